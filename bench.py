@@ -1,0 +1,444 @@
+"""Benchmark: OmniKVQuant decode step (cache append + fused split-K decode +
+combine/inverse rotation, every layer) on synthetic inputs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl omnikv|reference] [--workload 1]
+    torchrun --nproc-per-node N bench.py --gpus N ...   (one rank per GPU, weak scaling)
+
+Default workload: the Qwen2.5-Omni-3B-shaped decode (36 layers, 16 query / 2 KV
+heads, head dim 128, batch 1, 10,240 cached tokens of interleaved text / audio /
+video, K2/V2, 32-token windows); one step appends one text token per sequence to
+every layer's cache and runs decode attention for every layer. Each rank runs
+its own batch (different seed), so per-GPU work is fixed as N grows.
+
+Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events on
+the launching stream and preceded by an untimed L2 flush (a 512 MiB write);
+barrier + synchronize around the timed region; the max over ranks is reported.
+Each step is replayed from a CUDA graph that holds exactly the C-ABI calls of
+that step. `value` has all inputs resident in HBM; `e2e` also copies each step's
+inputs from pinned host memory and the step's outputs back to the host.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "2-bit decode attention tokens/s and achieved HBM GB/s vs ~8 TB/s (1 B200)"
+UNIT = "tokens/s"
+BYTES_PER_TOKEN_HEAD = {(2, 2): 82, (4, 4): 146}   # algorithmic packed bytes per token per kv head
+L2_FLUSH_BYTES = 512 << 20
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=64)
+    ap.add_argument("--warmup", type=int, default=4)
+    ap.add_argument("--impl", default="omnikv", choices=["omnikv", "reference"])
+    ap.add_argument("--workload", type=int, default=1)
+    ap.add_argument("--no-graphs", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", "clocks_rank%d.csv" % gpu_index)
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), "--query-gpu=" + self.Q,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = max(smax, float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# the GPU arm
+# ----------------------------------------------------------------------------
+class Workload:
+    """Per-layer constants and caches, prefilled (untimed), plus every step's inputs."""
+
+    def __init__(self, spec, seed, device, total_steps):
+        import bit_kv_cache_pack_b200 as m
+        from synth.workloads import (codebook, decode_inputs, key_drift, layer_params, prefill_inputs,
+                                     seq_lengths)
+        self.m, self.spec, self.dev = m, spec, device
+        self.lengths = seq_lengths(spec, seed)
+        self.cap = int(-(-(int(self.lengths.max()) + total_steps) // 32) * 32)
+        kb, vb = codebook(spec.key_bits), codebook(spec.value_bits)
+        self.consts, self.caches = [], []
+        qs, ks, vs, ms = [], [], [], []
+        for layer in range(spec.layers):
+            params = layer_params(spec, seed, layer)
+            c = m.LayerConstants(kb, vb, params["key_signs"], params["value_rot"], spec.num_q_heads, device)
+            cache = m.KVCache(spec.batch, spec.num_kv_heads, self.cap, spec.key_bits, spec.value_bits, device)
+            drift = key_drift(spec, seed, layer, self.cap // 32, device)
+            if spec.ragged:
+                for b in range(spec.batch):
+                    k, v, mod = prefill_inputs(spec, seed, layer, params, drift, self.lengths, device,
+                                               batch_index=[b])
+                    n = int(self.lengths[b])
+                    view = cache.sequence_view(b)
+                    m.omnikv_write_cache(c.struct, view, k[:, :, :n].contiguous(), v[:, :, :n].contiguous(),
+                                         mod[:, :n].contiguous(), n)
+                    del k, v, mod
+                cache.struct.max_seq_len = int(self.lengths.max())
+            else:
+                k, v, mod = prefill_inputs(spec, seed, layer, params, drift, self.lengths, device)
+                m.omnikv_write_cache(c.struct, cache.struct, k, v, mod, int(self.lengths[0]))
+                del k, v, mod
+            torch.cuda.synchronize(device)
+            self.consts.append(c)
+            self.caches.append(cache)
+            lq, lk, lv, lm = [], [], [], []
+            for s in range(total_steps):
+                q, kn, vn, mn = decode_inputs(spec, seed, layer, s, params, drift, self.lengths + s, device)
+                lq.append(q), lk.append(kn), lv.append(vn), lm.append(mn)
+            qs.append(torch.stack(lq)), ks.append(torch.stack(lk)), vs.append(torch.stack(lv))
+            ms.append(torch.stack(lm))
+        # [steps][layers][...] contiguous, so one step's inputs are one block
+        self.q = torch.stack(qs, 1).contiguous()
+        self.k = torch.stack(ks, 1).contiguous()
+        self.v = torch.stack(vs, 1).contiguous()
+        self.mod = torch.stack(ms, 1).contiguous()
+        self.S = max(1, m.omnikv_default_splits(self.consts[0].struct, self.caches[0].struct))
+        self.part = m.partials_tensor(spec.batch, spec.num_q_heads, self.S, device)
+        self.out = torch.empty(spec.layers, spec.batch, spec.num_q_heads, 128, dtype=torch.float32,
+                               device=device)
+
+    def step_calls(self, s, q, k, v, mod, stream, dec_events=None):
+        """The C-ABI calls of one decode step over all layers."""
+        m = self.m
+        n = self.spec.layers
+        for layer in range(n):
+            c, cache = self.consts[layer].struct, self.caches[layer].struct
+            m.omnikv_write_cache(c, cache, k[layer], v[layer], mod[layer], 1, stream)
+            if dec_events is not None:
+                dec_events[layer][0].record(stream)
+            m.omnikv_decode_attention(c, cache, q[layer], self.part, self.S, stream)
+            if dec_events is not None:
+                dec_events[layer][1].record(stream)
+            m.omnikv_combine(c, cache, self.part, self.S, self.out[layer], stream)
+
+    def launches_per_step(self):
+        return self.spec.layers * 4   # write + finish_write + decode + combine
+
+    def decode_bytes(self, s):
+        """Algorithmic bytes one decode launch reads at step s (per layer): packed
+        records per token and kv head, plus one modality byte per token."""
+        sp = self.spec
+        T = (self.lengths.astype(np.int64) + s + 1).sum()
+        return int(T * sp.num_kv_heads * BYTES_PER_TOKEN_HEAD[(sp.key_bits, sp.value_bits)] + T)
+
+
+def run_gpu(args):
+    import torch.distributed as dist
+    from synth.workloads import CONFIGS
+    world, rank, local = dist_env()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    spec = CONFIGS[args.workload]
+    seed = args.workload + 1000 * rank
+    K, W = args.steps, args.warmup
+    total = W + K + K + 1  # device-resident run, then the e2e run
+    wl = Workload(spec, seed, dev, total)
+    stream = torch.cuda.Stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    torch.cuda.synchronize(dev)
+
+    # --- device-resident steps, each from a captured graph ---------------------
+    dec_ev = [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in range(spec.layers)]
+              for _ in range(W + K)]
+    graphs = []
+    use_graphs = not args.no_graphs
+    if use_graphs:
+        pool = None
+        for s in range(W + K):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, pool=pool, stream=stream):
+                wl.step_calls(s, wl.q[s], wl.k[s], wl.v[s], wl.mod[s], torch.cuda.current_stream(),
+                              dec_ev[s])
+            pool = g.pool()
+            graphs.append(g)
+    torch.cuda.synchronize(dev)
+    t_steps = []
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    with torch.cuda.stream(stream):
+        for s in range(W + K):
+            flush.zero_()
+            if s == W:
+                torch.cuda.synchronize(dev)
+                if world > 1:
+                    dist.barrier()
+                clocks.start()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            if use_graphs:
+                graphs[s].replay()
+            else:
+                wl.step_calls(s, wl.q[s], wl.k[s], wl.v[s], wl.mod[s], stream, dec_ev[s])
+            e1.record(stream)
+            t_steps.append((e0, e1))
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in t_steps[W:]]
+    dec_ms = [dec_ev[s][l][0].elapsed_time(dec_ev[s][l][1]) for s in range(W, W + K) for l in range(spec.layers)]
+    dec_bytes = [wl.decode_bytes(s) for s in range(W, W + K) for _ in range(spec.layers)]
+    total_ms = float(np.sum(step_ms))
+
+    # --- end to end through the C ABI with host buffers ------------------------
+    hq = wl.q[W + K:].cpu().pin_memory()
+    hk = wl.k[W + K:].cpu().pin_memory()
+    hv = wl.v[W + K:].cpu().pin_memory()
+    hm = wl.mod[W + K:].cpu().pin_memory()
+    hout = torch.empty((K,) + tuple(wl.out.shape), dtype=torch.float32).pin_memory()
+    dq, dk, dv, dm = (torch.empty_like(wl.q[0]), torch.empty_like(wl.k[0]), torch.empty_like(wl.v[0]),
+                      torch.empty_like(wl.mod[0]))
+    e2e_graphs = []
+    if use_graphs:
+        for i in range(K):
+            s = W + K + i
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, pool=pool, stream=stream):
+                wl.step_calls(s, dq, dk, dv, dm, torch.cuda.current_stream())
+            e2e_graphs.append(g)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e2e_ev = []
+    with torch.cuda.stream(stream):
+        for i in range(K):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            dq.copy_(hq[i], non_blocking=True)
+            dk.copy_(hk[i], non_blocking=True)
+            dv.copy_(hv[i], non_blocking=True)
+            dm.copy_(hm[i], non_blocking=True)
+            if use_graphs:
+                e2e_graphs[i].replay()
+            else:
+                wl.step_calls(W + K + i, dq, dk, dv, dm, stream)
+            hout[i].copy_(wl.out, non_blocking=True)
+            e1.record(stream)
+            e2e_ev.append((e0, e1))
+    torch.cuda.synchronize(dev)
+    e2e_ms = float(np.sum([a.elapsed_time(b) for a, b in e2e_ev]))
+    assert torch.isfinite(hout).all(), "non-finite decode output"
+    h2d = int(dq.numel() * 2 + dk.numel() * 2 + dv.numel() * 2 + dm.numel())
+    d2h = int(wl.out.numel() * 4)
+
+    # --- max over ranks --------------------------------------------------------
+    t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, e2e_ms = float(t[0]), float(t[1])
+    tokens = world * spec.batch * K
+    value = tokens / (total_ms / 1e3)
+    e2e_value = tokens / (e2e_ms / 1e3)
+    avg_dec_s = float(np.mean(dec_ms)) / 1e3
+    achieved = float(np.mean(dec_bytes)) / avg_dec_s / 1e9
+    peak, peak_kind = peaks()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": W, "ms_per_step": round(total_ms / K, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "u2 codes, f32 accumulate",
+            "data": "synthetic",
+            "config": {"workload": spec.name, "layers": spec.layers, "global_batch": spec.batch * world,
+                       "context": int(wl.lengths.max()), "num_q_heads": spec.num_q_heads,
+                       "num_kv_heads": spec.num_kv_heads, "head_dim": 128, "key_bits": spec.key_bits,
+                       "value_bits": spec.value_bits, "window": 32, "num_splits": wl.S,
+                       "parallelism": "dp%d (independent sequences per rank)" % world,
+                       "l2": "flushed between timed steps (512 MiB write)",
+                       "launch": "CUDA graph per step" if use_graphs else "eager"},
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": None,
+                         "peak_source": peak_kind, "kernel": "decode_split_k",
+                         "avg_launch_us": round(avg_dec_s * 1e6, 3),
+                         "bytes_per_launch": int(np.mean(dec_bytes))},
+            "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": wl.launches_per_step() * K,
+            "clocks": clk,
+        }
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(spec, seed)
+        print(json.dumps(line), flush=True)
+    graphs.clear()
+    e2e_graphs.clear()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------
+# the CPU oracle, timed (baseline and reference arm)
+# ----------------------------------------------------------------------------
+def _oracle_layers(spec, seed, layers, extra_steps):
+    from oracle import codec
+    from synth.workloads import codebook, decode_inputs, key_drift, layer_params, prefill_inputs, seq_lengths
+    L = seq_lengths(spec, seed)
+    cap = int(-(-(int(L.max()) + extra_steps) // 32) * 32)
+    out = []
+    for layer in layers:
+        params = layer_params(spec, seed, layer)
+        ocfg = codec.OracleConfig(codebook(spec.key_bits), codebook(spec.value_bits),
+                                  params["key_signs"].numpy(), params["value_rot"].numpy(),
+                                  spec.num_q_heads, spec.num_kv_heads)
+        oc = codec.OracleCache(spec.batch, spec.num_kv_heads, cap, spec.key_bits, spec.value_bits)
+        drift = key_drift(spec, seed, layer, cap // 32, "cpu")
+        k, v, mod = prefill_inputs(spec, seed, layer, params, drift, L, "cpu")
+        for b in range(spec.batch):
+            sub = codec.OracleCache(1, spec.num_kv_heads, cap, spec.key_bits, spec.value_bits)
+            n = int(L[b])
+            codec.write_cache(ocfg, sub, k[b:b + 1, :, :n].numpy(), v[b:b + 1, :, :n].numpy(),
+                              mod[b:b + 1, :n].numpy())
+            oc.records[b], oc.key_tail[b], oc.modality[b], oc.seq_lens[b] = (
+                sub.records[0], sub.key_tail[0], sub.modality[0], sub.seq_lens[0])
+        steps = [decode_inputs(spec, seed, layer, s, params, drift, L + s, "cpu") for s in range(extra_steps)]
+        out.append((ocfg, oc, steps))
+    return out
+
+
+def _oracle_step(ocfg, oc, inputs, num_splits=4):
+    from oracle import codec
+    from oracle.attention import decode_fused
+    q, kn, vn, mn = inputs
+    codec.write_cache(ocfg, oc, kn.numpy(), vn.numpy(), mn.numpy())
+    return decode_fused(ocfg, oc, q.numpy(), num_splits)
+
+
+def cpu_baseline(spec, seed, sample_layers=12):
+    """The oracle as it stands (single process, numpy) on a bounded sample: one
+    decode step (append + fused decode + combine) over the first sample_layers
+    layers, scaled to all layers."""
+    n = min(sample_layers, spec.layers)
+    prepared = _oracle_layers(spec, seed, range(n), 1)
+    t0 = time.perf_counter()
+    for ocfg, oc, steps in prepared:
+        _oracle_step(ocfg, oc, steps[0])
+    dt = time.perf_counter() - t0
+    per_step = dt * spec.layers / n
+    return {"value": round(spec.batch / per_step, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": "1 decode step x %d of %d layers (append + fused decode + combine, numpy fp64), "
+                      "scaled to %d layers; %.1f s of CPU" % (n, spec.layers, spec.layers, dt)}
+
+
+def run_reference(args):
+    from synth.workloads import CONFIGS
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    spec = CONFIGS[args.workload]
+    seed = args.workload
+    K, W = args.steps, args.warmup
+    n_prep = min(4, spec.layers)
+    prepared = _oracle_layers(spec, seed, range(n_prep), (W + K) // n_prep + 2)
+    times = []
+    for s in range(W + K):
+        ocfg, oc, steps = prepared[s % n_prep]
+        t0 = time.perf_counter()
+        _oracle_step(ocfg, oc, steps[s // n_prep])
+        if s >= W:
+            times.append(time.perf_counter() - t0)
+    per_step = float(np.mean(times)) * spec.layers   # one sample = one layer of a step
+    value = spec.batch / per_step
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
+        "steps": K, "warmup": W, "ms_per_step": round(per_step * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic",
+        "config": {"workload": spec.name, "layers": spec.layers, "global_batch": spec.batch,
+                   "context": int(spec.context), "num_q_heads": spec.num_q_heads,
+                   "num_kv_heads": spec.num_kv_heads, "head_dim": 128, "key_bits": spec.key_bits,
+                   "value_bits": spec.value_bits, "window": 32},
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": "each step: one layer's append + fused decode + combine (numpy fp64), "
+                                   "x %d layers" % spec.layers},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,12 @@
+"""OmniKVQuant 2-bit KV-cache write and fused decode attention for B200 (sm_100a).
+
+The compute lives in libomnikv.so (hand-written CUDA behind the C ABI of
+include/omnikv.h); this package is its thin Python binding plus PyTorch
+allocation helpers.
+"""
+from ._abi import (OMNIKV_DEVERR_CAPACITY, OMNIKV_ERR_CAPACITY, OMNIKV_ERR_CUDA,  # noqa: F401
+                   OMNIKV_ERR_INVALID_ARG, OMNIKV_ERR_UNSUPPORTED, OMNIKV_OK, OmniKVCache,
+                   OmniKVConfig, OmniKVError, load, omnikv_abi_version, omnikv_combine,
+                   omnikv_decode_attention, omnikv_default_splits, omnikv_partials_bytes,
+                   omnikv_record_bytes, omnikv_write_cache, status_string)
+from .layer import KVCache, LayerConstants, partials_tensor  # noqa: F401

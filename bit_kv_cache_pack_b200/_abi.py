@@ -1,0 +1,153 @@
+"""ctypes binding of libomnikv.so: the C ABI declared in include/omnikv.h.
+
+Argument marshalling only: every step of the cache write and decode runs in the
+library's CUDA kernels. Functions keep the C names; tensors may be passed as
+torch tensors (their data_ptr() is used) or as integer device addresses.
+A non-OK status raises OmniKVError. Loading fails loudly if the library has not
+been built (python -m bit_kv_cache_pack_b200.build).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libomnikv.so")
+
+OMNIKV_OK = 0
+OMNIKV_ERR_INVALID_ARG = 1
+OMNIKV_ERR_UNSUPPORTED = 2
+OMNIKV_ERR_CAPACITY = 3
+OMNIKV_ERR_CUDA = 4
+OMNIKV_ERR_DEVICE_CHECK = 5
+OMNIKV_DEVERR_CAPACITY = 0x1
+OMNIKV_DEVERR_MODALITY = 0x2
+
+EXPORTED = (
+    "omnikv_record_bytes", "omnikv_partials_bytes", "omnikv_default_splits",
+    "omnikv_write_cache", "omnikv_decode_attention", "omnikv_combine",
+    "omnikv_status_string", "omnikv_abi_version",
+)
+
+
+class OmniKVError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__("%s: %s (status %d)" % (where, status_string(status), status))
+
+
+class OmniKVConfig(ctypes.Structure):
+    _fields_ = [
+        ("head_dim", ctypes.c_int32),
+        ("num_q_heads", ctypes.c_int32),
+        ("num_kv_heads", ctypes.c_int32),
+        ("window", ctypes.c_int32),
+        ("key_bits", ctypes.c_int32),
+        ("value_bits", ctypes.c_int32),
+        ("key_codebook", ctypes.c_void_p),
+        ("value_codebook", ctypes.c_void_p),
+        ("key_signs", ctypes.c_void_p),
+        ("value_rot", ctypes.c_void_p),
+    ]
+
+
+class OmniKVCache(ctypes.Structure):
+    _fields_ = [
+        ("records", ctypes.c_void_p),
+        ("key_tail", ctypes.c_void_p),
+        ("modality", ctypes.c_void_p),
+        ("seq_lens", ctypes.c_void_p),
+        ("error_word", ctypes.c_void_p),
+        ("batch", ctypes.c_int32),
+        ("cap_tokens", ctypes.c_int32),
+        ("max_seq_len", ctypes.c_int32),
+    ]
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """The loaded library; raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError("libomnikv.so is not built (%s); run python -m bit_kv_cache_pack_b200.build"
+                          % _LIB_PATH)
+    lib = ctypes.CDLL(_LIB_PATH)
+    P, I32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    cfgp, cachep = ctypes.POINTER(OmniKVConfig), ctypes.POINTER(OmniKVCache)
+    lib.omnikv_record_bytes.argtypes, lib.omnikv_record_bytes.restype = [I32, I32], SZ
+    lib.omnikv_partials_bytes.argtypes, lib.omnikv_partials_bytes.restype = [I32, I32, I32], SZ
+    lib.omnikv_default_splits.argtypes, lib.omnikv_default_splits.restype = [cfgp, cachep], I32
+    lib.omnikv_write_cache.argtypes = [cfgp, cachep, P, P, P, I32, P]
+    lib.omnikv_write_cache.restype = ctypes.c_int
+    lib.omnikv_decode_attention.argtypes = [cfgp, cachep, P, P, I32, P]
+    lib.omnikv_decode_attention.restype = ctypes.c_int
+    lib.omnikv_combine.argtypes = [cfgp, cachep, P, I32, P, P]
+    lib.omnikv_combine.restype = ctypes.c_int
+    lib.omnikv_status_string.argtypes, lib.omnikv_status_string.restype = [ctypes.c_int], ctypes.c_char_p
+    lib.omnikv_abi_version.argtypes, lib.omnikv_abi_version.restype = [], I32
+    _lib = lib
+    return lib
+
+
+def _ptr(x) -> int:
+    if x is None:
+        return 0
+    if isinstance(x, int):
+        return x
+    return int(x.data_ptr())
+
+
+def _stream(s) -> int:
+    if s is None:
+        return 0
+    if isinstance(s, int):
+        return s
+    return int(s.cuda_stream)
+
+
+def _check(status: int, where: str) -> None:
+    if status != OMNIKV_OK:
+        raise OmniKVError(status, where)
+
+
+def status_string(status: int) -> str:
+    return load().omnikv_status_string(status).decode()
+
+
+def omnikv_abi_version() -> int:
+    return int(load().omnikv_abi_version())
+
+
+def omnikv_record_bytes(key_bits: int, value_bits: int) -> int:
+    return int(load().omnikv_record_bytes(key_bits, value_bits))
+
+
+def omnikv_partials_bytes(batch: int, num_q_heads: int, num_splits: int) -> int:
+    return int(load().omnikv_partials_bytes(batch, num_q_heads, num_splits))
+
+
+def omnikv_default_splits(cfg: OmniKVConfig, cache: OmniKVCache) -> int:
+    return int(load().omnikv_default_splits(ctypes.byref(cfg), ctypes.byref(cache)))
+
+
+def omnikv_write_cache(cfg: OmniKVConfig, cache: OmniKVCache, k_new, v_new, modality_new, n_new: int,
+                       stream=None) -> None:
+    st = load().omnikv_write_cache(ctypes.byref(cfg), ctypes.byref(cache), _ptr(k_new), _ptr(v_new),
+                                   _ptr(modality_new), int(n_new), _stream(stream))
+    _check(st, "omnikv_write_cache")
+
+
+def omnikv_decode_attention(cfg: OmniKVConfig, cache: OmniKVCache, q, partials, num_splits: int = 0,
+                            stream=None) -> None:
+    st = load().omnikv_decode_attention(ctypes.byref(cfg), ctypes.byref(cache), _ptr(q), _ptr(partials),
+                                        int(num_splits), _stream(stream))
+    _check(st, "omnikv_decode_attention")
+
+
+def omnikv_combine(cfg: OmniKVConfig, cache: OmniKVCache, partials, num_splits: int, out, stream=None) -> None:
+    st = load().omnikv_combine(ctypes.byref(cfg), ctypes.byref(cache), _ptr(partials), int(num_splits),
+                               _ptr(out), _stream(stream))
+    _check(st, "omnikv_combine")

@@ -1,0 +1,170 @@
+// C ABI of the OmniKVQuant kernels: argument validation and launches.
+// Every check runs on the host before any launch; see include/omnikv.h.
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace omnikv;
+
+namespace {
+
+bool aligned(const void* ptr, size_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; }
+
+omnikv_status check_config(const omnikv_config* cfg) {
+  if (!cfg) return OMNIKV_ERR_INVALID_ARG;
+  if (cfg->head_dim != kHeadDim || cfg->window != kWindow) return OMNIKV_ERR_UNSUPPORTED;
+  if ((cfg->key_bits != 2 && cfg->key_bits != 4) || (cfg->value_bits != 2 && cfg->value_bits != 4))
+    return OMNIKV_ERR_UNSUPPORTED;
+  if (cfg->num_kv_heads < 1 || cfg->num_q_heads < 1 || cfg->num_q_heads % cfg->num_kv_heads)
+    return OMNIKV_ERR_INVALID_ARG;
+  if (cfg->num_q_heads / cfg->num_kv_heads > kMaxGroup) return OMNIKV_ERR_UNSUPPORTED;
+  if (!cfg->key_codebook || !cfg->value_codebook || !cfg->key_signs || !cfg->value_rot)
+    return OMNIKV_ERR_INVALID_ARG;
+  if (!aligned(cfg->key_signs, 16) || !aligned(cfg->value_rot, 16)) return OMNIKV_ERR_INVALID_ARG;
+  return OMNIKV_OK;
+}
+
+omnikv_status check_cache(const omnikv_cache* c) {
+  if (!c || !c->records || !c->key_tail || !c->modality || !c->seq_lens) return OMNIKV_ERR_INVALID_ARG;
+  if (c->batch < 1 || c->cap_tokens < kWindow || c->cap_tokens % kWindow) return OMNIKV_ERR_INVALID_ARG;
+  if (c->max_seq_len < 0 || c->max_seq_len > c->cap_tokens) return OMNIKV_ERR_INVALID_ARG;
+  if (!aligned(c->records, 16) || !aligned(c->key_tail, 16) || !aligned(c->modality, 16) ||
+      !aligned(c->seq_lens, 4) || (c->error_word && !aligned(c->error_word, 4)))
+    return OMNIKV_ERR_INVALID_ARG;
+  return OMNIKV_OK;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+int32_t resolve_splits(const omnikv_config* cfg, const omnikv_cache* c, int32_t requested) {
+  if (requested > 0) return requested;
+  const int nw = (c->max_seq_len + kWindow - 1) / kWindow;
+  if (nw <= 0) return 1;
+  const long long units = (long long)c->batch * cfg->num_kv_heads;
+  const long long target = 2LL * sm_count();
+  long long s = (target + units - 1) / units;
+  // keep at least a few windows per split so the per-CTA setup is amortised
+  const long long max_s = (nw + 3) / 4;
+  if (s > max_s) s = max_s;
+  if (s < 1) s = 1;
+  return (int32_t)s;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t omnikv_record_bytes(int32_t key_bits, int32_t value_bits) {
+  if ((key_bits != 2 && key_bits != 4) || (value_bits != 2 && value_bits != 4)) return 0;
+  return (size_t)RecordLayout(key_bits, value_bits).bytes;
+}
+
+size_t omnikv_partials_bytes(int32_t batch, int32_t num_q_heads, int32_t num_splits) {
+  if (batch < 1 || num_q_heads < 1 || num_splits < 1) return 0;
+  return (size_t)batch * num_q_heads * num_splits * sizeof(Partial);
+}
+
+int32_t omnikv_default_splits(const omnikv_config* cfg, const omnikv_cache* cache) {
+  if (check_config(cfg) != OMNIKV_OK || check_cache(cache) != OMNIKV_OK) return 0;
+  return resolve_splits(cfg, cache, 0);
+}
+
+omnikv_status omnikv_write_cache(const omnikv_config* cfg, omnikv_cache* cache, const void* k_new,
+                                 const void* v_new, const uint8_t* modality_new, int32_t n_new,
+                                 void* stream) {
+  omnikv_status st = check_config(cfg);
+  if (st != OMNIKV_OK) return st;
+  if ((st = check_cache(cache)) != OMNIKV_OK) return st;
+  if (n_new < 1 || !k_new || !v_new || !modality_new) return OMNIKV_ERR_INVALID_ARG;
+  if (!aligned(k_new, 16) || !aligned(v_new, 16)) return OMNIKV_ERR_INVALID_ARG;
+  if ((long long)cache->max_seq_len + n_new > cache->cap_tokens) return OMNIKV_ERR_CAPACITY;
+  WriteParams p;
+  p.key_cb = cfg->key_codebook;
+  p.val_cb = cfg->value_codebook;
+  p.key_signs = cfg->key_signs;
+  p.value_rot = cfg->value_rot;
+  p.key_bits = cfg->key_bits;
+  p.value_bits = cfg->value_bits;
+  p.num_kv_heads = cfg->num_kv_heads;
+  p.records = static_cast<uint8_t*>(cache->records);
+  p.key_tail = static_cast<__half*>(cache->key_tail);
+  p.modality = cache->modality;
+  p.seq_lens = cache->seq_lens;
+  p.error_word = cache->error_word;
+  p.cap_tokens = cache->cap_tokens;
+  p.cap_windows = cache->cap_tokens / kWindow;
+  p.k_new = static_cast<const __half*>(k_new);
+  p.v_new = static_cast<const __half*>(v_new);
+  p.mod_new = modality_new;
+  p.n_new = n_new;
+  if (launch_write(p, cache->batch, static_cast<cudaStream_t>(stream)) != cudaSuccess) return OMNIKV_ERR_CUDA;
+  cache->max_seq_len += n_new;
+  return OMNIKV_OK;
+}
+
+omnikv_status omnikv_decode_attention(const omnikv_config* cfg, const omnikv_cache* cache, const void* q,
+                                      void* partials, int32_t num_splits, void* stream) {
+  omnikv_status st = check_config(cfg);
+  if (st != OMNIKV_OK) return st;
+  if ((st = check_cache(cache)) != OMNIKV_OK) return st;
+  if (!q || !partials || num_splits < 0) return OMNIKV_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(partials, 16)) return OMNIKV_ERR_INVALID_ARG;
+  DecodeParams p;
+  p.key_cb = cfg->key_codebook;
+  p.val_cb = cfg->value_codebook;
+  p.key_signs = cfg->key_signs;
+  p.key_bits = cfg->key_bits;
+  p.value_bits = cfg->value_bits;
+  p.num_kv_heads = cfg->num_kv_heads;
+  p.group = cfg->num_q_heads / cfg->num_kv_heads;
+  p.records = static_cast<const uint8_t*>(cache->records);
+  p.modality = cache->modality;
+  p.seq_lens = cache->seq_lens;
+  p.cap_tokens = cache->cap_tokens;
+  p.cap_windows = cache->cap_tokens / kWindow;
+  p.q = static_cast<const __half*>(q);
+  p.partials = static_cast<Partial*>(partials);
+  p.num_splits = resolve_splits(cfg, cache, num_splits);
+  if (launch_decode(p, cache->batch, static_cast<cudaStream_t>(stream)) != cudaSuccess) return OMNIKV_ERR_CUDA;
+  return OMNIKV_OK;
+}
+
+omnikv_status omnikv_combine(const omnikv_config* cfg, const omnikv_cache* cache, const void* partials,
+                             int32_t num_splits, float* out, void* stream) {
+  omnikv_status st = check_config(cfg);
+  if (st != OMNIKV_OK) return st;
+  if ((st = check_cache(cache)) != OMNIKV_OK) return st;
+  if (!partials || !out || num_splits < 0) return OMNIKV_ERR_INVALID_ARG;
+  if (!aligned(partials, 16) || !aligned(out, 16)) return OMNIKV_ERR_INVALID_ARG;
+  CombineParams p;
+  p.value_rot = cfg->value_rot;
+  p.num_kv_heads = cfg->num_kv_heads;
+  p.group = cfg->num_q_heads / cfg->num_kv_heads;
+  p.partials = static_cast<const Partial*>(partials);
+  p.num_splits = resolve_splits(cfg, cache, num_splits);
+  p.out = out;
+  if (launch_combine(p, cache->batch, static_cast<cudaStream_t>(stream)) != cudaSuccess) return OMNIKV_ERR_CUDA;
+  return OMNIKV_OK;
+}
+
+const char* omnikv_status_string(omnikv_status s) {
+  switch (s) {
+    case OMNIKV_OK: return "ok";
+    case OMNIKV_ERR_INVALID_ARG: return "invalid argument";
+    case OMNIKV_ERR_UNSUPPORTED: return "unsupported configuration";
+    case OMNIKV_ERR_CAPACITY: return "cache capacity exceeded";
+    case OMNIKV_ERR_CUDA: return "CUDA launch failed";
+    case OMNIKV_ERR_DEVICE_CHECK: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+int32_t omnikv_abi_version(void) { return OMNIKV_ABI_VERSION; }
+
+}  // extern "C"

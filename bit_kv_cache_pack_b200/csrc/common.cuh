@@ -1,0 +1,94 @@
+// Shared device helpers for the OmniKVQuant kernels (sm_100a).
+//
+// Arithmetic that decides a stored bit (key rotation, window range, codes,
+// value scale) uses explicitly rounded intrinsics (__fadd_rn, __fsub_rn,
+// __fmul_rn, __fdiv_rn, __fsqrt_rn) so that the compiler never contracts a
+// multiply and an add into an FMA: the result is the IEEE value of each step.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "../../include/omnikv.h"
+
+namespace omnikv {
+
+constexpr int kHeadDim = 128;
+constexpr int kWindow = 32;
+constexpr int kMods = 3;
+constexpr int kMaxGroup = 8;  // query heads per kv head handled by one CTA
+
+// fp32(2^-3.5) = fp32(1/sqrt(128)), bit pattern 0x3DB504F3
+__device__ __forceinline__ float inv_sqrt_d() { return __int_as_float(0x3DB504F3); }
+
+struct RecordLayout {
+  int k_off, meta_off, v_off, sigma_off, bytes;
+  int key_bits, value_bits;
+  __host__ __device__ RecordLayout(int kb, int vb) : key_bits(kb), value_bits(vb) {
+    const int kbytes = kWindow * kHeadDim * kb / 8;
+    const int vbytes = kWindow * kHeadDim * vb / 8;
+    k_off = 0;
+    meta_off = kbytes;
+    v_off = meta_off + kHeadDim * 4;
+    sigma_off = v_off + vbytes;
+    bytes = sigma_off + kWindow * 2;
+  }
+};
+
+// One entry of the split-K partials buffer.
+struct Partial {
+  float acc[kMods][kHeadDim];
+  float m;
+  float l;
+};
+static_assert(sizeof(Partial) == 1544, "partials entry is 1544 bytes");
+
+// Sign flip, Sylvester-Hadamard butterflies with h = 1, 2, ..., 64, then the
+// fp32 scale 2^-3.5, on a 128-vector spread over a warp: lane L holds channels
+// 4L + r, r = 0..3, in x[r]. Stages h = 1, 2 stay inside the thread; stage h >= 4
+// pairs lane L with lane L ^ (h / 4). The lower index of a pair becomes a + b
+// and the upper a - b (a the lower, b the upper), exactly as the scalar order.
+__device__ __forceinline__ void warp_hadamard_rotate(float x[4], const float sign[4]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int r = 0; r < 4; ++r) x[r] = __fmul_rn(x[r], sign[r]);
+  {  // h = 1
+    const float a0 = x[0], b0 = x[1], a1 = x[2], b1 = x[3];
+    x[0] = __fadd_rn(a0, b0);
+    x[1] = __fsub_rn(a0, b0);
+    x[2] = __fadd_rn(a1, b1);
+    x[3] = __fsub_rn(a1, b1);
+  }
+  {  // h = 2
+    const float a0 = x[0], b0 = x[2], a1 = x[1], b1 = x[3];
+    x[0] = __fadd_rn(a0, b0);
+    x[2] = __fsub_rn(a0, b0);
+    x[1] = __fadd_rn(a1, b1);
+    x[3] = __fsub_rn(a1, b1);
+  }
+#pragma unroll
+  for (int hl = 1; hl < 32; hl <<= 1) {  // h = 4 * hl
+    const bool upper = (lane & hl) != 0;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float other = __shfl_xor_sync(0xffffffffu, x[r], hl);
+      x[r] = upper ? __fsub_rn(other, x[r]) : __fadd_rn(x[r], other);
+    }
+  }
+  const float s = inv_sqrt_d();
+#pragma unroll
+  for (int r = 0; r < 4; ++r) x[r] = __fmul_rn(x[r], s);
+}
+
+// code = #{ j : z > t_j } for the L-1 thresholds (strict comparison).
+__device__ __forceinline__ uint32_t count_above(float z, const float* thr, int nthr) {
+  uint32_t c = 0;
+  for (int j = 0; j < nthr; ++j) c += (z > thr[j]) ? 1u : 0u;
+  return c;
+}
+
+__device__ __forceinline__ void set_error(int32_t* word, int32_t bits) {
+  if (word) atomicOr(word, bits);
+}
+
+}  // namespace omnikv

@@ -1,0 +1,56 @@
+// Launch parameters and launchers of the OmniKVQuant kernels (internal).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace omnikv {
+
+struct Partial;
+
+struct WriteParams {
+  const float* key_cb;
+  const float* val_cb;
+  const float* key_signs;
+  const float* value_rot;
+  int key_bits, value_bits, num_kv_heads;
+  uint8_t* records;
+  __half* key_tail;
+  uint8_t* modality;
+  int32_t* seq_lens;
+  int32_t* error_word;
+  int cap_tokens, cap_windows;
+  const __half* k_new;
+  const __half* v_new;
+  const uint8_t* mod_new;
+  int n_new;
+};
+
+struct DecodeParams {
+  const float* key_cb;
+  const float* val_cb;
+  const float* key_signs;
+  int key_bits, value_bits, num_kv_heads, group;
+  const uint8_t* records;
+  const uint8_t* modality;
+  const int32_t* seq_lens;
+  int cap_tokens, cap_windows;
+  const __half* q;
+  Partial* partials;
+  int num_splits;
+};
+
+struct CombineParams {
+  const float* value_rot;
+  int num_kv_heads, group;
+  const Partial* partials;
+  int num_splits;
+  float* out;
+};
+
+cudaError_t launch_write(const WriteParams& p, int batch, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeParams& p, int batch, cudaStream_t stream);
+cudaError_t launch_combine(const CombineParams& p, int batch, cudaStream_t stream);
+
+}  // namespace omnikv

@@ -1,0 +1,172 @@
+/*
+ * omnikv.h -- C ABI of the OmniKVQuant 2-bit KV-cache write and fused decode
+ * attention for NVIDIA B200 (sm_100a).
+ *
+ * Method: "OmniKVQuant: KV Cache Quantization for Omni-LLMs" (arXiv:2609.11582).
+ *   - keys: sign-flip Hadamard rotation (the TurboQuant rotation kept for keys,
+ *     paperpeel.com section 2.2 "Temporal key drift"), then a per-channel
+ *     min-max range over each 32-token group (section 3.1 "Implementation
+ *     details"), stored as fp16 minimum m_gc and scale s_gc (section 3.3 "Error
+ *     comparison"), mapped onto a fixed codebook (pchao.org "方法概览").
+ *   - values: rotated with the orthogonal basis U_m of the token's modality
+ *     m in {V, A, L} (section 2.3 "Modality-aware value rotation"), then coded
+ *     on the same kind of fixed codebook with one fp16 scale per token.
+ *   - decode: the query is rotated once per head instead of inverse-rotating
+ *     every cached key, the 2-bit cache is unpacked inside attention in
+ *     FlashAttention order, and the inverse value rotations are batched across
+ *     head outputs, so no dense fp16 cache is built (section 1, last paragraph;
+ *     abstract on arxiv / thelatestinai.com).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller, except the
+ *     configuration and cache structs themselves, which live in host memory.
+ *     The library allocates nothing, frees nothing, never synchronises the
+ *     device and keeps no global state.
+ *   - `stream` is a cudaStream_t (passed as void*); NULL means the legacy
+ *     default stream. All work is stream-ordered on it.
+ *   - Host-side validation runs before any launch; a failed check returns an
+ *     error status and launches nothing. A launch failure returns
+ *     OMNIKV_ERR_CUDA. Conditions only the device can see (a sequence whose
+ *     length would pass cap_tokens) skip that sequence's work and set a bit in
+ *     the optional device error word (see omnikv_cache.error_word); they never
+ *     fault.
+ *   - fp16 tensors are IEEE binary16 (passed as void*), row-major, contiguous.
+ *
+ * Window record (one per sequence, kv head and 32-token window; all fields
+ * little-endian; bits = key_bits or value_bits; cpw = 32 / bits codes per u32):
+ *   K codes [32 tokens][128 / cpw] u32  token-major: channel c of token t is
+ *           in word (t, c / cpw) at bits [bits * (c % cpw), +bits)
+ *   meta    [128] { fp16 m_gc, fp16 s_gc }
+ *   V codes [32 / cpw][128] u32         channel-major: token t, channel c is in
+ *           word (t / cpw, c) at bits [bits * (t % cpw), +bits)
+ *   sigma   [32] fp16 (per-token value scale)
+ * Size: 2624 bytes for K2/V2, 4672 bytes for K4/V4 (omnikv_record_bytes).
+ * Dequantised rotated-space cache: k'_tc = m_gc + s_gc (c_j - c_0) for key code
+ * j; v'_tc = sigma_t c_j for value code j. Padded slots of a partial window hold
+ * code 0 and sigma 0.
+ */
+#ifndef OMNIKV_H_
+#define OMNIKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define OMNIKV_API __attribute__((visibility("default")))
+#else
+#define OMNIKV_API
+#endif
+
+#define OMNIKV_ABI_VERSION 1
+#define OMNIKV_HEAD_DIM 128
+#define OMNIKV_WINDOW 32
+#define OMNIKV_NUM_MODALITIES 3 /* 0 = text (L), 1 = audio (A), 2 = video (V) */
+
+typedef enum {
+  OMNIKV_OK = 0,
+  OMNIKV_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned pointer */
+  OMNIKV_ERR_UNSUPPORTED = 2,  /* head_dim != 128, window != 32, bits not 2/4, GQA group > 8 */
+  OMNIKV_ERR_CAPACITY = 3,     /* max_seq_len + n_new > cap_tokens */
+  OMNIKV_ERR_CUDA = 4,         /* a CUDA launch failed (cudaGetLastError) */
+  OMNIKV_ERR_DEVICE_CHECK = 5  /* reserved for device-side checks read back by the caller */
+} omnikv_status;
+
+/* Device error word bits (omnikv_cache.error_word). */
+#define OMNIKV_DEVERR_CAPACITY 0x1 /* a write would have passed cap_tokens; that sequence was skipped */
+#define OMNIKV_DEVERR_MODALITY 0x2 /* a modality id was > 2; it was stored and used as 2 (video) */
+
+/* Per-layer constants. All pointers are device pointers. */
+typedef struct {
+  int32_t head_dim;             /* must be 128 */
+  int32_t num_q_heads;          /* multiple of num_kv_heads; group size G = num_q_heads / num_kv_heads in 1..8 */
+  int32_t num_kv_heads;         /* >= 1 */
+  int32_t window;               /* must be 32 (the 32-token group g of section 3.1) */
+  int32_t key_bits;             /* 2 or 4 */
+  int32_t value_bits;           /* 2 or 4 */
+  const float* key_codebook;    /* [2^key_bits] fp32, strictly ascending (fixed codebook) */
+  const float* value_codebook;  /* [2^value_bits] fp32, strictly ascending */
+  const float* key_signs;       /* [128] fp32, each +1 or -1 (sign flip before the Hadamard transform) */
+  const float* value_rot;       /* [num_kv_heads][3][128][128] fp32: U_m row-major, its COLUMNS are the
+                                   basis: v' = U_m^T v, v = U_m v'. Must be orthogonal. */
+} omnikv_config;
+
+/* One layer's cache for a batch. Device memory is owned by the caller and must be
+ * zero-filled before the first write (records, modality, seq_lens). A view of
+ * one sequence (batch = 1, pointers advanced by its index) is itself a valid cache. */
+typedef struct {
+  void* records;        /* [batch][num_kv_heads][cap_tokens / 32] window records, 16-byte aligned */
+  void* key_tail;       /* [batch][num_kv_heads][32][128] fp16: raw keys of each partial last window */
+  uint8_t* modality;    /* [batch][cap_tokens] modality id of every cached token */
+  int32_t* seq_lens;    /* [batch] tokens cached per sequence; advanced by omnikv_write_cache */
+  int32_t* error_word;  /* optional [1] int32: OMNIKV_DEVERR_* bits are OR-ed in; may be NULL */
+  int32_t batch;        /* >= 1 */
+  int32_t cap_tokens;   /* capacity per sequence, a positive multiple of 32 */
+  int32_t max_seq_len;  /* HOST-side upper bound on every seq_lens[b]; sizes grids and checks capacity.
+                           omnikv_write_cache adds n_new to it on success. */
+} omnikv_cache;
+
+/* Bytes of one window record: 2624 for K2/V2, 4672 for K4/V4; 0 for unsupported bits. */
+OMNIKV_API size_t omnikv_record_bytes(int32_t key_bits, int32_t value_bits);
+
+/* Bytes of the split-K partials buffer for omnikv_decode_attention / omnikv_combine:
+ * [batch][num_q_heads][num_splits] entries of { fp32 acc[3][128], fp32 m, fp32 l } (1544 B each). */
+OMNIKV_API size_t omnikv_partials_bytes(int32_t batch, int32_t num_q_heads, int32_t num_splits);
+
+/* The split count used when omnikv_decode_attention is given num_splits = 0 (depends on the
+ * batch, the kv heads, max_seq_len and the device's SM count). Returns >= 1, or 0 on bad arguments. */
+OMNIKV_API int32_t omnikv_default_splits(const omnikv_config* cfg, const omnikv_cache* cache);
+
+/* Cache write (kv_quant_pack). Appends n_new tokens to EVERY sequence of the batch, at position
+ * seq_lens[b] (read on the device), then advances seq_lens[b] and cache->max_seq_len by n_new.
+ *   k_new, v_new : [batch][num_kv_heads][n_new][128] fp16, 16-byte aligned
+ *   modality_new : [batch][n_new] u8, each 0, 1 or 2 (larger ids: OMNIKV_DEVERR_MODALITY)
+ * Keys: every 32-token window touched by the new positions is (re)quantised over all its valid
+ * tokens: rotation k' = fp32(2^-3.5) H (s . k) (butterflies h = 1..64, fp32), per-channel
+ * m = fp16(min), s = fp16((max - min) / (c_last - c_0)), code = #{j : (k' - m) / s + c_0 > t_j},
+ * t_j = fp32((c_j + c_{j+1}) * 0.5), code 0 where s == 0. A window left partial keeps its raw keys in
+ * key_tail. Values: sigma = fp16(sqrt(pairwise-tree sum of v_c^2 / 128)) of the unrotated fp16 value,
+ * v' = U_m^T v (fp32 accumulation), code = #{j : v'_c / sigma > t_j}, 0 where sigma == 0.
+ * Key codes and metadata are bit-exact with a scalar fp32 evaluation in this order; value codes
+ * depend on the fp32-accumulated rotation and may differ from an fp64 rotation only where v'/sigma
+ * lies within rounding of a threshold.
+ * Errors: OMNIKV_ERR_CAPACITY if cache->max_seq_len + n_new > cap_tokens (nothing launched);
+ * OMNIKV_ERR_INVALID_ARG for n_new < 1 or a null / misaligned pointer. */
+OMNIKV_API omnikv_status omnikv_write_cache(const omnikv_config* cfg, omnikv_cache* cache,
+                                 const void* k_new, const void* v_new, const uint8_t* modality_new,
+                                 int32_t n_new, void* stream);
+
+/* Fused split-K decode attention over the packed cache (decode_split_k). For every sequence b,
+ * query head i (kv head i / G) and split s, over the windows [floor(s W / S), floor((s+1) W / S))
+ * of the W = ceil(seq_lens[b] / 32) windows: q' = fp32(2^-3.5) H (s . q_i); score_t = q' . k'_t /
+ * sqrt(128); a running max m and sum l of exp(score - m), and one rotated-space accumulator per
+ * modality acc_m = sum_{t of modality m} exp(score_t - m) v'_t. Written to `partials`.
+ *   q          : [batch][num_q_heads][128] fp16, 16-byte aligned
+ *   partials   : device buffer of omnikv_partials_bytes(batch, num_q_heads, S) bytes, 16-byte aligned
+ *   num_splits : S >= 1, or 0 for omnikv_default_splits(cfg, cache)
+ * Empty splits write m = -inf, l = 0, acc = 0. */
+OMNIKV_API omnikv_status omnikv_decode_attention(const omnikv_config* cfg, const omnikv_cache* cache,
+                                      const void* q, void* partials, int32_t num_splits, void* stream);
+
+/* Split-K combine and batched inverse value rotation (combine_inverse_rotate):
+ * M = max_s m_s, l = sum_s l_s e^(m_s - M), acc_m = sum_s acc_{s,m} e^(m_s - M),
+ * out = sum_m U_m acc_m / l (fp32). A sequence with no tokens yields zeros.
+ *   partials   : as written by omnikv_decode_attention with the same num_splits (0 resolves the same way)
+ *   out        : [batch][num_q_heads][128] fp32 */
+OMNIKV_API omnikv_status omnikv_combine(const omnikv_config* cfg, const omnikv_cache* cache,
+                             const void* partials, int32_t num_splits, float* out, void* stream);
+
+/* Static text for a status code. */
+OMNIKV_API const char* omnikv_status_string(omnikv_status status);
+
+/* OMNIKV_ABI_VERSION of the loaded library. */
+OMNIKV_API int32_t omnikv_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* OMNIKV_H_ */

@@ -1,0 +1,122 @@
+"""CPU-only checks of the C-ABI library: it loads, exports every function that
+include/omnikv.h declares, reports sizes, and rejects bad arguments on the host
+before launching anything (every call below fails validation, so no CUDA work
+is ever issued)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from bit_kv_cache_pack_b200 import _abi
+from bit_kv_cache_pack_b200._abi import OmniKVCache, OmniKVConfig
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", h)).read()
+            names += re.findall(r"OMNIKV_API\s+[\w\s\*]+?\b(omnikv_\w+)\s*\(", text)
+    return names
+
+
+def test_every_declared_symbol_is_exported():
+    names = _declared()
+    assert len(names) >= 8
+    lib = ctypes.CDLL(_abi._LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) >= set(_abi.EXPORTED)
+
+
+def test_sizes_and_version():
+    assert _abi.omnikv_abi_version() == 1
+    assert _abi.omnikv_record_bytes(2, 2) == 2624
+    assert _abi.omnikv_record_bytes(4, 4) == 4672
+    assert _abi.omnikv_record_bytes(2, 4) == 1024 + 512 + 2048 + 64
+    assert _abi.omnikv_record_bytes(3, 2) == 0
+    assert _abi.omnikv_partials_bytes(2, 16, 5) == 2 * 16 * 5 * 1544
+    assert _abi.omnikv_partials_bytes(0, 16, 5) == 0
+    assert _abi.status_string(_abi.OMNIKV_ERR_CAPACITY) == "cache capacity exceeded"
+
+
+FAKE = 0x10000  # 64 KiB-aligned fake device address; never dereferenced
+
+
+def _cfg(**kw):
+    c = OmniKVConfig(128, 16, 2, 32, 2, 2, FAKE, FAKE, FAKE, FAKE)
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+def _cache(**kw):
+    c = OmniKVCache(FAKE, FAKE, FAKE, FAKE, 0, 1, 2048, 0)
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+def _write_status(cfg, cache, n_new=1, k=FAKE, v=FAKE, mod=FAKE):
+    lib = _abi.load()
+    return lib.omnikv_write_cache(ctypes.byref(cfg), ctypes.byref(cache), k, v, mod, n_new, 0)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(head_dim=64), _abi.OMNIKV_ERR_UNSUPPORTED),
+    (dict(window=16), _abi.OMNIKV_ERR_UNSUPPORTED),
+    (dict(key_bits=3), _abi.OMNIKV_ERR_UNSUPPORTED),
+    (dict(value_bits=8), _abi.OMNIKV_ERR_UNSUPPORTED),
+    (dict(num_q_heads=15), _abi.OMNIKV_ERR_INVALID_ARG),
+    (dict(num_q_heads=32, num_kv_heads=2), _abi.OMNIKV_ERR_UNSUPPORTED),
+    (dict(num_kv_heads=0), _abi.OMNIKV_ERR_INVALID_ARG),
+    (dict(key_codebook=None), _abi.OMNIKV_ERR_INVALID_ARG),
+    (dict(value_rot=FAKE + 4), _abi.OMNIKV_ERR_INVALID_ARG),
+])
+def test_config_rejected(kw, want):
+    assert _write_status(_cfg(**kw), _cache()) == want
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(records=None), _abi.OMNIKV_ERR_INVALID_ARG),
+    (dict(records=FAKE + 8), _abi.OMNIKV_ERR_INVALID_ARG),
+    (dict(cap_tokens=100), _abi.OMNIKV_ERR_INVALID_ARG),
+    (dict(batch=0), _abi.OMNIKV_ERR_INVALID_ARG),
+    (dict(max_seq_len=4096), _abi.OMNIKV_ERR_INVALID_ARG),
+    (dict(max_seq_len=2048), _abi.OMNIKV_ERR_CAPACITY),
+    (dict(max_seq_len=2040), None),
+])
+def test_cache_rejected(kw, want):
+    if want is None:  # 2040 + 9 > 2048
+        assert _write_status(_cfg(), _cache(**kw), n_new=9) == _abi.OMNIKV_ERR_CAPACITY
+    else:
+        assert _write_status(_cfg(), _cache(**kw)) == want
+
+
+def test_write_arguments_rejected():
+    assert _write_status(_cfg(), _cache(), n_new=0) == _abi.OMNIKV_ERR_INVALID_ARG
+    assert _write_status(_cfg(), _cache(), k=None) == _abi.OMNIKV_ERR_INVALID_ARG
+    assert _write_status(_cfg(), _cache(), v=FAKE + 2) == _abi.OMNIKV_ERR_INVALID_ARG
+    assert _write_status(_cfg(), _cache(), mod=None) == _abi.OMNIKV_ERR_INVALID_ARG
+
+
+def test_decode_and_combine_arguments_rejected():
+    lib = _abi.load()
+    cfg, cache = _cfg(), _cache()
+    assert lib.omnikv_decode_attention(ctypes.byref(cfg), ctypes.byref(cache), None, FAKE, 0, 0) == \
+        _abi.OMNIKV_ERR_INVALID_ARG
+    assert lib.omnikv_decode_attention(ctypes.byref(cfg), ctypes.byref(cache), FAKE, FAKE + 4, 0, 0) == \
+        _abi.OMNIKV_ERR_INVALID_ARG
+    assert lib.omnikv_decode_attention(ctypes.byref(cfg), ctypes.byref(cache), FAKE, FAKE, -1, 0) == \
+        _abi.OMNIKV_ERR_INVALID_ARG
+    assert lib.omnikv_combine(ctypes.byref(cfg), ctypes.byref(cache), FAKE, 1, None, 0) == \
+        _abi.OMNIKV_ERR_INVALID_ARG
+    bad = _cfg(head_dim=256)
+    assert lib.omnikv_combine(ctypes.byref(bad), ctypes.byref(cache), FAKE, 1, FAKE, 0) == \
+        _abi.OMNIKV_ERR_UNSUPPORTED
+    assert lib.omnikv_default_splits(ctypes.byref(bad), ctypes.byref(cache)) == 0
+    with pytest.raises(_abi.OmniKVError):
+        _abi.omnikv_decode_attention(cfg, cache, None, FAKE)
