@@ -131,6 +131,7 @@ omnikv_status omnikv_decode_attention(const omnikv_config* cfg, const omnikv_cac
   p.q = static_cast<const __half*>(q);
   p.partials = static_cast<Partial*>(partials);
   p.num_splits = resolve_splits(cfg, cache, num_splits);
+  p.error_word = cache->error_word;
   if (launch_decode(p, cache->batch, static_cast<cudaStream_t>(stream)) != cudaSuccess) return OMNIKV_ERR_CUDA;
   return OMNIKV_OK;
 }

@@ -2,22 +2,67 @@
 //
 // paperpeel.com section 1 (last paragraph): the query is rotated once per head
 // instead of inverse-rotating every cached key, the cache is unpacked inside
-// attention in FlashAttention order (refs [4], [5]), and no dense fp16 cache
-// is built. One CTA per (split of the context, kv head, sequence); warp g owns
-// query head kvh * G + g and shares each staged window record with the other
-// query heads of its group (GQA). Per window: scores from the packed key codes
-// and the window's fp16 min / scale, an online softmax (running max and sum),
-// and one rotated-space accumulator per modality (values are stored in the
-// basis of their modality, so they are summed per modality and mapped back by
-// the combine kernel).
+// attention in FlashAttention order (refs [4], [5]), and no dense fp16 cache is
+// built. One CTA of 4 warps per (split of the context, kv head, sequence); all
+// query heads of the kv head (the GQA group, up to 8) are served by every load
+// of a window record.
+//
+// Tensor-core path (2-bit keys and values, symmetric codebook):
+//   * each warp streams its own windows (w0 + warp, w0 + warp + 4, ...) through
+//     a 4-stage shared-memory ring filled by 1-D bulk async copies (record +
+//     the window's 32 modality ids) completing on per-stage mbarriers;
+//   * scores use mma.sync m16n8k16 with the 8 query heads as N: the A operand
+//     (16 tokens x 16 channels) is built from the packed codes with one shift
+//     and one AND per register -- a code's low bit b0 lands on fp16 bit 13
+//     (value 2^-7 or 0) and its high bit b1 on bit 14 (value 2 or 0), exactly;
+//     with a symmetric codebook c_j - c_0 = (c_1 - c_0) b0 + (c_2 - c_0) b1, so
+//     two exact planes reproduce the codebook and the B operand carries
+//     q'_c s_gc (c_1 - c_0) * 128 and q'_c s_gc (c_2 - c_0) / 2 in fp16; the
+//     window minimum enters as the per-head offset sum_c q'_c m_gc;
+//   * online softmax per window (running max with exact rescale when it grows,
+//     per-lane partial sums reduced once at the end);
+//   * P (times the token's value scale sigma and the plane constants) becomes
+//     the B operand of the value product through movmatrix; values are stored
+//     channel-major so the A operand (16 channels x 16 tokens) again needs one
+//     shift and one AND per register; one fp32 accumulator set per modality
+//     (values of different modalities live in different rotated bases); the
+//     c_0 term is c_0 * sum_t p_t sigma_t per modality, added at the end;
+//   * the 4 warps merge (max, rescale, shared-memory reduction) and write one
+//     split-K partial per query head.
+// Token order inside a 16-token tile: fragment row / k-slot r holds token
+// tau(r) = r/2 + 8 (r%2) for r < 8 and 4 + (r-8)/2 + 8 (r%2) for r >= 8, so the
+// two tokens of every value-operand register (k-slots 2t, 2t+1 -> tokens t,
+// t+8) sit 16 bits apart in one channel-major code word.
+//
+// Generic path (4-bit codes, or a codebook that is not symmetric): a CUDA-core
+// loop with the same math (scores, online softmax, per-modality accumulators).
+//
+// Inputs must stay in the fp16 range of the operands: |q' s_gc| / sqrt(128)
+// below ~480 and value scales sigma below ~480; outside it the output is not
+// finite (the data would have to be far outside any realistic key / value range).
 #include "common.cuh"
 #include "kernels.h"
+#include "ptx.cuh"
 
 namespace omnikv {
 
 namespace {
 
-constexpr int kMaxRecordBytes = 4672;
+constexpr int kWarps = 4;
+constexpr int kThreads = 32 * kWarps;
+constexpr int kStages = 4;
+constexpr int kRec22 = 2624;                    // K2/V2 record bytes
+constexpr int kStageBytes = kRec22 + kWindow;   // record + modality ids
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: a bulk copy that takes longer is an error
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct __align__(16) DecodeSmem {
+  uint8_t stage[kWarps][kStages][kStageBytes];  // also reused by the generic path and the final merge
+  uint64_t bar[kWarps][kStages];
+  float q[kMaxGroup][kHeadDim];                 // rotated queries, times the softmax scale
+  float mw[kWarps][kMaxGroup];                  // per-warp running max, for the merge
+};
+static_assert(sizeof(DecodeSmem) <= 48 * 1024, "static shared memory");
 
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
@@ -31,57 +76,79 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-__global__ void __launch_bounds__(32 * kMaxGroup)
-decode_split_k_simt_kernel(const DecodeParams p) {
-  const int b = blockIdx.z;
-  const int kvh = blockIdx.y;
-  const int split = blockIdx.x;
+// Position of channel c of head g in the rotated-query buffer. Chunks of 4
+// channels inside each group of 32 are XOR-swizzled so that the 8 lanes of a
+// quarter warp (heads g, g+1 x channel groups t = 0..3) reading chunk i read 8
+// different bank groups.
+__device__ __forceinline__ int qpos(int g, int c) {
+  const int t = c >> 5, i4 = (c >> 2) & 7;
+  return g * kHeadDim + 32 * t + 4 * (i4 ^ ((4 * (g & 1) + t) & 7)) + (c & 3);
+}
+
+// q' = fp32(2^-3.5) H (s . q) for every head of the group, times 2^-3.5 more
+// (the softmax scale 1/sqrt(128)); heads >= G are zero. Stored at qpos(g, c).
+__device__ __forceinline__ void rotate_queries(const DecodeParams& p, int b, int kvh, float (*qs)[kHeadDim]) {
+  float* qflat = &qs[0][0];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.group;
-  const int g = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
   const int Hq = p.num_kv_heads * G;
-  const int qh = kvh * G + g;
+  float sg[4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) sg[r] = p.key_signs[4 * lane + r];
+  for (int g = warp; g < kMaxGroup; g += kWarps) {
+    if (g < G) {
+      const __half* q = p.q + ((size_t)b * Hq + kvh * G + g) * kHeadDim;
+      const uint2 raw = *reinterpret_cast<const uint2*>(q + 4 * lane);
+      const __half2 lo = *reinterpret_cast<const __half2*>(&raw.x);
+      const __half2 hi = *reinterpret_cast<const __half2*>(&raw.y);
+      float x[4] = {__low2float(lo), __high2float(lo), __low2float(hi), __high2float(hi)};
+      warp_hadamard_rotate(x, sg);
+#pragma unroll
+      for (int r = 0; r < 4; ++r) qflat[qpos(g, 4 * lane + r)] = x[r] * inv_sqrt_d();
+    } else {
+#pragma unroll
+      for (int r = 0; r < 4; ++r) qflat[qpos(g, 4 * lane + r)] = 0.0f;
+    }
+  }
+}
 
-  const int T = max(0, min(p.seq_lens[b], p.cap_tokens));
+__device__ __forceinline__ void split_range(const DecodeParams& p, int b, int split, int& T, int& w0, int& w1) {
+  T = max(0, min(p.seq_lens[b], p.cap_tokens));
   const int nw = (T + kWindow - 1) / kWindow;
-  const int w0 = (int)(((long long)split * nw) / p.num_splits);
-  const int w1 = (int)(((long long)(split + 1) * nw) / p.num_splits);
+  w0 = (int)(((long long)split * nw) / p.num_splits);
+  w1 = (int)(((long long)(split + 1) * nw) / p.num_splits);
+}
 
+// ---------------------------------------------------------------------------
+// generic CUDA-core path: warp w owns query heads w and w + 4 of the group
+// ---------------------------------------------------------------------------
+__device__ void decode_generic(const DecodeParams& p, DecodeSmem& sm, int b, int kvh, int split) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = p.group;
+  const int Hq = p.num_kv_heads * G;
+  int T, w0, w1;
+  split_range(p, b, split, T, w0, w1);
   const RecordLayout lay(p.key_bits, p.value_bits);
-  __shared__ __align__(16) uint8_t rec[kMaxRecordBytes];
-  __shared__ __align__(16) uint8_t mods[kWindow];
-  __shared__ float qs[kMaxGroup][kHeadDim];
-  __shared__ float cbk[16], cbv[16];
-
+  uint8_t* rec = &sm.stage[0][0][0];
+  uint8_t* mods = rec + 4672;
+  float* cbk = reinterpret_cast<float*>(rec + 4672 + 32);
+  float* cbv = cbk + 16;
   if (threadIdx.x < (1 << p.key_bits)) cbk[threadIdx.x] = p.key_cb[threadIdx.x];
   if (threadIdx.x < (1 << p.value_bits)) cbv[threadIdx.x] = p.val_cb[threadIdx.x];
-
-  // q' = fp32(2^-3.5) H (s . q), then the softmax scale 1/sqrt(128)
-  {
-    const __half* q = p.q + ((size_t)b * Hq + qh) * kHeadDim;
-    const uint2 raw = *reinterpret_cast<const uint2*>(q + 4 * lane);
-    const __half2 lo = *reinterpret_cast<const __half2*>(&raw.x);
-    const __half2 hi = *reinterpret_cast<const __half2*>(&raw.y);
-    float x[4] = {__low2float(lo), __high2float(lo), __low2float(hi), __high2float(hi)};
-    float sg[4];
-#pragma unroll
-    for (int r = 0; r < 4; ++r) sg[r] = p.key_signs[4 * lane + r];
-    warp_hadamard_rotate(x, sg);
-#pragma unroll
-    for (int r = 0; r < 4; ++r) qs[g][4 * lane + r] = x[r] * inv_sqrt_d();
-  }
 
   const int kcpw = 32 / p.key_bits, kwpt = kHeadDim / kcpw;
   const uint32_t kmask = (1u << p.key_bits) - 1u;
   const int vcpw = 32 / p.value_bits;
   const uint32_t vmask = (1u << p.value_bits) - 1u;
 
-  float m_run = -INFINITY, l_run = 0.0f;
-  float acc[kMods][4];
+  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.0f, 0.0f};
+  float acc[2][kMods][4];
 #pragma unroll
-  for (int m = 0; m < kMods; ++m)
+  for (int k = 0; k < 2; ++k)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) acc[m][j] = 0.0f;
+    for (int m = 0; m < kMods; ++m)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[k][m][j] = 0.0f;
 
   const uint8_t* rec_base = p.records + ((size_t)(b * p.num_kv_heads + kvh) * p.cap_windows) * lay.bytes;
   for (int w = w0; w < w1; ++w) {
@@ -95,70 +162,445 @@ decode_split_k_simt_kernel(const DecodeParams p) {
             reinterpret_cast<const uint4*>(p.modality + (size_t)b * p.cap_tokens + w * kWindow)[threadIdx.x];
     }
     __syncthreads();
-
     const int nvalid = min(kWindow, T - w * kWindow);
     const uint32_t* kw = reinterpret_cast<const uint32_t*>(rec + lay.k_off);
     const __half2* meta = reinterpret_cast<const __half2*>(rec + lay.meta_off);
     const uint32_t* vw = reinterpret_cast<const uint32_t*>(rec + lay.v_off);
     const __half* sig = reinterpret_cast<const __half*>(rec + lay.sigma_off);
-
-    // scores: lane = token of the window
-    float sc = 0.0f;
     const float c0 = cbk[0];
+    // scores: lane = token; both heads of this warp share the dequantised key
+    float sc[2] = {0.0f, 0.0f};
     for (int c = 0; c < kHeadDim; ++c) {
       const uint32_t code = (kw[lane * kwpt + c / kcpw] >> (p.key_bits * (c % kcpw))) & kmask;
       const float2 ms = __half22float2(meta[c]);
       const float kval = ms.x + ms.y * (cbk[code] - c0);
-      sc = fmaf(qs[g][c], kval, sc);
+      sc[0] = fmaf((&sm.q[0][0])[qpos(warp, c)], kval, sc[0]);
+      sc[1] = fmaf((&sm.q[0][0])[qpos(warp + kWarps, c)], kval, sc[1]);
     }
-    if (lane >= nvalid) sc = -INFINITY;
-    const float m_new = fmaxf(m_run, warp_max(sc));
-    const float alpha = expf(m_run - m_new);
-    const float pt = lane < nvalid ? expf(sc - m_new) : 0.0f;
-    l_run = l_run * alpha + warp_sum(pt);
+    float pt[2];
 #pragma unroll
-    for (int m = 0; m < kMods; ++m)
+    for (int k = 0; k < 2; ++k) {
+      if (lane >= nvalid) sc[k] = -INFINITY;
+      const float m_new = fmaxf(m_run[k], warp_max(sc[k]));
+      const float alpha = expf(m_run[k] - m_new);
+      pt[k] = lane < nvalid ? expf(sc[k] - m_new) : 0.0f;
+      l_run[k] = l_run[k] * alpha + warp_sum(pt[k]);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) acc[m][j] *= alpha;
-    m_run = m_new;
-
-    // per-modality rotated-space values: lane = channels lane + 32 j
+      for (int m = 0; m < kMods; ++m)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[k][m][j] *= alpha;
+      m_run[k] = m_new;
+    }
     for (int t = 0; t < nvalid; ++t) {
-      const float wt = __shfl_sync(0xffffffffu, pt, t) * __half2float(sig[t]);
+      const float s = __half2float(sig[t]);
+      const float wt0 = __shfl_sync(0xffffffffu, pt[0], t) * s;
+      const float wt1 = __shfl_sync(0xffffffffu, pt[1], t) * s;
       const int mod = mods[t];
       const uint32_t* vrow = vw + (t / vcpw) * kHeadDim;
       const int sh = p.value_bits * (t % vcpw);
       float val[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) val[j] = wt * cbv[(vrow[lane + 32 * j] >> sh) & vmask];
-      if (mod == 0) {
+      for (int j = 0; j < 4; ++j) val[j] = cbv[(vrow[lane + 32 * j] >> sh) & vmask];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[0][j] += val[j];
-      } else if (mod == 1) {
+      for (int m = 0; m < kMods; ++m) {
+        if (mod == m || (m == kMods - 1 && mod > m)) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[1][j] += val[j];
-      } else {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[2][j] += val[j];
+          for (int j = 0; j < 4; ++j) {
+            acc[0][m][j] = fmaf(wt0, val[j], acc[0][m][j]);
+            acc[1][m][j] = fmaf(wt1, val[j], acc[1][m][j]);
+          }
+        }
       }
     }
   }
-  Partial* out = p.partials + ((size_t)b * Hq + qh) * p.num_splits + split;
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int g = warp + kWarps * k;
+    if (g >= G) continue;
+    Partial* out = p.partials + ((size_t)b * Hq + kvh * G + g) * p.num_splits + split;
+#pragma unroll
+    for (int m = 0; m < kMods; ++m)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) out->acc[m][lane + 32 * j] = acc[k][m][j];
+    if (lane == 0) {
+      out->m = m_run[k];
+      out->l = l_run[k];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// tensor-core path (K2/V2, symmetric codebooks)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int tile_token(int r) {  // tau(r), r in 0..15
+  return r < 8 ? (r >> 1) + 8 * (r & 1) : 4 + ((r - 8) >> 1) + 8 * (r & 1);
+}
+
+constexpr uint32_t kPlane0 = 0x20002000u;  // bit 13 of each half: 2^-7
+constexpr uint32_t kPlane1 = 0x40004000u;  // bit 14 of each half: 2
+
+__device__ __forceinline__ uint32_t rotl(uint32_t x, int n) { return __funnelshift_l(x, x, n); }
+
+struct WarpState {
+  float m[2];           // running max for heads 2t, 2t+1 (warp-uniform per column)
+  float l[2];           // per-lane partial sum of p for heads 2t, 2t+1
+  float S[kMods][2];    // per-lane partial sum of p * sigma per modality
+  float acc[kMods][8][4];
+};
+
+__device__ __forceinline__ void issue_window(const DecodeParams& p, DecodeSmem& sm, int warp, int stage,
+                                             const uint8_t* rec_base, int b, int wi) {
+  uint64_t* bar = &sm.bar[warp][stage];
+  uint8_t* dst = &sm.stage[warp][stage][0];
+  mbar_arrive_expect_tx(bar, kStageBytes);
+  bulk_copy_g2s(dst, rec_base + (size_t)wi * kRec22, kRec22, bar);
+  bulk_copy_g2s(dst + kRec22, p.modality + (size_t)b * p.cap_tokens + (size_t)wi * kWindow, kWindow, bar);
+}
+
+__device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh, int split, float kK0, float kK1,
+                           float kV0, float kV1, float vc0) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int G = p.group;
+  const int Hq = p.num_kv_heads * G;
+  int T, w0, w1;
+  split_range(p, b, split, T, w0, w1);
+  const uint8_t* rec_base = p.records + ((size_t)(b * p.num_kv_heads + kvh) * p.cap_windows) * kRec22;
+  const int nmine = (w1 - w0 > warp) ? (w1 - w0 - warp + kWarps - 1) / kWarps : 0;
+
+  if (lane == 0) {
+#pragma unroll
+    for (int s = 0; s < kStages; ++s) mbar_init(&sm.bar[warp][s], 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
+  if (lane == 0)
+    for (int i = 0; i < kStages && i < nmine; ++i) issue_window(p, sm, warp, i, rec_base, b, w0 + warp + kWarps * i);
+
+  WarpState st;
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    st.m[j] = -INFINITY;
+    st.l[j] = 0.0f;
+#pragma unroll
+    for (int m = 0; m < kMods; ++m) st.S[m][j] = 0.0f;
+  }
 #pragma unroll
   for (int m = 0; m < kMods; ++m)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) out->acc[m][lane + 32 * j] = acc[m][j];
-  if (lane == 0) {
-    out->m = m_run;
-    out->l = l_run;
+    for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) st.acc[m][mt][r] = 0.0f;
+
+  int failed_at = -1;
+  for (int i = 0; i < nmine; ++i) {
+    const int s = i % kStages;
+    const int wi = w0 + warp + kWarps * i;
+    if (!mbar_wait_bounded(&sm.bar[warp][s], (i / kStages) & 1, kWaitLimitNs)) {
+      failed_at = i;
+      break;
+    }
+    const uint8_t* stg = &sm.stage[warp][s][0];
+    const uint32_t* kw = reinterpret_cast<const uint32_t*>(stg);
+    const __half2* meta = reinterpret_cast<const __half2*>(stg + 1024);
+    const uint32_t* vw = reinterpret_cast<const uint32_t*>(stg + 1536);
+    const __half* sig = reinterpret_cast<const __half*>(stg + 2560);
+    const uint8_t* mods = stg + kRec22;
+
+    // ---- per-window B operand of the score product: head g, channels 32t .. 32t+31
+    uint32_t B0[8][2], B1[8][2];
+    float off;
+    {
+      const float* qrow = &sm.q[g][32 * t];
+      const int qsw = (4 * (g & 1) + t) & 7;
+      const uint4* mv4 = reinterpret_cast<const uint4*>(meta + 32 * t);
+      float x[32];
+      off = 0.0f;
+#pragma unroll
+      for (int i4 = 0; i4 < 8; ++i4) {
+        const float4 qq = *reinterpret_cast<const float4*>(qrow + 4 * (i4 ^ qsw));
+        const uint4 mm = mv4[i4];
+        const float qa[4] = {qq.x, qq.y, qq.z, qq.w};
+        const uint32_t ma[4] = {mm.x, mm.y, mm.z, mm.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 ms = __half22float2(*reinterpret_cast<const __half2*>(&ma[j]));
+          off = fmaf(qa[j], ms.x, off);
+          x[4 * i4 + j] = qa[j] * ms.y;
+        }
+      }
+#pragma unroll
+      for (int kc = 0; kc < 8; ++kc) {
+        B0[kc][0] = pack_half2(x[kc] * kK0, x[kc + 8] * kK0);
+        B0[kc][1] = pack_half2(x[kc + 16] * kK0, x[kc + 24] * kK0);
+        B1[kc][0] = pack_half2(x[kc] * kK1, x[kc + 8] * kK1);
+        B1[kc][1] = pack_half2(x[kc + 16] * kK1, x[kc + 24] * kK1);
+      }
+      off += __shfl_xor_sync(0xffffffffu, off, 1);
+      off += __shfl_xor_sync(0xffffffffu, off, 2);
+    }
+    const float off0 = __shfl_sync(0xffffffffu, off, 8 * t);      // head 2t
+    const float off1 = __shfl_sync(0xffffffffu, off, 8 * t + 4);  // head 2t + 1
+
+    // ---- scores for the two 16-token tiles
+    float sc[2][4];
+    int tokA[2], tokB[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      tokA[h] = 16 * h + tile_token(g);
+      tokB[h] = 16 * h + tile_token(g + 8);
+      const uint2 kA = *reinterpret_cast<const uint2*>(kw + tokA[h] * 8 + 2 * t);
+      const uint2 kB = *reinterpret_cast<const uint2*>(kw + tokB[h] * 8 + 2 * t);
+      float d0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, d1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+      for (int kc = 0; kc < 8; ++kc) {
+        uint32_t r[4];
+        if (kc < 7) {
+          r[0] = kA.x << (13 - 2 * kc);
+          r[1] = kB.x << (13 - 2 * kc);
+          r[2] = kA.y << (13 - 2 * kc);
+          r[3] = kB.y << (13 - 2 * kc);
+        } else {
+          r[0] = kA.x >> 1;
+          r[1] = kB.x >> 1;
+          r[2] = kA.y >> 1;
+          r[3] = kB.y >> 1;
+        }
+        const uint32_t a0[4] = {r[0] & kPlane0, r[1] & kPlane0, r[2] & kPlane0, r[3] & kPlane0};
+        const uint32_t a1[4] = {r[0] & kPlane1, r[1] & kPlane1, r[2] & kPlane1, r[3] & kPlane1};
+        mma_f16_16816(d0, a0, B0[kc][0], B0[kc][1]);
+        mma_f16_16816(d1, a1, B1[kc][0], B1[kc][1]);
+      }
+      const int posA = wi * kWindow + tokA[h], posB = wi * kWindow + tokB[h];
+      sc[h][0] = posA < T ? d0[0] + d1[0] + off0 : -INFINITY;
+      sc[h][1] = posA < T ? d0[1] + d1[1] + off1 : -INFINITY;
+      sc[h][2] = posB < T ? d0[2] + d1[2] + off0 : -INFINITY;
+      sc[h][3] = posB < T ? d0[3] + d1[3] + off1 : -INFINITY;
+    }
+
+    // ---- online softmax over the window
+    float mx0 = fmaxf(fmaxf(sc[0][0], sc[0][2]), fmaxf(sc[1][0], sc[1][2]));
+    float mx1 = fmaxf(fmaxf(sc[0][1], sc[0][3]), fmaxf(sc[1][1], sc[1][3]));
+#pragma unroll
+    for (int o = 4; o <= 16; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+    }
+    const float mn0 = fmaxf(st.m[0], mx0), mn1 = fmaxf(st.m[1], mx1);
+    if (__any_sync(0xffffffffu, mn0 > st.m[0] || mn1 > st.m[1])) {
+      const float a0 = exp2f((st.m[0] - mn0) * kLog2e), a1 = exp2f((st.m[1] - mn1) * kLog2e);
+      st.l[0] *= a0;
+      st.l[1] *= a1;
+#pragma unroll
+      for (int m = 0; m < kMods; ++m) {
+        st.S[m][0] *= a0;
+        st.S[m][1] *= a1;
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          st.acc[m][mt][0] *= a0;
+          st.acc[m][mt][1] *= a1;
+          st.acc[m][mt][2] *= a0;
+          st.acc[m][mt][3] *= a1;
+        }
+      }
+      st.m[0] = mn0;
+      st.m[1] = mn1;
+    }
+    const float ms0 = st.m[0] * kLog2e, ms1 = st.m[1] * kLog2e;
+
+    // ---- value product per tile
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float p0 = exp2f(fmaf(sc[h][0], kLog2e, -ms0));
+      const float p1 = exp2f(fmaf(sc[h][1], kLog2e, -ms1));
+      const float p2 = exp2f(fmaf(sc[h][2], kLog2e, -ms0));
+      const float p3 = exp2f(fmaf(sc[h][3], kLog2e, -ms1));
+      st.l[0] += p0 + p2;
+      st.l[1] += p1 + p3;
+      const float sgA = __half2float(sig[tokA[h]]), sgB = __half2float(sig[tokB[h]]);
+      const float w0v = p0 * sgA, w1v = p1 * sgA, w2v = p2 * sgB, w3v = p3 * sgB;
+      const uint32_t bv0[2] = {movmatrix_trans(pack_half2(w0v * kV0, w1v * kV0)),
+                               movmatrix_trans(pack_half2(w2v * kV0, w3v * kV0))};
+      const uint32_t bv1[2] = {movmatrix_trans(pack_half2(w0v * kV1, w1v * kV1)),
+                               movmatrix_trans(pack_half2(w2v * kV1, w3v * kV1))};
+      // modalities of this tile (warp-uniform mask) and of this lane's tokens
+      const int mA = mods[tokA[h]], mB = mods[tokB[h]];
+      const uint32_t mbits = __reduce_or_sync(0xffffffffu, (1u << min(mA, 2)) | (1u << min(mB, 2)));
+      // V words of channels 16g .. 16g+15 for this tile's 16 tokens
+      uint32_t vwd[16];
+      {
+        const uint4* src = reinterpret_cast<const uint4*>(vw + h * kHeadDim + 16 * g);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const uint4 u = src[q4];
+          vwd[4 * q4 + 0] = u.x;
+          vwd[4 * q4 + 1] = u.y;
+          vwd[4 * q4 + 2] = u.z;
+          vwd[4 * q4 + 3] = u.w;
+        }
+      }
+      const int rlo = 13 - 2 * t, rhi = (5 - 2 * t) & 31;
+      if ((mbits & (mbits - 1)) == 0) {  // one modality in the tile
+        const int m = __ffs(mbits) - 1;
+#pragma unroll
+        for (int mm = 0; mm < kMods; ++mm) {
+          if (mm != m) continue;
+          st.S[mm][0] += w0v + w2v;
+          st.S[mm][1] += w1v + w3v;
+#pragma unroll
+          for (int mt = 0; mt < 8; ++mt) {
+            const uint32_t wg = vwd[2 * mt], wg8 = vwd[2 * mt + 1];
+            const uint32_t r[4] = {rotl(wg, rlo), rotl(wg8, rlo), rotl(wg, rhi), rotl(wg8, rhi)};
+            const uint32_t a0[4] = {r[0] & kPlane0, r[1] & kPlane0, r[2] & kPlane0, r[3] & kPlane0};
+            const uint32_t a1[4] = {r[0] & kPlane1, r[1] & kPlane1, r[2] & kPlane1, r[3] & kPlane1};
+            mma_f16_16816(st.acc[mm][mt], a0, bv0[0], bv0[1]);
+            mma_f16_16816(st.acc[mm][mt], a1, bv1[0], bv1[1]);
+          }
+        }
+      } else {  // mixed tile: one masked product per modality present
+        // k-slots of this lane's B registers: 2t, 2t+1 -> tokens t, t+8; 2t+8, 2t+9 -> t+4, t+12
+        const int base = 16 * h;
+        const int mk0 = min((int)mods[base + t], 2), mk1 = min((int)mods[base + t + 8], 2);
+        const int mk2 = min((int)mods[base + t + 4], 2), mk3 = min((int)mods[base + t + 12], 2);
+#pragma unroll
+        for (int mm = 0; mm < kMods; ++mm) {
+          if (!(mbits & (1u << mm))) continue;
+          const uint32_t msk01 = (mk0 == mm ? 0x0000FFFFu : 0u) | (mk1 == mm ? 0xFFFF0000u : 0u);
+          const uint32_t msk23 = (mk2 == mm ? 0x0000FFFFu : 0u) | (mk3 == mm ? 0xFFFF0000u : 0u);
+          const uint32_t b00 = bv0[0] & msk01, b01 = bv0[1] & msk23;
+          const uint32_t b10 = bv1[0] & msk01, b11 = bv1[1] & msk23;
+          st.S[mm][0] += (min(mA, 2) == mm ? w0v : 0.0f) + (min(mB, 2) == mm ? w2v : 0.0f);
+          st.S[mm][1] += (min(mA, 2) == mm ? w1v : 0.0f) + (min(mB, 2) == mm ? w3v : 0.0f);
+#pragma unroll
+          for (int mt = 0; mt < 8; ++mt) {
+            const uint32_t wg = vwd[2 * mt], wg8 = vwd[2 * mt + 1];
+            const uint32_t r[4] = {rotl(wg, rlo), rotl(wg8, rlo), rotl(wg, rhi), rotl(wg8, rhi)};
+            const uint32_t a0[4] = {r[0] & kPlane0, r[1] & kPlane0, r[2] & kPlane0, r[3] & kPlane0};
+            const uint32_t a1[4] = {r[0] & kPlane1, r[1] & kPlane1, r[2] & kPlane1, r[3] & kPlane1};
+            mma_f16_16816(st.acc[mm][mt], a0, b00, b01);
+            mma_f16_16816(st.acc[mm][mt], a1, b10, b11);
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0 && i + kStages < nmine) {
+      fence_proxy_async_smem();
+      issue_window(p, sm, warp, s, rec_base, b, w0 + warp + kWarps * (i + kStages));
+    }
   }
+
+  if (__any_sync(0xffffffffu, failed_at >= 0)) {
+    // a copy did not complete in time: report it, wait (bounded) for the copies
+    // still in flight (windows failed_at .. failed_at + kStages - 1), give up
+    const int f = __shfl_sync(0xffffffffu, failed_at, 0);
+    if (lane == 0) set_error(p.error_word, OMNIKV_DEVERR_TIMEOUT);
+    for (int j = f; j < nmine && j < f + kStages; ++j)
+      mbar_wait_bounded(&sm.bar[warp][j % kStages], (j / kStages) & 1, kWaitLimitNs);
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      st.m[j] = -INFINITY;
+      st.l[j] = 0.0f;
+    }
+  }
+
+  // ---- reduce the per-lane partial sums over the 8 lanes sharing a column
+#pragma unroll
+  for (int o = 4; o <= 16; o <<= 1) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      st.l[j] += __shfl_xor_sync(0xffffffffu, st.l[j], o);
+#pragma unroll
+      for (int m = 0; m < kMods; ++m) st.S[m][j] += __shfl_xor_sync(0xffffffffu, st.S[m][j], o);
+    }
+  }
+  // c_0 term of the value codebook
+#pragma unroll
+  for (int m = 0; m < kMods; ++m)
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      st.acc[m][mt][0] += vc0 * st.S[m][0];
+      st.acc[m][mt][1] += vc0 * st.S[m][1];
+      st.acc[m][mt][2] += vc0 * st.S[m][0];
+      st.acc[m][mt][3] += vc0 * st.S[m][1];
+    }
+
+  // ---- merge the 4 warps: max, rescale, shared-memory reduction ------------
+  if (g == 0) {
+    sm.mw[warp][2 * t] = st.m[0];
+    sm.mw[warp][2 * t + 1] = st.m[1];
+  }
+  __syncthreads();  // all warps are done with their stage buffers
+  float* macc = reinterpret_cast<float*>(&sm.stage[0][0][0]);  // [3][8][128]
+  float* ml = macc + kMods * kMaxGroup * kHeadDim;              // [8]
+  for (int i = threadIdx.x; i < kMods * kMaxGroup * kHeadDim + kMaxGroup; i += kThreads) macc[i] = 0.0f;
+  __syncthreads();
+  float sc2[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const int hcol = 2 * t + j;
+    float mm = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) mm = fmaxf(mm, sm.mw[w][hcol]);
+    sc2[j] = (st.m[j] == -INFINITY) ? 0.0f : exp2f((st.m[j] - mm) * kLog2e);
+  }
+  if (g == 0) {
+    atomicAdd(&ml[2 * t], st.l[0] * sc2[0]);
+    atomicAdd(&ml[2 * t + 1], st.l[1] * sc2[1]);
+  }
+#pragma unroll
+  for (int m = 0; m < kMods; ++m)
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      const int c0 = 16 * g + 2 * mt;  // row g -> channel 16g + 2mt, row g + 8 -> + 1
+      float* base = macc + (size_t)m * kMaxGroup * kHeadDim;
+      atomicAdd(&base[(2 * t) * kHeadDim + c0], st.acc[m][mt][0] * sc2[0]);
+      atomicAdd(&base[(2 * t + 1) * kHeadDim + c0], st.acc[m][mt][1] * sc2[1]);
+      atomicAdd(&base[(2 * t) * kHeadDim + c0 + 1], st.acc[m][mt][2] * sc2[0]);
+      atomicAdd(&base[(2 * t + 1) * kHeadDim + c0 + 1], st.acc[m][mt][3] * sc2[1]);
+    }
+  __syncthreads();
+  // ---- write one partial per query head of the group
+  for (int hh = warp; hh < G; hh += kWarps) {
+    Partial* out = p.partials + ((size_t)b * Hq + kvh * G + hh) * p.num_splits + split;
+#pragma unroll
+    for (int m = 0; m < kMods; ++m)
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        out->acc[m][lane + 32 * j] = macc[((size_t)m * kMaxGroup + hh) * kHeadDim + lane + 32 * j];
+    if (lane == 0) {
+      float mm = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) mm = fmaxf(mm, sm.mw[w][hh]);
+      out->m = mm;
+      out->l = ml[hh];
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 2) decode_split_k_kernel(const DecodeParams p) {
+  __shared__ DecodeSmem sm;
+  const int b = blockIdx.z, kvh = blockIdx.y, split = blockIdx.x;
+  rotate_queries(p, b, kvh, sm.q);
+  __syncthreads();
+  if (p.key_bits == 2 && p.value_bits == 2) {
+    const float k0 = p.key_cb[0], k1 = p.key_cb[1], k2 = p.key_cb[2], k3 = p.key_cb[3];
+    const float v0 = p.val_cb[0], v1 = p.val_cb[1], v2 = p.val_cb[2], v3 = p.val_cb[3];
+    const bool symmetric = (k0 == -k3) && (k1 == -k2) && (v0 == -v3) && (v1 == -v2);
+    if (symmetric) {
+      decode_mma(p, sm, b, kvh, split, (k1 - k0) * 128.0f, (k2 - k0) * 0.5f, (v1 - v0) * 128.0f,
+                 (v2 - v0) * 0.5f, v0);
+      return;
+    }
+  }
+  decode_generic(p, sm, b, kvh, split);
 }
 
 }  // namespace
 
 cudaError_t launch_decode(const DecodeParams& p, int batch, cudaStream_t stream) {
   dim3 grid(p.num_splits, p.num_kv_heads, batch);
-  decode_split_k_simt_kernel<<<grid, 32 * p.group, 0, stream>>>(p);
+  decode_split_k_kernel<<<grid, kThreads, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -39,6 +39,7 @@ struct DecodeParams {
   const __half* q;
   Partial* partials;
   int num_splits;
+  int32_t* error_word;
 };
 
 struct CombineParams {

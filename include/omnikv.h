@@ -78,6 +78,8 @@ typedef enum {
 /* Device error word bits (omnikv_cache.error_word). */
 #define OMNIKV_DEVERR_CAPACITY 0x1 /* a write would have passed cap_tokens; that sequence was skipped */
 #define OMNIKV_DEVERR_MODALITY 0x2 /* a modality id was > 2; it was stored and used as 2 (video) */
+#define OMNIKV_DEVERR_TIMEOUT 0x4  /* a staged copy did not complete within its wait limit; outputs of that
+                                      CTA are zero (never expected; the kernel returns instead of hanging) */
 
 /* Per-layer constants. All pointers are device pointers. */
 typedef struct {

@@ -167,3 +167,52 @@ def test_device_capacity_check_sets_error_word(cuda_device):
     assert int(gc.error_word.item()) & m.OMNIKV_DEVERR_CAPACITY
     assert int(gc.seq_lens.item()) == 60
     assert int(gc.records.sum().item()) == 0
+
+
+def test_asymmetric_codebook_uses_generic_path(cuda_device):
+    """A 2-bit codebook that is not symmetric takes the CUDA-core path inside
+    the same kernel; results still match the oracle."""
+    import dataclasses
+    m = _abi()
+    spec, seed = CONFIGS[0], 8
+    params, consts, ocfg = make_layer(spec, seed, 0, cuda_device)
+    cb = np.array([-1.2, -0.3, 0.5, 1.7], np.float32)
+    consts = m.LayerConstants(cb, cb, params["key_signs"], params["value_rot"], spec.num_q_heads, cuda_device)
+    ocfg = dataclasses.replace(ocfg, key_codebook=cb, value_codebook=cb)
+    L = np.array([500], np.int32)
+    drift = key_drift(spec, seed, 0, 16, cuda_device)
+    k, v, mod = prefill_inputs(spec, seed, 0, params, drift, L, cuda_device)
+    gc = m.KVCache(1, 2, 512, 2, 2, cuda_device)
+    oc = codec.OracleCache(1, 2, 512, 2, 2)
+    _write_both(consts, ocfg, gc, oc, k, v, mod)
+    _check_state(ocfg, oc, gc, v.cpu().numpy(), mod.cpu().numpy())
+    q = torch.randn(1, 16, 128, device=cuda_device).half()
+    ref = decode_dense(ocfg, oc, q.cpu().numpy())
+    check_decode(gpu_decode(consts, upload_oracle_cache(oc, cuda_device), q, 3), ref, "asymmetric")
+
+
+@pytest.mark.parametrize("G,hkv", [(1, 4), (4, 2), (8, 1)])
+def test_group_sizes(cuda_device, G, hkv):
+    """GQA groups smaller than 8 leave tensor-core columns unused; every group
+    size up to 8 must match the oracle."""
+    import dataclasses
+    m = _abi()
+    spec = dataclasses.replace(CONFIGS[0], num_q_heads=G * hkv, num_kv_heads=hkv)
+    seed = 9
+    params, consts, ocfg = make_layer(spec, seed, 0, cuda_device, per_head=True)
+    L = np.array([333, 70], np.int32)
+    spec2 = dataclasses.replace(spec, batch=2)
+    drift = key_drift(spec2, seed, 0, 16, cuda_device)
+    k, v, mod = prefill_inputs(spec2, seed, 0, params, drift, np.array([333, 333]), cuda_device)
+    oc = codec.OracleCache(2, hkv, 352, 2, 2)
+    for b in range(2):
+        sub = codec.OracleCache(1, hkv, 352, 2, 2)
+        n = int(L[b])
+        codec.write_cache(ocfg, sub, k[b:b + 1, :, :n].cpu().numpy(), v[b:b + 1, :, :n].cpu().numpy(),
+                          mod[b:b + 1, :n].cpu().numpy())
+        oc.records[b], oc.key_tail[b], oc.modality[b], oc.seq_lens[b] = (
+            sub.records[0], sub.key_tail[0], sub.modality[0], sub.seq_lens[0])
+    q = torch.randn(2, G * hkv, 128, device=cuda_device).half()
+    ref = decode_dense(ocfg, oc, q.cpu().numpy())
+    for S in (1, 4):
+        check_decode(gpu_decode(consts, upload_oracle_cache(oc, cuda_device), q, S), ref, "G=%d S=%d" % (G, S))
