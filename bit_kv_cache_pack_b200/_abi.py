@@ -22,6 +22,7 @@ OMNIKV_ERR_DEVICE_CHECK = 5
 OMNIKV_DEVERR_CAPACITY = 0x1
 OMNIKV_DEVERR_MODALITY = 0x2
 OMNIKV_DEVERR_TIMEOUT = 0x4
+OMNIKV_DEVERR_BOUND = 0x8
 
 EXPORTED = (
     "omnikv_record_bytes", "omnikv_partials_bytes", "omnikv_default_splits",

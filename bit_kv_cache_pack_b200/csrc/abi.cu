@@ -46,13 +46,15 @@ int32_t resolve_splits(const omnikv_config* cfg, const omnikv_cache* c, int32_t 
   if (requested > 0) return requested;
   const int nw = (c->max_seq_len + kWindow - 1) / kWindow;
   if (nw <= 0) return 1;
+  // aim at about two resident CTAs per SM over the whole batch, with at least
+  // 8 windows (2 per warp) per split so the per-CTA setup is amortised
   const long long units = (long long)c->batch * cfg->num_kv_heads;
   const long long target = 2LL * sm_count();
-  long long s = (target + units - 1) / units;
-  // keep at least a few windows per split so the per-CTA setup is amortised
-  const long long max_s = (nw + 3) / 4;
+  long long s = target / units;
+  const long long max_s = (nw + 7) / 8;
   if (s > max_s) s = max_s;
   if (s < 1) s = 1;
+  if (s > kMaxSplits) s = kMaxSplits;
   return (int32_t)s;
 }
 
@@ -131,6 +133,11 @@ omnikv_status omnikv_decode_attention(const omnikv_config* cfg, const omnikv_cac
   p.q = static_cast<const __half*>(q);
   p.partials = static_cast<Partial*>(partials);
   p.num_splits = resolve_splits(cfg, cache, num_splits);
+  if (p.num_splits > kMaxSplits) return OMNIKV_ERR_UNSUPPORTED;
+  {
+    const int nw = (cache->max_seq_len + kWindow - 1) / kWindow;
+    p.split_windows = nw > 0 ? (nw + p.num_splits - 1) / p.num_splits : 1;
+  }
   p.error_word = cache->error_word;
   if (launch_decode(p, cache->batch, static_cast<cudaStream_t>(stream)) != cudaSuccess) return OMNIKV_ERR_CUDA;
   return OMNIKV_OK;
@@ -149,6 +156,7 @@ omnikv_status omnikv_combine(const omnikv_config* cfg, const omnikv_cache* cache
   p.group = cfg->num_q_heads / cfg->num_kv_heads;
   p.partials = static_cast<const Partial*>(partials);
   p.num_splits = resolve_splits(cfg, cache, num_splits);
+  if (p.num_splits > kMaxSplits) return OMNIKV_ERR_UNSUPPORTED;
   p.out = out;
   if (launch_combine(p, cache->batch, static_cast<cudaStream_t>(stream)) != cudaSuccess) return OMNIKV_ERR_CUDA;
   return OMNIKV_OK;

@@ -1,12 +1,14 @@
 // combine_inverse_rotate: merges the split-K partials of decode_split_k and
-// applies the inverse value rotations, batched across the query heads of a kv
-// head (paperpeel.com section 1: inverse value rotations are batched across
-// head outputs instead of applied per cached value).
+// applies the inverse value rotations (paperpeel.com section 1: inverse value
+// rotations are applied to head outputs instead of to every cached value).
 //
-// Per (sequence, kv head): M = max_s m_s, l = sum_s l_s e^(m_s - M),
-// a_m = sum_s acc_{s,m} e^(m_s - M) / l, then out = sum_m U_m a_m for the G
-// query heads at once, i.e. the [G x 384] x [384 x 128] product with the
-// stacked bases.
+// One CTA per (query head, kv head, sequence):
+//   1. warp 0: M = max_s m_s, weights e_s = exp(m_s - M), l = sum_s l_s e_s;
+//   2. all threads: a_m[c] = sum_s acc_{s,m}[c] e_s / l, the splits read as
+//      16-byte vectors, two threads per vector column;
+//   3. out[j] = sum_m sum_c U_m[j][c] a_m[c]: one warp per output row, lanes over
+//      c (coalesced rows of U_m), warp reduction.
+// A sequence without tokens (all m_s = -inf) yields zeros.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -14,68 +16,98 @@ namespace omnikv {
 
 namespace {
 
-constexpr int kCombineThreads = 128;
+constexpr int kCombineThreads = 256;
+constexpr int kMaxSplitsSmem = 4096;
 
 __global__ void __launch_bounds__(kCombineThreads)
 combine_inverse_rotate_kernel(const CombineParams p) {
-  const int b = blockIdx.y;
-  const int kvh = blockIdx.x;
+  const int g = blockIdx.x;        // query head within the group
+  const int kvh = blockIdx.y;
+  const int b = blockIdx.z;
   const int G = p.group;
   const int Hq = p.num_kv_heads * G;
   const int S = p.num_splits;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qh = kvh * G + g;
+  const Partial* part = p.partials + ((size_t)b * Hq + qh) * S;
 
-  __shared__ float a[kMaxGroup][kMods][kHeadDim];
+  __shared__ float w[kMaxSplitsSmem];
+  __shared__ __align__(16) float4 red[2][96];
+  __shared__ __align__(16) float a[kMods * kHeadDim];
+  __shared__ float s_l;
 
-  // merge splits; thread = rotated-space channel
-  for (int g = 0; g < G; ++g) {
-    const Partial* part = p.partials + ((size_t)b * Hq + kvh * G + g) * S;
+  if (warp == 0) {
     float M = -INFINITY;
-    for (int s = 0; s < S; ++s) M = fmaxf(M, part[s].m);
-    float l = 0.0f, acc[kMods] = {0.0f, 0.0f, 0.0f};
-    if (M != -INFINITY) {
-      for (int s = 0; s < S; ++s) {
-        const float ms = part[s].m;
-        if (ms == -INFINITY) continue;
-        const float e = expf(ms - M);
-        l += part[s].l * e;
+    for (int s = lane; s < S; s += 32) M = fmaxf(M, part[s].m);
 #pragma unroll
-        for (int m = 0; m < kMods; ++m) acc[m] += part[s].acc[m][tid] * e;
-      }
+    for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float l = 0.0f;
+    for (int s = lane; s < S; s += 32) {
+      const float ms = part[s].m;
+      const float e = (ms == -INFINITY) ? 0.0f : expf(ms - M);
+      w[s] = e;
+      l += part[s].l * e;
     }
-    const float inv = l > 0.0f ? 1.0f / l : 0.0f;
 #pragma unroll
-    for (int m = 0; m < kMods; ++m) a[g][m][tid] = acc[m] * inv;
+    for (int o = 16; o >= 1; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    if (lane == 0) s_l = l;
   }
   __syncthreads();
 
-  // out[g][j] = sum_m sum_c U_m[j][c] a[g][m][c]; warp per output row j,
-  // lanes over c (coalesced reads of U_m rows)
-  const int warp = tid >> 5, lane = tid & 31;
-  const float* Ubase = p.value_rot + (size_t)kvh * kMods * kHeadDim * kHeadDim;
-  for (int j = warp; j < kHeadDim; j += kCombineThreads / 32) {
-    float part[kMaxGroup];
-#pragma unroll
-    for (int g = 0; g < kMaxGroup; ++g) part[g] = 0.0f;
-#pragma unroll
-    for (int m = 0; m < kMods; ++m) {
-      const float* row = Ubase + ((size_t)m * kHeadDim + j) * kHeadDim;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int c = lane + 32 * k;
-        const float u = row[c];
-#pragma unroll
-        for (int g = 0; g < kMaxGroup; ++g)
-          if (g < G) part[g] = fmaf(u, a[g][m][c], part[g]);
+  // weighted sum over splits: column c4 (of 96 float4), half h of the splits
+  {
+    const int c4 = tid & 127, h = tid >> 7;
+    if (c4 < 96) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+      for (int s = h; s < S; s += 2) {
+        const float e = w[s];
+        if (e == 0.0f) continue;  // empty split, or negligible weight
+        const float4 v = reinterpret_cast<const float4*>(part[s].acc)[c4];
+        acc.x = fmaf(v.x, e, acc.x);
+        acc.y = fmaf(v.y, e, acc.y);
+        acc.z = fmaf(v.z, e, acc.z);
+        acc.w = fmaf(v.w, e, acc.w);
       }
+      red[h][c4] = acc;
     }
+  }
+  __syncthreads();
+  if (tid < 96) {
+    const float inv = s_l > 0.0f ? 1.0f / s_l : 0.0f;
+    const float4 x = red[0][tid], y = red[1][tid];
+    reinterpret_cast<float4*>(a)[tid] =
+        make_float4((x.x + y.x) * inv, (x.y + y.y) * inv, (x.z + y.z) * inv, (x.w + y.w) * inv);
+  }
+  __syncthreads();
+
+  // out[j] = sum_m U_m[j][:] . a_m
+  const float* Ubase = p.value_rot + (size_t)kvh * kMods * kHeadDim * kHeadDim;
+  float* out = p.out + ((size_t)b * Hq + qh) * kHeadDim;
+  float4 xa[kMods];
 #pragma unroll
-    for (int g = 0; g < kMaxGroup; ++g) {
-      if (g >= G) break;
-      float v = part[g];
+  for (int m = 0; m < kMods; ++m) xa[m] = reinterpret_cast<const float4*>(a + m * kHeadDim)[lane];
+  constexpr int kRows = 4;  // rows per batch: their U loads are issued together
+  for (int j0 = warp * kRows; j0 < kHeadDim; j0 += kRows * (kCombineThreads / 32)) {
+    float4 u[kRows][kMods];
+#pragma unroll
+    for (int r = 0; r < kRows; ++r)
+#pragma unroll
+      for (int m = 0; m < kMods; ++m)
+        u[r][m] = reinterpret_cast<const float4*>(Ubase + ((size_t)m * kHeadDim + j0 + r) * kHeadDim)[lane];
+#pragma unroll
+    for (int r = 0; r < kRows; ++r) {
+      float v = 0.0f;
+#pragma unroll
+      for (int m = 0; m < kMods; ++m) {
+        v = fmaf(u[r][m].x, xa[m].x, v);
+        v = fmaf(u[r][m].y, xa[m].y, v);
+        v = fmaf(u[r][m].z, xa[m].z, v);
+        v = fmaf(u[r][m].w, xa[m].w, v);
+      }
 #pragma unroll
       for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0) p.out[((size_t)b * Hq + kvh * G + g) * kHeadDim + j] = v;
+      if (lane == 0) out[j0 + r] = v;
     }
   }
 }
@@ -83,7 +115,8 @@ combine_inverse_rotate_kernel(const CombineParams p) {
 }  // namespace
 
 cudaError_t launch_combine(const CombineParams& p, int batch, cudaStream_t stream) {
-  dim3 grid(p.num_kv_heads, batch);
+  if (p.num_splits > kMaxSplitsSmem) return cudaErrorInvalidValue;
+  dim3 grid(p.group, p.num_kv_heads, batch);
   combine_inverse_rotate_kernel<<<grid, kCombineThreads, 0, stream>>>(p);
   return cudaGetLastError();
 }

@@ -36,12 +36,15 @@ struct RecordLayout {
 };
 
 // One entry of the split-K partials buffer.
-struct Partial {
+struct __align__(16) Partial {
   float acc[kMods][kHeadDim];
   float m;
   float l;
+  float pad[2];
 };
-static_assert(sizeof(Partial) == 1544, "partials entry is 1544 bytes");
+static_assert(sizeof(Partial) == 1552, "partials entry is 1552 bytes");
+
+constexpr int kMaxSplits = 4096;
 
 // Sign flip, Sylvester-Hadamard butterflies with h = 1, 2, ..., 64, then the
 // fp32 scale 2^-3.5, on a 128-vector spread over a warp: lane L holds channels

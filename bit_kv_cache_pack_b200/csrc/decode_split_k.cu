@@ -11,18 +11,21 @@
 //   * each warp streams its own windows (w0 + warp, w0 + warp + 4, ...) through
 //     a 4-stage shared-memory ring filled by 1-D bulk async copies (record +
 //     the window's 32 modality ids) completing on per-stage mbarriers;
-//   * scores use mma.sync m16n8k16 with the 8 query heads as N: the A operand
-//     (16 tokens x 16 channels) is built from the packed codes with one shift
-//     and one AND per register -- a code's low bit b0 lands on fp16 bit 13
-//     (value 2^-7 or 0) and its high bit b1 on bit 14 (value 2 or 0), exactly;
-//     with a symmetric codebook c_j - c_0 = (c_1 - c_0) b0 + (c_2 - c_0) b1, so
-//     two exact planes reproduce the codebook and the B operand carries
-//     q'_c s_gc (c_1 - c_0) * 128 and q'_c s_gc (c_2 - c_0) / 2 in fp16; the
-//     window minimum enters as the per-head offset sum_c q'_c m_gc;
+//   * scores use mma.sync m16n8k16 with the 8 query heads as N. With a
+//     symmetric codebook c_j - c_0 = (c_1 - c_0) b0 + (c_2 - c_0) b1 for the
+//     code's bits b0, b1, so k'_tc - m_gc = s_gc ((c_1 - c_0) b0 + (c_2 - c_0) b1).
+//     The A operand (16 tokens x 16 channels) holds s_gc * 2^-7 * b0 and
+//     s_gc * 2 * b1, both exact in fp16: one shift and one AND put a code bit on
+//     fp16 bit 13 (2^-7) or 14 (2), and one HMUL2 by the window's fp16 scales.
+//     The B operand is q'_c (c_1 - c_0) * 128 and q'_c (c_2 - c_0) / 2, split
+//     into an fp16 high and low part (so the product keeps ~22 bits), built
+//     once per CTA in shared memory; the window minimum enters as the per-head
+//     offset sum_c q'_c m_gc;
 //   * online softmax per window (running max with exact rescale when it grows,
 //     per-lane partial sums reduced once at the end);
-//   * P (times the token's value scale sigma and the plane constants) becomes
-//     the B operand of the value product through movmatrix; values are stored
+//   * P (times the token's value scale sigma and the plane constants, split
+//     into fp16 high + low parts) becomes the B operand of the value product
+//     through movmatrix; values are stored
 //     channel-major so the A operand (16 channels x 16 tokens) again needs one
 //     shift and one AND per register; one fp32 accumulator set per modality
 //     (values of different modalities live in different rotated bases); the
@@ -50,7 +53,7 @@ namespace {
 
 constexpr int kWarps = 4;
 constexpr int kThreads = 32 * kWarps;
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kRec22 = 2624;                    // K2/V2 record bytes
 constexpr int kStageBytes = kRec22 + kWindow;   // record + modality ids
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: a bulk copy that takes longer is an error
@@ -58,6 +61,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 struct __align__(16) DecodeSmem {
   uint8_t stage[kWarps][kStages][kStageBytes];  // also reused by the generic path and the final merge
+  uint4 btab[8][2][32];                         // score B operand per (chunk, plane, lane): {hi, hi, lo, lo}
   uint64_t bar[kWarps][kStages];
   float q[kMaxGroup][kHeadDim];                 // rotated queries, times the softmax scale
   float mw[kWarps][kMaxGroup];                  // per-warp running max, for the merge
@@ -112,11 +116,16 @@ __device__ __forceinline__ void rotate_queries(const DecodeParams& p, int b, int
   }
 }
 
+// Split s covers windows [s C, min((s+1) C, W_b)) of sequence b, with C =
+// p.split_windows chosen on the host from the length bound, so a short sequence
+// leaves its last splits empty and every non-empty split has the same size.
 __device__ __forceinline__ void split_range(const DecodeParams& p, int b, int split, int& T, int& w0, int& w1) {
   T = max(0, min(p.seq_lens[b], p.cap_tokens));
   const int nw = (T + kWindow - 1) / kWindow;
-  w0 = (int)(((long long)split * nw) / p.num_splits);
-  w1 = (int)(((long long)(split + 1) * nw) / p.num_splits);
+  w0 = min(split * p.split_windows, nw);
+  w1 = min(w0 + p.split_windows, nw);
+  if (split == p.num_splits - 1 && threadIdx.x == 0 && nw > p.num_splits * p.split_windows)
+    set_error(p.error_word, OMNIKV_DEVERR_BOUND);
 }
 
 // ---------------------------------------------------------------------------
@@ -241,6 +250,16 @@ constexpr uint32_t kPlane1 = 0x40004000u;  // bit 14 of each half: 2
 
 __device__ __forceinline__ uint32_t rotl(uint32_t x, int n) { return __funnelshift_l(x, x, n); }
 
+// (lo, hi) -> fp16 pair h = fp16(x) and l = fp16(x - h), each transposed to the
+// B-fragment layout with movmatrix.
+__device__ __forceinline__ void split_pair_t(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(x0, x1);
+  const float2 f = __half22float2(h);
+  const __half2 l = __floats2half2_rn(x0 - f.x, x1 - f.y);
+  hi = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h));
+  lo = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&l));
+}
+
 struct WarpState {
   float m[2];           // running max for heads 2t, 2t+1 (warp-uniform per column)
   float l[2];           // per-lane partial sum of p for heads 2t, 2t+1
@@ -257,8 +276,8 @@ __device__ __forceinline__ void issue_window(const DecodeParams& p, DecodeSmem& 
   bulk_copy_g2s(dst + kRec22, p.modality + (size_t)b * p.cap_tokens + (size_t)wi * kWindow, kWindow, bar);
 }
 
-__device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh, int split, float kK0, float kK1,
-                           float kV0, float kV1, float vc0) {
+__device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh, int split, float kV0, float kV1,
+                           float vc0) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int G = p.group;
@@ -307,34 +326,36 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
     const __half* sig = reinterpret_cast<const __half*>(stg + 2560);
     const uint8_t* mods = stg + kRec22;
 
-    // ---- per-window B operand of the score product: head g, channels 32t .. 32t+31
-    uint32_t B0[8][2], B1[8][2];
+    // ---- per-window: fp16 scale pairs for the A operand, offset sum_c q'_c m_gc
+    // lane (g, t) covers channels 32t .. 32t+31 (k-slot pairs (c, c+8))
+    uint32_t sp[8][2];
     float off;
     {
       const float* qrow = &sm.q[g][32 * t];
       const int qsw = (4 * (g & 1) + t) & 7;
       const uint4* mv4 = reinterpret_cast<const uint4*>(meta + 32 * t);
-      float x[32];
+      uint32_t mv[32];
+#pragma unroll
+      for (int i4 = 0; i4 < 8; ++i4) {
+        const uint4 mm = mv4[i4];
+        mv[4 * i4 + 0] = mm.x;
+        mv[4 * i4 + 1] = mm.y;
+        mv[4 * i4 + 2] = mm.z;
+        mv[4 * i4 + 3] = mm.w;
+      }
       off = 0.0f;
 #pragma unroll
       for (int i4 = 0; i4 < 8; ++i4) {
         const float4 qq = *reinterpret_cast<const float4*>(qrow + 4 * (i4 ^ qsw));
-        const uint4 mm = mv4[i4];
         const float qa[4] = {qq.x, qq.y, qq.z, qq.w};
-        const uint32_t ma[4] = {mm.x, mm.y, mm.z, mm.w};
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float2 ms = __half22float2(*reinterpret_cast<const __half2*>(&ma[j]));
-          off = fmaf(qa[j], ms.x, off);
-          x[4 * i4 + j] = qa[j] * ms.y;
-        }
+        for (int j = 0; j < 4; ++j)
+          off = fmaf(qa[j], __low2float(*reinterpret_cast<const __half2*>(&mv[4 * i4 + j])), off);
       }
 #pragma unroll
-      for (int kc = 0; kc < 8; ++kc) {
-        B0[kc][0] = pack_half2(x[kc] * kK0, x[kc + 8] * kK0);
-        B0[kc][1] = pack_half2(x[kc + 16] * kK0, x[kc + 24] * kK0);
-        B1[kc][0] = pack_half2(x[kc] * kK1, x[kc + 8] * kK1);
-        B1[kc][1] = pack_half2(x[kc + 16] * kK1, x[kc + 24] * kK1);
+      for (int kc = 0; kc < 8; ++kc) {  // high halves (the scales) of channels (c, c+8)
+        sp[kc][0] = __byte_perm(mv[kc], mv[kc + 8], 0x7632);
+        sp[kc][1] = __byte_perm(mv[kc + 16], mv[kc + 24], 0x7632);
       }
       off += __shfl_xor_sync(0xffffffffu, off, 1);
       off += __shfl_xor_sync(0xffffffffu, off, 2);
@@ -366,10 +387,16 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
           r[2] = kA.y >> 1;
           r[3] = kB.y >> 1;
         }
-        const uint32_t a0[4] = {r[0] & kPlane0, r[1] & kPlane0, r[2] & kPlane0, r[3] & kPlane0};
-        const uint32_t a1[4] = {r[0] & kPlane1, r[1] & kPlane1, r[2] & kPlane1, r[3] & kPlane1};
-        mma_f16_16816(d0, a0, B0[kc][0], B0[kc][1]);
-        mma_f16_16816(d1, a1, B1[kc][0], B1[kc][1]);
+        const uint32_t s0 = sp[kc][0], s1 = sp[kc][1];
+        const uint32_t a0[4] = {hmul2_u32(s0, r[0] & kPlane0), hmul2_u32(s0, r[1] & kPlane0),
+                                hmul2_u32(s1, r[2] & kPlane0), hmul2_u32(s1, r[3] & kPlane0)};
+        const uint32_t a1[4] = {hmul2_u32(s0, r[0] & kPlane1), hmul2_u32(s0, r[1] & kPlane1),
+                                hmul2_u32(s1, r[2] & kPlane1), hmul2_u32(s1, r[3] & kPlane1)};
+        const uint4 bp0 = sm.btab[kc][0][lane], bp1 = sm.btab[kc][1][lane];
+        mma_f16_16816(d0, a0, bp0.x, bp0.y);
+        mma_f16_16816(d1, a1, bp1.x, bp1.y);
+        mma_f16_16816(d0, a0, bp0.z, bp0.w);
+        mma_f16_16816(d1, a1, bp1.z, bp1.w);
       }
       const int posA = wi * kWindow + tokA[h], posB = wi * kWindow + tokB[h];
       sc[h][0] = posA < T ? d0[0] + d1[0] + off0 : -INFINITY;
@@ -419,10 +446,12 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
       st.l[1] += p1 + p3;
       const float sgA = __half2float(sig[tokA[h]]), sgB = __half2float(sig[tokB[h]]);
       const float w0v = p0 * sgA, w1v = p1 * sgA, w2v = p2 * sgB, w3v = p3 * sgB;
-      const uint32_t bv0[2] = {movmatrix_trans(pack_half2(w0v * kV0, w1v * kV0)),
-                               movmatrix_trans(pack_half2(w2v * kV0, w3v * kV0))};
-      const uint32_t bv1[2] = {movmatrix_trans(pack_half2(w0v * kV1, w1v * kV1)),
-                               movmatrix_trans(pack_half2(w2v * kV1, w3v * kV1))};
+      // value-product B operand per plane, as fp16 high + low parts
+      uint32_t bv0[4], bv1[4];  // {hi(row g), hi(row g+8), lo(row g), lo(row g+8)}, transposed
+      split_pair_t(w0v * kV0, w1v * kV0, bv0[0], bv0[2]);
+      split_pair_t(w2v * kV0, w3v * kV0, bv0[1], bv0[3]);
+      split_pair_t(w0v * kV1, w1v * kV1, bv1[0], bv1[2]);
+      split_pair_t(w2v * kV1, w3v * kV1, bv1[1], bv1[3]);
       // modalities of this tile (warp-uniform mask) and of this lane's tokens
       const int mA = mods[tokA[h]], mB = mods[tokB[h]];
       const uint32_t mbits = __reduce_or_sync(0xffffffffu, (1u << min(mA, 2)) | (1u << min(mB, 2)));
@@ -455,6 +484,8 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
             const uint32_t a1[4] = {r[0] & kPlane1, r[1] & kPlane1, r[2] & kPlane1, r[3] & kPlane1};
             mma_f16_16816(st.acc[mm][mt], a0, bv0[0], bv0[1]);
             mma_f16_16816(st.acc[mm][mt], a1, bv1[0], bv1[1]);
+            mma_f16_16816(st.acc[mm][mt], a0, bv0[2], bv0[3]);
+            mma_f16_16816(st.acc[mm][mt], a1, bv1[2], bv1[3]);
           }
         }
       } else {  // mixed tile: one masked product per modality present
@@ -469,6 +500,8 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
           const uint32_t msk23 = (mk2 == mm ? 0x0000FFFFu : 0u) | (mk3 == mm ? 0xFFFF0000u : 0u);
           const uint32_t b00 = bv0[0] & msk01, b01 = bv0[1] & msk23;
           const uint32_t b10 = bv1[0] & msk01, b11 = bv1[1] & msk23;
+          const uint32_t c00 = bv0[2] & msk01, c01 = bv0[3] & msk23;
+          const uint32_t c10 = bv1[2] & msk01, c11 = bv1[3] & msk23;
           st.S[mm][0] += (min(mA, 2) == mm ? w0v : 0.0f) + (min(mB, 2) == mm ? w2v : 0.0f);
           st.S[mm][1] += (min(mA, 2) == mm ? w1v : 0.0f) + (min(mB, 2) == mm ? w3v : 0.0f);
 #pragma unroll
@@ -479,6 +512,8 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
             const uint32_t a1[4] = {r[0] & kPlane1, r[1] & kPlane1, r[2] & kPlane1, r[3] & kPlane1};
             mma_f16_16816(st.acc[mm][mt], a0, b00, b01);
             mma_f16_16816(st.acc[mm][mt], a1, b10, b11);
+            mma_f16_16816(st.acc[mm][mt], a0, c00, c01);
+            mma_f16_16816(st.acc[mm][mt], a1, c10, c11);
           }
         }
       }
@@ -525,62 +560,123 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
       st.acc[m][mt][3] += vc0 * st.S[m][1];
     }
 
-  // ---- merge the 4 warps: max, rescale, shared-memory reduction ------------
+  // ---- merge the 4 warps: common max, rescale, exchange in register order ---
+  // (every warp holds the same (channel, head) in the same register of the same
+  // lane, so a lane-major buffer is bank-conflict free)
   if (g == 0) {
     sm.mw[warp][2 * t] = st.m[0];
     sm.mw[warp][2 * t + 1] = st.m[1];
   }
-  __syncthreads();  // all warps are done with their stage buffers
-  float* macc = reinterpret_cast<float*>(&sm.stage[0][0][0]);  // [3][8][128]
-  float* ml = macc + kMods * kMaxGroup * kHeadDim;              // [8]
-  for (int i = threadIdx.x; i < kMods * kMaxGroup * kHeadDim + kMaxGroup; i += kThreads) macc[i] = 0.0f;
-  __syncthreads();
-  float sc2[2];
+  __syncthreads();  // also: all warps are done with their stage buffers
+  float M[2];
 #pragma unroll
   for (int j = 0; j < 2; ++j) {
-    const int hcol = 2 * t + j;
     float mm = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) mm = fmaxf(mm, sm.mw[w][hcol]);
-    sc2[j] = (st.m[j] == -INFINITY) ? 0.0f : exp2f((st.m[j] - mm) * kLog2e);
-  }
-  if (g == 0) {
-    atomicAdd(&ml[2 * t], st.l[0] * sc2[0]);
-    atomicAdd(&ml[2 * t + 1], st.l[1] * sc2[1]);
-  }
-#pragma unroll
-  for (int m = 0; m < kMods; ++m)
-#pragma unroll
-    for (int mt = 0; mt < 8; ++mt) {
-      const int c0 = 16 * g + 2 * mt;  // row g -> channel 16g + 2mt, row g + 8 -> + 1
-      float* base = macc + (size_t)m * kMaxGroup * kHeadDim;
-      atomicAdd(&base[(2 * t) * kHeadDim + c0], st.acc[m][mt][0] * sc2[0]);
-      atomicAdd(&base[(2 * t + 1) * kHeadDim + c0], st.acc[m][mt][1] * sc2[1]);
-      atomicAdd(&base[(2 * t) * kHeadDim + c0 + 1], st.acc[m][mt][2] * sc2[0]);
-      atomicAdd(&base[(2 * t + 1) * kHeadDim + c0 + 1], st.acc[m][mt][3] * sc2[1]);
-    }
-  __syncthreads();
-  // ---- write one partial per query head of the group
-  for (int hh = warp; hh < G; hh += kWarps) {
-    Partial* out = p.partials + ((size_t)b * Hq + kvh * G + hh) * p.num_splits + split;
+    for (int w = 0; w < kWarps; ++w) mm = fmaxf(mm, sm.mw[w][2 * t + j]);
+    M[j] = mm;
+    const float f = (st.m[j] == -INFINITY) ? 0.0f : exp2f((st.m[j] - mm) * kLog2e);
+    st.l[j] *= f;
 #pragma unroll
     for (int m = 0; m < kMods; ++m)
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        out->acc[m][lane + 32 * j] = macc[((size_t)m * kMaxGroup + hh) * kHeadDim + lane + 32 * j];
-    if (lane == 0) {
-      float mm = -INFINITY;
+      for (int mt = 0; mt < 8; ++mt) {
+        st.acc[m][mt][j] *= f;
+        st.acc[m][mt][j + 2] *= f;
+      }
+  }
+  constexpr int kVals = kMods * 8 * 4 + 2;
+  float* xbuf = reinterpret_cast<float*>(&sm.stage[0][0][0]);  // [2][kVals][32]
+  static_assert(2 * kVals * 32 * 4 <= kWarps * kStages * kStageBytes, "merge buffer");
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) mm = fmaxf(mm, sm.mw[w][hh]);
-      out->m = mm;
-      out->l = ml[hh];
+  for (int round = 0; round < 2; ++round) {
+    const int writers_lo = round == 0 ? 2 : 1;  // round 0: warps 2,3 -> 0,1; round 1: warp 1 -> 0
+    const bool writer = round == 0 ? (warp >= 2) : (warp == 1);
+    const bool reader = round == 0 ? (warp < 2) : (warp == 0);
+    if (writer) {
+      float* dst = xbuf + (size_t)(warp - writers_lo) * kVals * 32 + lane;
+#pragma unroll
+      for (int m = 0; m < kMods; ++m)
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+          for (int r = 0; r < 4; ++r) dst[((m * 8 + mt) * 4 + r) * 32] = st.acc[m][mt][r];
+      dst[(kVals - 2) * 32] = st.l[0];
+      dst[(kVals - 1) * 32] = st.l[1];
     }
+    __syncthreads();
+    if (reader) {
+      const float* src = xbuf + (size_t)warp * kVals * 32 + lane;
+#pragma unroll
+      for (int m = 0; m < kMods; ++m)
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+          for (int r = 0; r < 4; ++r) st.acc[m][mt][r] += src[((m * 8 + mt) * 4 + r) * 32];
+      st.l[0] += src[(kVals - 2) * 32];
+      st.l[1] += src[(kVals - 1) * 32];
+    }
+    __syncthreads();
+  }
+  // ---- warp 0 writes one partial per query head of the group
+  if (warp == 0) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int hh = 2 * t + j;
+      if (hh >= G) continue;
+      Partial* out = p.partials + ((size_t)b * Hq + kvh * G + hh) * p.num_splits + split;
+#pragma unroll
+      for (int m = 0; m < kMods; ++m)
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt)
+          *reinterpret_cast<float2*>(&out->acc[m][16 * g + 2 * mt]) =
+              make_float2(st.acc[m][mt][j], st.acc[m][mt][j + 2]);
+      if (g == 0) {
+        out->m = M[j];
+        out->l = st.l[j];
+      }
+    }
+  }
+}
+
+// Score B operand for lane (g, t), chunk kc, plane P: k-slots 2t, 2t+1 hold
+// channels 32t + kc and 32t + kc + 8, k-slots 2t+8, 2t+9 hold 32t + 16 + kc and
+// 32t + 24 + kc; column g is query head g. Entry {hi(slots 2t..), hi(slots
+// 2t+8..), lo(..), lo(..)} with lo = fp16(y - hi).
+__device__ __forceinline__ void build_score_operand(DecodeSmem& sm, float k0scale, float k1scale) {
+  const float* qflat = &sm.q[0][0];
+  for (int e = threadIdx.x; e < 8 * 2 * 32; e += kThreads) {
+    const int lane = e & 31, P = (e >> 5) & 1, kc = e >> 6;
+    const int g = lane >> 2, t = lane & 3;
+    const float sc = P == 0 ? k0scale : k1scale;
+    float y[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) y[j] = qflat[qpos(g, 32 * t + kc + 8 * j)] * sc;
+    const __half2 h01 = __floats2half2_rn(y[0], y[1]);
+    const __half2 h23 = __floats2half2_rn(y[2], y[3]);
+    const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+    const __half2 l01 = __floats2half2_rn(y[0] - f01.x, y[1] - f01.y);
+    const __half2 l23 = __floats2half2_rn(y[2] - f23.x, y[3] - f23.y);
+    sm.btab[kc][P][lane] = make_uint4(*reinterpret_cast<const uint32_t*>(&h01), *reinterpret_cast<const uint32_t*>(&h23),
+                                      *reinterpret_cast<const uint32_t*>(&l01), *reinterpret_cast<const uint32_t*>(&l23));
   }
 }
 
 __global__ void __launch_bounds__(kThreads, 2) decode_split_k_kernel(const DecodeParams p) {
   __shared__ DecodeSmem sm;
   const int b = blockIdx.z, kvh = blockIdx.y, split = blockIdx.x;
+  {
+    int T, w0, w1;
+    split_range(p, b, split, T, w0, w1);
+    if (w0 == w1) {  // empty split (short sequence): only m and l are read by the combine
+      if (threadIdx.x < p.group) {
+        Partial* out = p.partials + ((size_t)b * p.num_kv_heads * p.group + kvh * p.group + threadIdx.x) * p.num_splits + split;
+        out->m = -INFINITY;
+        out->l = 0.0f;
+      }
+      return;
+    }
+  }
   rotate_queries(p, b, kvh, sm.q);
   __syncthreads();
   if (p.key_bits == 2 && p.value_bits == 2) {
@@ -588,8 +684,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_split_k_kernel(const Decod
     const float v0 = p.val_cb[0], v1 = p.val_cb[1], v2 = p.val_cb[2], v3 = p.val_cb[3];
     const bool symmetric = (k0 == -k3) && (k1 == -k2) && (v0 == -v3) && (v1 == -v2);
     if (symmetric) {
-      decode_mma(p, sm, b, kvh, split, (k1 - k0) * 128.0f, (k2 - k0) * 0.5f, (v1 - v0) * 128.0f,
-                 (v2 - v0) * 0.5f, v0);
+      build_score_operand(sm, (k1 - k0) * 128.0f, (k2 - k0) * 0.5f);
+      __syncthreads();
+      decode_mma(p, sm, b, kvh, split, (v1 - v0) * 128.0f, (v2 - v0) * 0.5f, v0);
       return;
     }
   }

@@ -39,6 +39,7 @@ struct DecodeParams {
   const __half* q;
   Partial* partials;
   int num_splits;
+  int split_windows;  // windows per split (C)
   int32_t* error_word;
 };
 

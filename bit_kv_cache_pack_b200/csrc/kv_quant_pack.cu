@@ -157,8 +157,11 @@ kv_quant_pack_kernel(const WriteParams p) {
       int m = mnew[p0 + i - L0];
       if (m >= kMods) m = kMods - 1;  // out-of-range ids are flagged below and read as video
       const float* U = p.value_rot + ((size_t)(h * kMods + m) * kHeadDim) * kHeadDim + j;
-      float acc = 0.0f;
-      for (int c = 0; c < kHeadDim; ++c) acc = fmaf(U[(size_t)c * kHeadDim], kp[i][c], acc);
+      // column j of U_m against the value: independent loads, 8 partial sums
+      float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 32
+      for (int c = 0; c < kHeadDim; ++c) part[c & 7] = fmaf(U[(size_t)c * kHeadDim], kp[i][c], part[c & 7]);
+      const float acc = ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
       const float s = s_sigma[i];
       uint32_t code = 0;
       if (s != 0.0f) code = count_above(__fdiv_rn(acc, s), thr_v, LV - 1);

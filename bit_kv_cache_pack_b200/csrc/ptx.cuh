@@ -2,6 +2,7 @@
 // no multicast), legacy tensor-core MMA and register-fragment transpose.
 #pragma once
 
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 namespace omnikv {
@@ -85,6 +86,11 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
   uint32_t y;
   asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
   return y;
+}
+
+__device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
+  const __half2 r = __hmul2(*reinterpret_cast<const __half2*>(&a), *reinterpret_cast<const __half2*>(&b));
+  return *reinterpret_cast<const uint32_t*>(&r);
 }
 
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {

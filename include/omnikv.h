@@ -78,6 +78,8 @@ typedef enum {
 /* Device error word bits (omnikv_cache.error_word). */
 #define OMNIKV_DEVERR_CAPACITY 0x1 /* a write would have passed cap_tokens; that sequence was skipped */
 #define OMNIKV_DEVERR_MODALITY 0x2 /* a modality id was > 2; it was stored and used as 2 (video) */
+#define OMNIKV_DEVERR_BOUND 0x8    /* a sequence was longer than cache->max_seq_len promised; windows past
+                                      num_splits * ceil(ceil(max_seq_len / 32) / num_splits) were skipped */
 #define OMNIKV_DEVERR_TIMEOUT 0x4  /* a staged copy did not complete within its wait limit; outputs of that
                                       CTA are zero (never expected; the kernel returns instead of hanging) */
 
@@ -115,7 +117,8 @@ typedef struct {
 OMNIKV_API size_t omnikv_record_bytes(int32_t key_bits, int32_t value_bits);
 
 /* Bytes of the split-K partials buffer for omnikv_decode_attention / omnikv_combine:
- * [batch][num_q_heads][num_splits] entries of { fp32 acc[3][128], fp32 m, fp32 l } (1544 B each). */
+ * [batch][num_q_heads][num_splits] entries of { fp32 acc[3][128], fp32 m, fp32 l, 2 x fp32 padding }
+ * (1552 B each, 16-byte aligned). num_splits is at most 4096 (OMNIKV_ERR_UNSUPPORTED above). */
 OMNIKV_API size_t omnikv_partials_bytes(int32_t batch, int32_t num_q_heads, int32_t num_splits);
 
 /* The split count used when omnikv_decode_attention is given num_splits = 0 (depends on the
@@ -142,13 +145,14 @@ OMNIKV_API omnikv_status omnikv_write_cache(const omnikv_config* cfg, omnikv_cac
                                  int32_t n_new, void* stream);
 
 /* Fused split-K decode attention over the packed cache (decode_split_k). For every sequence b,
- * query head i (kv head i / G) and split s, over the windows [floor(s W / S), floor((s+1) W / S))
- * of the W = ceil(seq_lens[b] / 32) windows: q' = fp32(2^-3.5) H (s . q_i); score_t = q' . k'_t /
+ * query head i (kv head i / G) and split s, over the windows [s C, min((s+1) C, W)) of the
+ * W = ceil(seq_lens[b] / 32) windows, C = ceil(ceil(cache->max_seq_len / 32) / S):
+ * q' = fp32(2^-3.5) H (s . q_i); score_t = q' . k'_t /
  * sqrt(128); a running max m and sum l of exp(score - m), and one rotated-space accumulator per
  * modality acc_m = sum_{t of modality m} exp(score_t - m) v'_t. Written to `partials`.
  *   q          : [batch][num_q_heads][128] fp16, 16-byte aligned
  *   partials   : device buffer of omnikv_partials_bytes(batch, num_q_heads, S) bytes, 16-byte aligned
- *   num_splits : S >= 1, or 0 for omnikv_default_splits(cfg, cache)
+ *   num_splits : 1 <= S <= 4096, or 0 for omnikv_default_splits(cfg, cache)
  * Empty splits write m = -inf, l = 0, acc = 0. */
 OMNIKV_API omnikv_status omnikv_decode_attention(const omnikv_config* cfg, const omnikv_cache* cache,
                                       const void* q, void* partials, int32_t num_splits, void* stream);

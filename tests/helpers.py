@@ -13,6 +13,11 @@ MAX_REL_L2 = 1e-3  # decode output tolerance (relative L2)
 Z_TOL = 5e-5       # value-code disagreement allowed only this close to a threshold
 
 
+def seeded_randn(shape, device, seed):
+    g = torch.Generator(device=device).manual_seed(seed)
+    return torch.randn(*shape, device=device, generator=g)
+
+
 def make_layer(spec, seed, layer, device, per_head=False):
     from bit_kv_cache_pack_b200 import LayerConstants
     params = layer_params(spec, seed, layer, per_head)

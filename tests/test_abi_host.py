@@ -38,7 +38,7 @@ def test_sizes_and_version():
     assert _abi.omnikv_record_bytes(4, 4) == 4672
     assert _abi.omnikv_record_bytes(2, 4) == 1024 + 512 + 2048 + 64
     assert _abi.omnikv_record_bytes(3, 2) == 0
-    assert _abi.omnikv_partials_bytes(2, 16, 5) == 2 * 16 * 5 * 1544
+    assert _abi.omnikv_partials_bytes(2, 16, 5) == 2 * 16 * 5 * 1552
     assert _abi.omnikv_partials_bytes(0, 16, 5) == 0
     assert _abi.status_string(_abi.OMNIKV_ERR_CAPACITY) == "cache capacity exceeded"
 

@@ -14,7 +14,7 @@ from oracle import codec
 from oracle.attention import decode_dense
 from synth.workloads import CONFIGS, decode_inputs, key_drift, prefill_inputs, seq_lengths, with_bits
 
-from helpers import check_decode, compare_records, make_layer, upload_oracle_cache
+from helpers import check_decode, compare_records, make_layer, seeded_randn, upload_oracle_cache
 
 pytestmark = pytest.mark.gpu
 
@@ -104,7 +104,7 @@ def test_chunked_writes_and_tail(cuda_device, bits):
     for a, b_ in zip(cuts[:-1], cuts[1:]):
         _write_both(consts, ocfg, gc, oc, k[:, :, a:b_], v[:, :, a:b_], mod[:, a:b_])
         _check_state(ocfg, oc, gc, v.cpu().numpy(), mod.cpu().numpy())
-    q = torch.randn(1, 16, 128, device=cuda_device).half()
+    q = seeded_randn((1, 16, 128), cuda_device, 11).half()
     ref = decode_dense(ocfg, oc, q.cpu().numpy())
     check_decode(gpu_decode(consts, upload_oracle_cache(oc, cuda_device), q), ref, "bits=%d" % bits)
 
@@ -119,9 +119,12 @@ def test_decode_split_counts(cuda_device, splits):
     k, v, mod = prefill_inputs(spec, seed, 0, params, drift, L, cuda_device)
     oc = codec.OracleCache(1, 2, 1024, 2, 2)
     codec.write_cache(ocfg, oc, k.cpu().numpy(), v.cpu().numpy(), mod.cpu().numpy())
-    q = torch.randn(1, 16, 128, device=cuda_device).half()
-    ref = decode_dense(ocfg, oc, q.cpu().numpy())
-    check_decode(gpu_decode(consts, upload_oracle_cache(oc, cuda_device), q, splits), ref, "S=%d" % splits)
+    for scale in (1.0, 3.0):  # 3x sharpens the attention (larger error amplification)
+        g = torch.Generator(device=cuda_device).manual_seed(splits)
+        q = (scale * torch.randn(1, 16, 128, device=cuda_device, generator=g)).half()
+        ref = decode_dense(ocfg, oc, q.cpu().numpy())
+        check_decode(gpu_decode(consts, upload_oracle_cache(oc, cuda_device), q, splits), ref,
+                     "S=%d scale=%g" % (splits, scale))
 
 
 def test_decode_edge_cases(cuda_device):
@@ -144,7 +147,7 @@ def test_decode_edge_cases(cuda_device):
     gc.struct.max_seq_len = 70
     torch.cuda.synchronize()
     assert np.array_equal(gc.seq_lens.cpu().numpy(), [0, 1, 70, 32])
-    q = torch.randn(4, 16, 128, device=cuda_device).half()
+    q = seeded_randn((4, 16, 128), cuda_device, 12).half()
     q[2] = 0
     ref = decode_dense(ocfg, oc, q.cpu().numpy())
     out = gpu_decode(consts, upload_oracle_cache(oc, cuda_device), q)
@@ -160,7 +163,7 @@ def test_device_capacity_check_sets_error_word(cuda_device):
     params, consts, ocfg = make_layer(spec, seed, 0, cuda_device)
     gc = m.KVCache(1, 2, 64, 2, 2, cuda_device)
     gc.seq_lens.fill_(60)
-    k = torch.randn(1, 2, 8, 128, device=cuda_device).half()
+    k = seeded_randn((1, 2, 8, 128), cuda_device, 13).half()
     mod = torch.zeros(1, 8, dtype=torch.uint8, device=cuda_device)
     m.omnikv_write_cache(consts.struct, gc.struct, k, k.clone(), mod, 8)
     torch.cuda.synchronize()
@@ -186,7 +189,7 @@ def test_asymmetric_codebook_uses_generic_path(cuda_device):
     oc = codec.OracleCache(1, 2, 512, 2, 2)
     _write_both(consts, ocfg, gc, oc, k, v, mod)
     _check_state(ocfg, oc, gc, v.cpu().numpy(), mod.cpu().numpy())
-    q = torch.randn(1, 16, 128, device=cuda_device).half()
+    q = seeded_randn((1, 16, 128), cuda_device, 11).half()
     ref = decode_dense(ocfg, oc, q.cpu().numpy())
     check_decode(gpu_decode(consts, upload_oracle_cache(oc, cuda_device), q, 3), ref, "asymmetric")
 
@@ -212,7 +215,7 @@ def test_group_sizes(cuda_device, G, hkv):
                           mod[b:b + 1, :n].cpu().numpy())
         oc.records[b], oc.key_tail[b], oc.modality[b], oc.seq_lens[b] = (
             sub.records[0], sub.key_tail[0], sub.modality[0], sub.seq_lens[0])
-    q = torch.randn(2, G * hkv, 128, device=cuda_device).half()
+    q = seeded_randn((2, G * hkv, 128), cuda_device, 14 + G).half()
     ref = decode_dense(ocfg, oc, q.cpu().numpy())
     for S in (1, 4):
         check_decode(gpu_decode(consts, upload_oracle_cache(oc, cuda_device), q, S), ref, "G=%d S=%d" % (G, S))
