@@ -1,7 +1,7 @@
 """Benchmark: OmniKVQuant decode step (cache append + fused split-K decode +
 combine/inverse rotation, every layer) on synthetic inputs.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl omnikv|reference] [--workload 1]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl omnikv|reference] [--workload omni3b-b1]
     torchrun --nproc-per-node N bench.py --gpus N ...   (one rank per GPU, weak scaling)
 
 Default workload: the Qwen2.5-Omni-3B-shaped decode (36 layers, 16 query / 2 KV
@@ -32,6 +32,8 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+WORKLOADS_KEYS = ("tiny", "omni3b-b1", "omni3b-b16", "omni30b-b8", "ragged-b64")
+
 METRIC = "2-bit decode attention tokens/s and achieved HBM GB/s vs ~8 TB/s (1 B200)"
 UNIT = "tokens/s"
 BYTES_PER_TOKEN_HEAD = {(2, 2): 82, (4, 4): 146}   # algorithmic packed bytes per token per kv head
@@ -44,9 +46,10 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=64)
     ap.add_argument("--warmup", type=int, default=4)
     ap.add_argument("--impl", default="omnikv", choices=["omnikv", "reference"])
-    ap.add_argument("--workload", type=int, default=1)
+    ap.add_argument("--workload", default="omni3b-b1", choices=sorted(WORKLOADS_KEYS))
     ap.add_argument("--no-graphs", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clocks-csv", default=None, help="where to keep the nvidia-smi samples (default: a temp file)")
     return ap.parse_args()
 
 
@@ -74,10 +77,11 @@ class ClockSampler:
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, path=None):
+        import tempfile
         self.idx = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", "clocks_rank%d.csv" % gpu_index)
+        self.path = path or os.path.join(tempfile.gettempdir(), "omnikv_clocks_%d_%d.csv" % (os.getpid(), gpu_index))
 
     def start(self):
         try:
@@ -200,15 +204,15 @@ class Workload:
 
 def run_gpu(args):
     import torch.distributed as dist
-    from synth.workloads import CONFIGS
+    from synth.workloads import WORKLOADS
     world, rank, local = dist_env()
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
-    spec = CONFIGS[args.workload]
-    seed = args.workload + 1000 * rank
+    spec = WORKLOADS[args.workload]
+    seed = WORKLOADS_KEYS.index(args.workload) + 1000 * rank
     K, W = args.steps, args.warmup
     total = W + K + K + 1  # device-resident run, then the e2e run
     wl = Workload(spec, seed, dev, total)
@@ -232,7 +236,7 @@ def run_gpu(args):
             graphs.append(g)
     torch.cuda.synchronize(dev)
     t_steps = []
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(local, args.clocks_csv)
     if world > 1:
         dist.barrier()
     with torch.cuda.stream(stream):
@@ -398,12 +402,12 @@ def cpu_baseline(spec, seed, sample_layers=12):
 
 
 def run_reference(args):
-    from synth.workloads import CONFIGS
+    from synth.workloads import WORKLOADS
     world, rank, _ = dist_env()
     if rank != 0:
         return
-    spec = CONFIGS[args.workload]
-    seed = args.workload
+    spec = WORKLOADS[args.workload]
+    seed = WORKLOADS_KEYS.index(args.workload)
     K, W = args.steps, args.warmup
     n_prep = min(4, spec.layers)
     prepared = _oracle_layers(spec, seed, range(n_prep), (W + K) // n_prep + 2)

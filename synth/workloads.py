@@ -1,6 +1,6 @@
 """Workload recipes: shapes, modality layouts and seeded random tensors.
 
-Five workloads with the shapes of the models the OmniKVQuant pages evaluate
+Five workloads (WORKLOADS) with the shapes of the models the OmniKVQuant pages evaluate
 (Qwen2.5-Omni-3B: 36 layers, 16 query / 2 KV heads, head dim 128; Qwen3-Omni-
 30B-A3B: 48 layers, 32 / 4 heads), about 10k tokens per minute of audio-visual
 input (paperpeel.com section 1), 32-token windows (section 3.1). The pages
@@ -58,16 +58,21 @@ class WorkloadSpec:
     ragged: tuple = field(default=())   # (lo, hi) for ragged lengths
 
 
-CONFIGS = {
-    0: WorkloadSpec("tiny-1L-b1-16q2kv-ctx2048", 1, 1, 16, 2, 2048, "tavt", decode_steps=1),
-    1: WorkloadSpec("qwen2.5-omni-3b-36L-b1-ctx10240", 36, 1, 16, 2, 10240, "interleaved",
-                    decode_steps=128),
-    2: WorkloadSpec("qwen2.5-omni-3b-36L-b16-ctx32768", 36, 16, 16, 2, 32768, "interleaved",
-                    decode_steps=64),
-    3: WorkloadSpec("qwen3-omni-30b-48L-b8-ctx65536", 48, 8, 32, 4, 65536, "audio_heavy",
-                    drift_std=1.0, n_outliers=8, outlier_scale=16.0, decode_steps=32),
-    4: WorkloadSpec("ragged-36L-b64-ctx1024..32768", 36, 64, 16, 2, 0, "mixed",
-                    decode_steps=1, ragged=(1024, 32768)),
+WORKLOADS = {
+    # 1 layer, batch 1, 2,048 tokens: text 128 | audio 640 | video 1152 | text 128
+    "tiny": WorkloadSpec("tiny-1L-b1-16q2kv-ctx2048", 1, 1, 16, 2, 2048, "tavt", decode_steps=1),
+    # Qwen2.5-Omni-3B shape, batch 1, 10,240 tokens, 128 one-token decode steps
+    "omni3b-b1": WorkloadSpec("qwen2.5-omni-3b-36L-b1-ctx10240", 36, 1, 16, 2, 10240, "interleaved",
+                              decode_steps=128),
+    # same shape, batch 16, 32,768 tokens per sequence, 64 decode steps
+    "omni3b-b16": WorkloadSpec("qwen2.5-omni-3b-36L-b16-ctx32768", 36, 16, 16, 2, 32768, "interleaved",
+                               decode_steps=64),
+    # Qwen3-Omni-30B-A3B shape, batch 8, 65,536 tokens per sequence, audio-heavy, 32 decode steps
+    "omni30b-b8": WorkloadSpec("qwen3-omni-30b-48L-b8-ctx65536", 48, 8, 32, 4, 65536, "audio_heavy",
+                               drift_std=1.0, n_outliers=8, outlier_scale=16.0, decode_steps=32),
+    # ragged serving mix, batch 64, lengths uniform in [1024, 32768] (never a multiple of 32)
+    "ragged-b64": WorkloadSpec("ragged-36L-b64-ctx1024..32768", 36, 64, 16, 2, 0, "mixed",
+                               decode_steps=1, ragged=(1024, 32768)),
 }
 
 

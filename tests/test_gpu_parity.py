@@ -12,7 +12,7 @@ import torch
 
 from oracle import codec
 from oracle.attention import decode_dense
-from synth.workloads import CONFIGS, decode_inputs, key_drift, prefill_inputs, seq_lengths, with_bits
+from synth.workloads import WORKLOADS, decode_inputs, key_drift, prefill_inputs, seq_lengths, with_bits
 
 from helpers import check_decode, compare_records, make_layer, seeded_randn, upload_oracle_cache
 
@@ -65,7 +65,7 @@ def test_config0_write_append_decode(cuda_device):
     """The tiny configuration end to end: 2048-token prefill, one appended text
     token, one decode step."""
     m = _abi()
-    spec, seed = CONFIGS[0], 0
+    spec, seed = WORKLOADS["tiny"], 0
     params, consts, ocfg = make_layer(spec, seed, 0, cuda_device)
     L = seq_lengths(spec, seed)
     cap = 2048 + 32
@@ -92,7 +92,7 @@ def test_chunked_writes_and_tail(cuda_device, bits):
     """Prefill in ragged chunks (1, 2, 31, 33, ... tokens), per-head value bases:
     every partial-window path of the write."""
     m = _abi()
-    spec = with_bits(CONFIGS[0], bits, bits)
+    spec = with_bits(WORKLOADS["tiny"], bits, bits)
     seed = 3
     params, consts, ocfg = make_layer(spec, seed, 0, cuda_device, per_head=True)
     L = np.array([300], np.int32)
@@ -112,7 +112,7 @@ def test_chunked_writes_and_tail(cuda_device, bits):
 @pytest.mark.parametrize("splits", [1, 2, 7, 64, 200])
 def test_decode_split_counts(cuda_device, splits):
     m = _abi()
-    spec, seed = CONFIGS[0], 5
+    spec, seed = WORKLOADS["tiny"], 5
     params, consts, ocfg = make_layer(spec, seed, 0, cuda_device)
     L = np.array([1000], np.int32)
     drift = key_drift(spec, seed, 0, 32, cuda_device)
@@ -131,7 +131,7 @@ def test_decode_edge_cases(cuda_device):
     """Batch of four: an empty sequence (zeros), a single token, a zero query
     (mean of the values) and a one-window sequence."""
     m = _abi()
-    spec, seed = CONFIGS[0], 6
+    spec, seed = WORKLOADS["tiny"], 6
     params, consts, ocfg = make_layer(spec, seed, 0, cuda_device)
     drift = key_drift(spec, seed, 0, 4, cuda_device)
     oc = codec.OracleCache(4, 2, 96, 2, 2)
@@ -159,7 +159,7 @@ def test_device_capacity_check_sets_error_word(cuda_device):
     """A host bound that understates the device length: the kernel skips the
     write and reports it in the error word, without faulting."""
     m = _abi()
-    spec, seed = CONFIGS[0], 7
+    spec, seed = WORKLOADS["tiny"], 7
     params, consts, ocfg = make_layer(spec, seed, 0, cuda_device)
     gc = m.KVCache(1, 2, 64, 2, 2, cuda_device)
     gc.seq_lens.fill_(60)
@@ -177,7 +177,7 @@ def test_asymmetric_codebook_uses_generic_path(cuda_device):
     the same kernel; results still match the oracle."""
     import dataclasses
     m = _abi()
-    spec, seed = CONFIGS[0], 8
+    spec, seed = WORKLOADS["tiny"], 8
     params, consts, ocfg = make_layer(spec, seed, 0, cuda_device)
     cb = np.array([-1.2, -0.3, 0.5, 1.7], np.float32)
     consts = m.LayerConstants(cb, cb, params["key_signs"], params["value_rot"], spec.num_q_heads, cuda_device)
@@ -200,7 +200,7 @@ def test_group_sizes(cuda_device, G, hkv):
     size up to 8 must match the oracle."""
     import dataclasses
     m = _abi()
-    spec = dataclasses.replace(CONFIGS[0], num_q_heads=G * hkv, num_kv_heads=hkv)
+    spec = dataclasses.replace(WORKLOADS["tiny"], num_q_heads=G * hkv, num_kv_heads=hkv)
     seed = 9
     params, consts, ocfg = make_layer(spec, seed, 0, cuda_device, per_head=True)
     L = np.array([333, 70], np.int32)
