@@ -27,8 +27,9 @@ OMNIKV_DEVERR_BOUND = 0x8
 EXPORTED = (
     "omnikv_record_bytes", "omnikv_partials_bytes", "omnikv_default_splits",
     "omnikv_write_cache", "omnikv_decode_attention", "omnikv_combine",
-    "omnikv_status_string", "omnikv_abi_version",
+    "omnikv_status_string", "omnikv_abi_version", "omnikv_decode_static",
 )
+OMNIKV_DECODE_STATIC_SCRATCH_BYTES = 8 << 20
 
 
 class OmniKVError(RuntimeError):
@@ -88,6 +89,8 @@ def load() -> ctypes.CDLL:
     lib.omnikv_decode_attention.restype = ctypes.c_int
     lib.omnikv_combine.argtypes = [cfgp, cachep, P, I32, P, P]
     lib.omnikv_combine.restype = ctypes.c_int
+    lib.omnikv_decode_static.argtypes = [cfgp, cachep, P, P, I32, P]
+    lib.omnikv_decode_static.restype = ctypes.c_int
     lib.omnikv_status_string.argtypes, lib.omnikv_status_string.restype = [ctypes.c_int], ctypes.c_char_p
     lib.omnikv_abi_version.argtypes, lib.omnikv_abi_version.restype = [], I32
     _lib = lib
@@ -153,3 +156,11 @@ def omnikv_combine(cfg: OmniKVConfig, cache: OmniKVCache, partials, num_splits: 
     st = load().omnikv_combine(ctypes.byref(cfg), ctypes.byref(cache), _ptr(partials), int(num_splits),
                                _ptr(out), _stream(stream))
     _check(st, "omnikv_combine")
+
+
+def omnikv_decode_static(cfg: OmniKVConfig, cache: OmniKVCache, q, out, num_splits: int = 0, stream=None) -> None:
+    """Decode + combine with the split partials in the library's fixed device
+    array (no allocation by the caller or the library); see include/omnikv.h."""
+    st = load().omnikv_decode_static(ctypes.byref(cfg), ctypes.byref(cache), _ptr(q), _ptr(out), int(num_splits),
+                                     _stream(stream))
+    _check(st, "omnikv_decode_static")

@@ -2,6 +2,7 @@
 // Every check runs on the host before any launch; see include/omnikv.h.
 #include <cuda_runtime.h>
 
+#include "abi_internal.h"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -42,6 +43,10 @@ int sm_count() {
   return n;
 }
 
+}  // namespace
+
+namespace omnikv {
+
 int32_t resolve_splits(const omnikv_config* cfg, const omnikv_cache* c, int32_t requested) {
   if (requested > 0) return requested;
   const int nw = (c->max_seq_len + kWindow - 1) / kWindow;
@@ -58,7 +63,60 @@ int32_t resolve_splits(const omnikv_config* cfg, const omnikv_cache* c, int32_t 
   return (int32_t)s;
 }
 
-}  // namespace
+
+omnikv_status prepare_decode(const omnikv_config* cfg, const omnikv_cache* cache, const void* q, void* partials,
+                             int32_t num_splits, DecodeParams* p) {
+  omnikv_status st = check_config(cfg);
+  if (st != OMNIKV_OK) return st;
+  if ((st = check_cache(cache)) != OMNIKV_OK) return st;
+  if (!q || !partials || num_splits < 0) return OMNIKV_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(partials, 16)) return OMNIKV_ERR_INVALID_ARG;
+  p->key_cb = cfg->key_codebook;
+  p->val_cb = cfg->value_codebook;
+  p->key_signs = cfg->key_signs;
+  p->key_bits = cfg->key_bits;
+  p->value_bits = cfg->value_bits;
+  p->num_kv_heads = cfg->num_kv_heads;
+  p->group = cfg->num_q_heads / cfg->num_kv_heads;
+  p->records = static_cast<const uint8_t*>(cache->records);
+  p->modality = cache->modality;
+  p->seq_lens = cache->seq_lens;
+  p->cap_tokens = cache->cap_tokens;
+  p->cap_windows = cache->cap_tokens / kWindow;
+  p->q = static_cast<const __half*>(q);
+  p->partials = static_cast<Partial*>(partials);
+  p->num_splits = resolve_splits(cfg, cache, num_splits);
+  if (p->num_splits > kMaxSplits) return OMNIKV_ERR_UNSUPPORTED;
+  const int nw = (cache->max_seq_len + kWindow - 1) / kWindow;
+  p->split_windows = nw > 0 ? (nw + p->num_splits - 1) / p->num_splits : 1;
+  p->error_word = cache->error_word;
+  return OMNIKV_OK;
+}
+
+omnikv_status prepare_combine(const omnikv_config* cfg, const omnikv_cache* cache, const void* partials,
+                              int32_t num_splits, float* out, CombineParams* p) {
+  omnikv_status st = check_config(cfg);
+  if (st != OMNIKV_OK) return st;
+  if ((st = check_cache(cache)) != OMNIKV_OK) return st;
+  if (!partials || !out || num_splits < 0) return OMNIKV_ERR_INVALID_ARG;
+  if (!aligned(partials, 16) || !aligned(out, 16)) return OMNIKV_ERR_INVALID_ARG;
+  p->value_rot = cfg->value_rot;
+  p->num_kv_heads = cfg->num_kv_heads;
+  p->group = cfg->num_q_heads / cfg->num_kv_heads;
+  p->partials = static_cast<const Partial*>(partials);
+  p->num_splits = resolve_splits(cfg, cache, num_splits);
+  if (p->num_splits > kMaxSplits) return OMNIKV_ERR_UNSUPPORTED;
+  p->out = out;
+  return OMNIKV_OK;
+}
+
+omnikv_status validate_config_cache(const omnikv_config* cfg, const omnikv_cache* cache) {
+  omnikv_status st = check_config(cfg);
+  if (st != OMNIKV_OK) return st;
+  return check_cache(cache);
+}
+
+}  // namespace omnikv
 
 extern "C" {
 
@@ -112,52 +170,18 @@ omnikv_status omnikv_write_cache(const omnikv_config* cfg, omnikv_cache* cache, 
 
 omnikv_status omnikv_decode_attention(const omnikv_config* cfg, const omnikv_cache* cache, const void* q,
                                       void* partials, int32_t num_splits, void* stream) {
-  omnikv_status st = check_config(cfg);
-  if (st != OMNIKV_OK) return st;
-  if ((st = check_cache(cache)) != OMNIKV_OK) return st;
-  if (!q || !partials || num_splits < 0) return OMNIKV_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(partials, 16)) return OMNIKV_ERR_INVALID_ARG;
   DecodeParams p;
-  p.key_cb = cfg->key_codebook;
-  p.val_cb = cfg->value_codebook;
-  p.key_signs = cfg->key_signs;
-  p.key_bits = cfg->key_bits;
-  p.value_bits = cfg->value_bits;
-  p.num_kv_heads = cfg->num_kv_heads;
-  p.group = cfg->num_q_heads / cfg->num_kv_heads;
-  p.records = static_cast<const uint8_t*>(cache->records);
-  p.modality = cache->modality;
-  p.seq_lens = cache->seq_lens;
-  p.cap_tokens = cache->cap_tokens;
-  p.cap_windows = cache->cap_tokens / kWindow;
-  p.q = static_cast<const __half*>(q);
-  p.partials = static_cast<Partial*>(partials);
-  p.num_splits = resolve_splits(cfg, cache, num_splits);
-  if (p.num_splits > kMaxSplits) return OMNIKV_ERR_UNSUPPORTED;
-  {
-    const int nw = (cache->max_seq_len + kWindow - 1) / kWindow;
-    p.split_windows = nw > 0 ? (nw + p.num_splits - 1) / p.num_splits : 1;
-  }
-  p.error_word = cache->error_word;
+  const omnikv_status st = prepare_decode(cfg, cache, q, partials, num_splits, &p);
+  if (st != OMNIKV_OK) return st;
   if (launch_decode(p, cache->batch, static_cast<cudaStream_t>(stream)) != cudaSuccess) return OMNIKV_ERR_CUDA;
   return OMNIKV_OK;
 }
 
 omnikv_status omnikv_combine(const omnikv_config* cfg, const omnikv_cache* cache, const void* partials,
                              int32_t num_splits, float* out, void* stream) {
-  omnikv_status st = check_config(cfg);
-  if (st != OMNIKV_OK) return st;
-  if ((st = check_cache(cache)) != OMNIKV_OK) return st;
-  if (!partials || !out || num_splits < 0) return OMNIKV_ERR_INVALID_ARG;
-  if (!aligned(partials, 16) || !aligned(out, 16)) return OMNIKV_ERR_INVALID_ARG;
   CombineParams p;
-  p.value_rot = cfg->value_rot;
-  p.num_kv_heads = cfg->num_kv_heads;
-  p.group = cfg->num_q_heads / cfg->num_kv_heads;
-  p.partials = static_cast<const Partial*>(partials);
-  p.num_splits = resolve_splits(cfg, cache, num_splits);
-  if (p.num_splits > kMaxSplits) return OMNIKV_ERR_UNSUPPORTED;
-  p.out = out;
+  const omnikv_status st = prepare_combine(cfg, cache, partials, num_splits, out, &p);
+  if (st != OMNIKV_OK) return st;
   if (launch_combine(p, cache->batch, static_cast<cudaStream_t>(stream)) != cudaSuccess) return OMNIKV_ERR_CUDA;
   return OMNIKV_OK;
 }

@@ -165,6 +165,28 @@ OMNIKV_API omnikv_status omnikv_decode_attention(const omnikv_config* cfg, const
 OMNIKV_API omnikv_status omnikv_combine(const omnikv_config* cfg, const omnikv_cache* cache,
                              const void* partials, int32_t num_splits, float* out, void* stream);
 
+/* Decode attention and combine in one call, with the split-K partials in a fixed device array of
+ * OMNIKV_DECODE_STATIC_SCRATCH_BYTES owned by this library; the caller passes only inputs (q) and
+ * outputs (out), as for omnikv_decode_attention + omnikv_combine, and nothing is allocated.
+ * The paper has no counterpart: this entry point serves callers that cannot allocate device memory
+ * while decoding -- engines that reserved nearly all device memory for their own pool at start-up
+ * (a further cudaMalloc fails or fragments it), plug-ins whose host framework owns every allocation,
+ * and latency-critical loops that cannot pay for cudaMalloc / cudaFree, which may synchronise the
+ * device.
+ *   q, out, num_splits : as for omnikv_decode_attention / omnikv_combine; num_splits = 0 takes the
+ *                        default, lowered until batch * num_q_heads * num_splits partials (1552 B each)
+ *                        fit in the array
+ * Errors: OMNIKV_ERR_CAPACITY if the partials do not fit (an explicit num_splits too large, or
+ * batch * num_q_heads above 5405); OMNIKV_ERR_CUDA if the array's device address cannot be obtained.
+ * Every GPU that loads the library holds the array until the process exits. Its device address is
+ * looked up (cudaGetSymbolAddress) by the first call made on each device; make that first call
+ * before any stream capture. All calls share the array, which keeps the last call's contents (no
+ * part of it needs to start at zero); calls that overlap on the GPU race on it, so run them on one
+ * stream or otherwise ordered. */
+#define OMNIKV_DECODE_STATIC_SCRATCH_BYTES (8u << 20)
+OMNIKV_API omnikv_status omnikv_decode_static(const omnikv_config* cfg, const omnikv_cache* cache, const void* q,
+                                              float* out, int32_t num_splits, void* stream);
+
 /* Static text for a status code. */
 OMNIKV_API const char* omnikv_status_string(omnikv_status status);
 
