@@ -25,6 +25,7 @@ struct WriteParams {
   const __half* v_new;
   const uint8_t* mod_new;
   int n_new;
+  int tc_values;  // 1: values of windows filled completely by this write are done by vrot_tc
 };
 
 struct DecodeParams {
@@ -52,6 +53,7 @@ struct CombineParams {
 };
 
 cudaError_t launch_write(const WriteParams& p, int batch, cudaStream_t stream);
+cudaError_t launch_vrot_tc(const WriteParams& p, int batch, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeParams& p, int batch, cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams& p, int batch, cudaStream_t stream);
 

@@ -124,6 +124,17 @@ kv_quant_pack_kernel(const WriteParams p) {
   }
   __syncthreads();  // kp is reused for values below
 
+  // windows filled completely by this write get their values from vrot_tc
+  const bool tc_window = p.tc_values && p0 >= L0 && nvalid == kWindow;
+  if (tc_window) {
+    if (h == 0 && tid < kWindow) {
+      const int m = mnew[p0 + tid - L0];
+      if (m >= kMods) set_error(p.error_word, OMNIKV_DEVERR_MODALITY);
+      p.modality[(size_t)b * p.cap_tokens + p0 + tid] = (uint8_t)(m >= kMods ? kMods - 1 : m);
+    }
+    return;
+  }
+
   // ---- values: per-token scale (pairwise tree in a warp) ----------------------
   for (int i = inew0 + warp; i < nvalid; i += kWriteThreads / 32) {
     const __half* src = vnew + (size_t)(p0 + i - L0) * kHeadDim;
@@ -209,12 +220,18 @@ __global__ void finish_write_kernel(const WriteParams p) {
 
 }  // namespace
 
-cudaError_t launch_write(const WriteParams& p, int batch, cudaStream_t stream) {
+cudaError_t launch_write(const WriteParams& p_in, int batch, cudaStream_t stream) {
+  WriteParams p = p_in;
+  p.tc_values = p.n_new >= kWindow ? 1 : 0;  // a write this long can fill whole windows
   const int slots = (p.n_new + kWindow - 1) / kWindow + 1;
   dim3 grid(slots, p.num_kv_heads, batch);
   kv_quant_pack_kernel<<<grid, kWriteThreads, 0, stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (p.tc_values) {
+    e = launch_vrot_tc(p, batch, stream);
+    if (e != cudaSuccess) return e;
+  }
   finish_write_kernel<<<batch, 128, 0, stream>>>(p);
   return cudaGetLastError();
 }

@@ -134,7 +134,9 @@ OMNIKV_API int32_t omnikv_default_splits(const omnikv_config* cfg, const omnikv_
  * m = fp16(min), s = fp16((max - min) / (c_last - c_0)), code = #{j : (k' - m) / s + c_0 > t_j},
  * t_j = fp32((c_j + c_{j+1}) * 0.5), code 0 where s == 0. A window left partial keeps its raw keys in
  * key_tail. Values: sigma = fp16(sqrt(pairwise-tree sum of v_c^2 / 128)) of the unrotated fp16 value,
- * v' = U_m^T v (fp32 accumulation), code = #{j : v'_c / sigma > t_j}, 0 where sigma == 0.
+ * v' = U_m^T v (windows the write fills completely: tcgen05 tensor cores, fp16 values times U split into
+ * fp16 high + low parts, fp32 accumulation; other tokens: fp32 FMA), code = #{j : v'_c / sigma > t_j},
+ * 0 where sigma == 0.
  * Key codes and metadata are bit-exact with a scalar fp32 evaluation in this order; value codes
  * depend on the fp32-accumulated rotation and may differ from an fp64 rotation only where v'/sigma
  * lies within rounding of a threshold.
