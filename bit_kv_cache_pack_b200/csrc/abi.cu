@@ -74,6 +74,7 @@ omnikv_status prepare_decode(const omnikv_config* cfg, const omnikv_cache* cache
   p->key_cb = cfg->key_codebook;
   p->val_cb = cfg->value_codebook;
   p->key_signs = cfg->key_signs;
+  p->value_rot = cfg->value_rot;
   p->key_bits = cfg->key_bits;
   p->value_bits = cfg->value_bits;
   p->num_kv_heads = cfg->num_kv_heads;

@@ -276,6 +276,20 @@ __device__ __forceinline__ void issue_window(const DecodeParams& p, DecodeSmem& 
   bulk_copy_g2s(dst + kRec22, p.modality + (size_t)b * p.cap_tokens + (size_t)wi * kWindow, kWindow, bar);
 }
 
+// Each warp's first kStages windows: barrier set-up and bulk copies (lane 0).
+__device__ __forceinline__ void prime_pipeline(const DecodeParams& p, DecodeSmem& sm, int b, int kvh, int w0, int w1) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint8_t* rec_base = p.records + ((size_t)(b * p.num_kv_heads + kvh) * p.cap_windows) * kRec22;
+  const int nmine = (w1 - w0 > warp) ? (w1 - w0 - warp + kWarps - 1) / kWarps : 0;
+  if (lane == 0) {
+#pragma unroll
+    for (int s = 0; s < kStages; ++s) mbar_init(&sm.bar[warp][s], 1);
+    fence_barrier_init();
+    for (int i = 0; i < kStages && i < nmine; ++i) issue_window(p, sm, warp, i, rec_base, b, w0 + warp + kWarps * i);
+  }
+  __syncwarp();
+}
+
 __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh, int split, float kV0, float kV1,
                            float vc0) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -286,15 +300,6 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
   split_range(p, b, split, T, w0, w1);
   const uint8_t* rec_base = p.records + ((size_t)(b * p.num_kv_heads + kvh) * p.cap_windows) * kRec22;
   const int nmine = (w1 - w0 > warp) ? (w1 - w0 - warp + kWarps - 1) / kWarps : 0;
-
-  if (lane == 0) {
-#pragma unroll
-    for (int s = 0; s < kStages; ++s) mbar_init(&sm.bar[warp][s], 1);
-    fence_barrier_init();
-  }
-  __syncwarp();
-  if (lane == 0)
-    for (int i = 0; i < kStages && i < nmine; ++i) issue_window(p, sm, warp, i, rec_base, b, w0 + warp + kWarps * i);
 
   WarpState st;
 #pragma unroll
@@ -665,30 +670,42 @@ __device__ __forceinline__ void build_score_operand(DecodeSmem& sm, float k0scal
 __global__ void __launch_bounds__(kThreads, 2) decode_split_k_kernel(const DecodeParams p) {
   __shared__ DecodeSmem sm;
   const int b = blockIdx.z, kvh = blockIdx.y, split = blockIdx.x;
-  {
-    int T, w0, w1;
-    split_range(p, b, split, T, w0, w1);
-    if (w0 == w1) {  // empty split (short sequence): only m and l are read by the combine
-      if (threadIdx.x < p.group) {
-        Partial* out = p.partials + ((size_t)b * p.num_kv_heads * p.group + kvh * p.group + threadIdx.x) * p.num_splits + split;
-        out->m = -INFINITY;
-        out->l = 0.0f;
-      }
-      return;
+  int T, w0, w1;
+  split_range(p, b, split, T, w0, w1);
+  if (w0 == w1) {  // empty split (short sequence): only m and l are read by the combine
+    if (threadIdx.x < p.group) {
+      Partial* out = p.partials + ((size_t)b * p.num_kv_heads * p.group + kvh * p.group + threadIdx.x) * p.num_splits + split;
+      out->m = -INFINITY;
+      out->l = 0.0f;
     }
+    return;
+  }
+  bool fast = false;
+  float k0 = 0.f, k1 = 0.f, k2 = 0.f, v0 = 0.f, v1 = 0.f, v2 = 0.f;
+  if (p.key_bits == 2 && p.value_bits == 2) {
+    k0 = p.key_cb[0], k1 = p.key_cb[1], k2 = p.key_cb[2];
+    const float k3 = p.key_cb[3];
+    v0 = p.val_cb[0], v1 = p.val_cb[1], v2 = p.val_cb[2];
+    const float v3 = p.val_cb[3];
+    fast = (k0 == -k3) && (k1 == -k2) && (v0 == -v3) && (v1 == -v2);
+  }
+  if (fast) prime_pipeline(p, sm, b, kvh, w0, w1);  // window copies start before the query work
+  // warm the L2 with this split's share of the value bases, read by the combine
+  {
+    const size_t ubytes = (size_t)kMods * kHeadDim * kHeadDim * sizeof(float);
+    const size_t share = (ubytes + p.num_splits - 1) / p.num_splits;
+    const char* ub = reinterpret_cast<const char*>(p.value_rot) + (size_t)kvh * ubytes;
+    for (size_t off = (size_t)split * share + 128 * threadIdx.x; off < min(ubytes, (size_t)(split + 1) * share);
+         off += 128 * kThreads)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(ub + off));
   }
   rotate_queries(p, b, kvh, sm.q);
   __syncthreads();
-  if (p.key_bits == 2 && p.value_bits == 2) {
-    const float k0 = p.key_cb[0], k1 = p.key_cb[1], k2 = p.key_cb[2], k3 = p.key_cb[3];
-    const float v0 = p.val_cb[0], v1 = p.val_cb[1], v2 = p.val_cb[2], v3 = p.val_cb[3];
-    const bool symmetric = (k0 == -k3) && (k1 == -k2) && (v0 == -v3) && (v1 == -v2);
-    if (symmetric) {
-      build_score_operand(sm, (k1 - k0) * 128.0f, (k2 - k0) * 0.5f);
-      __syncthreads();
-      decode_mma(p, sm, b, kvh, split, (v1 - v0) * 128.0f, (v2 - v0) * 0.5f, v0);
-      return;
-    }
+  if (fast) {
+    build_score_operand(sm, (k1 - k0) * 128.0f, (k2 - k0) * 0.5f);
+    __syncthreads();
+    decode_mma(p, sm, b, kvh, split, (v1 - v0) * 128.0f, (v2 - v0) * 0.5f, v0);
+    return;
   }
   decode_generic(p, sm, b, kvh, split);
 }

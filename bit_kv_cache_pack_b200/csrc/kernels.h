@@ -32,6 +32,7 @@ struct DecodeParams {
   const float* key_cb;
   const float* val_cb;
   const float* key_signs;
+  const float* value_rot;  // only prefetched into L2 (for the combine)
   int key_bits, value_bits, num_kv_heads, group;
   const uint8_t* records;
   const uint8_t* modality;

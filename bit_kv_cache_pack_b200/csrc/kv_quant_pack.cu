@@ -61,14 +61,38 @@ kv_quant_pack_kernel(const WriteParams p) {
   const float kc0 = p.key_cb[0];
   const float kspan = __fsub_rn(p.key_cb[LK - 1], kc0);
 
+  // ---- issue every raw-key load of the window first (one memory round trip),
+  // and prefetch the value basis of the first new token into L2 so that the
+  // value rotation below reads it from L2
+  constexpr int kPerWarp = kWindow / (kWriteThreads / 32);
+  uint2 raws[kPerWarp];
+#pragma unroll
+  for (int k = 0; k < kPerWarp; ++k) {
+    const int i = warp + (kWriteThreads / 32) * k;
+    if (i < nvalid) {
+      const int pos = p0 + i;
+      const __half* src = pos < L0 ? tail + i * kHeadDim : knew + (size_t)(pos - L0) * kHeadDim;
+      raws[k] = *reinterpret_cast<const uint2*>(src + 4 * lane);
+    }
+  }
+  if (!(p.tc_values && p0 >= L0 && nvalid == kWindow)) {
+    int m0 = mnew[p0 + inew0 - L0];
+    m0 = m0 >= kMods ? kMods - 1 : m0;
+    const float* U = p.value_rot + ((size_t)(h * kMods + m0) * kHeadDim + tid) * kHeadDim;  // row tid
+#pragma unroll
+    for (int q = 0; q < 4; ++q) asm volatile("prefetch.global.L2 [%0];" ::"l"(U + 32 * q));
+  }
+
   // ---- keys: rotate every valid token of the window -------------------------
   float sg[4];
 #pragma unroll
   for (int r = 0; r < 4; ++r) sg[r] = p.key_signs[4 * lane + r];
-  for (int i = warp; i < nvalid; i += kWriteThreads / 32) {
+#pragma unroll
+  for (int k = 0; k < kPerWarp; ++k) {
+    const int i = warp + (kWriteThreads / 32) * k;
+    if (i >= nvalid) break;
     const int pos = p0 + i;
-    const __half* src = pos < L0 ? tail + i * kHeadDim : knew + (size_t)(pos - L0) * kHeadDim;
-    const uint2 raw = *reinterpret_cast<const uint2*>(src + 4 * lane);
+    const uint2 raw = raws[k];
     // the tail is written here only when this window is also the first one
     // touched (it reads old slots < L0 - p0 and writes new ones); a distinct
     // partial last window is copied by finish_write_kernel after this kernel.
