@@ -98,10 +98,14 @@ def load() -> ctypes.CDLL:
 
 
 def _ptr(x) -> int:
+    """Device address of a tensor (which must be contiguous: the C ABI takes
+    row-major dense arrays) or an integer address passed through."""
     if x is None:
         return 0
     if isinstance(x, int):
         return x
+    if hasattr(x, "is_contiguous") and not x.is_contiguous():
+        raise ValueError("tensor arguments of the C ABI must be contiguous (got strides %s)" % (x.stride(),))
     return int(x.data_ptr())
 
 

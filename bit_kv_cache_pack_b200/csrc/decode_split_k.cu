@@ -250,6 +250,13 @@ constexpr uint32_t kPlane1 = 0x40004000u;  // bit 14 of each half: 2
 
 __device__ __forceinline__ uint32_t rotl(uint32_t x, int n) { return __funnelshift_l(x, x, n); }
 
+// 2^x with the hardware approximation (relative error below 2^-22); -inf -> 0.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // (lo, hi) -> fp16 pair h = fp16(x) and l = fp16(x - h), each transposed to the
 // B-fragment layout with movmatrix.
 __device__ __forceinline__ void split_pair_t(float x0, float x1, uint32_t& hi, uint32_t& lo) {
@@ -368,46 +375,57 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
     const float off0 = __shfl_sync(0xffffffffu, off, 8 * t);      // head 2t
     const float off1 = __shfl_sync(0xffffffffu, off, 8 * t + 4);  // head 2t + 1
 
-    // ---- scores for the two 16-token tiles
+    // ---- scores for the two 16-token tiles, issued interleaved per chunk (4
+    // independent accumulator chains)
     float sc[2][4];
     int tokA[2], tokB[2];
+    uint2 kA[2], kB[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       tokA[h] = 16 * h + tile_token(g);
       tokB[h] = 16 * h + tile_token(g + 8);
-      const uint2 kA = *reinterpret_cast<const uint2*>(kw + tokA[h] * 8 + 2 * t);
-      const uint2 kB = *reinterpret_cast<const uint2*>(kw + tokB[h] * 8 + 2 * t);
-      float d0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, d1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      kA[h] = *reinterpret_cast<const uint2*>(kw + tokA[h] * 8 + 2 * t);
+      kB[h] = *reinterpret_cast<const uint2*>(kw + tokB[h] * 8 + 2 * t);
+    }
+    {
+      float d0[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      float d1[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
       for (int kc = 0; kc < 8; ++kc) {
-        uint32_t r[4];
-        if (kc < 7) {
-          r[0] = kA.x << (13 - 2 * kc);
-          r[1] = kB.x << (13 - 2 * kc);
-          r[2] = kA.y << (13 - 2 * kc);
-          r[3] = kB.y << (13 - 2 * kc);
-        } else {
-          r[0] = kA.x >> 1;
-          r[1] = kB.x >> 1;
-          r[2] = kA.y >> 1;
-          r[3] = kB.y >> 1;
-        }
         const uint32_t s0 = sp[kc][0], s1 = sp[kc][1];
-        const uint32_t a0[4] = {hmul2_u32(s0, r[0] & kPlane0), hmul2_u32(s0, r[1] & kPlane0),
-                                hmul2_u32(s1, r[2] & kPlane0), hmul2_u32(s1, r[3] & kPlane0)};
-        const uint32_t a1[4] = {hmul2_u32(s0, r[0] & kPlane1), hmul2_u32(s0, r[1] & kPlane1),
-                                hmul2_u32(s1, r[2] & kPlane1), hmul2_u32(s1, r[3] & kPlane1)};
         const uint4 bp0 = sm.btab[kc][0][lane], bp1 = sm.btab[kc][1][lane];
-        mma_f16_16816(d0, a0, bp0.x, bp0.y);
-        mma_f16_16816(d1, a1, bp1.x, bp1.y);
-        mma_f16_16816(d0, a0, bp0.z, bp0.w);
-        mma_f16_16816(d1, a1, bp1.z, bp1.w);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t r[4];
+          if (kc < 7) {
+            r[0] = kA[h].x << (13 - 2 * kc);
+            r[1] = kB[h].x << (13 - 2 * kc);
+            r[2] = kA[h].y << (13 - 2 * kc);
+            r[3] = kB[h].y << (13 - 2 * kc);
+          } else {
+            r[0] = kA[h].x >> 1;
+            r[1] = kB[h].x >> 1;
+            r[2] = kA[h].y >> 1;
+            r[3] = kB[h].y >> 1;
+          }
+          const uint32_t a0[4] = {hmul2_u32(s0, r[0] & kPlane0), hmul2_u32(s0, r[1] & kPlane0),
+                                  hmul2_u32(s1, r[2] & kPlane0), hmul2_u32(s1, r[3] & kPlane0)};
+          const uint32_t a1[4] = {hmul2_u32(s0, r[0] & kPlane1), hmul2_u32(s0, r[1] & kPlane1),
+                                  hmul2_u32(s1, r[2] & kPlane1), hmul2_u32(s1, r[3] & kPlane1)};
+          mma_f16_16816(d0[h], a0, bp0.x, bp0.y);
+          mma_f16_16816(d1[h], a1, bp1.x, bp1.y);
+          mma_f16_16816(d0[h], a0, bp0.z, bp0.w);
+          mma_f16_16816(d1[h], a1, bp1.z, bp1.w);
+        }
       }
-      const int posA = wi * kWindow + tokA[h], posB = wi * kWindow + tokB[h];
-      sc[h][0] = posA < T ? d0[0] + d1[0] + off0 : -INFINITY;
-      sc[h][1] = posA < T ? d0[1] + d1[1] + off1 : -INFINITY;
-      sc[h][2] = posB < T ? d0[2] + d1[2] + off0 : -INFINITY;
-      sc[h][3] = posB < T ? d0[3] + d1[3] + off1 : -INFINITY;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int posA = wi * kWindow + tokA[h], posB = wi * kWindow + tokB[h];
+        sc[h][0] = posA < T ? d0[h][0] + d1[h][0] + off0 : -INFINITY;
+        sc[h][1] = posA < T ? d0[h][1] + d1[h][1] + off1 : -INFINITY;
+        sc[h][2] = posB < T ? d0[h][2] + d1[h][2] + off0 : -INFINITY;
+        sc[h][3] = posB < T ? d0[h][3] + d1[h][3] + off1 : -INFINITY;
+      }
     }
 
     // ---- online softmax over the window
@@ -420,7 +438,7 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
     }
     const float mn0 = fmaxf(st.m[0], mx0), mn1 = fmaxf(st.m[1], mx1);
     if (__any_sync(0xffffffffu, mn0 > st.m[0] || mn1 > st.m[1])) {
-      const float a0 = exp2f((st.m[0] - mn0) * kLog2e), a1 = exp2f((st.m[1] - mn1) * kLog2e);
+      const float a0 = fast_exp2((st.m[0] - mn0) * kLog2e), a1 = fast_exp2((st.m[1] - mn1) * kLog2e);
       st.l[0] *= a0;
       st.l[1] *= a1;
 #pragma unroll
@@ -443,10 +461,10 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
     // ---- value product per tile
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const float p0 = exp2f(fmaf(sc[h][0], kLog2e, -ms0));
-      const float p1 = exp2f(fmaf(sc[h][1], kLog2e, -ms1));
-      const float p2 = exp2f(fmaf(sc[h][2], kLog2e, -ms0));
-      const float p3 = exp2f(fmaf(sc[h][3], kLog2e, -ms1));
+      const float p0 = fast_exp2(fmaf(sc[h][0], kLog2e, -ms0));
+      const float p1 = fast_exp2(fmaf(sc[h][1], kLog2e, -ms1));
+      const float p2 = fast_exp2(fmaf(sc[h][2], kLog2e, -ms0));
+      const float p3 = fast_exp2(fmaf(sc[h][3], kLog2e, -ms1));
       st.l[0] += p0 + p2;
       st.l[1] += p1 + p3;
       const float sgA = __half2float(sig[tokA[h]]), sgB = __half2float(sig[tokB[h]]);
@@ -580,7 +598,7 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) mm = fmaxf(mm, sm.mw[w][2 * t + j]);
     M[j] = mm;
-    const float f = (st.m[j] == -INFINITY) ? 0.0f : exp2f((st.m[j] - mm) * kLog2e);
+    const float f = (st.m[j] == -INFINITY) ? 0.0f : fast_exp2((st.m[j] - mm) * kLog2e);
     st.l[j] *= f;
 #pragma unroll
     for (int m = 0; m < kMods; ++m)

@@ -218,23 +218,21 @@ def pack_value_codes(codes, bits):
 
 
 def unpack_key_codes(words, bits):
+    """[32][128/cpw] u32 -> [32][128] codes (inverse of pack_key_codes)."""
     cpw = codes_per_word(bits)
     w = np.asarray(words, dtype=np.uint32).reshape(WINDOW, HEAD_DIM // cpw)
-    mask = np.uint32((1 << bits) - 1)
-    out = np.zeros((WINDOW, HEAD_DIM), dtype=np.uint32)
-    for c in range(HEAD_DIM):
-        out[:, c] = (w[:, c // cpw] >> np.uint32(bits * (c % cpw))) & mask
-    return out
+    c = np.arange(HEAD_DIM)
+    shifts = (bits * (c % cpw)).astype(np.uint32)
+    return (w[:, c // cpw] >> shifts[None, :]) & np.uint32((1 << bits) - 1)
 
 
 def unpack_value_codes(words, bits):
+    """[32/cpw][128] u32 -> [32][128] codes (inverse of pack_value_codes)."""
     cpw = codes_per_word(bits)
     w = np.asarray(words, dtype=np.uint32).reshape(WINDOW // cpw, HEAD_DIM)
-    mask = np.uint32((1 << bits) - 1)
-    out = np.zeros((WINDOW, HEAD_DIM), dtype=np.uint32)
-    for t in range(WINDOW):
-        out[t, :] = (w[t // cpw, :] >> np.uint32(bits * (t % cpw))) & mask
-    return out
+    t = np.arange(WINDOW)
+    shifts = (bits * (t % cpw)).astype(np.uint32)
+    return (w[t // cpw, :] >> shifts[:, None]) & np.uint32((1 << bits) - 1)
 
 
 # ----------------------------------------------------------------------------

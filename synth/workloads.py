@@ -253,9 +253,9 @@ def prefill_inputs(spec: WorkloadSpec, seed: int, layer: int, params, drift, len
     v = mu_t + sd_t * e
     valid = (torch.arange(T, device=device)[None, :] < torch.as_tensor(
         [int(lengths[b]) for b in bidx], device=device)[:, None])
-    k = (k * valid[:, None, :, None]).to(torch.float16)
-    v = (v * valid[:, None, :, None]).to(torch.float16)
-    return k, v, mod
+    k = (k * valid[:, None, :, None]).to(torch.float16).contiguous()
+    v = (v * valid[:, None, :, None]).to(torch.float16).contiguous()
+    return k, v, mod.contiguous()
 
 
 def decode_inputs(spec: WorkloadSpec, seed: int, layer: int, step: int, params, drift, positions, device):
@@ -271,6 +271,6 @@ def decode_inputs(spec: WorkloadSpec, seed: int, layer: int, step: int, params, 
     e = torch.randn(B, H, 1, HEAD_DIM, generator=g, device=device)
     mu = params["mu"].to(device)[:, TEXT]
     sd = params["lam"].to(device)[:, TEXT].sqrt()
-    v = (mu[None, :, None, :] + sd[None, :, None, :] * e).to(torch.float16)
+    v = (mu[None, :, None, :] + sd[None, :, None, :] * e).to(torch.float16).contiguous()
     mod = torch.zeros(B, 1, dtype=torch.uint8, device=device)
-    return q, k, v, mod
+    return q.contiguous(), k.contiguous(), v, mod

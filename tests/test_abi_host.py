@@ -120,3 +120,11 @@ def test_decode_and_combine_arguments_rejected():
     assert lib.omnikv_default_splits(ctypes.byref(bad), ctypes.byref(cache)) == 0
     with pytest.raises(_abi.OmniKVError):
         _abi.omnikv_decode_attention(cfg, cache, None, FAKE)
+
+
+def test_binding_rejects_non_contiguous_tensors():
+    import torch
+    t = torch.zeros(4, 8).t()
+    with pytest.raises(ValueError):
+        _abi._ptr(t)
+    assert _abi._ptr(torch.zeros(3)) != 0
