@@ -60,6 +60,20 @@ def dist_env():
     return world, rank, local
 
 
+def rank_seed(workload: str, rank: int) -> int:
+    """Each rank decodes its own batch (weak scaling): a different seed per rank."""
+    return WORKLOADS_KEYS.index(workload) + 1000 * rank
+
+
+def max_over_ranks(values, device, world):
+    """Elementwise maximum over all ranks of a list of timings (ms)."""
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -212,7 +226,7 @@ def run_gpu(args):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     spec = WORKLOADS[args.workload]
-    seed = WORKLOADS_KEYS.index(args.workload) + 1000 * rank
+    seed = rank_seed(args.workload, rank)
     K, W = args.steps, args.warmup
     total = W + K + K + 1  # device-resident run, then the e2e run
     wl = Workload(spec, seed, dev, total)
@@ -304,11 +318,11 @@ def run_gpu(args):
     h2d = int(dq.numel() * 2 + dk.numel() * 2 + dv.numel() * 2 + dm.numel())
     d2h = int(wl.out.numel() * 4)
 
+    # --- dense bf16 decode over the same context (comparison baseline) --------
+    dense = dense_baseline(spec, wl, dev, K, W, flush, stream)
+
     # --- max over ranks --------------------------------------------------------
-    t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, e2e_ms = float(t[0]), float(t[1])
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev, world)
     tokens = world * spec.batch * K
     value = tokens / (total_ms / 1e3)
     e2e_value = tokens / (e2e_ms / 1e3)
@@ -337,6 +351,7 @@ def run_gpu(args):
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": wl.launches_per_step() * K,
             "clocks": clk,
+            "dense_bf16": dense,
         }
         if not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(spec, seed)
@@ -346,6 +361,52 @@ def run_gpu(args):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def dense_baseline(spec, wl, dev, K, W, flush, stream):
+    """The library's dense bf16 split-K decode over an unquantised cache of the
+    same shape and context (random bf16 K/V), every layer, K timed steps with the
+    same L2 flush; compared with the packed path's decode + combine."""
+    import bit_kv_cache_pack_b200 as m
+    B, H, Hq = spec.batch, spec.num_kv_heads, spec.num_q_heads
+    T = wl.lengths.astype(np.int64) + W + K
+    cap = int(-(-int(T.max()) // 32) * 32)
+    g = torch.Generator(device=dev).manual_seed(99)
+    ks, vs, qs = [], [], []
+    for _ in range(spec.layers):
+        ks.append(torch.randn(B, H, cap, 128, generator=g, device=dev).to(torch.bfloat16))
+        vs.append(torch.randn(B, H, cap, 128, generator=g, device=dev).to(torch.bfloat16))
+        qs.append(torch.randn(B, Hq, 128, generator=g, device=dev).to(torch.bfloat16))
+    lens = torch.as_tensor(T, dtype=torch.int32, device=dev)
+    S = 0
+    part = torch.empty(m.omnikv_dense_partials_bytes(B, Hq, 4096) // 4, device=dev)
+    out = torch.empty(spec.layers, B, Hq, 128, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def step(st):
+        for layer in range(spec.layers):
+            m.omnikv_dense_decode_bf16(ks[layer], vs[layer], lens, B, Hq, H, cap, int(T.max()), qs[layer], part, S,
+                                       out[layer], err, st)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step(torch.cuda.current_stream())
+    times = []
+    with torch.cuda.stream(stream):
+        for i in range(W + K):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            graph.replay()
+            e1.record(stream)
+            times.append((e0, e1))
+    torch.cuda.synchronize(dev)
+    ms = float(np.mean([a.elapsed_time(b) for a, b in times[W:]]))
+    assert int(err.item()) == 0 and torch.isfinite(out).all()
+    bytes_step = spec.layers * (int(T.sum()) * H * 512 + B * Hq * 128 * 2)
+    del graph
+    return {"ms_per_step": round(ms, 4), "us_per_layer": round(ms * 1e3 / spec.layers, 3),
+            "tokens_per_s": round(B / (ms / 1e3), 3), "achieved_GBps": round(bytes_step / (ms / 1e3) / 1e9, 1),
+            "bytes_per_token_head": 512, "what": "decode attention only (no cache append), same context, bf16 K/V"}
 
 
 # ----------------------------------------------------------------------------

@@ -28,6 +28,7 @@ EXPORTED = (
     "omnikv_record_bytes", "omnikv_partials_bytes", "omnikv_default_splits",
     "omnikv_write_cache", "omnikv_decode_attention", "omnikv_combine",
     "omnikv_status_string", "omnikv_abi_version", "omnikv_decode_static",
+    "omnikv_dense_partials_bytes", "omnikv_dense_decode_bf16",
 )
 OMNIKV_DECODE_STATIC_SCRATCH_BYTES = 8 << 20
 
@@ -89,6 +90,9 @@ def load() -> ctypes.CDLL:
     lib.omnikv_decode_attention.restype = ctypes.c_int
     lib.omnikv_combine.argtypes = [cfgp, cachep, P, I32, P, P]
     lib.omnikv_combine.restype = ctypes.c_int
+    lib.omnikv_dense_partials_bytes.argtypes, lib.omnikv_dense_partials_bytes.restype = [I32, I32, I32], SZ
+    lib.omnikv_dense_decode_bf16.argtypes = [P, P, P, I32, I32, I32, I32, I32, P, P, I32, P, P, P]
+    lib.omnikv_dense_decode_bf16.restype = ctypes.c_int
     lib.omnikv_decode_static.argtypes = [cfgp, cachep, P, P, I32, P]
     lib.omnikv_decode_static.restype = ctypes.c_int
     lib.omnikv_status_string.argtypes, lib.omnikv_status_string.restype = [ctypes.c_int], ctypes.c_char_p
@@ -168,3 +172,17 @@ def omnikv_decode_static(cfg: OmniKVConfig, cache: OmniKVCache, q, out, num_spli
     st = load().omnikv_decode_static(ctypes.byref(cfg), ctypes.byref(cache), _ptr(q), _ptr(out), int(num_splits),
                                      _stream(stream))
     _check(st, "omnikv_decode_static")
+
+
+def omnikv_dense_partials_bytes(batch: int, num_q_heads: int, num_splits: int) -> int:
+    return int(load().omnikv_dense_partials_bytes(batch, num_q_heads, num_splits))
+
+
+def omnikv_dense_decode_bf16(k_cache, v_cache, seq_lens, batch: int, num_q_heads: int, num_kv_heads: int,
+                             cap_tokens: int, max_seq_len: int, q, partials, num_splits: int, out,
+                             error_word=None, stream=None) -> None:
+    """Dense bf16 split-K decode (comparison baseline); see include/omnikv.h."""
+    st = load().omnikv_dense_decode_bf16(_ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), int(batch), int(num_q_heads),
+                                         int(num_kv_heads), int(cap_tokens), int(max_seq_len), _ptr(q), _ptr(partials),
+                                         int(num_splits), _ptr(out), _ptr(error_word), _stream(stream))
+    _check(st, "omnikv_dense_decode_bf16")

@@ -187,6 +187,47 @@ omnikv_status omnikv_combine(const omnikv_config* cfg, const omnikv_cache* cache
   return OMNIKV_OK;
 }
 
+size_t omnikv_dense_partials_bytes(int32_t batch, int32_t num_q_heads, int32_t num_splits) {
+  if (batch < 1 || num_q_heads < 1 || num_splits < 1) return 0;
+  return (size_t)batch * num_q_heads * num_splits * kDensePartialFloats * sizeof(float);
+}
+
+omnikv_status omnikv_dense_decode_bf16(const void* k_cache, const void* v_cache, const int32_t* seq_lens, int32_t batch,
+                                       int32_t num_q_heads, int32_t num_kv_heads, int32_t cap_tokens,
+                                       int32_t max_seq_len, const void* q, void* partials, int32_t num_splits,
+                                       float* out, int32_t* error_word, void* stream) {
+  if (!k_cache || !v_cache || !seq_lens || !q || !partials || !out) return OMNIKV_ERR_INVALID_ARG;
+  if (batch < 1 || num_kv_heads < 1 || num_q_heads < 1 || num_q_heads % num_kv_heads) return OMNIKV_ERR_INVALID_ARG;
+  if (num_q_heads / num_kv_heads > kMaxGroup) return OMNIKV_ERR_UNSUPPORTED;
+  if (cap_tokens < 1 || max_seq_len < 0 || max_seq_len > cap_tokens || num_splits < 0) return OMNIKV_ERR_INVALID_ARG;
+  if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(q, 4) || !aligned(partials, 16) || !aligned(out, 16))
+    return OMNIKV_ERR_INVALID_ARG;
+  DenseParams p;
+  p.k = static_cast<const __nv_bfloat16*>(k_cache);
+  p.v = static_cast<const __nv_bfloat16*>(v_cache);
+  p.seq_lens = seq_lens;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.partials = static_cast<float*>(partials);
+  p.out = out;
+  p.error_word = error_word;
+  p.num_kv_heads = num_kv_heads;
+  p.group = num_q_heads / num_kv_heads;
+  p.cap_tokens = cap_tokens;
+  const int nc = (max_seq_len + 31) / 32;
+  int S = num_splits;
+  if (S == 0) {
+    const long long units = (long long)batch * num_kv_heads;
+    long long s = sm_count() / units;
+    if (s > (nc + 7) / 8) s = (nc + 7) / 8;
+    S = (int)(s < 1 ? 1 : s);
+  }
+  if (S > kMaxSplits) return OMNIKV_ERR_UNSUPPORTED;
+  p.num_splits = S;
+  p.split_chunks = nc > 0 ? (nc + S - 1) / S : 1;
+  if (launch_dense(p, batch, static_cast<cudaStream_t>(stream)) != cudaSuccess) return OMNIKV_ERR_CUDA;
+  return OMNIKV_OK;
+}
+
 const char* omnikv_status_string(omnikv_status s) {
   switch (s) {
     case OMNIKV_OK: return "ok";

@@ -1,6 +1,7 @@
 // Launch parameters and launchers of the OmniKVQuant kernels (internal).
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -52,6 +53,20 @@ struct CombineParams {
   int num_splits;
   float* out;
 };
+
+// Dense bf16 decode (comparison baseline).
+constexpr int kDensePartialFloats = 132;  // acc[128], m, l, 2 pad
+struct DenseParams {
+  const __nv_bfloat16* k;  // [B][H_kv][cap][128]
+  const __nv_bfloat16* v;
+  const int32_t* seq_lens;
+  const __nv_bfloat16* q;  // [B][H_q][128]
+  float* partials;         // [B][H_q][S][132]
+  float* out;              // [B][H_q][128]
+  int32_t* error_word;
+  int num_kv_heads, group, cap_tokens, num_splits, split_chunks;
+};
+cudaError_t launch_dense(const DenseParams& p, int batch, cudaStream_t stream);
 
 cudaError_t launch_write(const WriteParams& p, int batch, cudaStream_t stream);
 cudaError_t launch_vrot_tc(const WriteParams& p, int batch, cudaStream_t stream);

@@ -189,6 +189,21 @@ OMNIKV_API omnikv_status omnikv_combine(const omnikv_config* cfg, const omnikv_c
 OMNIKV_API omnikv_status omnikv_decode_static(const omnikv_config* cfg, const omnikv_cache* cache, const void* q,
                                               float* out, int32_t num_splits, void* stream);
 
+/* Dense bf16 split-K decode attention over an unquantised cache: the comparison baseline for the
+ * packed kernels (the same attention read at 512 B per token and kv head). Not part of the method.
+ *   k_cache, v_cache : [batch][num_kv_heads][cap_tokens][128] bf16, 16-byte aligned
+ *   seq_lens         : [batch] device; max_seq_len a host bound on them
+ *   q                : [batch][num_q_heads][128] bf16; scores q.k / sqrt(128)
+ *   partials         : device buffer of omnikv_dense_partials_bytes(batch, num_q_heads, S) bytes
+ *   num_splits       : S >= 1, or 0 for a default; out: [batch][num_q_heads][128] fp32
+ *   error_word       : optional device int32 (OMNIKV_DEVERR_TIMEOUT) */
+OMNIKV_API size_t omnikv_dense_partials_bytes(int32_t batch, int32_t num_q_heads, int32_t num_splits);
+OMNIKV_API omnikv_status omnikv_dense_decode_bf16(const void* k_cache, const void* v_cache, const int32_t* seq_lens,
+                                                  int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                                                  int32_t cap_tokens, int32_t max_seq_len, const void* q,
+                                                  void* partials, int32_t num_splits, float* out,
+                                                  int32_t* error_word, void* stream);
+
 /* Static text for a status code. */
 OMNIKV_API const char* omnikv_status_string(omnikv_status status);
 
