@@ -52,11 +52,11 @@ int32_t resolve_splits(const omnikv_config* cfg, const omnikv_cache* c, int32_t 
   const int nw = (c->max_seq_len + kWindow - 1) / kWindow;
   if (nw <= 0) return 1;
   // aim at about two resident CTAs per SM over the whole batch, with at least
-  // 8 windows (2 per warp) per split so the per-CTA setup is amortised
+  // 4 windows (one per warp) per split
   const long long units = (long long)c->batch * cfg->num_kv_heads;
   const long long target = 2LL * sm_count();
   long long s = target / units;
-  const long long max_s = (nw + 7) / 8;
+  const long long max_s = (nw + 3) / 4;
   if (s > max_s) s = max_s;
   if (s < 1) s = 1;
   if (s > kMaxSplits) s = kMaxSplits;
