@@ -13,9 +13,11 @@ its own batch (different seed), so per-GPU work is fixed as N grows.
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events on
 the launching stream and preceded by an untimed L2 flush (a 512 MiB write);
 barrier + synchronize around the timed region; the max over ranks is reported.
-Each step is replayed from a CUDA graph that holds exactly the C-ABI calls of
-that step. `value` has all inputs resident in HBM; `e2e` also copies each step's
-inputs from pinned host memory and the step's outputs back to the host.
+All steps are replayed from one CUDA graph holding, per step, the L2 flush, the
+step's start event, exactly the C-ABI calls of the step, and its end event (no
+host gaps between steps). `value` has all inputs resident in HBM; `e2e` also
+copies each step's inputs from pinned host memory and the step's outputs back to
+the host (captured the same way).
 """
 from __future__ import annotations
 
@@ -187,26 +189,42 @@ class Workload:
         self.v = torch.stack(vs, 1).contiguous()
         self.mod = torch.stack(ms, 1).contiguous()
         self.S = max(1, m.omnikv_default_splits(self.consts[0].struct, self.caches[0].struct))
-        self.part = m.partials_tensor(spec.batch, spec.num_q_heads, self.S, device)
+        # the step's default split count grows (slightly) with the context: size
+        # the partials for its value at the longest context of the run
+        c0 = self.caches[0].struct
+        saved = c0.max_seq_len
+        c0.max_seq_len = int(self.lengths.max()) + total_steps
+        s_max = max(self.S, m.omnikv_default_splits(self.consts[0].struct, c0))
+        c0.max_seq_len = saved
+        self.part = m.partials_tensor(spec.batch, spec.num_q_heads, s_max, device)
         self.out = torch.empty(spec.layers, spec.batch, spec.num_q_heads, 128, dtype=torch.float32,
                                device=device)
 
     def step_calls(self, s, q, k, v, mod, stream, dec_events=None):
-        """The C-ABI calls of one decode step over all layers."""
+        """The C-ABI calls of one decode step over all layers: omnikv_decode_step
+        per layer (append + decode in one launch, then the combine launch). With
+        `dec_events` (a start/end pair), layer s % layers instead makes the same
+        step as three calls (write, decode, combine; identical results) with the
+        decode launch between the two events, so the decode kernel is timed in
+        place once per step."""
         m = self.m
         n = self.spec.layers
         for layer in range(n):
             c, cache = self.consts[layer].struct, self.caches[layer].struct
-            m.omnikv_write_cache(c, cache, k[layer], v[layer], mod[layer], 1, stream)
-            if dec_events is not None:
-                dec_events[layer][0].record(stream)
-            m.omnikv_decode_attention(c, cache, q[layer], self.part, self.S, stream)
-            if dec_events is not None:
-                dec_events[layer][1].record(stream)
-            m.omnikv_combine(c, cache, self.part, self.S, self.out[layer], stream)
+            if dec_events is not None and layer == s % n:
+                m.omnikv_write_cache(c, cache, k[layer], v[layer], mod[layer], 1, stream)
+                dec_events[0].record(stream)
+                m.omnikv_decode_attention(c, cache, q[layer], self.part, self.S, stream)
+                dec_events[1].record(stream)
+                m.omnikv_combine(c, cache, self.part, self.S, self.out[layer], stream)
+            else:
+                m.omnikv_decode_step(c, cache, q[layer], k[layer], v[layer], mod[layer], self.part, 0,
+                                     self.out[layer], stream)
 
-    def launches_per_step(self):
-        return self.spec.layers * 4   # write + finish_write + decode + combine
+    def launches_per_step(self, instrumented):
+        """Library kernel launches in one step: 2 per layer (decode step +
+        combine), 3 in the instrumented layer (append + decode + combine)."""
+        return 2 * self.spec.layers + (1 if instrumented else 0)
 
     def decode_bytes(self, s):
         """Algorithmic bytes one decode launch reads at step s (per layer): packed
@@ -234,49 +252,46 @@ def run_gpu(args):
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     torch.cuda.synchronize(dev)
 
-    # --- device-resident steps, each from a captured graph ---------------------
-    dec_ev = [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in range(spec.layers)]
-              for _ in range(W + K)]
-    graphs = []
+    # --- device-resident steps: one graph holding, per step, the L2 flush, the
+    # start event, the step's C-ABI calls and the end event (no host gaps) -------
+    ev = lambda: torch.cuda.Event(enable_timing=True, external=True)
+    dec_ev = [(ev(), ev()) for _ in range(W + K)]
+    step_ev = [(ev(), ev()) for _ in range(W + K)]
     use_graphs = not args.no_graphs
+    graph = None
     if use_graphs:
-        pool = None
-        for s in range(W + K):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, pool=pool, stream=stream):
-                wl.step_calls(s, wl.q[s], wl.k[s], wl.v[s], wl.mod[s], torch.cuda.current_stream(),
-                              dec_ev[s])
-            pool = g.pool()
-            graphs.append(g)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            cs = torch.cuda.current_stream()
+            for s in range(W + K):
+                flush.zero_()
+                step_ev[s][0].record(cs)
+                wl.step_calls(s, wl.q[s], wl.k[s], wl.v[s], wl.mod[s], cs, dec_ev[s])
+                step_ev[s][1].record(cs)
     torch.cuda.synchronize(dev)
-    t_steps = []
     clocks = ClockSampler(local, args.clocks_csv)
     if world > 1:
         dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
     with torch.cuda.stream(stream):
-        for s in range(W + K):
-            flush.zero_()
-            if s == W:
-                torch.cuda.synchronize(dev)
-                if world > 1:
-                    dist.barrier()
-                clocks.start()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            if use_graphs:
-                graphs[s].replay()
-            else:
+        if use_graphs:
+            graph.replay()
+        else:
+            for s in range(W + K):
+                flush.zero_()
+                step_ev[s][0].record(stream)
                 wl.step_calls(s, wl.q[s], wl.k[s], wl.v[s], wl.mod[s], stream, dec_ev[s])
-            e1.record(stream)
-            t_steps.append((e0, e1))
+                step_ev[s][1].record(stream)
     torch.cuda.synchronize(dev)
     clk = clocks.stop()
-    step_ms = [a.elapsed_time(b) for a, b in t_steps[W:]]
-    dec_ms = [dec_ev[s][l][0].elapsed_time(dec_ev[s][l][1]) for s in range(W, W + K) for l in range(spec.layers)]
-    dec_bytes = [wl.decode_bytes(s) for s in range(W, W + K) for _ in range(spec.layers)]
+    step_ms = [a.elapsed_time(b) for a, b in step_ev[W:]]
+    dec_ms = [dec_ev[s][0].elapsed_time(dec_ev[s][1]) for s in range(W, W + K)]
+    dec_bytes = [wl.decode_bytes(s) for s in range(W, W + K)]
     total_ms = float(np.sum(step_ms))
 
-    # --- end to end through the C ABI with host buffers ------------------------
+    # --- end to end through the C ABI with host buffers: per step the H2D copy of
+    # the step's inputs from pinned memory and the D2H copy of its outputs --------
     hq = wl.q[W + K:].cpu().pin_memory()
     hk = wl.k[W + K:].cpu().pin_memory()
     hv = wl.v[W + K:].cpu().pin_memory()
@@ -284,34 +299,32 @@ def run_gpu(args):
     hout = torch.empty((K,) + tuple(wl.out.shape), dtype=torch.float32).pin_memory()
     dq, dk, dv, dm = (torch.empty_like(wl.q[0]), torch.empty_like(wl.k[0]), torch.empty_like(wl.v[0]),
                       torch.empty_like(wl.mod[0]))
-    e2e_graphs = []
-    if use_graphs:
-        for i in range(K):
-            s = W + K + i
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, pool=pool, stream=stream):
-                wl.step_calls(s, dq, dk, dv, dm, torch.cuda.current_stream())
-            e2e_graphs.append(g)
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
-    e2e_ev = []
-    with torch.cuda.stream(stream):
+    e2e_ev = [(ev(), ev()) for _ in range(K)]
+
+    def e2e_steps(cs):
         for i in range(K):
             flush.zero_()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
+            e2e_ev[i][0].record(cs)
             dq.copy_(hq[i], non_blocking=True)
             dk.copy_(hk[i], non_blocking=True)
             dv.copy_(hv[i], non_blocking=True)
             dm.copy_(hm[i], non_blocking=True)
-            if use_graphs:
-                e2e_graphs[i].replay()
-            else:
-                wl.step_calls(W + K + i, dq, dk, dv, dm, stream)
+            wl.step_calls(W + K + i, dq, dk, dv, dm, cs)
             hout[i].copy_(wl.out, non_blocking=True)
-            e1.record(stream)
-            e2e_ev.append((e0, e1))
+            e2e_ev[i][1].record(cs)
+    g2 = None
+    if use_graphs:
+        g2 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g2, stream=stream):
+            e2e_steps(torch.cuda.current_stream())
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    with torch.cuda.stream(stream):
+        if use_graphs:
+            g2.replay()
+        else:
+            e2e_steps(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = float(np.sum([a.elapsed_time(b) for a, b in e2e_ev]))
     assert torch.isfinite(hout).all(), "non-finite decode output"
@@ -341,7 +354,8 @@ def run_gpu(args):
                        "value_bits": spec.value_bits, "window": 32, "num_splits": wl.S,
                        "parallelism": "dp%d (independent sequences per rank)" % world,
                        "l2": "flushed between timed steps (512 MiB write)",
-                       "launch": "CUDA graph per step" if use_graphs else "eager"},
+                       "launch": "one CUDA graph for all steps (flush + events + C-ABI calls)" if use_graphs
+                       else "eager"},
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": None,
                          "peak_source": peak_kind, "kernel": "decode_split_k",
@@ -349,15 +363,14 @@ def run_gpu(args):
                          "bytes_per_launch": int(np.mean(dec_bytes))},
             "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": wl.launches_per_step() * K,
+            "gpu_launches": wl.launches_per_step(True) * K,
             "clocks": clk,
             "dense_bf16": dense,
         }
         if not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(spec, seed)
         print(json.dumps(line), flush=True)
-    graphs.clear()
-    e2e_graphs.clear()
+    del graph, g2
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

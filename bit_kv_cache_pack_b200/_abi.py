@@ -28,7 +28,7 @@ EXPORTED = (
     "omnikv_record_bytes", "omnikv_partials_bytes", "omnikv_default_splits",
     "omnikv_write_cache", "omnikv_decode_attention", "omnikv_combine",
     "omnikv_status_string", "omnikv_abi_version", "omnikv_decode_static",
-    "omnikv_dense_partials_bytes", "omnikv_dense_decode_bf16",
+    "omnikv_dense_partials_bytes", "omnikv_dense_decode_bf16", "omnikv_decode_step",
 )
 OMNIKV_DECODE_STATIC_SCRATCH_BYTES = 8 << 20
 
@@ -64,6 +64,7 @@ class OmniKVCache(ctypes.Structure):
         ("batch", ctypes.c_int32),
         ("cap_tokens", ctypes.c_int32),
         ("max_seq_len", ctypes.c_int32),
+        ("step_flags", ctypes.c_void_p),
     ]
 
 
@@ -93,6 +94,8 @@ def load() -> ctypes.CDLL:
     lib.omnikv_dense_partials_bytes.argtypes, lib.omnikv_dense_partials_bytes.restype = [I32, I32, I32], SZ
     lib.omnikv_dense_decode_bf16.argtypes = [P, P, P, I32, I32, I32, I32, I32, P, P, I32, P, P, P]
     lib.omnikv_dense_decode_bf16.restype = ctypes.c_int
+    lib.omnikv_decode_step.argtypes = [cfgp, cachep, P, P, P, P, P, I32, P, P]
+    lib.omnikv_decode_step.restype = ctypes.c_int
     lib.omnikv_decode_static.argtypes = [cfgp, cachep, P, P, I32, P]
     lib.omnikv_decode_static.restype = ctypes.c_int
     lib.omnikv_status_string.argtypes, lib.omnikv_status_string.restype = [ctypes.c_int], ctypes.c_char_p
@@ -164,6 +167,15 @@ def omnikv_combine(cfg: OmniKVConfig, cache: OmniKVCache, partials, num_splits: 
     st = load().omnikv_combine(ctypes.byref(cfg), ctypes.byref(cache), _ptr(partials), int(num_splits),
                                _ptr(out), _stream(stream))
     _check(st, "omnikv_combine")
+
+
+def omnikv_decode_step(cfg: OmniKVConfig, cache: OmniKVCache, q, k_new, v_new, modality_new, partials,
+                       num_splits: int, out, stream=None) -> None:
+    """Append one token per sequence, decode and combine (see include/omnikv.h);
+    the cache needs its step_flags array."""
+    st = load().omnikv_decode_step(ctypes.byref(cfg), ctypes.byref(cache), _ptr(q), _ptr(k_new), _ptr(v_new),
+                                   _ptr(modality_new), _ptr(partials), int(num_splits), _ptr(out), _stream(stream))
+    _check(st, "omnikv_decode_step")
 
 
 def omnikv_decode_static(cfg: OmniKVConfig, cache: OmniKVCache, q, out, num_splits: int = 0, stream=None) -> None:

@@ -51,10 +51,11 @@ int32_t resolve_splits(const omnikv_config* cfg, const omnikv_cache* c, int32_t 
   if (requested > 0) return requested;
   const int nw = (c->max_seq_len + kWindow - 1) / kWindow;
   if (nw <= 0) return 1;
-  // aim at about two resident CTAs per SM over the whole batch, with at least
-  // 4 windows (one per warp) per split
+  // aim at one full wave of resident decode CTAs over the whole batch (a
+  // second, partial wave would double the time), with at least 4 windows (one
+  // per warp) per split
   const long long units = (long long)c->batch * cfg->num_kv_heads;
-  const long long target = 2LL * sm_count();
+  const long long target = (long long)decode_ctas_per_sm() * sm_count();
   long long s = target / units;
   const long long max_s = (nw + 3) / 4;
   if (s > max_s) s = max_s;
@@ -91,6 +92,9 @@ omnikv_status prepare_decode(const omnikv_config* cfg, const omnikv_cache* cache
   const int nw = (cache->max_seq_len + kWindow - 1) / kWindow;
   p->split_windows = nw > 0 ? (nw + p->num_splits - 1) / p->num_splits : 1;
   p->error_word = cache->error_word;
+  p->batch = cache->batch;
+  p->len_add = 0;
+  p->step_flags = nullptr;
   return OMNIKV_OK;
 }
 
@@ -108,6 +112,9 @@ omnikv_status prepare_combine(const omnikv_config* cfg, const omnikv_cache* cach
   p->num_splits = resolve_splits(cfg, cache, num_splits);
   if (p->num_splits > kMaxSplits) return OMNIKV_ERR_UNSUPPORTED;
   p->out = out;
+  p->seq_lens = cache->seq_lens;
+  p->len_add = 0;
+  p->cap_tokens = cache->cap_tokens;
   return OMNIKV_OK;
 }
 
@@ -136,6 +143,34 @@ int32_t omnikv_default_splits(const omnikv_config* cfg, const omnikv_cache* cach
   return resolve_splits(cfg, cache, 0);
 }
 
+namespace {
+
+void fill_write_params(const omnikv_config* cfg, const omnikv_cache* cache, const void* k_new, const void* v_new,
+                       const uint8_t* modality_new, int32_t n_new, WriteParams* p) {
+  p->key_cb = cfg->key_codebook;
+  p->val_cb = cfg->value_codebook;
+  p->key_signs = cfg->key_signs;
+  p->value_rot = cfg->value_rot;
+  p->key_bits = cfg->key_bits;
+  p->value_bits = cfg->value_bits;
+  p->num_kv_heads = cfg->num_kv_heads;
+  p->records = static_cast<uint8_t*>(cache->records);
+  p->key_tail = static_cast<__half*>(cache->key_tail);
+  p->modality = cache->modality;
+  p->seq_lens = cache->seq_lens;
+  p->error_word = cache->error_word;
+  p->cap_tokens = cache->cap_tokens;
+  p->cap_windows = cache->cap_tokens / kWindow;
+  p->k_new = static_cast<const __half*>(k_new);
+  p->v_new = static_cast<const __half*>(v_new);
+  p->mod_new = modality_new;
+  p->n_new = n_new;
+  p->tc_values = 0;
+  p->step_flags = nullptr;
+}
+
+}  // namespace
+
 omnikv_status omnikv_write_cache(const omnikv_config* cfg, omnikv_cache* cache, const void* k_new,
                                  const void* v_new, const uint8_t* modality_new, int32_t n_new,
                                  void* stream) {
@@ -146,24 +181,7 @@ omnikv_status omnikv_write_cache(const omnikv_config* cfg, omnikv_cache* cache, 
   if (!aligned(k_new, 16) || !aligned(v_new, 16)) return OMNIKV_ERR_INVALID_ARG;
   if ((long long)cache->max_seq_len + n_new > cache->cap_tokens) return OMNIKV_ERR_CAPACITY;
   WriteParams p;
-  p.key_cb = cfg->key_codebook;
-  p.val_cb = cfg->value_codebook;
-  p.key_signs = cfg->key_signs;
-  p.value_rot = cfg->value_rot;
-  p.key_bits = cfg->key_bits;
-  p.value_bits = cfg->value_bits;
-  p.num_kv_heads = cfg->num_kv_heads;
-  p.records = static_cast<uint8_t*>(cache->records);
-  p.key_tail = static_cast<__half*>(cache->key_tail);
-  p.modality = cache->modality;
-  p.seq_lens = cache->seq_lens;
-  p.error_word = cache->error_word;
-  p.cap_tokens = cache->cap_tokens;
-  p.cap_windows = cache->cap_tokens / kWindow;
-  p.k_new = static_cast<const __half*>(k_new);
-  p.v_new = static_cast<const __half*>(v_new);
-  p.mod_new = modality_new;
-  p.n_new = n_new;
+  fill_write_params(cfg, cache, k_new, v_new, modality_new, n_new, &p);
   if (launch_write(p, cache->batch, static_cast<cudaStream_t>(stream)) != cudaSuccess) return OMNIKV_ERR_CUDA;
   cache->max_seq_len += n_new;
   return OMNIKV_OK;
@@ -184,6 +202,52 @@ omnikv_status omnikv_combine(const omnikv_config* cfg, const omnikv_cache* cache
   const omnikv_status st = prepare_combine(cfg, cache, partials, num_splits, out, &p);
   if (st != OMNIKV_OK) return st;
   if (launch_combine(p, cache->batch, static_cast<cudaStream_t>(stream)) != cudaSuccess) return OMNIKV_ERR_CUDA;
+  return OMNIKV_OK;
+}
+
+omnikv_status omnikv_decode_step(const omnikv_config* cfg, omnikv_cache* cache, const void* q, const void* k_new,
+                                 const void* v_new, const uint8_t* modality_new, void* partials, int32_t num_splits,
+                                 float* out, void* stream) {
+  omnikv_status st = check_config(cfg);
+  if (st != OMNIKV_OK) return st;
+  if ((st = check_cache(cache)) != OMNIKV_OK) return st;
+  if (!cache->step_flags || !q || !k_new || !v_new || !modality_new || !partials || !out) return OMNIKV_ERR_INVALID_ARG;
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(cache->step_flags, 4)) return OMNIKV_ERR_INVALID_ARG;
+  if ((long long)cache->max_seq_len + 1 > cache->cap_tokens) return OMNIKV_ERR_CAPACITY;
+  omnikv_cache after = *cache;  // the decode and combine see the appended token
+  after.max_seq_len += 1;
+  // fused (append CTAs inside the decode launch) only when every CTA of that
+  // launch is resident at once, so a waiting warp never waits on an unscheduled CTA
+  const long long units = (long long)cache->batch * cfg->num_kv_heads;
+  const long long resident = (long long)decode_ctas_per_sm() * sm_count();
+  int32_t S = resolve_splits(cfg, &after, num_splits);
+  bool fused = units * (1 + (long long)S) <= resident;
+  if (!fused && num_splits == 0) {
+    const long long s_res = resident / units - 1;
+    if (s_res >= 1 && 2 * s_res >= S) {
+      S = (int32_t)s_res;
+      fused = true;
+    }
+  }
+  DecodeParams dp;
+  if ((st = prepare_decode(cfg, &after, q, partials, S, &dp)) != OMNIKV_OK) return st;
+  CombineParams cp;
+  if ((st = prepare_combine(cfg, &after, partials, S, out, &cp)) != OMNIKV_OK) return st;
+  WriteParams wp;
+  fill_write_params(cfg, cache, k_new, v_new, modality_new, 1, &wp);
+  wp.step_flags = cache->step_flags;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (fused) {
+    dp.len_add = 1;
+    dp.step_flags = cache->step_flags;
+    cp.len_add = 1;
+    if (launch_decode_step(dp, wp, s) != cudaSuccess) return OMNIKV_ERR_CUDA;
+  } else {
+    if (launch_write(wp, cache->batch, s) != cudaSuccess) return OMNIKV_ERR_CUDA;
+    if (launch_decode(dp, cache->batch, s) != cudaSuccess) return OMNIKV_ERR_CUDA;
+  }
+  if (launch_combine(cp, cache->batch, s) != cudaSuccess) return OMNIKV_ERR_CUDA;
+  cache->max_seq_len += 1;
   return OMNIKV_OK;
 }
 

@@ -1,0 +1,223 @@
+// The per-window body of the OmniKVQuant cache write, shared by the write
+// kernels (kv_quant_pack.cu) and the decode-step kernel (decode_split_k.cu).
+// See kv_quant_pack.cu for the method and its sources.
+#pragma once
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace omnikv {
+namespace {
+
+constexpr int kWriteThreads = 128;  // one group of 128 threads per (window, kv head)
+
+struct __align__(16) WindowSmem {  // 16-byte multiple: per-group copies stay float4-aligned
+  float kp[kWindow][kHeadDim];  // rotated keys, then reused for fp32 values
+  float s_min[kHeadDim], s_scale[kHeadDim];
+  float s_sigma[kWindow];
+  float thr_k[15], thr_v[15];
+};
+
+static_assert(sizeof(WindowSmem) % 16 == 0, "per-group shared memory must keep 16-byte alignment");
+
+// Barrier over the 128 threads of one group (id 0 is __syncthreads).
+__device__ __forceinline__ void group_sync(int id) { asm volatile("bar.sync %0, 128;\n" ::"r"(id) : "memory"); }
+
+// Re-quantise window w of (sequence b, kv head h) after the append of
+// positions [L0, L1), by the 128 threads of one group (tid 0..127, barrier
+// bar_id). tail_any: this group also handles every other window the append
+// touches, in order, so a partial window always keeps its new raw keys in the
+// tail (otherwise only the first touched window does, and finish_write_kernel
+// copies those of a distinct partial last window).
+__device__ void quantize_window(const WriteParams& p, int b, int h, int w, int L0, int L1, WindowSmem& sm, int tid,
+                                int bar_id, bool tail_any) {
+  const int H = p.num_kv_heads;
+  const int p0 = w * kWindow;
+  const int p1 = min(p0 + kWindow, L1);
+  const int nvalid = p1 - p0;
+  const int inew0 = max(L0 - p0, 0);  // first slot of this window holding a new token
+
+  const RecordLayout lay(p.key_bits, p.value_bits);
+  uint8_t* rec = p.records + ((size_t)(b * H + h) * p.cap_windows + w) * lay.bytes;
+  const size_t seq_head = (size_t)b * H + h;
+  __half* tail = p.key_tail + seq_head * kWindow * kHeadDim;
+  const __half* knew = p.k_new + seq_head * p.n_new * kHeadDim;
+  const __half* vnew = p.v_new + seq_head * p.n_new * kHeadDim;
+  const uint8_t* mnew = p.mod_new + (size_t)b * p.n_new;
+
+  float (*kp)[kHeadDim] = sm.kp;
+  float* s_min = sm.s_min;
+  float* s_scale = sm.s_scale;
+  float* s_sigma = sm.s_sigma;
+  float* thr_k = sm.thr_k;
+  float* thr_v = sm.thr_v;
+
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int LK = 1 << p.key_bits;
+  const int LV = 1 << p.value_bits;
+  if (tid < LK - 1) thr_k[tid] = __fmul_rn(__fadd_rn(p.key_cb[tid], p.key_cb[tid + 1]), 0.5f);
+  if (tid < LV - 1) thr_v[tid] = __fmul_rn(__fadd_rn(p.val_cb[tid], p.val_cb[tid + 1]), 0.5f);
+  const float kc0 = p.key_cb[0];
+  const float kspan = __fsub_rn(p.key_cb[LK - 1], kc0);
+
+  // ---- issue every raw-key load of the window first (one memory round trip),
+  // and prefetch the value basis of the first new token into L2 so that the
+  // value rotation below reads it from L2
+  constexpr int kPerWarp = kWindow / (kWriteThreads / 32);
+  uint2 raws[kPerWarp];
+#pragma unroll
+  for (int k = 0; k < kPerWarp; ++k) {
+    const int i = warp + (kWriteThreads / 32) * k;
+    if (i < nvalid) {
+      const int pos = p0 + i;
+      const __half* src = pos < L0 ? tail + i * kHeadDim : knew + (size_t)(pos - L0) * kHeadDim;
+      raws[k] = *reinterpret_cast<const uint2*>(src + 4 * lane);
+    }
+  }
+  if (!(p.tc_values && p0 >= L0 && nvalid == kWindow)) {
+    int m0 = mnew[p0 + inew0 - L0];
+    m0 = m0 >= kMods ? kMods - 1 : m0;
+    const float* U = p.value_rot + ((size_t)(h * kMods + m0) * kHeadDim + tid) * kHeadDim;  // row tid
+#pragma unroll
+    for (int q = 0; q < 4; ++q) asm volatile("prefetch.global.L2 [%0];" ::"l"(U + 32 * q));
+  }
+
+  // ---- keys: rotate every valid token of the window -------------------------
+  float sg[4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) sg[r] = p.key_signs[4 * lane + r];
+#pragma unroll
+  for (int k = 0; k < kPerWarp; ++k) {
+    const int i = warp + (kWriteThreads / 32) * k;
+    if (i >= nvalid) break;
+    const int pos = p0 + i;
+    const uint2 raw = raws[k];
+    // the tail keeps the new raw keys of a window left partial (see tail_any)
+    if (nvalid < kWindow && pos >= L0 && (tail_any || w == L0 / kWindow))
+      *reinterpret_cast<uint2*>(tail + i * kHeadDim + 4 * lane) = raw;
+    const __half2 lo = *reinterpret_cast<const __half2*>(&raw.x);
+    const __half2 hi = *reinterpret_cast<const __half2*>(&raw.y);
+    float x[4] = {__low2float(lo), __high2float(lo), __low2float(hi), __high2float(hi)};
+    warp_hadamard_rotate(x, sg);
+    *reinterpret_cast<float4*>(&kp[i][4 * lane]) = make_float4(x[0], x[1], x[2], x[3]);
+  }
+  group_sync(bar_id);
+
+  // ---- window range per channel -> fp16 metadata -----------------------------
+  {
+    const int c = tid;
+    float mn = kp[0][c], mx = kp[0][c];
+    for (int i = 1; i < nvalid; ++i) {
+      mn = fminf(mn, kp[i][c]);
+      mx = fmaxf(mx, kp[i][c]);
+    }
+    const __half m16 = __float2half_rn(mn);
+    const __half s16 = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), kspan));
+    reinterpret_cast<__half2*>(rec + lay.meta_off)[c] = __halves2half2(m16, s16);
+    s_min[c] = __half2float(m16);
+    s_scale[c] = __half2float(s16);
+  }
+  group_sync(bar_id);
+
+  // ---- key codes, token-major words -----------------------------------------
+  {
+    const int cpw = 32 / p.key_bits;
+    const int wpt = kHeadDim / cpw;
+    uint32_t* kw = reinterpret_cast<uint32_t*>(rec + lay.k_off);
+    for (int wi = tid; wi < kWindow * wpt; wi += kWriteThreads) {
+      const int t = wi / wpt;
+      const int word = wi - t * wpt;
+      uint32_t bits = 0;
+      if (t < nvalid) {
+        for (int k = 0; k < cpw; ++k) {
+          const int ch = word * cpw + k;
+          const float s = s_scale[ch];
+          uint32_t code = 0;
+          if (s != 0.0f) {
+            const float z = __fadd_rn(__fdiv_rn(__fsub_rn(kp[t][ch], s_min[ch]), s), kc0);
+            code = count_above(z, thr_k, LK - 1);
+          }
+          bits |= code << (p.key_bits * k);
+        }
+      }
+      kw[wi] = bits;
+    }
+  }
+  group_sync(bar_id);  // kp is reused for values below
+
+  // windows filled completely by this write get their values from vrot_tc
+  const bool tc_window = p.tc_values && p0 >= L0 && nvalid == kWindow;
+  if (tc_window) {
+    if (h == 0 && tid < kWindow) {
+      const int m = mnew[p0 + tid - L0];
+      if (m >= kMods) set_error(p.error_word, OMNIKV_DEVERR_MODALITY);
+      p.modality[(size_t)b * p.cap_tokens + p0 + tid] = (uint8_t)(m >= kMods ? kMods - 1 : m);
+    }
+    return;
+  }
+
+  // ---- values: per-token scale (pairwise tree in a warp) ----------------------
+  for (int i = inew0 + warp; i < nvalid; i += kWriteThreads / 32) {
+    const __half* src = vnew + (size_t)(p0 + i - L0) * kHeadDim;
+    float x[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      x[j] = __half2float(src[lane + 32 * j]);
+      kp[i][lane + 32 * j] = x[j];
+    }
+    // tree: h = 64 pairs j with j + 2, h = 32 pairs the two results, then lanes
+    const float a = __fadd_rn(__fmul_rn(x[0], x[0]), __fmul_rn(x[2], x[2]));
+    const float c = __fadd_rn(__fmul_rn(x[1], x[1]), __fmul_rn(x[3], x[3]));
+    float z = __fadd_rn(a, c);
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) z = __fadd_rn(z, __shfl_xor_sync(0xffffffffu, z, o));
+    if (lane == 0) s_sigma[i] = __half2float(__float2half_rn(__fsqrt_rn(__fmul_rn(z, 0.0078125f))));
+  }
+  group_sync(bar_id);
+
+  // ---- values: rotation, codes, channel-major packing --------------------------
+  {
+    const int j = tid;  // output channel
+    const int cpw = 32 / p.value_bits;
+    const int ngroups = kWindow / cpw;
+    const uint32_t mask = (1u << p.value_bits) - 1u;
+    uint32_t* vw = reinterpret_cast<uint32_t*>(rec + lay.v_off);
+    uint32_t words[4];
+#pragma unroll
+    for (int g = 0; g < 4; ++g) words[g] = g < ngroups ? vw[g * kHeadDim + j] : 0u;
+    for (int i = inew0; i < nvalid; ++i) {
+      int m = mnew[p0 + i - L0];
+      if (m >= kMods) m = kMods - 1;  // out-of-range ids are flagged below and read as video
+      const float* U = p.value_rot + ((size_t)(h * kMods + m) * kHeadDim) * kHeadDim + j;
+      // column j of U_m against the value: independent loads, 8 partial sums
+      float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 32
+      for (int c = 0; c < kHeadDim; ++c) part[c & 7] = fmaf(U[(size_t)c * kHeadDim], kp[i][c], part[c & 7]);
+      const float acc = ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
+      const float s = s_sigma[i];
+      uint32_t code = 0;
+      if (s != 0.0f) code = count_above(__fdiv_rn(acc, s), thr_v, LV - 1);
+      const int g = i / cpw;
+      const int sh = p.value_bits * (i - g * cpw);
+#pragma unroll
+      for (int gg = 0; gg < 4; ++gg)
+        if (gg == g) words[gg] = (words[gg] & ~(mask << sh)) | (code << sh);
+    }
+#pragma unroll
+    for (int g = 0; g < 4; ++g)
+      if (g < ngroups) vw[g * kHeadDim + j] = words[g];
+  }
+  if (tid >= inew0 && tid < nvalid) {
+    reinterpret_cast<__half*>(rec + lay.sigma_off)[tid] = __float2half_rn(s_sigma[tid]);
+    if (h == 0) {
+      const int m = mnew[p0 + tid - L0];
+      if (m >= kMods) set_error(p.error_word, OMNIKV_DEVERR_MODALITY);
+      p.modality[(size_t)b * p.cap_tokens + p0 + tid] = (uint8_t)(m >= kMods ? kMods - 1 : m);
+    }
+  }
+}
+
+
+}  // namespace
+}  // namespace omnikv

@@ -2,26 +2,34 @@
 // applies the inverse value rotations (paperpeel.com section 1: inverse value
 // rotations are applied to head outputs instead of to every cached value).
 //
-// One CTA per (query head, kv head, sequence):
+// One CTA per (query head, block of 32 output rows, kv head, sequence):
+//   0. before waiting on the decode launch: this warp's 4 rows of U_m for the 3
+//      modalities go into registers (they do not depend on the decode);
 //   1. warp 0: M = max_s m_s, weights e_s = exp(m_s - M), l = sum_s l_s e_s;
-//   2. all threads: a_m[c] = sum_s acc_{s,m}[c] e_s / l, the splits read as
-//      16-byte vectors, two threads per vector column;
-//   3. out[j] = sum_m sum_c U_m[j][c] a_m[c]: one warp per output row, lanes over
-//      c (coalesced rows of U_m), warp reduction.
+//   2. a_m[c] = sum_s acc_{s,m}[c] e_s / l, the splits read as 16-byte vectors,
+//      two threads per vector column, splits of weight 0 skipped;
+//   3. out[j] = sum_m sum_c U_m[j][c] a_m[c] for the block's rows: one warp per 4
+//      rows, lanes over c, warp reduction.
+// The 4 row blocks of a head merge the same partials (read from L2); splitting
+// the rows keeps every step one memory round trip deep.
 // A sequence without tokens (all m_s = -inf) yields zeros.
 #include "common.cuh"
 #include "kernels.h"
+#include "ptx.cuh"
 
 namespace omnikv {
 
 namespace {
 
 constexpr int kCombineThreads = 256;
+constexpr int kRowBlocks = 4;                        // blocks of 32 output rows
+constexpr int kRowsPerWarp = kHeadDim / kRowBlocks / (kCombineThreads / 32);  // 4
 constexpr int kMaxSplitsSmem = 4096;
 
 __global__ void __launch_bounds__(kCombineThreads)
 combine_inverse_rotate_kernel(const CombineParams p) {
-  const int g = blockIdx.x;        // query head within the group
+  const int g = blockIdx.x / kRowBlocks;  // query head within the group
+  const int rb = blockIdx.x % kRowBlocks;
   const int kvh = blockIdx.y;
   const int b = blockIdx.z;
   const int G = p.group;
@@ -29,24 +37,46 @@ combine_inverse_rotate_kernel(const CombineParams p) {
   const int S = p.num_splits;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qh = kvh * G + g;
-  const Partial* part = p.partials + ((size_t)b * Hq + qh) * S;
 
   __shared__ float w[kMaxSplitsSmem];
   __shared__ __align__(16) float4 red[2][96];
   __shared__ __align__(16) float a[kMods * kHeadDim];
   __shared__ float s_l;
 
+  griddep_launch_dependents();
+  // ---- 0. value-basis rows (constant input): rows j0 .. j0 + 3, lanes over c
+  const int j0 = rb * (kHeadDim / kRowBlocks) + warp * kRowsPerWarp;
+  const float* Ubase = p.value_rot + (size_t)kvh * kMods * kHeadDim * kHeadDim;
+  float4 u[kRowsPerWarp][kMods];
+#pragma unroll
+  for (int r = 0; r < kRowsPerWarp; ++r)
+#pragma unroll
+    for (int m = 0; m < kMods; ++m)
+      u[r][m] = reinterpret_cast<const float4*>(Ubase + ((size_t)m * kHeadDim + j0 + r) * kHeadDim)[lane];
+
+  griddep_wait();  // the partials come from the decode launch just before
+  const Partial* part = p.partials + ((size_t)b * Hq + qh) * S;
+  if (p.len_add > 0 && blockIdx.x == 0 && kvh == 0 && tid == 0) {  // decode step: advance the length
+    const int L = p.seq_lens[b];
+    if (L >= 0 && L + p.len_add <= p.cap_tokens) p.seq_lens[b] = L + p.len_add;
+  }
+
+  // ---- 1. split weights
   if (warp == 0) {
     float M = -INFINITY;
-    for (int s = lane; s < S; s += 32) M = fmaxf(M, part[s].m);
+    for (int s = lane; s < S; s += 32) {
+      const float ms = part[s].m;
+      w[s] = ms;
+      M = fmaxf(M, ms);
+    }
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float l = 0.0f;
     for (int s = lane; s < S; s += 32) {
-      const float ms = part[s].m;
+      const float ms = w[s];
       const float e = (ms == -INFINITY) ? 0.0f : expf(ms - M);
       w[s] = e;
-      l += part[s].l * e;
+      if (e != 0.0f) l += part[s].l * e;
     }
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
@@ -54,7 +84,7 @@ combine_inverse_rotate_kernel(const CombineParams p) {
   }
   __syncthreads();
 
-  // weighted sum over splits: column c4 (of 96 float4), half h of the splits
+  // ---- 2. weighted sum over splits: column c4 (of 96 float4), half h of the splits
   {
     const int c4 = tid & 127, h = tid >> 7;
     if (c4 < 96) {
@@ -81,34 +111,24 @@ combine_inverse_rotate_kernel(const CombineParams p) {
   }
   __syncthreads();
 
-  // out[j] = sum_m U_m[j][:] . a_m
-  const float* Ubase = p.value_rot + (size_t)kvh * kMods * kHeadDim * kHeadDim;
+  // ---- 3. out[j] = sum_m U_m[j][:] . a_m for this warp's rows
   float* out = p.out + ((size_t)b * Hq + qh) * kHeadDim;
   float4 xa[kMods];
 #pragma unroll
   for (int m = 0; m < kMods; ++m) xa[m] = reinterpret_cast<const float4*>(a + m * kHeadDim)[lane];
-  constexpr int kRows = 4;  // rows per batch: their U loads are issued together
-  for (int j0 = warp * kRows; j0 < kHeadDim; j0 += kRows * (kCombineThreads / 32)) {
-    float4 u[kRows][kMods];
 #pragma unroll
-    for (int r = 0; r < kRows; ++r)
+  for (int r = 0; r < kRowsPerWarp; ++r) {
+    float v = 0.0f;
 #pragma unroll
-      for (int m = 0; m < kMods; ++m)
-        u[r][m] = reinterpret_cast<const float4*>(Ubase + ((size_t)m * kHeadDim + j0 + r) * kHeadDim)[lane];
-#pragma unroll
-    for (int r = 0; r < kRows; ++r) {
-      float v = 0.0f;
-#pragma unroll
-      for (int m = 0; m < kMods; ++m) {
-        v = fmaf(u[r][m].x, xa[m].x, v);
-        v = fmaf(u[r][m].y, xa[m].y, v);
-        v = fmaf(u[r][m].z, xa[m].z, v);
-        v = fmaf(u[r][m].w, xa[m].w, v);
-      }
-#pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0) out[j0 + r] = v;
+    for (int m = 0; m < kMods; ++m) {
+      v = fmaf(u[r][m].x, xa[m].x, v);
+      v = fmaf(u[r][m].y, xa[m].y, v);
+      v = fmaf(u[r][m].z, xa[m].z, v);
+      v = fmaf(u[r][m].w, xa[m].w, v);
     }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) out[j0 + r] = v;
   }
 }
 
@@ -116,9 +136,8 @@ combine_inverse_rotate_kernel(const CombineParams p) {
 
 cudaError_t launch_combine(const CombineParams& p, int batch, cudaStream_t stream) {
   if (p.num_splits > kMaxSplitsSmem) return cudaErrorInvalidValue;
-  dim3 grid(p.group, p.num_kv_heads, batch);
-  combine_inverse_rotate_kernel<<<grid, kCombineThreads, 0, stream>>>(p);
-  return cudaGetLastError();
+  dim3 grid(p.group * kRowBlocks, p.num_kv_heads, batch);
+  return launch_pdl(combine_inverse_rotate_kernel, grid, dim3(kCombineThreads), 0, stream, p);
 }
 
 }  // namespace omnikv

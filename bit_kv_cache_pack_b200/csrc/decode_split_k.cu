@@ -8,8 +8,8 @@
 // of a window record.
 //
 // Tensor-core path (2-bit keys and values, symmetric codebook):
-//   * each warp streams its own windows (w0 + warp, w0 + warp + 4, ...) through
-//     a 4-stage shared-memory ring filled by 1-D bulk async copies (record +
+//   * each warp streams its own contiguous run of the split's windows through
+//     a 3-stage shared-memory ring filled by 1-D bulk async copies (record +
 //     the window's 32 modality ids) completing on per-stage mbarriers;
 //   * scores use mma.sync m16n8k16 with the 8 query heads as N. With a
 //     symmetric codebook c_j - c_0 = (c_1 - c_0) b0 + (c_2 - c_0) b1 for the
@@ -28,10 +28,14 @@
 //     through movmatrix; values are stored
 //     channel-major so the A operand (16 channels x 16 tokens) again needs one
 //     shift and one AND per register; one fp32 accumulator set per modality
-//     (values of different modalities live in different rotated bases); the
-//     c_0 term is c_0 * sum_t p_t sigma_t per modality, added at the end;
-//   * the 4 warps merge (max, rescale, shared-memory reduction) and write one
-//     split-K partial per query head.
+//     (values of different modalities live in different rotated bases): the
+//     active modality's set is in registers, the others are parked in the
+//     warp's tensor-memory lanes (tcgen05.st / tcgen05.ld, 32 columns each)
+//     together with the running max they were parked at, and are rescaled to
+//     the current max when a tile of that modality brings them back; the c_0
+//     term is c_0 * sum_t p_t sigma_t per modality, added at the end;
+//   * the 4 warps merge (common max, rescale, shared-memory reduction), one
+//     modality at a time, and write one split-K partial per query head.
 // Token order inside a 16-token tile: fragment row / k-slot r holds token
 // tau(r) = r/2 + 8 (r%2) for r < 8 and 4 + (r-8)/2 + 8 (r%2) for r >= 8, so the
 // two tokens of every value-operand register (k-slots 2t, 2t+1 -> tokens t,
@@ -43,6 +47,9 @@
 // Inputs must stay in the fp16 range of the operands: |q' s_gc| / sqrt(128)
 // below ~480 and value scales sigma below ~480; outside it the output is not
 // finite (the data would have to be far outside any realistic key / value range).
+#include <atomic>
+
+#include "append.cuh"
 #include "common.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
@@ -58,6 +65,8 @@ constexpr int kRec22 = 2624;                    // K2/V2 record bytes
 constexpr int kStageBytes = kRec22 + kWindow;   // record + modality ids
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: a bulk copy that takes longer is an error
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kCtasPerSm = 2;      // resident CTAs per SM the register budget is set for
+constexpr uint32_t kTmemCols = 128;  // per CTA: 3 parked accumulators x 32 columns in each warp's lanes
 
 struct __align__(16) DecodeSmem {
   uint8_t stage[kWarps][kStages][kStageBytes];  // also reused by the generic path and the final merge
@@ -65,6 +74,8 @@ struct __align__(16) DecodeSmem {
   uint64_t bar[kWarps][kStages];
   float q[kMaxGroup][kHeadDim];                 // rotated queries, times the softmax scale
   float mw[kWarps][kMaxGroup];                  // per-warp running max, for the merge
+  float lw[kWarps][kMaxGroup];                  // per-warp softmax denominators, for the merge
+  uint32_t tmem_base;                           // TMEM columns of the parked accumulators
 };
 static_assert(sizeof(DecodeSmem) <= 48 * 1024, "static shared memory");
 
@@ -120,12 +131,44 @@ __device__ __forceinline__ void rotate_queries(const DecodeParams& p, int b, int
 // p.split_windows chosen on the host from the length bound, so a short sequence
 // leaves its last splits empty and every non-empty split has the same size.
 __device__ __forceinline__ void split_range(const DecodeParams& p, int b, int split, int& T, int& w0, int& w1) {
-  T = max(0, min(p.seq_lens[b], p.cap_tokens));
+  const int L = p.seq_lens[b];
+  const int La = L + p.len_add;  // a decode step's append happens only within the capacity
+  T = max(0, min(La <= p.cap_tokens ? La : L, p.cap_tokens));
   const int nw = (T + kWindow - 1) / kWindow;
   w0 = min(split * p.split_windows, nw);
   w1 = min(w0 + p.split_windows, nw);
   if (split == p.num_splits - 1 && threadIdx.x == 0 && nw > p.num_splits * p.split_windows)
     set_error(p.error_word, OMNIKV_DEVERR_BOUND);
+}
+
+// Decode step: the window that receives the appended token, and the flag value
+// that marks its record as written (window -1: nothing to wait for).
+__device__ __forceinline__ void step_window(const DecodeParams& p, int b, int& win, int& val) {
+  win = -1;
+  val = 0;
+  if (p.len_add > 0 && p.step_flags != nullptr) {
+    const int L = p.seq_lens[b];
+    if (L >= 0 && L + p.len_add <= p.cap_tokens) {
+      val = L + p.len_add;
+      win = (val - 1) / kWindow;
+    }
+  }
+}
+
+// Bounded acquire-spin until *flag == val (written with release by the append
+// CTA of the same launch); false after about `limit_ns`.
+__device__ __forceinline__ bool wait_flag(const int32_t* flag, int val, uint64_t limit_ns) {
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 0;; ++it) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+    if (v == val) break;
+    if ((it & 63u) == 63u && global_timer_ns() - t0 > limit_ns) return false;
+    __nanosleep(64);
+  }
+  // the record is then read through the async proxy (bulk copy)
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  return true;
 }
 
 // ---------------------------------------------------------------------------
@@ -160,7 +203,12 @@ __device__ void decode_generic(const DecodeParams& p, DecodeSmem& sm, int b, int
       for (int j = 0; j < 4; ++j) acc[k][m][j] = 0.0f;
 
   const uint8_t* rec_base = p.records + ((size_t)(b * p.num_kv_heads + kvh) * p.cap_windows) * lay.bytes;
+  int wait_win, wait_val;
+  step_window(p, b, wait_win, wait_val);
   for (int w = w0; w < w1; ++w) {
+    if (w == wait_win && threadIdx.x == 0 &&
+        !wait_flag(p.step_flags + (size_t)b * p.num_kv_heads + kvh, wait_val, kWaitLimitNs))
+      set_error(p.error_word, OMNIKV_DEVERR_TIMEOUT);
     __syncthreads();
     {
       const uint4* src = reinterpret_cast<const uint4*>(rec_base + (size_t)w * lay.bytes);
@@ -267,15 +315,84 @@ __device__ __forceinline__ void split_pair_t(float x0, float x1, uint32_t& hi, u
   lo = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&l));
 }
 
+// Per-warp decode state. Only the accumulator of the active modality lives in
+// registers; the others are parked in this warp's TMEM lanes (columns 32 m ..
+// 32 m + 31 for modality m), each with the running max it was parked at, and are
+// rescaled to the current max when they are brought back.
 struct WarpState {
-  float m[2];           // running max for heads 2t, 2t+1 (warp-uniform per column)
-  float l[2];           // per-lane partial sum of p for heads 2t, 2t+1
-  float S[kMods][2];    // per-lane partial sum of p * sigma per modality
-  float acc[kMods][8][4];
+  float m[2];              // running max for heads 2t, 2t+1 (warp-uniform per column)
+  float l[2];              // per-lane partial sum of p for heads 2t, 2t+1
+  float S[kMods][2];       // per-lane partial sum of p * sigma per modality (kept at the running max)
+  float mref[kMods][2];    // running max at which a parked accumulator was stored
+  float acc[8][4];         // accumulator of the active modality
+  int cur;                 // active modality, -1 if none (warp-uniform)
+  uint32_t parked;         // bit m set: modality m's accumulator is parked in TMEM (warp-uniform)
 };
 
+__device__ __forceinline__ uint32_t slot_addr(uint32_t tbase, int warp, int m) {
+  return tbase + ((uint32_t)(32 * warp) << 16) + 32u * (uint32_t)m;
+}
+
+__device__ __forceinline__ void park_active(WarpState& st, uint32_t tbase, int warp) {
+  tmem_st32(slot_addr(tbase, warp, st.cur), reinterpret_cast<const uint32_t*>(&st.acc[0][0]));
+#pragma unroll
+  for (int mm = 0; mm < kMods; ++mm)
+    if (mm == st.cur) {
+      st.mref[mm][0] = st.m[0];
+      st.mref[mm][1] = st.m[1];
+    }
+  st.parked |= 1u << st.cur;
+}
+
+// Load modality m's parked accumulator into acc, scaled by 2^((mref - target) log2 e)
+// per column, or zeros if it was never parked. Warp-collective.
+__device__ __forceinline__ void unpark(WarpState& st, int m, uint32_t tbase, int warp, float tgt0, float tgt1) {
+  if (st.parked & (1u << m)) {
+    tmem_ld32(slot_addr(tbase, warp, m), reinterpret_cast<uint32_t*>(&st.acc[0][0]));
+    float r0 = 0.f, r1 = 0.f;
+#pragma unroll
+    for (int mm = 0; mm < kMods; ++mm)
+      if (mm == m) {
+        r0 = st.mref[mm][0];
+        r1 = st.mref[mm][1];
+      }
+    const float f0 = fast_exp2((r0 - tgt0) * kLog2e), f1 = fast_exp2((r1 - tgt1) * kLog2e);
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      st.acc[mt][0] *= f0;
+      st.acc[mt][1] *= f1;
+      st.acc[mt][2] *= f0;
+      st.acc[mt][3] *= f1;
+    }
+  } else {
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) st.acc[mt][r] = 0.0f;
+  }
+}
+
+// Make modality m the active one (warp-uniform m).
+__device__ __forceinline__ void activate(WarpState& st, int m, uint32_t tbase, int warp) {
+  if (m == st.cur) return;
+  if (st.cur >= 0) park_active(st, tbase, warp);
+  unpark(st, m, tbase, warp, st.m[0], st.m[1]);
+  st.cur = m;
+}
+
+// Warp `warp` of the CTA decodes the contiguous windows [*a, *e) of [w0, w1).
+__device__ __forceinline__ void warp_windows(int w0, int w1, int warp, int& a, int& e) {
+  const int per = (w1 - w0 + kWarps - 1) / kWarps;
+  a = min(w0 + warp * per, w1);
+  e = min(a + per, w1);
+}
+
 __device__ __forceinline__ void issue_window(const DecodeParams& p, DecodeSmem& sm, int warp, int stage,
-                                             const uint8_t* rec_base, int b, int wi) {
+                                             const uint8_t* rec_base, int b, int kvh, int wi, int wait_win,
+                                             int wait_val) {
+  if (wi == wait_win &&
+      !wait_flag(p.step_flags + (size_t)b * p.num_kv_heads + kvh, wait_val, kWaitLimitNs))
+    set_error(p.error_word, OMNIKV_DEVERR_TIMEOUT);
   uint64_t* bar = &sm.bar[warp][stage];
   uint8_t* dst = &sm.stage[warp][stage][0];
   mbar_arrive_expect_tx(bar, kStageBytes);
@@ -287,18 +404,21 @@ __device__ __forceinline__ void issue_window(const DecodeParams& p, DecodeSmem& 
 __device__ __forceinline__ void prime_pipeline(const DecodeParams& p, DecodeSmem& sm, int b, int kvh, int w0, int w1) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint8_t* rec_base = p.records + ((size_t)(b * p.num_kv_heads + kvh) * p.cap_windows) * kRec22;
-  const int nmine = (w1 - w0 > warp) ? (w1 - w0 - warp + kWarps - 1) / kWarps : 0;
+  int wa, we, wait_win, wait_val;
+  warp_windows(w0, w1, warp, wa, we);
+  step_window(p, b, wait_win, wait_val);
   if (lane == 0) {
 #pragma unroll
     for (int s = 0; s < kStages; ++s) mbar_init(&sm.bar[warp][s], 1);
     fence_barrier_init();
-    for (int i = 0; i < kStages && i < nmine; ++i) issue_window(p, sm, warp, i, rec_base, b, w0 + warp + kWarps * i);
+    for (int i = 0; i < kStages && wa + i < we; ++i)
+      issue_window(p, sm, warp, i, rec_base, b, kvh, wa + i, wait_win, wait_val);
   }
   __syncwarp();
 }
 
 __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh, int split, float kV0, float kV1,
-                           float vc0) {
+                           float vc0, uint32_t tbase) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int G = p.group;
@@ -306,7 +426,10 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
   int T, w0, w1;
   split_range(p, b, split, T, w0, w1);
   const uint8_t* rec_base = p.records + ((size_t)(b * p.num_kv_heads + kvh) * p.cap_windows) * kRec22;
-  const int nmine = (w1 - w0 > warp) ? (w1 - w0 - warp + kWarps - 1) / kWarps : 0;
+  int wa, we, wait_win, wait_val;
+  warp_windows(w0, w1, warp, wa, we);
+  step_window(p, b, wait_win, wait_val);
+  const int nmine = we - wa;
 
   WarpState st;
 #pragma unroll
@@ -314,19 +437,22 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
     st.m[j] = -INFINITY;
     st.l[j] = 0.0f;
 #pragma unroll
-    for (int m = 0; m < kMods; ++m) st.S[m][j] = 0.0f;
+    for (int m = 0; m < kMods; ++m) {
+      st.S[m][j] = 0.0f;
+      st.mref[m][j] = -INFINITY;
+    }
   }
 #pragma unroll
-  for (int m = 0; m < kMods; ++m)
+  for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
-    for (int mt = 0; mt < 8; ++mt)
-#pragma unroll
-      for (int r = 0; r < 4; ++r) st.acc[m][mt][r] = 0.0f;
+    for (int r = 0; r < 4; ++r) st.acc[mt][r] = 0.0f;
+  st.cur = -1;
+  st.parked = 0;
 
   int failed_at = -1;
   for (int i = 0; i < nmine; ++i) {
     const int s = i % kStages;
-    const int wi = w0 + warp + kWarps * i;
+    const int wi = wa + i;
     if (!mbar_wait_bounded(&sm.bar[warp][s], (i / kStages) & 1, kWaitLimitNs)) {
       failed_at = i;
       break;
@@ -428,7 +554,8 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
       }
     }
 
-    // ---- online softmax over the window
+    // ---- online softmax over the window (parked accumulators keep their own
+    // reference max and are rescaled when brought back)
     float mx0 = fmaxf(fmaxf(sc[0][0], sc[0][2]), fmaxf(sc[1][0], sc[1][2]));
     float mx1 = fmaxf(fmaxf(sc[0][1], sc[0][3]), fmaxf(sc[1][1], sc[1][3]));
 #pragma unroll
@@ -445,13 +572,13 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
       for (int m = 0; m < kMods; ++m) {
         st.S[m][0] *= a0;
         st.S[m][1] *= a1;
+      }
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt) {
-          st.acc[m][mt][0] *= a0;
-          st.acc[m][mt][1] *= a1;
-          st.acc[m][mt][2] *= a0;
-          st.acc[m][mt][3] *= a1;
-        }
+      for (int mt = 0; mt < 8; ++mt) {
+        st.acc[mt][0] *= a0;
+        st.acc[mt][1] *= a1;
+        st.acc[mt][2] *= a0;
+        st.acc[mt][3] *= a1;
       }
       st.m[0] = mn0;
       st.m[1] = mn1;
@@ -476,75 +603,61 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
       split_pair_t(w0v * kV1, w1v * kV1, bv1[0], bv1[2]);
       split_pair_t(w2v * kV1, w3v * kV1, bv1[1], bv1[3]);
       // modalities of this tile (warp-uniform mask) and of this lane's tokens
-      const int mA = mods[tokA[h]], mB = mods[tokB[h]];
-      const uint32_t mbits = __reduce_or_sync(0xffffffffu, (1u << min(mA, 2)) | (1u << min(mB, 2)));
-      // V words of channels 16g .. 16g+15 for this tile's 16 tokens
-      uint32_t vwd[16];
-      {
-        const uint4* src = reinterpret_cast<const uint4*>(vw + h * kHeadDim + 16 * g);
+      const int mA = min((int)mods[tokA[h]], 2), mB = min((int)mods[tokB[h]], 2);
+      const uint32_t mbits = __reduce_or_sync(0xffffffffu, (1u << mA) | (1u << mB));
+      // k-slots of this lane's B registers: 2t, 2t+1 -> tokens t, t+8; 2t+8, 2t+9 -> t+4, t+12
+      const int base = 16 * h;
+      const int mk0 = min((int)mods[base + t], 2), mk1 = min((int)mods[base + t + 8], 2);
+      const int mk2 = min((int)mods[base + t + 4], 2), mk3 = min((int)mods[base + t + 12], 2);
+      const int rlo = 13 - 2 * t, rhi = (5 - 2 * t) & 31;
+      const uint4* vsrc = reinterpret_cast<const uint4*>(vw + h * kHeadDim + 16 * g);
+      // one (masked) product per modality present, the active one first
+      uint32_t todo = mbits;
+      int mm = (st.cur >= 0 && ((todo >> st.cur) & 1u)) ? st.cur : __ffs(todo) - 1;
+#pragma unroll 1
+      while (true) {
+        activate(st, mm, tbase, warp);
+        const bool single = mbits == (1u << mm);
+        const uint32_t msk01 = single ? 0xFFFFFFFFu : ((mk0 == mm ? 0x0000FFFFu : 0u) | (mk1 == mm ? 0xFFFF0000u : 0u));
+        const uint32_t msk23 = single ? 0xFFFFFFFFu : ((mk2 == mm ? 0x0000FFFFu : 0u) | (mk3 == mm ? 0xFFFF0000u : 0u));
+        const uint32_t b00 = bv0[0] & msk01, b01 = bv0[1] & msk23;
+        const uint32_t b10 = bv1[0] & msk01, b11 = bv1[1] & msk23;
+        const uint32_t c00 = bv0[2] & msk01, c01 = bv0[3] & msk23;
+        const uint32_t c10 = bv1[2] & msk01, c11 = bv1[3] & msk23;
+        const float u0 = (mA == mm ? w0v : 0.0f) + (mB == mm ? w2v : 0.0f);
+        const float u1 = (mA == mm ? w1v : 0.0f) + (mB == mm ? w3v : 0.0f);
+#pragma unroll
+        for (int k = 0; k < kMods; ++k)
+          if (k == mm) {
+            st.S[k][0] += u0;
+            st.S[k][1] += u1;
+          }
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
-          const uint4 u = src[q4];
-          vwd[4 * q4 + 0] = u.x;
-          vwd[4 * q4 + 1] = u.y;
-          vwd[4 * q4 + 2] = u.z;
-          vwd[4 * q4 + 3] = u.w;
-        }
-      }
-      const int rlo = 13 - 2 * t, rhi = (5 - 2 * t) & 31;
-      if ((mbits & (mbits - 1)) == 0) {  // one modality in the tile
-        const int m = __ffs(mbits) - 1;
+          const uint4 u = vsrc[q4];  // V words of channels 16g + 4 q4 .. + 3
+          const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-        for (int mm = 0; mm < kMods; ++mm) {
-          if (mm != m) continue;
-          st.S[mm][0] += w0v + w2v;
-          st.S[mm][1] += w1v + w3v;
-#pragma unroll
-          for (int mt = 0; mt < 8; ++mt) {
-            const uint32_t wg = vwd[2 * mt], wg8 = vwd[2 * mt + 1];
+          for (int e = 0; e < 2; ++e) {
+            const int mt = 2 * q4 + e;
+            const uint32_t wg = wv[2 * e], wg8 = wv[2 * e + 1];
             const uint32_t r[4] = {rotl(wg, rlo), rotl(wg8, rlo), rotl(wg, rhi), rotl(wg8, rhi)};
             const uint32_t a0[4] = {r[0] & kPlane0, r[1] & kPlane0, r[2] & kPlane0, r[3] & kPlane0};
             const uint32_t a1[4] = {r[0] & kPlane1, r[1] & kPlane1, r[2] & kPlane1, r[3] & kPlane1};
-            mma_f16_16816(st.acc[mm][mt], a0, bv0[0], bv0[1]);
-            mma_f16_16816(st.acc[mm][mt], a1, bv1[0], bv1[1]);
-            mma_f16_16816(st.acc[mm][mt], a0, bv0[2], bv0[3]);
-            mma_f16_16816(st.acc[mm][mt], a1, bv1[2], bv1[3]);
+            mma_f16_16816(st.acc[mt], a0, b00, b01);
+            mma_f16_16816(st.acc[mt], a1, b10, b11);
+            mma_f16_16816(st.acc[mt], a0, c00, c01);
+            mma_f16_16816(st.acc[mt], a1, c10, c11);
           }
         }
-      } else {  // mixed tile: one masked product per modality present
-        // k-slots of this lane's B registers: 2t, 2t+1 -> tokens t, t+8; 2t+8, 2t+9 -> t+4, t+12
-        const int base = 16 * h;
-        const int mk0 = min((int)mods[base + t], 2), mk1 = min((int)mods[base + t + 8], 2);
-        const int mk2 = min((int)mods[base + t + 4], 2), mk3 = min((int)mods[base + t + 12], 2);
-#pragma unroll
-        for (int mm = 0; mm < kMods; ++mm) {
-          if (!(mbits & (1u << mm))) continue;
-          const uint32_t msk01 = (mk0 == mm ? 0x0000FFFFu : 0u) | (mk1 == mm ? 0xFFFF0000u : 0u);
-          const uint32_t msk23 = (mk2 == mm ? 0x0000FFFFu : 0u) | (mk3 == mm ? 0xFFFF0000u : 0u);
-          const uint32_t b00 = bv0[0] & msk01, b01 = bv0[1] & msk23;
-          const uint32_t b10 = bv1[0] & msk01, b11 = bv1[1] & msk23;
-          const uint32_t c00 = bv0[2] & msk01, c01 = bv0[3] & msk23;
-          const uint32_t c10 = bv1[2] & msk01, c11 = bv1[3] & msk23;
-          st.S[mm][0] += (min(mA, 2) == mm ? w0v : 0.0f) + (min(mB, 2) == mm ? w2v : 0.0f);
-          st.S[mm][1] += (min(mA, 2) == mm ? w1v : 0.0f) + (min(mB, 2) == mm ? w3v : 0.0f);
-#pragma unroll
-          for (int mt = 0; mt < 8; ++mt) {
-            const uint32_t wg = vwd[2 * mt], wg8 = vwd[2 * mt + 1];
-            const uint32_t r[4] = {rotl(wg, rlo), rotl(wg8, rlo), rotl(wg, rhi), rotl(wg8, rhi)};
-            const uint32_t a0[4] = {r[0] & kPlane0, r[1] & kPlane0, r[2] & kPlane0, r[3] & kPlane0};
-            const uint32_t a1[4] = {r[0] & kPlane1, r[1] & kPlane1, r[2] & kPlane1, r[3] & kPlane1};
-            mma_f16_16816(st.acc[mm][mt], a0, b00, b01);
-            mma_f16_16816(st.acc[mm][mt], a1, b10, b11);
-            mma_f16_16816(st.acc[mm][mt], a0, c00, c01);
-            mma_f16_16816(st.acc[mm][mt], a1, c10, c11);
-          }
-        }
+        todo &= ~(1u << mm);
+        if (!todo) break;
+        mm = __ffs(todo) - 1;
       }
     }
     __syncwarp();
     if (lane == 0 && i + kStages < nmine) {
       fence_proxy_async_smem();
-      issue_window(p, sm, warp, s, rec_base, b, w0 + warp + kWarps * (i + kStages));
+      issue_window(p, sm, warp, s, rec_base, b, kvh, wa + i + kStages, wait_win, wait_val);
     }
   }
 
@@ -559,8 +672,13 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
     for (int j = 0; j < 2; ++j) {
       st.m[j] = -INFINITY;
       st.l[j] = 0.0f;
+#pragma unroll
+      for (int m = 0; m < kMods; ++m) st.S[m][j] = 0.0f;
     }
+    st.cur = -1;
+    st.parked = 0;
   }
+  if (st.cur >= 0) park_active(st, tbase, warp);
 
   // ---- reduce the per-lane partial sums over the 8 lanes sharing a column
 #pragma unroll
@@ -572,20 +690,8 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
       for (int m = 0; m < kMods; ++m) st.S[m][j] += __shfl_xor_sync(0xffffffffu, st.S[m][j], o);
     }
   }
-  // c_0 term of the value codebook
-#pragma unroll
-  for (int m = 0; m < kMods; ++m)
-#pragma unroll
-    for (int mt = 0; mt < 8; ++mt) {
-      st.acc[m][mt][0] += vc0 * st.S[m][0];
-      st.acc[m][mt][1] += vc0 * st.S[m][1];
-      st.acc[m][mt][2] += vc0 * st.S[m][0];
-      st.acc[m][mt][3] += vc0 * st.S[m][1];
-    }
 
-  // ---- merge the 4 warps: common max, rescale, exchange in register order ---
-  // (every warp holds the same (channel, head) in the same register of the same
-  // lane, so a lane-major buffer is bank-conflict free)
+  // ---- merge the 4 warps at their common max, one modality at a time ------
   if (g == 0) {
     sm.mw[warp][2 * t] = st.m[0];
     sm.mw[warp][2 * t + 1] = st.m[1];
@@ -601,63 +707,56 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
     const float f = (st.m[j] == -INFINITY) ? 0.0f : fast_exp2((st.m[j] - mm) * kLog2e);
     st.l[j] *= f;
 #pragma unroll
-    for (int m = 0; m < kMods; ++m)
+    for (int m = 0; m < kMods; ++m) st.S[m][j] *= f;
+  }
+  if (g == 0) {
+    sm.lw[warp][2 * t] = st.l[0];
+    sm.lw[warp][2 * t + 1] = st.l[1];
+  }
+  float* xbuf = reinterpret_cast<float*>(&sm.stage[0][0][0]);  // [warp][32 registers][32 lanes]
+  static_assert(kWarps * 32 * 32 * 4 <= kWarps * kStages * kStageBytes, "merge buffer");
 #pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        st.acc[m][mt][j] *= f;
-        st.acc[m][mt][j + 2] *= f;
+  for (int m = 0; m < kMods; ++m) {
+    unpark(st, m, tbase, warp, M[0], M[1]);  // zeros if this warp never saw modality m
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+        xbuf[(warp * 32 + mt * 4 + r) * 32 + lane] = st.acc[mt][r] + vc0 * st.S[m][r & 1];
+    __syncthreads();
+    // warp w sums registers of m-tiles 2w, 2w+1 over the 4 warps and writes them
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int mt = 2 * warp + e;
+      float v[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        float x = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) x += xbuf[(w * 32 + mt * 4 + r) * 32 + lane];
+        v[r] = x;
       }
-  }
-  constexpr int kVals = kMods * 8 * 4 + 2;
-  float* xbuf = reinterpret_cast<float*>(&sm.stage[0][0][0]);  // [2][kVals][32]
-  static_assert(2 * kVals * 32 * 4 <= kWarps * kStages * kStageBytes, "merge buffer");
 #pragma unroll
-  for (int round = 0; round < 2; ++round) {
-    const int writers_lo = round == 0 ? 2 : 1;  // round 0: warps 2,3 -> 0,1; round 1: warp 1 -> 0
-    const bool writer = round == 0 ? (warp >= 2) : (warp == 1);
-    const bool reader = round == 0 ? (warp < 2) : (warp == 0);
-    if (writer) {
-      float* dst = xbuf + (size_t)(warp - writers_lo) * kVals * 32 + lane;
-#pragma unroll
-      for (int m = 0; m < kMods; ++m)
-#pragma unroll
-        for (int mt = 0; mt < 8; ++mt)
-#pragma unroll
-          for (int r = 0; r < 4; ++r) dst[((m * 8 + mt) * 4 + r) * 32] = st.acc[m][mt][r];
-      dst[(kVals - 2) * 32] = st.l[0];
-      dst[(kVals - 1) * 32] = st.l[1];
-    }
-    __syncthreads();
-    if (reader) {
-      const float* src = xbuf + (size_t)warp * kVals * 32 + lane;
-#pragma unroll
-      for (int m = 0; m < kMods; ++m)
-#pragma unroll
-        for (int mt = 0; mt < 8; ++mt)
-#pragma unroll
-          for (int r = 0; r < 4; ++r) st.acc[m][mt][r] += src[((m * 8 + mt) * 4 + r) * 32];
-      st.l[0] += src[(kVals - 2) * 32];
-      st.l[1] += src[(kVals - 1) * 32];
+      for (int j = 0; j < 2; ++j) {
+        const int hh = 2 * t + j;
+        if (hh >= G) continue;
+        Partial* out = p.partials + ((size_t)b * Hq + kvh * G + hh) * p.num_splits + split;
+        *reinterpret_cast<float2*>(&out->acc[m][16 * g + 2 * mt]) = make_float2(v[j], v[j + 2]);
+      }
     }
     __syncthreads();
   }
-  // ---- warp 0 writes one partial per query head of the group
-  if (warp == 0) {
+  if (warp == 0 && g == 0) {
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
       const int hh = 2 * t + j;
       if (hh >= G) continue;
+      float l = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) l += sm.lw[w][hh];
       Partial* out = p.partials + ((size_t)b * Hq + kvh * G + hh) * p.num_splits + split;
-#pragma unroll
-      for (int m = 0; m < kMods; ++m)
-#pragma unroll
-        for (int mt = 0; mt < 8; ++mt)
-          *reinterpret_cast<float2*>(&out->acc[m][16 * g + 2 * mt]) =
-              make_float2(st.acc[m][mt][j], st.acc[m][mt][j + 2]);
-      if (g == 0) {
-        out->m = M[j];
-        out->l = st.l[j];
-      }
+      out->m = M[j];
+      out->l = l;
     }
   }
 }
@@ -685,19 +784,11 @@ __device__ __forceinline__ void build_score_operand(DecodeSmem& sm, float k0scal
   }
 }
 
-__global__ void __launch_bounds__(kThreads, 2) decode_split_k_kernel(const DecodeParams p) {
-  __shared__ DecodeSmem sm;
-  const int b = blockIdx.z, kvh = blockIdx.y, split = blockIdx.x;
-  int T, w0, w1;
-  split_range(p, b, split, T, w0, w1);
-  if (w0 == w1) {  // empty split (short sequence): only m and l are read by the combine
-    if (threadIdx.x < p.group) {
-      Partial* out = p.partials + ((size_t)b * p.num_kv_heads * p.group + kvh * p.group + threadIdx.x) * p.num_splits + split;
-      out->m = -INFINITY;
-      out->l = 0.0f;
-    }
-    return;
-  }
+// One decode CTA: split `split` of kv head kvh of sequence b.
+__device__ __forceinline__ void decode_cta(const DecodeParams& p, DecodeSmem& sm, int b, int kvh, int split) {
+  // ---- independent of the cache (overlaps the previous launch of the stream):
+  // query rotation, score operand, L2 prefetch of this split's share of the
+  // value bases (read by the combine)
   bool fast = false;
   float k0 = 0.f, k1 = 0.f, k2 = 0.f, v0 = 0.f, v1 = 0.f, v2 = 0.f;
   if (p.key_bits == 2 && p.value_bits == 2) {
@@ -707,8 +798,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_split_k_kernel(const Decod
     const float v3 = p.val_cb[3];
     fast = (k0 == -k3) && (k1 == -k2) && (v0 == -v3) && (v1 == -v2);
   }
-  if (fast) prime_pipeline(p, sm, b, kvh, w0, w1);  // window copies start before the query work
-  // warm the L2 with this split's share of the value bases, read by the combine
   {
     const size_t ubytes = (size_t)kMods * kHeadDim * kHeadDim * sizeof(float);
     const size_t share = (ubytes + p.num_splits - 1) / p.num_splits;
@@ -719,21 +808,156 @@ __global__ void __launch_bounds__(kThreads, 2) decode_split_k_kernel(const Decod
   }
   rotate_queries(p, b, kvh, sm.q);
   __syncthreads();
+  if (fast) build_score_operand(sm, (k1 - k0) * 128.0f, (k2 - k0) * 0.5f);
+
+  // ---- the cache: lengths and records may come from the previous launch
+  griddep_wait();
+  int T, w0, w1;
+  split_range(p, b, split, T, w0, w1);
+  if (w0 == w1) {  // empty split (short sequence): only m and l are read by the combine
+    if (threadIdx.x < p.group) {
+      Partial* out = p.partials + ((size_t)b * p.num_kv_heads * p.group + kvh * p.group + threadIdx.x) * p.num_splits + split;
+      out->m = -INFINITY;
+      out->l = 0.0f;
+    }
+    return;
+  }
   if (fast) {
-    build_score_operand(sm, (k1 - k0) * 128.0f, (k2 - k0) * 0.5f);
+    prime_pipeline(p, sm, b, kvh, w0, w1);
+    if (threadIdx.x < 32) tmem_alloc(&sm.tmem_base, kTmemCols);
+    tc_fence_before();
     __syncthreads();
-    decode_mma(p, sm, b, kvh, split, (v1 - v0) * 128.0f, (v2 - v0) * 0.5f, v0);
+    tc_fence_after();
+    const uint32_t tbase = sm.tmem_base;
+    decode_mma(p, sm, b, kvh, split, (v1 - v0) * 128.0f, (v2 - v0) * 0.5f, v0, tbase);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (threadIdx.x < 32) tmem_dealloc(tbase, kTmemCols);
     return;
   }
   decode_generic(p, sm, b, kvh, split);
 }
 
+__global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_split_k_kernel(const DecodeParams p) {
+  __shared__ DecodeSmem sm;
+  griddep_launch_dependents();
+  decode_cta(p, sm, blockIdx.z, blockIdx.y, blockIdx.x);
+}
+
+// Decode step: CTAs [0, batch * H) append one token to (sequence, kv head) and
+// then publish the new length in the step flag; the others are decode CTAs
+// (split fastest, then kv head, then sequence). Only the warp decoding the
+// window that receives the token waits for the flag, before copying it.
+__global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_step_kernel(const DecodeParams p, const WriteParams w) {
+  __shared__ DecodeSmem sm;
+  static_assert(sizeof(WindowSmem) <= sizeof(DecodeSmem), "append uses the decode shared memory");
+  griddep_launch_dependents();
+  const int H = p.num_kv_heads;
+  const int nappend = p.batch * H;
+  if ((int)blockIdx.x < nappend) {
+    griddep_wait();
+    const int b = blockIdx.x / H, h = blockIdx.x % H;
+    const int L0 = w.seq_lens[b];
+    const int L1 = L0 + 1;
+    if (L0 >= 0 && L1 <= w.cap_tokens) {
+      quantize_window(w, b, h, L0 / kWindow, L0, L1, *reinterpret_cast<WindowSmem*>(&sm), threadIdx.x, 1, true);
+      if (h > 0 && threadIdx.x == 0) {  // the decode of head h reads the token's modality after h's flag
+        const int m = w.mod_new[b];
+        w.modality[(size_t)b * w.cap_tokens + L0] = (uint8_t)(m >= kMods ? kMods - 1 : m);
+      }
+      __threadfence();
+      __syncthreads();
+      if (threadIdx.x == 0)
+        asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(w.step_flags + (size_t)b * H + h), "r"(L1)
+                     : "memory");
+    } else if (threadIdx.x == 0 && h == 0) {
+      set_error(w.error_word, OMNIKV_DEVERR_CAPACITY);
+    }
+    return;
+  }
+  const int r = blockIdx.x - nappend;
+  decode_cta(p, sm, r / (p.num_splits * H), (r / p.num_splits) % H, r % p.num_splits);
+}
+
+// Several decode CTAs share an SM only if the SM's unified L1 / shared memory is
+// split in favour of shared memory; without a preference the runtime may pick a
+// split that holds one CTA. Set once per device (bit d of the mask).
+std::atomic<uint64_t> g_carveout_set{0};
+
+cudaError_t prefer_shared_carveout() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (1ull << dev) : 0ull;
+  if (bit && (g_carveout_set.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(decode_split_k_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared);
+  if (e == cudaSuccess && bit) g_carveout_set.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
+
 }  // namespace
 
+// Resident decode CTAs per SM, from the kernel's registers and shared memory and
+// the TMEM columns each CTA allocates (computed from the attributes rather than
+// the runtime occupancy query, which does not report the residency seen on
+// sm_100a for this kernel). Cached per device.
+int decode_ctas_per_sm() {
+  static std::atomic<int> cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return kCtasPerSm;
+  if (dev < 64) {
+    const int c = cached[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
+  cudaFuncAttributes a;
+  int regs_sm = 0, smem_sm = 0, smem_rsv = 0;
+  if (prefer_shared_carveout() != cudaSuccess || cudaFuncGetAttributes(&a, decode_split_k_kernel) != cudaSuccess ||
+      cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&smem_rsv, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess)
+    return kCtasPerSm;
+  const int warp_regs = ((a.numRegs * 32 + 255) / 256) * 256;  // allocated per warp in units of 256
+  const int by_regs = regs_sm / (warp_regs * kWarps);
+  const int by_smem = smem_sm / ((int)a.sharedSizeBytes + smem_rsv);
+  const int by_tmem = 512 / (int)kTmemCols;
+  const int n = max(1, min(by_regs, min(by_smem, by_tmem)));
+  if (dev < 64) cached[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+cudaError_t launch_decode_step(const DecodeParams& p, const WriteParams& w, cudaStream_t stream) {
+  cudaError_t e = prefer_shared_carveout();
+  if (e != cudaSuccess) return e;
+  static std::atomic<uint64_t> step_carveout{0};
+  int dev = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (1ull << dev) : 0ull;
+  if (!bit || !(step_carveout.load(std::memory_order_acquire) & bit)) {
+    e = cudaFuncSetAttribute(decode_step_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    if (bit) step_carveout.fetch_or(bit, std::memory_order_acq_rel);
+  }
+  const int ctas = p.batch * p.num_kv_heads * (1 + p.num_splits);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ctas);
+  cfg.blockDim = dim3(kThreads);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_step_kernel, p, w);
+}
+
 cudaError_t launch_decode(const DecodeParams& p, int batch, cudaStream_t stream) {
+  const cudaError_t e = prefer_shared_carveout();
+  if (e != cudaSuccess) return e;
   dim3 grid(p.num_splits, p.num_kv_heads, batch);
-  decode_split_k_kernel<<<grid, kThreads, 0, stream>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(decode_split_k_kernel, grid, dim3(kThreads), 0, stream, p);
 }
 
 }  // namespace omnikv

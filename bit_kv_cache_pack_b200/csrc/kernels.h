@@ -27,6 +27,7 @@ struct WriteParams {
   const uint8_t* mod_new;
   int n_new;
   int tc_values;  // 1: values of windows filled completely by this write are done by vrot_tc
+  int32_t* step_flags;  // decode step only: [batch][kv heads], set to the new length once written
 };
 
 struct DecodeParams {
@@ -44,6 +45,11 @@ struct DecodeParams {
   int num_splits;
   int split_windows;  // windows per split (C)
   int32_t* error_word;
+  int batch;
+  // decode step only: the length seen is seq_lens[b] + len_add, and the window
+  // holding the appended position is read once step_flags[b][h] == that length
+  int len_add;
+  const int32_t* step_flags;
 };
 
 struct CombineParams {
@@ -52,6 +58,9 @@ struct CombineParams {
   const Partial* partials;
   int num_splits;
   float* out;
+  // decode step only: seq_lens[b] += len_add (when within cap_tokens) after the merge
+  int32_t* seq_lens;
+  int len_add, cap_tokens;
 };
 
 // Dense bf16 decode (comparison baseline).
@@ -68,9 +77,33 @@ struct DenseParams {
 };
 cudaError_t launch_dense(const DenseParams& p, int batch, cudaStream_t stream);
 
+// Launch with programmatic stream serialisation: the kernel may start while
+// the previous kernel of the stream is still running; it calls griddep_wait()
+// before touching anything that kernel may write, and griddep_launch_dependents()
+// to let its own successor start early.
+template <typename Kernel, typename Params>
+cudaError_t launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, const Params& p) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
 cudaError_t launch_write(const WriteParams& p, int batch, cudaStream_t stream);
 cudaError_t launch_vrot_tc(const WriteParams& p, int batch, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeParams& p, int batch, cudaStream_t stream);
+// The decode launch of a decode step: batch * kv heads append CTAs (one token per
+// sequence, described by w) followed by the decode CTAs of p.
+cudaError_t launch_decode_step(const DecodeParams& p, const WriteParams& w, cudaStream_t stream);
+
+int decode_ctas_per_sm();  // resident decode CTAs per SM on the current device
 cudaError_t launch_combine(const CombineParams& p, int batch, cudaStream_t stream);
 
 }  // namespace omnikv

@@ -72,16 +72,6 @@ __device__ __forceinline__ uint64_t make_desc_sw128(uint32_t saddr) {
 // K-major, N = 128, M = 128.
 constexpr uint32_t kIdesc = (1u << 4) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 
-__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(dst_smem)),
-               "r"(ncols));
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::);
-}
-
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(taddr), "r"(ncols));
-}
-
 __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                          uint32_t accumulate) {
   asm volatile(
@@ -98,29 +88,11 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
                : "memory");
 }
 
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
-
-// 32 consecutive fp32 columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float v[32]) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
 __global__ void __launch_bounds__(kVThreads, 1) vrot_tc_kernel(const WriteParams p) {
   extern __shared__ uint8_t dyn_smem[];
   VrotSmem& sm = *reinterpret_cast<VrotSmem*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
+  griddep_launch_dependents();
+  griddep_wait();  // kv_quant_pack (just before) writes the records' key parts
   const int b = blockIdx.z, h = blockIdx.y;
   const int H = p.num_kv_heads;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -247,13 +219,13 @@ __global__ void __launch_bounds__(kVThreads, 1) vrot_tc_kernel(const WriteParams
       const uint32_t row_addr = tmem + ((uint32_t)(32 * warp) << 16);
 #pragma unroll
       for (int cb = 0; cb < 4; ++cb) {
-        float v[32];
+        uint32_t v[32];
         tmem_ld32(row_addr + 32 * cb, v);  // warp-collective: every lane loads
         if (mine) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             uint32_t code = 0;
-            if (s != 0.0f) code = count_above(__fdiv_rn(v[i], s), sm.thr, LV - 1);
+            if (s != 0.0f) code = count_above(__fdiv_rn(__uint_as_float(v[i]), s), sm.thr, LV - 1);
             sm.codes[32 * cb + i][r] = (uint8_t)code;
           }
         }
@@ -303,8 +275,7 @@ cudaError_t launch_vrot_tc(const WriteParams& p, int batch, cudaStream_t stream)
   if (e != cudaSuccess) return e;
   const int tiles = (p.n_new / kWindow + 1 + 3) / 4;  // full windows <= n_new / 32 (+1 for alignment)
   dim3 grid(tiles, p.num_kv_heads, batch);
-  vrot_tc_kernel<<<grid, kVThreads, smem, stream>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(vrot_tc_kernel, grid, dim3(kVThreads), (size_t)smem, stream, p);
 }
 
 }  // namespace omnikv

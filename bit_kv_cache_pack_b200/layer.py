@@ -50,8 +50,10 @@ class KVCache:
         self.modality = torch.zeros(batch, cap_tokens, dtype=torch.uint8, device=dev)
         self.seq_lens = torch.zeros(batch, dtype=torch.int32, device=dev)
         self.error_word = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.step_flags = torch.zeros(batch, num_kv_heads, dtype=torch.int32, device=dev)
         self.struct = OmniKVCache(self.records.data_ptr(), self.key_tail.data_ptr(), self.modality.data_ptr(),
-                                  self.seq_lens.data_ptr(), self.error_word.data_ptr(), batch, cap_tokens, 0)
+                                  self.seq_lens.data_ptr(), self.error_word.data_ptr(), batch, cap_tokens, 0,
+                                  self.step_flags.data_ptr())
 
     @property
     def max_seq_len(self) -> int:
@@ -62,7 +64,7 @@ class KVCache:
         is the batch-wide bound."""
         return OmniKVCache(self.records[b].data_ptr(), self.key_tail[b].data_ptr(), self.modality[b].data_ptr(),
                            self.seq_lens[b:].data_ptr(), self.error_word.data_ptr(), 1, self.cap_tokens,
-                           self.struct.max_seq_len)
+                           self.struct.max_seq_len, self.step_flags[b].data_ptr())
 
 
 def partials_tensor(batch: int, num_q_heads: int, num_splits: int, device="cuda") -> torch.Tensor:

@@ -61,7 +61,7 @@ extern "C" {
 #define OMNIKV_API
 #endif
 
-#define OMNIKV_ABI_VERSION 1
+#define OMNIKV_ABI_VERSION 2
 #define OMNIKV_HEAD_DIM 128
 #define OMNIKV_WINDOW 32
 #define OMNIKV_NUM_MODALITIES 3 /* 0 = text (L), 1 = audio (A), 2 = video (V) */
@@ -111,6 +111,9 @@ typedef struct {
   int32_t cap_tokens;   /* capacity per sequence, a positive multiple of 32 */
   int32_t max_seq_len;  /* HOST-side upper bound on every seq_lens[b]; sizes grids and checks capacity.
                            omnikv_write_cache adds n_new to it on success. */
+  int32_t* step_flags;  /* optional [batch][num_kv_heads] int32, zero-filled with the cache; used (and
+                           required) only by omnikv_decode_step, which stores the new length there once
+                           the appended token's window record is written; may be NULL otherwise */
 } omnikv_cache;
 
 /* Bytes of one window record: 2624 for K2/V2, 4672 for K4/V4; 0 for unsupported bits. */
@@ -166,6 +169,23 @@ OMNIKV_API omnikv_status omnikv_decode_attention(const omnikv_config* cfg, const
  *   out        : [batch][num_q_heads][128] fp32 */
 OMNIKV_API omnikv_status omnikv_combine(const omnikv_config* cfg, const omnikv_cache* cache,
                              const void* partials, int32_t num_splits, float* out, void* stream);
+
+/* One decode step: append ONE token to every sequence (as omnikv_write_cache with n_new = 1), then
+ * decode attention over the cache including it and combine (as omnikv_decode_attention +
+ * omnikv_combine), in two launches instead of four: the append runs in CTAs of the decode launch,
+ * concurrently with the decode of the other windows; only the warp that decodes a sequence's last
+ * window waits (bounded, OMNIKV_DEVERR_TIMEOUT on expiry) until cache->step_flags[b][h] holds the
+ * new length, and the combine launch advances seq_lens[b]. Results are identical to the four calls.
+ *   q                     : [batch][num_q_heads][128] fp16 (the step's queries)
+ *   k_new, v_new          : [batch][num_kv_heads][1][128] fp16; modality_new: [batch] u8
+ *   partials, num_splits  : as for omnikv_decode_attention (num_splits = 0: the default, lowered if
+ *                           needed so that every CTA of the launch is resident at once)
+ *   out                   : [batch][num_q_heads][128] fp32
+ * Requires cache->step_flags (OMNIKV_ERR_INVALID_ARG without it);
+ * OMNIKV_ERR_CAPACITY if cache->max_seq_len + 1 > cap_tokens; advances cache->max_seq_len by 1. */
+OMNIKV_API omnikv_status omnikv_decode_step(const omnikv_config* cfg, omnikv_cache* cache, const void* q,
+                                            const void* k_new, const void* v_new, const uint8_t* modality_new,
+                                            void* partials, int32_t num_splits, float* out, void* stream);
 
 /* Decode attention and combine in one call, with the split-K partials in a fixed device array of
  * OMNIKV_DECODE_STATIC_SCRATCH_BYTES owned by this library; the caller passes only inputs (q) and

@@ -32,8 +32,15 @@ def test_every_declared_symbol_is_exported():
     assert set(names) >= set(_abi.EXPORTED)
 
 
+def test_package_exports_every_binding():
+    import bit_kv_cache_pack_b200 as pkg
+    for n in _abi.EXPORTED:
+        if n not in ("omnikv_status_string",):
+            assert hasattr(pkg, n), n
+
+
 def test_sizes_and_version():
-    assert _abi.omnikv_abi_version() == 1
+    assert _abi.omnikv_abi_version() == 2
     assert _abi.omnikv_record_bytes(2, 2) == 2624
     assert _abi.omnikv_record_bytes(4, 4) == 4672
     assert _abi.omnikv_record_bytes(2, 4) == 1024 + 512 + 2048 + 64
@@ -54,7 +61,7 @@ def _cfg(**kw):
 
 
 def _cache(**kw):
-    c = OmniKVCache(FAKE, FAKE, FAKE, FAKE, 0, 1, 2048, 0)
+    c = OmniKVCache(FAKE, FAKE, FAKE, FAKE, 0, 1, 2048, 0, FAKE)
     for k, v in kw.items():
         setattr(c, k, v)
     return c
@@ -128,3 +135,20 @@ def test_binding_rejects_non_contiguous_tensors():
     with pytest.raises(ValueError):
         _abi._ptr(t)
     assert _abi._ptr(torch.zeros(3)) != 0
+
+
+def _step_status(cfg, cache, q=FAKE, k=FAKE, v=FAKE, mod=FAKE, part=FAKE, out=FAKE):
+    lib = _abi.load()
+    return lib.omnikv_decode_step(ctypes.byref(cfg), ctypes.byref(cache), q, k, v, mod, part, 0, out, 0)
+
+
+def test_decode_step_arguments_rejected():
+    """The fused step needs the cache's step flags and every buffer, and checks
+    the capacity for its one appended token, all before any launch."""
+    assert _step_status(_cfg(), _cache(step_flags=None)) == _abi.OMNIKV_ERR_INVALID_ARG
+    assert _step_status(_cfg(), _cache(step_flags=FAKE + 2)) == _abi.OMNIKV_ERR_INVALID_ARG
+    for kw in ("q", "k", "v", "mod", "part", "out"):
+        assert _step_status(_cfg(), _cache(), **{kw: None}) == _abi.OMNIKV_ERR_INVALID_ARG, kw
+    assert _step_status(_cfg(), _cache(), k=FAKE + 8) == _abi.OMNIKV_ERR_INVALID_ARG
+    assert _step_status(_cfg(), _cache(max_seq_len=2048)) == _abi.OMNIKV_ERR_CAPACITY
+    assert _step_status(_cfg(key_bits=3), _cache()) == _abi.OMNIKV_ERR_UNSUPPORTED

@@ -30,10 +30,10 @@ def test_static_scratch_rejects_what_does_not_fit():
     fake = 0x10000
     cfg = OmniKVConfig(128, 16, 2, 32, 2, 2, fake, fake, fake, fake)
     lib = _abi.load()
-    big = OmniKVCache(fake, fake, fake, fake, 0, 400, 2048, 2048)     # 400 * 16 = 6400 entries > 5405
+    big = OmniKVCache(fake, fake, fake, fake, 0, 400, 2048, 2048, 0)     # 400 * 16 = 6400 entries > 5405
     assert lib.omnikv_decode_static(ctypes.byref(cfg), ctypes.byref(big), fake, fake, 1, 0) == \
         _abi.OMNIKV_ERR_CAPACITY
-    small = OmniKVCache(fake, fake, fake, fake, 0, 1, 2048, 2048)     # 16 entries per split
+    small = OmniKVCache(fake, fake, fake, fake, 0, 1, 2048, 2048, 0)     # 16 entries per split
     assert lib.omnikv_decode_static(ctypes.byref(cfg), ctypes.byref(small), fake, fake, 400, 0) == \
         _abi.OMNIKV_ERR_CAPACITY                                      # 6400 entries again
     assert lib.omnikv_decode_static(ctypes.byref(cfg), ctypes.byref(small), None, fake, 1, 0) == \
