@@ -15,13 +15,39 @@ struct __align__(16) WindowSmem {  // 16-byte multiple: per-group copies stay fl
   float kp[kWindow][kHeadDim];  // rotated keys, then reused for fp32 values
   float s_min[kHeadDim], s_scale[kHeadDim];
   float s_sigma[kWindow];
-  float thr_k[15], thr_v[15];
+  CodeBound bk[15], bv[15];  // code decision bounds (keys: after + c_0; values: none added)
 };
 
 static_assert(sizeof(WindowSmem) % 16 == 0, "per-group shared memory must keep 16-byte alignment");
 
 // Barrier over the 128 threads of one group (id 0 is __syncthreads).
 __device__ __forceinline__ void group_sync(int id) { asm volatile("bar.sync %0, 128;\n" ::"r"(id) : "memory"); }
+
+// Key codes of the window's valid tokens, 32 / BITS per token-major word:
+// code = #{j : (k' - m) / s + c_0 > t_j}, 0 where s == 0.
+template <int BITS>
+__device__ __forceinline__ void key_code_words(const WriteParams& p, const WindowSmem& sm, uint8_t* kout, int nvalid,
+                                               int tid) {
+  constexpr int cpw = 32 / BITS, wpt = kHeadDim / cpw;
+  const CodeBounds<(1 << BITS) - 1> bk = load_bounds<(1 << BITS) - 1>(sm.bk);
+  uint32_t* kw = reinterpret_cast<uint32_t*>(kout);
+  for (int wi = tid; wi < kWindow * wpt; wi += kWriteThreads) {
+    const int t = wi / wpt;
+    const int word = wi - t * wpt;
+    uint32_t bits = 0;
+    if (t < nvalid) {
+#pragma unroll
+      for (int k = 0; k < cpw; ++k) {
+        const int ch = word * cpw + k;
+        const float s = sm.s_scale[ch];
+        uint32_t code = 0;
+        if (s != 0.0f) code = code_from_bounds(bk, (double)__fsub_rn(sm.kp[t][ch], sm.s_min[ch]), (double)s);
+        bits |= code << (BITS * k);
+      }
+    }
+    kw[wi] = bits;
+  }
+}
 
 // Re-quantise window w of (sequence b, kv head h) after the append of
 // positions [L0, L1), by the 128 threads of one group (tid 0..127, barrier
@@ -49,16 +75,17 @@ __device__ void quantize_window(const WriteParams& p, int b, int h, int w, int L
   float* s_min = sm.s_min;
   float* s_scale = sm.s_scale;
   float* s_sigma = sm.s_sigma;
-  float* thr_k = sm.thr_k;
-  float* thr_v = sm.thr_v;
 
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const int LK = 1 << p.key_bits;
   const int LV = 1 << p.value_bits;
-  if (tid < LK - 1) thr_k[tid] = __fmul_rn(__fadd_rn(p.key_cb[tid], p.key_cb[tid + 1]), 0.5f);
-  if (tid < LV - 1) thr_v[tid] = __fmul_rn(__fadd_rn(p.val_cb[tid], p.val_cb[tid + 1]), 0.5f);
   const float kc0 = p.key_cb[0];
+  if (tid < LK - 1) sm.bk[tid] = make_code_bound(__fmul_rn(__fadd_rn(p.key_cb[tid], p.key_cb[tid + 1]), 0.5f), kc0);
+  if (tid >= 32 && tid - 32 < LV - 1) {
+    const int j = tid - 32;
+    sm.bv[j] = make_code_bound(__fmul_rn(__fadd_rn(p.val_cb[j], p.val_cb[j + 1]), 0.5f), 0.0f);
+  }
   const float kspan = __fsub_rn(p.key_cb[LK - 1], kc0);
 
   // ---- issue every raw-key load of the window first (one memory round trip),
@@ -121,29 +148,10 @@ __device__ void quantize_window(const WriteParams& p, int b, int h, int w, int L
   group_sync(bar_id);
 
   // ---- key codes, token-major words -----------------------------------------
-  {
-    const int cpw = 32 / p.key_bits;
-    const int wpt = kHeadDim / cpw;
-    uint32_t* kw = reinterpret_cast<uint32_t*>(rec + lay.k_off);
-    for (int wi = tid; wi < kWindow * wpt; wi += kWriteThreads) {
-      const int t = wi / wpt;
-      const int word = wi - t * wpt;
-      uint32_t bits = 0;
-      if (t < nvalid) {
-        for (int k = 0; k < cpw; ++k) {
-          const int ch = word * cpw + k;
-          const float s = s_scale[ch];
-          uint32_t code = 0;
-          if (s != 0.0f) {
-            const float z = __fadd_rn(__fdiv_rn(__fsub_rn(kp[t][ch], s_min[ch]), s), kc0);
-            code = count_above(z, thr_k, LK - 1);
-          }
-          bits |= code << (p.key_bits * k);
-        }
-      }
-      kw[wi] = bits;
-    }
-  }
+  if (p.key_bits == 2)
+    key_code_words<2>(p, sm, rec + lay.k_off, nvalid, tid);
+  else
+    key_code_words<4>(p, sm, rec + lay.k_off, nvalid, tid);
   group_sync(bar_id);  // kp is reused for values below
 
   // windows filled completely by this write get their values from vrot_tc
@@ -196,8 +204,10 @@ __device__ void quantize_window(const WriteParams& p, int b, int h, int w, int L
       for (int c = 0; c < kHeadDim; ++c) part[c & 7] = fmaf(U[(size_t)c * kHeadDim], kp[i][c], part[c & 7]);
       const float acc = ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
       const float s = s_sigma[i];
-      uint32_t code = 0;
-      if (s != 0.0f) code = count_above(__fdiv_rn(acc, s), thr_v, LV - 1);
+      uint32_t code = 0;  // #{j : v' / sigma > t_j}, 0 where sigma == 0
+      if (s != 0.0f)
+        code = p.value_bits == 2 ? code_from_bounds(load_bounds<3>(sm.bv), (double)acc, (double)s)
+                                 : code_from_bounds(load_bounds<15>(sm.bv), (double)acc, (double)s);
       const int g = i / cpw;
       const int sh = p.value_bits * (i - g * cpw);
 #pragma unroll

@@ -90,6 +90,62 @@ __device__ __forceinline__ uint32_t count_above(float z, const float* thr, int n
   return c;
 }
 
+// Division-free, exact form of the code decision  fl(fl(a / s) + c) > t  for
+// s > 0 (fl: fp32 round to nearest even). y -> fl(y + c) is monotone, so the
+// decision is  fl(a / s) >= F  for F the smallest float with fl(F + c) > t; and
+// fl(x) >= F  iff  x > mid  or  (x == mid and F has an even significand), mid
+// the midpoint of F and its predecessor (the rounding boundary). The sign of
+// a - mid * s is exact in one fp64 FMA: mid has at most 25 significant bits,
+// s (an fp16 value) 11 and a (fp32) 24, so mid * s is exact and the FMA rounds
+// only its exact result. s = +inf gives the decision for a / s = 0.
+struct CodeBound {
+  double mid;
+  int tie_up;  // 1: a / s == mid rounds up to F
+};
+
+__device__ inline CodeBound make_code_bound(float t, float c) {
+  float y = __fsub_rn(t, c);
+  for (int i = 0; i < 64 && __fadd_rn(y, c) > t; ++i) y = nextafterf(y, -INFINITY);
+  for (int i = 0; i < 64 && !(__fadd_rn(y, c) > t); ++i) y = nextafterf(y, INFINITY);
+  const float prev = nextafterf(y, -INFINITY);
+  CodeBound b;
+  b.mid = 0.5 * ((double)prev + (double)y);
+  b.tie_up = (__float_as_uint(y) & 1u) == 0u;
+  return b;
+}
+
+// The NB = 2^bits - 1 bounds of one code, in registers.
+template <int NB>
+struct CodeBounds {
+  double mid[NB];
+  uint32_t tie_up;  // bit j: a / s == mid[j] rounds up past threshold j
+};
+
+template <int NB>
+__device__ __forceinline__ CodeBounds<NB> load_bounds(const CodeBound* bd) {
+  CodeBounds<NB> r;
+  r.tie_up = 0;
+#pragma unroll
+  for (int j = 0; j < NB; ++j) {
+    r.mid[j] = bd[j].mid;
+    r.tie_up |= (uint32_t)bd[j].tie_up << j;
+  }
+  return r;
+}
+
+// #{ j : fl(fl(a / s) + c) > t_j }: every threshold decided independently and
+// without branches (no dependent chain), for the ascending thresholds of `b`.
+template <int NB>
+__device__ __forceinline__ uint32_t code_from_bounds(const CodeBounds<NB>& b, double a, double s) {
+  uint32_t code = 0;
+#pragma unroll
+  for (int j = 0; j < NB; ++j) {
+    const double d = fma(-b.mid[j], s, a);
+    code += (uint32_t)(d > 0.0) | ((uint32_t)(d == 0.0) & ((b.tie_up >> j) & 1u));
+  }
+  return code;
+}
+
 __device__ __forceinline__ void set_error(int32_t* word, int32_t bits) {
   if (word) atomicOr(word, bits);
 }

@@ -81,8 +81,8 @@ cudaError_t launch_dense(const DenseParams& p, int batch, cudaStream_t stream);
 // the previous kernel of the stream is still running; it calls griddep_wait()
 // before touching anything that kernel may write, and griddep_launch_dependents()
 // to let its own successor start early.
-template <typename Kernel, typename Params>
-cudaError_t launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, const Params& p) {
+template <typename Kernel, typename... Args>
+cudaError_t launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, const Args&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -93,7 +93,7 @@ cudaError_t launch_pdl(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaSt
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, p);
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
 cudaError_t launch_write(const WriteParams& p, int batch, cudaStream_t stream);
