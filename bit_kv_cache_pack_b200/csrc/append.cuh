@@ -16,6 +16,7 @@ struct __align__(16) WindowSmem {  // 16-byte multiple: per-group copies stay fl
   float s_min[kHeadDim], s_scale[kHeadDim];
   float s_sigma[kWindow];
   CodeBound bk[15], bv[15];  // code decision bounds (keys: after + c_0; values: none added)
+  uint8_t codes[kWindow][kHeadDim];  // key codes (token, channel) before packing
 };
 
 static_assert(sizeof(WindowSmem) % 16 == 0, "per-group shared memory must keep 16-byte alignment");
@@ -23,28 +24,28 @@ static_assert(sizeof(WindowSmem) % 16 == 0, "per-group shared memory must keep 1
 // Barrier over the 128 threads of one group (id 0 is __syncthreads).
 __device__ __forceinline__ void group_sync(int id) { asm volatile("bar.sync %0, 128;\n" ::"r"(id) : "memory"); }
 
-// Key codes of the window's valid tokens, 32 / BITS per token-major word:
-// code = #{j : (k' - m) / s + c_0 > t_j}, 0 where s == 0.
+// Key codes of the window's valid tokens, code = #{j : (k' - m) / s + c_0 > t_j}
+// (0 where s == 0): thread c decides channel c for every token with the
+// channel's fp32 bounds, then the codes are packed 32 / BITS per token-major word.
 template <int BITS>
-__device__ __forceinline__ void key_code_words(const WriteParams& p, const WindowSmem& sm, uint8_t* kout, int nvalid,
-                                               int tid) {
-  constexpr int cpw = 32 / BITS, wpt = kHeadDim / cpw;
-  const CodeBounds<(1 << BITS) - 1> bk = load_bounds<(1 << BITS) - 1>(sm.bk);
+__device__ __forceinline__ void key_code_words(WindowSmem& sm, uint8_t* kout, int nvalid, int tid, int bar_id) {
+  constexpr int NB = (1 << BITS) - 1, cpw = 32 / BITS, wpt = kHeadDim / cpw;
+  {
+    const int c = tid;
+    const float s = sm.s_scale[c], m = sm.s_min[c];
+    const ScaledBounds<NB> sb = scale_bounds(load_bounds<NB>(sm.bk), s);
+    for (int t = 0; t < kWindow; ++t)
+      sm.codes[t][c] = (uint8_t)((t < nvalid && s != 0.0f) ? code_from_scaled(sb, __fsub_rn(sm.kp[t][c], m)) : 0u);
+  }
+  group_sync(bar_id);
   uint32_t* kw = reinterpret_cast<uint32_t*>(kout);
   for (int wi = tid; wi < kWindow * wpt; wi += kWriteThreads) {
     const int t = wi / wpt;
     const int word = wi - t * wpt;
+    const uint8_t* src = &sm.codes[t][word * cpw];
     uint32_t bits = 0;
-    if (t < nvalid) {
 #pragma unroll
-      for (int k = 0; k < cpw; ++k) {
-        const int ch = word * cpw + k;
-        const float s = sm.s_scale[ch];
-        uint32_t code = 0;
-        if (s != 0.0f) code = code_from_bounds(bk, (double)__fsub_rn(sm.kp[t][ch], sm.s_min[ch]), (double)s);
-        bits |= code << (BITS * k);
-      }
-    }
+    for (int k = 0; k < cpw; ++k) bits |= (uint32_t)src[k] << (BITS * k);
     kw[wi] = bits;
   }
 }
@@ -149,9 +150,9 @@ __device__ void quantize_window(const WriteParams& p, int b, int h, int w, int L
 
   // ---- key codes, token-major words -----------------------------------------
   if (p.key_bits == 2)
-    key_code_words<2>(p, sm, rec + lay.k_off, nvalid, tid);
+    key_code_words<2>(sm, rec + lay.k_off, nvalid, tid, bar_id);
   else
-    key_code_words<4>(p, sm, rec + lay.k_off, nvalid, tid);
+    key_code_words<4>(sm, rec + lay.k_off, nvalid, tid, bar_id);
   group_sync(bar_id);  // kp is reused for values below
 
   // windows filled completely by this write get their values from vrot_tc
@@ -206,8 +207,8 @@ __device__ void quantize_window(const WriteParams& p, int b, int h, int w, int L
       const float s = s_sigma[i];
       uint32_t code = 0;  // #{j : v' / sigma > t_j}, 0 where sigma == 0
       if (s != 0.0f)
-        code = p.value_bits == 2 ? code_from_bounds(load_bounds<3>(sm.bv), (double)acc, (double)s)
-                                 : code_from_bounds(load_bounds<15>(sm.bv), (double)acc, (double)s);
+        code = p.value_bits == 2 ? code_from_scaled(scale_bounds(load_bounds<3>(sm.bv), s), acc)
+                                 : code_from_scaled(scale_bounds(load_bounds<15>(sm.bv), s), acc);
       const int g = i / cpw;
       const int sh = p.value_bits * (i - g * cpw);
 #pragma unroll

@@ -133,16 +133,36 @@ __device__ __forceinline__ CodeBounds<NB> load_bounds(const CodeBound* bd) {
   return r;
 }
 
-// #{ j : fl(fl(a / s) + c) > t_j }: every threshold decided independently and
-// without branches (no dependent chain), for the ascending thresholds of `b`.
+// The decisions for one scale s > 0 as fp32 bounds: decision j  <=>  a > b[j].
+// With T = mid_j * s (exact in fp64), a > T or (a == T and ties round up):
+// for T not an fp32 value, a > T <=> a > RD(T) (a is fp32); for T an fp32
+// value, a >= T <=> a > pred(T). s = +inf maps to +-inf bounds, the decisions
+// for a / s = 0.
 template <int NB>
-__device__ __forceinline__ uint32_t code_from_bounds(const CodeBounds<NB>& b, double a, double s) {
-  uint32_t code = 0;
+struct ScaledBounds {
+  float b[NB];
+};
+
+template <int NB>
+__device__ __forceinline__ ScaledBounds<NB> scale_bounds(const CodeBounds<NB>& cb, float s) {
+  ScaledBounds<NB> r;
+  const double sd = (double)s;
 #pragma unroll
   for (int j = 0; j < NB; ++j) {
-    const double d = fma(-b.mid[j], s, a);
-    code += (uint32_t)(d > 0.0) | ((uint32_t)(d == 0.0) & ((b.tie_up >> j) & 1u));
+    const double T = cb.mid[j] * sd;
+    float B = __double2float_rd(T);
+    if ((double)B == T && ((cb.tie_up >> j) & 1u)) B = nextafterf(B, -INFINITY);
+    r.b[j] = B;
   }
+  return r;
+}
+
+// #{ j : fl(fl(a / s) + c) > t_j } for the ascending thresholds behind `sb`.
+template <int NB>
+__device__ __forceinline__ uint32_t code_from_scaled(const ScaledBounds<NB>& sb, float a) {
+  uint32_t code = 0;
+#pragma unroll
+  for (int j = 0; j < NB; ++j) code += (a > sb.b[j]) ? 1u : 0u;
   return code;
 }
 

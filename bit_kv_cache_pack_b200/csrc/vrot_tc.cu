@@ -171,13 +171,13 @@ __device__ __forceinline__ void epilogue_codes(VrotSmem& sm, uint32_t tmem, int 
   const int r = 32 * (warp & 3) + lane, cb = warp >> 2;
   const bool mine = r < ntok && sm.mods[r] == m;
   const float sg = sm.sigma[r];
-  const double sd = (double)sg;
+  const ScaledBounds<(1 << BITS) - 1> sb = scale_bounds(bv, sg);
   uint32_t v[32];
   tmem_ld32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + 32 * cb, v);  // warp-collective
   if (mine) {
 #pragma unroll
     for (int c = 0; c < 32; ++c) {
-      const uint32_t code = code_from_bounds(bv, (double)__uint_as_float(v[c]), sd);
+      const uint32_t code = code_from_scaled(sb, __uint_as_float(v[c]));
       sm.codes[32 * cb + c][r] = (uint8_t)(sg != 0.0f ? code : 0u);
     }
   }
