@@ -24,6 +24,15 @@ static_assert(sizeof(WindowSmem) % 16 == 0, "per-group shared memory must keep 1
 // Barrier over the 128 threads of one group (id 0 is __syncthreads).
 __device__ __forceinline__ void group_sync(int id) { asm volatile("bar.sync %0, 128;\n" ::"r"(id) : "memory"); }
 
+// Column of channel c of token t in the rotated-key buffer: the 4-float chunks
+// of each 32-channel block are XOR-permuted by (t % 2, block), so that the 8
+// threads of a quarter warp storing one chunk each (2 tokens x 4 blocks) hit 8
+// different bank groups. Readers of a whole row see a permutation of it.
+__device__ __forceinline__ int kp_col(int t, int c) {
+  const int q = c >> 5, j = (c >> 2) & 7;
+  return 32 * q + 4 * (j ^ ((t & 1) | (q << 1))) + (c & 3);
+}
+
 // Key codes of the window's valid tokens, code = #{j : (k' - m) / s + c_0 > t_j}
 // (0 where s == 0): thread c decides channel c for every token with the
 // channel's fp32 bounds, then the codes are packed 32 / BITS per token-major word.
@@ -35,7 +44,7 @@ __device__ __forceinline__ void key_code_words(WindowSmem& sm, uint8_t* kout, in
     const float s = sm.s_scale[c], m = sm.s_min[c];
     const ScaledBounds<NB> sb = scale_bounds(load_bounds<NB>(sm.bk), s);
     for (int t = 0; t < kWindow; ++t)
-      sm.codes[t][c] = (uint8_t)((t < nvalid && s != 0.0f) ? code_from_scaled(sb, __fsub_rn(sm.kp[t][c], m)) : 0u);
+      sm.codes[t][c] = (uint8_t)((t < nvalid && s != 0.0f) ? code_from_scaled(sb, __fsub_rn(sm.kp[t][kp_col(t, c)], m)) : 0u);
   }
   group_sync(bar_id);
   uint32_t* kw = reinterpret_cast<uint32_t*>(kout);
@@ -91,17 +100,16 @@ __device__ void quantize_window(const WriteParams& p, int b, int h, int w, int L
 
   // ---- issue every raw-key load of the window first (one memory round trip),
   // and prefetch the value basis of the first new token into L2 so that the
-  // value rotation below reads it from L2
-  constexpr int kPerWarp = kWindow / (kWriteThreads / 32);
-  uint2 raws[kPerWarp];
+  // value rotation below reads it from L2. Four threads per token: thread
+  // (i = tid / 4, q = tid % 4) holds channels 32 q .. 32 q + 31 of token i.
+  const int ti = tid >> 2, tq = tid & 3;
+  uint4 raw[4] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u),
+                  make_uint4(0u, 0u, 0u, 0u)};
+  if (ti < nvalid) {
+    const int pos = p0 + ti;
+    const __half* src = (pos < L0 ? tail + ti * kHeadDim : knew + (size_t)(pos - L0) * kHeadDim) + 32 * tq;
 #pragma unroll
-  for (int k = 0; k < kPerWarp; ++k) {
-    const int i = warp + (kWriteThreads / 32) * k;
-    if (i < nvalid) {
-      const int pos = p0 + i;
-      const __half* src = pos < L0 ? tail + i * kHeadDim : knew + (size_t)(pos - L0) * kHeadDim;
-      raws[k] = *reinterpret_cast<const uint2*>(src + 4 * lane);
-    }
+    for (int j = 0; j < 4; ++j) raw[j] = reinterpret_cast<const uint4*>(src)[j];
   }
   if (!(p.tc_values && p0 >= L0 && nvalid == kWindow)) {
     int m0 = mnew[p0 + inew0 - L0];
@@ -111,34 +119,76 @@ __device__ void quantize_window(const WriteParams& p, int b, int h, int w, int L
     for (int q = 0; q < 4; ++q) asm volatile("prefetch.global.L2 [%0];" ::"l"(U + 32 * q));
   }
 
-  // ---- keys: rotate every valid token of the window -------------------------
-  float sg[4];
-#pragma unroll
-  for (int r = 0; r < 4; ++r) sg[r] = p.key_signs[4 * lane + r];
-#pragma unroll
-  for (int k = 0; k < kPerWarp; ++k) {
-    const int i = warp + (kWriteThreads / 32) * k;
-    if (i >= nvalid) break;
-    const int pos = p0 + i;
-    const uint2 raw = raws[k];
+  // ---- keys: rotate every valid token of the window: sign flip, butterflies
+  // h = 1 .. 16 inside the thread's 32 channels, h = 32 and 64 with the threads
+  // of the same token holding channels c + h (the lower index of a pair becomes
+  // a + b, the upper a - b, as in the scalar order), then the scale 2^-3.5.
+  if (ti < nvalid) {
+    const int pos = p0 + ti;
     // the tail keeps the new raw keys of a window left partial (see tail_any)
-    if (nvalid < kWindow && pos >= L0 && (tail_any || w == L0 / kWindow))
-      *reinterpret_cast<uint2*>(tail + i * kHeadDim + 4 * lane) = raw;
-    const __half2 lo = *reinterpret_cast<const __half2*>(&raw.x);
-    const __half2 hi = *reinterpret_cast<const __half2*>(&raw.y);
-    float x[4] = {__low2float(lo), __high2float(lo), __low2float(hi), __high2float(hi)};
-    warp_hadamard_rotate(x, sg);
-    *reinterpret_cast<float4*>(&kp[i][4 * lane]) = make_float4(x[0], x[1], x[2], x[3]);
+    if (nvalid < kWindow && pos >= L0 && (tail_any || w == L0 / kWindow)) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) reinterpret_cast<uint4*>(tail + ti * kHeadDim + 32 * tq)[j] = raw[j];
+    }
+  }
+  {
+    float x[32];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const __half2* hp = reinterpret_cast<const __half2*>(&raw[j]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __half22float2(hp[e]);
+        x[8 * j + 2 * e] = f.x;
+        x[8 * j + 2 * e + 1] = f.y;
+      }
+    }
+    const float4* sgn = reinterpret_cast<const float4*>(p.key_signs + 32 * tq);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float4 g = sgn[j];
+      x[4 * j] = __fmul_rn(x[4 * j], g.x);
+      x[4 * j + 1] = __fmul_rn(x[4 * j + 1], g.y);
+      x[4 * j + 2] = __fmul_rn(x[4 * j + 2], g.z);
+      x[4 * j + 3] = __fmul_rn(x[4 * j + 3], g.w);
+    }
+#pragma unroll
+    for (int hh = 1; hh < 32; hh <<= 1)
+#pragma unroll
+      for (int c = 0; c < 32; ++c)
+        if (!(c & hh)) {
+          const float a = x[c], b = x[c + hh];
+          x[c] = __fadd_rn(a, b);
+          x[c + hh] = __fsub_rn(a, b);
+        }
+#pragma unroll
+    for (int d = 1; d <= 2; d <<= 1) {  // h = 32 (partner q ^ 1), h = 64 (partner q ^ 2)
+      const bool upper = (tq & d) != 0;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const float other = __shfl_xor_sync(0xffffffffu, x[c], d);
+        x[c] = upper ? __fsub_rn(other, x[c]) : __fadd_rn(x[c], other);
+      }
+    }
+    const float sc = inv_sqrt_d();
+    if (ti < nvalid) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        *reinterpret_cast<float4*>(&kp[ti][kp_col(ti, 32 * tq + 4 * j)]) =
+            make_float4(__fmul_rn(x[4 * j], sc), __fmul_rn(x[4 * j + 1], sc), __fmul_rn(x[4 * j + 2], sc),
+                        __fmul_rn(x[4 * j + 3], sc));
+    }
   }
   group_sync(bar_id);
 
   // ---- window range per channel -> fp16 metadata -----------------------------
   {
     const int c = tid;
-    float mn = kp[0][c], mx = kp[0][c];
+    float mn = kp[0][kp_col(0, c)], mx = mn;
     for (int i = 1; i < nvalid; ++i) {
-      mn = fminf(mn, kp[i][c]);
-      mx = fmaxf(mx, kp[i][c]);
+      const float v = kp[i][kp_col(i, c)];
+      mn = fminf(mn, v);
+      mx = fmaxf(mx, v);
     }
     const __half m16 = __float2half_rn(mn);
     const __half s16 = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), kspan));
