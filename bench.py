@@ -188,13 +188,13 @@ class Workload:
         self.k = torch.stack(ks, 1).contiguous()
         self.v = torch.stack(vs, 1).contiguous()
         self.mod = torch.stack(ms, 1).contiguous()
-        self.S = max(1, m.omnikv_default_splits(self.consts[0].struct, self.caches[0].struct))
+        self.S, self.fused = m.omnikv_step_splits(self.consts[0].struct, self.caches[0].struct, 0)
         # the step's default split count grows (slightly) with the context: size
         # the partials for its value at the longest context of the run
         c0 = self.caches[0].struct
         saved = c0.max_seq_len
-        c0.max_seq_len = int(self.lengths.max()) + total_steps
-        s_max = max(self.S, m.omnikv_default_splits(self.consts[0].struct, c0))
+        c0.max_seq_len = int(self.lengths.max()) + total_steps - 1
+        s_max = max(self.S, m.omnikv_step_splits(self.consts[0].struct, c0, 0)[0])
         c0.max_seq_len = saved
         self.part = m.partials_tensor(spec.batch, spec.num_q_heads, s_max, device)
         self.out = torch.empty(spec.layers, spec.batch, spec.num_q_heads, 128, dtype=torch.float32,
@@ -202,36 +202,41 @@ class Workload:
 
     def step_calls(self, s, q, k, v, mod, stream, dec_events=None):
         """The C-ABI calls of one decode step over all layers: omnikv_decode_step
-        per layer (append + decode in one launch, then the combine launch). With
-        `dec_events` (a start/end pair), layer s % layers instead makes the same
-        step as three calls (write, decode, combine; identical results) with the
-        decode launch between the two events, so the decode kernel is timed in
-        place once per step."""
+        per layer (the append-and-decode launch, then the combine launch). With
+        `dec_events` (a start/end pair), layer s % layers makes the same step as
+        its two calls, omnikv_append_decode between the events, so the dominant
+        kernel (decode_step_kernel) is timed in place once per step."""
         m = self.m
         n = self.spec.layers
         for layer in range(n):
             c, cache = self.consts[layer].struct, self.caches[layer].struct
             if dec_events is not None and layer == s % n:
-                m.omnikv_write_cache(c, cache, k[layer], v[layer], mod[layer], 1, stream)
                 dec_events[0].record(stream)
-                m.omnikv_decode_attention(c, cache, q[layer], self.part, self.S, stream)
+                m.omnikv_append_decode(c, cache, q[layer], k[layer], v[layer], mod[layer], self.part, 0, stream)
                 dec_events[1].record(stream)
-                m.omnikv_combine(c, cache, self.part, self.S, self.out[layer], stream)
+                m.omnikv_combine_step(c, cache, self.part, 0, self.out[layer], stream)
             else:
                 m.omnikv_decode_step(c, cache, q[layer], k[layer], v[layer], mod[layer], self.part, 0,
                                      self.out[layer], stream)
 
     def launches_per_step(self, instrumented):
-        """Library kernel launches in one step: 2 per layer (decode step +
-        combine), 3 in the instrumented layer (append + decode + combine)."""
-        return 2 * self.spec.layers + (1 if instrumented else 0)
+        """Library kernel launches in one step: 2 per layer (the append-and-decode
+        launch and the combine launch) when the step's grid is resident at once,
+        else 4 (append, decode, combine; the append is one launch for a token)."""
+        return (2 if self.fused else 3) * self.spec.layers
 
     def decode_bytes(self, s):
-        """Algorithmic bytes one decode launch reads at step s (per layer): packed
-        records per token and kv head, plus one modality byte per token."""
+        """Algorithmic bytes of one append-and-decode launch at step s (one
+        layer): the packed records of every cached token and kv head after the
+        append, 1 modality id per token, and the append itself per kv head (the
+        new fp16 key and value read, the raw keys of the partial window read from
+        the tail, the window record written)."""
         sp = self.spec
-        T = (self.lengths.astype(np.int64) + s + 1).sum()
-        return int(T * sp.num_kv_heads * BYTES_PER_TOKEN_HEAD[(sp.key_bits, sp.value_bits)] + T)
+        L = self.lengths.astype(np.int64) + s
+        T = (L + 1).sum()
+        rec = BYTES_PER_TOKEN_HEAD[(sp.key_bits, sp.value_bits)] * 32
+        append = sp.num_kv_heads * int((512 + 256 * (L % 32) + rec).sum())
+        return int(T * sp.num_kv_heads * BYTES_PER_TOKEN_HEAD[(sp.key_bits, sp.value_bits)] + T + append)
 
 
 def run_gpu(args):
@@ -358,7 +363,9 @@ def run_gpu(args):
                        else "eager"},
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": None,
-                         "peak_source": peak_kind, "kernel": "decode_split_k",
+                         "peak_source": peak_kind,
+                         "kernel": "decode_step_kernel (append + decode launch)" if wl.fused
+                         else "kv_append_kernel + decode_split_k launches",
                          "avg_launch_us": round(avg_dec_s * 1e6, 3),
                          "bytes_per_launch": int(np.mean(dec_bytes))},
             "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": h2d,

@@ -29,6 +29,7 @@ EXPORTED = (
     "omnikv_write_cache", "omnikv_decode_attention", "omnikv_combine",
     "omnikv_status_string", "omnikv_abi_version", "omnikv_decode_static",
     "omnikv_dense_partials_bytes", "omnikv_dense_decode_bf16", "omnikv_decode_step",
+    "omnikv_append_decode", "omnikv_combine_step", "omnikv_step_splits",
 )
 OMNIKV_DECODE_STATIC_SCRATCH_BYTES = 8 << 20
 
@@ -96,6 +97,12 @@ def load() -> ctypes.CDLL:
     lib.omnikv_dense_decode_bf16.restype = ctypes.c_int
     lib.omnikv_decode_step.argtypes = [cfgp, cachep, P, P, P, P, P, I32, P, P]
     lib.omnikv_decode_step.restype = ctypes.c_int
+    lib.omnikv_step_splits.argtypes = [cfgp, cachep, I32, ctypes.POINTER(I32)]
+    lib.omnikv_step_splits.restype = I32
+    lib.omnikv_append_decode.argtypes = [cfgp, cachep, P, P, P, P, P, I32, P]
+    lib.omnikv_append_decode.restype = ctypes.c_int
+    lib.omnikv_combine_step.argtypes = [cfgp, cachep, P, I32, P, P]
+    lib.omnikv_combine_step.restype = ctypes.c_int
     lib.omnikv_decode_static.argtypes = [cfgp, cachep, P, P, I32, P]
     lib.omnikv_decode_static.restype = ctypes.c_int
     lib.omnikv_status_string.argtypes, lib.omnikv_status_string.restype = [ctypes.c_int], ctypes.c_char_p
@@ -176,6 +183,28 @@ def omnikv_decode_step(cfg: OmniKVConfig, cache: OmniKVCache, q, k_new, v_new, m
     st = load().omnikv_decode_step(ctypes.byref(cfg), ctypes.byref(cache), _ptr(q), _ptr(k_new), _ptr(v_new),
                                    _ptr(modality_new), _ptr(partials), int(num_splits), _ptr(out), _stream(stream))
     _check(st, "omnikv_decode_step")
+
+
+def omnikv_step_splits(cfg: OmniKVConfig, cache: OmniKVCache, num_splits: int = 0):
+    """(split count, fused) of the next decode step; see include/omnikv.h."""
+    f = ctypes.c_int32(0)
+    S = int(load().omnikv_step_splits(ctypes.byref(cfg), ctypes.byref(cache), int(num_splits), ctypes.byref(f)))
+    return S, bool(f.value)
+
+
+def omnikv_append_decode(cfg: OmniKVConfig, cache: OmniKVCache, q, k_new, v_new, modality_new, partials,
+                         num_splits: int, stream=None) -> None:
+    """First launch of omnikv_decode_step (append + decode into the partials)."""
+    st = load().omnikv_append_decode(ctypes.byref(cfg), ctypes.byref(cache), _ptr(q), _ptr(k_new), _ptr(v_new),
+                                     _ptr(modality_new), _ptr(partials), int(num_splits), _stream(stream))
+    _check(st, "omnikv_append_decode")
+
+
+def omnikv_combine_step(cfg: OmniKVConfig, cache: OmniKVCache, partials, num_splits: int, out, stream=None) -> None:
+    """Second launch of omnikv_decode_step (combine + length advance)."""
+    st = load().omnikv_combine_step(ctypes.byref(cfg), ctypes.byref(cache), _ptr(partials), int(num_splits),
+                                    _ptr(out), _stream(stream))
+    _check(st, "omnikv_combine_step")
 
 
 def omnikv_decode_static(cfg: OmniKVConfig, cache: OmniKVCache, q, out, num_splits: int = 0, stream=None) -> None:

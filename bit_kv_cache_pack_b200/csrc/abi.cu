@@ -205,34 +205,61 @@ omnikv_status omnikv_combine(const omnikv_config* cfg, const omnikv_cache* cache
   return OMNIKV_OK;
 }
 
-omnikv_status omnikv_decode_step(const omnikv_config* cfg, omnikv_cache* cache, const void* q, const void* k_new,
-                                 const void* v_new, const uint8_t* modality_new, void* partials, int32_t num_splits,
-                                 float* out, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The split count of a decode step and whether its append runs inside the decode
+// launch, for the cache as the step sees it (max_seq_len already counting the
+// appended token). Fused only when every CTA of that launch is resident at once,
+// so a waiting warp never waits on an unscheduled CTA; with num_splits = 0 the
+// default is lowered (by at most half) to make it so.
+void plan_step(const omnikv_config* cfg, const omnikv_cache* after, int32_t num_splits, int32_t* S, bool* fused) {
+  const long long units = (long long)after->batch * cfg->num_kv_heads;
+  const long long resident = (long long)decode_ctas_per_sm() * sm_count();
+  *S = resolve_splits(cfg, after, num_splits);
+  *fused = units * (1 + (long long)*S) <= resident;
+  if (!*fused && num_splits == 0) {
+    const long long s_res = resident / units - 1;
+    if (s_res >= 1 && 2 * s_res >= *S) {
+      *S = (int32_t)s_res;
+      *fused = true;
+    }
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t omnikv_step_splits(const omnikv_config* cfg, const omnikv_cache* cache, int32_t num_splits, int32_t* fused) {
+  if (check_config(cfg) != OMNIKV_OK || check_cache(cache) != OMNIKV_OK || num_splits < 0) return 0;
+  omnikv_cache after = *cache;
+  after.max_seq_len = cache->max_seq_len < cache->cap_tokens ? cache->max_seq_len + 1 : cache->max_seq_len;
+  int32_t S;
+  bool f;
+  plan_step(cfg, &after, num_splits, &S, &f);
+  if (fused) *fused = f ? 1 : 0;
+  return S;
+}
+
+omnikv_status omnikv_append_decode(const omnikv_config* cfg, omnikv_cache* cache, const void* q, const void* k_new,
+                                   const void* v_new, const uint8_t* modality_new, void* partials,
+                                   int32_t num_splits, void* stream) {
   omnikv_status st = check_config(cfg);
   if (st != OMNIKV_OK) return st;
   if ((st = check_cache(cache)) != OMNIKV_OK) return st;
-  if (!cache->step_flags || !q || !k_new || !v_new || !modality_new || !partials || !out) return OMNIKV_ERR_INVALID_ARG;
+  if (!cache->step_flags || !q || !k_new || !v_new || !modality_new || !partials || num_splits < 0)
+    return OMNIKV_ERR_INVALID_ARG;
   if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(cache->step_flags, 4)) return OMNIKV_ERR_INVALID_ARG;
   if ((long long)cache->max_seq_len + 1 > cache->cap_tokens) return OMNIKV_ERR_CAPACITY;
-  omnikv_cache after = *cache;  // the decode and combine see the appended token
+  omnikv_cache after = *cache;  // the decode sees the appended token
   after.max_seq_len += 1;
-  // fused (append CTAs inside the decode launch) only when every CTA of that
-  // launch is resident at once, so a waiting warp never waits on an unscheduled CTA
-  const long long units = (long long)cache->batch * cfg->num_kv_heads;
-  const long long resident = (long long)decode_ctas_per_sm() * sm_count();
-  int32_t S = resolve_splits(cfg, &after, num_splits);
-  bool fused = units * (1 + (long long)S) <= resident;
-  if (!fused && num_splits == 0) {
-    const long long s_res = resident / units - 1;
-    if (s_res >= 1 && 2 * s_res >= S) {
-      S = (int32_t)s_res;
-      fused = true;
-    }
-  }
+  int32_t S;
+  bool fused;
+  plan_step(cfg, &after, num_splits, &S, &fused);
   DecodeParams dp;
   if ((st = prepare_decode(cfg, &after, q, partials, S, &dp)) != OMNIKV_OK) return st;
-  CombineParams cp;
-  if ((st = prepare_combine(cfg, &after, partials, S, out, &cp)) != OMNIKV_OK) return st;
   WriteParams wp;
   fill_write_params(cfg, cache, k_new, v_new, modality_new, 1, &wp);
   wp.step_flags = cache->step_flags;
@@ -240,15 +267,38 @@ omnikv_status omnikv_decode_step(const omnikv_config* cfg, omnikv_cache* cache, 
   if (fused) {
     dp.len_add = 1;
     dp.step_flags = cache->step_flags;
-    cp.len_add = 1;
     if (launch_decode_step(dp, wp, s) != cudaSuccess) return OMNIKV_ERR_CUDA;
   } else {
     if (launch_write(wp, cache->batch, s) != cudaSuccess) return OMNIKV_ERR_CUDA;
     if (launch_decode(dp, cache->batch, s) != cudaSuccess) return OMNIKV_ERR_CUDA;
   }
-  if (launch_combine(cp, cache->batch, s) != cudaSuccess) return OMNIKV_ERR_CUDA;
   cache->max_seq_len += 1;
   return OMNIKV_OK;
+}
+
+omnikv_status omnikv_combine_step(const omnikv_config* cfg, omnikv_cache* cache, const void* partials,
+                                  int32_t num_splits, float* out, void* stream) {
+  omnikv_status st = check_config(cfg);
+  if (st != OMNIKV_OK) return st;
+  if ((st = check_cache(cache)) != OMNIKV_OK) return st;
+  if (!partials || !out || num_splits < 0) return OMNIKV_ERR_INVALID_ARG;
+  int32_t S;
+  bool fused;
+  plan_step(cfg, cache, num_splits, &S, &fused);  // the same plan as omnikv_append_decode made
+  CombineParams cp;
+  if ((st = prepare_combine(cfg, cache, partials, S, out, &cp)) != OMNIKV_OK) return st;
+  cp.len_add = fused ? 1 : 0;  // the fused append leaves the length to this launch
+  if (launch_combine(cp, cache->batch, static_cast<cudaStream_t>(stream)) != cudaSuccess) return OMNIKV_ERR_CUDA;
+  return OMNIKV_OK;
+}
+
+omnikv_status omnikv_decode_step(const omnikv_config* cfg, omnikv_cache* cache, const void* q, const void* k_new,
+                                 const void* v_new, const uint8_t* modality_new, void* partials, int32_t num_splits,
+                                 float* out, void* stream) {
+  if (!out) return OMNIKV_ERR_INVALID_ARG;
+  omnikv_status st = omnikv_append_decode(cfg, cache, q, k_new, v_new, modality_new, partials, num_splits, stream);
+  if (st != OMNIKV_OK) return st;
+  return omnikv_combine_step(cfg, cache, partials, num_splits, out, stream);
 }
 
 size_t omnikv_dense_partials_bytes(int32_t batch, int32_t num_q_heads, int32_t num_splits) {

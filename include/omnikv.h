@@ -158,7 +158,8 @@ OMNIKV_API omnikv_status omnikv_write_cache(const omnikv_config* cfg, omnikv_cac
  *   q          : [batch][num_q_heads][128] fp16, 16-byte aligned
  *   partials   : device buffer of omnikv_partials_bytes(batch, num_q_heads, S) bytes, 16-byte aligned
  *   num_splits : 1 <= S <= 4096, or 0 for omnikv_default_splits(cfg, cache)
- * Empty splits write m = -inf, l = 0, acc = 0. */
+ * Empty splits write m = -inf and l = 0 only (their accumulators are not written; the combine gives
+ * them weight 0). */
 OMNIKV_API omnikv_status omnikv_decode_attention(const omnikv_config* cfg, const omnikv_cache* cache,
                                       const void* q, void* partials, int32_t num_splits, void* stream);
 
@@ -186,6 +187,24 @@ OMNIKV_API omnikv_status omnikv_combine(const omnikv_config* cfg, const omnikv_c
 OMNIKV_API omnikv_status omnikv_decode_step(const omnikv_config* cfg, omnikv_cache* cache, const void* q,
                                             const void* k_new, const void* v_new, const uint8_t* modality_new,
                                             void* partials, int32_t num_splits, float* out, void* stream);
+
+/* The split count the next omnikv_decode_step (or omnikv_append_decode) uses with this num_splits
+ * (0: default) for the cache as it is now (partials must hold that many splits), and in *fused whether
+ * its append runs inside the decode launch (1; 2 launches per step) or before it (0; 3 launches).
+ * Returns 0 on bad arguments. */
+OMNIKV_API int32_t omnikv_step_splits(const omnikv_config* cfg, const omnikv_cache* cache, int32_t num_splits,
+                                      int32_t* fused);
+
+/* The two launches of omnikv_decode_step as separate calls (omnikv_decode_step = this pair), e.g. to
+ * time them apart or to schedule other work between them. omnikv_append_decode appends the token and
+ * writes the split partials (arguments as above) and advances cache->max_seq_len by 1;
+ * omnikv_combine_step must follow it on the same stream with the same cache, partials and
+ * num_splits: it merges them into out and advances seq_lens where the append left that to it. */
+OMNIKV_API omnikv_status omnikv_append_decode(const omnikv_config* cfg, omnikv_cache* cache, const void* q,
+                                              const void* k_new, const void* v_new, const uint8_t* modality_new,
+                                              void* partials, int32_t num_splits, void* stream);
+OMNIKV_API omnikv_status omnikv_combine_step(const omnikv_config* cfg, omnikv_cache* cache, const void* partials,
+                                             int32_t num_splits, float* out, void* stream);
 
 /* Decode attention and combine in one call, with the split-K partials in a fixed device array of
  * OMNIKV_DECODE_STATIC_SCRATCH_BYTES owned by this library; the caller passes only inputs (q) and

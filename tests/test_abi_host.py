@@ -152,3 +152,18 @@ def test_decode_step_arguments_rejected():
     assert _step_status(_cfg(), _cache(), k=FAKE + 8) == _abi.OMNIKV_ERR_INVALID_ARG
     assert _step_status(_cfg(), _cache(max_seq_len=2048)) == _abi.OMNIKV_ERR_CAPACITY
     assert _step_status(_cfg(key_bits=3), _cache()) == _abi.OMNIKV_ERR_UNSUPPORTED
+
+
+def test_step_splits_and_two_phase_arguments_rejected():
+    lib = _abi.load()
+    f = ctypes.c_int32(7)
+    assert lib.omnikv_step_splits(ctypes.byref(_cfg(key_bits=3)), ctypes.byref(_cache()), 0, ctypes.byref(f)) == 0
+    assert lib.omnikv_step_splits(ctypes.byref(_cfg()), ctypes.byref(_cache()), -1, ctypes.byref(f)) == 0
+    cfg, cache = _cfg(), _cache(step_flags=None)
+    assert lib.omnikv_append_decode(ctypes.byref(cfg), ctypes.byref(cache), FAKE, FAKE, FAKE, FAKE, FAKE, 0, 0) == \
+        _abi.OMNIKV_ERR_INVALID_ARG
+    cache = _cache(max_seq_len=2048)
+    assert lib.omnikv_append_decode(ctypes.byref(cfg), ctypes.byref(cache), FAKE, FAKE, FAKE, FAKE, FAKE, 0, 0) == \
+        _abi.OMNIKV_ERR_CAPACITY
+    assert lib.omnikv_combine_step(ctypes.byref(cfg), ctypes.byref(_cache()), FAKE, 0, None, 0) == \
+        _abi.OMNIKV_ERR_INVALID_ARG

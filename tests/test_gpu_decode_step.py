@@ -80,7 +80,11 @@ def test_decode_step_matches_four_calls_and_oracle(cuda_device, hkv, G, lengths,
         mn = torch.tensor([(s + b) % 3 for b in range(B)], dtype=torch.uint8, device=dev)
         out_f = torch.full((B, Hq, 128), float("nan"), device=dev)
         out_p = torch.full((B, Hq, 128), float("nan"), device=dev)
-        m.omnikv_decode_step(consts.struct, fused.struct, q, kn, vn, mn, part_f, splits, out_f)
+        if s % 2:  # the same step as its two launches
+            m.omnikv_append_decode(consts.struct, fused.struct, q, kn, vn, mn, part_f, splits)
+            m.omnikv_combine_step(consts.struct, fused.struct, part_f, splits, out_f)
+        else:
+            m.omnikv_decode_step(consts.struct, fused.struct, q, kn, vn, mn, part_f, splits, out_f)
         m.omnikv_write_cache(consts.struct, plain.struct, kn, vn, mn, 1)
         Sp = splits or m.omnikv_default_splits(consts.struct, plain.struct)
         m.omnikv_decode_attention(consts.struct, plain.struct, q, part_p, Sp)
