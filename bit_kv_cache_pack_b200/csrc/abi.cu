@@ -55,7 +55,7 @@ int32_t resolve_splits(const omnikv_config* cfg, const omnikv_cache* c, int32_t 
   // second, partial wave would double the time), with at least 4 windows (one
   // per warp) per split
   const long long units = (long long)c->batch * cfg->num_kv_heads;
-  const long long target = (long long)decode_ctas_per_sm() * sm_count();
+  const long long target = (long long)decode_ctas_per_sm(cfg->key_bits, cfg->value_bits) * sm_count();
   long long s = target / units;
   const long long max_s = (nw + 3) / 4;
   if (s > max_s) s = max_s;
@@ -216,7 +216,7 @@ namespace {
 // default is lowered (by at most half) to make it so.
 void plan_step(const omnikv_config* cfg, const omnikv_cache* after, int32_t num_splits, int32_t* S, bool* fused) {
   const long long units = (long long)after->batch * cfg->num_kv_heads;
-  const long long resident = (long long)decode_ctas_per_sm() * sm_count();
+  const long long resident = (long long)decode_ctas_per_sm(cfg->key_bits, cfg->value_bits) * sm_count();
   *S = resolve_splits(cfg, after, num_splits);
   *fused = units * (1 + (long long)*S) <= resident;
   if (!*fused && num_splits == 0) {

@@ -171,119 +171,257 @@ __device__ __forceinline__ bool wait_flag(const int32_t* flag, int val, uint64_t
   return true;
 }
 
+// 2^x with the hardware approximation (relative error below 2^-22); -inf -> 0.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // ---------------------------------------------------------------------------
-// generic CUDA-core path: warp w owns query heads w and w + 4 of the group
+// CUDA-core path (4-bit codes, or a codebook that is not symmetric): the CTA
+// decodes the split's windows one at a time from a double-buffered ring of bulk
+// copies. Scores: four threads per token, thread q of token t holding channels
+// 4 j + q (j = 0..31), each dequantised once, k'_tc = m_c + s_c (c_code - c_0),
+// and used for the 8 query heads; two shuffles complete the dot products.
+// Values: thread c owns channel c and one fp32 accumulator per (modality, head).
 // ---------------------------------------------------------------------------
-__device__ void decode_generic(const DecodeParams& p, DecodeSmem& sm, int b, int kvh, int split) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+constexpr int kGenStages = 2;
+
+struct GenSmem {                 // laid over DecodeSmem::stage
+  uint8_t rec[kGenStages][4704];  // window record + 32 modality ids (largest record: 4672 B)
+  float qT[kHeadDim][kMaxGroup];  // rotated queries, channel-major
+  float pw[kWindow][kMaxGroup];   // p_ht * sigma_t of the current window
+  float dk[16], dv[16];           // c_j - c_0 (keys), c_j (values)
+  float wmax[kWarps][kMaxGroup];
+  uint64_t bar[kGenStages];
+};
+static_assert(sizeof(GenSmem) <= sizeof(DecodeSmem::stage), "generic path shared memory");
+
+__device__ __forceinline__ void gen_issue(const DecodeParams& p, GenSmem& g, int stage, const uint8_t* rec_base,
+                                          int rec_bytes, int b, int kvh, int wi, int wait_win, int wait_val) {
+  if (wi == wait_win &&
+      !wait_flag(p.step_flags + (size_t)b * p.num_kv_heads + kvh, wait_val, kWaitLimitNs))
+    set_error(p.error_word, OMNIKV_DEVERR_TIMEOUT);
+  mbar_arrive_expect_tx(&g.bar[stage], rec_bytes + kWindow);
+  bulk_copy_g2s(g.rec[stage], rec_base + (size_t)wi * rec_bytes, rec_bytes, &g.bar[stage]);
+  bulk_copy_g2s(g.rec[stage] + rec_bytes, p.modality + (size_t)b * p.cap_tokens + (size_t)wi * kWindow, kWindow,
+                &g.bar[stage]);
+}
+
+template <int KB, int VB>
+__device__ void decode_generic_t(const DecodeParams& p, DecodeSmem& sm, int b, int kvh, int split) {
+  GenSmem& g = *reinterpret_cast<GenSmem*>(&sm.stage[0][0][0]);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = p.group;
   const int Hq = p.num_kv_heads * G;
   int T, w0, w1;
   split_range(p, b, split, T, w0, w1);
-  const RecordLayout lay(p.key_bits, p.value_bits);
-  uint8_t* rec = &sm.stage[0][0][0];
-  uint8_t* mods = rec + 4672;
-  float* cbk = reinterpret_cast<float*>(rec + 4672 + 32);
-  float* cbv = cbk + 16;
-  if (threadIdx.x < (1 << p.key_bits)) cbk[threadIdx.x] = p.key_cb[threadIdx.x];
-  if (threadIdx.x < (1 << p.value_bits)) cbv[threadIdx.x] = p.val_cb[threadIdx.x];
-
-  const int kcpw = 32 / p.key_bits, kwpt = kHeadDim / kcpw;
-  const uint32_t kmask = (1u << p.key_bits) - 1u;
-  const int vcpw = 32 / p.value_bits;
-  const uint32_t vmask = (1u << p.value_bits) - 1u;
-
-  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.0f, 0.0f};
-  float acc[2][kMods][4];
-#pragma unroll
-  for (int k = 0; k < 2; ++k)
-#pragma unroll
-    for (int m = 0; m < kMods; ++m)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) acc[k][m][j] = 0.0f;
-
-  const uint8_t* rec_base = p.records + ((size_t)(b * p.num_kv_heads + kvh) * p.cap_windows) * lay.bytes;
   int wait_win, wait_val;
   step_window(p, b, wait_win, wait_val);
-  for (int w = w0; w < w1; ++w) {
-    if (w == wait_win && threadIdx.x == 0 &&
-        !wait_flag(p.step_flags + (size_t)b * p.num_kv_heads + kvh, wait_val, kWaitLimitNs))
-      set_error(p.error_word, OMNIKV_DEVERR_TIMEOUT);
-    __syncthreads();
-    {
-      const uint4* src = reinterpret_cast<const uint4*>(rec_base + (size_t)w * lay.bytes);
-      uint4* dst = reinterpret_cast<uint4*>(rec);
-      for (int i = threadIdx.x; i < lay.bytes / 16; i += blockDim.x) dst[i] = src[i];
-      if (threadIdx.x < 2)
-        reinterpret_cast<uint4*>(mods)[threadIdx.x] =
-            reinterpret_cast<const uint4*>(p.modality + (size_t)b * p.cap_tokens + w * kWindow)[threadIdx.x];
+  const RecordLayout lay(p.key_bits, p.value_bits);
+  const uint8_t* rec_base = p.records + ((size_t)(b * p.num_kv_heads + kvh) * p.cap_windows) * lay.bytes;
+  const int nwin = w1 - w0;
+  if (tid == 0) {
+    for (int s = 0; s < kGenStages; ++s) mbar_init(&g.bar[s], 1);
+    fence_barrier_init();
+    for (int s = 0; s < kGenStages && s < nwin; ++s) gen_issue(p, g, s, rec_base, lay.bytes, b, kvh, w0 + s, wait_win, wait_val);
+  }
+  const int LK = 1 << p.key_bits, LV = 1 << p.value_bits;
+  if (tid < LK) g.dk[tid] = p.key_cb[tid] - p.key_cb[0];
+  if (tid >= 32 && tid - 32 < LV) g.dv[tid - 32] = p.val_cb[tid - 32];
+#pragma unroll
+  for (int h = 0; h < kMaxGroup; ++h) g.qT[tid][h] = (&sm.q[0][0])[qpos(h, tid)];
+  __syncthreads();
+
+  // score threads: token t = tid / 4, channel phase q = tid % 4
+  const int st = tid >> 2, sq = tid & 3;
+  constexpr uint32_t kmask = (1u << KB) - 1u, vmask = (1u << VB) - 1u;
+  constexpr int kcpw = 32 / KB, kwpt = kHeadDim / kcpw, vcpw = 32 / VB;
+  float m_run[kMaxGroup], l_part[kMaxGroup];  // running max (CTA-uniform), per-thread partial sums of p
+  float acc[kMods][kMaxGroup];               // thread c = tid: channel c
+#pragma unroll
+  for (int h = 0; h < kMaxGroup; ++h) {
+    m_run[h] = -INFINITY;
+    l_part[h] = 0.0f;
+#pragma unroll
+    for (int m = 0; m < kMods; ++m) acc[m][h] = 0.0f;
+  }
+
+  int failed_at = -1;
+  for (int i = 0; i < nwin; ++i) {
+    const int s = i % kGenStages;
+    const int wi = w0 + i;
+    if (__syncthreads_or(!mbar_wait_bounded(&g.bar[s], (i / kGenStages) & 1, kWaitLimitNs))) {
+      failed_at = i;
+      break;
     }
-    __syncthreads();
-    const int nvalid = min(kWindow, T - w * kWindow);
+    const uint8_t* rec = g.rec[s];
     const uint32_t* kw = reinterpret_cast<const uint32_t*>(rec + lay.k_off);
     const __half2* meta = reinterpret_cast<const __half2*>(rec + lay.meta_off);
     const uint32_t* vw = reinterpret_cast<const uint32_t*>(rec + lay.v_off);
     const __half* sig = reinterpret_cast<const __half*>(rec + lay.sigma_off);
-    const float c0 = cbk[0];
-    // scores: lane = token; both heads of this warp share the dequantised key
-    float sc[2] = {0.0f, 0.0f};
-    for (int c = 0; c < kHeadDim; ++c) {
-      const uint32_t code = (kw[lane * kwpt + c / kcpw] >> (p.key_bits * (c % kcpw))) & kmask;
-      const float2 ms = __half22float2(meta[c]);
-      const float kval = ms.x + ms.y * (cbk[code] - c0);
-      sc[0] = fmaf((&sm.q[0][0])[qpos(warp, c)], kval, sc[0]);
-      sc[1] = fmaf((&sm.q[0][0])[qpos(warp + kWarps, c)], kval, sc[1]);
-    }
-    float pt[2];
+    const uint8_t* mods = rec + lay.bytes;
+
+    // ---- scores of token st for the 8 heads over channels 4 j + sq
+    float sc[kMaxGroup];
 #pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      if (lane >= nvalid) sc[k] = -INFINITY;
-      const float m_new = fmaxf(m_run[k], warp_max(sc[k]));
-      const float alpha = expf(m_run[k] - m_new);
-      pt[k] = lane < nvalid ? expf(sc[k] - m_new) : 0.0f;
-      l_run[k] = l_run[k] * alpha + warp_sum(pt[k]);
+    for (int h = 0; h < kMaxGroup; ++h) sc[h] = 0.0f;
+    {
+      uint32_t row[kwpt];  // this token's key words (every channel 4 j + sq of word j * 4 / kcpw)
+#pragma unroll
+      for (int k4 = 0; k4 < kwpt / 4; ++k4) {
+        const uint4 u = reinterpret_cast<const uint4*>(kw + st * kwpt)[k4];
+        row[4 * k4] = u.x;
+        row[4 * k4 + 1] = u.y;
+        row[4 * k4 + 2] = u.z;
+        row[4 * k4 + 3] = u.w;
+      }
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int c = 4 * j + sq;
+        const uint32_t code = (row[(4 * j) / kcpw] >> (KB * (c % kcpw))) & kmask;
+        const float2 ms = __half22float2(meta[c]);
+        const float kv = fmaf(ms.y, g.dk[code], ms.x);
+        const float4 qa = *reinterpret_cast<const float4*>(&g.qT[c][0]);
+        const float4 qb = *reinterpret_cast<const float4*>(&g.qT[c][4]);
+        sc[0] = fmaf(qa.x, kv, sc[0]);
+        sc[1] = fmaf(qa.y, kv, sc[1]);
+        sc[2] = fmaf(qa.z, kv, sc[2]);
+        sc[3] = fmaf(qa.w, kv, sc[3]);
+        sc[4] = fmaf(qb.x, kv, sc[4]);
+        sc[5] = fmaf(qb.y, kv, sc[5]);
+        sc[6] = fmaf(qb.z, kv, sc[6]);
+        sc[7] = fmaf(qb.w, kv, sc[7]);
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; ++h) {
+      sc[h] += __shfl_xor_sync(0xffffffffu, sc[h], 1);
+      sc[h] += __shfl_xor_sync(0xffffffffu, sc[h], 2);
+      if (wi * kWindow + st >= T || h >= G) sc[h] = -INFINITY;
+    }
+    // ---- window max per head: lanes of a warp (8 tokens), then the 4 warps
+    float mx[kMaxGroup];
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; ++h) {
+      float v = sc[h];
+      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+      mx[h] = v;
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int h = 0; h < kMaxGroup; ++h) g.wmax[warp][h] = mx[h];
+    }
+    __syncthreads();
+    float alpha[kMaxGroup];
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; ++h) {
+      float v = fmaxf(fmaxf(g.wmax[0][h], g.wmax[1][h]), fmaxf(g.wmax[2][h], g.wmax[3][h]));
+      const float mn = fmaxf(m_run[h], v);
+      alpha[h] = (mn == -INFINITY) ? 1.0f : fast_exp2((m_run[h] - mn) * kLog2e);
+      m_run[h] = mn;
+    }
+    // ---- p = exp(score - max); thread (st, sq) stores heads 2 sq, 2 sq + 1 of token st
+    {
+      const float sgm = __half2float(sig[st]);
+#pragma unroll
+      for (int h = 0; h < kMaxGroup; ++h) {
+        const float pp = (sc[h] == -INFINITY) ? 0.0f : fast_exp2((sc[h] - m_run[h]) * kLog2e);
+        l_part[h] = l_part[h] * alpha[h] + (sq == 0 ? pp : 0.0f);
+        if ((h >> 1) == sq) g.pw[st][h] = pp * sgm;
+      }
+    }
+    __syncthreads();
+    // ---- values: channel c = tid over the window's valid tokens
+    {
 #pragma unroll
       for (int m = 0; m < kMods; ++m)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[k][m][j] *= alpha;
-      m_run[k] = m_new;
-    }
-    for (int t = 0; t < nvalid; ++t) {
-      const float s = __half2float(sig[t]);
-      const float wt0 = __shfl_sync(0xffffffffu, pt[0], t) * s;
-      const float wt1 = __shfl_sync(0xffffffffu, pt[1], t) * s;
-      const int mod = mods[t];
-      const uint32_t* vrow = vw + (t / vcpw) * kHeadDim;
-      const int sh = p.value_bits * (t % vcpw);
-      float val[4];
+        for (int h = 0; h < kMaxGroup; ++h) acc[m][h] *= alpha[h];
+      const int nvalid = min(kWindow, T - wi * kWindow);
+      for (int t = 0; t < nvalid; ++t) {
+        const uint32_t code = (vw[(t / vcpw) * kHeadDim + tid] >> (VB * (t % vcpw))) & vmask;
+        const float d = g.dv[code];
+        const float4 pa = *reinterpret_cast<const float4*>(&g.pw[t][0]);
+        const float4 pb = *reinterpret_cast<const float4*>(&g.pw[t][4]);
+        const int mod = min((int)mods[t], kMods - 1);  // the same for every thread
 #pragma unroll
-      for (int j = 0; j < 4; ++j) val[j] = cbv[(vrow[lane + 32 * j] >> sh) & vmask];
-#pragma unroll
-      for (int m = 0; m < kMods; ++m) {
-        if (mod == m || (m == kMods - 1 && mod > m)) {
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            acc[0][m][j] = fmaf(wt0, val[j], acc[0][m][j]);
-            acc[1][m][j] = fmaf(wt1, val[j], acc[1][m][j]);
-          }
+        for (int m = 0; m < kMods; ++m) {
+          if (mod != m) continue;
+          acc[m][0] = fmaf(pa.x, d, acc[m][0]);
+          acc[m][1] = fmaf(pa.y, d, acc[m][1]);
+          acc[m][2] = fmaf(pa.z, d, acc[m][2]);
+          acc[m][3] = fmaf(pa.w, d, acc[m][3]);
+          acc[m][4] = fmaf(pb.x, d, acc[m][4]);
+          acc[m][5] = fmaf(pb.y, d, acc[m][5]);
+          acc[m][6] = fmaf(pb.z, d, acc[m][6]);
+          acc[m][7] = fmaf(pb.w, d, acc[m][7]);
         }
       }
     }
-  }
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const int g = warp + kWarps * k;
-    if (g >= G) continue;
-    Partial* out = p.partials + ((size_t)b * Hq + kvh * G + g) * p.num_splits + split;
-#pragma unroll
-    for (int m = 0; m < kMods; ++m)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) out->acc[m][lane + 32 * j] = acc[k][m][j];
-    if (lane == 0) {
-      out->m = m_run[k];
-      out->l = l_run[k];
+    __syncthreads();  // stage s and pw are free again
+    if (tid == 0 && i + kGenStages < nwin) {
+      fence_proxy_async_smem();
+      gen_issue(p, g, s, rec_base, lay.bytes, b, kvh, w0 + i + kGenStages, wait_win, wait_val);
     }
   }
+  if (failed_at >= 0) {
+    if (tid == 0) set_error(p.error_word, OMNIKV_DEVERR_TIMEOUT);
+    // the copies still in flight (windows failed_at, failed_at + 1) land before
+    // this CTA's shared memory is released
+    for (int j = failed_at; j < nwin && j < failed_at + kGenStages; ++j)
+      mbar_wait_bounded(&g.bar[j % kGenStages], (j / kGenStages) & 1, kWaitLimitNs);
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; ++h) {
+      m_run[h] = -INFINITY;
+      l_part[h] = 0.0f;
+#pragma unroll
+      for (int m = 0; m < kMods; ++m) acc[m][h] = 0.0f;
+    }
+  }
+
+  // ---- l per head: thread sums over the tokens it owns (sq == 0), CTA reduction
+  {
+#pragma unroll
+    for (int h = 0; h < kMaxGroup; ++h) {
+      float v = l_part[h];
+      v += __shfl_xor_sync(0xffffffffu, v, 4);
+      v += __shfl_xor_sync(0xffffffffu, v, 8);
+      v += __shfl_xor_sync(0xffffffffu, v, 16);
+      l_part[h] = v;
+    }
+    __syncthreads();
+    if (lane == 0) {
+#pragma unroll
+      for (int h = 0; h < kMaxGroup; ++h) g.wmax[warp][h] = l_part[h];
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int h = 0; h < kMaxGroup; ++h) {
+    if (h >= G) continue;
+    Partial* out = p.partials + ((size_t)b * Hq + kvh * G + h) * p.num_splits + split;
+#pragma unroll
+    for (int m = 0; m < kMods; ++m) out->acc[m][tid] = acc[m][h];
+    if (tid == 0) {
+      out->m = m_run[h];
+      out->l = g.wmax[0][h] + g.wmax[1][h] + g.wmax[2][h] + g.wmax[3][h];
+    }
+  }
+}
+
+__device__ void decode_generic(const DecodeParams& p, DecodeSmem& sm, int b, int kvh, int split) {
+  if (p.key_bits == 2 && p.value_bits == 2)
+    decode_generic_t<2, 2>(p, sm, b, kvh, split);
+  else if (p.key_bits == 2)
+    decode_generic_t<2, 4>(p, sm, b, kvh, split);
+  else if (p.value_bits == 2)
+    decode_generic_t<4, 2>(p, sm, b, kvh, split);
+  else
+    decode_generic_t<4, 4>(p, sm, b, kvh, split);
 }
 
 // ---------------------------------------------------------------------------
@@ -298,12 +436,6 @@ constexpr uint32_t kPlane1 = 0x40004000u;  // bit 14 of each half: 2
 
 __device__ __forceinline__ uint32_t rotl(uint32_t x, int n) { return __funnelshift_l(x, x, n); }
 
-// 2^x with the hardware approximation (relative error below 2^-22); -inf -> 0.
-__device__ __forceinline__ float fast_exp2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
 
 // (lo, hi) -> fp16 pair h = fp16(x) and l = fp16(x - h), each transposed to the
 // B-fragment layout with movmatrix.
@@ -784,14 +916,18 @@ __device__ __forceinline__ void build_score_operand(DecodeSmem& sm, float k0scal
   }
 }
 
-// One decode CTA: split `split` of kv head kvh of sequence b.
+// One decode CTA: split `split` of kv head kvh of sequence b. kGen: the build of
+// the kernel that serves 4-bit caches (CUDA-core path only, no TMEM, more CTAs
+// per SM); otherwise the tensor-core path, with the CUDA-core path for 2-bit
+// codebooks that are not symmetric.
+template <bool kGen>
 __device__ __forceinline__ void decode_cta(const DecodeParams& p, DecodeSmem& sm, int b, int kvh, int split) {
   // ---- independent of the cache (overlaps the previous launch of the stream):
   // query rotation, score operand, L2 prefetch of this split's share of the
   // value bases (read by the combine)
   bool fast = false;
   float k0 = 0.f, k1 = 0.f, k2 = 0.f, v0 = 0.f, v1 = 0.f, v2 = 0.f;
-  if (p.key_bits == 2 && p.value_bits == 2) {
+  if (!kGen && p.key_bits == 2 && p.value_bits == 2) {
     k0 = p.key_cb[0], k1 = p.key_cb[1], k2 = p.key_cb[2];
     const float k3 = p.key_cb[3];
     v0 = p.val_cb[0], v1 = p.val_cb[1], v2 = p.val_cb[2];
@@ -822,7 +958,7 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, DecodeSmem& sm
     }
     return;
   }
-  if (fast) {
+  if (!kGen && fast) {
     prime_pipeline(p, sm, b, kvh, w0, w1);
     if (threadIdx.x < 32) tmem_alloc(&sm.tmem_base, kTmemCols);
     tc_fence_before();
@@ -839,17 +975,23 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, DecodeSmem& sm
   decode_generic(p, sm, b, kvh, split);
 }
 
-__global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_split_k_kernel(const DecodeParams p) {
+constexpr int kGenCtasPerSm = 4;  // the 4-bit build: registers for 4 resident CTAs
+
+template <bool kGen>
+__global__ void __launch_bounds__(kThreads, kGen ? kGenCtasPerSm : kCtasPerSm)
+    decode_split_k_kernel(const DecodeParams p) {
   __shared__ DecodeSmem sm;
   griddep_launch_dependents();
-  decode_cta(p, sm, blockIdx.z, blockIdx.y, blockIdx.x);
+  decode_cta<kGen>(p, sm, blockIdx.z, blockIdx.y, blockIdx.x);
 }
 
 // Decode step: CTAs [0, batch * H) append one token to (sequence, kv head) and
 // then publish the new length in the step flag; the others are decode CTAs
 // (split fastest, then kv head, then sequence). Only the warp decoding the
 // window that receives the token waits for the flag, before copying it.
-__global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_step_kernel(const DecodeParams p, const WriteParams w) {
+template <bool kGen>
+__global__ void __launch_bounds__(kThreads, kGen ? kGenCtasPerSm : kCtasPerSm)
+    decode_step_kernel(const DecodeParams p, const WriteParams w) {
   __shared__ DecodeSmem sm;
   static_assert(sizeof(WindowSmem) <= sizeof(DecodeSmem), "append uses the decode shared memory");
   griddep_launch_dependents();
@@ -877,87 +1019,90 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_step_kernel(const
     return;
   }
   const int r = blockIdx.x - nappend;
-  decode_cta(p, sm, r / (p.num_splits * H), (r / p.num_splits) % H, r % p.num_splits);
+  decode_cta<kGen>(p, sm, r / (p.num_splits * H), (r / p.num_splits) % H, r % p.num_splits);
 }
 
 // Several decode CTAs share an SM only if the SM's unified L1 / shared memory is
 // split in favour of shared memory; without a preference the runtime may pick a
-// split that holds one CTA. Set once per device (bit d of the mask).
-std::atomic<uint64_t> g_carveout_set{0};
-
-cudaError_t prefer_shared_carveout() {
+// split that holds one CTA. Set once per device and kernel (bit d of a mask).
+template <typename Kernel>
+cudaError_t prefer_shared_carveout(Kernel kernel, std::atomic<uint64_t>& done) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   const uint64_t bit = dev < 64 ? (1ull << dev) : 0ull;
-  if (bit && (g_carveout_set.load(std::memory_order_acquire) & bit)) return cudaSuccess;
-  e = cudaFuncSetAttribute(decode_split_k_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                           cudaSharedmemCarveoutMaxShared);
-  if (e == cudaSuccess && bit) g_carveout_set.fetch_or(bit, std::memory_order_acq_rel);
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
   return e;
+}
+
+std::atomic<uint64_t> g_carveout[4];  // decode <fast, gen>, step <fast, gen>
+
+cudaError_t prepare_kernels(bool gen) {
+  cudaError_t e = gen ? prefer_shared_carveout(decode_split_k_kernel<true>, g_carveout[1])
+                      : prefer_shared_carveout(decode_split_k_kernel<false>, g_carveout[0]);
+  if (e != cudaSuccess) return e;
+  return gen ? prefer_shared_carveout(decode_step_kernel<true>, g_carveout[3])
+             : prefer_shared_carveout(decode_step_kernel<false>, g_carveout[2]);
 }
 
 }  // namespace
 
+bool decode_uses_generic_build(int key_bits, int value_bits) { return key_bits != 2 || value_bits != 2; }
+
 // Resident decode CTAs per SM, from the kernel's registers and shared memory and
 // the TMEM columns each CTA allocates (computed from the attributes rather than
 // the runtime occupancy query, which does not report the residency seen on
-// sm_100a for this kernel). Cached per device.
-int decode_ctas_per_sm() {
-  static std::atomic<int> cached[64];
+// sm_100a for this kernel). Cached per device and build.
+int decode_ctas_per_sm(int key_bits, int value_bits) {
+  static std::atomic<int> cached[2][64];
+  const bool gen = decode_uses_generic_build(key_bits, value_bits);
+  const int fallback = gen ? kGenCtasPerSm : kCtasPerSm;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return kCtasPerSm;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fallback;
   if (dev < 64) {
-    const int c = cached[dev].load(std::memory_order_relaxed);
+    const int c = cached[gen][dev].load(std::memory_order_relaxed);
     if (c > 0) return c;
   }
   cudaFuncAttributes a;
   int regs_sm = 0, smem_sm = 0, smem_rsv = 0;
-  if (prefer_shared_carveout() != cudaSuccess || cudaFuncGetAttributes(&a, decode_split_k_kernel) != cudaSuccess ||
+  if (prepare_kernels(gen) != cudaSuccess ||
+      cudaFuncGetAttributes(&a, gen ? decode_step_kernel<true> : decode_step_kernel<false>) != cudaSuccess ||
       cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&smem_rsv, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess)
-    return kCtasPerSm;
+    return fallback;
+  // the step build uses at least as many registers as the decode build: size both by it
+  cudaFuncAttributes a2;
+  if (cudaFuncGetAttributes(&a2, gen ? decode_split_k_kernel<true> : decode_split_k_kernel<false>) == cudaSuccess &&
+      a2.numRegs > a.numRegs)
+    a.numRegs = a2.numRegs;
   const int warp_regs = ((a.numRegs * 32 + 255) / 256) * 256;  // allocated per warp in units of 256
   const int by_regs = regs_sm / (warp_regs * kWarps);
   const int by_smem = smem_sm / ((int)a.sharedSizeBytes + smem_rsv);
-  const int by_tmem = 512 / (int)kTmemCols;
+  const int by_tmem = gen ? 64 : 512 / (int)kTmemCols;  // the 4-bit build holds no tensor memory
   const int n = max(1, min(by_regs, min(by_smem, by_tmem)));
-  if (dev < 64) cached[dev].store(n, std::memory_order_relaxed);
+  if (dev < 64) cached[gen][dev].store(n, std::memory_order_relaxed);
   return n;
 }
 
 cudaError_t launch_decode_step(const DecodeParams& p, const WriteParams& w, cudaStream_t stream) {
-  cudaError_t e = prefer_shared_carveout();
+  const bool gen = decode_uses_generic_build(p.key_bits, p.value_bits);
+  const cudaError_t e = prepare_kernels(gen);
   if (e != cudaSuccess) return e;
-  static std::atomic<uint64_t> step_carveout{0};
-  int dev = 0;
-  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-  const uint64_t bit = dev < 64 ? (1ull << dev) : 0ull;
-  if (!bit || !(step_carveout.load(std::memory_order_acquire) & bit)) {
-    e = cudaFuncSetAttribute(decode_step_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             cudaSharedmemCarveoutMaxShared);
-    if (e != cudaSuccess) return e;
-    if (bit) step_carveout.fetch_or(bit, std::memory_order_acq_rel);
-  }
   const int ctas = p.batch * p.num_kv_heads * (1 + p.num_splits);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(ctas);
-  cfg.blockDim = dim3(kThreads);
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_step_kernel, p, w);
+  return gen ? launch_pdl(decode_step_kernel<true>, dim3(ctas), dim3(kThreads), 0, stream, p, w)
+             : launch_pdl(decode_step_kernel<false>, dim3(ctas), dim3(kThreads), 0, stream, p, w);
 }
 
 cudaError_t launch_decode(const DecodeParams& p, int batch, cudaStream_t stream) {
-  const cudaError_t e = prefer_shared_carveout();
+  const bool gen = decode_uses_generic_build(p.key_bits, p.value_bits);
+  const cudaError_t e = prepare_kernels(gen);
   if (e != cudaSuccess) return e;
   dim3 grid(p.num_splits, p.num_kv_heads, batch);
-  return launch_pdl(decode_split_k_kernel, grid, dim3(kThreads), 0, stream, p);
+  return gen ? launch_pdl(decode_split_k_kernel<true>, grid, dim3(kThreads), 0, stream, p)
+             : launch_pdl(decode_split_k_kernel<false>, grid, dim3(kThreads), 0, stream, p);
 }
 
 }  // namespace omnikv

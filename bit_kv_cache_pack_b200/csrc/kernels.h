@@ -103,7 +103,7 @@ cudaError_t launch_decode(const DecodeParams& p, int batch, cudaStream_t stream)
 // sequence, described by w) followed by the decode CTAs of p.
 cudaError_t launch_decode_step(const DecodeParams& p, const WriteParams& w, cudaStream_t stream);
 
-int decode_ctas_per_sm();  // resident decode CTAs per SM on the current device
+int decode_ctas_per_sm(int key_bits, int value_bits);  // resident decode CTAs per SM on the current device
 cudaError_t launch_combine(const CombineParams& p, int batch, cudaStream_t stream);
 
 }  // namespace omnikv

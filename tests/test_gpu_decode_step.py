@@ -42,28 +42,29 @@ def _prefill(m, consts, cache, spec, params, drift, lengths, dev, seed):
 
 
 CASES = [
-    # (kv heads, group, lengths, steps, explicit splits: 0 = default (fused))
-    (2, 8, [93], 5, 0),                 # crosses the window boundary at 96
-    (2, 8, [31, 64, 0], 3, 0),           # a full window, a fresh window, an empty sequence
-    (4, 8, [200, 17], 4, 0),             # 4 kv heads, 32 query heads
-    (2, 8, [93, 40], 4, 200),            # 2 x (1 + 200) CTAs: beyond residency -> four-call fallback
+    # (kv heads, group, lengths, steps, explicit splits: 0 = default (fused), bits)
+    (2, 8, [93], 5, 0, 2),                 # crosses the window boundary at 96
+    (2, 8, [31, 64, 0], 3, 0, 2),           # a full window, a fresh window, an empty sequence
+    (4, 8, [200, 17], 4, 0, 2),             # 4 kv heads, 32 query heads
+    (2, 8, [93, 40], 4, 200, 2),            # 2 x (1 + 200) CTAs: beyond residency -> four-call fallback
+    (2, 8, [93, 250], 4, 0, 4),             # K4V4: the CUDA-core decode path with the fused append
 ]
 
 
-@pytest.mark.parametrize("hkv,G,lengths,steps,splits", CASES,
-                         ids=["b1-boundary", "ragged-b3", "h4", "fallback"])
-def test_decode_step_matches_four_calls_and_oracle(cuda_device, hkv, G, lengths, steps, splits):
+@pytest.mark.parametrize("hkv,G,lengths,steps,splits,bits", CASES,
+                         ids=["b1-boundary", "ragged-b3", "h4", "fallback", "k4"])
+def test_decode_step_matches_four_calls_and_oracle(cuda_device, hkv, G, lengths, steps, splits, bits):
     import bit_kv_cache_pack_b200 as m
     dev = cuda_device
     seed = 21 + hkv + len(lengths)
-    spec = dataclasses.replace(with_bits(WORKLOADS["tiny"], 2, 2), num_kv_heads=hkv, num_q_heads=hkv * G,
+    spec = dataclasses.replace(with_bits(WORKLOADS["tiny"], bits, bits), num_kv_heads=hkv, num_q_heads=hkv * G,
                                batch=len(lengths))
     params, consts, ocfg = make_layer(spec, seed, 0, dev)
     B = len(lengths)
     cap = 320
     drift = key_drift(spec, seed, 0, cap // 32, dev)
-    fused = m.KVCache(B, hkv, cap, 2, 2, dev)
-    plain = m.KVCache(B, hkv, cap, 2, 2, dev)
+    fused = m.KVCache(B, hkv, cap, bits, bits, dev)
+    plain = m.KVCache(B, hkv, cap, bits, bits, dev)
     kept = _prefill(m, consts, fused, spec, params, drift, lengths, dev, seed)
     _prefill(m, consts, plain, spec, params, drift, lengths, dev, seed)
     torch.cuda.synchronize()
@@ -106,7 +107,7 @@ def test_decode_step_matches_four_calls_and_oracle(cuda_device, hkv, G, lengths,
     # the oracle, writing the same prefill and appends, decodes the last step's query
     ref_all = []
     for b in range(B):
-        oc = codec.OracleCache(1, hkv, cap, 2, 2)
+        oc = codec.OracleCache(1, hkv, cap, bits, bits)
         kb, vb, mb = kept[b]
         if lengths[b]:
             codec.write_cache(ocfg, oc, kb[None], vb[None], mb[None])
