@@ -413,9 +413,17 @@ __device__ void decode_generic_t(const DecodeParams& p, DecodeSmem& sm, int b, i
   }
 }
 
-__device__ void decode_generic(const DecodeParams& p, DecodeSmem& sm, int b, int kvh, int split) {
-  if (p.key_bits == 2 && p.value_bits == 2)
-    decode_generic_t<2, 2>(p, sm, b, kvh, split);
+// The 2-bit build reaches the CUDA-core path only for a codebook that is not
+// symmetric: out of line there, so that the tensor-core path stays compact in
+// the instruction cache. The 4-bit build inlines its three instances.
+__device__ __noinline__ void decode_generic_asym(const DecodeParams& p, DecodeSmem& sm, int b, int kvh, int split) {
+  decode_generic_t<2, 2>(p, sm, b, kvh, split);
+}
+
+template <bool kGen>
+__device__ __forceinline__ void decode_generic(const DecodeParams& p, DecodeSmem& sm, int b, int kvh, int split) {
+  if (!kGen)
+    decode_generic_asym(p, sm, b, kvh, split);
   else if (p.key_bits == 2)
     decode_generic_t<2, 4>(p, sm, b, kvh, split);
   else if (p.value_bits == 2)
@@ -972,7 +980,7 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, DecodeSmem& sm
     if (threadIdx.x < 32) tmem_dealloc(tbase, kTmemCols);
     return;
   }
-  decode_generic(p, sm, b, kvh, split);
+  decode_generic<kGen>(p, sm, b, kvh, split);
 }
 
 constexpr int kGenCtasPerSm = 4;  // the 4-bit build: registers for 4 resident CTAs
