@@ -39,6 +39,30 @@ WORKLOADS_KEYS = ("tiny", "omni3b-b1", "omni3b-b16", "omni30b-b8", "ragged-b64")
 METRIC = "2-bit decode attention tokens/s and achieved HBM GB/s vs ~8 TB/s (1 B200)"
 UNIT = "tokens/s"
 BYTES_PER_TOKEN_HEAD = {(2, 2): 82, (4, 4): 146}   # algorithmic packed bytes per token per kv head
+
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the
+# timed kernel on the default workload, from an ncu capture of this benchmark
+# (profiles/decode_step.omni3b-b1.md), valid for the kernel sources with this
+# SHA-256; any change to them makes the field null until the next capture.
+TRAFFIC_CAPTURE = {"sources_sha256": "4137738ab039f35cf3880972dd0b5ef2438eedee4d952f92bf42902e7f5c6281",
+                   "bytes_per_launch": 2226176}
+KERNEL_SOURCES = ("decode_split_k.cu", "append.cuh", "common.cuh", "ptx.cuh", "kernels.h")
+
+
+def kernel_sources_sha256():
+    import hashlib
+    h = hashlib.sha256()
+    d = os.path.join(os.path.dirname(os.path.abspath(__file__)), "bit_kv_cache_pack_b200", "csrc")
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(d, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def captured_traffic(workload_name):
+    if workload_name != "qwen2.5-omni-3b-36L-b1-ctx10240" or TRAFFIC_CAPTURE["sources_sha256"] is None:
+        return None
+    return TRAFFIC_CAPTURE["bytes_per_launch"] if kernel_sources_sha256() == TRAFFIC_CAPTURE["sources_sha256"] else None
 L2_FLUSH_BYTES = 512 << 20
 
 
@@ -50,6 +74,12 @@ def parse_args():
     ap.add_argument("--impl", default="omnikv", choices=["omnikv", "reference"])
     ap.add_argument("--workload", default="omni3b-b1", choices=sorted(WORKLOADS_KEYS))
     ap.add_argument("--no-graphs", action="store_true")
+    ap.add_argument("--layer", choices=["decode", "write"], default=None,
+                    help="time one layer's decode (+ combine) or prefill cache write on --workload instead of "
+                         "the decode step; prints one JSON line per split count")
+    ap.add_argument("--bits", type=int, default=0, help="with --layer: 2 or 4 (default: the workload's)")
+    ap.add_argument("--batch", type=int, default=0, help="with --layer: override the workload's batch")
+    ap.add_argument("--splits", default="0", help="with --layer decode: comma-separated split counts (0: default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--clocks-csv", default=None, help="where to keep the nvidia-smi samples (default: a temp file)")
     return ap.parse_args()
@@ -362,7 +392,7 @@ def run_gpu(args):
                        "launch": "one CUDA graph for all steps (flush + events + C-ABI calls)" if use_graphs
                        else "eager"},
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                         "frac": round(achieved / peak, 4), "traffic": None,
+                         "frac": round(achieved / peak, 4), "traffic": captured_traffic(spec.name),
                          "peak_source": peak_kind,
                          "kernel": "decode_step_kernel (append + decode launch)" if wl.fused
                          else "kv_append_kernel + decode_split_k launches",
@@ -517,9 +547,92 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_layer(args):
+    """One layer of --workload: the prefill cache write of the whole batch, or
+    decode + combine over that cache (split counts from --splits), each timed
+    with CUDA events after warm-up, L2 flushed before every timed call. Bytes:
+    write 512 B of fp16 K and V in + the packed record out per token and kv head;
+    decode the packed records per token and kv head + 1 modality byte per token."""
+    import dataclasses
+    import bit_kv_cache_pack_b200 as m
+    from synth.workloads import (WORKLOADS, codebook, key_drift, layer_params, prefill_inputs, seq_lengths,
+                                 with_bits)
+    spec = WORKLOADS[args.workload]
+    bits = args.bits or spec.key_bits
+    spec = with_bits(spec, bits, bits)
+    if args.batch:
+        spec = dataclasses.replace(spec, batch=args.batch)
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    seed = 7
+    L = seq_lengths(spec, seed)
+    T = int(L.max())
+    cap = int(-(-(T + 8) // 32) * 32)
+    params = layer_params(spec, seed, 0)
+    consts = m.LayerConstants(codebook(bits), codebook(bits), params["key_signs"], params["value_rot"],
+                              spec.num_q_heads, dev)
+    drift = key_drift(spec, seed, 0, cap // 32, dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    per_token = BYTES_PER_TOKEN_HEAD[(bits, bits)]
+    peak, _ = peaks()
+    iters, warm = 5, 2
+
+    def timed(fn, prep=None):
+        ts = []
+        for it in range(iters + warm):
+            if prep is not None:
+                prep()
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize(dev)
+            if it >= warm:
+                ts.append(e0.elapsed_time(e1) * 1e3)
+        return float(np.median(ts))
+
+    if args.layer == "write":
+        k, v, mod = prefill_inputs(spec, seed, 0, params, drift, np.full(spec.batch, T), dev)
+        c = m.KVCache(spec.batch, spec.num_kv_heads, cap, bits, bits, dev)
+
+        def empty():  # the prefill of an empty cache, every time
+            c.seq_lens.zero_()
+            c.struct.max_seq_len = 0
+
+        us = timed(lambda: m.omnikv_write_cache(consts.struct, c.struct, k, v, mod, T), empty)
+        byts = spec.batch * T * spec.num_kv_heads * (512 + per_token) + spec.batch * T
+        print(json.dumps({"layer": "write", "workload": spec.name, "tokens": spec.batch * T, "us": round(us, 2),
+                          "GBps": round(byts / us / 1e3, 1), "frac": round(byts / us / 1e3 / peak, 4),
+                          "error_word": int(c.error_word.item())}), flush=True)
+        return
+    cache = m.KVCache(spec.batch, spec.num_kv_heads, cap, bits, bits, dev)
+    for b in range(spec.batch):
+        k, v, mod = prefill_inputs(spec, seed, 0, params, drift, L, dev, batch_index=[b])
+        n = int(L[b])
+        m.omnikv_write_cache(consts.struct, cache.sequence_view(b), k[:, :, :n].contiguous(),
+                             v[:, :, :n].contiguous(), mod[:, :n].contiguous(), n)
+        del k, v, mod
+    cache.struct.max_seq_len = T
+    q = torch.randn(spec.batch, spec.num_q_heads, 128, device=dev).half()
+    byts = int(L.astype(np.int64).sum()) * spec.num_kv_heads * per_token + int(L.sum())
+    for S in [int(x) for x in args.splits.split(",")]:
+        S = S or m.omnikv_default_splits(consts.struct, cache.struct)
+        part = m.partials_tensor(spec.batch, spec.num_q_heads, S, dev)
+        out = torch.empty(spec.batch, spec.num_q_heads, 128, device=dev)
+        dec = timed(lambda: m.omnikv_decode_attention(consts.struct, cache.struct, q, part, S))
+        comb = timed(lambda: m.omnikv_combine(consts.struct, cache.struct, part, S, out))
+        print(json.dumps({"layer": "decode", "workload": spec.name, "splits": S, "decode_us": round(dec, 2),
+                          "combine_us": round(comb, 2), "GBps": round(byts / dec / 1e3, 1),
+                          "frac": round(byts / dec / 1e3 / peak, 4), "error_word": int(cache.error_word.item())}),
+              flush=True)
+
+
 def main():
     args = parse_args()
-    if args.impl == "reference":
+    if args.layer:
+        run_layer(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_gpu(args)

@@ -251,7 +251,7 @@ __device__ void quantize_window(const WriteParams& p, int b, int h, int w, int L
       const float* U = p.value_rot + ((size_t)(h * kMods + m) * kHeadDim) * kHeadDim + j;
       // column j of U_m against the value: independent loads, 8 partial sums
       float part[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll 32
+#pragma unroll  // every load of the column issued before the first FMA needs it
       for (int c = 0; c < kHeadDim; ++c) part[c & 7] = fmaf(U[(size_t)c * kHeadDim], kp[i][c], part[c & 7]);
       const float acc = ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
       const float s = s_sigma[i];

@@ -2,7 +2,9 @@
 // applies the inverse value rotations (paperpeel.com section 1: inverse value
 // rotations are applied to head outputs instead of to every cached value).
 //
-// One CTA per (query head, block of 32 output rows, kv head, sequence):
+// One CTA per (query head, block of output rows, kv head, sequence), the rows
+// split in 4 blocks of 32 when the heads alone would not fill the GPU, else one
+// block of 128:
 //   0. before waiting on the decode launch: this warp's 4 rows of U_m for the 3
 //      modalities go into registers (they do not depend on the decode);
 //   1. warp 0: M = max_s m_s, weights e_s = exp(m_s - M), l = sum_s l_s e_s;
@@ -10,8 +12,8 @@
 //      two threads per vector column, splits of weight 0 skipped;
 //   3. out[j] = sum_m sum_c U_m[j][c] a_m[c] for the block's rows: one warp per 4
 //      rows, lanes over c, warp reduction.
-// The 4 row blocks of a head merge the same partials (read from L2); splitting
-// the rows keeps every step one memory round trip deep.
+// The row blocks of a head merge the same partials (read from L2); splitting the
+// rows keeps every step one memory round trip deep when there are few heads.
 // A sequence without tokens (all m_s = -inf) yields zeros.
 #include "common.cuh"
 #include "kernels.h"
@@ -22,12 +24,13 @@ namespace omnikv {
 namespace {
 
 constexpr int kCombineThreads = 256;
-constexpr int kRowBlocks = 4;                        // blocks of 32 output rows
-constexpr int kRowsPerWarp = kHeadDim / kRowBlocks / (kCombineThreads / 32);  // 4
+constexpr int kWarpsC = kCombineThreads / 32;
 constexpr int kMaxSplitsSmem = 4096;
 
+template <int kRowBlocks>
 __global__ void __launch_bounds__(kCombineThreads)
 combine_inverse_rotate_kernel(const CombineParams p) {
+  constexpr int kRowsPerWarp = kHeadDim / kRowBlocks / kWarpsC;  // 4 or 16
   const int g = blockIdx.x / kRowBlocks;  // query head within the group
   const int rb = blockIdx.x % kRowBlocks;
   const int kvh = blockIdx.y;
@@ -44,12 +47,15 @@ combine_inverse_rotate_kernel(const CombineParams p) {
   __shared__ float s_l;
 
   griddep_launch_dependents();
-  // ---- 0. value-basis rows (constant input): rows j0 .. j0 + 3, lanes over c
+  // ---- 0. value-basis rows (constant input): this warp's rows j0 .., lanes over
+  // c; with 4 row blocks all of them (4 rows x 3 modalities) are loaded before
+  // the wait, with one block the first 4
   const int j0 = rb * (kHeadDim / kRowBlocks) + warp * kRowsPerWarp;
   const float* Ubase = p.value_rot + (size_t)kvh * kMods * kHeadDim * kHeadDim;
-  float4 u[kRowsPerWarp][kMods];
+  constexpr int kPre = 4;
+  float4 u[kPre][kMods];
 #pragma unroll
-  for (int r = 0; r < kRowsPerWarp; ++r)
+  for (int r = 0; r < kPre; ++r)
 #pragma unroll
     for (int m = 0; m < kMods; ++m)
       u[r][m] = reinterpret_cast<const float4*>(Ubase + ((size_t)m * kHeadDim + j0 + r) * kHeadDim)[lane];
@@ -111,24 +117,34 @@ combine_inverse_rotate_kernel(const CombineParams p) {
   }
   __syncthreads();
 
-  // ---- 3. out[j] = sum_m U_m[j][:] . a_m for this warp's rows
+  // ---- 3. out[j] = sum_m U_m[j][:] . a_m for this warp's rows, 4 at a time
   float* out = p.out + ((size_t)b * Hq + qh) * kHeadDim;
   float4 xa[kMods];
 #pragma unroll
   for (int m = 0; m < kMods; ++m) xa[m] = reinterpret_cast<const float4*>(a + m * kHeadDim)[lane];
 #pragma unroll
-  for (int r = 0; r < kRowsPerWarp; ++r) {
-    float v = 0.0f;
+  for (int rr = 0; rr < kRowsPerWarp; rr += kPre) {
+    if (rr > 0) {
 #pragma unroll
-    for (int m = 0; m < kMods; ++m) {
-      v = fmaf(u[r][m].x, xa[m].x, v);
-      v = fmaf(u[r][m].y, xa[m].y, v);
-      v = fmaf(u[r][m].z, xa[m].z, v);
-      v = fmaf(u[r][m].w, xa[m].w, v);
+      for (int r = 0; r < kPre; ++r)
+#pragma unroll
+        for (int m = 0; m < kMods; ++m)
+          u[r][m] = reinterpret_cast<const float4*>(Ubase + ((size_t)m * kHeadDim + j0 + rr + r) * kHeadDim)[lane];
     }
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (lane == 0) out[j0 + r] = v;
+    for (int r = 0; r < kPre; ++r) {
+      float v = 0.0f;
+#pragma unroll
+      for (int m = 0; m < kMods; ++m) {
+        v = fmaf(u[r][m].x, xa[m].x, v);
+        v = fmaf(u[r][m].y, xa[m].y, v);
+        v = fmaf(u[r][m].z, xa[m].z, v);
+        v = fmaf(u[r][m].w, xa[m].w, v);
+      }
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0) out[j0 + rr + r] = v;
+    }
   }
 }
 
@@ -136,8 +152,15 @@ combine_inverse_rotate_kernel(const CombineParams p) {
 
 cudaError_t launch_combine(const CombineParams& p, int batch, cudaStream_t stream) {
   if (p.num_splits > kMaxSplitsSmem) return cudaErrorInvalidValue;
-  dim3 grid(p.group * kRowBlocks, p.num_kv_heads, batch);
-  return launch_pdl(combine_inverse_rotate_kernel, grid, dim3(kCombineThreads), 0, stream, p);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long heads = (long long)batch * p.num_kv_heads * p.group;
+  if (heads >= sms) {  // enough heads to fill the GPU: one CTA per head
+    dim3 grid(p.group, p.num_kv_heads, batch);
+    return launch_pdl(combine_inverse_rotate_kernel<1>, grid, dim3(kCombineThreads), 0, stream, p);
+  }
+  dim3 grid(p.group * 4, p.num_kv_heads, batch);
+  return launch_pdl(combine_inverse_rotate_kernel<4>, grid, dim3(kCombineThreads), 0, stream, p);
 }
 
 }  // namespace omnikv
