@@ -43,18 +43,28 @@ __device__ __forceinline__ void key_code_words(WindowSmem& sm, uint8_t* kout, in
     const int c = tid;
     const float s = sm.s_scale[c], m = sm.s_min[c];
     const ScaledBounds<NB> sb = scale_bounds(load_bounds<NB>(sm.bk), s);
+    const int col0 = kp_col(0, c), col1 = kp_col(1, c);  // the column depends on the token's parity only
+#pragma unroll 4
     for (int t = 0; t < kWindow; ++t)
-      sm.codes[t][c] = (uint8_t)((t < nvalid && s != 0.0f) ? code_from_scaled(sb, __fsub_rn(sm.kp[t][kp_col(t, c)], m)) : 0u);
+      sm.codes[t][c] = (uint8_t)((t < nvalid && s != 0.0f)
+                                     ? code_from_scaled(sb, __fsub_rn(sm.kp[t][(t & 1) ? col1 : col0], m))
+                                     : 0u);
   }
   group_sync(bar_id);
   uint32_t* kw = reinterpret_cast<uint32_t*>(kout);
   for (int wi = tid; wi < kWindow * wpt; wi += kWriteThreads) {
     const int t = wi / wpt;
     const int word = wi - t * wpt;
-    const uint8_t* src = &sm.codes[t][word * cpw];
+    // cpw code bytes, 4 per u32, compacted to BITS-bit fields (bytes hold codes < 2^BITS)
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(&sm.codes[t][word * cpw]);
     uint32_t bits = 0;
 #pragma unroll
-    for (int k = 0; k < cpw; ++k) bits |= (uint32_t)src[k] << (BITS * k);
+    for (int q = 0; q < cpw / 4; ++q) {
+      const uint32_t x = src[q];
+      const uint32_t f = (x & 0xFFu) | ((x >> (8 - BITS)) & (0xFFu << BITS)) | ((x >> (16 - 2 * BITS)) & (0xFFu << (2 * BITS))) |
+                         ((x >> (24 - 3 * BITS)) & (0xFFu << (3 * BITS)));
+      bits |= (f & ((1u << (4 * BITS)) - 1u)) << (4 * BITS * q);
+    }
     kw[wi] = bits;
   }
 }
@@ -184,9 +194,10 @@ __device__ void quantize_window(const WriteParams& p, int b, int h, int w, int L
   // ---- window range per channel -> fp16 metadata -----------------------------
   {
     const int c = tid;
-    float mn = kp[0][kp_col(0, c)], mx = mn;
+    const int col0 = kp_col(0, c), col1 = kp_col(1, c);  // the column depends on the token's parity only
+    float mn = kp[0][col0], mx = mn;
     for (int i = 1; i < nvalid; ++i) {
-      const float v = kp[i][kp_col(i, c)];
+      const float v = kp[i][(i & 1) ? col1 : col0];
       mn = fminf(mn, v);
       mx = fmaxf(mx, v);
     }
