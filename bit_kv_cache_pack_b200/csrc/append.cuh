@@ -121,6 +121,13 @@ __device__ void quantize_window(const WriteParams& p, int b, int h, int w, int L
 #pragma unroll
     for (int j = 0; j < 4; ++j) raw[j] = reinterpret_cast<const uint4*>(src)[j];
   }
+  // the value of this warp's first new token (used after the keys, loaded now)
+  __half vfirst[4] = {__float2half(0.f), __float2half(0.f), __float2half(0.f), __float2half(0.f)};
+  if (!(p.tc_values && p0 >= L0 && nvalid == kWindow) && inew0 + warp < nvalid) {
+    const __half* src = vnew + (size_t)(p0 + inew0 + warp - L0) * kHeadDim;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) vfirst[j] = src[lane + 32 * j];
+  }
   if (!(p.tc_values && p0 >= L0 && nvalid == kWindow)) {
     int m0 = mnew[p0 + inew0 - L0];
     m0 = m0 >= kMods ? kMods - 1 : m0;
@@ -229,13 +236,17 @@ __device__ void quantize_window(const WriteParams& p, int b, int h, int w, int L
 
   // ---- values: per-token scale (pairwise tree in a warp) ----------------------
   for (int i = inew0 + warp; i < nvalid; i += kWriteThreads / 32) {
-    const __half* src = vnew + (size_t)(p0 + i - L0) * kHeadDim;
     float x[4];
+    if (i == inew0 + warp) {  // the warp's first new value was loaded at the start
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      x[j] = __half2float(src[lane + 32 * j]);
-      kp[i][lane + 32 * j] = x[j];
+      for (int j = 0; j < 4; ++j) x[j] = __half2float(vfirst[j]);
+    } else {
+      const __half* src = vnew + (size_t)(p0 + i - L0) * kHeadDim;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) x[j] = __half2float(src[lane + 32 * j]);
     }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) kp[i][lane + 32 * j] = x[j];
     // tree: h = 64 pairs j with j + 2, h = 32 pairs the two results, then lanes
     const float a = __fadd_rn(__fmul_rn(x[0], x[0]), __fmul_rn(x[2], x[2]));
     const float c = __fadd_rn(__fmul_rn(x[1], x[1]), __fmul_rn(x[3], x[3]));
