@@ -42,8 +42,9 @@ BYTES_PER_TOKEN_HEAD = {(2, 2): 82, (4, 4): 146}   # algorithmic packed bytes pe
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the
 # timed kernel on the default workload, from an ncu capture of this benchmark
-# (profiles/decode_step.omni3b-b1.md), valid for the kernel sources with this
-# SHA-256; any change to them makes the field null until the next capture.
+# (its summary is kept with the other profiles), valid for the kernel sources
+# with this SHA-256; any change to them makes the field null until the next
+# capture.
 TRAFFIC_CAPTURE = {"sources_sha256": "4137738ab039f35cf3880972dd0b5ef2438eedee4d952f92bf42902e7f5c6281",
                    "bytes_per_launch": 2226176}
 KERNEL_SOURCES = ("decode_split_k.cu", "append.cuh", "common.cuh", "ptx.cuh", "kernels.h")

@@ -83,13 +83,6 @@ __device__ __forceinline__ void warp_hadamard_rotate(float x[4], const float sig
   for (int r = 0; r < 4; ++r) x[r] = __fmul_rn(x[r], s);
 }
 
-// code = #{ j : z > t_j } for the L-1 thresholds (strict comparison).
-__device__ __forceinline__ uint32_t count_above(float z, const float* thr, int nthr) {
-  uint32_t c = 0;
-  for (int j = 0; j < nthr; ++j) c += (z > thr[j]) ? 1u : 0u;
-  return c;
-}
-
 // Division-free, exact form of the code decision  fl(fl(a / s) + c) > t  for
 // s > 0 (fl: fp32 round to nearest even). y -> fl(y + c) is monotone, so the
 // decision is  fl(a / s) >= F  for F the smallest float with fl(F + c) > t; and

@@ -41,8 +41,19 @@
 // two tokens of every value-operand register (k-slots 2t, 2t+1 -> tokens t,
 // t+8) sit 16 bits apart in one channel-major code word.
 //
-// Generic path (4-bit codes, or a codebook that is not symmetric): a CUDA-core
-// loop with the same math (scores, online softmax, per-modality accumulators).
+// CUDA-core path (4-bit codes, or a codebook that is not symmetric): the CTA
+// decodes a window at a time (four threads per token for the scores, a thread per
+// channel for the values), built into its own kernel for 4-bit caches (more CTAs
+// per SM, no tensor memory).
+//
+// Decode step (decode_step_kernel): the first batch x kv-head CTAs of the launch
+// append one token per (sequence, kv head) and publish the new length in a flag;
+// the decode CTAs read the cache at that length, and only the warp whose window
+// receives the token waits (bounded) for the flag before copying it.
+//
+// Launches use programmatic dependent launch: everything that does not depend on
+// the cache (query rotation, score operand, L2 prefetch of the value bases for the
+// combine) runs before griddepcontrol.wait.
 //
 // Inputs must stay in the fp16 range of the operands: |q' s_gc| / sqrt(128)
 // below ~480 and value scales sigma below ~480; outside it the output is not

@@ -4,10 +4,12 @@
 // a short append one CTA per sequence (one 128-thread group per kv head).
 // Keys (paperpeel.com section 2.2 "Temporal key drift", 3.1 "32-token groups g",
 // 3.3 "FP16 minimum m_gc and scale s_gc"): every touched window is re-quantised
-// over all its valid tokens -- sign flip + Hadamard butterflies in a warp
-// (4 channels per lane), per-channel min / max over the window, fp16 metadata,
-// codes on the fixed codebook, 16 (or 8) codes per u32. A window left partial
-// keeps its raw fp16 keys in the tail so a later append can re-quantise it.
+// over all its valid tokens -- sign flip + Hadamard butterflies (four threads
+// per token), per-channel min / max over the window, fp16 metadata, codes on the
+// fixed codebook (decided exactly without the division, see common.cuh), 16 (or
+// 8) codes per u32. A window left partial keeps its raw fp16 keys in the tail so
+// a later append can re-quantise it. The per-window body is quantize_window
+// (append.cuh); values of windows a long write fills completely go to vrot_tc.
 // Values (section 2.3 "Modality-aware value rotation"): per token, the fp16
 // scale sigma (pairwise-tree sum of squares in a warp), the rotation
 // v' = U_m^T v, and codes v'/sigma on the fixed codebook, packed channel-major

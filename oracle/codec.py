@@ -18,7 +18,7 @@ pchao.org "方法概览"):
             m in {V, A, L} (section 2.3, "Modality-aware value rotation"), then
             quantise on the fixed codebook with a per-token scale (reading r6).
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent (the same readings the kernels implement):
   r1  affine map of [min, max] onto [c_0, c_{L-1}]:  x_hat = m + s (c_j - c_0),
       s = (max - min) / (c_{L-1} - c_0).
   r3  m and s are rounded to fp16 (round to nearest even) BEFORE codes are
