@@ -47,15 +47,13 @@ int sm_count() {
 
 namespace omnikv {
 
-int32_t resolve_splits(const omnikv_config* cfg, const omnikv_cache* c, int32_t requested) {
-  if (requested > 0) return requested;
-  const int nw = (c->max_seq_len + kWindow - 1) / kWindow;
-  if (nw <= 0) return 1;
-  // aim at one full wave of resident decode CTAs over the whole batch (a
-  // second, partial wave would double the time), with at least 4 windows (one
-  // per warp) per split
-  const long long units = (long long)c->batch * cfg->num_kv_heads;
-  const long long target = (long long)decode_ctas_per_sm(cfg->key_bits, cfg->value_bits) * sm_count();
+namespace {
+
+// Splits for one full wave of `per_sm` resident decode CTAs per SM over the whole
+// batch (a second, partial wave would double the time), with at least 4 windows
+// (one per warp) per split.
+int32_t wave_splits(long long units, int per_sm, int nw) {
+  const long long target = (long long)per_sm * sm_count();
   long long s = target / units;
   // a large batch leaves little split parallelism, and its lengths may differ
   // (fixed-size splits of short sequences are empty): at least 8 splits (on the
@@ -69,6 +67,32 @@ int32_t resolve_splits(const omnikv_config* cfg, const omnikv_cache* c, int32_t 
   return (int32_t)s;
 }
 
+int split_windows_of(const omnikv_cache* c, int32_t S) {
+  const int nw = (c->max_seq_len + kWindow - 1) / kWindow;
+  return nw > 0 ? (nw + S - 1) / S : 1;
+}
+
+}  // namespace
+
+// The library's split count: one wave of the body that will run it. For 2-bit
+// caches the cooperative body takes the split if its wave leaves at most
+// kCoopMaxWindows windows per split, else the per-warp body sizes it.
+int32_t resolve_splits(const omnikv_config* cfg, const omnikv_cache* c, int32_t requested) {
+  if (requested > 0) return requested;
+  const int nw = (c->max_seq_len + kWindow - 1) / kWindow;
+  if (nw <= 0) return 1;
+  const long long units = (long long)c->batch * cfg->num_kv_heads;
+  if (cfg->key_bits != 2 || cfg->value_bits != 2) return wave_splits(units, decode_ctas_per_sm(kBodyGeneric), nw);
+  const int32_t s = wave_splits(units, decode_ctas_per_sm(kBodyCoop), nw);
+  if (split_windows_of(c, s) <= kCoopMaxWindows) return s;
+  return wave_splits(units, decode_ctas_per_sm(kBodyWarp), nw);
+}
+
+// Resident CTAs of a decode-step launch with S splits (the residency of its body).
+long long step_residency(const omnikv_config* cfg, const omnikv_cache* c, int32_t S) {
+  const int body = decode_body(cfg->key_bits, cfg->value_bits, split_windows_of(c, S));
+  return (long long)decode_ctas_per_sm(body) * sm_count();
+}
 
 omnikv_status prepare_decode(const omnikv_config* cfg, const omnikv_cache* cache, const void* q, void* partials,
                              int32_t num_splits, DecodeParams* p) {
@@ -221,12 +245,12 @@ namespace {
 // default is lowered (by at most half) to make it so.
 void plan_step(const omnikv_config* cfg, const omnikv_cache* after, int32_t num_splits, int32_t* S, bool* fused) {
   const long long units = (long long)after->batch * cfg->num_kv_heads;
-  const long long resident = (long long)decode_ctas_per_sm(cfg->key_bits, cfg->value_bits) * sm_count();
   *S = resolve_splits(cfg, after, num_splits);
+  const long long resident = step_residency(cfg, after, *S);
   *fused = units * (1 + (long long)*S) <= resident;
   if (!*fused && num_splits == 0) {
     const long long s_res = resident / units - 1;
-    if (s_res >= 1 && 2 * s_res >= *S) {
+    if (s_res >= 1 && 2 * s_res >= *S && units * (1 + s_res) <= step_residency(cfg, after, (int32_t)s_res)) {
       *S = (int32_t)s_res;
       *fused = true;
     }

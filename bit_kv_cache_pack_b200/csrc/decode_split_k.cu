@@ -8,9 +8,6 @@
 // of a window record.
 //
 // Tensor-core path (2-bit keys and values, symmetric codebook):
-//   * each warp streams its own contiguous run of the split's windows through
-//     a 3-stage shared-memory ring filled by 1-D bulk async copies (record +
-//     the window's 32 modality ids) completing on per-stage mbarriers;
 //   * scores use mma.sync m16n8k16 with the 8 query heads as N. With a
 //     symmetric codebook c_j - c_0 = (c_1 - c_0) b0 + (c_2 - c_0) b1 for the
 //     code's bits b0, b1, so k'_tc - m_gc = s_gc ((c_1 - c_0) b0 + (c_2 - c_0) b1).
@@ -21,21 +18,32 @@
 //     into an fp16 high and low part (so the product keeps ~22 bits), built
 //     once per CTA in shared memory; the window minimum enters as the per-head
 //     offset sum_c q'_c m_gc;
-//   * online softmax per window (running max with exact rescale when it grows,
-//     per-lane partial sums reduced once at the end);
+//   * online softmax (running max with exact rescale when it grows, per-lane
+//     partial sums reduced once at the end);
 //   * P (times the token's value scale sigma and the plane constants, split
 //     into fp16 high + low parts) becomes the B operand of the value product
-//     through movmatrix; values are stored
-//     channel-major so the A operand (16 channels x 16 tokens) again needs one
-//     shift and one AND per register; one fp32 accumulator set per modality
-//     (values of different modalities live in different rotated bases): the
-//     active modality's set is in registers, the others are parked in the
-//     warp's tensor-memory lanes (tcgen05.st / tcgen05.ld, 32 columns each)
-//     together with the running max they were parked at, and are rescaled to
-//     the current max when a tile of that modality brings them back; the c_0
-//     term is c_0 * sum_t p_t sigma_t per modality, added at the end;
-//   * the 4 warps merge (common max, rescale, shared-memory reduction), one
-//     modality at a time, and write one split-K partial per query head.
+//     through movmatrix; values are stored channel-major so the A operand (16
+//     channels x 16 tokens) again needs one shift and one AND per register; one
+//     fp32 accumulator set per modality (values of different modalities live in
+//     different rotated bases); the c_0 term is c_0 * sum_t p_t sigma_t per
+//     modality, added at the end.
+// Two bodies run this arithmetic; the host picks by the split length:
+//   * per-warp body (long splits): each warp streams its own contiguous run of
+//     the split's windows through a 3-stage ring of 1-D bulk async copies (record
+//     + the window's 32 modality ids) and owns all 128 channels of the value
+//     product; the active modality's accumulator is in registers, the others are
+//     parked in the warp's tensor-memory lanes (tcgen05.st / tcgen05.ld) with the
+//     running max they were parked at; the 4 warps merge at the end (common max,
+//     shared-memory reduction, one modality at a time). ~240 registers, 2 CTAs
+//     per SM;
+//   * cooperative body (splits of at most 16 windows): the CTA takes 4 windows
+//     at a time (one 2-stage ring of group copies); warp w scores window w, the
+//     CTA shares one running max, warp w writes its window's value-product B
+//     operand to shared memory, and every warp then runs the value product of
+//     the whole group for its own 32 channels (all three modality accumulators
+//     in registers, no merge). ~168 registers, 3 CTAs per SM; the shorter
+//     critical path wins when a split has few windows (decode steps at small
+//     batch), the per-warp body when it streams many.
 // Token order inside a 16-token tile: fragment row / k-slot r holds token
 // tau(r) = r/2 + 8 (r%2) for r < 8 and 4 + (r-8)/2 + 8 (r%2) for r >= 8, so the
 // two tokens of every value-operand register (k-slots 2t, 2t+1 -> tokens t,
@@ -48,8 +56,8 @@
 //
 // Decode step (decode_step_kernel): the first batch x kv-head CTAs of the launch
 // append one token per (sequence, kv head) and publish the new length in a flag;
-// the decode CTAs read the cache at that length, and only the warp whose window
-// receives the token waits (bounded) for the flag before copying it.
+// the decode CTAs read the cache at that length, and only the copy of the window
+// that receives the token waits (bounded) for the flag.
 //
 // Launches use programmatic dependent launch: everything that does not depend on
 // the cache (query rotation, score operand, L2 prefetch of the value bases for the
@@ -71,36 +79,37 @@ namespace {
 
 constexpr int kWarps = 4;
 constexpr int kThreads = 32 * kWarps;
-constexpr int kStages = 3;
+constexpr int kStages = 3;                      // per-warp body: windows in flight per warp
 constexpr int kRec22 = 2624;                    // K2/V2 record bytes
 constexpr int kStageBytes = kRec22 + kWindow;   // record + modality ids
+constexpr int kCoop = kWarps;                   // cooperative body: windows per group (one per warp for the scores)
+constexpr int kCoopStages = 2;                  // cooperative body: window groups in flight per CTA
+constexpr int kGroupBytes = kCoop * kStageBytes;  // kCoop records, then their modality ids
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: a bulk copy that takes longer is an error
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kCtasPerSm = 2;      // resident CTAs per SM the register budget is set for
-constexpr uint32_t kTmemCols = 128;  // per CTA: 3 parked accumulators x 32 columns in each warp's lanes
+constexpr uint32_t kTmemCols = 128;  // per-warp body, per CTA: 3 parked accumulators x 32 columns in each warp's lanes
 
 struct __align__(16) DecodeSmem {
-  uint8_t stage[kWarps][kStages][kStageBytes];  // also reused by the generic path and the final merge
-  uint4 btab[8][2][32];                         // score B operand per (chunk, plane, lane): {hi, hi, lo, lo}
+  union {
+    struct {
+      uint8_t stage[kWarps][kStages][kStageBytes];  // per-warp rings; also the final merge buffer
+    } w;
+    struct {
+      uint8_t stage[kCoopStages][kGroupBytes];     // window groups
+      uint4 pfrag[kCoop][2][2][32];                 // value B operand per (window, tile, plane, lane): {hi b0, hi b1, lo b0, lo b1}
+    } c;
+  } u;                                            // also the generic path's buffers
+  uint4 btab[8][2][32];                           // score B operand per (chunk, plane, lane): {hi, hi, lo, lo}
   uint64_t bar[kWarps][kStages];
-  float q[kMaxGroup][kHeadDim];                 // rotated queries, times the softmax scale
-  float mw[kWarps][kMaxGroup];                  // per-warp running max, for the merge
-  float lw[kWarps][kMaxGroup];                  // per-warp softmax denominators, for the merge
-  uint32_t tmem_base;                           // TMEM columns of the parked accumulators
+  uint64_t cbar[kCoopStages];
+  float q[kMaxGroup][kHeadDim];                   // rotated queries, times the softmax scale
+  float mw[kWarps][kMaxGroup];                    // per-warp running max (per-warp body merge; cooperative body: window max)
+  float lw[kWarps][kMaxGroup];                    // per-warp softmax denominators, for the merge
+  float red[kWarps][1 + kMods][kMaxGroup];        // cooperative body: per-warp sums of p and of p sigma per modality
+  uint32_t tmask[kCoop][2];                       // cooperative body: modality bits of each tile of the group (0: no window)
+  uint32_t tmem_base;                             // per-warp body: TMEM columns of the parked accumulators
 };
 static_assert(sizeof(DecodeSmem) <= 48 * 1024, "static shared memory");
-
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
 
 // Position of channel c of head g in the rotated-query buffer. Chunks of 4
 // channels inside each group of 32 are XOR-swizzled so that the 8 lanes of a
@@ -207,7 +216,7 @@ struct GenSmem {                 // laid over DecodeSmem::stage
   float wmax[kWarps][kMaxGroup];
   uint64_t bar[kGenStages];
 };
-static_assert(sizeof(GenSmem) <= sizeof(DecodeSmem::stage), "generic path shared memory");
+static_assert(sizeof(GenSmem) <= sizeof(DecodeSmem::u), "generic path shared memory");
 
 __device__ __forceinline__ void gen_issue(const DecodeParams& p, GenSmem& g, int stage, const uint8_t* rec_base,
                                           int rec_bytes, int b, int kvh, int wi, int wait_win, int wait_val) {
@@ -222,7 +231,7 @@ __device__ __forceinline__ void gen_issue(const DecodeParams& p, GenSmem& g, int
 
 template <int KB, int VB>
 __device__ void decode_generic_t(const DecodeParams& p, DecodeSmem& sm, int b, int kvh, int split) {
-  GenSmem& g = *reinterpret_cast<GenSmem*>(&sm.stage[0][0][0]);
+  GenSmem& g = *reinterpret_cast<GenSmem*>(&sm.u);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = p.group;
   const int Hq = p.num_kv_heads * G;
@@ -545,7 +554,7 @@ __device__ __forceinline__ void issue_window(const DecodeParams& p, DecodeSmem& 
       !wait_flag(p.step_flags + (size_t)b * p.num_kv_heads + kvh, wait_val, kWaitLimitNs))
     set_error(p.error_word, OMNIKV_DEVERR_TIMEOUT);
   uint64_t* bar = &sm.bar[warp][stage];
-  uint8_t* dst = &sm.stage[warp][stage][0];
+  uint8_t* dst = &sm.u.w.stage[warp][stage][0];
   mbar_arrive_expect_tx(bar, kStageBytes);
   bulk_copy_g2s(dst, rec_base + (size_t)wi * kRec22, kRec22, bar);
   bulk_copy_g2s(dst + kRec22, p.modality + (size_t)b * p.cap_tokens + (size_t)wi * kWindow, kWindow, bar);
@@ -608,7 +617,7 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
       failed_at = i;
       break;
     }
-    const uint8_t* stg = &sm.stage[warp][s][0];
+    const uint8_t* stg = &sm.u.w.stage[warp][s][0];
     const uint32_t* kw = reinterpret_cast<const uint32_t*>(stg);
     const __half2* meta = reinterpret_cast<const __half2*>(stg + 1024);
     const uint32_t* vw = reinterpret_cast<const uint32_t*>(stg + 1536);
@@ -864,7 +873,7 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
     sm.lw[warp][2 * t] = st.l[0];
     sm.lw[warp][2 * t + 1] = st.l[1];
   }
-  float* xbuf = reinterpret_cast<float*>(&sm.stage[0][0][0]);  // [warp][32 registers][32 lanes]
+  float* xbuf = reinterpret_cast<float*>(&sm.u.w.stage[0][0][0]);  // [warp][32 registers][32 lanes]
   static_assert(kWarps * 32 * 32 * 4 <= kWarps * kStages * kStageBytes, "merge buffer");
 #pragma unroll
   for (int m = 0; m < kMods; ++m) {
@@ -912,6 +921,448 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
   }
 }
 
+// Value-product accumulators of one warp: the warp owns channels 32 w + 4 g + 2 mt
+// (fragment row g) and + 1 (row g + 8) for m-tiles mt = 0, 1, and the query
+// heads 2t, 2t+1 as columns. The active modality accumulates in act (one chain
+// per m-tile and code plane); the totals of the other modalities wait in st, and
+// are exchanged when a tile of another modality comes (rare: modality runs are
+// long).
+struct PvAcc {
+  float act[2][2][4];      // [m-tile][plane][fragment] of the active modality
+  float st[kMods][2][4];   // [modality][m-tile][fragment], inactive modalities
+  int cur;                 // active modality, -1 before the first tile (warp-uniform)
+};
+
+__device__ __forceinline__ void pv_activate(PvAcc& a, int k) {
+  if (k == a.cur) return;
+#pragma unroll
+  for (int kk = 0; kk < kMods; ++kk)
+    if (kk == a.cur) {
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) a.st[kk][mt][r] = a.act[mt][0][r] + a.act[mt][1][r];
+    }
+#pragma unroll
+  for (int kk = 0; kk < kMods; ++kk)
+    if (kk == k) {
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          a.act[mt][0][r] = a.st[kk][mt][r];
+          a.act[mt][1][r] = 0.0f;
+        }
+    }
+  a.cur = k;
+}
+
+// 8 MMAs of one 16-token tile into the active accumulator: B = {hi b0, hi b1,
+// lo b0, lo b1} per plane, k-slot halves masked with m01 (b0) and m23 (b1).
+__device__ __forceinline__ void pv_tile(PvAcc& a, const uint32_t (&a0)[2][4], const uint32_t (&a1)[2][4],
+                                        const uint4& f0, const uint4& f1, uint32_t m01, uint32_t m23) {
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt) {
+    mma_f16_16816(a.act[mt][0], a0[mt], f0.x & m01, f0.y & m23);
+    mma_f16_16816(a.act[mt][1], a1[mt], f1.x & m01, f1.y & m23);
+  }
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt) {
+    mma_f16_16816(a.act[mt][0], a0[mt], f0.z & m01, f0.w & m23);
+    mma_f16_16816(a.act[mt][1], a1[mt], f1.z & m01, f1.w & m23);
+  }
+}
+
+__device__ __forceinline__ void pv_scale(PvAcc& a, float f0, float f1) {
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int P = 0; P < 2; ++P) {
+      a.act[mt][P][0] *= f0;
+      a.act[mt][P][1] *= f1;
+      a.act[mt][P][2] *= f0;
+      a.act[mt][P][3] *= f1;
+    }
+#pragma unroll
+  for (int k = 0; k < kMods; ++k)
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+      a.st[k][mt][0] *= f0;
+      a.st[k][mt][1] *= f1;
+      a.st[k][mt][2] *= f0;
+      a.st[k][mt][3] *= f1;
+    }
+}
+
+// Copies of window group `gi` (windows wfirst .. wfirst + nwin - 1): the records
+// (contiguous in the cache) and then their modality ids, completing on the
+// stage's mbarrier. In a decode step the window that receives the new token is
+// copied only after its flag shows the append (bounded wait); the records before
+// it go first. Thread 0.
+__device__ __forceinline__ void issue_group(const DecodeParams& p, DecodeSmem& sm, int stage, const uint8_t* rec_base,
+                                            int b, int kvh, int wfirst, int nwin, int wait_win, int wait_val) {
+  uint64_t* bar = &sm.cbar[stage];
+  uint8_t* dst = &sm.u.c.stage[stage][0];
+  mbar_arrive_expect_tx(bar, (uint32_t)nwin * (kRec22 + kWindow));
+  int nfree = nwin;  // records that need no wait
+  if (wait_win >= wfirst && wait_win < wfirst + nwin) nfree = wait_win - wfirst;
+  if (nfree > 0) bulk_copy_g2s(dst, rec_base + (size_t)wfirst * kRec22, (uint32_t)nfree * kRec22, bar);
+  if (nfree < nwin) {
+    if (!wait_flag(p.step_flags + (size_t)b * p.num_kv_heads + kvh, wait_val, kWaitLimitNs))
+      set_error(p.error_word, OMNIKV_DEVERR_TIMEOUT);
+    bulk_copy_g2s(dst + nfree * kRec22, rec_base + (size_t)(wfirst + nfree) * kRec22, (uint32_t)(nwin - nfree) * kRec22,
+                  bar);
+  }
+  bulk_copy_g2s(dst + kCoop * kRec22, p.modality + (size_t)b * p.cap_tokens + (size_t)wfirst * kWindow,
+                (uint32_t)nwin * kWindow, bar);
+}
+
+// The tensor-core decode of one split. Windows are taken kCoop at a time (a
+// group, one shared-memory stage): warp w scores window w of the group (both
+// 16-token tiles), the CTA takes the common running max, warp w turns its
+// probabilities into the value-product B operand in shared memory, and then every
+// warp runs the value product of the whole group for its own 32 channels.
+__device__ void decode_coop(const DecodeParams& p, DecodeSmem& sm, int b, int kvh, int split, float kV0, float kV1,
+                            float vc0) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int G = p.group;
+  const int Hq = p.num_kv_heads * G;
+  int T, w0, w1;
+  split_range(p, b, split, T, w0, w1);
+  const uint8_t* rec_base = p.records + ((size_t)(b * p.num_kv_heads + kvh) * p.cap_windows) * kRec22;
+  int wait_win, wait_val;
+  step_window(p, b, wait_win, wait_val);
+  const int ngroups = (w1 - w0 + kCoop - 1) / kCoop;
+  int issued = 0;  // groups whose copies were issued (meaningful in thread 0)
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int s = 0; s < kCoopStages; ++s) mbar_init(&sm.cbar[s], 1);
+    fence_barrier_init();
+    for (; issued < kCoopStages && issued < ngroups; ++issued)
+      issue_group(p, sm, issued, rec_base, b, kvh, w0 + kCoop * issued, min(kCoop, w1 - w0 - kCoop * issued),
+                  wait_win, wait_val);
+  }
+  __syncthreads();  // barrier initialisation (and the score operand) visible to every thread
+
+  float m_run[2] = {-INFINITY, -INFINITY};  // running max of heads 2t, 2t+1 (the same in every warp)
+  float l_part[2] = {0.0f, 0.0f};           // per-lane partial sums of p over this warp's windows
+  float S_part[kMods][2];                   // per-lane partial sums of p * sigma per modality
+#pragma unroll
+  for (int k = 0; k < kMods; ++k) S_part[k][0] = S_part[k][1] = 0.0f;
+  PvAcc pv;
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      pv.act[mt][0][r] = pv.act[mt][1][r] = 0.0f;
+#pragma unroll
+      for (int k = 0; k < kMods; ++k) pv.st[k][mt][r] = 0.0f;
+    }
+  pv.cur = -1;
+  const int rlo = 13 - 2 * t, rhi = (5 - 2 * t) & 31;
+
+  int failed_at = -1;
+  for (int it = 0; it < ngroups; ++it) {
+    const int s = it % kCoopStages;
+    const int wi = w0 + kCoop * it + warp;  // this warp's window for the scores
+    const bool have = wi < w1;              // warp-uniform
+    const uint8_t* stg = &sm.u.c.stage[s][0];
+    const bool ok = mbar_wait_bounded(&sm.cbar[s], (it / kCoopStages) & 1, kWaitLimitNs);
+    const bool wok = __all_sync(0xffffffffu, ok);
+
+    // ---- scores of this warp's window (both tiles) -------------------------
+    const uint8_t* rec = stg + warp * kRec22;
+    const uint8_t* mods = stg + kCoop * kRec22 + warp * kWindow;
+    float sc[2][4];
+    int tokA[2], tokB[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      tokA[h] = 16 * h + tile_token(g);
+      tokB[h] = 16 * h + tile_token(g + 8);
+#pragma unroll
+      for (int r = 0; r < 4; ++r) sc[h][r] = -INFINITY;
+    }
+    if (have && wok) {
+      const uint32_t* kw = reinterpret_cast<const uint32_t*>(rec);
+      const __half2* meta = reinterpret_cast<const __half2*>(rec + 1024);
+      // fp16 scale pairs of the A operand and the offset sum_c q'_c m_gc; lane
+      // (g, t) covers channels 32t .. 32t+31 (k-slot pairs (c, c+8))
+      uint32_t sp[8][2];
+      float off;
+      {
+        const float* qrow = &sm.q[g][32 * t];
+        const int qsw = (4 * (g & 1) + t) & 7;
+        const uint4* mv4 = reinterpret_cast<const uint4*>(meta + 32 * t);
+        uint32_t mv[32];
+#pragma unroll
+        for (int i4 = 0; i4 < 8; ++i4) {
+          const uint4 mm = mv4[i4];
+          mv[4 * i4 + 0] = mm.x;
+          mv[4 * i4 + 1] = mm.y;
+          mv[4 * i4 + 2] = mm.z;
+          mv[4 * i4 + 3] = mm.w;
+        }
+        off = 0.0f;
+#pragma unroll
+        for (int i4 = 0; i4 < 8; ++i4) {
+          const float4 qq = *reinterpret_cast<const float4*>(qrow + 4 * (i4 ^ qsw));
+          const float qa[4] = {qq.x, qq.y, qq.z, qq.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            off = fmaf(qa[j], __low2float(*reinterpret_cast<const __half2*>(&mv[4 * i4 + j])), off);
+        }
+#pragma unroll
+        for (int kc = 0; kc < 8; ++kc) {  // high halves (the scales) of channels (c, c+8)
+          sp[kc][0] = __byte_perm(mv[kc], mv[kc + 8], 0x7632);
+          sp[kc][1] = __byte_perm(mv[kc + 16], mv[kc + 24], 0x7632);
+        }
+        off += __shfl_xor_sync(0xffffffffu, off, 1);
+        off += __shfl_xor_sync(0xffffffffu, off, 2);
+      }
+      const float off0 = __shfl_sync(0xffffffffu, off, 8 * t);      // head 2t
+      const float off1 = __shfl_sync(0xffffffffu, off, 8 * t + 4);  // head 2t + 1
+      uint2 kA[2], kB[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        kA[h] = *reinterpret_cast<const uint2*>(kw + tokA[h] * 8 + 2 * t);
+        kB[h] = *reinterpret_cast<const uint2*>(kw + tokB[h] * 8 + 2 * t);
+      }
+      float d0[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      float d1[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+      for (int kc = 0; kc < 8; ++kc) {
+        const uint32_t s0 = sp[kc][0], s1 = sp[kc][1];
+        const uint4 bp0 = sm.btab[kc][0][lane], bp1 = sm.btab[kc][1][lane];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t r[4];
+          if (kc < 7) {
+            r[0] = kA[h].x << (13 - 2 * kc);
+            r[1] = kB[h].x << (13 - 2 * kc);
+            r[2] = kA[h].y << (13 - 2 * kc);
+            r[3] = kB[h].y << (13 - 2 * kc);
+          } else {
+            r[0] = kA[h].x >> 1;
+            r[1] = kB[h].x >> 1;
+            r[2] = kA[h].y >> 1;
+            r[3] = kB[h].y >> 1;
+          }
+          const uint32_t a0[4] = {hmul2_u32(s0, r[0] & kPlane0), hmul2_u32(s0, r[1] & kPlane0),
+                                  hmul2_u32(s1, r[2] & kPlane0), hmul2_u32(s1, r[3] & kPlane0)};
+          const uint32_t a1[4] = {hmul2_u32(s0, r[0] & kPlane1), hmul2_u32(s0, r[1] & kPlane1),
+                                  hmul2_u32(s1, r[2] & kPlane1), hmul2_u32(s1, r[3] & kPlane1)};
+          mma_f16_16816(d0[h], a0, bp0.x, bp0.y);
+          mma_f16_16816(d1[h], a1, bp1.x, bp1.y);
+          mma_f16_16816(d0[h], a0, bp0.z, bp0.w);
+          mma_f16_16816(d1[h], a1, bp1.z, bp1.w);
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int posA = wi * kWindow + tokA[h], posB = wi * kWindow + tokB[h];
+        sc[h][0] = posA < T ? d0[h][0] + d1[h][0] + off0 : -INFINITY;
+        sc[h][1] = posA < T ? d0[h][1] + d1[h][1] + off1 : -INFINITY;
+        sc[h][2] = posB < T ? d0[h][2] + d1[h][2] + off0 : -INFINITY;
+        sc[h][3] = posB < T ? d0[h][3] + d1[h][3] + off1 : -INFINITY;
+      }
+    }
+    {
+      float mx0 = fmaxf(fmaxf(sc[0][0], sc[0][2]), fmaxf(sc[1][0], sc[1][2]));
+      float mx1 = fmaxf(fmaxf(sc[0][1], sc[0][3]), fmaxf(sc[1][1], sc[1][3]));
+#pragma unroll
+      for (int o = 4; o <= 16; o <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+      }
+      if (g == 0) *reinterpret_cast<float2*>(&sm.mw[warp][2 * t]) = make_float2(mx0, mx1);
+    }
+    if (__syncthreads_or(!ok)) {  // a copy did not complete in time (the whole CTA stops here)
+      failed_at = it;
+      break;
+    }
+    // every warp is past the value product of group it - 1: its stage may be refilled
+    if (threadIdx.x == 0 && issued < ngroups && issued == it + kCoopStages - 1) {
+      fence_proxy_async_smem();
+      issue_group(p, sm, issued % kCoopStages, rec_base, b, kvh, w0 + kCoop * issued,
+                  min(kCoop, w1 - w0 - kCoop * issued), wait_win, wait_val);
+      ++issued;
+    }
+
+    // ---- common running max; rescale when it grows ------------------------
+    {
+      float mn0 = m_run[0], mn1 = m_run[1];
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const float2 x = *reinterpret_cast<const float2*>(&sm.mw[w][2 * t]);
+        mn0 = fmaxf(mn0, x.x);
+        mn1 = fmaxf(mn1, x.y);
+      }
+      if (__any_sync(0xffffffffu, mn0 > m_run[0] || mn1 > m_run[1])) {
+        const float a0 = fast_exp2((m_run[0] - mn0) * kLog2e), a1 = fast_exp2((m_run[1] - mn1) * kLog2e);
+        l_part[0] *= a0;
+        l_part[1] *= a1;
+#pragma unroll
+        for (int k = 0; k < kMods; ++k) {
+          S_part[k][0] *= a0;
+          S_part[k][1] *= a1;
+        }
+        pv_scale(pv, a0, a1);
+        m_run[0] = mn0;
+        m_run[1] = mn1;
+      }
+    }
+    const float ms0 = m_run[0] * kLog2e, ms1 = m_run[1] * kLog2e;
+
+    // ---- this warp's window: p, the sums, the value-product B operand --------
+    if (have) {
+      const __half* sig = reinterpret_cast<const __half*>(rec + 2560);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float p0 = fast_exp2(fmaf(sc[h][0], kLog2e, -ms0));
+        const float p1 = fast_exp2(fmaf(sc[h][1], kLog2e, -ms1));
+        const float p2 = fast_exp2(fmaf(sc[h][2], kLog2e, -ms0));
+        const float p3 = fast_exp2(fmaf(sc[h][3], kLog2e, -ms1));
+        l_part[0] += p0 + p2;
+        l_part[1] += p1 + p3;
+        const float sgA = __half2float(sig[tokA[h]]), sgB = __half2float(sig[tokB[h]]);
+        const float w0v = p0 * sgA, w1v = p1 * sgA, w2v = p2 * sgB, w3v = p3 * sgB;
+        uint32_t bv0[4], bv1[4];  // per plane {hi b0, hi b1, lo b0, lo b1}, transposed
+        split_pair_t(w0v * kV0, w1v * kV0, bv0[0], bv0[2]);
+        split_pair_t(w2v * kV0, w3v * kV0, bv0[1], bv0[3]);
+        split_pair_t(w0v * kV1, w1v * kV1, bv1[0], bv1[2]);
+        split_pair_t(w2v * kV1, w3v * kV1, bv1[1], bv1[3]);
+        sm.u.c.pfrag[warp][h][0][lane] = make_uint4(bv0[0], bv0[1], bv0[2], bv0[3]);
+        sm.u.c.pfrag[warp][h][1][lane] = make_uint4(bv1[0], bv1[1], bv1[2], bv1[3]);
+        const int mA = min((int)mods[tokA[h]], kMods - 1), mB = min((int)mods[tokB[h]], kMods - 1);
+#pragma unroll
+        for (int k = 0; k < kMods; ++k) {
+          S_part[k][0] += (mA == k ? w0v : 0.0f) + (mB == k ? w2v : 0.0f);
+          S_part[k][1] += (mA == k ? w1v : 0.0f) + (mB == k ? w3v : 0.0f);
+        }
+        const uint32_t tm = __reduce_or_sync(0xffffffffu, (1u << mA) | (1u << mB));
+        if (lane == 0) sm.tmask[warp][h] = tm;
+      }
+    } else if (lane == 0) {
+      sm.tmask[warp][0] = 0u;
+      sm.tmask[warp][1] = 0u;
+    }
+    __syncthreads();
+
+    // ---- value product of the group for this warp's 32 channels -------------
+#pragma unroll 1
+    for (int ww = 0; ww < kCoop; ++ww) {
+      const uint8_t* rv = stg + ww * kRec22 + 1536;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t tm = sm.tmask[ww][h];
+        if (tm == 0u) continue;  // no window (the group's tail)
+        const uint4 u = *reinterpret_cast<const uint4*>(rv + 4 * (h * kHeadDim + 32 * warp + 4 * g));
+        const uint4 f0 = sm.u.c.pfrag[ww][h][0][lane], f1 = sm.u.c.pfrag[ww][h][1][lane];
+        uint32_t a0[2][4], a1[2][4];
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+          const uint32_t wg = mt ? u.z : u.x, wg8 = mt ? u.w : u.y;
+          const uint32_t r[4] = {rotl(wg, rlo), rotl(wg8, rlo), rotl(wg, rhi), rotl(wg8, rhi)};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            a0[mt][j] = r[j] & kPlane0;
+            a1[mt][j] = r[j] & kPlane1;
+          }
+        }
+        if ((tm & (tm - 1u)) == 0u) {  // one modality (the common case)
+          pv_activate(pv, __ffs(tm) - 1);
+          pv_tile(pv, a0, a1, f0, f1, 0xFFFFFFFFu, 0xFFFFFFFFu);
+        } else {  // masked products, one per modality present, the active one first
+          const uint8_t* md = stg + kCoop * kRec22 + ww * kWindow + 16 * h;
+          // k-slots of this lane's B registers: 2t, 2t+1 -> tokens t, t+8; 2t+8, 2t+9 -> t+4, t+12
+          const int mk0 = min((int)md[t], kMods - 1), mk1 = min((int)md[t + 8], kMods - 1);
+          const int mk2 = min((int)md[t + 4], kMods - 1), mk3 = min((int)md[t + 12], kMods - 1);
+          uint32_t todo = tm;
+          int mm = (pv.cur >= 0 && ((todo >> pv.cur) & 1u)) ? pv.cur : __ffs(todo) - 1;
+#pragma unroll 1
+          while (true) {
+            pv_activate(pv, mm);
+            const uint32_t m01 = (mk0 == mm ? 0x0000FFFFu : 0u) | (mk1 == mm ? 0xFFFF0000u : 0u);
+            const uint32_t m23 = (mk2 == mm ? 0x0000FFFFu : 0u) | (mk3 == mm ? 0xFFFF0000u : 0u);
+            pv_tile(pv, a0, a1, f0, f1, m01, m23);
+            todo &= ~(1u << mm);
+            if (!todo) break;
+            mm = __ffs(todo) - 1;
+          }
+        }
+      }
+    }
+  }
+
+  if (failed_at >= 0) {
+    // a copy did not complete in time: report it, wait (bounded) for the copies
+    // still in flight, and leave an empty split
+    if (threadIdx.x == 0) {
+      set_error(p.error_word, OMNIKV_DEVERR_TIMEOUT);
+      for (int j = failed_at; j < issued; ++j) mbar_wait_bounded(&sm.cbar[j % kCoopStages], (j / kCoopStages) & 1, kWaitLimitNs);
+    }
+    m_run[0] = m_run[1] = -INFINITY;
+    l_part[0] = l_part[1] = 0.0f;
+#pragma unroll
+    for (int k = 0; k < kMods; ++k) S_part[k][0] = S_part[k][1] = 0.0f;
+    pv_scale(pv, 0.0f, 0.0f);
+  }
+  pv_activate(pv, kMods);  // parks the active modality (index kMods: none)
+
+  // ---- sums over the 8 lanes of a column, then over the warps ---------------
+#pragma unroll
+  for (int o = 4; o <= 16; o <<= 1) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      l_part[j] += __shfl_xor_sync(0xffffffffu, l_part[j], o);
+#pragma unroll
+      for (int k = 0; k < kMods; ++k) S_part[k][j] += __shfl_xor_sync(0xffffffffu, S_part[k][j], o);
+    }
+  }
+  if (g == 0) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      sm.red[warp][0][2 * t + j] = l_part[j];
+#pragma unroll
+      for (int k = 0; k < kMods; ++k) sm.red[warp][1 + k][2 * t + j] = S_part[k][j];
+    }
+  }
+  __syncthreads();
+  float Lsum[2], Ssum[kMods][2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    Lsum[j] = 0.0f;
+#pragma unroll
+    for (int k = 0; k < kMods; ++k) Ssum[k][j] = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      Lsum[j] += sm.red[w][0][2 * t + j];
+#pragma unroll
+      for (int k = 0; k < kMods; ++k) Ssum[k][j] += sm.red[w][1 + k][2 * t + j];
+    }
+  }
+  // ---- this warp's channels of the split partial, per query head ------------
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const int hh = 2 * t + j;
+    if (hh >= G) continue;
+    Partial* out = p.partials + ((size_t)b * Hq + kvh * G + hh) * p.num_splits + split;
+#pragma unroll
+    for (int k = 0; k < kMods; ++k)
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        const float c0 = vc0 * Ssum[k][j];
+        *reinterpret_cast<float2*>(&out->acc[k][32 * warp + 4 * g + 2 * mt]) =
+            make_float2(pv.st[k][mt][j] + c0, pv.st[k][mt][j + 2] + c0);
+      }
+    if (warp == 0 && g == 0) {
+      out->m = m_run[j];
+      out->l = Lsum[j];
+    }
+  }
+}
+
 // Score B operand for lane (g, t), chunk kc, plane P: k-slots 2t, 2t+1 hold
 // channels 32t + kc and 32t + kc + 8, k-slots 2t+8, 2t+9 hold 32t + 16 + kc and
 // 32t + 24 + kc; column g is query head g. Entry {hi(slots 2t..), hi(slots
@@ -935,12 +1386,13 @@ __device__ __forceinline__ void build_score_operand(DecodeSmem& sm, float k0scal
   }
 }
 
-// One decode CTA: split `split` of kv head kvh of sequence b. kGen: the build of
-// the kernel that serves 4-bit caches (CUDA-core path only, no TMEM, more CTAs
-// per SM); otherwise the tensor-core path, with the CUDA-core path for 2-bit
-// codebooks that are not symmetric.
-template <bool kGen>
+// One decode CTA: split `split` of kv head kvh of sequence b. kBody: the 4-bit
+// build (CUDA-core path only, no TMEM, more CTAs per SM), or a tensor-core build
+// (per-warp or cooperative body), whose kernels fall back to the CUDA-core path for
+// 2-bit codebooks that are not symmetric.
+template <int kBody>
 __device__ __forceinline__ void decode_cta(const DecodeParams& p, DecodeSmem& sm, int b, int kvh, int split) {
+  constexpr bool kGen = kBody == kBodyGeneric;
   // ---- independent of the cache (overlaps the previous launch of the stream):
   // query rotation, score operand, L2 prefetch of this split's share of the
   // value bases (read by the combine)
@@ -977,7 +1429,11 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, DecodeSmem& sm
     }
     return;
   }
-  if (!kGen && fast) {
+  if (kBody == kBodyCoop && fast) {
+    decode_coop(p, sm, b, kvh, split, (v1 - v0) * 128.0f, (v2 - v0) * 0.5f, v0);
+    return;
+  }
+  if (kBody == kBodyWarp && fast) {
     prime_pipeline(p, sm, b, kvh, w0, w1);
     if (threadIdx.x < 32) tmem_alloc(&sm.tmem_base, kTmemCols);
     tc_fence_before();
@@ -994,22 +1450,25 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, DecodeSmem& sm
   decode_generic<kGen>(p, sm, b, kvh, split);
 }
 
-constexpr int kGenCtasPerSm = 4;  // the 4-bit build: registers for 4 resident CTAs
+// Registers for this many resident CTAs per SM: per-warp body 2 (its accumulators
+// need ~240 registers), cooperative body 3, 4-bit build 4.
+__host__ __device__ constexpr int body_ctas_per_sm(int body) {
+  return body == kBodyWarp ? 2 : body == kBodyCoop ? 3 : 4;
+}
 
-template <bool kGen>
-__global__ void __launch_bounds__(kThreads, kGen ? kGenCtasPerSm : kCtasPerSm)
-    decode_split_k_kernel(const DecodeParams p) {
+template <int kBody>
+__global__ void __launch_bounds__(kThreads, body_ctas_per_sm(kBody)) decode_split_k_kernel(const DecodeParams p) {
   __shared__ DecodeSmem sm;
   griddep_launch_dependents();
-  decode_cta<kGen>(p, sm, blockIdx.z, blockIdx.y, blockIdx.x);
+  decode_cta<kBody>(p, sm, blockIdx.z, blockIdx.y, blockIdx.x);
 }
 
 // Decode step: CTAs [0, batch * H) append one token to (sequence, kv head) and
 // then publish the new length in the step flag; the others are decode CTAs
-// (split fastest, then kv head, then sequence). Only the warp decoding the
-// window that receives the token waits for the flag, before copying it.
-template <bool kGen>
-__global__ void __launch_bounds__(kThreads, kGen ? kGenCtasPerSm : kCtasPerSm)
+// (split fastest, then kv head, then sequence). Only the copy of the window that
+// receives the token waits for the flag.
+template <int kBody>
+__global__ void __launch_bounds__(kThreads, body_ctas_per_sm(kBody))
     decode_step_kernel(const DecodeParams p, const WriteParams w) {
   __shared__ DecodeSmem sm;
   static_assert(sizeof(WindowSmem) <= sizeof(DecodeSmem), "append uses the decode shared memory");
@@ -1038,7 +1497,7 @@ __global__ void __launch_bounds__(kThreads, kGen ? kGenCtasPerSm : kCtasPerSm)
     return;
   }
   const int r = blockIdx.x - nappend;
-  decode_cta<kGen>(p, sm, r / (p.num_splits * H), (r / p.num_splits) % H, r % p.num_splits);
+  decode_cta<kBody>(p, sm, r / (p.num_splits * H), (r / p.num_splits) % H, r % p.num_splits);
 }
 
 // Several decode CTAs share an SM only if the SM's unified L1 / shared memory is
@@ -1056,72 +1515,92 @@ cudaError_t prefer_shared_carveout(Kernel kernel, std::atomic<uint64_t>& done) {
   return e;
 }
 
-std::atomic<uint64_t> g_carveout[4];  // decode <fast, gen>, step <fast, gen>
+std::atomic<uint64_t> g_carveout[2][kNumBodies];  // [decode, step][body]
 
-cudaError_t prepare_kernels(bool gen) {
-  cudaError_t e = gen ? prefer_shared_carveout(decode_split_k_kernel<true>, g_carveout[1])
-                      : prefer_shared_carveout(decode_split_k_kernel<false>, g_carveout[0]);
+template <int kBody>
+cudaError_t prepare_body() {
+  const cudaError_t e = prefer_shared_carveout(decode_split_k_kernel<kBody>, g_carveout[0][kBody]);
   if (e != cudaSuccess) return e;
-  return gen ? prefer_shared_carveout(decode_step_kernel<true>, g_carveout[3])
-             : prefer_shared_carveout(decode_step_kernel<false>, g_carveout[2]);
+  return prefer_shared_carveout(decode_step_kernel<kBody>, g_carveout[1][kBody]);
+}
+
+cudaError_t prepare_kernels(int body) {
+  return body == kBodyWarp ? prepare_body<kBodyWarp>()
+       : body == kBodyCoop ? prepare_body<kBodyCoop>()
+                           : prepare_body<kBodyGeneric>();
+}
+
+template <int kBody>
+cudaError_t body_attributes(cudaFuncAttributes* a) {
+  cudaError_t e = cudaFuncGetAttributes(a, decode_step_kernel<kBody>);
+  if (e != cudaSuccess) return e;
+  cudaFuncAttributes a2;
+  e = cudaFuncGetAttributes(&a2, decode_split_k_kernel<kBody>);
+  if (e != cudaSuccess) return e;
+  // size both kernels of the body by the larger register count
+  if (a2.numRegs > a->numRegs) a->numRegs = a2.numRegs;
+  if (a2.sharedSizeBytes > a->sharedSizeBytes) a->sharedSizeBytes = a2.sharedSizeBytes;
+  return cudaSuccess;
 }
 
 }  // namespace
 
-bool decode_uses_generic_build(int key_bits, int value_bits) { return key_bits != 2 || value_bits != 2; }
+int decode_body(int key_bits, int value_bits, int split_windows) {
+  if (key_bits != 2 || value_bits != 2) return kBodyGeneric;
+  return split_windows <= kCoopMaxWindows ? kBodyCoop : kBodyWarp;
+}
 
-// Resident decode CTAs per SM, from the kernel's registers and shared memory and
-// the TMEM columns each CTA allocates (computed from the attributes rather than
-// the runtime occupancy query, which does not report the residency seen on
-// sm_100a for this kernel). Cached per device and build.
-int decode_ctas_per_sm(int key_bits, int value_bits) {
-  static std::atomic<int> cached[2][64];
-  const bool gen = decode_uses_generic_build(key_bits, value_bits);
-  const int fallback = gen ? kGenCtasPerSm : kCtasPerSm;
+// Resident decode CTAs per SM of a body, from its kernels' registers and shared
+// memory and the TMEM columns each CTA allocates (computed from the attributes
+// rather than the runtime occupancy query, which does not report the residency
+// seen on sm_100a for these kernels). Cached per device and body.
+int decode_ctas_per_sm(int body) {
+  static std::atomic<int> cached[kNumBodies][64];
+  if (body < 0 || body >= kNumBodies) body = kBodyGeneric;
+  const int fallback = body_ctas_per_sm(body);
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return fallback;
   if (dev < 64) {
-    const int c = cached[gen][dev].load(std::memory_order_relaxed);
+    const int c = cached[body][dev].load(std::memory_order_relaxed);
     if (c > 0) return c;
   }
   cudaFuncAttributes a;
   int regs_sm = 0, smem_sm = 0, smem_rsv = 0;
-  if (prepare_kernels(gen) != cudaSuccess ||
-      cudaFuncGetAttributes(&a, gen ? decode_step_kernel<true> : decode_step_kernel<false>) != cudaSuccess ||
+  const cudaError_t ea = body == kBodyWarp ? body_attributes<kBodyWarp>(&a)
+                       : body == kBodyCoop ? body_attributes<kBodyCoop>(&a)
+                                           : body_attributes<kBodyGeneric>(&a);
+  if (prepare_kernels(body) != cudaSuccess || ea != cudaSuccess ||
       cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&smem_rsv, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess)
     return fallback;
-  // the step build uses at least as many registers as the decode build: size both by it
-  cudaFuncAttributes a2;
-  if (cudaFuncGetAttributes(&a2, gen ? decode_split_k_kernel<true> : decode_split_k_kernel<false>) == cudaSuccess &&
-      a2.numRegs > a.numRegs)
-    a.numRegs = a2.numRegs;
   const int warp_regs = ((a.numRegs * 32 + 255) / 256) * 256;  // allocated per warp in units of 256
   const int by_regs = regs_sm / (warp_regs * kWarps);
   const int by_smem = smem_sm / ((int)a.sharedSizeBytes + smem_rsv);
-  const int by_tmem = gen ? 64 : 512 / (int)kTmemCols;  // the 4-bit build holds no tensor memory
+  const int by_tmem = body == kBodyWarp ? 512 / (int)kTmemCols : 64;  // only the per-warp body holds tensor memory
   const int n = max(1, min(by_regs, min(by_smem, by_tmem)));
-  if (dev < 64) cached[gen][dev].store(n, std::memory_order_relaxed);
+  if (dev < 64) cached[body][dev].store(n, std::memory_order_relaxed);
   return n;
 }
 
 cudaError_t launch_decode_step(const DecodeParams& p, const WriteParams& w, cudaStream_t stream) {
-  const bool gen = decode_uses_generic_build(p.key_bits, p.value_bits);
-  const cudaError_t e = prepare_kernels(gen);
+  const int body = decode_body(p.key_bits, p.value_bits, p.split_windows);
+  const cudaError_t e = prepare_kernels(body);
   if (e != cudaSuccess) return e;
-  const int ctas = p.batch * p.num_kv_heads * (1 + p.num_splits);
-  return gen ? launch_pdl(decode_step_kernel<true>, dim3(ctas), dim3(kThreads), 0, stream, p, w)
-             : launch_pdl(decode_step_kernel<false>, dim3(ctas), dim3(kThreads), 0, stream, p, w);
+  const dim3 grid(p.batch * p.num_kv_heads * (1 + p.num_splits));
+  return body == kBodyWarp ? launch_pdl(decode_step_kernel<kBodyWarp>, grid, dim3(kThreads), 0, stream, p, w)
+       : body == kBodyCoop ? launch_pdl(decode_step_kernel<kBodyCoop>, grid, dim3(kThreads), 0, stream, p, w)
+                           : launch_pdl(decode_step_kernel<kBodyGeneric>, grid, dim3(kThreads), 0, stream, p, w);
 }
 
 cudaError_t launch_decode(const DecodeParams& p, int batch, cudaStream_t stream) {
-  const bool gen = decode_uses_generic_build(p.key_bits, p.value_bits);
-  const cudaError_t e = prepare_kernels(gen);
+  const int body = decode_body(p.key_bits, p.value_bits, p.split_windows);
+  const cudaError_t e = prepare_kernels(body);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.num_splits, p.num_kv_heads, batch);
-  return gen ? launch_pdl(decode_split_k_kernel<true>, grid, dim3(kThreads), 0, stream, p)
-             : launch_pdl(decode_split_k_kernel<false>, grid, dim3(kThreads), 0, stream, p);
+  const dim3 grid(p.num_splits, p.num_kv_heads, batch);
+  return body == kBodyWarp ? launch_pdl(decode_split_k_kernel<kBodyWarp>, grid, dim3(kThreads), 0, stream, p)
+       : body == kBodyCoop ? launch_pdl(decode_split_k_kernel<kBodyCoop>, grid, dim3(kThreads), 0, stream, p)
+                           : launch_pdl(decode_split_k_kernel<kBodyGeneric>, grid, dim3(kThreads), 0, stream, p);
 }
 
 }  // namespace omnikv

@@ -103,7 +103,14 @@ cudaError_t launch_decode(const DecodeParams& p, int batch, cudaStream_t stream)
 // sequence, described by w) followed by the decode CTAs of p.
 cudaError_t launch_decode_step(const DecodeParams& p, const WriteParams& w, cudaStream_t stream);
 
-int decode_ctas_per_sm(int key_bits, int value_bits);  // resident decode CTAs per SM on the current device
+// Decode kernel bodies. 2-bit caches: the per-warp body (each warp streams its own
+// run of windows; registers for 2 CTAs per SM) for long splits, the cooperative
+// body (the CTA takes 4 windows at a time; 3 CTAs per SM) for splits of at most
+// kCoopMaxWindows windows; 4-bit caches: the CUDA-core build.
+enum DecodeBody { kBodyWarp = 0, kBodyCoop = 1, kBodyGeneric = 2, kNumBodies = 3 };
+constexpr int kCoopMaxWindows = 16;
+int decode_body(int key_bits, int value_bits, int split_windows);
+int decode_ctas_per_sm(int body);  // resident decode CTAs per SM of a body on the current device
 cudaError_t launch_combine(const CombineParams& p, int batch, cudaStream_t stream);
 
 }  // namespace omnikv

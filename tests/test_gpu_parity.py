@@ -109,8 +109,11 @@ def test_chunked_writes_and_tail(cuda_device, bits):
     check_decode(gpu_decode(consts, upload_oracle_cache(oc, cuda_device), q), ref, "bits=%d" % bits)
 
 
-@pytest.mark.parametrize("splits", [1, 2, 7, 64, 200])
+@pytest.mark.parametrize("splits", [1, 2, 3, 5, 7, 64, 200])
 def test_decode_split_counts(cuda_device, splits):
+    """1,000 tokens (32 windows): one split of 32 windows runs the per-warp body; 16, 11,
+    7, 5 and 1 windows per split run the cooperative body (whole and partial window
+    groups)."""
     m = _abi()
     spec, seed = WORKLOADS["tiny"], 5
     params, consts, ocfg = make_layer(spec, seed, 0, cuda_device)
