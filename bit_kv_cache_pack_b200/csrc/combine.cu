@@ -7,9 +7,11 @@
 // block of 128:
 //   0. before waiting on the decode launch: this warp's 4 rows of U_m for the 3
 //      modalities go into registers (they do not depend on the decode);
-//   1. warp 0: M = max_s m_s, weights e_s = exp(m_s - M), l = sum_s l_s e_s;
+//   1. warp 0: M = max_s m_s, weights e_s = exp(m_s - M), l = sum_s l_s e_s,
+//      each lane's (m, l) pairs loaded together;
 //   2. a_m[c] = sum_s acc_{s,m}[c] e_s / l, the splits read as 16-byte vectors,
-//      two threads per vector column, splits of weight 0 skipped;
+//      two threads per vector column, 16 loads in flight per thread, splits of
+//      weight 0 not read;
 //   3. out[j] = sum_m sum_c U_m[j][c] a_m[c] for the block's rows: one warp per 4
 //      rows, lanes over c, warp reduction.
 // The row blocks of a head merge the same partials (read from L2); splitting the
@@ -41,7 +43,8 @@ combine_inverse_rotate_kernel(const CombineParams p) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qh = kvh * G + g;
 
-  __shared__ float w[kMaxSplitsSmem];
+  __shared__ float w[kMaxSplitsSmem];   // split maxima, then weights
+  __shared__ float wl[kMaxSplitsSmem];  // split denominators
   __shared__ __align__(16) float4 red[2][96];
   __shared__ __align__(16) float a[kMods * kHeadDim];
   __shared__ float s_l;
@@ -67,13 +70,28 @@ combine_inverse_rotate_kernel(const CombineParams p) {
     if (L >= 0 && L + p.len_add <= p.cap_tokens) p.seq_lens[b] = L + p.len_add;
   }
 
-  // ---- 1. split weights
+  // ---- 1. split weights (warp 0): every lane loads (m, l) of all its splits at
+  // once (one memory round trip for up to 128 splits), then the max, the weights
+  // e_s and l = sum_s l_s e_s
   if (warp == 0) {
+    constexpr int kPer = 4;  // splits per lane per pass
     float M = -INFINITY;
-    for (int s = lane; s < S; s += 32) {
-      const float ms = part[s].m;
-      w[s] = ms;
-      M = fmaxf(M, ms);
+    for (int base = 0; base < S; base += 32 * kPer) {
+      float2 ml[kPer];
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {
+        const int s = base + 32 * i + lane;
+        ml[i] = s < S ? *reinterpret_cast<const float2*>(&part[s].m) : make_float2(-INFINITY, 0.0f);
+      }
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {
+        const int s = base + 32 * i + lane;
+        if (s < S) {
+          w[s] = ml[i].x;
+          wl[s] = ml[i].y;
+        }
+        M = fmaxf(M, ml[i].x);
+      }
     }
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
@@ -82,7 +100,7 @@ combine_inverse_rotate_kernel(const CombineParams p) {
       const float ms = w[s];
       const float e = (ms == -INFINITY) ? 0.0f : expf(ms - M);
       w[s] = e;
-      if (e != 0.0f) l += part[s].l * e;
+      if (e != 0.0f) l += wl[s] * e;
     }
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
@@ -90,20 +108,29 @@ combine_inverse_rotate_kernel(const CombineParams p) {
   }
   __syncthreads();
 
-  // ---- 2. weighted sum over splits: column c4 (of 96 float4), half h of the splits
+  // ---- 2. weighted sum over splits: column c4 (of 96 float4), half h of the
+  // splits, kU loads in flight per thread (splits of weight 0 are not read)
   {
     const int c4 = tid & 127, h = tid >> 7;
     if (c4 < 96) {
+      constexpr int kU = 16;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-      for (int s = h; s < S; s += 2) {
-        const float e = w[s];
-        if (e == 0.0f) continue;  // empty split, or negligible weight
-        const float4 v = reinterpret_cast<const float4*>(part[s].acc)[c4];
-        acc.x = fmaf(v.x, e, acc.x);
-        acc.y = fmaf(v.y, e, acc.y);
-        acc.z = fmaf(v.z, e, acc.z);
-        acc.w = fmaf(v.w, e, acc.w);
+      for (int s0 = h; s0 < S; s0 += 2 * kU) {
+        float4 v[kU];
+        float e[kU];
+#pragma unroll
+        for (int i = 0; i < kU; ++i) {
+          const int s = s0 + 2 * i;
+          e[i] = s < S ? w[s] : 0.0f;
+          v[i] = e[i] != 0.0f ? reinterpret_cast<const float4*>(part[s].acc)[c4] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int i = 0; i < kU; ++i) {
+          acc.x = fmaf(v[i].x, e[i], acc.x);
+          acc.y = fmaf(v[i].y, e[i], acc.y);
+          acc.z = fmaf(v[i].z, e[i], acc.z);
+          acc.w = fmaf(v[i].w, e[i], acc.w);
+        }
       }
       red[h][c4] = acc;
     }
