@@ -215,6 +215,7 @@ struct GenSmem {                 // laid over DecodeSmem::stage
   float dk[16], dv[16];           // c_j - c_0 (keys), c_j (values)
   float wmax[kWarps][kMaxGroup];
   uint64_t bar[kGenStages];
+  uint32_t runs;                  // bit t: token t of the current window starts a run of one modality
 };
 static_assert(sizeof(GenSmem) <= sizeof(DecodeSmem::u), "generic path shared memory");
 
@@ -344,6 +345,13 @@ __device__ void decode_generic_t(const DecodeParams& p, DecodeSmem& sm, int b, i
       alpha[h] = (mn == -INFINITY) ? 1.0f : fast_exp2((m_run[h] - mn) * kLog2e);
       m_run[h] = mn;
     }
+    // ---- where the window's modality runs start (warp 0; read after the barrier)
+    if (warp == 0) {
+      const int mt = min((int)mods[lane], kMods - 1);
+      const int mp = lane > 0 ? min((int)mods[lane - 1], kMods - 1) : -1;
+      const uint32_t starts = __ballot_sync(0xffffffffu, mt != mp);
+      if (lane == 0) g.runs = starts;
+    }
     // ---- p = exp(score - max); thread (st, sq) stores heads 2 sq, 2 sq + 1 of token st
     {
       const float sgm = __half2float(sig[st]);
@@ -355,31 +363,55 @@ __device__ void decode_generic_t(const DecodeParams& p, DecodeSmem& sm, int b, i
       }
     }
     __syncthreads();
-    // ---- values: channel c = tid over the window's valid tokens
+    // ---- values: channel c = tid over the window's valid tokens, taken in runs
+    // of one modality (one accumulator set per run, no per-token selection)
     {
+      bool grew = false;
 #pragma unroll
-      for (int m = 0; m < kMods; ++m)
+      for (int h = 0; h < kMaxGroup; ++h) grew |= alpha[h] != 1.0f;
+      if (grew) {  // the same decision in every thread
 #pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h) acc[m][h] *= alpha[h];
+        for (int m = 0; m < kMods; ++m)
+#pragma unroll
+          for (int h = 0; h < kMaxGroup; ++h) acc[m][h] *= alpha[h];
+      }
       const int nvalid = min(kWindow, T - wi * kWindow);
-      for (int t = 0; t < nvalid; ++t) {
-        const uint32_t code = (vw[(t / vcpw) * kHeadDim + tid] >> (VB * (t % vcpw))) & vmask;
-        const float d = g.dv[code];
-        const float4 pa = *reinterpret_cast<const float4*>(&g.pw[t][0]);
-        const float4 pb = *reinterpret_cast<const float4*>(&g.pw[t][4]);
+      const uint32_t starts = g.runs;
+      for (int t = 0; t < nvalid;) {
         const int mod = min((int)mods[t], kMods - 1);  // the same for every thread
+        const uint32_t later = starts & ~((2u << t) - 1u);  // runs starting after token t
+        const int e = later ? min(nvalid, __ffs(later) - 1) : nvalid;
+        float a[kMaxGroup];
 #pragma unroll
-        for (int m = 0; m < kMods; ++m) {
-          if (mod != m) continue;
-          acc[m][0] = fmaf(pa.x, d, acc[m][0]);
-          acc[m][1] = fmaf(pa.y, d, acc[m][1]);
-          acc[m][2] = fmaf(pa.z, d, acc[m][2]);
-          acc[m][3] = fmaf(pa.w, d, acc[m][3]);
-          acc[m][4] = fmaf(pb.x, d, acc[m][4]);
-          acc[m][5] = fmaf(pb.y, d, acc[m][5]);
-          acc[m][6] = fmaf(pb.z, d, acc[m][6]);
-          acc[m][7] = fmaf(pb.w, d, acc[m][7]);
+        for (int h = 0; h < kMaxGroup; ++h) a[h] = 0.0f;
+#pragma unroll
+        for (int m = 0; m < kMods; ++m)
+          if (m == mod) {
+#pragma unroll
+            for (int h = 0; h < kMaxGroup; ++h) a[h] = acc[m][h];
+          }
+#pragma unroll 4
+        for (int tt = t; tt < e; ++tt) {
+          const uint32_t code = (vw[(tt / vcpw) * kHeadDim + tid] >> (VB * (tt % vcpw))) & vmask;
+          const float d = g.dv[code];
+          const float4 pa = *reinterpret_cast<const float4*>(&g.pw[tt][0]);
+          const float4 pb = *reinterpret_cast<const float4*>(&g.pw[tt][4]);
+          a[0] = fmaf(pa.x, d, a[0]);
+          a[1] = fmaf(pa.y, d, a[1]);
+          a[2] = fmaf(pa.z, d, a[2]);
+          a[3] = fmaf(pa.w, d, a[3]);
+          a[4] = fmaf(pb.x, d, a[4]);
+          a[5] = fmaf(pb.y, d, a[5]);
+          a[6] = fmaf(pb.z, d, a[6]);
+          a[7] = fmaf(pb.w, d, a[7]);
         }
+#pragma unroll
+        for (int m = 0; m < kMods; ++m)
+          if (m == mod) {
+#pragma unroll
+            for (int h = 0; h < kMaxGroup; ++h) acc[m][h] = a[h];
+          }
+        t = e;
       }
     }
     __syncthreads();  // stage s and pw are free again
