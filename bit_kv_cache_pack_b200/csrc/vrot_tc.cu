@@ -11,9 +11,10 @@
 //     B = U_m^T split into fp16 high and low parts (U = hi + lo to ~22 bits);
 //     both in shared memory in the K-major 128-byte-swizzled layout, written with
 //     16-byte stores whose chunk index is XOR-ed with the row (conflict free);
-//     U_m arrives as one 64 KB bulk copy (fp32) into a staging buffer, is
-//     converted once, and stays while the following tiles need the same
-//     modality; the next basis needed is prefetched into the staging buffer;
+//     two converted bases stay resident (slots tagged with modality and kv head,
+//     least recently used replaced), so a stream that alternates two modalities
+//     (audio and video blocks) converts each basis once; a missing basis is read
+//     from global memory (coalesced over the output channel) and converted;
 //   * one elected thread issues tcgen05.mma kind::f16 (M = N = 128, K = 16,
 //     8 k-steps x {hi, lo}) into a 128-column fp32 accumulator in TMEM and
 //     commits to an mbarrier (bounded wait);
@@ -38,25 +39,22 @@ constexpr int kTile = 128;                 // tokens per tile = MMA M
 constexpr int kVThreads = 512;             // 16 warps: 4 per TMEM lane quarter
 constexpr uint32_t kTmemCols = 128;        // one fp32 accumulator of N = 128 columns
 constexpr uint64_t kMmaWaitNs = 2000000000ull;
-constexpr uint32_t kUBytes = kHeadDim * kHeadDim * sizeof(float);
 
 // operand: [2 k-atoms][128 rows][128 B], 16-byte chunks XOR-swizzled by row % 8
 constexpr int kOperandBytes = 2 * 128 * 128;   // 32 KB of fp16
 
+constexpr int kSlots = 2;  // converted bases resident in shared memory
+
 struct __align__(1024) VrotSmem {
-  uint8_t a[2][kOperandBytes];     // values (A), double buffer
-  uint8_t bhi[kOperandBytes];      // U_m^T high part (B)
-  uint8_t blo[kOperandBytes];      // U_m^T low part (B)
-  float ustage[kHeadDim * kHeadDim];   // U_m (fp32, row-major) staged by one bulk copy
-  uint8_t codes[kHeadDim][kTile + 4];  // code of (channel, token); rows padded against bank conflicts
+  uint8_t a[2][kOperandBytes];          // values (A), double buffer
+  uint8_t b[kSlots][2][kOperandBytes];  // U_m^T per slot: high, low part (B)
+  uint8_t codes[kHeadDim][kTile + 4];   // code of (channel, token); rows padded against bank conflicts
   float sigma[kTile];
   uint8_t mods[kTile];
-  CodeBound bv[15];                    // value code decision bounds
+  CodeBound bv[15];                     // value code decision bounds
   uint64_t mma_bar;
-  uint64_t u_bar;
   uint32_t tmem_base;
-  int present;                         // modality bits of the current tile
-  int present_next;                    // ... of the next tile
+  int present;                          // modality bits of the current tile
 };
 
 __device__ __forceinline__ uint32_t swz_offset(int row, int k16) {  // k16: 16-byte chunk index 0..15 along K
@@ -102,13 +100,20 @@ struct TileItem {
   bool valid;
 };
 
-__device__ __forceinline__ TileItem tile_item(const WriteParams& p, int i, int tiles_per_seq) {
+// (lb, lL0): the last sequence whose length was read and that length (the
+// lengths do not change during the launch), so that consecutive tiles of one
+// sequence wait on no global load.
+__device__ __forceinline__ TileItem tile_item(const WriteParams& p, int i, int tiles_per_seq, int& lb, int& lL0) {
   TileItem t;
   const int H = p.num_kv_heads;
   const int bh = i / tiles_per_seq, tile = i - bh * tiles_per_seq;
   t.b = bh / H;
   t.h = bh - t.b * H;
-  t.L0 = p.seq_lens[t.b];
+  if (t.b != lb) {
+    lL0 = p.seq_lens[t.b];
+    lb = t.b;
+  }
+  t.L0 = lL0;
   t.wt0 = 0;
   t.nwin = 0;
   t.valid = false;
@@ -161,6 +166,33 @@ __device__ __forceinline__ void gather_present(int* dst, int mod) {
   if ((threadIdx.x & 31) == 0 && bits) atomicOr(dst, (int)bits);
 }
 
+// U^T (U: one basis, fp32 row-major, global memory) -> slot `slot` of B as fp16
+// high and low parts: thread = output channel j = B row, 16-byte chunks 4 q ..
+// 4 q + 3 along K; the 32 loads of a thread are in flight together.
+__device__ __forceinline__ void convert_basis(VrotSmem& sm, int slot, const float* U, int tid) {
+  const int j = tid & (kHeadDim - 1), q = tid >> 7;
+  float u[4][8];
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) u[kk][e] = U[(size_t)(8 * (4 * q + kk) + e) * kHeadDim + j];
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk) {
+    const int k16 = 4 * q + kk;
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const __half2 hv = __floats2half2_rn(u[kk][2 * e], u[kk][2 * e + 1]);
+      const float2 hf = __half22float2(hv);
+      const __half2 lv = __floats2half2_rn(u[kk][2 * e] - hf.x, u[kk][2 * e + 1] - hf.y);
+      hi[e] = *reinterpret_cast<const uint32_t*>(&hv);
+      lo[e] = *reinterpret_cast<const uint32_t*>(&lv);
+    }
+    *reinterpret_cast<uint4*>(sm.b[slot][0] + swz_offset(j, k16)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(sm.b[slot][1] + swz_offset(j, k16)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+  }
+}
+
 // Epilogue of one modality pass: warp w reads TMEM lanes 32 (w % 4) .. + 31
 // (token rows) and columns 32 (w / 4) .. + 31 (channels); each lane computes its
 // token's codes code = #{j : v' / sigma > t_j} (0 where sigma == 0) for the
@@ -202,14 +234,13 @@ __global__ void __launch_bounds__(kVThreads, 1) vrot_tc_kernel(const WriteParams
   if (warp == 0) tmem_alloc(&sm.tmem_base, kTmemCols);
   if (tid == 0) {
     mbar_init(&sm.mma_bar, 1);
-    mbar_init(&sm.u_bar, 1);
     fence_barrier_init();
     sm.present = 0;
-    sm.present_next = 0;
   }
   // the first tile's values
   int i = i0;
-  TileItem cur = tile_item(p, i, tiles_per_seq);
+  int last_b = -1, last_L0 = 0;
+  TileItem cur = tile_item(p, i, tiles_per_seq, last_b, last_L0);
   uint4 regs[kChunks];
   int mod_tok;
   load_tile(p, cur, tid, regs, mod_tok);
@@ -224,24 +255,21 @@ __global__ void __launch_bounds__(kVThreads, 1) vrot_tc_kernel(const WriteParams
   const uint32_t tmem = sm.tmem_base;
 
   int buf = 0;
-  int bmod = -1, bhead = -1;    // basis currently converted into B (modality, kv head)
-  int upend = -1, uhead = -1;   // basis in flight into the staging buffer
-  uint32_t u_phase = 0, mma_phase = 0;
+  int slot_m[kSlots], slot_h[kSlots], slot_use[kSlots];  // basis held by each slot (every thread: the same)
+#pragma unroll
+  for (int sl = 0; sl < kSlots; ++sl) {
+    slot_m[sl] = -1;
+    slot_h[sl] = -1;
+    slot_use[sl] = -1;
+  }
+  int npass = 0;  // modality passes so far (slot recency)
+  uint32_t mma_phase = 0;
   bool timed_out = false;
-  const float* Ubase = p.value_rot;
-  auto issue_u = [&](int m, int h) {  // thread 0; every thread tracks the same state
-    if (tid == 0) {
-      mbar_arrive_expect_tx(&sm.u_bar, kUBytes);
-      bulk_copy_g2s(sm.ustage, Ubase + ((size_t)h * kMods + m) * kHeadDim * kHeadDim, kUBytes, &sm.u_bar);
-    }
-    upend = m;
-    uhead = h;
-  };
 
   while (true) {
     // ---- the next tile's loads are issued now and land during this tile's work
     int inext = i + 1;
-    TileItem nxt = tile_item(p, inext < i1 ? inext : i, tiles_per_seq);
+    TileItem nxt = tile_item(p, inext < i1 ? inext : i, tiles_per_seq, last_b, last_L0);
     if (inext >= i1) nxt.valid = false;
     int mod_next;
     load_tile(p, nxt, tid, regs, mod_next);
@@ -276,66 +304,29 @@ __global__ void __launch_bounds__(kVThreads, 1) vrot_tc_kernel(const WriteParams
       __syncthreads();
       const int present = sm.present;
 
-      // ---- one pass per modality present, the one already in B first
+      // ---- one pass per modality present, those whose basis is resident first
       int todo = present;
-      int m = (bhead == cur.h && bmod >= 0 && ((todo >> bmod) & 1)) ? bmod : __ffs(todo) - 1;
       while (todo) {
-        if (!(bmod == m && bhead == cur.h)) {
-          if (!(upend == m && uhead == cur.h)) {
-            if (upend >= 0) {  // a prefetch of another basis is in flight: let it land first
-              if (__syncthreads_or(!mbar_wait_bounded(&sm.u_bar, u_phase, kMmaWaitNs))) {
-                timed_out = true;
-                break;
-              }
-              u_phase ^= 1u;
-              upend = -1;
-            }
-            issue_u(m, cur.h);
-          }
-          if (__syncthreads_or(!mbar_wait_bounded(&sm.u_bar, u_phase, kMmaWaitNs))) {
-            timed_out = true;
-            break;
-          }
-          u_phase ^= 1u;
-          upend = -1;
-          // U_m^T -> B (high, low): thread = output channel j = B row, chunks 4 q .. 4 q + 3
-          {
-            const int j = tid & (kHeadDim - 1), q = tid >> 7;
-            const float* U = sm.ustage + j;
+        int m = -1, slot = -1;
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const int k16 = 4 * q + kk;
-              float u[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) u[e] = U[(8 * k16 + e) * kHeadDim];
-              uint32_t hi[4], lo[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const __half2 hv = __floats2half2_rn(u[2 * e], u[2 * e + 1]);
-                const float2 hf = __half22float2(hv);
-                const __half2 lv = __floats2half2_rn(u[2 * e] - hf.x, u[2 * e + 1] - hf.y);
-                hi[e] = *reinterpret_cast<const uint32_t*>(&hv);
-                lo[e] = *reinterpret_cast<const uint32_t*>(&lv);
-              }
-              *reinterpret_cast<uint4*>(sm.bhi + swz_offset(j, k16)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-              *reinterpret_cast<uint4*>(sm.blo + swz_offset(j, k16)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-            }
+        for (int sl = 0; sl < kSlots; ++sl)
+          if (m < 0 && slot_h[sl] == cur.h && slot_m[sl] >= 0 && ((todo >> slot_m[sl]) & 1)) {
+            m = slot_m[sl];
+            slot = sl;
           }
-          bmod = m;
-          bhead = cur.h;
+        if (m < 0) {  // convert the basis into the least recently used slot
+          m = __ffs(todo) - 1;
+          slot = slot_use[0] <= slot_use[1] ? 0 : 1;
+          convert_basis(sm, slot, p.value_rot + ((size_t)cur.h * kMods + m) * kHeadDim * kHeadDim, tid);
+          slot_m[slot] = m;
+          slot_h[slot] = cur.h;
           fence_proxy_async_smem();  // generic-proxy operand writes -> visible to the tensor core
-          __syncthreads();           // also: every thread is done reading the staging buffer
-          // prefetch the next basis needed: this tile's next modality, else the next tile's first
-          {
-            const int rest = todo & ~(1 << m);
-            if (rest) {
-              issue_u(__ffs(rest) - 1, cur.h);
-            }
-          }
+          __syncthreads();
         }
+        slot_use[slot] = npass++;
         tc_fence_after();
         if (tid == 0) {
-          const uint32_t a0 = smem_u32(sm.a[buf]), bh0 = smem_u32(sm.bhi), bl0 = smem_u32(sm.blo);
+          const uint32_t a0 = smem_u32(sm.a[buf]), bh0 = smem_u32(sm.b[slot][0]), bl0 = smem_u32(sm.b[slot][1]);
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) {
             const uint32_t off = (uint32_t)((ks >> 2) * (128 * 128) + (ks & 3) * 32);
@@ -357,9 +348,8 @@ __global__ void __launch_bounds__(kVThreads, 1) vrot_tc_kernel(const WriteParams
         else
           epilogue_codes<4>(sm, tmem, warp, lane, ntok, m);
         tc_fence_before();
-        __syncthreads();  // the accumulator is reused by the next pass
+        __syncthreads();  // the accumulator is reused by the next pass (and B may be replaced)
         todo &= ~(1 << m);
-        if (todo) m = __ffs(todo) - 1;
       }
       if (timed_out) break;
 
@@ -393,18 +383,11 @@ __global__ void __launch_bounds__(kVThreads, 1) vrot_tc_kernel(const WriteParams
     gather_present(&sm.present, mod_next);
     if (tid < kTile) sm.mods[tid] = (uint8_t)(mod_next < 0 ? 0 : mod_next);
     __syncthreads();
-    // prefetch the basis of the next tile's first modality if B does not hold one it needs
-    if (upend < 0) {
-      const int np = sm.present;
-      if (np && !(bhead == nxt.h && bmod >= 0 && ((np >> bmod) & 1))) issue_u(__ffs(np) - 1, nxt.h);
-    }
     cur = nxt;
     i = inext;
   }
 
   if (timed_out && tid == 0) set_error(p.error_word, OMNIKV_DEVERR_TIMEOUT);
-  // a basis copy still in flight must land before this CTA's shared memory is released
-  if (upend >= 0) mbar_wait_bounded(&sm.u_bar, u_phase, kMmaWaitNs);
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
