@@ -167,3 +167,35 @@ def test_step_splits_and_two_phase_arguments_rejected():
         _abi.OMNIKV_ERR_CAPACITY
     assert lib.omnikv_combine_step(ctypes.byref(cfg), ctypes.byref(_cache()), FAKE, 0, None, 0) == \
         _abi.OMNIKV_ERR_INVALID_ARG
+
+
+# The library's split counts on the host without a GPU: residency falls back to
+# each decode body's register budget (per-warp body 2 CTAs per SM, cooperative
+# body 3, 4-bit build 4) on 148 SMs. The expected counts are the ones the B200
+# runs use (same SM count and residencies there).
+@pytest.mark.parametrize("batch,tokens,bits,want", [
+    (1, 10240, 2, 80),    # 2 units: cooperative wave 222, capped at one window per warp (4 per split)
+    (2, 32768, 2, 111),   # cooperative wave, 10 windows per split (<= 16)
+    (4, 32768, 2, 37),    # cooperative wave would give 19 windows per split: per-warp wave 296 / 8
+    (16, 32768, 2, 9),    # per-warp wave 296 / 32
+    (64, 32768, 2, 8),    # large batch: at least 8 splits
+    (16, 32768, 4, 18),   # 4-bit build: 592 / 32
+])
+def test_default_split_rule(batch, tokens, bits, want):
+    lib = _abi.load()
+    cfg = _cfg(key_bits=bits, value_bits=bits)
+    cache = _cache(batch=batch, cap_tokens=65536, max_seq_len=tokens)
+    assert lib.omnikv_default_splits(ctypes.byref(cfg), ctypes.byref(cache)) == want
+
+
+@pytest.mark.parametrize("batch,tokens,want_s,want_fused", [
+    (1, 10240, 81, 1),    # 10,241 tokens after the append: 81 splits of 4 windows, 164 CTAs fit
+    (16, 32768, 8, 1),    # 9 per-warp splits would need 320 CTAs > 296: lowered to 8 (288 fit)
+    (64, 32768, 8, 0),    # 128 units x 9 CTAs do not fit: append launch, then decode launch
+])
+def test_step_split_rule(batch, tokens, want_s, want_fused):
+    lib = _abi.load()
+    f = ctypes.c_int32(-1)
+    cache = _cache(batch=batch, cap_tokens=65536, max_seq_len=tokens)
+    assert lib.omnikv_step_splits(ctypes.byref(_cfg()), ctypes.byref(cache), 0, ctypes.byref(f)) == want_s
+    assert f.value == want_fused
