@@ -151,20 +151,26 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.f.close()
+        return self.parse(self.path)
+
+    @staticmethod
+    def parse(path):
+        """Median SM clock, the maximum, and the throttle reasons seen active in an
+        nvidia-smi CSV of the query Q (None without samples)."""
         sm, smax, reasons = [], 0.0, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
+        for line in open(path):
             parts = [x.strip() for x in line.split(",")]
             if len(parts) < 9:
                 continue
+            for n, v in zip(names, parts[5:9]):  # a reason counts even where a clock is unreadable
+                if v.lower() == "active":
+                    reasons.add(n)
             try:
                 sm.append(float(parts[1]))
                 smax = max(smax, float(parts[2]))
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
         if not sm:
             return None
         return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": smax, "reasons": sorted(reasons),
