@@ -125,7 +125,11 @@ OMNIKV_API size_t omnikv_record_bytes(int32_t key_bits, int32_t value_bits);
 OMNIKV_API size_t omnikv_partials_bytes(int32_t batch, int32_t num_q_heads, int32_t num_splits);
 
 /* The split count used when omnikv_decode_attention is given num_splits = 0 (depends on the
- * batch, the kv heads, max_seq_len and the device's SM count). Returns >= 1, or 0 on bad arguments. */
+ * batch, the kv heads, max_seq_len, the bit widths and the device's SM count): one wave of resident
+ * decode CTAs over batch x kv heads, at most one split per 4 windows, at least 8 splits for large
+ * batches. The decode kernel body depends on the split length (2-bit caches: splits of at most 16
+ * windows run a body with more resident CTAs per SM), and the wave is sized for that body.
+ * Returns >= 1, or 0 on bad arguments. */
 OMNIKV_API int32_t omnikv_default_splits(const omnikv_config* cfg, const omnikv_cache* cache);
 
 /* Cache write (kv_quant_pack). Appends n_new tokens to EVERY sequence of the batch, at position
