@@ -17,6 +17,8 @@ Modules:
                cache-write state machine (fp32, op-for-op)
   attention -- dequantisation and decode attention in fp64, two ways (dense in
                the original basis; fused rotated-space split-K per modality)
+  mxmeta    -- MXFP4 key metadata (the pages' default format): E2M1 minima and
+               scales with shared E8M0 exponents, codes and byte layout
 
 Parity status: every function is pinned by ``tests/test_oracle_*.py`` against
 closed forms, textbook values, brute force or invariants, except the claims the
