@@ -71,19 +71,24 @@ def codes_per_word(bits: int) -> int:
     return 32 // bits
 
 
-def record_offsets(key_bits: int, value_bits: int):
+META_FORMATS = ("fp16", "mx")  # key metadata: fp16 (m, s) pairs, or MXFP4 (oracle/mxmeta.py)
+
+
+def record_offsets(key_bits: int, value_bits: int, meta_format: str = "fp16"):
+    if meta_format not in META_FORMATS:
+        raise ValueError(meta_format)
     k_bytes = WINDOW * HEAD_DIM * key_bits // 8
     v_bytes = WINDOW * HEAD_DIM * value_bits // 8
     meta = k_bytes
-    v = meta + HEAD_DIM * 4
+    v = meta + (HEAD_DIM * 4 if meta_format == "fp16" else 144)
     sig = v + v_bytes
     total = sig + WINDOW * 2
     return {"k": 0, "meta": meta, "v": v, "sigma": sig, "total": total,
             "k_bytes": k_bytes, "v_bytes": v_bytes}
 
 
-def record_bytes(key_bits: int, value_bits: int) -> int:
-    return record_offsets(key_bits, value_bits)["total"]
+def record_bytes(key_bits: int, value_bits: int, meta_format: str = "fp16") -> int:
+    return record_offsets(key_bits, value_bits, meta_format)["total"]
 
 
 # ----------------------------------------------------------------------------
@@ -260,10 +265,11 @@ class OracleConfig:
 class OracleCache:
     """Window records, fp16 key tail, modality ids and lengths of a batch."""
 
-    def __init__(self, batch, num_kv_heads, cap_tokens, key_bits, value_bits):
+    def __init__(self, batch, num_kv_heads, cap_tokens, key_bits, value_bits, meta_format="fp16"):
         if cap_tokens % WINDOW:
             raise ValueError("cap_tokens must be a multiple of 32")
-        self.off = record_offsets(key_bits, value_bits)
+        self.off = record_offsets(key_bits, value_bits, meta_format)
+        self.meta_format = meta_format
         self.key_bits, self.value_bits = key_bits, value_bits
         self.records = np.zeros((batch, num_kv_heads, cap_tokens // WINDOW, self.off["total"]), np.uint8)
         self.key_tail = np.zeros((batch, num_kv_heads, WINDOW, HEAD_DIM), F16)
@@ -277,8 +283,24 @@ class OracleCache:
         return self.records[b, h, w, o["k"]:o["meta"]].view(np.uint32).reshape(WINDOW, -1)
 
     def meta(self, b, h, w):
+        """fp16 format: the [128] {m16, s16} pairs of the record."""
         o = self.off
+        if self.meta_format != "fp16":
+            raise ValueError("the record holds MXFP4 metadata")
         return self.records[b, h, w, o["meta"]:o["v"]].view(F16).reshape(HEAD_DIM, 2)
+
+    def meta_bytes(self, b, h, w):
+        o = self.off
+        return self.records[b, h, w, o["meta"]:o["v"]]
+
+    def key_meta_f32(self, b, h, w):
+        """The window's decoded minimum and scale per channel, (m, s) fp32 [128]."""
+        if self.meta_format == "fp16":
+            mt = self.meta(b, h, w)
+            return mt[:, 0].astype(F32), mt[:, 1].astype(F32)
+        from . import mxmeta
+        unpacked = mxmeta.unpack_meta_mx(self.meta_bytes(b, h, w))
+        return unpacked[4], unpacked[5]
 
     def v_words(self, b, h, w):
         o = self.off
@@ -301,6 +323,18 @@ def quantize_key_window(cfg: OracleConfig, raw_keys_fp16):
     codes = np.zeros((WINDOW, HEAD_DIM), np.uint32)
     codes[:n] = key_codes(kp, m16, s16, cfg.key_codebook)
     return pack_key_codes(codes, cfg.key_bits), m16, s16
+
+
+def quantize_key_window_mx(cfg: OracleConfig, raw_keys_fp16):
+    """The same window with MXFP4 metadata (oracle/mxmeta.py) -> (packed words,
+    the 144 metadata bytes)."""
+    from . import mxmeta
+    n = raw_keys_fp16.shape[0]
+    kp = rotate_keys(raw_keys_fp16, cfg.key_signs)
+    m_codes, m_exps, s_codes, s_exps, m_hat, s_hat = mxmeta.window_meta_mx(kp, cfg.key_codebook)
+    codes = np.zeros((WINDOW, HEAD_DIM), np.uint32)
+    codes[:n] = mxmeta.key_codes_mx(kp, m_hat, s_hat, cfg.key_codebook)
+    return pack_key_codes(codes, cfg.key_bits), mxmeta.pack_meta_mx(m_codes, m_exps, s_codes, s_exps)
 
 
 def encode_values(cfg: OracleConfig, head: int, v_fp16, modality):
@@ -342,11 +376,15 @@ def write_cache(cfg: OracleConfig, cache: OracleCache, k_new, v_new, modality_ne
                 raw = np.zeros((p1 - p0, HEAD_DIM), F16)
                 for p in range(p0, p1):
                     raw[p - p0] = cache.key_tail[b, h, p - p0] if p < L0 else k_new[b, h, p - L0]
-                words, m16, s16 = quantize_key_window(cfg, raw)
+                if cache.meta_format == "fp16":
+                    words, m16, s16 = quantize_key_window(cfg, raw)
+                    meta = cache.meta(b, h, w)
+                    meta[:, 0] = m16
+                    meta[:, 1] = s16
+                else:
+                    words, mbytes = quantize_key_window_mx(cfg, raw)
+                    cache.meta_bytes(b, h, w)[:] = mbytes
                 cache.k_words(b, h, w)[:] = words
-                meta = cache.meta(b, h, w)
-                meta[:, 0] = m16
-                meta[:, 1] = s16
                 if p1 - p0 < WINDOW:  # partial window: keep its raw keys
                     cache.key_tail[b, h, :p1 - p0] = raw
             # values: per token

@@ -192,3 +192,65 @@ def test_meta_byte_layout():
     assert packed[0] == (0 | 1 << 4) and packed[1] == (2 | 3 << 4) and packed[63] == (14 | 15 << 4)
     assert packed[64] == (0 | 7 << 4) and packed[65] == (14 | 5 << 4)
     assert list(packed[128:136]) == [0, 126, 127, 254, 130, 129, 128, 127]
+
+
+# ---- the MXFP4 format inside the oracle's cache state machine ---------------------
+def _cache_cfg(rng, bits):
+    from test_oracle_codec import _cfg
+    return _cfg(rng, bits, bits)
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_mx_cache_chunked_writes_equal_one_shot(bits):
+    """Appends in pieces re-quantise partial windows from the fp16 tail and give the
+    records a single prefill writes, with MXFP4 metadata too."""
+    from test_oracle_codec import _inputs
+    rng = np.random.default_rng(31)
+    cfg = _cache_cfg(rng, bits)
+    B, H, n = 2, 2, 101
+    k, v, mod = _inputs(rng, B, H, n)
+    one = codec.OracleCache(B, H, 128, bits, bits, meta_format="mx")
+    codec.write_cache(cfg, one, k, v, mod)
+    many = codec.OracleCache(B, H, 128, bits, bits, meta_format="mx")
+    cuts = [0, 1, 2, 31, 33, 64, 65, 90, 100, 101]
+    for a, b_ in zip(cuts[:-1], cuts[1:]):
+        codec.write_cache(cfg, many, k[:, :, a:b_], v[:, :, a:b_], mod[:, a:b_])
+    assert one.records.shape[-1] == mxmeta.record_bytes_mx(bits, bits)
+    assert np.array_equal(one.records, many.records)
+
+
+def test_mx_cache_records_follow_the_window_functions():
+    """Each stored window holds pack(codes) and pack(metadata) of its valid keys,
+    and its value fields are those of the fp16-metadata cache (same values path)."""
+    from test_oracle_codec import _inputs
+    rng = np.random.default_rng(32)
+    cfg = _cache_cfg(rng, 2)
+    k, v, mod = _inputs(rng, 1, 2, 77)
+    mx = codec.OracleCache(1, 2, 96, 2, 2, meta_format="mx")
+    fp = codec.OracleCache(1, 2, 96, 2, 2)
+    codec.write_cache(cfg, mx, k, v, mod)
+    codec.write_cache(cfg, fp, k, v, mod)
+    for h in range(2):
+        for w, (p0, p1) in enumerate([(0, 32), (32, 64), (64, 77)]):
+            kp = codec.rotate_keys(k[0, h, p0:p1], cfg.key_signs)
+            meta = mxmeta.window_meta_mx(kp, cfg.key_codebook)
+            codes = np.zeros((32, 128), np.uint32)
+            codes[:p1 - p0] = mxmeta.key_codes_mx(kp, meta[4], meta[5], cfg.key_codebook)
+            assert np.array_equal(mx.k_words(0, h, w), codec.pack_key_codes(codes, 2))
+            assert np.array_equal(mx.meta_bytes(0, h, w), mxmeta.pack_meta_mx(*meta[:4]))
+            assert np.array_equal(mx.v_words(0, h, w), fp.v_words(0, h, w))
+            assert np.array_equal(mx.sigma(0, h, w), fp.sigma(0, h, w))
+
+
+def test_mx_cache_decode_fused_equals_dense():
+    from test_oracle_codec import _inputs
+    from oracle.attention import decode_dense, decode_fused
+    rng = np.random.default_rng(33)
+    cfg = _cache_cfg(rng, 2)
+    c = codec.OracleCache(2, 2, 256, 2, 2, meta_format="mx")
+    k, v, mod = _inputs(rng, 2, 2, 150)
+    codec.write_cache(cfg, c, k, v, mod)
+    q = (rng.normal(size=(2, 16, 128)) * 1.5).astype(np.float16)
+    d = decode_dense(cfg, c, q)
+    for splits in (1, 3, 7):
+        assert np.abs(d - decode_fused(cfg, c, q, num_splits=splits)).max() < 1e-10
