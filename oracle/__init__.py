@@ -19,6 +19,8 @@ Modules:
                the original basis; fused rotated-space split-K per modality)
   mxmeta    -- MXFP4 key metadata (the pages' default format): E2M1 minima and
                scales with shared E8M0 exponents, codes and byte layout
+  codec_error -- key reconstruction MSE, attention KL and output MSE of the
+               codecs (fp16 / MXFP4 metadata, TurboQuant) on synthetic inputs
 
 Parity status: every function is pinned by ``tests/test_oracle_*.py`` against
 closed forms, textbook values, brute force or invariants, except the claims the
