@@ -8,7 +8,8 @@ Codecs (keys; values), every quantiser on the fixed Lloyd-Max codebook:
   omni-fp16 -- OmniKVQuant (oracle/codec.py): sign-flip Hadamard keys with a
                per-channel min-max range per 32-token window, fp16 metadata;
                values rotated by the basis U_m of their modality, per-token scale.
-  omni-mx   -- the same with MXFP4 window metadata (oracle/mxmeta.py).
+  omni-mx   -- the same with MXFP4 window metadata (oracle/mxmeta.py, its default
+               nearest rounding).
   turbo     -- TurboQuant as the pages describe it (pchao.org 关联工作; paperpeel
                section 2.2 "Temporal key drift", section 2.3): one random rotation
                (the same sign-flip Hadamard) for keys and values, and a per-token

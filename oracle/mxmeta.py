@@ -17,10 +17,17 @@ power-of-two E8M0 scale per block of 32) and states each choice:
   x3  the shared exponent e (stored as the E8M0 byte e + 127) is the smallest
       integer in [-127, 127] with max_c |x_c| <= 6 * 2^e over the block, so no
       element saturates; an all-zero block takes e = -127.
-  x4  the window minimum rounds toward -inf and the scale toward +inf on the
-      grid {+-magnitude * 2^e}, so that [m^, m^ + s^ (c_{L-1} - c_0)] covers the
-      channel's keys: m^ first (from the fp32 minimum), then the scale it needs,
-      s_req = fp32(fp32(max - m^) / (c_{L-1} - c_0)), rounded up to s^.
+  x4  rounding on the grid {+-magnitude * 2^e}: the minimum first (from the fp32
+      minimum), then the scale that minimum needs, s_req = fp32(fp32(max - m^) /
+      (c_{L-1} - c_0)) (0 if negative). Default ("nearest", the MX conversion rule):
+      both round to the nearest grid value, ties to the even code; keys outside
+      [m^, m^ + s^ (c_{L-1} - c_0)] take the end codes. Option ("cover"): the
+      minimum rounds toward -inf and the scale toward +inf, so the range covers
+      every key of the channel. On the workloads' synthetic keys with 2-bit codes
+      the covering option roughly doubles the errors of the fp16 format while the
+      nearest one stays within ~10 % of it (oracle/codec_error.py; with 4-bit codes
+      the covering one is the closer), and the pages report MXFP4 as their accurate
+      default at the 2-bit budget, hence the default.
   x5  codes as in the fp16 format with (m^, s^) in place of (m16, s16):
       z = (k' - m^) / s^ + c_0 in fp32, code = #{j : z > t_j}; s^ == 0 -> 0;
       reconstruction k^' = m^ + s^ (c_j - c_0).
@@ -87,6 +94,19 @@ def round_down(x, e):
     return _code_of(g), g * 2.0 ** e
 
 
+def round_nearest(x, e):
+    """Nearest grid value g * 2^e to x, ties to the even code (x4, default).
+    Returns (code, value)."""
+    q = float(x) / 2.0 ** e
+    grid = _signed_grid()
+    d = np.abs(grid - q)
+    best = np.flatnonzero(d == d.min())
+    if len(best) > 1:   # a tie between two neighbours: the even code
+        best = [i for i in best if _code_of(float(grid[i])) % 2 == 0]
+    g = float(grid[best[0]])
+    return _code_of(g), g * 2.0 ** e
+
+
 def round_up(x, e):
     """Smallest grid value g * 2^e >= x (x4, for the scale). Returns (code, value)."""
     q = float(x) / 2.0 ** e
@@ -96,11 +116,16 @@ def round_up(x, e):
     return _code_of(g), g * 2.0 ** e
 
 
-def window_meta_mx(kp_valid, codebook):
+def window_meta_mx(kp_valid, codebook, rounding="nearest"):
     """MXFP4 metadata of one window from its rotated fp32 keys (valid tokens only):
-    per channel the minimum rounded down, then the scale it needs rounded up (x3,
-    x4). Returns (m_codes [128], m_exps [4], s_codes [128], s_exps [4], m_hat [128],
-    s_hat [128]); m_hat and s_hat are exact in fp32."""
+    per channel the minimum, then the scale it needs, each rounded on its block's
+    grid (x3, x4; rounding "nearest" or "cover"). Returns (m_codes [128], m_exps [4],
+    s_codes [128], s_exps [4], m_hat [128], s_hat [128]); m_hat and s_hat are exact
+    in fp32."""
+    if rounding not in ("nearest", "cover"):
+        raise ValueError(rounding)
+    rnd_m = round_nearest if rounding == "nearest" else round_down
+    rnd_s = round_nearest if rounding == "nearest" else round_up
     kp = np.asarray(kp_valid, dtype=F32)
     c = np.asarray(codebook, dtype=F32)
     mn = kp.min(axis=0)
@@ -117,16 +142,17 @@ def window_meta_mx(kp_valid, codebook):
         e = block_exponent(mn[ch])
         m_exps[b] = e
         for cc in range(BLOCK * b, BLOCK * (b + 1)):
-            m_codes[cc], m_hat[cc] = round_down(mn[cc], e)
+            m_codes[cc], m_hat[cc] = rnd_m(mn[cc], e)
     # the scale each channel needs with its rounded minimum, in fp32
     with np.errstate(over="ignore"):
         s_req = ((mx - m_hat.astype(F32)) / span).astype(F32)
+    s_req = np.maximum(s_req, F32(0.0))   # a minimum rounded above the maximum: no range
     for b in range(BLOCKS):
         ch = slice(BLOCK * b, BLOCK * (b + 1))
         e = block_exponent(s_req[ch])
         s_exps[b] = e
         for cc in range(BLOCK * b, BLOCK * (b + 1)):
-            s_codes[cc], s_hat[cc] = round_up(s_req[cc], e)
+            s_codes[cc], s_hat[cc] = rnd_s(s_req[cc], e)
     return m_codes, m_exps, s_codes, s_exps, m_hat.astype(F32), s_hat.astype(F32)
 
 

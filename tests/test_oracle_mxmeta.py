@@ -60,10 +60,25 @@ def test_rounding_directions_by_enumeration(seed):
         vals = _grid_values(e)
         cd, vd = mxmeta.round_down(x, e)
         cu, vu = mxmeta.round_up(x, e)
+        cn, vn = mxmeta.round_nearest(x, e)
         assert vd == max(v for v in vals if v <= x)
         assert vu == min(v for v in vals if v >= x)
+        best = min(abs(v - x) for v in vals)
+        assert abs(vn - x) == best
         assert mxmeta.e2m1_decode(cd) * 2.0 ** e == vd
         assert mxmeta.e2m1_decode(cu) * 2.0 ** e == vu
+        assert mxmeta.e2m1_decode(cn) * 2.0 ** e == vn
+
+
+def test_nearest_ties_go_to_the_even_code():
+    # midpoints of the E2M1 grid: 0.25 0.75 1.25 1.75 2.5 3.5 5 -> 0 1 1 2 2 4 4
+    mids = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]
+    want = [0.0, 1.0, 1.0, 2.0, 2.0, 4.0, 4.0]
+    for e in (-3, 0, 2):
+        for x, w in zip(mids, want):
+            for sgn in (1.0, -1.0):
+                code, val = mxmeta.round_nearest(sgn * x * 2.0 ** e, e)
+                assert val == sgn * w * 2.0 ** e and code % 2 == 0
 
 
 def test_zero_is_positive_code():
@@ -81,25 +96,35 @@ def _synthetic_window(seed, n=32, outliers=4):
     return codec.rotate_keys(raw.astype(np.float16), signs)
 
 
+@pytest.mark.parametrize("rounding", ["nearest", "cover"])
 @pytest.mark.parametrize("bits,seed", [(2, 0), (2, 1), (2, 2), (4, 3), (4, 4)])
-def test_window_range_is_covered_and_error_bounded(bits, seed):
+def test_window_metadata_and_error_bounds(bits, seed, rounding):
     cb = _codebook(bits)
     kp = _synthetic_window(seed, n=32 if seed % 2 == 0 else 17)
-    m_codes, m_exps, s_codes, s_exps, m_hat, s_hat = mxmeta.window_meta_mx(kp, cb)
-    mn, mx = kp.min(axis=0), kp.max(axis=0)
+    m_codes, m_exps, s_codes, s_exps, m_hat, s_hat = mxmeta.window_meta_mx(kp, cb, rounding)
+    mn, mx = kp.min(axis=0).astype(np.float64), kp.max(axis=0).astype(np.float64)
+    m64, s64 = m_hat.astype(np.float64), s_hat.astype(np.float64)
     span = float(cb[-1]) - float(cb[0])
-    # the rounded minimum never exceeds the true one; the range reaches the maximum
-    # (up to the fp32 rounding of the required scale)
-    assert np.all(m_hat.astype(np.float64) <= mn.astype(np.float64))
-    top = m_hat.astype(np.float64) + s_hat.astype(np.float64) * span
-    assert np.all(top >= mx.astype(np.float64) - 1e-6 * np.abs(mx.astype(np.float64)))
-    # reconstruction within half the largest codebook gap (times the scale) plus
-    # the fp32 rounding of z
+    top = m64 + s64 * span
+    em = np.repeat(m_exps, 32).astype(np.float64)
+    if rounding == "cover":
+        # the rounded minimum never exceeds the true one; the range reaches the
+        # maximum (up to the fp32 rounding of the required scale)
+        assert np.all(m64 <= mn)
+        assert np.all(top >= mx - 1e-6 * np.abs(mx))
+    else:
+        # within half the widest grid gap (2 * 2^e between 4 and 6) of the minimum
+        assert np.all(np.abs(m64 - mn) <= 2.0 ** em)
+    # reconstruction: half a codebook gap times the scale inside the stored range,
+    # plus the distance by which a key lies outside it (end codes), plus the fp32
+    # rounding of z
     codes = mxmeta.key_codes_mx(kp, m_hat, s_hat, cb)
     rec = mxmeta.dequantize_keys_mx(codes, m_hat, s_hat, cb)
+    k64 = kp.astype(np.float64)
     gap = float(np.max(np.diff(cb.astype(np.float64))))
-    bound = s_hat.astype(np.float64) * (gap / 2.0) * (1 + 1e-5) + 1e-6 * (np.abs(kp) + 1)
-    assert np.all(np.abs(rec - kp.astype(np.float64)) <= bound)
+    outside = np.maximum(m64[None, :] - k64, 0) + np.maximum(k64 - top[None, :], 0)
+    bound = s64 * (gap / 2.0) * (1 + 1e-5) + outside + 1e-6 * (np.abs(k64) + 1)
+    assert np.all(np.abs(rec - k64) <= bound)
     assert codes.max() < (1 << bits)
 
 
@@ -125,8 +150,9 @@ def test_grid_minimum_is_reproduced():
     kp = (m[None, :].astype(np.float64) + s[None, :].astype(np.float64)
           * (cb[j].astype(np.float64) - float(cb[0]))).astype(F32)
     assert np.array_equal(kp.min(axis=0), m)
-    m_hat = mxmeta.window_meta_mx(kp, cb)[4]
-    assert np.array_equal(m_hat, m)
+    for rounding in ("nearest", "cover"):
+        m_hat = mxmeta.window_meta_mx(kp, cb, rounding)[4]
+        assert np.array_equal(m_hat, m)
 
 
 def test_power_of_two_scales_recover_scale_and_codes():
@@ -142,15 +168,17 @@ def test_power_of_two_scales_recover_scale_and_codes():
             s[32 * b:32 * b + 32] = 2.0 ** (es + rng.integers(-1, 3, 32))   # 0.5 .. 4 times 2^es
         j = _codes_every_level(rng, 1 << bits)
         kp = (s[None, :].astype(np.float64) * (cb[j].astype(np.float64) - float(cb[0]))).astype(F32)
-        m_codes, m_exps, s_codes, s_exps, m_hat, s_hat = mxmeta.window_meta_mx(kp, cb)
-        assert not m_hat.any()
-        assert np.array_equal(s_hat, s)
-        np.testing.assert_array_equal(mxmeta.key_codes_mx(kp, m_hat, s_hat, cb), j)
+        for rounding in ("nearest", "cover"):
+            m_codes, m_exps, s_codes, s_exps, m_hat, s_hat = mxmeta.window_meta_mx(kp, cb, rounding)
+            assert not m_hat.any()
+            assert np.array_equal(s_hat, s)
+            np.testing.assert_array_equal(mxmeta.key_codes_mx(kp, m_hat, s_hat, cb), j)
 
 
 def test_constant_channels():
-    """A constant channel on the grid keeps s^ = 0 and codes 0 (reading r5); off
-    the grid its minimum rounds down and a nonzero scale covers the value."""
+    """A constant channel on the grid keeps s^ = 0 and codes 0 (reading r5), with
+    either rounding; off the grid, the covering rounding takes the minimum down and
+    a nonzero scale that reaches the value."""
     cb = _codebook(2)
     kp = _synthetic_window(11)
     rng = np.random.default_rng(12)
@@ -159,13 +187,15 @@ def test_constant_channels():
     vals[0] = F32(-6.0)                     # block 0 exponent 0: every value on its grid
     kp[:, 0:32] = vals[None, :]
     kp[:, 40] = F32(1.25)                   # off the grid of block 1
-    m_codes, m_exps, s_codes, s_exps, m_hat, s_hat = mxmeta.window_meta_mx(kp, cb)
-    codes = mxmeta.key_codes_mx(kp, m_hat, s_hat, cb)
-    assert m_exps[0] == 0 and s_exps[0] == -127
-    assert np.array_equal(m_hat[0:32], vals) and not s_hat[0:32].any() and not codes[:, 0:32].any()
-    assert m_hat[40] < 1.25 < m_hat[40] + s_hat[40] * (float(cb[-1]) - float(cb[0]))
-    rec = mxmeta.dequantize_keys_mx(codes, m_hat, s_hat, cb)[:, 40]
-    assert np.all(np.abs(rec - 1.25) <= s_hat[40] * float(np.max(np.diff(cb))) / 2 * (1 + 1e-5))
+    for rounding in ("nearest", "cover"):
+        m_codes, m_exps, s_codes, s_exps, m_hat, s_hat = mxmeta.window_meta_mx(kp, cb, rounding)
+        codes = mxmeta.key_codes_mx(kp, m_hat, s_hat, cb)
+        assert m_exps[0] == 0 and s_exps[0] == -127
+        assert np.array_equal(m_hat[0:32], vals) and not s_hat[0:32].any() and not codes[:, 0:32].any()
+        if rounding == "cover":
+            assert m_hat[40] < 1.25 < m_hat[40] + s_hat[40] * (float(cb[-1]) - float(cb[0]))
+            rec = mxmeta.dequantize_keys_mx(codes, m_hat, s_hat, cb)[:, 40]
+            assert np.all(np.abs(rec - 1.25) <= s_hat[40] * float(np.max(np.diff(cb))) / 2 * (1 + 1e-5))
 
 
 def test_meta_bytes_round_trip_and_record_size():
