@@ -417,7 +417,7 @@ def run_gpu(args):
             "clocks": clk,
             "dense_bf16": dense,
         }
-        if not args.no_cpu_baseline:
+        if not args.no_cpu_baseline and world == 1:  # the oracle is timed at N = 1 only
             line["cpu_baseline"] = cpu_baseline(spec, seed)
         print(json.dumps(line), flush=True)
     del graph, g2
