@@ -21,6 +21,8 @@ Modules:
                scales with shared E8M0 exponents, codes and byte layout
   codec_error -- key reconstruction MSE, attention KL and output MSE of the
                codecs (fp16 / MXFP4 metadata, TurboQuant) on synthetic inputs
+  calibration -- per-modality value bases from attention-weighted covariances
+               (eigenbasis composed with the Hadamard rotation)
 
 Parity status: every function is pinned by ``tests/test_oracle_*.py`` against
 closed forms, textbook values, brute force or invariants, except the claims the

@@ -337,6 +337,13 @@ def quantize_key_window_mx(cfg: OracleConfig, raw_keys_fp16):
     return pack_key_codes(codes, cfg.key_bits), mxmeta.pack_meta_mx(m_codes, m_exps, s_codes, s_exps)
 
 
+def encode_values_with_basis(v_fp16, basis, codebook):
+    """Values of one modality rotated by `basis` -> (codes [n][128], sigma16 [n])."""
+    v = np.asarray(v_fp16, dtype=F16)
+    sg = value_sigma(v)
+    return value_codes(rotate_values(v, basis), sg, codebook), sg
+
+
 def encode_values(cfg: OracleConfig, head: int, v_fp16, modality):
     """Values of n tokens of one kv head -> (codes [n][128], sigma16 [n])."""
     v = np.asarray(v_fp16, dtype=F16)
