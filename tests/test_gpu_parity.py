@@ -200,19 +200,20 @@ def test_asymmetric_codebook_uses_generic_path(cuda_device):
 @pytest.mark.parametrize("G,hkv", [(1, 4), (4, 2), (8, 1)])
 def test_group_sizes(cuda_device, G, hkv):
     """GQA groups smaller than 8 leave tensor-core columns unused; every group
-    size up to 8 must match the oracle."""
+    size up to 8 must match the oracle, with both 2-bit decode bodies (600 tokens:
+    one split of 19 windows runs the per-warp body, 4 splits the cooperative one)."""
     import dataclasses
     m = _abi()
     spec = dataclasses.replace(WORKLOADS["tiny"], num_q_heads=G * hkv, num_kv_heads=hkv)
     seed = 9
     params, consts, ocfg = make_layer(spec, seed, 0, cuda_device, per_head=True)
-    L = np.array([333, 70], np.int32)
+    L = np.array([600, 70], np.int32)
     spec2 = dataclasses.replace(spec, batch=2)
-    drift = key_drift(spec2, seed, 0, 16, cuda_device)
-    k, v, mod = prefill_inputs(spec2, seed, 0, params, drift, np.array([333, 333]), cuda_device)
-    oc = codec.OracleCache(2, hkv, 352, 2, 2)
+    drift = key_drift(spec2, seed, 0, 20, cuda_device)
+    k, v, mod = prefill_inputs(spec2, seed, 0, params, drift, np.array([600, 600]), cuda_device)
+    oc = codec.OracleCache(2, hkv, 640, 2, 2)
     for b in range(2):
-        sub = codec.OracleCache(1, hkv, 352, 2, 2)
+        sub = codec.OracleCache(1, hkv, 640, 2, 2)
         n = int(L[b])
         codec.write_cache(ocfg, sub, k[b:b + 1, :, :n].cpu().numpy(), v[b:b + 1, :, :n].cpu().numpy(),
                           mod[b:b + 1, :n].cpu().numpy())
