@@ -48,11 +48,12 @@ CASES = [
     (4, 8, [200, 17], 4, 0, 2),             # 4 kv heads, 32 query heads
     (2, 8, [93, 40], 4, 200, 2),            # 2 x (1 + 200) CTAs: beyond residency -> four-call fallback
     (2, 8, [93, 250], 4, 0, 4),             # K4V4: the CUDA-core decode path with the fused append
+    (2, 8, [700], 3, 1, 2),                 # one split of 22 windows: the per-warp body in the fused launch
 ]
 
 
 @pytest.mark.parametrize("hkv,G,lengths,steps,splits,bits", CASES,
-                         ids=["b1-boundary", "ragged-b3", "h4", "fallback", "k4"])
+                         ids=["b1-boundary", "ragged-b3", "h4", "fallback", "k4", "per-warp"])
 def test_decode_step_matches_four_calls_and_oracle(cuda_device, hkv, G, lengths, steps, splits, bits):
     import bit_kv_cache_pack_b200 as m
     dev = cuda_device
@@ -61,7 +62,7 @@ def test_decode_step_matches_four_calls_and_oracle(cuda_device, hkv, G, lengths,
                                batch=len(lengths))
     params, consts, ocfg = make_layer(spec, seed, 0, dev)
     B = len(lengths)
-    cap = 320
+    cap = max(320, -(-(max(lengths) + steps) // 32) * 32)
     drift = key_drift(spec, seed, 0, cap // 32, dev)
     fused = m.KVCache(B, hkv, cap, bits, bits, dev)
     plain = m.KVCache(B, hkv, cap, bits, bits, dev)
