@@ -1,14 +1,15 @@
 """Benchmark: OmniKVQuant decode step (cache append + fused split-K decode +
 combine/inverse rotation, every layer) on synthetic inputs.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl omnikv|reference] [--workload omni3b-b1]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl omnikv|reference] [--workload omni30b-b8]
     torchrun --nproc-per-node N bench.py --gpus N ...   (one rank per GPU, weak scaling)
 
-Default workload: the Qwen2.5-Omni-3B-shaped decode (36 layers, 16 query / 2 KV
-heads, head dim 128, batch 1, 10,240 cached tokens of interleaved text / audio /
-video, K2/V2, 32-token windows); one step appends one text token per sequence to
-every layer's cache and runs decode attention for every layer. Each rank runs
-its own batch (different seed), so per-GPU work is fixed as N grows.
+Default workload: the largest single-GPU configuration, the Qwen3-Omni-30B-A3B-
+shaped decode (48 layers, 32 query / 4 KV heads, head dim 128, batch 8, 65,536
+cached tokens per sequence in an audio-heavy interleaved layout, K2/V2, 32-token
+windows); one step appends one text token per sequence to every layer's cache
+and runs decode attention for every layer. Each rank runs its own batch
+(different seed), so per-GPU work is fixed as N grows.
 
 Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events on
 the launching stream and preceded by an untimed L2 flush (a 512 MiB write);
@@ -29,6 +30,10 @@ import subprocess
 import sys
 import time
 
+if "reference" in sys.argv:  # the oracle arm: one thread per BLAS / OpenMP pool from the start
+    for _var in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+        os.environ.setdefault(_var, "1")
+
 import numpy as np
 import torch
 
@@ -46,8 +51,11 @@ BYTES_PER_TOKEN_HEAD = {(2, 2): 82, (4, 4): 146}   # algorithmic packed bytes pe
 # (its summary is kept with the other profiles), valid for the kernel sources
 # with this SHA-256; any change to them makes the field null until the next
 # capture.
-TRAFFIC_CAPTURE = {"sources_sha256": "71ad72e9edf4bc86edda2a2bba852d6d1b21129c1b76a859aceb750e9a300447",
-                   "bytes_per_launch": 2198016}
+TRAFFIC_CAPTURES = {
+    "qwen2.5-omni-3b-36L-b1-ctx10240": {
+        "sources_sha256": "71ad72e9edf4bc86edda2a2bba852d6d1b21129c1b76a859aceb750e9a300447",
+        "bytes_per_launch": 2198016},
+}
 KERNEL_SOURCES = ("decode_split_k.cu", "append.cuh", "common.cuh", "ptx.cuh", "kernels.h")
 
 
@@ -62,19 +70,22 @@ def kernel_sources_sha256():
 
 
 def captured_traffic(workload_name):
-    if workload_name != "qwen2.5-omni-3b-36L-b1-ctx10240" or TRAFFIC_CAPTURE["sources_sha256"] is None:
+    cap = TRAFFIC_CAPTURES.get(workload_name)
+    if cap is None:
         return None
-    return TRAFFIC_CAPTURE["bytes_per_launch"] if kernel_sources_sha256() == TRAFFIC_CAPTURE["sources_sha256"] else None
+    return cap["bytes_per_launch"] if kernel_sources_sha256() == cap["sources_sha256"] else None
+
+
 L2_FLUSH_BYTES = 512 << 20
 
 
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=64)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=4)
     ap.add_argument("--impl", default="omnikv", choices=["omnikv", "reference"])
-    ap.add_argument("--workload", default="omni3b-b1", choices=sorted(WORKLOADS_KEYS))
+    ap.add_argument("--workload", default="omni30b-b8", choices=sorted(WORKLOADS_KEYS))
     ap.add_argument("--no-graphs", action="store_true")
     ap.add_argument("--layer", choices=["decode", "write"], default=None,
                     help="time one layer's decode (+ combine) or prefill cache write on --workload instead of "
@@ -97,6 +108,19 @@ def dist_env():
 def rank_seed(workload: str, rank: int) -> int:
     """Each rank decodes its own batch (weak scaling): a different seed per rank."""
     return WORKLOADS_KEYS.index(workload) + 1000 * rank
+
+
+def workload_config(spec, world):
+    """The `config` object of both arms' JSON lines: the workload and how it is
+    measured (the same dict for the GPU arm and the oracle arm)."""
+    from synth.workloads import seq_lengths
+    L = seq_lengths(spec, 0)
+    return {"workload": spec.name, "layers": spec.layers, "global_batch": spec.batch * world,
+            "context": int(L.max()) if not spec.ragged else "%d..%d" % spec.ragged,
+            "num_q_heads": spec.num_q_heads, "num_kv_heads": spec.num_kv_heads, "head_dim": 128,
+            "key_bits": spec.key_bits, "value_bits": spec.value_bits, "window": 32,
+            "parallelism": "dp%d (independent sequences per rank)" % world,
+            "l2": "GPU arm: flushed between timed steps (512 MiB write)"}
 
 
 def max_over_ranks(values, device, world):
@@ -396,13 +420,9 @@ def run_gpu(args):
             "warmup": W, "ms_per_step": round(total_ms / K, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "u2 codes, f32 accumulate",
             "data": "synthetic",
-            "config": {"workload": spec.name, "layers": spec.layers, "global_batch": spec.batch * world,
-                       "context": int(wl.lengths.max()), "num_q_heads": spec.num_q_heads,
-                       "num_kv_heads": spec.num_kv_heads, "head_dim": 128, "key_bits": spec.key_bits,
-                       "value_bits": spec.value_bits, "window": 32, "num_splits": wl.S,
-                       "parallelism": "dp%d (independent sequences per rank)" % world,
-                       "l2": "flushed between timed steps (512 MiB write)",
-                       "launch": "one CUDA graph for all steps (flush + events + C-ABI calls)" if use_graphs
+            "config": workload_config(spec, world),
+            "launch": {"num_splits": wl.S, "fused_append": bool(wl.fused),
+                       "graph": "one CUDA graph for all steps (flush + events + C-ABI calls)" if use_graphs
                        else "eager"},
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": captured_traffic(spec.name),
@@ -475,7 +495,56 @@ def dense_baseline(spec, wl, dev, K, W, flush, stream):
 # ----------------------------------------------------------------------------
 # the CPU oracle, timed (baseline and reference arm)
 # ----------------------------------------------------------------------------
-def _oracle_layers(spec, seed, layers, extra_steps):
+def host_info():
+    """Host cores and CPU model of the machine the oracle is timed on."""
+    model = ""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count(), "cpu_model": model}
+
+
+class OneCore:
+    """Context: the oracle runs on one host core -- BLAS / OpenMP pools limited to
+    one thread, torch's intra-op pool to one thread, and the process pinned to a
+    single CPU of its allowed set -- restored on exit."""
+
+    def __enter__(self):
+        import threadpoolctl
+        self.limits = threadpoolctl.threadpool_limits(1)
+        self.threads = torch.get_num_threads()
+        torch.set_num_threads(1)
+        self.aff = os.sched_getaffinity(0)
+        os.sched_setaffinity(0, {min(self.aff)})
+        return self
+
+    def __exit__(self, *exc):
+        os.sched_setaffinity(0, self.aff)
+        torch.set_num_threads(self.threads)
+        self.limits.restore_original_limits()
+        return False
+
+
+def oracle_sample_shape(spec):
+    """Layers and sequences of the workload the oracle is timed on: all of it when
+    one layer holds at most ~100k token-heads, else one layer and up to 4 sequences
+    (the oracle decodes ~1 s per 65,536-token sequence and kv-head set)."""
+    from synth.workloads import seq_lengths
+    per_layer = int(seq_lengths(spec, 0).astype(np.int64).sum()) * spec.num_kv_heads
+    if per_layer <= 100_000:
+        return min(spec.layers, 12), spec.batch
+    return 1, min(spec.batch, 4)
+
+
+def _oracle_sequences(spec, seed, layers, seqs, extra_steps):
+    """The oracle's caches of the sampled (layer, sequence) pairs, each a batch-1
+    cache prefilled with that sequence's context (untimed), and every layer's
+    decode inputs for extra_steps steps."""
     from oracle import codec
     from synth.workloads import codebook, decode_inputs, key_drift, layer_params, prefill_inputs, seq_lengths
     L = seq_lengths(spec, seed)
@@ -486,46 +555,58 @@ def _oracle_layers(spec, seed, layers, extra_steps):
         ocfg = codec.OracleConfig(codebook(spec.key_bits), codebook(spec.value_bits),
                                   params["key_signs"].numpy(), params["value_rot"].numpy(),
                                   spec.num_q_heads, spec.num_kv_heads)
-        oc = codec.OracleCache(spec.batch, spec.num_kv_heads, cap, spec.key_bits, spec.value_bits)
         drift = key_drift(spec, seed, layer, cap // 32, "cpu")
-        k, v, mod = prefill_inputs(spec, seed, layer, params, drift, L, "cpu")
-        for b in range(spec.batch):
-            sub = codec.OracleCache(1, spec.num_kv_heads, cap, spec.key_bits, spec.value_bits)
+        caches = []
+        for b in seqs:
+            k, v, mod = prefill_inputs(spec, seed, layer, params, drift, L, "cpu", batch_index=[b])
             n = int(L[b])
-            codec.write_cache(ocfg, sub, k[b:b + 1, :, :n].numpy(), v[b:b + 1, :, :n].numpy(),
-                              mod[b:b + 1, :n].numpy())
-            oc.records[b], oc.key_tail[b], oc.modality[b], oc.seq_lens[b] = (
-                sub.records[0], sub.key_tail[0], sub.modality[0], sub.seq_lens[0])
+            oc = codec.OracleCache(1, spec.num_kv_heads, cap, spec.key_bits, spec.value_bits)
+            codec.write_cache(ocfg, oc, k[:, :, :n].numpy(), v[:, :, :n].numpy(), mod[:, :n].numpy())
+            caches.append(oc)
+            del k, v, mod
         steps = [decode_inputs(spec, seed, layer, s, params, drift, L + s, "cpu") for s in range(extra_steps)]
-        out.append((ocfg, oc, steps))
+        out.append((ocfg, caches, steps))
     return out
 
 
-def _oracle_step(ocfg, oc, inputs, num_splits=4):
+def _oracle_step(ocfg, oc, inputs, b, num_splits=4):
+    """One decode step of sequence b through the oracle: append its token, then
+    the fused split-K decode and combine."""
     from oracle import codec
     from oracle.attention import decode_fused
-    q, kn, vn, mn = inputs
-    codec.write_cache(ocfg, oc, kn.numpy(), vn.numpy(), mn.numpy())
-    return decode_fused(ocfg, oc, q.numpy(), num_splits)
+    q, kn, vn, mn = (x[b:b + 1].numpy() for x in inputs)
+    codec.write_cache(ocfg, oc, kn, vn, mn)
+    return decode_fused(ocfg, oc, q, num_splits)
 
 
-def cpu_baseline(spec, seed, sample_layers=12):
-    """The oracle as it stands (single process, numpy) on a bounded sample: one
-    decode step (append + fused decode + combine) over the first sample_layers
-    layers, scaled to all layers."""
-    n = min(sample_layers, spec.layers)
-    prepared = _oracle_layers(spec, seed, range(n), 1)
-    t0 = time.perf_counter()
-    for ocfg, oc, steps in prepared:
-        _oracle_step(ocfg, oc, steps[0])
-    dt = time.perf_counter() - t0
-    per_step = dt * spec.layers / n
-    return {"value": round(spec.batch / per_step, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": "1 decode step x %d of %d layers (append + fused decode + combine, numpy fp64), "
-                      "scaled to %d layers; %.1f s of CPU" % (n, spec.layers, spec.layers, dt)}
+def cpu_baseline(spec, seed):
+    """The oracle as it stands (numpy fp64, one pinned core) on a bounded sample of
+    the workload -- one decode step of the sampled layers and sequences -- scaled
+    linearly to the whole step (all layers, all sequences)."""
+    n_layers, n_seq = oracle_sample_shape(spec)
+    prepared = _oracle_sequences(spec, seed, range(n_layers), range(n_seq), 1)
+    with OneCore():
+        t0 = time.perf_counter()
+        for ocfg, caches, steps in prepared:
+            for b, oc in enumerate(caches):
+                _oracle_step(ocfg, oc, steps[0], b)
+        dt = time.perf_counter() - t0
+    scale = (spec.layers / n_layers) * (spec.batch / n_seq)
+    per_step = dt * scale
+    d = {"value": round(spec.batch / per_step, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
+         "sample": "1 decode step (append + fused decode + combine, numpy fp64) of %d of %d layers x %d of %d "
+                   "sequences, %.1f s of CPU on one pinned core, scaled x%g to the whole step"
+                   % (n_layers, spec.layers, n_seq, spec.batch, dt, scale),
+         "extrapolated": scale != 1.0}
+    d.update(host_info())
+    return d
 
 
 def run_reference(args):
+    """The reference arm: the oracle, timed on the host. Each timed step is one
+    (layer, sequence) sample of the workload's decode step (append + fused decode +
+    combine), rotating over the sampled sequences; the full step's time is that
+    sample's mean time x layers x sequences."""
     from synth.workloads import WORKLOADS
     world, rank, _ = dist_env()
     if rank != 0:
@@ -533,28 +614,34 @@ def run_reference(args):
     spec = WORKLOADS[args.workload]
     seed = WORKLOADS_KEYS.index(args.workload)
     K, W = args.steps, args.warmup
-    n_prep = min(4, spec.layers)
-    prepared = _oracle_layers(spec, seed, range(n_prep), (W + K) // n_prep + 2)
+    n_seq = min(spec.batch, 2)
+    prepared = _oracle_sequences(spec, seed, [0], range(n_seq), (W + K) // n_seq + 2)
+    ocfg, caches, steps = prepared[0]
     times = []
-    for s in range(W + K):
-        ocfg, oc, steps = prepared[s % n_prep]
-        t0 = time.perf_counter()
-        _oracle_step(ocfg, oc, steps[s // n_prep])
-        if s >= W:
-            times.append(time.perf_counter() - t0)
-    per_step = float(np.mean(times)) * spec.layers   # one sample = one layer of a step
+    with OneCore():
+        for s in range(W + K):
+            b = s % n_seq
+            t0 = time.perf_counter()
+            _oracle_step(ocfg, caches[b], steps[s // n_seq], b)
+            if s >= W:
+                times.append(time.perf_counter() - t0)
+    sample_s = float(np.mean(times))
+    scale = spec.layers * spec.batch
+    per_step = sample_s * scale
     value = spec.batch / per_step
+    base = {"value": round(value, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": "each timed step: one layer's decode step (append + fused decode + combine, numpy fp64) "
+                      "of one of %d sequences, on one pinned core; the whole step = x%d (%d layers x %d "
+                      "sequences)" % (n_seq, scale, spec.layers, spec.batch),
+            "extrapolated": scale != 1}
+    base.update(host_info())
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
         "steps": K, "warmup": W, "ms_per_step": round(per_step * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic",
-        "config": {"workload": spec.name, "layers": spec.layers, "global_batch": spec.batch,
-                   "context": int(spec.context), "num_q_heads": spec.num_q_heads,
-                   "num_kv_heads": spec.num_kv_heads, "head_dim": 128, "key_bits": spec.key_bits,
-                   "value_bits": spec.value_bits, "window": 32},
-        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": "each step: one layer's append + fused decode + combine (numpy fp64), "
-                                   "x %d layers" % spec.layers},
+        "config": workload_config(spec, world),
+        "extrapolated": scale != 1, "sample_ms_per_step": round(sample_s * 1e3, 3),
+        "cpu_baseline": base,
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

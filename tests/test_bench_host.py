@@ -36,15 +36,48 @@ def test_clock_record_empty(tmp_path):
 
 
 def test_traffic_reported_only_for_the_captured_sources(monkeypatch):
-    wl = "qwen2.5-omni-3b-36L-b1-ctx10240"
-    monkeypatch.setattr(bench, "TRAFFIC_CAPTURE", {"sources_sha256": bench.kernel_sources_sha256(),
-                                                   "bytes_per_launch": 123})
+    wl = "qwen3-omni-30b-48L-b8-ctx65536"
+    monkeypatch.setattr(bench, "TRAFFIC_CAPTURES", {wl: {"sources_sha256": bench.kernel_sources_sha256(),
+                                                         "bytes_per_launch": 123}})
     assert bench.captured_traffic(wl) == 123
     assert bench.captured_traffic("qwen2.5-omni-3b-36L-b16-ctx32768") is None  # another workload
-    monkeypatch.setattr(bench, "TRAFFIC_CAPTURE", {"sources_sha256": "0" * 64, "bytes_per_launch": 123})
+    monkeypatch.setattr(bench, "TRAFFIC_CAPTURES", {wl: {"sources_sha256": "0" * 64, "bytes_per_launch": 123}})
     assert bench.captured_traffic(wl) is None                                  # sources changed since
-    monkeypatch.setattr(bench, "TRAFFIC_CAPTURE", {"sources_sha256": None, "bytes_per_launch": None})
-    assert bench.captured_traffic(wl) is None
+
+
+def test_both_arms_share_the_config_object():
+    """The GPU arm and the oracle arm print the same `config` dict, and the
+    default workload is the largest single-GPU configuration (48 layers, 8 x
+    65,536 tokens)."""
+    import sys
+    from synth.workloads import WORKLOADS
+    argv = sys.argv
+    try:
+        sys.argv = ["bench.py"]
+        default = bench.parse_args().workload
+    finally:
+        sys.argv = argv
+    spec = WORKLOADS[default]
+    cfg = bench.workload_config(spec, 1)
+    assert cfg["workload"] == "qwen3-omni-30b-48L-b8-ctx65536"
+    assert cfg["layers"] == 48 and cfg["global_batch"] == 8 and cfg["context"] == 65536
+    assert bench.workload_config(spec, 1) == cfg
+
+
+def test_oracle_sample_is_bounded():
+    """The timed oracle sample of the big workloads is one layer of at most four
+    sequences; small workloads are timed (nearly) whole."""
+    from synth.workloads import WORKLOADS
+    assert bench.oracle_sample_shape(WORKLOADS["omni30b-b8"]) == (1, 4)
+    assert bench.oracle_sample_shape(WORKLOADS["omni3b-b1"]) == (12, 1)
+    assert bench.oracle_sample_shape(WORKLOADS["tiny"]) == (1, 1)
+
+
+def test_one_core_context_restores_affinity():
+    before = os.sched_getaffinity(0)
+    with bench.OneCore():
+        assert len(os.sched_getaffinity(0)) == 1
+    assert os.sched_getaffinity(0) == before
 
 
 def test_peak_source():
