@@ -11,9 +11,10 @@
 //
 // The scratch is a file-scope __device__ array of kScratchBytes (8 MiB) that
 // every GPU loading this library holds until the process exits. Host code only
-// sees a stand-in for it, so its device address is looked up once per device
-// with cudaGetSymbolAddress (on the first call made with that device current)
-// and passed to the kernels. All calls share the one array and it keeps the last
+// sees a stand-in for it, so its device address is looked up with
+// cudaGetSymbolAddress once per device and context (on the first call made with
+// that device current, and again after the device's context is recreated) and
+// passed to the kernels. All calls share the one array and it keeps the last
 // call's contents: nothing in it needs to start at zero (every split the combine
 // reads is written first by the same call), but calls that overlap on the GPU --
 // on different streams, or from different host threads -- race on it.
@@ -34,19 +35,48 @@ constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) uint8_t g_decode_scratch[kScratchBytes];
 
-std::atomic<void*> g_scratch_addr[kMaxDevices];
+// The array's device address per device, with the context it was looked up in:
+// a device reset (or any new context of the device) loads the module again,
+// possibly at another address, so the address is looked up again when the
+// current context differs from the one cached.
+struct ScratchAddr {
+  std::atomic<void*> ctx{nullptr};
+  std::atomic<void*> addr{nullptr};
+};
+ScratchAddr g_scratch[kMaxDevices];
 
-// Device address of g_decode_scratch on the current device (set up once).
+using CtxGetCurrentFn = int (*)(void** ctx);  // the driver's cuCtxGetCurrent (CUresult, CUcontext*)
+
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      f = nullptr;
+    return reinterpret_cast<CtxGetCurrentFn>(f);
+  }();
+  return fn;
+}
+
+// Device address of g_decode_scratch in the current context of the current device.
 cudaError_t scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  void* p = g_scratch_addr[dev].load(std::memory_order_acquire);
-  if (p == nullptr) {
-    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+  const CtxGetCurrentFn get = ctx_get_current();
+  if (get == nullptr) return cudaErrorInitializationError;
+  void* ctx = nullptr;  // null until the runtime has made its context current on this thread
+  if (get(&ctx) != 0) return cudaErrorInitializationError;
+  ScratchAddr& c = g_scratch[dev];
+  void* p = c.addr.load(std::memory_order_acquire);
+  if (p == nullptr || ctx == nullptr || c.ctx.load(std::memory_order_acquire) != ctx) {
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);  // makes the runtime's context current
     if (e != cudaSuccess) return e;
-    g_scratch_addr[dev].store(p, std::memory_order_release);
+    if (get(&ctx) != 0 || ctx == nullptr) return cudaErrorInitializationError;
+    c.addr.store(p, std::memory_order_release);
+    c.ctx.store(ctx, std::memory_order_release);
   }
   *out = p;
   return cudaSuccess;

@@ -20,8 +20,9 @@
  * Conventions for every entry point:
  *   - All tensor pointers are DEVICE pointers owned by the caller, except the
  *     configuration and cache structs themselves, which live in host memory.
- *     The library allocates nothing, frees nothing, never synchronises the
- *     device and keeps no global state.
+ *     The library allocates nothing, frees nothing and never synchronises the
+ *     device. It keeps no global state, with one exception: omnikv_decode_static
+ *     (below) keeps its split partials in a fixed device array of the library.
  *   - `stream` is a cudaStream_t (passed as void*); NULL means the legacy
  *     default stream. All work is stream-ordered on it.
  *   - Host-side validation runs before any launch; a failed check returns an
@@ -224,8 +225,9 @@ OMNIKV_API omnikv_status omnikv_combine_step(const omnikv_config* cfg, omnikv_ca
  * Errors: OMNIKV_ERR_CAPACITY if the partials do not fit (an explicit num_splits too large, or
  * batch * num_q_heads above 5405); OMNIKV_ERR_CUDA if the array's device address cannot be obtained.
  * Every GPU that loads the library holds the array until the process exits. Its device address is
- * looked up (cudaGetSymbolAddress) by the first call made on each device; make that first call
- * before any stream capture. All calls share the array, which keeps the last call's contents (no
+ * looked up (cudaGetSymbolAddress) by the first call made on each device, and again by the first
+ * call made in a new context of that device (after cudaDeviceReset, for example); make that first
+ * call before any stream capture. All calls share the array, which keeps the last call's contents (no
  * part of it needs to start at zero); calls that overlap on the GPU race on it, so run them on one
  * stream or otherwise ordered. */
 #define OMNIKV_DECODE_STATIC_SCRATCH_BYTES (8u << 20)

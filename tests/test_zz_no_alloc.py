@@ -4,14 +4,17 @@ It exists for callers that cannot allocate device memory while decoding: an
 engine that reserved nearly all device memory for its own pool, a plug-in whose
 host framework owns every allocation, a latency-critical loop that cannot pay for
 cudaMalloc. It keeps the split partials in the library's fixed device array, so
-its results must equal those of omnikv_decode_attention + omnikv_combine with a
-caller-allocated partials buffer, call after call, even though the array still
-holds the previous call's contents.
+its results must equal -- bit for bit, at the same split count -- those of
+omnikv_decode_attention + omnikv_combine with a caller-allocated partials buffer,
+call after call, even though the array still holds the previous call's contents;
+and, like them, the oracle's fp64 attention over the same dequantised cache within
+the decode tolerance.
 
 This file is collected last so that a stop-at-first-failure run has already run
 every other test.
 """
 import ctypes
+import dataclasses
 
 import numpy as np
 import pytest
@@ -19,9 +22,14 @@ import torch
 
 from bit_kv_cache_pack_b200 import _abi
 from bit_kv_cache_pack_b200._abi import OmniKVCache, OmniKVConfig
+from oracle import codec
+from oracle.attention import decode_dense
 from synth.workloads import WORKLOADS, key_drift, prefill_inputs, seq_lengths
 
-from helpers import check_decode, make_layer, seeded_randn
+from helpers import check_decode, make_layer, seeded_randn, upload_oracle_cache
+
+SCRATCH_BYTES = 8 << 20   # OMNIKV_DECODE_STATIC_SCRATCH_BYTES
+PARTIAL_BYTES = 1552      # one split-K partials entry
 
 
 def test_static_scratch_rejects_what_does_not_fit():
@@ -40,33 +48,73 @@ def test_static_scratch_rejects_what_does_not_fit():
         _abi.OMNIKV_ERR_INVALID_ARG
 
 
+def _oracle_cache(spec, seed, ocfg, params):
+    """The oracle's own cache of the workload's prefill (never the GPU's), and its
+    capacity in tokens."""
+    L = seq_lengths(spec, seed)
+    cap = int(-(-int(L.max()) // 32) * 32) + 32
+    drift = key_drift(spec, seed, 0, cap // 32, "cpu")
+    k, v, mod = prefill_inputs(spec, seed, 0, params, drift, L, "cpu")
+    oc = codec.OracleCache(spec.batch, spec.num_kv_heads, cap, spec.key_bits, spec.value_bits)
+    codec.write_cache(ocfg, oc, k.numpy(), v.numpy(), mod.numpy())
+    return oc
+
+
+def _allocated(m, consts, cache, q, S):
+    B, Hq = q.shape[:2]
+    part = m.partials_tensor(B, Hq, S, q.device)
+    out = torch.empty(B, Hq, 128, dtype=torch.float32, device=q.device)
+    m.omnikv_decode_attention(consts.struct, cache.struct, q, part, S)
+    m.omnikv_combine(consts.struct, cache.struct, part, S, out)
+    torch.cuda.synchronize()
+    return out.cpu().numpy()
+
+
+def _static(m, consts, cache, q, S):
+    B, Hq = q.shape[:2]
+    out = torch.full((B, Hq, 128), float("nan"), dtype=torch.float32, device=q.device)
+    m.omnikv_decode_static(consts.struct, cache.struct, q, out, S)
+    torch.cuda.synchronize()
+    return out.cpu().numpy()
+
+
 @pytest.mark.gpu
 def test_static_scratch_matches_allocated_partials(cuda_device):
+    """Two calls in a row (different queries and split counts; the second runs
+    over the first's leftover scratch contents): bit-identical to the allocating
+    entry points at the same split count, and within tolerance of the oracle."""
     import bit_kv_cache_pack_b200 as m
     spec, seed = WORKLOADS["tiny"], 21
-    params, consts, _ = make_layer(spec, seed, 0, cuda_device)
-    L = seq_lengths(spec, seed)
-    drift = key_drift(spec, seed, 0, 65, cuda_device)
-    k, v, mod = prefill_inputs(spec, seed, 0, params, drift, L, cuda_device)
-    cache = m.KVCache(1, spec.num_kv_heads, 2080, 2, 2, cuda_device)
-    m.omnikv_write_cache(consts.struct, cache.struct, k, v, mod, int(L[0]))
-
-    def with_allocated_partials(q, S):
-        S = S or m.omnikv_default_splits(consts.struct, cache.struct)
-        part = m.partials_tensor(1, spec.num_q_heads, S, cuda_device)
-        out = torch.empty(1, spec.num_q_heads, 128, dtype=torch.float32, device=cuda_device)
-        m.omnikv_decode_attention(consts.struct, cache.struct, q, part, S)
-        m.omnikv_combine(consts.struct, cache.struct, part, S, out)
-        torch.cuda.synchronize()
-        return out.cpu().numpy().astype(np.float64)
-
-    # two calls in a row, different queries and split counts: the second call
-    # runs over the first call's leftover scratch contents
+    params, consts, ocfg = make_layer(spec, seed, 0, cuda_device)
+    oc = _oracle_cache(spec, seed, ocfg, params)
+    cache = upload_oracle_cache(oc, cuda_device)
     for call, (qseed, S) in enumerate([(1, 7), (2, 0)]):
         q = seeded_randn((1, spec.num_q_heads, 128), cuda_device, qseed).half()
-        ref = with_allocated_partials(q, S)
-        out = torch.full((1, spec.num_q_heads, 128), float("nan"), dtype=torch.float32, device=cuda_device)
-        m.omnikv_decode_static(consts.struct, cache.struct, q, out, S)
-        torch.cuda.synchronize()
-        check_decode(out.cpu().numpy(), ref, "static scratch, call %d" % (call + 1))
+        S_used = S or m.omnikv_default_splits(consts.struct, cache.struct)
+        got = _static(m, consts, cache, q, S)
+        assert np.array_equal(got, _allocated(m, consts, cache, q, S_used)), "call %d" % (call + 1)
+        check_decode(got, decode_dense(ocfg, oc, q.cpu().numpy()), "static scratch, call %d" % (call + 1))
+    assert int(cache.error_word.item()) == 0
+
+
+@pytest.mark.gpu
+def test_static_scratch_lowers_the_default_split_count(cuda_device):
+    """Batch 64 x 16 query heads: the default split count does not fit the array
+    (5405 entries hold 5 splits), so the call lowers it to 5 -- which also moves the
+    decode to longer splits -- and must equal the allocating path at 5 splits."""
+    import bit_kv_cache_pack_b200 as m
+    spec = dataclasses.replace(WORKLOADS["tiny"], batch=64)
+    seed = 23
+    params, consts, ocfg = make_layer(spec, seed, 0, cuda_device)
+    oc = _oracle_cache(spec, seed, ocfg, params)
+    cache = upload_oracle_cache(oc, cuda_device)
+    fit = SCRATCH_BYTES // (spec.batch * spec.num_q_heads * PARTIAL_BYTES)
+    assert fit == 5
+    default = m.omnikv_default_splits(consts.struct, cache.struct)
+    assert default > fit
+    for call in range(2):
+        q = seeded_randn((spec.batch, spec.num_q_heads, 128), cuda_device, 40 + call).half()
+        got = _static(m, consts, cache, q, 0)
+        assert np.array_equal(got, _allocated(m, consts, cache, q, fit)), "call %d" % (call + 1)
+        check_decode(got, decode_dense(ocfg, oc, q.cpu().numpy()), "static scratch, batch 64, call %d" % (call + 1))
     assert int(cache.error_word.item()) == 0
