@@ -23,13 +23,17 @@ OMNIKV_DEVERR_CAPACITY = 0x1
 OMNIKV_DEVERR_MODALITY = 0x2
 OMNIKV_DEVERR_TIMEOUT = 0x4
 OMNIKV_DEVERR_BOUND = 0x8
+OMNIKV_DEVERR_RANGE = 0x10
+OMNIKV_META_FP16 = 0
+OMNIKV_META_MXFP4 = 1
 
 EXPORTED = (
     "omnikv_record_bytes", "omnikv_partials_bytes", "omnikv_default_splits",
     "omnikv_write_cache", "omnikv_decode_attention", "omnikv_combine",
     "omnikv_status_string", "omnikv_abi_version", "omnikv_decode_static",
     "omnikv_dense_partials_bytes", "omnikv_dense_decode_bf16", "omnikv_decode_step",
-    "omnikv_append_decode", "omnikv_combine_step", "omnikv_step_splits",
+    "omnikv_append_decode", "omnikv_combine_step", "omnikv_step_splits", "omnikv_write_cache_rotations",
+    "omnikv_test_decode_pending", "omnikv_record_bytes_meta",
 )
 OMNIKV_DECODE_STATIC_SCRATCH_BYTES = 8 << 20
 
@@ -52,6 +56,7 @@ class OmniKVConfig(ctypes.Structure):
         ("value_codebook", ctypes.c_void_p),
         ("key_signs", ctypes.c_void_p),
         ("value_rot", ctypes.c_void_p),
+        ("key_meta_format", ctypes.c_int32),
     ]
 
 
@@ -84,10 +89,15 @@ def load() -> ctypes.CDLL:
     P, I32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
     cfgp, cachep = ctypes.POINTER(OmniKVConfig), ctypes.POINTER(OmniKVCache)
     lib.omnikv_record_bytes.argtypes, lib.omnikv_record_bytes.restype = [I32, I32], SZ
+    lib.omnikv_record_bytes_meta.argtypes, lib.omnikv_record_bytes_meta.restype = [I32, I32, I32], SZ
     lib.omnikv_partials_bytes.argtypes, lib.omnikv_partials_bytes.restype = [I32, I32, I32], SZ
     lib.omnikv_default_splits.argtypes, lib.omnikv_default_splits.restype = [cfgp, cachep], I32
     lib.omnikv_write_cache.argtypes = [cfgp, cachep, P, P, P, I32, P]
     lib.omnikv_write_cache.restype = ctypes.c_int
+    lib.omnikv_write_cache_rotations.argtypes = [cfgp, cachep, P, P, P, I32, P, P]
+    lib.omnikv_write_cache_rotations.restype = ctypes.c_int
+    lib.omnikv_test_decode_pending.argtypes = [cfgp, cachep, P, P, I32, ctypes.c_uint64, P]
+    lib.omnikv_test_decode_pending.restype = ctypes.c_int
     lib.omnikv_decode_attention.argtypes = [cfgp, cachep, P, P, I32, P]
     lib.omnikv_decode_attention.restype = ctypes.c_int
     lib.omnikv_combine.argtypes = [cfgp, cachep, P, I32, P, P]
@@ -148,6 +158,10 @@ def omnikv_record_bytes(key_bits: int, value_bits: int) -> int:
     return int(load().omnikv_record_bytes(key_bits, value_bits))
 
 
+def omnikv_record_bytes_meta(key_bits: int, value_bits: int, key_meta_format: int) -> int:
+    return int(load().omnikv_record_bytes_meta(key_bits, value_bits, key_meta_format))
+
+
 def omnikv_partials_bytes(batch: int, num_q_heads: int, num_splits: int) -> int:
     return int(load().omnikv_partials_bytes(batch, num_q_heads, num_splits))
 
@@ -161,6 +175,20 @@ def omnikv_write_cache(cfg: OmniKVConfig, cache: OmniKVCache, k_new, v_new, moda
     st = load().omnikv_write_cache(ctypes.byref(cfg), ctypes.byref(cache), _ptr(k_new), _ptr(v_new),
                                    _ptr(modality_new), int(n_new), _stream(stream))
     _check(st, "omnikv_write_cache")
+
+
+def omnikv_write_cache_rotations(cfg: OmniKVConfig, cache: OmniKVCache, k_new, v_new, modality_new, n_new: int,
+                                 v_rot, stream=None) -> None:
+    st = load().omnikv_write_cache_rotations(ctypes.byref(cfg), ctypes.byref(cache), _ptr(k_new), _ptr(v_new),
+                                             _ptr(modality_new), int(n_new), _ptr(v_rot), _stream(stream))
+    _check(st, "omnikv_write_cache_rotations")
+
+
+def omnikv_test_decode_pending(cfg: OmniKVConfig, cache: OmniKVCache, q, partials, num_splits: int,
+                               flag_wait_ns: int, stream=None) -> None:
+    st = load().omnikv_test_decode_pending(ctypes.byref(cfg), ctypes.byref(cache), _ptr(q), _ptr(partials),
+                                           int(num_splits), int(flag_wait_ns), _stream(stream))
+    _check(st, "omnikv_test_decode_pending")
 
 
 def omnikv_decode_attention(cfg: OmniKVConfig, cache: OmniKVCache, q, partials, num_splits: int = 0,

@@ -34,7 +34,7 @@ def _nvcc() -> str:
 def build(verbose_ptxas: bool = False, force: bool = False) -> str:
     sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     headers = glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh")) + \
-        [os.path.join(ROOT, "include", "omnikv.h")]
+        glob.glob(os.path.join(ROOT, "include", "*.h"))
     os.makedirs(BUILD_DIR, exist_ok=True)
     newest_header = max(os.path.getmtime(h) for h in headers)
     objs = []

@@ -2,6 +2,7 @@
 // Every check runs on the host before any launch; see include/omnikv.h.
 #include <cuda_runtime.h>
 
+#include "../../include/omnikv_testing.h"
 #include "abi_internal.h"
 #include "common.cuh"
 #include "kernels.h"
@@ -23,6 +24,8 @@ omnikv_status check_config(const omnikv_config* cfg) {
   if (!cfg->key_codebook || !cfg->value_codebook || !cfg->key_signs || !cfg->value_rot)
     return OMNIKV_ERR_INVALID_ARG;
   if (!aligned(cfg->key_signs, 16) || !aligned(cfg->value_rot, 16)) return OMNIKV_ERR_INVALID_ARG;
+  if (cfg->key_meta_format != OMNIKV_META_FP16 && cfg->key_meta_format != OMNIKV_META_MXFP4)
+    return OMNIKV_ERR_UNSUPPORTED;
   return OMNIKV_OK;
 }
 
@@ -107,6 +110,7 @@ omnikv_status prepare_decode(const omnikv_config* cfg, const omnikv_cache* cache
   p->value_rot = cfg->value_rot;
   p->key_bits = cfg->key_bits;
   p->value_bits = cfg->value_bits;
+  p->key_meta = cfg->key_meta_format == OMNIKV_META_MXFP4 ? kMetaMx : kMetaFp16;
   p->num_kv_heads = cfg->num_kv_heads;
   p->group = cfg->num_q_heads / cfg->num_kv_heads;
   p->records = static_cast<const uint8_t*>(cache->records);
@@ -124,6 +128,7 @@ omnikv_status prepare_decode(const omnikv_config* cfg, const omnikv_cache* cache
   p->batch = cache->batch;
   p->len_add = 0;
   p->step_flags = nullptr;
+  p->flag_wait_ns = kFlagWaitNs;
   return OMNIKV_OK;
 }
 
@@ -162,6 +167,12 @@ size_t omnikv_record_bytes(int32_t key_bits, int32_t value_bits) {
   return (size_t)RecordLayout(key_bits, value_bits).bytes;
 }
 
+size_t omnikv_record_bytes_meta(int32_t key_bits, int32_t value_bits, int32_t key_meta_format) {
+  if ((key_bits != 2 && key_bits != 4) || (value_bits != 2 && value_bits != 4)) return 0;
+  if (key_meta_format != OMNIKV_META_FP16 && key_meta_format != OMNIKV_META_MXFP4) return 0;
+  return (size_t)RecordLayout(key_bits, value_bits, key_meta_format == OMNIKV_META_MXFP4 ? kMetaMx : kMetaFp16).bytes;
+}
+
 size_t omnikv_partials_bytes(int32_t batch, int32_t num_q_heads, int32_t num_splits) {
   if (batch < 1 || num_q_heads < 1 || num_splits < 1) return 0;
   return (size_t)batch * num_q_heads * num_splits * sizeof(Partial);
@@ -182,6 +193,7 @@ void fill_write_params(const omnikv_config* cfg, const omnikv_cache* cache, cons
   p->value_rot = cfg->value_rot;
   p->key_bits = cfg->key_bits;
   p->value_bits = cfg->value_bits;
+  p->key_meta = cfg->key_meta_format == OMNIKV_META_MXFP4 ? kMetaMx : kMetaFp16;
   p->num_kv_heads = cfg->num_kv_heads;
   p->records = static_cast<uint8_t*>(cache->records);
   p->key_tail = static_cast<__half*>(cache->key_tail);
@@ -196,6 +208,7 @@ void fill_write_params(const omnikv_config* cfg, const omnikv_cache* cache, cons
   p->n_new = n_new;
   p->tc_values = 0;
   p->step_flags = nullptr;
+  p->vrot_dump = nullptr;
 }
 
 }  // namespace
@@ -211,6 +224,23 @@ omnikv_status omnikv_write_cache(const omnikv_config* cfg, omnikv_cache* cache, 
   if ((long long)cache->max_seq_len + n_new > cache->cap_tokens) return OMNIKV_ERR_CAPACITY;
   WriteParams p;
   fill_write_params(cfg, cache, k_new, v_new, modality_new, n_new, &p);
+  if (launch_write(p, cache->batch, static_cast<cudaStream_t>(stream)) != cudaSuccess) return OMNIKV_ERR_CUDA;
+  cache->max_seq_len += n_new;
+  return OMNIKV_OK;
+}
+
+omnikv_status omnikv_write_cache_rotations(const omnikv_config* cfg, omnikv_cache* cache, const void* k_new,
+                                           const void* v_new, const uint8_t* modality_new, int32_t n_new,
+                                           float* v_rot, void* stream) {
+  omnikv_status st = check_config(cfg);
+  if (st != OMNIKV_OK) return st;
+  if ((st = check_cache(cache)) != OMNIKV_OK) return st;
+  if (n_new < 1 || !k_new || !v_new || !modality_new || !v_rot) return OMNIKV_ERR_INVALID_ARG;
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(v_rot, 16)) return OMNIKV_ERR_INVALID_ARG;
+  if ((long long)cache->max_seq_len + n_new > cache->cap_tokens) return OMNIKV_ERR_CAPACITY;
+  WriteParams p;
+  fill_write_params(cfg, cache, k_new, v_new, modality_new, n_new, &p);
+  p.vrot_dump = v_rot;
   if (launch_write(p, cache->batch, static_cast<cudaStream_t>(stream)) != cudaSuccess) return OMNIKV_ERR_CUDA;
   cache->max_seq_len += n_new;
   return OMNIKV_OK;
@@ -260,6 +290,24 @@ void plan_step(const omnikv_config* cfg, const omnikv_cache* after, int32_t num_
 }  // namespace
 
 extern "C" {
+
+omnikv_status omnikv_test_decode_pending(const omnikv_config* cfg, const omnikv_cache* cache, const void* q,
+                                         void* partials, int32_t num_splits, uint64_t flag_wait_ns, void* stream) {
+  omnikv_status st = check_config(cfg);
+  if (st != OMNIKV_OK) return st;
+  if ((st = check_cache(cache)) != OMNIKV_OK) return st;
+  if (!cache->step_flags || !aligned(cache->step_flags, 4)) return OMNIKV_ERR_INVALID_ARG;
+  if ((long long)cache->max_seq_len + 1 > cache->cap_tokens) return OMNIKV_ERR_CAPACITY;
+  omnikv_cache after = *cache;  // the decode reads the cache as if the token were appended
+  after.max_seq_len += 1;
+  DecodeParams dp;
+  if ((st = prepare_decode(cfg, &after, q, partials, num_splits, &dp)) != OMNIKV_OK) return st;
+  dp.len_add = 1;
+  dp.step_flags = cache->step_flags;
+  dp.flag_wait_ns = flag_wait_ns;
+  if (launch_decode(dp, cache->batch, static_cast<cudaStream_t>(stream)) != cudaSuccess) return OMNIKV_ERR_CUDA;
+  return OMNIKV_OK;
+}
 
 int32_t omnikv_step_splits(const omnikv_config* cfg, const omnikv_cache* cache, int32_t num_splits, int32_t* fused) {
   if (check_config(cfg) != OMNIKV_OK || check_cache(cache) != OMNIKV_OK || num_splits < 0) return 0;

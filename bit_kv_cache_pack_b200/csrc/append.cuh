@@ -83,7 +83,7 @@ __device__ void quantize_window(const WriteParams& p, int b, int h, int w, int L
   const int nvalid = p1 - p0;
   const int inew0 = max(L0 - p0, 0);  // first slot of this window holding a new token
 
-  const RecordLayout lay(p.key_bits, p.value_bits);
+  const RecordLayout lay(p.key_bits, p.value_bits, p.key_meta);
   uint8_t* rec = p.records + ((size_t)(b * H + h) * p.cap_windows + w) * lay.bytes;
   const size_t seq_head = (size_t)b * H + h;
   __half* tail = p.key_tail + seq_head * kWindow * kHeadDim;
@@ -208,11 +208,43 @@ __device__ void quantize_window(const WriteParams& p, int b, int h, int w, int L
       mn = fminf(mn, v);
       mx = fmaxf(mx, v);
     }
-    const __half m16 = __float2half_rn(mn);
-    const __half s16 = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), kspan));
-    reinterpret_cast<__half2*>(rec + lay.meta_off)[c] = __halves2half2(m16, s16);
-    s_min[c] = __half2float(m16);
-    s_scale[c] = __half2float(s16);
+    if (p.key_meta == kMetaMx) {
+      // MXFP4: the warp's 32 channels form one block. The minimum is rounded to
+      // the nearest E2M1 value of its block's exponent, then the scale it needs,
+      // fp32((max - m^) / (c_last - c_0)) (0 if negative), on the scale block's grid.
+      uint8_t* meta = rec + lay.meta_off;
+      float am = fabsf(mn);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+      const int em = mx_block_exp(am);
+      uint32_t mcode, scode;
+      const float mhat = mx_round_nearest(mn, em, &mcode);
+      const float sreq = fmaxf(__fdiv_rn(__fsub_rn(mx, mhat), kspan), 0.0f);
+      float as = sreq;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) as = fmaxf(as, __shfl_xor_sync(0xffffffffu, as, o));
+      const int es = mx_block_exp(as);
+      const float shat = mx_round_nearest(sreq, es, &scode);
+      const uint32_t mnext = __shfl_down_sync(0xffffffffu, mcode, 1);
+      const uint32_t snext = __shfl_down_sync(0xffffffffu, scode, 1);
+      if (!(c & 1)) {  // byte c / 2: channel c in the low nibble, c + 1 in the high one
+        meta[c >> 1] = (uint8_t)(mcode | (mnext << 4));
+        meta[64 + (c >> 1)] = (uint8_t)(scode | (snext << 4));
+      }
+      if ((c & 31) == 0) {
+        meta[128 + (c >> 5)] = (uint8_t)(em + 127);
+        meta[132 + (c >> 5)] = (uint8_t)(es + 127);
+      }
+      if (c < 8) meta[136 + c] = 0;
+      s_min[c] = mhat;
+      s_scale[c] = shat;
+    } else {
+      const __half m16 = __float2half_rn(mn);
+      const __half s16 = __float2half_rn(__fdiv_rn(__fsub_rn(mx, mn), kspan));
+      reinterpret_cast<__half2*>(rec + lay.meta_off)[c] = __halves2half2(m16, s16);
+      s_min[c] = __half2float(m16);
+      s_scale[c] = __half2float(s16);
+    }
   }
   group_sync(bar_id);
 
@@ -276,6 +308,7 @@ __device__ void quantize_window(const WriteParams& p, int b, int h, int w, int L
 #pragma unroll  // every load of the column issued before the first FMA needs it
       for (int c = 0; c < kHeadDim; ++c) part[c & 7] = fmaf(U[(size_t)c * kHeadDim], kp[i][c], part[c & 7]);
       const float acc = ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
+      if (p.vrot_dump) p.vrot_dump[((size_t)(b * H + h) * p.n_new + (p0 + i - L0)) * kHeadDim + j] = acc;
       const float s = s_sigma[i];
       uint32_t code = 0;  // #{j : v' / sigma > t_j}, 0 where sigma == 0
       if (s != 0.0f)

@@ -21,19 +21,65 @@ constexpr int kMaxGroup = 8;  // query heads per kv head handled by one CTA
 // fp32(2^-3.5) = fp32(1/sqrt(128)), bit pattern 0x3DB504F3
 __device__ __forceinline__ float inv_sqrt_d() { return __int_as_float(0x3DB504F3); }
 
+// Key metadata formats of a window: fp16 (m, s) pairs per channel (512 B), or
+// MXFP4 -- E2M1 elements sharing an E8M0 exponent per 32 channels (144 B).
+constexpr int kMetaFp16 = 0, kMetaMx = 1;
+constexpr int kMetaFp16Bytes = 512, kMetaMxBytes = 144;
+
+__host__ __device__ constexpr int meta_bytes_of(int key_meta) { return key_meta == kMetaMx ? kMetaMxBytes : kMetaFp16Bytes; }
+
 struct RecordLayout {
   int k_off, meta_off, v_off, sigma_off, bytes;
   int key_bits, value_bits;
-  __host__ __device__ RecordLayout(int kb, int vb) : key_bits(kb), value_bits(vb) {
+  __host__ __device__ RecordLayout(int kb, int vb, int key_meta = kMetaFp16) : key_bits(kb), value_bits(vb) {
     const int kbytes = kWindow * kHeadDim * kb / 8;
     const int vbytes = kWindow * kHeadDim * vb / 8;
     k_off = 0;
     meta_off = kbytes;
-    v_off = meta_off + kHeadDim * 4;
+    v_off = meta_off + meta_bytes_of(key_meta);
     sigma_off = v_off + vbytes;
     bytes = sigma_off + kWindow * 2;
   }
 };
+
+// ---- MXFP4 key metadata (E2M1 elements, one E8M0 exponent per 32 channels) ----
+// The shared exponent of a block: the smallest e in [-127, 127] with
+// amax <= 6 * 2^e (no element saturates); -127 for an all-zero block.
+__device__ __forceinline__ int mx_block_exp(float amax) {
+  if (!(amax > 0.0f)) return -127;
+  const int f = ilogbf(amax);  // 2^f <= amax < 2^(f + 1)
+  int e = (amax <= ldexpf(1.5f, f)) ? f - 2 : f - 1;  // 6 * 2^(f-2) = 1.5 * 2^f
+  return max(-127, min(127, e));
+}
+
+// Value of an E2M1 code (sign << 3 | magnitude index; magnitudes 0, 0.5, 1, 1.5,
+// 2, 3, 4, 6) times 2^e, exact in fp32 (subnormal results included).
+__device__ __forceinline__ float mx_value(uint32_t code, int e) {
+  const uint32_t idx = code & 7u;
+  float v = 0.0f;
+  if (idx != 0u) {
+    const int ex = (idx >= 2u ? (int)(idx >> 1) - 1 : -1) + e;  // 2^ex * (1 or 1.5)
+    const bool half_up = idx >= 2u && (idx & 1u);
+    if (ex > 127)
+      v = INFINITY;
+    else if (ex >= -126)
+      v = __uint_as_float(((uint32_t)(ex + 127) << 23) | (half_up ? (1u << 22) : 0u));
+    else
+      v = ldexpf(half_up ? 1.5f : 1.0f, ex);
+  }
+  return (code & 8u) ? -v : v;
+}
+
+// Nearest E2M1 grid value g * 2^e to x (|x| <= 6 * 2^e), ties to the even code;
+// a zero is coded +0. Returns the value; *code receives the E2M1 code.
+__device__ __forceinline__ float mx_round_nearest(float x, int e, uint32_t* code) {
+  const float a = fabsf(ldexpf(x, -e));  // exact scaling by a power of two
+  // midpoints 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5: a tie goes to the even index
+  uint32_t idx = (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) + (a > 2.5f) + (a >= 3.5f) + (a > 5.0f);
+  const uint32_t c = idx | ((idx != 0u && x < 0.0f) ? 8u : 0u);
+  *code = c;
+  return mx_value(c, e);
+}
 
 // One entry of the split-K partials buffer.
 struct __align__(16) Partial {

@@ -63,30 +63,36 @@
 // the cache (query rotation, score operand, L2 prefetch of the value bases for the
 // combine) runs before griddepcontrol.wait.
 //
-// Inputs must stay in the fp16 range of the operands: |q' s_gc| / sqrt(128)
-// below ~480 and value scales sigma below ~480; outside it the output is not
-// finite (the data would have to be far outside any realistic key / value range).
+// Operand range: the score operand carries a per-CTA power of two, so queries of
+// any finite magnitude are exact to ~22 bits; key scales s_gc up to 32752 (the
+// A operand holds s_gc * 2) and value scales sigma below 565 (the value operand
+// holds p sigma (c_1 - c_0) 128 with p <= 1) stay inside fp16. Beyond them a
+// split's partial is not finite: it is written empty (weight 0 in the combine) and
+// OMNIKV_DEVERR_RANGE is set. Key scales below 2^-7 lose relative precision in the
+// s_gc * 2^-7 plane (fp16 subnormals); realistic key ranges are far above.
 #include <atomic>
 
-#include "append.cuh"
-#include "common.cuh"
-#include "kernels.h"
-#include "ptx.cuh"
+#include "decode_common.cuh"
 
 namespace omnikv {
 
 namespace {
 
-constexpr int kWarps = 4;
-constexpr int kThreads = 32 * kWarps;
 constexpr int kStages = 3;                      // per-warp body: windows in flight per warp
-constexpr int kRec22 = 2624;                    // K2/V2 record bytes
+constexpr int kRec22 = 2624;                    // K2/V2 record bytes with fp16 key metadata (the largest)
 constexpr int kStageBytes = kRec22 + kWindow;   // record + modality ids
+
+// Offsets of a K2/V2 record with key metadata format kMeta.
+template <int kMeta>
+struct Rec22 {
+  static constexpr int meta = 1024;
+  static constexpr int v = meta + meta_bytes_of(kMeta);
+  static constexpr int sigma = v + 1024;
+  static constexpr int bytes = sigma + 64;
+};
 constexpr int kCoop = kWarps;                   // cooperative body: windows per group (one per warp for the scores)
 constexpr int kCoopStages = 2;                  // cooperative body: window groups in flight per CTA
 constexpr int kGroupBytes = kCoop * kStageBytes;  // kCoop records, then their modality ids
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: a bulk copy that takes longer is an error
-constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kTmemCols = 128;  // per-warp body, per CTA: 3 parked accumulators x 32 columns in each warp's lanes
 
 struct __align__(16) DecodeSmem {
@@ -108,381 +114,13 @@ struct __align__(16) DecodeSmem {
   float red[kWarps][1 + kMods][kMaxGroup];        // cooperative body: per-warp sums of p and of p sigma per modality
   uint32_t tmask[kCoop][2];                       // cooperative body: modality bits of each tile of the group (0: no window)
   uint32_t tmem_base;                             // per-warp body: TMEM columns of the parked accumulators
+  uint32_t mxpairs[kWarps][kHeadDim];             // MXFP4 caches: a warp's window metadata as fp16 (m, s) pairs
+  uint32_t bad_heads;                             // bit h: head h's partial is not finite (written empty)
+  int abort;                                      // cooperative body: a step flag never arrived
+  int wabort[kWarps];                             // per-warp body: a step flag of warp w never arrived
 };
 static_assert(sizeof(DecodeSmem) <= 48 * 1024, "static shared memory");
-
-// Position of channel c of head g in the rotated-query buffer. Chunks of 4
-// channels inside each group of 32 are XOR-swizzled so that the 8 lanes of a
-// quarter warp (heads g, g+1 x channel groups t = 0..3) reading chunk i read 8
-// different bank groups.
-__device__ __forceinline__ int qpos(int g, int c) {
-  const int t = c >> 5, i4 = (c >> 2) & 7;
-  return g * kHeadDim + 32 * t + 4 * (i4 ^ ((4 * (g & 1) + t) & 7)) + (c & 3);
-}
-
-// q' = fp32(2^-3.5) H (s . q) for every head of the group, times 2^-3.5 more
-// (the softmax scale 1/sqrt(128)); heads >= G are zero. Stored at qpos(g, c).
-__device__ __forceinline__ void rotate_queries(const DecodeParams& p, int b, int kvh, float (*qs)[kHeadDim]) {
-  float* qflat = &qs[0][0];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int G = p.group;
-  const int Hq = p.num_kv_heads * G;
-  float sg[4];
-#pragma unroll
-  for (int r = 0; r < 4; ++r) sg[r] = p.key_signs[4 * lane + r];
-  for (int g = warp; g < kMaxGroup; g += kWarps) {
-    if (g < G) {
-      const __half* q = p.q + ((size_t)b * Hq + kvh * G + g) * kHeadDim;
-      const uint2 raw = *reinterpret_cast<const uint2*>(q + 4 * lane);
-      const __half2 lo = *reinterpret_cast<const __half2*>(&raw.x);
-      const __half2 hi = *reinterpret_cast<const __half2*>(&raw.y);
-      float x[4] = {__low2float(lo), __high2float(lo), __low2float(hi), __high2float(hi)};
-      warp_hadamard_rotate(x, sg);
-#pragma unroll
-      for (int r = 0; r < 4; ++r) qflat[qpos(g, 4 * lane + r)] = x[r] * inv_sqrt_d();
-    } else {
-#pragma unroll
-      for (int r = 0; r < 4; ++r) qflat[qpos(g, 4 * lane + r)] = 0.0f;
-    }
-  }
-}
-
-// Split s covers windows [s C, min((s+1) C, W_b)) of sequence b, with C =
-// p.split_windows chosen on the host from the length bound, so a short sequence
-// leaves its last splits empty and every non-empty split has the same size.
-__device__ __forceinline__ void split_range(const DecodeParams& p, int b, int split, int& T, int& w0, int& w1) {
-  const int L = p.seq_lens[b];
-  const int La = L + p.len_add;  // a decode step's append happens only within the capacity
-  T = max(0, min(La <= p.cap_tokens ? La : L, p.cap_tokens));
-  const int nw = (T + kWindow - 1) / kWindow;
-  w0 = min(split * p.split_windows, nw);
-  w1 = min(w0 + p.split_windows, nw);
-  if (split == p.num_splits - 1 && threadIdx.x == 0 && nw > p.num_splits * p.split_windows)
-    set_error(p.error_word, OMNIKV_DEVERR_BOUND);
-}
-
-// Decode step: the window that receives the appended token, and the flag value
-// that marks its record as written (window -1: nothing to wait for).
-__device__ __forceinline__ void step_window(const DecodeParams& p, int b, int& win, int& val) {
-  win = -1;
-  val = 0;
-  if (p.len_add > 0 && p.step_flags != nullptr) {
-    const int L = p.seq_lens[b];
-    if (L >= 0 && L + p.len_add <= p.cap_tokens) {
-      val = L + p.len_add;
-      win = (val - 1) / kWindow;
-    }
-  }
-}
-
-// Bounded acquire-spin until *flag == val (written with release by the append
-// CTA of the same launch); false after about `limit_ns`.
-__device__ __forceinline__ bool wait_flag(const int32_t* flag, int val, uint64_t limit_ns) {
-  const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 0;; ++it) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
-    if (v == val) break;
-    if ((it & 63u) == 63u && global_timer_ns() - t0 > limit_ns) return false;
-    __nanosleep(64);
-  }
-  // the record is then read through the async proxy (bulk copy)
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-  return true;
-}
-
-// 2^x with the hardware approximation (relative error below 2^-22); -inf -> 0.
-__device__ __forceinline__ float fast_exp2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// ---------------------------------------------------------------------------
-// CUDA-core path (4-bit codes, or a codebook that is not symmetric): the CTA
-// decodes the split's windows one at a time from a double-buffered ring of bulk
-// copies. Scores: four threads per token, thread q of token t holding channels
-// 4 j + q (j = 0..31), each dequantised once, k'_tc = m_c + s_c (c_code - c_0),
-// and used for the 8 query heads; two shuffles complete the dot products.
-// Values: thread c owns channel c and one fp32 accumulator per (modality, head).
-// ---------------------------------------------------------------------------
-constexpr int kGenStages = 2;
-
-struct GenSmem {                 // laid over DecodeSmem::stage
-  uint8_t rec[kGenStages][4704];  // window record + 32 modality ids (largest record: 4672 B)
-  float qT[kHeadDim][kMaxGroup];  // rotated queries, channel-major
-  float pw[kWindow][kMaxGroup];   // p_ht * sigma_t of the current window
-  float dk[16], dv[16];           // c_j - c_0 (keys), c_j (values)
-  float wmax[kWarps][kMaxGroup];
-  uint64_t bar[kGenStages];
-  uint32_t runs;                  // bit t: token t of the current window starts a run of one modality
-};
-static_assert(sizeof(GenSmem) <= sizeof(DecodeSmem::u), "generic path shared memory");
-
-__device__ __forceinline__ void gen_issue(const DecodeParams& p, GenSmem& g, int stage, const uint8_t* rec_base,
-                                          int rec_bytes, int b, int kvh, int wi, int wait_win, int wait_val) {
-  if (wi == wait_win &&
-      !wait_flag(p.step_flags + (size_t)b * p.num_kv_heads + kvh, wait_val, kWaitLimitNs))
-    set_error(p.error_word, OMNIKV_DEVERR_TIMEOUT);
-  mbar_arrive_expect_tx(&g.bar[stage], rec_bytes + kWindow);
-  bulk_copy_g2s(g.rec[stage], rec_base + (size_t)wi * rec_bytes, rec_bytes, &g.bar[stage]);
-  bulk_copy_g2s(g.rec[stage] + rec_bytes, p.modality + (size_t)b * p.cap_tokens + (size_t)wi * kWindow, kWindow,
-                &g.bar[stage]);
-}
-
-template <int KB, int VB>
-__device__ void decode_generic_t(const DecodeParams& p, DecodeSmem& sm, int b, int kvh, int split) {
-  GenSmem& g = *reinterpret_cast<GenSmem*>(&sm.u);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int G = p.group;
-  const int Hq = p.num_kv_heads * G;
-  int T, w0, w1;
-  split_range(p, b, split, T, w0, w1);
-  int wait_win, wait_val;
-  step_window(p, b, wait_win, wait_val);
-  const RecordLayout lay(p.key_bits, p.value_bits);
-  const uint8_t* rec_base = p.records + ((size_t)(b * p.num_kv_heads + kvh) * p.cap_windows) * lay.bytes;
-  const int nwin = w1 - w0;
-  if (tid == 0) {
-    for (int s = 0; s < kGenStages; ++s) mbar_init(&g.bar[s], 1);
-    fence_barrier_init();
-    for (int s = 0; s < kGenStages && s < nwin; ++s) gen_issue(p, g, s, rec_base, lay.bytes, b, kvh, w0 + s, wait_win, wait_val);
-  }
-  const int LK = 1 << p.key_bits, LV = 1 << p.value_bits;
-  if (tid < LK) g.dk[tid] = p.key_cb[tid] - p.key_cb[0];
-  if (tid >= 32 && tid - 32 < LV) g.dv[tid - 32] = p.val_cb[tid - 32];
-#pragma unroll
-  for (int h = 0; h < kMaxGroup; ++h) g.qT[tid][h] = (&sm.q[0][0])[qpos(h, tid)];
-  __syncthreads();
-
-  // score threads: token t = tid / 4, channel phase q = tid % 4
-  const int st = tid >> 2, sq = tid & 3;
-  constexpr uint32_t kmask = (1u << KB) - 1u, vmask = (1u << VB) - 1u;
-  constexpr int kcpw = 32 / KB, kwpt = kHeadDim / kcpw, vcpw = 32 / VB;
-  float m_run[kMaxGroup], l_part[kMaxGroup];  // running max (CTA-uniform), per-thread partial sums of p
-  float acc[kMods][kMaxGroup];               // thread c = tid: channel c
-#pragma unroll
-  for (int h = 0; h < kMaxGroup; ++h) {
-    m_run[h] = -INFINITY;
-    l_part[h] = 0.0f;
-#pragma unroll
-    for (int m = 0; m < kMods; ++m) acc[m][h] = 0.0f;
-  }
-
-  int failed_at = -1;
-  for (int i = 0; i < nwin; ++i) {
-    const int s = i % kGenStages;
-    const int wi = w0 + i;
-    if (__syncthreads_or(!mbar_wait_bounded(&g.bar[s], (i / kGenStages) & 1, kWaitLimitNs))) {
-      failed_at = i;
-      break;
-    }
-    const uint8_t* rec = g.rec[s];
-    const uint32_t* kw = reinterpret_cast<const uint32_t*>(rec + lay.k_off);
-    const __half2* meta = reinterpret_cast<const __half2*>(rec + lay.meta_off);
-    const uint32_t* vw = reinterpret_cast<const uint32_t*>(rec + lay.v_off);
-    const __half* sig = reinterpret_cast<const __half*>(rec + lay.sigma_off);
-    const uint8_t* mods = rec + lay.bytes;
-
-    // ---- scores of token st for the 8 heads over channels 4 j + sq
-    float sc[kMaxGroup];
-#pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h) sc[h] = 0.0f;
-    {
-      uint32_t row[kwpt];  // this token's key words (every channel 4 j + sq of word j * 4 / kcpw)
-#pragma unroll
-      for (int k4 = 0; k4 < kwpt / 4; ++k4) {
-        const uint4 u = reinterpret_cast<const uint4*>(kw + st * kwpt)[k4];
-        row[4 * k4] = u.x;
-        row[4 * k4 + 1] = u.y;
-        row[4 * k4 + 2] = u.z;
-        row[4 * k4 + 3] = u.w;
-      }
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int c = 4 * j + sq;
-        const uint32_t code = (row[(4 * j) / kcpw] >> (KB * (c % kcpw))) & kmask;
-        const float2 ms = __half22float2(meta[c]);
-        const float kv = fmaf(ms.y, g.dk[code], ms.x);
-        const float4 qa = *reinterpret_cast<const float4*>(&g.qT[c][0]);
-        const float4 qb = *reinterpret_cast<const float4*>(&g.qT[c][4]);
-        sc[0] = fmaf(qa.x, kv, sc[0]);
-        sc[1] = fmaf(qa.y, kv, sc[1]);
-        sc[2] = fmaf(qa.z, kv, sc[2]);
-        sc[3] = fmaf(qa.w, kv, sc[3]);
-        sc[4] = fmaf(qb.x, kv, sc[4]);
-        sc[5] = fmaf(qb.y, kv, sc[5]);
-        sc[6] = fmaf(qb.z, kv, sc[6]);
-        sc[7] = fmaf(qb.w, kv, sc[7]);
-      }
-    }
-#pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h) {
-      sc[h] += __shfl_xor_sync(0xffffffffu, sc[h], 1);
-      sc[h] += __shfl_xor_sync(0xffffffffu, sc[h], 2);
-      if (wi * kWindow + st >= T || h >= G) sc[h] = -INFINITY;
-    }
-    // ---- window max per head: lanes of a warp (8 tokens), then the 4 warps
-    float mx[kMaxGroup];
-#pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h) {
-      float v = sc[h];
-      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
-      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
-      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-      mx[h] = v;
-    }
-    if (lane == 0) {
-#pragma unroll
-      for (int h = 0; h < kMaxGroup; ++h) g.wmax[warp][h] = mx[h];
-    }
-    __syncthreads();
-    float alpha[kMaxGroup];
-#pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h) {
-      float v = fmaxf(fmaxf(g.wmax[0][h], g.wmax[1][h]), fmaxf(g.wmax[2][h], g.wmax[3][h]));
-      const float mn = fmaxf(m_run[h], v);
-      alpha[h] = (mn == -INFINITY) ? 1.0f : fast_exp2((m_run[h] - mn) * kLog2e);
-      m_run[h] = mn;
-    }
-    // ---- where the window's modality runs start (warp 0; read after the barrier)
-    if (warp == 0) {
-      const int mt = min((int)mods[lane], kMods - 1);
-      const int mp = lane > 0 ? min((int)mods[lane - 1], kMods - 1) : -1;
-      const uint32_t starts = __ballot_sync(0xffffffffu, mt != mp);
-      if (lane == 0) g.runs = starts;
-    }
-    // ---- p = exp(score - max); thread (st, sq) stores heads 2 sq, 2 sq + 1 of token st
-    {
-      const float sgm = __half2float(sig[st]);
-#pragma unroll
-      for (int h = 0; h < kMaxGroup; ++h) {
-        const float pp = (sc[h] == -INFINITY) ? 0.0f : fast_exp2((sc[h] - m_run[h]) * kLog2e);
-        l_part[h] = l_part[h] * alpha[h] + (sq == 0 ? pp : 0.0f);
-        if ((h >> 1) == sq) g.pw[st][h] = pp * sgm;
-      }
-    }
-    __syncthreads();
-    // ---- values: channel c = tid over the window's valid tokens, taken in runs
-    // of one modality (one accumulator set per run, no per-token selection)
-    {
-      bool grew = false;
-#pragma unroll
-      for (int h = 0; h < kMaxGroup; ++h) grew |= alpha[h] != 1.0f;
-      if (grew) {  // the same decision in every thread
-#pragma unroll
-        for (int m = 0; m < kMods; ++m)
-#pragma unroll
-          for (int h = 0; h < kMaxGroup; ++h) acc[m][h] *= alpha[h];
-      }
-      const int nvalid = min(kWindow, T - wi * kWindow);
-      const uint32_t starts = g.runs;
-      for (int t = 0; t < nvalid;) {
-        const int mod = min((int)mods[t], kMods - 1);  // the same for every thread
-        const uint32_t later = starts & ~((2u << t) - 1u);  // runs starting after token t
-        const int e = later ? min(nvalid, __ffs(later) - 1) : nvalid;
-        float a[kMaxGroup];
-#pragma unroll
-        for (int h = 0; h < kMaxGroup; ++h) a[h] = 0.0f;
-#pragma unroll
-        for (int m = 0; m < kMods; ++m)
-          if (m == mod) {
-#pragma unroll
-            for (int h = 0; h < kMaxGroup; ++h) a[h] = acc[m][h];
-          }
-#pragma unroll 4
-        for (int tt = t; tt < e; ++tt) {
-          const uint32_t code = (vw[(tt / vcpw) * kHeadDim + tid] >> (VB * (tt % vcpw))) & vmask;
-          const float d = g.dv[code];
-          const float4 pa = *reinterpret_cast<const float4*>(&g.pw[tt][0]);
-          const float4 pb = *reinterpret_cast<const float4*>(&g.pw[tt][4]);
-          a[0] = fmaf(pa.x, d, a[0]);
-          a[1] = fmaf(pa.y, d, a[1]);
-          a[2] = fmaf(pa.z, d, a[2]);
-          a[3] = fmaf(pa.w, d, a[3]);
-          a[4] = fmaf(pb.x, d, a[4]);
-          a[5] = fmaf(pb.y, d, a[5]);
-          a[6] = fmaf(pb.z, d, a[6]);
-          a[7] = fmaf(pb.w, d, a[7]);
-        }
-#pragma unroll
-        for (int m = 0; m < kMods; ++m)
-          if (m == mod) {
-#pragma unroll
-            for (int h = 0; h < kMaxGroup; ++h) acc[m][h] = a[h];
-          }
-        t = e;
-      }
-    }
-    __syncthreads();  // stage s and pw are free again
-    if (tid == 0 && i + kGenStages < nwin) {
-      fence_proxy_async_smem();
-      gen_issue(p, g, s, rec_base, lay.bytes, b, kvh, w0 + i + kGenStages, wait_win, wait_val);
-    }
-  }
-  if (failed_at >= 0) {
-    if (tid == 0) set_error(p.error_word, OMNIKV_DEVERR_TIMEOUT);
-    // the copies still in flight (windows failed_at, failed_at + 1) land before
-    // this CTA's shared memory is released
-    for (int j = failed_at; j < nwin && j < failed_at + kGenStages; ++j)
-      mbar_wait_bounded(&g.bar[j % kGenStages], (j / kGenStages) & 1, kWaitLimitNs);
-#pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h) {
-      m_run[h] = -INFINITY;
-      l_part[h] = 0.0f;
-#pragma unroll
-      for (int m = 0; m < kMods; ++m) acc[m][h] = 0.0f;
-    }
-  }
-
-  // ---- l per head: thread sums over the tokens it owns (sq == 0), CTA reduction
-  {
-#pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h) {
-      float v = l_part[h];
-      v += __shfl_xor_sync(0xffffffffu, v, 4);
-      v += __shfl_xor_sync(0xffffffffu, v, 8);
-      v += __shfl_xor_sync(0xffffffffu, v, 16);
-      l_part[h] = v;
-    }
-    __syncthreads();
-    if (lane == 0) {
-#pragma unroll
-      for (int h = 0; h < kMaxGroup; ++h) g.wmax[warp][h] = l_part[h];
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int h = 0; h < kMaxGroup; ++h) {
-    if (h >= G) continue;
-    Partial* out = p.partials + ((size_t)b * Hq + kvh * G + h) * p.num_splits + split;
-#pragma unroll
-    for (int m = 0; m < kMods; ++m) out->acc[m][tid] = acc[m][h];
-    if (tid == 0) {
-      out->m = m_run[h];
-      out->l = g.wmax[0][h] + g.wmax[1][h] + g.wmax[2][h] + g.wmax[3][h];
-    }
-  }
-}
-
-// The 2-bit build reaches the CUDA-core path only for a codebook that is not
-// symmetric: out of line there, so that the tensor-core path stays compact in
-// the instruction cache. The 4-bit build inlines its three instances.
-__device__ __noinline__ void decode_generic_asym(const DecodeParams& p, DecodeSmem& sm, int b, int kvh, int split) {
-  decode_generic_t<2, 2>(p, sm, b, kvh, split);
-}
-
-template <bool kGen>
-__device__ __forceinline__ void decode_generic(const DecodeParams& p, DecodeSmem& sm, int b, int kvh, int split) {
-  if (!kGen)
-    decode_generic_asym(p, sm, b, kvh, split);
-  else if (p.key_bits == 2)
-    decode_generic_t<2, 4>(p, sm, b, kvh, split);
-  else if (p.value_bits == 2)
-    decode_generic_t<4, 2>(p, sm, b, kvh, split);
-  else
-    decode_generic_t<4, 4>(p, sm, b, kvh, split);
-}
+static_assert(sizeof(GenSmem) <= sizeof(DecodeSmem::u), "CUDA-core path shared memory");
 
 // ---------------------------------------------------------------------------
 // tensor-core path (K2/V2, symmetric codebooks)
@@ -505,6 +143,41 @@ __device__ __forceinline__ void split_pair_t(float x0, float x1, uint32_t& hi, u
   const __half2 l = __floats2half2_rn(x0 - f.x, x1 - f.y);
   hi = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h));
   lo = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&l));
+}
+
+// The window's key metadata as fp16 (m_c, s_c) pairs, channel c at index c: the
+// record's own for fp16 metadata; for MXFP4 the warp converts its window's E2M1
+// values (exact in fp16 for block exponents in [-16, 12]; a scale beyond makes the
+// split non-finite, reported as OMNIKV_DEVERR_RANGE) into its buffer.
+__device__ __noinline__ void mx_window_pairs(const uint8_t* meta, uint32_t* out, int lane) {
+  __syncwarp();  // the previous window's readers are done
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int c = lane + 32 * k;
+    const float2 ms = mx_meta_channel(meta, c);
+    const __half2 h = __floats2half2_rn(ms.x, ms.y);
+    out[c] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  __syncwarp();
+}
+
+template <int kMeta>
+__device__ __forceinline__ const __half2* window_meta_pairs(DecodeSmem& sm, const uint8_t* rec, int warp, int lane) {
+  if (kMeta != kMetaMx) return reinterpret_cast<const __half2*>(rec + Rec22<kMeta>::meta);
+  mx_window_pairs(rec + Rec22<kMeta>::meta, sm.mxpairs[warp], lane);
+  return reinterpret_cast<const __half2*>(sm.mxpairs[warp]);
+}
+
+// The split's maximum and denominator of head h; a split whose partial is not
+// finite (inputs outside the fp16 range of the operands) is reported and written
+// empty, so the combine gives it weight 0 and never reads its accumulators.
+__device__ __forceinline__ void write_split_ml(const DecodeParams& p, const DecodeSmem& sm, int b, int kvh, int h,
+                                               int split, float m, float l) {
+  Partial* out = p.partials + ((size_t)b * p.num_kv_heads * p.group + kvh * p.group + h) * p.num_splits + split;
+  const bool bad = ((sm.bad_heads >> h) & 1u) || !isfinite(l) || isnan(m) || m == INFINITY;
+  if (bad) set_error(p.error_word, OMNIKV_DEVERR_RANGE);
+  out->m = bad ? -INFINITY : m;
+  out->l = bad ? 0.0f : l;
 }
 
 // Per-warp decode state. Only the accumulator of the active modality lives in
@@ -579,45 +252,58 @@ __device__ __forceinline__ void warp_windows(int w0, int w1, int warp, int& a, i
   e = min(a + per, w1);
 }
 
+template <int kMeta>
 __device__ __forceinline__ void issue_window(const DecodeParams& p, DecodeSmem& sm, int warp, int stage,
                                              const uint8_t* rec_base, int b, int kvh, int wi, int wait_win,
                                              int wait_val) {
-  if (wi == wait_win &&
-      !wait_flag(p.step_flags + (size_t)b * p.num_kv_heads + kvh, wait_val, kWaitLimitNs))
-    set_error(p.error_word, OMNIKV_DEVERR_TIMEOUT);
   uint64_t* bar = &sm.bar[warp][stage];
+  if (wi == wait_win &&
+      !wait_flag(p.step_flags + (size_t)b * p.num_kv_heads + kvh, wait_val, p.flag_wait_ns)) {
+    // the appended token's record never became ready: no copy of a stale record;
+    // the warp's split is written empty
+    set_error(p.error_word, OMNIKV_DEVERR_TIMEOUT);
+    sm.wabort[warp] = 1;
+    mbar_arrive_expect_tx(bar, 0);
+    return;
+  }
   uint8_t* dst = &sm.u.w.stage[warp][stage][0];
-  mbar_arrive_expect_tx(bar, kStageBytes);
-  bulk_copy_g2s(dst, rec_base + (size_t)wi * kRec22, kRec22, bar);
-  bulk_copy_g2s(dst + kRec22, p.modality + (size_t)b * p.cap_tokens + (size_t)wi * kWindow, kWindow, bar);
+  constexpr int rb = Rec22<kMeta>::bytes;
+  mbar_arrive_expect_tx(bar, rb + kWindow);
+  bulk_copy_g2s(dst, rec_base + (size_t)wi * rb, rb, bar);
+  bulk_copy_g2s(dst + rb, p.modality + (size_t)b * p.cap_tokens + (size_t)wi * kWindow, kWindow, bar);
 }
 
 // Each warp's first kStages windows: barrier set-up and bulk copies (lane 0).
+template <int kMeta>
 __device__ __forceinline__ void prime_pipeline(const DecodeParams& p, DecodeSmem& sm, int b, int kvh, int w0, int w1) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint8_t* rec_base = p.records + ((size_t)(b * p.num_kv_heads + kvh) * p.cap_windows) * kRec22;
+  const uint8_t* rec_base =
+      p.records + ((size_t)(b * p.num_kv_heads + kvh) * p.cap_windows) * Rec22<kMeta>::bytes;
   int wa, we, wait_win, wait_val;
   warp_windows(w0, w1, warp, wa, we);
   step_window(p, b, wait_win, wait_val);
   if (lane == 0) {
+    sm.wabort[warp] = 0;
 #pragma unroll
     for (int s = 0; s < kStages; ++s) mbar_init(&sm.bar[warp][s], 1);
     fence_barrier_init();
     for (int i = 0; i < kStages && wa + i < we; ++i)
-      issue_window(p, sm, warp, i, rec_base, b, kvh, wa + i, wait_win, wait_val);
+      issue_window<kMeta>(p, sm, warp, i, rec_base, b, kvh, wa + i, wait_win, wait_val);
   }
   __syncwarp();
 }
 
+template <int kMeta>
 __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh, int split, float kV0, float kV1,
-                           float vc0, uint32_t tbase) {
+                           float vc0, uint32_t tbase, float escale) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int G = p.group;
   const int Hq = p.num_kv_heads * G;
   int T, w0, w1;
   split_range(p, b, split, T, w0, w1);
-  const uint8_t* rec_base = p.records + ((size_t)(b * p.num_kv_heads + kvh) * p.cap_windows) * kRec22;
+  const uint8_t* rec_base =
+      p.records + ((size_t)(b * p.num_kv_heads + kvh) * p.cap_windows) * Rec22<kMeta>::bytes;
   int wa, we, wait_win, wait_val;
   warp_windows(w0, w1, warp, wa, we);
   step_window(p, b, wait_win, wait_val);
@@ -645,16 +331,18 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
   for (int i = 0; i < nmine; ++i) {
     const int s = i % kStages;
     const int wi = wa + i;
-    if (!mbar_wait_bounded(&sm.bar[warp][s], (i / kStages) & 1, kWaitLimitNs)) {
+    if (!mbar_wait_bounded(&sm.bar[warp][s], (i / kStages) & 1, kWaitLimitNs) ||
+        *reinterpret_cast<volatile int*>(&sm.wabort[warp]) != 0) {
       failed_at = i;
       break;
     }
     const uint8_t* stg = &sm.u.w.stage[warp][s][0];
     const uint32_t* kw = reinterpret_cast<const uint32_t*>(stg);
-    const __half2* meta = reinterpret_cast<const __half2*>(stg + 1024);
-    const uint32_t* vw = reinterpret_cast<const uint32_t*>(stg + 1536);
-    const __half* sig = reinterpret_cast<const __half*>(stg + 2560);
-    const uint8_t* mods = stg + kRec22;
+    using L = Rec22<kMeta>;
+    const __half2* meta = window_meta_pairs<kMeta>(sm, stg, warp, lane);
+    const uint32_t* vw = reinterpret_cast<const uint32_t*>(stg + L::v);
+    const __half* sig = reinterpret_cast<const __half*>(stg + L::sigma);
+    const uint8_t* mods = stg + L::bytes;
 
     // ---- per-window: fp16 scale pairs for the A operand, offset sum_c q'_c m_gc
     // lane (g, t) covers channels 32t .. 32t+31 (k-slot pairs (c, c+8))
@@ -739,10 +427,10 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int posA = wi * kWindow + tokA[h], posB = wi * kWindow + tokB[h];
-        sc[h][0] = posA < T ? d0[h][0] + d1[h][0] + off0 : -INFINITY;
-        sc[h][1] = posA < T ? d0[h][1] + d1[h][1] + off1 : -INFINITY;
-        sc[h][2] = posB < T ? d0[h][2] + d1[h][2] + off0 : -INFINITY;
-        sc[h][3] = posB < T ? d0[h][3] + d1[h][3] + off1 : -INFINITY;
+        sc[h][0] = posA < T ? fmaf(d0[h][0] + d1[h][0], escale, off0) : -INFINITY;
+        sc[h][1] = posA < T ? fmaf(d0[h][1] + d1[h][1], escale, off1) : -INFINITY;
+        sc[h][2] = posB < T ? fmaf(d0[h][2] + d1[h][2], escale, off0) : -INFINITY;
+        sc[h][3] = posB < T ? fmaf(d0[h][3] + d1[h][3], escale, off1) : -INFINITY;
       }
     }
 
@@ -849,7 +537,7 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
     __syncwarp();
     if (lane == 0 && i + kStages < nmine) {
       fence_proxy_async_smem();
-      issue_window(p, sm, warp, s, rec_base, b, kvh, wa + i + kStages, wait_win, wait_val);
+      issue_window<kMeta>(p, sm, warp, s, rec_base, b, kvh, wa + i + kStages, wait_win, wait_val);
     }
   }
 
@@ -934,6 +622,7 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
         if (hh >= G) continue;
         Partial* out = p.partials + ((size_t)b * Hq + kvh * G + hh) * p.num_splits + split;
         *reinterpret_cast<float2*>(&out->acc[m][16 * g + 2 * mt]) = make_float2(v[j], v[j + 2]);
+        if (!isfinite(v[j]) || !isfinite(v[j + 2])) atomicOr(&sm.bad_heads, 1u << hh);
       }
     }
     __syncthreads();
@@ -946,9 +635,7 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
       float l = 0.0f;
 #pragma unroll
       for (int w = 0; w < kWarps; ++w) l += sm.lw[w][hh];
-      Partial* out = p.partials + ((size_t)b * Hq + kvh * G + hh) * p.num_splits + split;
-      out->m = M[j];
-      out->l = l;
+      write_split_ml(p, sm, b, kvh, hh, split, M[j], l);
     }
   }
 }
@@ -1031,22 +718,35 @@ __device__ __forceinline__ void pv_scale(PvAcc& a, float f0, float f1) {
 // stage's mbarrier. In a decode step the window that receives the new token is
 // copied only after its flag shows the append (bounded wait); the records before
 // it go first. Thread 0.
+template <int kMeta>
 __device__ __forceinline__ void issue_group(const DecodeParams& p, DecodeSmem& sm, int stage, const uint8_t* rec_base,
                                             int b, int kvh, int wfirst, int nwin, int wait_win, int wait_val) {
   uint64_t* bar = &sm.cbar[stage];
   uint8_t* dst = &sm.u.c.stage[stage][0];
-  mbar_arrive_expect_tx(bar, (uint32_t)nwin * (kRec22 + kWindow));
   int nfree = nwin;  // records that need no wait
   if (wait_win >= wfirst && wait_win < wfirst + nwin) nfree = wait_win - wfirst;
-  if (nfree > 0) bulk_copy_g2s(dst, rec_base + (size_t)wfirst * kRec22, (uint32_t)nfree * kRec22, bar);
-  if (nfree < nwin) {
-    if (!wait_flag(p.step_flags + (size_t)b * p.num_kv_heads + kvh, wait_val, kWaitLimitNs))
-      set_error(p.error_word, OMNIKV_DEVERR_TIMEOUT);
-    bulk_copy_g2s(dst + nfree * kRec22, rec_base + (size_t)(wfirst + nfree) * kRec22, (uint32_t)(nwin - nfree) * kRec22,
-                  bar);
-  }
-  bulk_copy_g2s(dst + kCoop * kRec22, p.modality + (size_t)b * p.cap_tokens + (size_t)wfirst * kWindow,
+  // the records that need no wait and the modality ids are copied first; the
+  // phase cannot complete before the arrive below
+  constexpr int rb = Rec22<kMeta>::bytes;
+  mbar_expect_tx(bar, (uint32_t)nfree * rb + (uint32_t)nwin * kWindow);
+  if (nfree > 0) bulk_copy_g2s(dst, rec_base + (size_t)wfirst * rb, (uint32_t)nfree * rb, bar);
+  bulk_copy_g2s(dst + kCoop * rb, p.modality + (size_t)b * p.cap_tokens + (size_t)wfirst * kWindow,
                 (uint32_t)nwin * kWindow, bar);
+  if (nfree == nwin) {
+    mbar_arrive_expect_tx(bar, 0);
+    return;
+  }
+  if (!wait_flag(p.step_flags + (size_t)b * p.num_kv_heads + kvh, wait_val, p.flag_wait_ns)) {
+    // the appended token's record never became ready: no copy of a stale record;
+    // the split is written empty
+    set_error(p.error_word, OMNIKV_DEVERR_TIMEOUT);
+    sm.abort = 1;
+    mbar_arrive_expect_tx(bar, 0);
+    return;
+  }
+  mbar_arrive_expect_tx(bar, (uint32_t)(nwin - nfree) * rb);
+  bulk_copy_g2s(dst + nfree * rb, rec_base + (size_t)(wfirst + nfree) * rb, (uint32_t)(nwin - nfree) * rb,
+                bar);
 }
 
 // The tensor-core decode of one split. Windows are taken kCoop at a time (a
@@ -1054,25 +754,28 @@ __device__ __forceinline__ void issue_group(const DecodeParams& p, DecodeSmem& s
 // 16-token tiles), the CTA takes the common running max, warp w turns its
 // probabilities into the value-product B operand in shared memory, and then every
 // warp runs the value product of the whole group for its own 32 channels.
+template <int kMeta>
 __device__ void decode_coop(const DecodeParams& p, DecodeSmem& sm, int b, int kvh, int split, float kV0, float kV1,
-                            float vc0) {
+                            float vc0, float escale) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int G = p.group;
   const int Hq = p.num_kv_heads * G;
   int T, w0, w1;
   split_range(p, b, split, T, w0, w1);
-  const uint8_t* rec_base = p.records + ((size_t)(b * p.num_kv_heads + kvh) * p.cap_windows) * kRec22;
+  const uint8_t* rec_base =
+      p.records + ((size_t)(b * p.num_kv_heads + kvh) * p.cap_windows) * Rec22<kMeta>::bytes;
   int wait_win, wait_val;
   step_window(p, b, wait_win, wait_val);
   const int ngroups = (w1 - w0 + kCoop - 1) / kCoop;
   int issued = 0;  // groups whose copies were issued (meaningful in thread 0)
   if (threadIdx.x == 0) {
+    sm.abort = 0;
 #pragma unroll
     for (int s = 0; s < kCoopStages; ++s) mbar_init(&sm.cbar[s], 1);
     fence_barrier_init();
     for (; issued < kCoopStages && issued < ngroups; ++issued)
-      issue_group(p, sm, issued, rec_base, b, kvh, w0 + kCoop * issued, min(kCoop, w1 - w0 - kCoop * issued),
+      issue_group<kMeta>(p, sm, issued, rec_base, b, kvh, w0 + kCoop * issued, min(kCoop, w1 - w0 - kCoop * issued),
                   wait_win, wait_val);
   }
   __syncthreads();  // barrier initialisation (and the score operand) visible to every thread
@@ -1100,12 +803,14 @@ __device__ void decode_coop(const DecodeParams& p, DecodeSmem& sm, int b, int kv
     const int wi = w0 + kCoop * it + warp;  // this warp's window for the scores
     const bool have = wi < w1;              // warp-uniform
     const uint8_t* stg = &sm.u.c.stage[s][0];
-    const bool ok = mbar_wait_bounded(&sm.cbar[s], (it / kCoopStages) & 1, kWaitLimitNs);
+    const bool ok = mbar_wait_bounded(&sm.cbar[s], (it / kCoopStages) & 1, kWaitLimitNs) &&
+                    *reinterpret_cast<volatile int*>(&sm.abort) == 0;
     const bool wok = __all_sync(0xffffffffu, ok);
 
     // ---- scores of this warp's window (both tiles) -------------------------
-    const uint8_t* rec = stg + warp * kRec22;
-    const uint8_t* mods = stg + kCoop * kRec22 + warp * kWindow;
+    using L = Rec22<kMeta>;
+    const uint8_t* rec = stg + warp * L::bytes;
+    const uint8_t* mods = stg + kCoop * L::bytes + warp * kWindow;
     float sc[2][4];
     int tokA[2], tokB[2];
 #pragma unroll
@@ -1117,7 +822,7 @@ __device__ void decode_coop(const DecodeParams& p, DecodeSmem& sm, int b, int kv
     }
     if (have && wok) {
       const uint32_t* kw = reinterpret_cast<const uint32_t*>(rec);
-      const __half2* meta = reinterpret_cast<const __half2*>(rec + 1024);
+      const __half2* meta = window_meta_pairs<kMeta>(sm, rec, warp, lane);
       // fp16 scale pairs of the A operand and the offset sum_c q'_c m_gc; lane
       // (g, t) covers channels 32t .. 32t+31 (k-slot pairs (c, c+8))
       uint32_t sp[8][2];
@@ -1193,10 +898,10 @@ __device__ void decode_coop(const DecodeParams& p, DecodeSmem& sm, int b, int kv
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int posA = wi * kWindow + tokA[h], posB = wi * kWindow + tokB[h];
-        sc[h][0] = posA < T ? d0[h][0] + d1[h][0] + off0 : -INFINITY;
-        sc[h][1] = posA < T ? d0[h][1] + d1[h][1] + off1 : -INFINITY;
-        sc[h][2] = posB < T ? d0[h][2] + d1[h][2] + off0 : -INFINITY;
-        sc[h][3] = posB < T ? d0[h][3] + d1[h][3] + off1 : -INFINITY;
+        sc[h][0] = posA < T ? fmaf(d0[h][0] + d1[h][0], escale, off0) : -INFINITY;
+        sc[h][1] = posA < T ? fmaf(d0[h][1] + d1[h][1], escale, off1) : -INFINITY;
+        sc[h][2] = posB < T ? fmaf(d0[h][2] + d1[h][2], escale, off0) : -INFINITY;
+        sc[h][3] = posB < T ? fmaf(d0[h][3] + d1[h][3], escale, off1) : -INFINITY;
       }
     }
     {
@@ -1216,7 +921,7 @@ __device__ void decode_coop(const DecodeParams& p, DecodeSmem& sm, int b, int kv
     // every warp is past the value product of group it - 1: its stage may be refilled
     if (threadIdx.x == 0 && issued < ngroups && issued == it + kCoopStages - 1) {
       fence_proxy_async_smem();
-      issue_group(p, sm, issued % kCoopStages, rec_base, b, kvh, w0 + kCoop * issued,
+      issue_group<kMeta>(p, sm, issued % kCoopStages, rec_base, b, kvh, w0 + kCoop * issued,
                   min(kCoop, w1 - w0 - kCoop * issued), wait_win, wait_val);
       ++issued;
     }
@@ -1248,7 +953,7 @@ __device__ void decode_coop(const DecodeParams& p, DecodeSmem& sm, int b, int kv
 
     // ---- this warp's window: p, the sums, the value-product B operand --------
     if (have) {
-      const __half* sig = reinterpret_cast<const __half*>(rec + 2560);
+      const __half* sig = reinterpret_cast<const __half*>(rec + L::sigma);
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const float p0 = fast_exp2(fmaf(sc[h][0], kLog2e, -ms0));
@@ -1284,7 +989,7 @@ __device__ void decode_coop(const DecodeParams& p, DecodeSmem& sm, int b, int kv
     // ---- value product of the group for this warp's 32 channels -------------
 #pragma unroll 1
     for (int ww = 0; ww < kCoop; ++ww) {
-      const uint8_t* rv = stg + ww * kRec22 + 1536;
+      const uint8_t* rv = stg + ww * L::bytes + L::v;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const uint32_t tm = sm.tmask[ww][h];
@@ -1306,7 +1011,7 @@ __device__ void decode_coop(const DecodeParams& p, DecodeSmem& sm, int b, int kv
           pv_activate(pv, __ffs(tm) - 1);
           pv_tile(pv, a0, a1, f0, f1, 0xFFFFFFFFu, 0xFFFFFFFFu);
         } else {  // masked products, one per modality present, the active one first
-          const uint8_t* md = stg + kCoop * kRec22 + ww * kWindow + 16 * h;
+          const uint8_t* md = stg + kCoop * L::bytes + ww * kWindow + 16 * h;
           // k-slots of this lane's B registers: 2t, 2t+1 -> tokens t, t+8; 2t+8, 2t+9 -> t+4, t+12
           const int mk0 = min((int)md[t], kMods - 1), mk1 = min((int)md[t + 8], kMods - 1);
           const int mk2 = min((int)md[t + 4], kMods - 1), mk3 = min((int)md[t + 12], kMods - 1);
@@ -1380,18 +1085,23 @@ __device__ void decode_coop(const DecodeParams& p, DecodeSmem& sm, int b, int kv
     const int hh = 2 * t + j;
     if (hh >= G) continue;
     Partial* out = p.partials + ((size_t)b * Hq + kvh * G + hh) * p.num_splits + split;
+    bool fin = true;
 #pragma unroll
     for (int k = 0; k < kMods; ++k)
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt) {
         const float c0 = vc0 * Ssum[k][j];
-        *reinterpret_cast<float2*>(&out->acc[k][32 * warp + 4 * g + 2 * mt]) =
-            make_float2(pv.st[k][mt][j] + c0, pv.st[k][mt][j + 2] + c0);
+        const float2 v = make_float2(pv.st[k][mt][j] + c0, pv.st[k][mt][j + 2] + c0);
+        *reinterpret_cast<float2*>(&out->acc[k][32 * warp + 4 * g + 2 * mt]) = v;
+        fin = fin && isfinite(v.x) && isfinite(v.y);
       }
-    if (warp == 0 && g == 0) {
-      out->m = m_run[j];
-      out->l = Lsum[j];
-    }
+    if (!fin) atomicOr(&sm.bad_heads, 1u << hh);
+  }
+  __syncthreads();
+  if (warp == 0 && g == 0) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+      if (2 * t + j < G) write_split_ml(p, sm, b, kvh, 2 * t + j, split, m_run[j], Lsum[j]);
   }
 }
 
@@ -1421,8 +1131,9 @@ __device__ __forceinline__ void build_score_operand(DecodeSmem& sm, float k0scal
 // One decode CTA: split `split` of kv head kvh of sequence b. kBody: the 4-bit
 // build (CUDA-core path only, no TMEM, more CTAs per SM), or a tensor-core build
 // (per-warp or cooperative body), whose kernels fall back to the CUDA-core path for
-// 2-bit codebooks that are not symmetric.
-template <int kBody>
+// 2-bit codebooks that are not symmetric. kMeta: the key metadata format the
+// tensor-core builds are compiled for (the CUDA-core path reads it at run time).
+template <int kBody, int kMeta>
 __device__ __forceinline__ void decode_cta(const DecodeParams& p, DecodeSmem& sm, int b, int kvh, int split) {
   constexpr bool kGen = kBody == kBodyGeneric;
   // ---- independent of the cache (overlaps the previous launch of the stream):
@@ -1445,9 +1156,29 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, DecodeSmem& sm
          off += 128 * kThreads)
       asm volatile("prefetch.global.L2 [%0];" ::"l"(ub + off));
   }
-  rotate_queries(p, b, kvh, sm.q);
+  rotate_queries(p, b, kvh, &sm.q[0][0]);
+  if (threadIdx.x == 0) sm.bad_heads = 0u;
+  // the score operand carries a power of two 2^-E that keeps its largest entry at
+  // most 2^14 (so large queries stay inside the fp16 range); scores are scaled back
+  // by 2^E in fp32
+  {
+    float qm = 0.0f;
+    for (int i = threadIdx.x; i < kMaxGroup * kHeadDim; i += kThreads) qm = fmaxf(qm, fabsf((&sm.q[0][0])[i]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) qm = fmaxf(qm, __shfl_xor_sync(0xffffffffu, qm, o));
+    if ((threadIdx.x & 31) == 0) sm.lw[threadIdx.x >> 5][0] = qm;
+  }
   __syncthreads();
-  if (fast) build_score_operand(sm, (k1 - k0) * 128.0f, (k2 - k0) * 0.5f);
+  float escale = 1.0f;
+  if (fast) {
+    const float c0k = (k1 - k0) * 128.0f, c1k = (k2 - k0) * 0.5f;
+    const float xmax = fmaxf(fmaxf(sm.lw[0][0], sm.lw[1][0]), fmaxf(sm.lw[2][0], sm.lw[3][0])) *
+                       fmaxf(fabsf(c0k), fabsf(c1k));
+    int E = 0;
+    if (xmax > 0.0f && isfinite(xmax)) E = max(-24, min(100, (int)ceilf(log2f(xmax / 16384.0f))));
+    escale = ldexpf(1.0f, E);
+    build_score_operand(sm, c0k * ldexpf(1.0f, -E), c1k * ldexpf(1.0f, -E));
+  }
 
   // ---- the cache: lengths and records may come from the previous launch
   griddep_wait();
@@ -1462,24 +1193,24 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, DecodeSmem& sm
     return;
   }
   if (kBody == kBodyCoop && fast) {
-    decode_coop(p, sm, b, kvh, split, (v1 - v0) * 128.0f, (v2 - v0) * 0.5f, v0);
+    decode_coop<kMeta>(p, sm, b, kvh, split, (v1 - v0) * 128.0f, (v2 - v0) * 0.5f, v0, escale);
     return;
   }
   if (kBody == kBodyWarp && fast) {
-    prime_pipeline(p, sm, b, kvh, w0, w1);
+    prime_pipeline<kMeta>(p, sm, b, kvh, w0, w1);
     if (threadIdx.x < 32) tmem_alloc(&sm.tmem_base, kTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = sm.tmem_base;
-    decode_mma(p, sm, b, kvh, split, (v1 - v0) * 128.0f, (v2 - v0) * 0.5f, v0, tbase);
+    decode_mma<kMeta>(p, sm, b, kvh, split, (v1 - v0) * 128.0f, (v2 - v0) * 0.5f, v0, tbase, escale);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (threadIdx.x < 32) tmem_dealloc(tbase, kTmemCols);
     return;
   }
-  decode_generic<kGen>(p, sm, b, kvh, split);
+  decode_generic<kGen, SyncCta>(p, *reinterpret_cast<GenSmem*>(&sm.u), &sm.q[0][0], b, kvh, split);
 }
 
 // Registers for this many resident CTAs per SM: per-warp body 2 (its accumulators
@@ -1488,18 +1219,18 @@ __host__ __device__ constexpr int body_ctas_per_sm(int body) {
   return body == kBodyWarp ? 2 : body == kBodyCoop ? 3 : 4;
 }
 
-template <int kBody>
+template <int kBody, int kMeta>
 __global__ void __launch_bounds__(kThreads, body_ctas_per_sm(kBody)) decode_split_k_kernel(const DecodeParams p) {
   __shared__ DecodeSmem sm;
   griddep_launch_dependents();
-  decode_cta<kBody>(p, sm, blockIdx.z, blockIdx.y, blockIdx.x);
+  decode_cta<kBody, kMeta>(p, sm, blockIdx.z, blockIdx.y, blockIdx.x);
 }
 
 // Decode step: CTAs [0, batch * H) append one token to (sequence, kv head) and
 // then publish the new length in the step flag; the others are decode CTAs
 // (split fastest, then kv head, then sequence). Only the copy of the window that
 // receives the token waits for the flag.
-template <int kBody>
+template <int kBody, int kMeta>
 __global__ void __launch_bounds__(kThreads, body_ctas_per_sm(kBody))
     decode_step_kernel(const DecodeParams p, const WriteParams w) {
   __shared__ DecodeSmem sm;
@@ -1529,7 +1260,7 @@ __global__ void __launch_bounds__(kThreads, body_ctas_per_sm(kBody))
     return;
   }
   const int r = blockIdx.x - nappend;
-  decode_cta<kBody>(p, sm, r / (p.num_splits * H), (r / p.num_splits) % H, r % p.num_splits);
+  decode_cta<kBody, kMeta>(p, sm, r / (p.num_splits * H), (r / p.num_splits) % H, r % p.num_splits);
 }
 
 // Several decode CTAs share an SM only if the SM's unified L1 / shared memory is
@@ -1547,29 +1278,42 @@ cudaError_t prefer_shared_carveout(Kernel kernel, std::atomic<uint64_t>& done) {
   return e;
 }
 
-std::atomic<uint64_t> g_carveout[2][kNumBodies];  // [decode, step][body]
+std::atomic<uint64_t> g_carveout[2][kNumBodies][2];  // [decode, step][body][key metadata format]
 
-template <int kBody>
+template <int kBody, int kMeta>
 cudaError_t prepare_body() {
-  const cudaError_t e = prefer_shared_carveout(decode_split_k_kernel<kBody>, g_carveout[0][kBody]);
+  const cudaError_t e = prefer_shared_carveout(decode_split_k_kernel<kBody, kMeta>, g_carveout[0][kBody][kMeta]);
   if (e != cudaSuccess) return e;
-  return prefer_shared_carveout(decode_step_kernel<kBody>, g_carveout[1][kBody]);
+  return prefer_shared_carveout(decode_step_kernel<kBody, kMeta>, g_carveout[1][kBody][kMeta]);
 }
 
-cudaError_t prepare_kernels(int body) {
-  return body == kBodyWarp ? prepare_body<kBodyWarp>()
-       : body == kBodyCoop ? prepare_body<kBodyCoop>()
-                           : prepare_body<kBodyGeneric>();
+// The 4-bit build reads the metadata format at run time: one instance.
+cudaError_t prepare_kernels(int body, int meta) {
+  if (body == kBodyGeneric) return prepare_body<kBodyGeneric, kMetaFp16>();
+  if (meta == kMetaMx) return body == kBodyWarp ? prepare_body<kBodyWarp, kMetaMx>() : prepare_body<kBodyCoop, kMetaMx>();
+  return body == kBodyWarp ? prepare_body<kBodyWarp, kMetaFp16>() : prepare_body<kBodyCoop, kMetaFp16>();
 }
 
-template <int kBody>
-cudaError_t body_attributes(cudaFuncAttributes* a) {
-  cudaError_t e = cudaFuncGetAttributes(a, decode_step_kernel<kBody>);
+template <int kBody, int kMeta>
+cudaError_t body_attributes_of(cudaFuncAttributes* a) {
+  cudaError_t e = cudaFuncGetAttributes(a, decode_step_kernel<kBody, kMeta>);
   if (e != cudaSuccess) return e;
   cudaFuncAttributes a2;
-  e = cudaFuncGetAttributes(&a2, decode_split_k_kernel<kBody>);
+  e = cudaFuncGetAttributes(&a2, decode_split_k_kernel<kBody, kMeta>);
   if (e != cudaSuccess) return e;
   // size both kernels of the body by the larger register count
+  if (a2.numRegs > a->numRegs) a->numRegs = a2.numRegs;
+  if (a2.sharedSizeBytes > a->sharedSizeBytes) a->sharedSizeBytes = a2.sharedSizeBytes;
+  return cudaSuccess;
+}
+
+// Attributes of a body, over both metadata formats (the residency of the larger).
+template <int kBody>
+cudaError_t body_attributes(cudaFuncAttributes* a) {
+  cudaError_t e = body_attributes_of<kBody, kMetaFp16>(a);
+  if (e != cudaSuccess || kBody == kBodyGeneric) return e;
+  cudaFuncAttributes a2;
+  if ((e = body_attributes_of<kBody, kMetaMx>(&a2)) != cudaSuccess) return e;
   if (a2.numRegs > a->numRegs) a->numRegs = a2.numRegs;
   if (a2.sharedSizeBytes > a->sharedSizeBytes) a->sharedSizeBytes = a2.sharedSizeBytes;
   return cudaSuccess;
@@ -1601,7 +1345,8 @@ int decode_ctas_per_sm(int body) {
   const cudaError_t ea = body == kBodyWarp ? body_attributes<kBodyWarp>(&a)
                        : body == kBodyCoop ? body_attributes<kBodyCoop>(&a)
                                            : body_attributes<kBodyGeneric>(&a);
-  if (prepare_kernels(body) != cudaSuccess || ea != cudaSuccess ||
+  if (prepare_kernels(body, kMetaFp16) != cudaSuccess || (body != kBodyGeneric && prepare_kernels(body, kMetaMx) != cudaSuccess) ||
+      ea != cudaSuccess ||
       cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&smem_rsv, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess)
@@ -1617,22 +1362,32 @@ int decode_ctas_per_sm(int body) {
 
 cudaError_t launch_decode_step(const DecodeParams& p, const WriteParams& w, cudaStream_t stream) {
   const int body = decode_body(p.key_bits, p.value_bits, p.split_windows);
-  const cudaError_t e = prepare_kernels(body);
+  const int meta = p.key_meta;
+  const cudaError_t e = prepare_kernels(body, meta);
   if (e != cudaSuccess) return e;
   const dim3 grid(p.batch * p.num_kv_heads * (1 + p.num_splits));
-  return body == kBodyWarp ? launch_pdl(decode_step_kernel<kBodyWarp>, grid, dim3(kThreads), 0, stream, p, w)
-       : body == kBodyCoop ? launch_pdl(decode_step_kernel<kBodyCoop>, grid, dim3(kThreads), 0, stream, p, w)
-                           : launch_pdl(decode_step_kernel<kBodyGeneric>, grid, dim3(kThreads), 0, stream, p, w);
+  const dim3 block(kThreads);
+  if (body == kBodyGeneric) return launch_pdl(decode_step_kernel<kBodyGeneric, kMetaFp16>, grid, block, 0, stream, p, w);
+  if (meta == kMetaMx)
+    return body == kBodyWarp ? launch_pdl(decode_step_kernel<kBodyWarp, kMetaMx>, grid, block, 0, stream, p, w)
+                             : launch_pdl(decode_step_kernel<kBodyCoop, kMetaMx>, grid, block, 0, stream, p, w);
+  return body == kBodyWarp ? launch_pdl(decode_step_kernel<kBodyWarp, kMetaFp16>, grid, block, 0, stream, p, w)
+                           : launch_pdl(decode_step_kernel<kBodyCoop, kMetaFp16>, grid, block, 0, stream, p, w);
 }
 
 cudaError_t launch_decode(const DecodeParams& p, int batch, cudaStream_t stream) {
   const int body = decode_body(p.key_bits, p.value_bits, p.split_windows);
-  const cudaError_t e = prepare_kernels(body);
+  const int meta = p.key_meta;
+  const cudaError_t e = prepare_kernels(body, meta);
   if (e != cudaSuccess) return e;
   const dim3 grid(p.num_splits, p.num_kv_heads, batch);
-  return body == kBodyWarp ? launch_pdl(decode_split_k_kernel<kBodyWarp>, grid, dim3(kThreads), 0, stream, p)
-       : body == kBodyCoop ? launch_pdl(decode_split_k_kernel<kBodyCoop>, grid, dim3(kThreads), 0, stream, p)
-                           : launch_pdl(decode_split_k_kernel<kBodyGeneric>, grid, dim3(kThreads), 0, stream, p);
+  const dim3 block(kThreads);
+  if (body == kBodyGeneric) return launch_pdl(decode_split_k_kernel<kBodyGeneric, kMetaFp16>, grid, block, 0, stream, p);
+  if (meta == kMetaMx)
+    return body == kBodyWarp ? launch_pdl(decode_split_k_kernel<kBodyWarp, kMetaMx>, grid, block, 0, stream, p)
+                             : launch_pdl(decode_split_k_kernel<kBodyCoop, kMetaMx>, grid, block, 0, stream, p);
+  return body == kBodyWarp ? launch_pdl(decode_split_k_kernel<kBodyWarp, kMetaFp16>, grid, block, 0, stream, p)
+                           : launch_pdl(decode_split_k_kernel<kBodyCoop, kMetaFp16>, grid, block, 0, stream, p);
 }
 
 }  // namespace omnikv

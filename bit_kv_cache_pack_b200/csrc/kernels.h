@@ -16,6 +16,7 @@ struct WriteParams {
   const float* key_signs;
   const float* value_rot;
   int key_bits, value_bits, num_kv_heads;
+  int key_meta;  // kMetaFp16 or kMetaMx
   uint8_t* records;
   __half* key_tail;
   uint8_t* modality;
@@ -28,7 +29,10 @@ struct WriteParams {
   int n_new;
   int tc_values;  // 1: values of windows filled completely by this write are done by vrot_tc
   int32_t* step_flags;  // decode step only: [batch][kv heads], set to the new length once written
+  float* vrot_dump;     // optional: [batch][kv heads][n_new][128] fp32 rotated values v' of the written tokens
 };
+
+constexpr uint64_t kFlagWaitNs = 2000000000ull;  // default limit of a decode step's flag wait (2 s)
 
 struct DecodeParams {
   const float* key_cb;
@@ -36,6 +40,7 @@ struct DecodeParams {
   const float* key_signs;
   const float* value_rot;  // only prefetched into L2 (for the combine)
   int key_bits, value_bits, num_kv_heads, group;
+  int key_meta;  // kMetaFp16 or kMetaMx
   const uint8_t* records;
   const uint8_t* modality;
   const int32_t* seq_lens;
@@ -50,6 +55,7 @@ struct DecodeParams {
   // holding the appended position is read once step_flags[b][h] == that length
   int len_add;
   const int32_t* step_flags;
+  uint64_t flag_wait_ns;  // how long a copy waits for its step flag before giving up (OMNIKV_DEVERR_TIMEOUT)
 };
 
 struct CombineParams {

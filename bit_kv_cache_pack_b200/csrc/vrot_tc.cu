@@ -198,7 +198,8 @@ __device__ __forceinline__ void convert_basis(VrotSmem& sm, int slot, const floa
 // token's codes code = #{j : v' / sigma > t_j} (0 where sigma == 0) for the
 // tokens of modality m.
 template <int BITS>
-__device__ __forceinline__ void epilogue_codes(VrotSmem& sm, uint32_t tmem, int warp, int lane, int ntok, int m) {
+__device__ __forceinline__ void epilogue_codes(VrotSmem& sm, uint32_t tmem, int warp, int lane, int ntok, int m,
+                                               float* dump) {
   const CodeBounds<(1 << BITS) - 1> bv = load_bounds<(1 << BITS) - 1>(sm.bv);
   const int r = 32 * (warp & 3) + lane, cb = warp >> 2;
   const bool mine = r < ntok && sm.mods[r] == m;
@@ -211,6 +212,13 @@ __device__ __forceinline__ void epilogue_codes(VrotSmem& sm, uint32_t tmem, int 
     for (int c = 0; c < 32; ++c) {
       const uint32_t code = code_from_scaled(sb, __uint_as_float(v[c]));
       sm.codes[32 * cb + c][r] = (uint8_t)(sg != 0.0f ? code : 0u);
+    }
+    if (dump) {  // test hook: this token's v' for channels 32 cb .. 32 cb + 31
+      float4* d = reinterpret_cast<float4*>(dump + 32 * cb);
+#pragma unroll
+      for (int c4 = 0; c4 < 8; ++c4)
+        d[c4] = make_float4(__uint_as_float(v[4 * c4]), __uint_as_float(v[4 * c4 + 1]), __uint_as_float(v[4 * c4 + 2]),
+                            __uint_as_float(v[4 * c4 + 3]));
     }
   }
 }
@@ -228,7 +236,7 @@ __global__ void __launch_bounds__(kVThreads, 1) vrot_tc_kernel(const WriteParams
   const int i0 = blockIdx.x * per, i1 = min(i0 + per, n_items);
   if (i0 >= i1) return;
   const int LV = 1 << p.value_bits;
-  const RecordLayout lay(p.key_bits, p.value_bits);
+  const RecordLayout lay(p.key_bits, p.value_bits, p.key_meta);
 
   if (tid < LV - 1) sm.bv[tid] = make_code_bound(__fmul_rn(__fadd_rn(p.val_cb[tid], p.val_cb[tid + 1]), 0.5f), 0.0f);
   if (warp == 0) tmem_alloc(&sm.tmem_base, kTmemCols);
@@ -343,10 +351,15 @@ __global__ void __launch_bounds__(kVThreads, 1) vrot_tc_kernel(const WriteParams
           break;
         }
         // ---- epilogue: this thread's token (TMEM lane 32 warp + lane)
+        float* dump = nullptr;  // test hook: where this thread's token's v' goes
+        if (p.vrot_dump) {
+          const int tok = cur.wt0 * kWindow + 32 * (warp & 3) + lane - cur.L0;
+          dump = p.vrot_dump + (((size_t)cur.b * p.num_kv_heads + cur.h) * p.n_new + tok) * kHeadDim;
+        }
         if (p.value_bits == 2)
-          epilogue_codes<2>(sm, tmem, warp, lane, ntok, m);
+          epilogue_codes<2>(sm, tmem, warp, lane, ntok, m, dump);
         else
-          epilogue_codes<4>(sm, tmem, warp, lane, ntok, m);
+          epilogue_codes<4>(sm, tmem, warp, lane, ntok, m, dump);
         tc_fence_before();
         __syncthreads();  // the accumulator is reused by the next pass (and B may be replaced)
         todo &= ~(1 << m);

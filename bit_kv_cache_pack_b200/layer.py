@@ -18,7 +18,7 @@ WINDOW = 32
 
 class LayerConstants:
     def __init__(self, key_codebook, value_codebook, key_signs, value_rot, num_q_heads: int,
-                 device="cuda"):
+                 device="cuda", key_meta_format: int = _abi.OMNIKV_META_FP16):
         dev = torch.device(device)
         f32 = dict(dtype=torch.float32, device=dev)
         self.key_codebook = torch.as_tensor(key_codebook, **f32).contiguous()
@@ -29,19 +29,20 @@ class LayerConstants:
         self.num_q_heads = int(num_q_heads)
         self.key_bits = int(self.key_codebook.numel()).bit_length() - 1
         self.value_bits = int(self.value_codebook.numel()).bit_length() - 1
+        self.key_meta_format = int(key_meta_format)
         self.struct = OmniKVConfig(
             HEAD_DIM, self.num_q_heads, self.num_kv_heads, WINDOW, self.key_bits, self.value_bits,
             self.key_codebook.data_ptr(), self.value_codebook.data_ptr(), self.key_signs.data_ptr(),
-            self.value_rot.data_ptr())
+            self.value_rot.data_ptr(), self.key_meta_format)
 
 
 class KVCache:
     def __init__(self, batch: int, num_kv_heads: int, cap_tokens: int, key_bits: int = 2,
-                 value_bits: int = 2, device="cuda"):
+                 value_bits: int = 2, device="cuda", key_meta_format: int = _abi.OMNIKV_META_FP16):
         dev = torch.device(device)
         if cap_tokens % WINDOW:
             raise ValueError("cap_tokens must be a multiple of 32")
-        self.record_bytes = _abi.omnikv_record_bytes(key_bits, value_bits)
+        self.record_bytes = _abi.omnikv_record_bytes_meta(key_bits, value_bits, key_meta_format)
         self.batch, self.num_kv_heads, self.cap_tokens = batch, num_kv_heads, cap_tokens
         self.key_bits, self.value_bits = key_bits, value_bits
         self.records = torch.zeros(batch, num_kv_heads, cap_tokens // WINDOW, self.record_bytes,

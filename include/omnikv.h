@@ -37,11 +37,19 @@
  * little-endian; bits = key_bits or value_bits; cpw = 32 / bits codes per u32):
  *   K codes [32 tokens][128 / cpw] u32  token-major: channel c of token t is
  *           in word (t, c / cpw) at bits [bits * (c % cpw), +bits)
- *   meta    [128] { fp16 m_gc, fp16 s_gc }
+ *   meta    key metadata of the window, in the config's key_meta_format:
+ *           OMNIKV_META_FP16 (512 B): [128] { fp16 m_gc, fp16 s_gc };
+ *           OMNIKV_META_MXFP4 (144 B; the pages' default metadata, section 3.1):
+ *           E2M1 codes (sign << 3 | magnitude index, magnitudes 0, 0.5, 1, 1.5,
+ *           2, 3, 4, 6) of the 128 minima, two per byte (even channel in the low
+ *           nibble), then of the 128 scales; then the E8M0 exponents (e + 127) of
+ *           the 4 blocks of 32 channels of the minima, then of the scales; 8 zero
+ *           bytes. m_gc = E2M1(m code) 2^e_m, s_gc = E2M1(s code) 2^e_s.
  *   V codes [32 / cpw][128] u32         channel-major: token t, channel c is in
  *           word (t / cpw, c) at bits [bits * (t % cpw), +bits)
  *   sigma   [32] fp16 (per-token value scale)
- * Size: 2624 bytes for K2/V2, 4672 bytes for K4/V4 (omnikv_record_bytes).
+ * Size (omnikv_record_bytes_meta): 2624 bytes for K2/V2 and 4672 for K4/V4 with
+ * fp16 metadata; 2256 and 4304 with MXFP4 metadata.
  * Dequantised rotated-space cache: k'_tc = m_gc + s_gc (c_j - c_0) for key code
  * j; v'_tc = sigma_t c_j for value code j. Padded slots of a partial window hold
  * code 0 and sigma 0.
@@ -62,10 +70,12 @@ extern "C" {
 #define OMNIKV_API
 #endif
 
-#define OMNIKV_ABI_VERSION 2
+#define OMNIKV_ABI_VERSION 3
 #define OMNIKV_HEAD_DIM 128
 #define OMNIKV_WINDOW 32
 #define OMNIKV_NUM_MODALITIES 3 /* 0 = text (L), 1 = audio (A), 2 = video (V) */
+#define OMNIKV_META_FP16 0      /* key window metadata: fp16 minimum and scale per channel */
+#define OMNIKV_META_MXFP4 1     /* key window metadata: MXFP4 (E2M1 values, one E8M0 exponent per 32 channels) */
 
 typedef enum {
   OMNIKV_OK = 0,
@@ -83,6 +93,11 @@ typedef enum {
                                       num_splits * ceil(ceil(max_seq_len / 32) / num_splits) were skipped */
 #define OMNIKV_DEVERR_TIMEOUT 0x4  /* a staged copy did not complete within its wait limit; outputs of that
                                       CTA are zero (never expected; the kernel returns instead of hanging) */
+#define OMNIKV_DEVERR_RANGE 0x10   /* a decode split produced a non-finite partial and was written empty
+                                      (weight 0 in the combine): inputs outside the range of the fp16
+                                      tensor-core operands of 2-bit decoding -- key window scales s_gc
+                                      above 32752, value scales sigma of 565 or more -- or non-finite
+                                      queries or cache entries. Queries of any finite size are supported. */
 
 /* Per-layer constants. All pointers are device pointers. */
 typedef struct {
@@ -97,6 +112,13 @@ typedef struct {
   const float* key_signs;       /* [128] fp32, each +1 or -1 (sign flip before the Hadamard transform) */
   const float* value_rot;       /* [num_kv_heads][3][128][128] fp32: U_m row-major, its COLUMNS are the
                                    basis: v' = U_m^T v, v = U_m v'. Must be orthogonal. */
+  int32_t key_meta_format;      /* OMNIKV_META_FP16 (0) or OMNIKV_META_MXFP4 (1): how a window's key minima and
+                                   scales are stored (section 3.1 "Implementation details": MXFP4 by default;
+                                   section 3.3: fp16). With MXFP4, per block of 32 channels the shared exponent
+                                   is the smallest e in [-127, 127] with max |x| <= 6 2^e (-127 for a zero
+                                   block); the minimum rounds to the nearest E2M1 value times 2^e (ties to the
+                                   even code), then the scale it needs, fp32((max - m^) / (c_last - c_0)) (0 if
+                                   negative), on its block's grid the same way. Codes as with fp16 metadata. */
 } omnikv_config;
 
 /* One layer's cache for a batch. Device memory is owned by the caller and must be
@@ -117,8 +139,14 @@ typedef struct {
                            the appended token's window record is written; may be NULL otherwise */
 } omnikv_cache;
 
-/* Bytes of one window record: 2624 for K2/V2, 4672 for K4/V4; 0 for unsupported bits. */
+/* Bytes of one window record with fp16 key metadata: 2624 for K2/V2, 4672 for K4/V4; 0 for
+ * unsupported bits. */
 OMNIKV_API size_t omnikv_record_bytes(int32_t key_bits, int32_t value_bits);
+
+/* Bytes of one window record in a key metadata format (OMNIKV_META_FP16: as omnikv_record_bytes;
+ * OMNIKV_META_MXFP4: 2256 for K2/V2, 4304 for K4/V4); 0 for unsupported arguments. The cache's
+ * records array holds [batch][num_kv_heads][cap_tokens / 32] records of this size. */
+OMNIKV_API size_t omnikv_record_bytes_meta(int32_t key_bits, int32_t value_bits, int32_t key_meta_format);
 
 /* Bytes of the split-K partials buffer for omnikv_decode_attention / omnikv_combine:
  * [batch][num_q_heads][num_splits] entries of { fp32 acc[3][128], fp32 m, fp32 l, 2 x fp32 padding }
@@ -153,6 +181,17 @@ OMNIKV_API int32_t omnikv_default_splits(const omnikv_config* cfg, const omnikv_
 OMNIKV_API omnikv_status omnikv_write_cache(const omnikv_config* cfg, omnikv_cache* cache,
                                  const void* k_new, const void* v_new, const uint8_t* modality_new,
                                  int32_t n_new, void* stream);
+
+/* omnikv_write_cache that also returns the rotated values v' = U_m^T v the kernels computed for the
+ * written tokens (section 2.3 "Modality-aware value rotation"; the value codes are decided from exactly
+ * these fp32 numbers), so a caller can check the value codes against v' / sigma bit for bit and v' against
+ * an exact rotation. Arguments as omnikv_write_cache, plus
+ *   v_rot : [batch][num_kv_heads][n_new][128] fp32, 16-byte aligned; every entry is written.
+ * Slower than omnikv_write_cache (an extra 512 B written per token and kv head); meant for tests. */
+OMNIKV_API omnikv_status omnikv_write_cache_rotations(const omnikv_config* cfg, omnikv_cache* cache,
+                                                      const void* k_new, const void* v_new,
+                                                      const uint8_t* modality_new, int32_t n_new, float* v_rot,
+                                                      void* stream);
 
 /* Fused split-K decode attention over the packed cache (decode_split_k). For every sequence b,
  * query head i (kv head i / G) and split s, over the windows [s C, min((s+1) C, W)) of the
