@@ -44,19 +44,17 @@ WORKLOADS_KEYS = ("tiny", "omni3b-b1", "omni3b-b16", "omni30b-b8", "ragged-b64")
 
 METRIC = "2-bit decode attention tokens/s and achieved HBM GB/s vs ~8 TB/s (1 B200)"
 UNIT = "tokens/s"
-BYTES_PER_TOKEN_HEAD = {(2, 2): 82, (4, 4): 146}   # algorithmic packed bytes per token per kv head
+# algorithmic packed bytes per token per kv head: (key bits, value bits, key metadata format)
+BYTES_PER_TOKEN_HEAD = {(2, 2, "fp16"): 82, (4, 4, "fp16"): 146, (2, 2, "mx"): 70.5, (4, 4, "mx"): 134.5}
+META_FORMATS = {"fp16": 0, "mx": 1}   # omnikv_config.key_meta_format
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the
-# timed kernel on the default workload, from an ncu capture of this benchmark
-# (its summary is kept with the other profiles), valid for the kernel sources
-# with this SHA-256; any change to them makes the field null until the next
-# capture.
-TRAFFIC_CAPTURES = {
-    "qwen2.5-omni-3b-36L-b1-ctx10240": {
-        "sources_sha256": "71ad72e9edf4bc86edda2a2bba852d6d1b21129c1b76a859aceb750e9a300447",
-        "bytes_per_launch": 2198016},
-}
-KERNEL_SOURCES = ("decode_split_k.cu", "append.cuh", "common.cuh", "ptx.cuh", "kernels.h")
+# timed kernel, per (workload, key metadata format), from an ncu capture of this
+# benchmark (its summary is kept with the other profiles), valid for the kernel
+# sources with this SHA-256; any change to them makes the field null until the
+# next capture.
+TRAFFIC_CAPTURES = {}
+KERNEL_SOURCES = ("decode_split_k.cu", "decode_common.cuh", "append.cuh", "common.cuh", "ptx.cuh", "kernels.h")
 
 
 def kernel_sources_sha256():
@@ -69,8 +67,8 @@ def kernel_sources_sha256():
     return h.hexdigest()
 
 
-def captured_traffic(workload_name):
-    cap = TRAFFIC_CAPTURES.get(workload_name)
+def captured_traffic(workload_name, meta="fp16"):
+    cap = TRAFFIC_CAPTURES.get((workload_name, meta))
     if cap is None:
         return None
     return cap["bytes_per_launch"] if kernel_sources_sha256() == cap["sources_sha256"] else None
@@ -91,6 +89,8 @@ def parse_args():
                     help="time one layer's decode (+ combine) or prefill cache write on --workload instead of "
                          "the decode step; prints one JSON line per split count")
     ap.add_argument("--bits", type=int, default=0, help="with --layer: 2 or 4 (default: the workload's)")
+    ap.add_argument("--meta", default="fp16", choices=sorted(META_FORMATS),
+                    help="key metadata format: fp16 (m, s) pairs or mx (MXFP4, the pages' default)")
     ap.add_argument("--batch", type=int, default=0, help="with --layer: override the workload's batch")
     ap.add_argument("--splits", default="0", help="with --layer decode: comma-separated split counts (0: default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -110,7 +110,7 @@ def rank_seed(workload: str, rank: int) -> int:
     return WORKLOADS_KEYS.index(workload) + 1000 * rank
 
 
-def workload_config(spec, world):
+def workload_config(spec, world, meta="fp16"):
     """The `config` object of both arms' JSON lines: the workload and how it is
     measured (the same dict for the GPU arm and the oracle arm)."""
     from synth.workloads import seq_lengths
@@ -119,6 +119,7 @@ def workload_config(spec, world):
             "context": int(L.max()) if not spec.ragged else "%d..%d" % spec.ragged,
             "num_q_heads": spec.num_q_heads, "num_kv_heads": spec.num_kv_heads, "head_dim": 128,
             "key_bits": spec.key_bits, "value_bits": spec.value_bits, "window": 32,
+            "key_meta_format": "mxfp4" if meta == "mx" else "fp16",
             "parallelism": "dp%d (independent sequences per rank)" % world,
             "l2": "GPU arm: flushed between timed steps (512 MiB write)"}
 
@@ -207,11 +208,11 @@ class ClockSampler:
 class Workload:
     """Per-layer constants and caches, prefilled (untimed), plus every step's inputs."""
 
-    def __init__(self, spec, seed, device, total_steps):
+    def __init__(self, spec, seed, device, total_steps, meta="fp16"):
         import bit_kv_cache_pack_b200 as m
         from synth.workloads import (codebook, decode_inputs, key_drift, layer_params, prefill_inputs,
                                      seq_lengths)
-        self.m, self.spec, self.dev = m, spec, device
+        self.m, self.spec, self.dev, self.meta = m, spec, device, meta
         self.lengths = seq_lengths(spec, seed)
         self.cap = int(-(-(int(self.lengths.max()) + total_steps) // 32) * 32)
         kb, vb = codebook(spec.key_bits), codebook(spec.value_bits)
@@ -219,8 +220,10 @@ class Workload:
         qs, ks, vs, ms = [], [], [], []
         for layer in range(spec.layers):
             params = layer_params(spec, seed, layer)
-            c = m.LayerConstants(kb, vb, params["key_signs"], params["value_rot"], spec.num_q_heads, device)
-            cache = m.KVCache(spec.batch, spec.num_kv_heads, self.cap, spec.key_bits, spec.value_bits, device)
+            c = m.LayerConstants(kb, vb, params["key_signs"], params["value_rot"], spec.num_q_heads, device,
+                                 key_meta_format=META_FORMATS[meta])
+            cache = m.KVCache(spec.batch, spec.num_kv_heads, self.cap, spec.key_bits, spec.value_bits, device,
+                              key_meta_format=META_FORMATS[meta])
             drift = key_drift(spec, seed, layer, self.cap // 32, device)
             if spec.ragged:
                 for b in range(spec.batch):
@@ -296,9 +299,10 @@ class Workload:
         sp = self.spec
         L = self.lengths.astype(np.int64) + s
         T = (L + 1).sum()
-        rec = BYTES_PER_TOKEN_HEAD[(sp.key_bits, sp.value_bits)] * 32
+        per_token = BYTES_PER_TOKEN_HEAD[(sp.key_bits, sp.value_bits, self.meta)]
+        rec = int(per_token * 32)
         append = sp.num_kv_heads * int((512 + 256 * (L % 32) + rec).sum())
-        return int(T * sp.num_kv_heads * BYTES_PER_TOKEN_HEAD[(sp.key_bits, sp.value_bits)] + T + append)
+        return int(T * sp.num_kv_heads * per_token + T + append)
 
 
 def run_gpu(args):
@@ -314,7 +318,7 @@ def run_gpu(args):
     seed = rank_seed(args.workload, rank)
     K, W = args.steps, args.warmup
     total = W + K + K + 1  # device-resident run, then the e2e run
-    wl = Workload(spec, seed, dev, total)
+    wl = Workload(spec, seed, dev, total, args.meta)
     stream = torch.cuda.Stream(dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     torch.cuda.synchronize(dev)
@@ -420,12 +424,12 @@ def run_gpu(args):
             "warmup": W, "ms_per_step": round(total_ms / K, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "u2 codes, f32 accumulate",
             "data": "synthetic",
-            "config": workload_config(spec, world),
+            "config": workload_config(spec, world, args.meta),
             "launch": {"num_splits": wl.S, "fused_append": bool(wl.fused),
                        "graph": "one CUDA graph for all steps (flush + events + C-ABI calls)" if use_graphs
                        else "eager"},
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                         "frac": round(achieved / peak, 4), "traffic": captured_traffic(spec.name),
+                         "frac": round(achieved / peak, 4), "traffic": captured_traffic(spec.name, args.meta),
                          "peak_source": peak_kind,
                          "kernel": "decode_step_kernel (append + decode launch)" if wl.fused
                          else "kv_append_kernel + decode_split_k launches",
@@ -438,7 +442,7 @@ def run_gpu(args):
             "dense_bf16": dense,
         }
         if not args.no_cpu_baseline and world == 1:  # the oracle is timed at N = 1 only
-            line["cpu_baseline"] = cpu_baseline(spec, seed)
+            line["cpu_baseline"] = cpu_baseline(spec, seed, args.meta)
         print(json.dumps(line), flush=True)
     del graph, g2
     if world > 1:
@@ -541,7 +545,7 @@ def oracle_sample_shape(spec):
     return 1, min(spec.batch, 4)
 
 
-def _oracle_sequences(spec, seed, layers, seqs, extra_steps):
+def _oracle_sequences(spec, seed, layers, seqs, extra_steps, meta="fp16"):
     """The oracle's caches of the sampled (layer, sequence) pairs, each a batch-1
     cache prefilled with that sequence's context (untimed), and every layer's
     decode inputs for extra_steps steps."""
@@ -560,7 +564,7 @@ def _oracle_sequences(spec, seed, layers, seqs, extra_steps):
         for b in seqs:
             k, v, mod = prefill_inputs(spec, seed, layer, params, drift, L, "cpu", batch_index=[b])
             n = int(L[b])
-            oc = codec.OracleCache(1, spec.num_kv_heads, cap, spec.key_bits, spec.value_bits)
+            oc = codec.OracleCache(1, spec.num_kv_heads, cap, spec.key_bits, spec.value_bits, meta_format=meta)
             codec.write_cache(ocfg, oc, k[:, :, :n].numpy(), v[:, :, :n].numpy(), mod[:, :n].numpy())
             caches.append(oc)
             del k, v, mod
@@ -579,12 +583,12 @@ def _oracle_step(ocfg, oc, inputs, b, num_splits=4):
     return decode_fused(ocfg, oc, q, num_splits)
 
 
-def cpu_baseline(spec, seed):
+def cpu_baseline(spec, seed, meta="fp16"):
     """The oracle as it stands (numpy fp64, one pinned core) on a bounded sample of
     the workload -- one decode step of the sampled layers and sequences -- scaled
     linearly to the whole step (all layers, all sequences)."""
     n_layers, n_seq = oracle_sample_shape(spec)
-    prepared = _oracle_sequences(spec, seed, range(n_layers), range(n_seq), 1)
+    prepared = _oracle_sequences(spec, seed, range(n_layers), range(n_seq), 1, meta)
     with OneCore():
         t0 = time.perf_counter()
         for ocfg, caches, steps in prepared:
@@ -615,7 +619,7 @@ def run_reference(args):
     seed = WORKLOADS_KEYS.index(args.workload)
     K, W = args.steps, args.warmup
     n_seq = min(spec.batch, 2)
-    prepared = _oracle_sequences(spec, seed, [0], range(n_seq), (W + K) // n_seq + 2)
+    prepared = _oracle_sequences(spec, seed, [0], range(n_seq), (W + K) // n_seq + 2, args.meta)
     ocfg, caches, steps = prepared[0]
     times = []
     with OneCore():
@@ -639,7 +643,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
         "steps": K, "warmup": W, "ms_per_step": round(per_step * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic",
-        "config": workload_config(spec, world),
+        "config": workload_config(spec, world, args.meta),
         "extrapolated": scale != 1, "sample_ms_per_step": round(sample_s * 1e3, 3),
         "cpu_baseline": base,
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -669,11 +673,12 @@ def run_layer(args):
     T = int(L.max())
     cap = int(-(-(T + 8) // 32) * 32)
     params = layer_params(spec, seed, 0)
+    fmt = META_FORMATS[args.meta]
     consts = m.LayerConstants(codebook(bits), codebook(bits), params["key_signs"], params["value_rot"],
-                              spec.num_q_heads, dev)
+                              spec.num_q_heads, dev, key_meta_format=fmt)
     drift = key_drift(spec, seed, 0, cap // 32, dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    per_token = BYTES_PER_TOKEN_HEAD[(bits, bits)]
+    per_token = BYTES_PER_TOKEN_HEAD[(bits, bits, args.meta)]
     peak, _ = peaks()
     iters, warm = 5, 2
 
@@ -694,19 +699,19 @@ def run_layer(args):
 
     if args.layer == "write":
         k, v, mod = prefill_inputs(spec, seed, 0, params, drift, np.full(spec.batch, T), dev)
-        c = m.KVCache(spec.batch, spec.num_kv_heads, cap, bits, bits, dev)
+        c = m.KVCache(spec.batch, spec.num_kv_heads, cap, bits, bits, dev, key_meta_format=fmt)
 
         def empty():  # the prefill of an empty cache, every time
             c.seq_lens.zero_()
             c.struct.max_seq_len = 0
 
         us = timed(lambda: m.omnikv_write_cache(consts.struct, c.struct, k, v, mod, T), empty)
-        byts = spec.batch * T * spec.num_kv_heads * (512 + per_token) + spec.batch * T
-        print(json.dumps({"layer": "write", "workload": spec.name, "tokens": spec.batch * T, "us": round(us, 2),
+        byts = int(spec.batch * T * spec.num_kv_heads * (512 + per_token) + spec.batch * T)
+        print(json.dumps({"layer": "write", "workload": spec.name, "meta": args.meta, "tokens": spec.batch * T, "us": round(us, 2),
                           "GBps": round(byts / us / 1e3, 1), "frac": round(byts / us / 1e3 / peak, 4),
                           "error_word": int(c.error_word.item())}), flush=True)
         return
-    cache = m.KVCache(spec.batch, spec.num_kv_heads, cap, bits, bits, dev)
+    cache = m.KVCache(spec.batch, spec.num_kv_heads, cap, bits, bits, dev, key_meta_format=fmt)
     for b in range(spec.batch):
         k, v, mod = prefill_inputs(spec, seed, 0, params, drift, L, dev, batch_index=[b])
         n = int(L[b])
@@ -715,14 +720,14 @@ def run_layer(args):
         del k, v, mod
     cache.struct.max_seq_len = T
     q = torch.randn(spec.batch, spec.num_q_heads, 128, device=dev).half()
-    byts = int(L.astype(np.int64).sum()) * spec.num_kv_heads * per_token + int(L.sum())
+    byts = int(int(L.astype(np.int64).sum()) * spec.num_kv_heads * per_token + int(L.sum()))
     for S in [int(x) for x in args.splits.split(",")]:
         S = S or m.omnikv_default_splits(consts.struct, cache.struct)
         part = m.partials_tensor(spec.batch, spec.num_q_heads, S, dev)
         out = torch.empty(spec.batch, spec.num_q_heads, 128, device=dev)
         dec = timed(lambda: m.omnikv_decode_attention(consts.struct, cache.struct, q, part, S))
         comb = timed(lambda: m.omnikv_combine(consts.struct, cache.struct, part, S, out))
-        print(json.dumps({"layer": "decode", "workload": spec.name, "splits": S, "decode_us": round(dec, 2),
+        print(json.dumps({"layer": "decode", "workload": spec.name, "meta": args.meta, "splits": S, "decode_us": round(dec, 2),
                           "combine_us": round(comb, 2), "GBps": round(byts / dec / 1e3, 1),
                           "frac": round(byts / dec / 1e3 / peak, 4), "error_word": int(cache.error_word.item())}),
               flush=True)

@@ -3,6 +3,8 @@
 // path (4-bit caches and codebooks that are not symmetric).
 #pragma once
 
+#include <cstddef>
+
 #include "append.cuh"
 #include "common.cuh"
 #include "kernels.h"
@@ -132,6 +134,9 @@ struct GenSmem {                 // laid over the calling body's staging buffers
   uint32_t runs;                  // bit t: token t of the current window starts a run of one modality
   int abort;                      // a step flag never arrived: the split is written empty
 };
+
+static_assert(offsetof(GenSmem, qT) % 16 == 0 && offsetof(GenSmem, pw) % 16 == 0, "16-byte vector fields");
+static_assert(offsetof(GenSmem, mxm) % 8 == 0 && offsetof(GenSmem, bar) % 8 == 0, "8-byte fields");
 
 // (m^, s^) of channel c from a window's MXFP4 key metadata: E2M1 codes two per
 // byte (even channel in the low nibble), minima then scales, then the E8M0

@@ -71,6 +71,7 @@
 // OMNIKV_DEVERR_RANGE is set. Key scales below 2^-7 lose relative precision in the
 // s_gc * 2^-7 plane (fp16 subnormals); realistic key ranges are far above.
 #include <atomic>
+#include <cstddef>
 
 #include "decode_common.cuh"
 
@@ -114,12 +115,18 @@ struct __align__(16) DecodeSmem {
   float red[kWarps][1 + kMods][kMaxGroup];        // cooperative body: per-warp sums of p and of p sigma per modality
   uint32_t tmask[kCoop][2];                       // cooperative body: modality bits of each tile of the group (0: no window)
   uint32_t tmem_base;                             // per-warp body: TMEM columns of the parked accumulators
-  uint32_t mxpairs[kWarps][kHeadDim];             // MXFP4 caches: a warp's window metadata as fp16 (m, s) pairs
+  alignas(16) uint32_t mxpairs[kWarps][kHeadDim]; // MXFP4 caches: a warp's window metadata as fp16 (m, s) pairs
+                                                  // (read as 16-byte vectors)
   uint32_t bad_heads;                             // bit h: head h's partial is not finite (written empty)
   int abort;                                      // cooperative body: a step flag never arrived
   int wabort[kWarps];                             // per-warp body: a step flag of warp w never arrived
 };
 static_assert(sizeof(DecodeSmem) <= 48 * 1024, "static shared memory");
+// fields read or written as 16-byte / 8-byte vectors, and mbarriers
+static_assert(offsetof(DecodeSmem, btab) % 16 == 0 && offsetof(DecodeSmem, q) % 16 == 0 &&
+                  offsetof(DecodeSmem, mxpairs) % 16 == 0, "16-byte vector fields");
+static_assert(offsetof(DecodeSmem, mw) % 8 == 0 && offsetof(DecodeSmem, bar) % 8 == 0 &&
+                  offsetof(DecodeSmem, cbar) % 8 == 0, "8-byte fields");
 static_assert(sizeof(GenSmem) <= sizeof(DecodeSmem::u), "CUDA-core path shared memory");
 
 // ---------------------------------------------------------------------------
@@ -331,8 +338,11 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
   for (int i = 0; i < nmine; ++i) {
     const int s = i % kStages;
     const int wi = wa + i;
-    if (!mbar_wait_bounded(&sm.bar[warp][s], (i / kStages) & 1, kWaitLimitNs) ||
-        *reinterpret_cast<volatile int*>(&sm.wabort[warp]) != 0) {
+    // the warp leaves together: a lane whose wait ran out, or lane 0 (the lane
+    // that issues the copies) having given up on a step flag, stops every lane
+    const bool ok = mbar_wait_bounded(&sm.bar[warp][s], (i / kStages) & 1, kWaitLimitNs) &&
+                    *reinterpret_cast<volatile int*>(&sm.wabort[warp]) == 0;
+    if (!__all_sync(0xffffffffu, ok)) {
       failed_at = i;
       break;
     }
@@ -723,18 +733,22 @@ __device__ __forceinline__ void issue_group(const DecodeParams& p, DecodeSmem& s
                                             int b, int kvh, int wfirst, int nwin, int wait_win, int wait_val) {
   uint64_t* bar = &sm.cbar[stage];
   uint8_t* dst = &sm.u.c.stage[stage][0];
+  constexpr int rb = Rec22<kMeta>::bytes;
   int nfree = nwin;  // records that need no wait
   if (wait_win >= wfirst && wait_win < wfirst + nwin) nfree = wait_win - wfirst;
-  // the records that need no wait and the modality ids are copied first; the
-  // phase cannot complete before the arrive below
-  constexpr int rb = Rec22<kMeta>::bytes;
-  mbar_expect_tx(bar, (uint32_t)nfree * rb + (uint32_t)nwin * kWindow);
-  if (nfree > 0) bulk_copy_g2s(dst, rec_base + (size_t)wfirst * rb, (uint32_t)nfree * rb, bar);
-  bulk_copy_g2s(dst + kCoop * rb, p.modality + (size_t)b * p.cap_tokens + (size_t)wfirst * kWindow,
-                (uint32_t)nwin * kWindow, bar);
   if (nfree == nwin) {
-    mbar_arrive_expect_tx(bar, 0);
+    mbar_arrive_expect_tx(bar, (uint32_t)nwin * (rb + kWindow));
+    bulk_copy_g2s(dst, rec_base + (size_t)wfirst * rb, (uint32_t)nwin * rb, bar);
+    bulk_copy_g2s(dst + kCoop * rb, p.modality + (size_t)b * p.cap_tokens + (size_t)wfirst * kWindow,
+                  (uint32_t)nwin * kWindow, bar);
     return;
+  }
+  // the records that need no wait are copied first; the phase cannot complete
+  // before the arrive below. The modality ids (the appended token's is written by
+  // its append CTA before the flag) and the waited-for records follow the flag.
+  if (nfree > 0) {
+    mbar_expect_tx(bar, (uint32_t)nfree * rb);
+    bulk_copy_g2s(dst, rec_base + (size_t)wfirst * rb, (uint32_t)nfree * rb, bar);
   }
   if (!wait_flag(p.step_flags + (size_t)b * p.num_kv_heads + kvh, wait_val, p.flag_wait_ns)) {
     // the appended token's record never became ready: no copy of a stale record;
@@ -744,9 +758,10 @@ __device__ __forceinline__ void issue_group(const DecodeParams& p, DecodeSmem& s
     mbar_arrive_expect_tx(bar, 0);
     return;
   }
-  mbar_arrive_expect_tx(bar, (uint32_t)(nwin - nfree) * rb);
-  bulk_copy_g2s(dst + nfree * rb, rec_base + (size_t)(wfirst + nfree) * rb, (uint32_t)(nwin - nfree) * rb,
-                bar);
+  mbar_arrive_expect_tx(bar, (uint32_t)(nwin - nfree) * rb + (uint32_t)nwin * kWindow);
+  bulk_copy_g2s(dst + nfree * rb, rec_base + (size_t)(wfirst + nfree) * rb, (uint32_t)(nwin - nfree) * rb, bar);
+  bulk_copy_g2s(dst + kCoop * rb, p.modality + (size_t)b * p.cap_tokens + (size_t)wfirst * kWindow,
+                (uint32_t)nwin * kWindow, bar);
 }
 
 // The tensor-core decode of one split. Windows are taken kCoop at a time (a
@@ -1158,6 +1173,7 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, DecodeSmem& sm
   }
   rotate_queries(p, b, kvh, &sm.q[0][0]);
   if (threadIdx.x == 0) sm.bad_heads = 0u;
+  __syncthreads();  // every warp's rotated queries are written before they are scanned
   // the score operand carries a power of two 2^-E that keeps its largest entry at
   // most 2^14 (so large queries stay inside the fp16 range); scores are scaled back
   // by 2^E in fp32

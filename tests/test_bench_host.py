@@ -37,12 +37,31 @@ def test_clock_record_empty(tmp_path):
 
 def test_traffic_reported_only_for_the_captured_sources(monkeypatch):
     wl = "qwen3-omni-30b-48L-b8-ctx65536"
-    monkeypatch.setattr(bench, "TRAFFIC_CAPTURES", {wl: {"sources_sha256": bench.kernel_sources_sha256(),
-                                                         "bytes_per_launch": 123}})
+    monkeypatch.setattr(bench, "TRAFFIC_CAPTURES", {(wl, "fp16"): {"sources_sha256": bench.kernel_sources_sha256(),
+                                                                   "bytes_per_launch": 123}})
     assert bench.captured_traffic(wl) == 123
+    assert bench.captured_traffic(wl, "mx") is None                            # another metadata format
     assert bench.captured_traffic("qwen2.5-omni-3b-36L-b16-ctx32768") is None  # another workload
-    monkeypatch.setattr(bench, "TRAFFIC_CAPTURES", {wl: {"sources_sha256": "0" * 64, "bytes_per_launch": 123}})
+    monkeypatch.setattr(bench, "TRAFFIC_CAPTURES", {(wl, "fp16"): {"sources_sha256": "0" * 64,
+                                                                   "bytes_per_launch": 123}})
     assert bench.captured_traffic(wl) is None                                  # sources changed since
+
+
+def test_kernel_sources_cover_the_decode_sources():
+    """Every kernel source the decode and step kernels include is hashed (the
+    public header outside the source folder holds declarations only)."""
+    import os
+    import re
+    d = os.path.join(os.path.dirname(bench.__file__), "bit_kv_cache_pack_b200", "csrc")
+    seen, todo = set(), ["decode_split_k.cu"]
+    while todo:
+        name = todo.pop()
+        if name in seen or "/" in name or not os.path.exists(os.path.join(d, name)):
+            continue
+        seen.add(name)
+        with open(os.path.join(d, name)) as f:
+            todo += re.findall(r'#include "([^"]+)"', f.read())
+    assert seen <= set(bench.KERNEL_SOURCES), sorted(seen - set(bench.KERNEL_SOURCES))
 
 
 def test_both_arms_share_the_config_object():
