@@ -53,7 +53,11 @@ META_FORMATS = {"fp16": 0, "mx": 1}   # omnikv_config.key_meta_format
 # benchmark (its summary is kept with the other profiles), valid for the kernel
 # sources with this SHA-256; any change to them makes the field null until the
 # next capture.
-TRAFFIC_CAPTURES = {}
+TRAFFIC_CAPTURES = {
+    ("qwen3-omni-30b-48L-b8-ctx65536", "fp16"): {
+        "sources_sha256": "799cd4759c72a470928c8d49d5aae5d6bc7a99b927e0bf951309ec3e40f878e9",
+        "bytes_per_launch": 173718528 + 8225024},
+}
 KERNEL_SOURCES = ("decode_split_k.cu", "decode_common.cuh", "append.cuh", "common.cuh", "ptx.cuh", "kernels.h")
 
 
