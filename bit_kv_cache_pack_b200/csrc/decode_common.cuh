@@ -141,10 +141,22 @@ static_assert(offsetof(GenSmem, mxm) % 8 == 0 && offsetof(GenSmem, bar) % 8 == 0
 // (m^, s^) of channel c from a window's MXFP4 key metadata: E2M1 codes two per
 // byte (even channel in the low nibble), minima then scales, then the E8M0
 // exponents (e + 127) of the 4 minimum blocks and the 4 scale blocks.
+// E2M1 code (sign << 3 | magnitude index i) times 2^(eb - 127) for a block exponent
+// byte eb, without branches: the magnitude's fp32 bits (0, 0.5, or (1 + (i & 1)/2) *
+// 2^(i/2 - 1) for i >= 2) times the fp32 power of two (2^-127 is subnormal; eb = 255
+// is taken as 2^127 * 2). Exact, and the same value as mx_value(code, eb - 127).
+__device__ __forceinline__ float mx_decode(uint32_t code, uint32_t eb) {
+  const uint32_t i = code & 7u;
+  const uint32_t mag = i >= 2u ? (i << 22) + 0x3F000000u : (i != 0u ? 0x3F000000u : 0u);
+  const float p2 = __uint_as_float(eb == 0u ? 0x00400000u : (eb == 255u ? 254u << 23 : eb << 23));
+  const float v = __uint_as_float(mag | ((code & 8u) << 28)) * p2;
+  return eb == 255u ? v * 2.0f : v;
+}
+
 __device__ __forceinline__ float2 mx_meta_channel(const uint8_t* meta, int c) {
   const uint32_t mb = meta[c >> 1], sb = meta[64 + (c >> 1)];
   const uint32_t mc = (c & 1) ? (mb >> 4) : (mb & 15u), sc = (c & 1) ? (sb >> 4) : (sb & 15u);
-  return make_float2(mx_value(mc, (int)meta[128 + (c >> 5)] - 127), mx_value(sc, (int)meta[132 + (c >> 5)] - 127));
+  return make_float2(mx_decode(mc, meta[128 + (c >> 5)]), mx_decode(sc, meta[132 + (c >> 5)]));
 }
 
 __device__ __forceinline__ void gen_issue(const DecodeParams& p, GenSmem& g, int stage, const uint8_t* rec_base,

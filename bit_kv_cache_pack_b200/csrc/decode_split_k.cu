@@ -156,7 +156,7 @@ __device__ __forceinline__ void split_pair_t(float x0, float x1, uint32_t& hi, u
 // record's own for fp16 metadata; for MXFP4 the warp converts its window's E2M1
 // values (exact in fp16 for block exponents in [-16, 12]; a scale beyond makes the
 // split non-finite, reported as OMNIKV_DEVERR_RANGE) into its buffer.
-__device__ __noinline__ void mx_window_pairs(const uint8_t* meta, uint32_t* out, int lane) {
+__device__ __forceinline__ void mx_window_pairs(const uint8_t* meta, uint32_t* out, int lane) {
   __syncwarp();  // the previous window's readers are done
 #pragma unroll
   for (int k = 0; k < 4; ++k) {

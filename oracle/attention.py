@@ -43,7 +43,8 @@ def key_rotation_matrix(signs):
 def dequantize(cfg: OracleConfig, cache: OracleCache, b: int, h: int):
     """Rotated-space dequantised cache of one (sequence, kv head):
     k_hat'[t][c] = m + s (c_j - c_0) with the record's decoded metadata (fp16 m16, s16, or
-    MXFP4 m^, s^), v_hat'[t][c] = sigma16 c_j  (fp64),
+    MXFP4 m^, s^), or k_hat'[t][c] = sigma16_t c_j for the TurboQuant key codec (one
+    scale per token); v_hat'[t][c] = sigma16 c_j  (fp64),
     and the modality id of every token. Returns (kq [T][128], vq [T][128], mod [T])."""
     T = int(cache.seq_lens[b])
     ck = np.asarray(cfg.key_codebook, dtype=np.float32).astype(F64)
@@ -53,8 +54,11 @@ def dequantize(cfg: OracleConfig, cache: OracleCache, b: int, h: int):
     vq = np.zeros((nw * WINDOW, HEAD_DIM), F64)
     for w in range(nw):
         kc = unpack_key_codes(cache.k_words(b, h, w), cache.key_bits)
-        m, s = (x.astype(F64) for x in cache.key_meta_f32(b, h, w))
-        kq[w * WINDOW:(w + 1) * WINDOW] = m[None, :] + s[None, :] * (ck[kc] - ck[0])
+        if cache.meta_format == "turbo":
+            kq[w * WINDOW:(w + 1) * WINDOW] = cache.key_sigma(b, h, w).astype(F64)[:, None] * ck[kc]
+        else:
+            m, s = (x.astype(F64) for x in cache.key_meta_f32(b, h, w))
+            kq[w * WINDOW:(w + 1) * WINDOW] = m[None, :] + s[None, :] * (ck[kc] - ck[0])
         vc = unpack_value_codes(cache.v_words(b, h, w), cache.value_bits)
         sg = cache.sigma(b, h, w).astype(F64)
         vq[w * WINDOW:(w + 1) * WINDOW] = sg[:, None] * cv[vc]

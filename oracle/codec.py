@@ -71,7 +71,10 @@ def codes_per_word(bits: int) -> int:
     return 32 // bits
 
 
-META_FORMATS = ("fp16", "mx")  # key metadata: fp16 (m, s) pairs, or MXFP4 (oracle/mxmeta.py)
+# key metadata: fp16 (m, s) pairs per window channel, MXFP4 (oracle/mxmeta.py), or the
+# TurboQuant key codec ("turbo": one fp16 scale per token, no window statistics)
+META_FORMATS = ("fp16", "mx", "turbo")
+META_BYTES = {"fp16": HEAD_DIM * 4, "mx": 144, "turbo": WINDOW * 2}
 
 
 def record_offsets(key_bits: int, value_bits: int, meta_format: str = "fp16"):
@@ -80,7 +83,7 @@ def record_offsets(key_bits: int, value_bits: int, meta_format: str = "fp16"):
     k_bytes = WINDOW * HEAD_DIM * key_bits // 8
     v_bytes = WINDOW * HEAD_DIM * value_bits // 8
     meta = k_bytes
-    v = meta + (HEAD_DIM * 4 if meta_format == "fp16" else 144)
+    v = meta + META_BYTES[meta_format]
     sig = v + v_bytes
     total = sig + WINDOW * 2
     return {"k": 0, "meta": meta, "v": v, "sigma": sig, "total": total,
@@ -289,6 +292,13 @@ class OracleCache:
             raise ValueError("the record holds MXFP4 metadata")
         return self.records[b, h, w, o["meta"]:o["v"]].view(F16).reshape(HEAD_DIM, 2)
 
+    def key_sigma(self, b, h, w):
+        """turbo format: the [32] fp16 key scales of the record's tokens."""
+        o = self.off
+        if self.meta_format != "turbo":
+            raise ValueError("the record holds window metadata")
+        return self.records[b, h, w, o["meta"]:o["v"]].view(F16)
+
     def meta_bytes(self, b, h, w):
         o = self.off
         return self.records[b, h, w, o["meta"]:o["v"]]
@@ -298,6 +308,8 @@ class OracleCache:
         if self.meta_format == "fp16":
             mt = self.meta(b, h, w)
             return mt[:, 0].astype(F32), mt[:, 1].astype(F32)
+        if self.meta_format == "turbo":
+            raise ValueError("turbo records have per-token key scales, not window metadata")
         from . import mxmeta
         unpacked = mxmeta.unpack_meta_mx(self.meta_bytes(b, h, w))
         return unpacked[4], unpacked[5]
@@ -335,6 +347,23 @@ def quantize_key_window_mx(cfg: OracleConfig, raw_keys_fp16):
     codes = np.zeros((WINDOW, HEAD_DIM), np.uint32)
     codes[:n] = mxmeta.key_codes_mx(kp, m_hat, s_hat, cfg.key_codebook)
     return pack_key_codes(codes, cfg.key_bits), mxmeta.pack_meta_mx(m_codes, m_exps, s_codes, s_exps)
+
+
+def quantize_key_window_turbo(cfg: OracleConfig, raw_keys_fp16):
+    """The TurboQuant key codec on one window of raw fp16 keys (pchao.org 关联工作;
+    paperpeel.com section 2.2 "Temporal key drift": one random rotation and a
+    per-token scale, no window statistics). Each token on its own: k' = R k (a1),
+    sigma16 = fp16(||k|| / sqrt(128)) from the unrotated key (the value scale's
+    rule, reading r6), code = #{j : k'_c / sigma16 > t_j} (the value code's rule).
+    Returns (packed words, sigma16 [32]); padded rows get code 0 and scale 0."""
+    n = raw_keys_fp16.shape[0]
+    kp = rotate_keys(raw_keys_fp16, cfg.key_signs)
+    sg = np.zeros(WINDOW, F16)
+    codes = np.zeros((WINDOW, HEAD_DIM), np.uint32)
+    if n:
+        sg[:n] = value_sigma(raw_keys_fp16)
+        codes[:n] = value_codes(kp, sg[:n], cfg.key_codebook)
+    return pack_key_codes(codes, cfg.key_bits), sg
 
 
 def encode_values_with_basis(v_fp16, basis, codebook):
@@ -388,6 +417,9 @@ def write_cache(cfg: OracleConfig, cache: OracleCache, k_new, v_new, modality_ne
                     meta = cache.meta(b, h, w)
                     meta[:, 0] = m16
                     meta[:, 1] = s16
+                elif cache.meta_format == "turbo":
+                    words, ksg = quantize_key_window_turbo(cfg, raw)
+                    cache.key_sigma(b, h, w)[:] = ksg
                 else:
                     words, mbytes = quantize_key_window_mx(cfg, raw)
                     cache.meta_bytes(b, h, w)[:] = mbytes
