@@ -45,8 +45,9 @@ WORKLOADS_KEYS = ("tiny", "omni3b-b1", "omni3b-b16", "omni30b-b8", "ragged-b64")
 METRIC = "2-bit decode attention tokens/s and achieved HBM GB/s vs ~8 TB/s (1 B200)"
 UNIT = "tokens/s"
 # algorithmic packed bytes per token per kv head: (key bits, value bits, key metadata format)
-BYTES_PER_TOKEN_HEAD = {(2, 2, "fp16"): 82, (4, 4, "fp16"): 146, (2, 2, "mx"): 70.5, (4, 4, "mx"): 134.5}
-META_FORMATS = {"fp16": 0, "mx": 1}   # omnikv_config.key_meta_format
+BYTES_PER_TOKEN_HEAD = {(2, 2, "fp16"): 82, (4, 4, "fp16"): 146, (2, 2, "mx"): 70.5, (4, 4, "mx"): 134.5,
+                        (2, 2, "turbo"): 68, (4, 4, "turbo"): 132}
+META_FORMATS = {"fp16": 0, "mx": 1, "turbo": 2}   # omnikv_config.key_meta_format
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the
 # timed kernel, per (workload, key metadata format), from an ncu capture of this
@@ -94,7 +95,8 @@ def parse_args():
                          "the decode step; prints one JSON line per split count")
     ap.add_argument("--bits", type=int, default=0, help="with --layer: 2 or 4 (default: the workload's)")
     ap.add_argument("--meta", default="fp16", choices=sorted(META_FORMATS),
-                    help="key metadata format: fp16 (m, s) pairs or mx (MXFP4, the pages' default)")
+                    help="key metadata format: fp16 (m, s) pairs, mx (MXFP4, the pages' default) or turbo "
+                         "(the TurboQuant key codec the pages compare against: one scale per token)")
     ap.add_argument("--batch", type=int, default=0, help="with --layer: override the workload's batch")
     ap.add_argument("--splits", default="0", help="with --layer decode: comma-separated split counts (0: default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -123,7 +125,7 @@ def workload_config(spec, world, meta="fp16"):
             "context": int(L.max()) if not spec.ragged else "%d..%d" % spec.ragged,
             "num_q_heads": spec.num_q_heads, "num_kv_heads": spec.num_kv_heads, "head_dim": 128,
             "key_bits": spec.key_bits, "value_bits": spec.value_bits, "window": 32,
-            "key_meta_format": "mxfp4" if meta == "mx" else "fp16",
+            "key_meta_format": {"fp16": "fp16", "mx": "mxfp4", "turbo": "turbo (per-token key scale)"}[meta],
             "parallelism": "dp%d (independent sequences per rank)" % world,
             "l2": "GPU arm: flushed between timed steps (512 MiB write)"}
 

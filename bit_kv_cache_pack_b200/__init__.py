@@ -5,7 +5,7 @@ include/omnikv.h); this package is its thin Python binding plus PyTorch
 allocation helpers.
 """
 from ._abi import (OMNIKV_DEVERR_CAPACITY, OMNIKV_ERR_CAPACITY, OMNIKV_ERR_CUDA,  # noqa: F401
-                   OMNIKV_META_FP16, OMNIKV_META_MXFP4, omnikv_record_bytes_meta,
+                   OMNIKV_META_FP16, OMNIKV_META_MXFP4, OMNIKV_META_TURBO, omnikv_record_bytes_meta,
                    OMNIKV_ERR_INVALID_ARG, OMNIKV_ERR_UNSUPPORTED, OMNIKV_OK, OmniKVCache,
                    OmniKVConfig, OmniKVError, load, omnikv_abi_version, omnikv_combine,
                    omnikv_append_decode, omnikv_combine_step, omnikv_decode_attention, omnikv_decode_static,

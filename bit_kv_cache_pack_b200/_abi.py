@@ -26,6 +26,7 @@ OMNIKV_DEVERR_BOUND = 0x8
 OMNIKV_DEVERR_RANGE = 0x10
 OMNIKV_META_FP16 = 0
 OMNIKV_META_MXFP4 = 1
+OMNIKV_META_TURBO = 2
 
 EXPORTED = (
     "omnikv_record_bytes", "omnikv_partials_bytes", "omnikv_default_splits",

@@ -13,6 +13,11 @@ namespace {
 
 bool aligned(const void* ptr, size_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; }
 
+// the kernels' key metadata format of a validated omnikv_config.key_meta_format
+int meta_of(int32_t key_meta_format) {
+  return key_meta_format == OMNIKV_META_MXFP4 ? kMetaMx : key_meta_format == OMNIKV_META_TURBO ? kMetaTurbo : kMetaFp16;
+}
+
 omnikv_status check_config(const omnikv_config* cfg) {
   if (!cfg) return OMNIKV_ERR_INVALID_ARG;
   if (cfg->head_dim != kHeadDim || cfg->window != kWindow) return OMNIKV_ERR_UNSUPPORTED;
@@ -24,7 +29,8 @@ omnikv_status check_config(const omnikv_config* cfg) {
   if (!cfg->key_codebook || !cfg->value_codebook || !cfg->key_signs || !cfg->value_rot)
     return OMNIKV_ERR_INVALID_ARG;
   if (!aligned(cfg->key_signs, 16) || !aligned(cfg->value_rot, 16)) return OMNIKV_ERR_INVALID_ARG;
-  if (cfg->key_meta_format != OMNIKV_META_FP16 && cfg->key_meta_format != OMNIKV_META_MXFP4)
+  if (cfg->key_meta_format != OMNIKV_META_FP16 && cfg->key_meta_format != OMNIKV_META_MXFP4 &&
+      cfg->key_meta_format != OMNIKV_META_TURBO)
     return OMNIKV_ERR_UNSUPPORTED;
   return OMNIKV_OK;
 }
@@ -110,7 +116,7 @@ omnikv_status prepare_decode(const omnikv_config* cfg, const omnikv_cache* cache
   p->value_rot = cfg->value_rot;
   p->key_bits = cfg->key_bits;
   p->value_bits = cfg->value_bits;
-  p->key_meta = cfg->key_meta_format == OMNIKV_META_MXFP4 ? kMetaMx : kMetaFp16;
+  p->key_meta = meta_of(cfg->key_meta_format);
   p->num_kv_heads = cfg->num_kv_heads;
   p->group = cfg->num_q_heads / cfg->num_kv_heads;
   p->records = static_cast<const uint8_t*>(cache->records);
@@ -169,8 +175,10 @@ size_t omnikv_record_bytes(int32_t key_bits, int32_t value_bits) {
 
 size_t omnikv_record_bytes_meta(int32_t key_bits, int32_t value_bits, int32_t key_meta_format) {
   if ((key_bits != 2 && key_bits != 4) || (value_bits != 2 && value_bits != 4)) return 0;
-  if (key_meta_format != OMNIKV_META_FP16 && key_meta_format != OMNIKV_META_MXFP4) return 0;
-  return (size_t)RecordLayout(key_bits, value_bits, key_meta_format == OMNIKV_META_MXFP4 ? kMetaMx : kMetaFp16).bytes;
+  if (key_meta_format != OMNIKV_META_FP16 && key_meta_format != OMNIKV_META_MXFP4 &&
+      key_meta_format != OMNIKV_META_TURBO)
+    return 0;
+  return (size_t)RecordLayout(key_bits, value_bits, meta_of(key_meta_format)).bytes;
 }
 
 size_t omnikv_partials_bytes(int32_t batch, int32_t num_q_heads, int32_t num_splits) {
@@ -193,7 +201,7 @@ void fill_write_params(const omnikv_config* cfg, const omnikv_cache* cache, cons
   p->value_rot = cfg->value_rot;
   p->key_bits = cfg->key_bits;
   p->value_bits = cfg->value_bits;
-  p->key_meta = cfg->key_meta_format == OMNIKV_META_MXFP4 ? kMetaMx : kMetaFp16;
+  p->key_meta = meta_of(cfg->key_meta_format);
   p->num_kv_heads = cfg->num_kv_heads;
   p->records = static_cast<uint8_t*>(cache->records);
   p->key_tail = static_cast<__half*>(cache->key_tail);

@@ -34,12 +34,15 @@ __device__ __forceinline__ int kp_col(int t, int c) {
 }
 
 // Key codes of the window's valid tokens, code = #{j : (k' - m) / s + c_0 > t_j}
-// (0 where s == 0): thread c decides channel c for every token with the
-// channel's fp32 bounds, then the codes are packed 32 / BITS per token-major word.
+// (0 where s == 0) with window metadata, or code = #{j : k' / ksigma_t > t_j} (0
+// where ksigma_t == 0) for TurboQuant keys (scales in s_scale[0..31], bounds built
+// without c_0): thread c decides channel c for every token, then the codes are
+// packed 32 / BITS per token-major word.
 template <int BITS>
-__device__ __forceinline__ void key_code_words(WindowSmem& sm, uint8_t* kout, int nvalid, int tid, int bar_id) {
+__device__ __forceinline__ void key_code_words(WindowSmem& sm, uint8_t* kout, int nvalid, int tid, int bar_id,
+                                               bool turbo) {
   constexpr int NB = (1 << BITS) - 1, cpw = 32 / BITS, wpt = kHeadDim / cpw;
-  {
+  if (!turbo) {
     const int c = tid;
     const float s = sm.s_scale[c], m = sm.s_min[c];
     const ScaledBounds<NB> sb = scale_bounds(load_bounds<NB>(sm.bk), s);
@@ -49,6 +52,17 @@ __device__ __forceinline__ void key_code_words(WindowSmem& sm, uint8_t* kout, in
       sm.codes[t][c] = (uint8_t)((t < nvalid && s != 0.0f)
                                      ? code_from_scaled(sb, __fsub_rn(sm.kp[t][(t & 1) ? col1 : col0], m))
                                      : 0u);
+  } else {
+    const int c = tid;
+    const CodeBounds<NB> bd = load_bounds<NB>(sm.bk);
+    const int col0 = kp_col(0, c), col1 = kp_col(1, c);
+#pragma unroll 2
+    for (int t = 0; t < kWindow; ++t) {
+      const float s = sm.s_scale[t];
+      sm.codes[t][c] = (uint8_t)((t < nvalid && s != 0.0f)
+                                     ? code_from_scaled(scale_bounds(bd, s), sm.kp[t][(t & 1) ? col1 : col0])
+                                     : 0u);
+    }
   }
   group_sync(bar_id);
   uint32_t* kw = reinterpret_cast<uint32_t*>(kout);
@@ -100,8 +114,10 @@ __device__ void quantize_window(const WriteParams& p, int b, int h, int w, int L
   const int lane = tid & 31;
   const int LK = 1 << p.key_bits;
   const int LV = 1 << p.value_bits;
+  const bool turbo = p.key_meta == kMetaTurbo;
   const float kc0 = p.key_cb[0];
-  if (tid < LK - 1) sm.bk[tid] = make_code_bound(__fmul_rn(__fadd_rn(p.key_cb[tid], p.key_cb[tid + 1]), 0.5f), kc0);
+  if (tid < LK - 1)
+    sm.bk[tid] = make_code_bound(__fmul_rn(__fadd_rn(p.key_cb[tid], p.key_cb[tid + 1]), 0.5f), turbo ? 0.0f : kc0);
   if (tid >= 32 && tid - 32 < LV - 1) {
     const int j = tid - 32;
     sm.bv[j] = make_code_bound(__fmul_rn(__fadd_rn(p.val_cb[j], p.val_cb[j + 1]), 0.5f), 0.0f);
@@ -198,6 +214,35 @@ __device__ void quantize_window(const WriteParams& p, int b, int h, int w, int L
   }
   group_sync(bar_id);
 
+  // ---- TurboQuant keys: one scale per token from the unrotated fp16 key, the
+  // pairwise tree of the value scale (h = 64 across threads q ^ 2, h = 32 across
+  // q ^ 1, then h = 16 .. 1 inside the thread's 32 channels)
+  if (turbo) {
+    float x[32];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const __half2* hp = reinterpret_cast<const __half2*>(&raw[j]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __half22float2(hp[e]);
+        x[8 * j + 2 * e] = __fmul_rn(f.x, f.x);  // exact: an fp16 square fits in fp32
+        x[8 * j + 2 * e + 1] = __fmul_rn(f.y, f.y);
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < 32; ++c) x[c] = __fadd_rn(x[c], __shfl_xor_sync(0xffffffffu, x[c], 2));
+#pragma unroll
+    for (int c = 0; c < 32; ++c) x[c] = __fadd_rn(x[c], __shfl_xor_sync(0xffffffffu, x[c], 1));
+#pragma unroll
+    for (int hh = 16; hh >= 1; hh >>= 1)
+#pragma unroll
+      for (int c = 0; c < hh; ++c) x[c] = __fadd_rn(x[c], x[c + hh]);
+    if (tq == 0 && ti < kWindow) {
+      const __half s16 = ti < nvalid ? __float2half_rn(__fsqrt_rn(__fmul_rn(x[0], 0.0078125f))) : __float2half(0.0f);
+      reinterpret_cast<__half*>(rec + lay.meta_off)[ti] = s16;
+      s_scale[ti] = __half2float(s16);
+    }
+  } else {
   // ---- window range per channel -> fp16 metadata -----------------------------
   {
     const int c = tid;
@@ -246,13 +291,14 @@ __device__ void quantize_window(const WriteParams& p, int b, int h, int w, int L
       s_scale[c] = __half2float(s16);
     }
   }
+  }
   group_sync(bar_id);
 
   // ---- key codes, token-major words -----------------------------------------
   if (p.key_bits == 2)
-    key_code_words<2>(sm, rec + lay.k_off, nvalid, tid, bar_id);
+    key_code_words<2>(sm, rec + lay.k_off, nvalid, tid, bar_id, turbo);
   else
-    key_code_words<4>(sm, rec + lay.k_off, nvalid, tid, bar_id);
+    key_code_words<4>(sm, rec + lay.k_off, nvalid, tid, bar_id, turbo);
   group_sync(bar_id);  // kp is reused for values below
 
   // windows filled completely by this write get their values from vrot_tc

@@ -23,10 +23,14 @@ __device__ __forceinline__ float inv_sqrt_d() { return __int_as_float(0x3DB504F3
 
 // Key metadata formats of a window: fp16 (m, s) pairs per channel (512 B), or
 // MXFP4 -- E2M1 elements sharing an E8M0 exponent per 32 channels (144 B).
-constexpr int kMetaFp16 = 0, kMetaMx = 1;
-constexpr int kMetaFp16Bytes = 512, kMetaMxBytes = 144;
+// key metadata formats: fp16 (m, s) per window channel; MXFP4 blocks of them; the
+// TurboQuant key codec (one fp16 scale per token, no window statistics)
+constexpr int kMetaFp16 = 0, kMetaMx = 1, kMetaTurbo = 2;
+constexpr int kMetaFp16Bytes = 512, kMetaMxBytes = 144, kMetaTurboBytes = 64;
 
-__host__ __device__ constexpr int meta_bytes_of(int key_meta) { return key_meta == kMetaMx ? kMetaMxBytes : kMetaFp16Bytes; }
+__host__ __device__ constexpr int meta_bytes_of(int key_meta) {
+  return key_meta == kMetaMx ? kMetaMxBytes : key_meta == kMetaTurbo ? kMetaTurboBytes : kMetaFp16Bytes;
+}
 
 struct RecordLayout {
   int k_off, meta_off, v_off, sigma_off, bytes;

@@ -194,7 +194,8 @@ __device__ void decode_generic_t(const DecodeParams& p, GenSmem& g, const float*
     for (int s = 0; s < kGenStages && s < nwin; ++s) gen_issue(p, g, s, rec_base, lay.bytes, b, kvh, w0 + s, wait_win, wait_val);
   }
   const int LK = 1 << p.key_bits, LV = 1 << p.value_bits;
-  if (tid < LK) g.dk[tid] = p.key_cb[tid] - p.key_cb[0];
+  const bool tqfmt = p.key_meta == kMetaTurbo;  // TurboQuant keys: k'_tc = ksigma_t c_j
+  if (tid < LK) g.dk[tid] = tqfmt ? p.key_cb[tid] : p.key_cb[tid] - p.key_cb[0];
   if (tid >= 32 && tid - 32 < LV) g.dv[tid - 32] = p.val_cb[tid - 32];
 #pragma unroll
   for (int h = 0; h < kMaxGroup; ++h) g.qT[tid][h] = qflat[qpos(h, tid)];
@@ -254,7 +255,7 @@ __device__ void decode_generic_t(const DecodeParams& p, GenSmem& g, const float*
       for (int j = 0; j < 32; ++j) {
         const int c = 4 * j + sq;
         const uint32_t code = (row[(4 * j) / kcpw] >> (KB * (c % kcpw))) & kmask;
-        const float2 ms = mxfmt ? g.mxm[c] : __half22float2(meta[c]);
+        const float2 ms = mxfmt ? g.mxm[c] : tqfmt ? make_float2(0.0f, 1.0f) : __half22float2(meta[c]);
         const float kv = fmaf(ms.y, g.dk[code], ms.x);
         const float4 qa = *reinterpret_cast<const float4*>(&g.qT[c][0]);
         const float4 qb = *reinterpret_cast<const float4*>(&g.qT[c][4]);
@@ -268,10 +269,12 @@ __device__ void decode_generic_t(const DecodeParams& p, GenSmem& g, const float*
         sc[7] = fmaf(qb.w, kv, sc[7]);
       }
     }
+    const float ksg = tqfmt ? __half2float(reinterpret_cast<const __half*>(rec + lay.meta_off)[st]) : 1.0f;
 #pragma unroll
     for (int h = 0; h < kMaxGroup; ++h) {
       sc[h] += __shfl_xor_sync(0xffffffffu, sc[h], 1);
       sc[h] += __shfl_xor_sync(0xffffffffu, sc[h], 2);
+      sc[h] *= ksg;
       if (wi * kWindow + st >= T || h >= G) sc[h] = -INFINITY;
     }
     // ---- window max per head: lanes of a warp (8 tokens), then the 4 warps

@@ -117,6 +117,7 @@ struct __align__(16) DecodeSmem {
   uint32_t tmem_base;                             // per-warp body: TMEM columns of the parked accumulators
   alignas(16) uint32_t mxpairs[kWarps][kHeadDim]; // MXFP4 caches: a warp's window metadata as fp16 (m, s) pairs
                                                   // (read as 16-byte vectors)
+  float qoff[kMaxGroup];                          // TurboQuant keys: c_0 sum_c q'_c per head
   uint32_t bad_heads;                             // bit h: head h's partial is not finite (written empty)
   int abort;                                      // cooperative body: a step flag never arrived
   int wabort[kWarps];                             // per-warp body: a step flag of warp w never arrived
@@ -350,6 +351,7 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
     const uint32_t* kw = reinterpret_cast<const uint32_t*>(stg);
     using L = Rec22<kMeta>;
     const __half2* meta = window_meta_pairs<kMeta>(sm, stg, warp, lane);
+    const __half* ksig = reinterpret_cast<const __half*>(stg + L::meta);  // TurboQuant keys: per-token scales
     const uint32_t* vw = reinterpret_cast<const uint32_t*>(stg + L::v);
     const __half* sig = reinterpret_cast<const __half*>(stg + L::sigma);
     const uint8_t* mods = stg + L::bytes;
@@ -357,8 +359,11 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
     // ---- per-window: fp16 scale pairs for the A operand, offset sum_c q'_c m_gc
     // lane (g, t) covers channels 32t .. 32t+31 (k-slot pairs (c, c+8))
     uint32_t sp[8][2];
-    float off;
-    {
+    float off = 0.0f;
+    if constexpr (kMeta == kMetaTurbo) {
+#pragma unroll
+      for (int kc = 0; kc < 8; ++kc) sp[kc][0] = sp[kc][1] = 0u;  // no window scales
+    } else {
       const float* qrow = &sm.q[g][32 * t];
       const int qsw = (4 * (g & 1) + t) & 7;
       const uint4* mv4 = reinterpret_cast<const uint4*>(meta + 32 * t);
@@ -388,8 +393,9 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
       off += __shfl_xor_sync(0xffffffffu, off, 1);
       off += __shfl_xor_sync(0xffffffffu, off, 2);
     }
-    const float off0 = __shfl_sync(0xffffffffu, off, 8 * t);      // head 2t
-    const float off1 = __shfl_sync(0xffffffffu, off, 8 * t + 4);  // head 2t + 1
+    // TurboQuant keys: the window-independent c_0 sum_c q'_c of heads 2t, 2t+1
+    const float off0 = kMeta == kMetaTurbo ? sm.qoff[2 * t] : __shfl_sync(0xffffffffu, off, 8 * t);
+    const float off1 = kMeta == kMetaTurbo ? sm.qoff[2 * t + 1] : __shfl_sync(0xffffffffu, off, 8 * t + 4);
 
     // ---- scores for the two 16-token tiles, issued interleaved per chunk (4
     // independent accumulator chains)
@@ -424,10 +430,19 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
             r[2] = kA[h].y >> 1;
             r[3] = kB[h].y >> 1;
           }
-          const uint32_t a0[4] = {hmul2_u32(s0, r[0] & kPlane0), hmul2_u32(s0, r[1] & kPlane0),
-                                  hmul2_u32(s1, r[2] & kPlane0), hmul2_u32(s1, r[3] & kPlane0)};
-          const uint32_t a1[4] = {hmul2_u32(s0, r[0] & kPlane1), hmul2_u32(s0, r[1] & kPlane1),
-                                  hmul2_u32(s1, r[2] & kPlane1), hmul2_u32(s1, r[3] & kPlane1)};
+          uint32_t a0[4], a1[4];
+          if constexpr (kMeta == kMetaTurbo) {  // the code planes alone (the scale is per token)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              a0[k] = r[k] & kPlane0;
+              a1[k] = r[k] & kPlane1;
+            }
+          } else {
+            a0[0] = hmul2_u32(s0, r[0] & kPlane0), a0[1] = hmul2_u32(s0, r[1] & kPlane0);
+            a0[2] = hmul2_u32(s1, r[2] & kPlane0), a0[3] = hmul2_u32(s1, r[3] & kPlane0);
+            a1[0] = hmul2_u32(s0, r[0] & kPlane1), a1[1] = hmul2_u32(s0, r[1] & kPlane1);
+            a1[2] = hmul2_u32(s1, r[2] & kPlane1), a1[3] = hmul2_u32(s1, r[3] & kPlane1);
+          }
           mma_f16_16816(d0[h], a0, bp0.x, bp0.y);
           mma_f16_16816(d1[h], a1, bp1.x, bp1.y);
           mma_f16_16816(d0[h], a0, bp0.z, bp0.w);
@@ -437,10 +452,13 @@ __device__ void decode_mma(const DecodeParams& p, DecodeSmem& sm, int b, int kvh
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int posA = wi * kWindow + tokA[h], posB = wi * kWindow + tokB[h];
-        sc[h][0] = posA < T ? fmaf(d0[h][0] + d1[h][0], escale, off0) : -INFINITY;
-        sc[h][1] = posA < T ? fmaf(d0[h][1] + d1[h][1], escale, off1) : -INFINITY;
-        sc[h][2] = posB < T ? fmaf(d0[h][2] + d1[h][2], escale, off0) : -INFINITY;
-        sc[h][3] = posB < T ? fmaf(d0[h][3] + d1[h][3], escale, off1) : -INFINITY;
+        // TurboQuant keys: k'_tc = ksigma_t c_j, so the score is ksigma_t times the sum
+        const float kgA = kMeta == kMetaTurbo ? __half2float(ksig[tokA[h]]) : 1.0f;
+        const float kgB = kMeta == kMetaTurbo ? __half2float(ksig[tokB[h]]) : 1.0f;
+        sc[h][0] = posA < T ? kgA * fmaf(d0[h][0] + d1[h][0], escale, off0) : -INFINITY;
+        sc[h][1] = posA < T ? kgA * fmaf(d0[h][1] + d1[h][1], escale, off1) : -INFINITY;
+        sc[h][2] = posB < T ? kgB * fmaf(d0[h][2] + d1[h][2], escale, off0) : -INFINITY;
+        sc[h][3] = posB < T ? kgB * fmaf(d0[h][3] + d1[h][3], escale, off1) : -INFINITY;
       }
     }
 
@@ -838,11 +856,15 @@ __device__ void decode_coop(const DecodeParams& p, DecodeSmem& sm, int b, int kv
     if (have && wok) {
       const uint32_t* kw = reinterpret_cast<const uint32_t*>(rec);
       const __half2* meta = window_meta_pairs<kMeta>(sm, rec, warp, lane);
+      const __half* ksig = reinterpret_cast<const __half*>(rec + L::meta);  // TurboQuant keys: per-token scales
       // fp16 scale pairs of the A operand and the offset sum_c q'_c m_gc; lane
       // (g, t) covers channels 32t .. 32t+31 (k-slot pairs (c, c+8))
       uint32_t sp[8][2];
-      float off;
-      {
+      float off = 0.0f;
+      if constexpr (kMeta == kMetaTurbo) {
+#pragma unroll
+        for (int kc = 0; kc < 8; ++kc) sp[kc][0] = sp[kc][1] = 0u;  // no window scales
+      } else {
         const float* qrow = &sm.q[g][32 * t];
         const int qsw = (4 * (g & 1) + t) & 7;
         const uint4* mv4 = reinterpret_cast<const uint4*>(meta + 32 * t);
@@ -872,8 +894,9 @@ __device__ void decode_coop(const DecodeParams& p, DecodeSmem& sm, int b, int kv
         off += __shfl_xor_sync(0xffffffffu, off, 1);
         off += __shfl_xor_sync(0xffffffffu, off, 2);
       }
-      const float off0 = __shfl_sync(0xffffffffu, off, 8 * t);      // head 2t
-      const float off1 = __shfl_sync(0xffffffffu, off, 8 * t + 4);  // head 2t + 1
+      // TurboQuant keys: the window-independent c_0 sum_c q'_c of heads 2t, 2t+1
+      const float off0 = kMeta == kMetaTurbo ? sm.qoff[2 * t] : __shfl_sync(0xffffffffu, off, 8 * t);
+      const float off1 = kMeta == kMetaTurbo ? sm.qoff[2 * t + 1] : __shfl_sync(0xffffffffu, off, 8 * t + 4);
       uint2 kA[2], kB[2];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -900,10 +923,19 @@ __device__ void decode_coop(const DecodeParams& p, DecodeSmem& sm, int b, int kv
             r[2] = kA[h].y >> 1;
             r[3] = kB[h].y >> 1;
           }
-          const uint32_t a0[4] = {hmul2_u32(s0, r[0] & kPlane0), hmul2_u32(s0, r[1] & kPlane0),
-                                  hmul2_u32(s1, r[2] & kPlane0), hmul2_u32(s1, r[3] & kPlane0)};
-          const uint32_t a1[4] = {hmul2_u32(s0, r[0] & kPlane1), hmul2_u32(s0, r[1] & kPlane1),
-                                  hmul2_u32(s1, r[2] & kPlane1), hmul2_u32(s1, r[3] & kPlane1)};
+          uint32_t a0[4], a1[4];
+          if constexpr (kMeta == kMetaTurbo) {  // the code planes alone (the scale is per token)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              a0[k] = r[k] & kPlane0;
+              a1[k] = r[k] & kPlane1;
+            }
+          } else {
+            a0[0] = hmul2_u32(s0, r[0] & kPlane0), a0[1] = hmul2_u32(s0, r[1] & kPlane0);
+            a0[2] = hmul2_u32(s1, r[2] & kPlane0), a0[3] = hmul2_u32(s1, r[3] & kPlane0);
+            a1[0] = hmul2_u32(s0, r[0] & kPlane1), a1[1] = hmul2_u32(s0, r[1] & kPlane1);
+            a1[2] = hmul2_u32(s1, r[2] & kPlane1), a1[3] = hmul2_u32(s1, r[3] & kPlane1);
+          }
           mma_f16_16816(d0[h], a0, bp0.x, bp0.y);
           mma_f16_16816(d1[h], a1, bp1.x, bp1.y);
           mma_f16_16816(d0[h], a0, bp0.z, bp0.w);
@@ -913,10 +945,13 @@ __device__ void decode_coop(const DecodeParams& p, DecodeSmem& sm, int b, int kv
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int posA = wi * kWindow + tokA[h], posB = wi * kWindow + tokB[h];
-        sc[h][0] = posA < T ? fmaf(d0[h][0] + d1[h][0], escale, off0) : -INFINITY;
-        sc[h][1] = posA < T ? fmaf(d0[h][1] + d1[h][1], escale, off1) : -INFINITY;
-        sc[h][2] = posB < T ? fmaf(d0[h][2] + d1[h][2], escale, off0) : -INFINITY;
-        sc[h][3] = posB < T ? fmaf(d0[h][3] + d1[h][3], escale, off1) : -INFINITY;
+        // TurboQuant keys: k'_tc = ksigma_t c_j, so the score is ksigma_t times the sum
+        const float kgA = kMeta == kMetaTurbo ? __half2float(ksig[tokA[h]]) : 1.0f;
+        const float kgB = kMeta == kMetaTurbo ? __half2float(ksig[tokB[h]]) : 1.0f;
+        sc[h][0] = posA < T ? kgA * fmaf(d0[h][0] + d1[h][0], escale, off0) : -INFINITY;
+        sc[h][1] = posA < T ? kgA * fmaf(d0[h][1] + d1[h][1], escale, off1) : -INFINITY;
+        sc[h][2] = posB < T ? kgB * fmaf(d0[h][2] + d1[h][2], escale, off0) : -INFINITY;
+        sc[h][3] = posB < T ? kgB * fmaf(d0[h][3] + d1[h][3], escale, off1) : -INFINITY;
       }
     }
     {
@@ -1184,6 +1219,19 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, DecodeSmem& sm
     for (int o = 16; o > 0; o >>= 1) qm = fmaxf(qm, __shfl_xor_sync(0xffffffffu, qm, o));
     if ((threadIdx.x & 31) == 0) sm.lw[threadIdx.x >> 5][0] = qm;
   }
+  if constexpr (kMeta == kMetaTurbo) {
+    // c_0 sum_c q'_c per head: the codebook's c_0 term of every score (warp w sums
+    // the rows of heads w and w + 4, in any channel order)
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    for (int g = w; g < kMaxGroup; g += kWarps) {
+      float x = 0.0f;
+#pragma unroll
+      for (int c = l; c < kHeadDim; c += 32) x += sm.q[g][c];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+      if (l == 0) sm.qoff[g] = p.key_cb[0] * x;
+    }
+  }
   __syncthreads();
   float escale = 1.0f;
   if (fast) {
@@ -1294,7 +1342,7 @@ cudaError_t prefer_shared_carveout(Kernel kernel, std::atomic<uint64_t>& done) {
   return e;
 }
 
-std::atomic<uint64_t> g_carveout[2][kNumBodies][2];  // [decode, step][body][key metadata format]
+std::atomic<uint64_t> g_carveout[2][kNumBodies][3];  // [decode, step][body][key metadata format]
 
 template <int kBody, int kMeta>
 cudaError_t prepare_body() {
@@ -1307,6 +1355,8 @@ cudaError_t prepare_body() {
 cudaError_t prepare_kernels(int body, int meta) {
   if (body == kBodyGeneric) return prepare_body<kBodyGeneric, kMetaFp16>();
   if (meta == kMetaMx) return body == kBodyWarp ? prepare_body<kBodyWarp, kMetaMx>() : prepare_body<kBodyCoop, kMetaMx>();
+  if (meta == kMetaTurbo)
+    return body == kBodyWarp ? prepare_body<kBodyWarp, kMetaTurbo>() : prepare_body<kBodyCoop, kMetaTurbo>();
   return body == kBodyWarp ? prepare_body<kBodyWarp, kMetaFp16>() : prepare_body<kBodyCoop, kMetaFp16>();
 }
 
@@ -1323,13 +1373,16 @@ cudaError_t body_attributes_of(cudaFuncAttributes* a) {
   return cudaSuccess;
 }
 
-// Attributes of a body, over both metadata formats (the residency of the larger).
+// Attributes of a body, over every key metadata format (the residency of the largest).
 template <int kBody>
 cudaError_t body_attributes(cudaFuncAttributes* a) {
   cudaError_t e = body_attributes_of<kBody, kMetaFp16>(a);
   if (e != cudaSuccess || kBody == kBodyGeneric) return e;
   cudaFuncAttributes a2;
   if ((e = body_attributes_of<kBody, kMetaMx>(&a2)) != cudaSuccess) return e;
+  if (a2.numRegs > a->numRegs) a->numRegs = a2.numRegs;
+  if (a2.sharedSizeBytes > a->sharedSizeBytes) a->sharedSizeBytes = a2.sharedSizeBytes;
+  if ((e = body_attributes_of<kBody, kMetaTurbo>(&a2)) != cudaSuccess) return e;
   if (a2.numRegs > a->numRegs) a->numRegs = a2.numRegs;
   if (a2.sharedSizeBytes > a->sharedSizeBytes) a->sharedSizeBytes = a2.sharedSizeBytes;
   return cudaSuccess;
@@ -1361,7 +1414,9 @@ int decode_ctas_per_sm(int body) {
   const cudaError_t ea = body == kBodyWarp ? body_attributes<kBodyWarp>(&a)
                        : body == kBodyCoop ? body_attributes<kBodyCoop>(&a)
                                            : body_attributes<kBodyGeneric>(&a);
-  if (prepare_kernels(body, kMetaFp16) != cudaSuccess || (body != kBodyGeneric && prepare_kernels(body, kMetaMx) != cudaSuccess) ||
+  if (prepare_kernels(body, kMetaFp16) != cudaSuccess ||
+      (body != kBodyGeneric && (prepare_kernels(body, kMetaMx) != cudaSuccess ||
+                                prepare_kernels(body, kMetaTurbo) != cudaSuccess)) ||
       ea != cudaSuccess ||
       cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
@@ -1387,6 +1442,9 @@ cudaError_t launch_decode_step(const DecodeParams& p, const WriteParams& w, cuda
   if (meta == kMetaMx)
     return body == kBodyWarp ? launch_pdl(decode_step_kernel<kBodyWarp, kMetaMx>, grid, block, 0, stream, p, w)
                              : launch_pdl(decode_step_kernel<kBodyCoop, kMetaMx>, grid, block, 0, stream, p, w);
+  if (meta == kMetaTurbo)
+    return body == kBodyWarp ? launch_pdl(decode_step_kernel<kBodyWarp, kMetaTurbo>, grid, block, 0, stream, p, w)
+                             : launch_pdl(decode_step_kernel<kBodyCoop, kMetaTurbo>, grid, block, 0, stream, p, w);
   return body == kBodyWarp ? launch_pdl(decode_step_kernel<kBodyWarp, kMetaFp16>, grid, block, 0, stream, p, w)
                            : launch_pdl(decode_step_kernel<kBodyCoop, kMetaFp16>, grid, block, 0, stream, p, w);
 }
@@ -1402,6 +1460,9 @@ cudaError_t launch_decode(const DecodeParams& p, int batch, cudaStream_t stream)
   if (meta == kMetaMx)
     return body == kBodyWarp ? launch_pdl(decode_split_k_kernel<kBodyWarp, kMetaMx>, grid, block, 0, stream, p)
                              : launch_pdl(decode_split_k_kernel<kBodyCoop, kMetaMx>, grid, block, 0, stream, p);
+  if (meta == kMetaTurbo)
+    return body == kBodyWarp ? launch_pdl(decode_split_k_kernel<kBodyWarp, kMetaTurbo>, grid, block, 0, stream, p)
+                             : launch_pdl(decode_split_k_kernel<kBodyCoop, kMetaTurbo>, grid, block, 0, stream, p);
   return body == kBodyWarp ? launch_pdl(decode_split_k_kernel<kBodyWarp, kMetaFp16>, grid, block, 0, stream, p)
                            : launch_pdl(decode_split_k_kernel<kBodyCoop, kMetaFp16>, grid, block, 0, stream, p);
 }

@@ -16,7 +16,7 @@ struct WriteParams {
   const float* key_signs;
   const float* value_rot;
   int key_bits, value_bits, num_kv_heads;
-  int key_meta;  // kMetaFp16 or kMetaMx
+  int key_meta;  // kMetaFp16, kMetaMx or kMetaTurbo
   uint8_t* records;
   __half* key_tail;
   uint8_t* modality;
@@ -40,7 +40,7 @@ struct DecodeParams {
   const float* key_signs;
   const float* value_rot;  // only prefetched into L2 (for the combine)
   int key_bits, value_bits, num_kv_heads, group;
-  int key_meta;  // kMetaFp16 or kMetaMx
+  int key_meta;  // kMetaFp16, kMetaMx or kMetaTurbo
   const uint8_t* records;
   const uint8_t* modality;
   const int32_t* seq_lens;

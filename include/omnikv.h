@@ -44,15 +44,19 @@
  *           2, 3, 4, 6) of the 128 minima, two per byte (even channel in the low
  *           nibble), then of the 128 scales; then the E8M0 exponents (e + 127) of
  *           the 4 blocks of 32 channels of the minima, then of the scales; 8 zero
- *           bytes. m_gc = E2M1(m code) 2^e_m, s_gc = E2M1(s code) 2^e_s.
+ *           bytes. m_gc = E2M1(m code) 2^e_m, s_gc = E2M1(s code) 2^e_s;
+ *           OMNIKV_META_TURBO (64 B; the TurboQuant key codec the pages compare
+ *           against, pchao.org related work / paperpeel.com section 2.2): [32]
+ *           fp16 key scales, one per token (0 for padded slots).
  *   V codes [32 / cpw][128] u32         channel-major: token t, channel c is in
  *           word (t / cpw, c) at bits [bits * (t % cpw), +bits)
  *   sigma   [32] fp16 (per-token value scale)
  * Size (omnikv_record_bytes_meta): 2624 bytes for K2/V2 and 4672 for K4/V4 with
- * fp16 metadata; 2256 and 4304 with MXFP4 metadata.
+ * fp16 metadata; 2256 and 4304 with MXFP4 metadata; 2176 and 4224 with TurboQuant
+ * keys.
  * Dequantised rotated-space cache: k'_tc = m_gc + s_gc (c_j - c_0) for key code
- * j; v'_tc = sigma_t c_j for value code j. Padded slots of a partial window hold
- * code 0 and sigma 0.
+ * j (window metadata) or k'_tc = ksigma_t c_j (TurboQuant keys); v'_tc = sigma_t
+ * c_j for value code j. Padded slots of a partial window hold code 0 and sigma 0.
  */
 #ifndef OMNIKV_H_
 #define OMNIKV_H_
@@ -76,6 +80,7 @@ extern "C" {
 #define OMNIKV_NUM_MODALITIES 3 /* 0 = text (L), 1 = audio (A), 2 = video (V) */
 #define OMNIKV_META_FP16 0      /* key window metadata: fp16 minimum and scale per channel */
 #define OMNIKV_META_MXFP4 1     /* key window metadata: MXFP4 (E2M1 values, one E8M0 exponent per 32 channels) */
+#define OMNIKV_META_TURBO 2     /* TurboQuant key codec: one fp16 scale per token, no window statistics */
 
 typedef enum {
   OMNIKV_OK = 0,
@@ -118,7 +123,12 @@ typedef struct {
                                    is the smallest e in [-127, 127] with max |x| <= 6 2^e (-127 for a zero
                                    block); the minimum rounds to the nearest E2M1 value times 2^e (ties to the
                                    even code), then the scale it needs, fp32((max - m^) / (c_last - c_0)) (0 if
-                                   negative), on its block's grid the same way. Codes as with fp16 metadata. */
+                                   negative), on its block's grid the same way. Codes as with fp16 metadata.
+                                   OMNIKV_META_TURBO (2): the TurboQuant key codec, per token: ksigma =
+                                   fp16(sqrt(sum_c k_c^2 / 128)) of the unrotated fp16 key (the value scale's
+                                   rule) and code = #{j : k'_c / ksigma > t_j} (0 where ksigma == 0); the
+                                   values are unchanged (TurboQuant proper passes the transposed key rotation
+                                   R^T as every modality's value basis: one shared rotation). */
 } omnikv_config;
 
 /* One layer's cache for a batch. Device memory is owned by the caller and must be
@@ -144,7 +154,8 @@ typedef struct {
 OMNIKV_API size_t omnikv_record_bytes(int32_t key_bits, int32_t value_bits);
 
 /* Bytes of one window record in a key metadata format (OMNIKV_META_FP16: as omnikv_record_bytes;
- * OMNIKV_META_MXFP4: 2256 for K2/V2, 4304 for K4/V4); 0 for unsupported arguments. The cache's
+ * OMNIKV_META_MXFP4: 2256 for K2/V2, 4304 for K4/V4; OMNIKV_META_TURBO: 2176 for K2/V2, 4224 for
+ * K4/V4); 0 for unsupported arguments. The cache's
  * records array holds [batch][num_kv_heads][cap_tokens / 32] records of this size. */
 OMNIKV_API size_t omnikv_record_bytes_meta(int32_t key_bits, int32_t value_bits, int32_t key_meta_format);
 

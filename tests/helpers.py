@@ -50,7 +50,7 @@ def upload_oracle_cache(oc: codec.OracleCache, device):
     from bit_kv_cache_pack_b200 import KVCache
     B, H, _, _ = oc.records.shape
     c = KVCache(B, H, oc.cap_tokens, oc.key_bits, oc.value_bits, device,
-                key_meta_format=1 if oc.meta_format == "mx" else 0)
+                key_meta_format={"fp16": 0, "mx": 1, "turbo": 2}[oc.meta_format])
     c.records.copy_(torch.from_numpy(oc.records))
     c.key_tail.copy_(torch.from_numpy(oc.key_tail))
     c.modality.copy_(torch.from_numpy(oc.modality))

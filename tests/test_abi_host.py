@@ -48,7 +48,9 @@ def test_sizes_and_version():
     assert _abi.omnikv_record_bytes_meta(2, 2, _abi.OMNIKV_META_FP16) == 2624
     assert _abi.omnikv_record_bytes_meta(2, 2, _abi.OMNIKV_META_MXFP4) == 2256   # 1024 + 144 + 1024 + 64
     assert _abi.omnikv_record_bytes_meta(4, 4, _abi.OMNIKV_META_MXFP4) == 4304
-    assert _abi.omnikv_record_bytes_meta(2, 2, 2) == 0
+    assert _abi.omnikv_record_bytes_meta(2, 2, _abi.OMNIKV_META_TURBO) == 2176   # 1024 + 64 + 1024 + 64
+    assert _abi.omnikv_record_bytes_meta(4, 4, _abi.OMNIKV_META_TURBO) == 4224
+    assert _abi.omnikv_record_bytes_meta(2, 2, 3) == 0
     assert _abi.omnikv_partials_bytes(2, 16, 5) == 2 * 16 * 5 * 1552
     assert _abi.omnikv_partials_bytes(0, 16, 5) == 0
     assert _abi.status_string(_abi.OMNIKV_ERR_CAPACITY) == "cache capacity exceeded"
@@ -86,7 +88,7 @@ def _write_status(cfg, cache, n_new=1, k=FAKE, v=FAKE, mod=FAKE):
     (dict(num_kv_heads=0), _abi.OMNIKV_ERR_INVALID_ARG),
     (dict(key_codebook=None), _abi.OMNIKV_ERR_INVALID_ARG),
     (dict(value_rot=FAKE + 4), _abi.OMNIKV_ERR_INVALID_ARG),
-    (dict(key_meta_format=2), _abi.OMNIKV_ERR_UNSUPPORTED),
+    (dict(key_meta_format=3), _abi.OMNIKV_ERR_UNSUPPORTED),
 ])
 def test_config_rejected(kw, want):
     assert _write_status(_cfg(**kw), _cache()) == want

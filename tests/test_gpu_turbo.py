@@ -1,0 +1,178 @@
+"""The TurboQuant key codec on the GPU (the baseline the pages compare against:
+pchao.org related work; paperpeel.com section 2.2 "Temporal key drift"): one
+sign-flip Hadamard rotation and one fp16 scale per token, no window statistics
+(oracle/codec.py quantize_key_window_turbo).
+
+Cache write: key codes and the 32 per-token key scales of every window bit-exact,
+value scales bit-exact, value codes as for the window formats (at a threshold
+within the rotation's error bound); 2,176-byte records for K2/V2. Decode: the GPU's
+decode + combine over turbo caches against the oracle's fp64 attention over the
+same dequantised cache, on both 2-bit decode bodies, the 4-bit build and the fused
+decode step. The codec-error comparison (paperpeel.com section 3.3, Table 3:
+key reconstruction MSE, attention KL divergence, attention-output MSE) computed
+from GPU-written caches of the three codecs equals the oracle's.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import codec
+from oracle.attention import decode_dense, dequantize, key_rotation_matrix
+from oracle.codec_error import attention_metrics
+from synth.workloads import WORKLOADS, codebook, decode_inputs, key_drift, prefill_inputs, seq_lengths, with_bits
+
+from helpers import check_decode, compare_records, make_layer, seeded_randn, upload_oracle_cache
+
+pytestmark = pytest.mark.gpu
+
+TURBO = 2
+
+
+def _write_both(m, consts, ocfg, gc, oc, k, v, mod):
+    n = k.shape[2]
+    m.omnikv_write_cache(consts.struct, gc.struct, k.contiguous(), v.contiguous(), mod.contiguous(), n)
+    codec.write_cache(ocfg, oc, k.cpu().numpy(), v.cpu().numpy(), mod.cpu().numpy())
+    torch.cuda.synchronize()
+
+
+def _check(ocfg, oc, gc, v_all, mod_all):
+    grec = gc.records.cpu().numpy()
+    assert grec.shape[-1] == oc.records.shape[-1]
+    assert np.array_equal(gc.seq_lens.cpu().numpy(), oc.seq_lens)
+    assert int(gc.error_word.item()) == 0
+    mism = 0
+    for b in range(grec.shape[0]):
+        T = int(oc.seq_lens[b])
+        for h in range(grec.shape[1]):
+            mism += compare_records(ocfg, oc, grec, b, h, range((T + 31) // 32), v_all[b, h], mod_all[b])
+    return mism
+
+
+def _decode(m, consts, cache, q, S, Hq):
+    S = S or m.omnikv_default_splits(consts.struct, cache.struct)
+    part = m.partials_tensor(q.shape[0], Hq, S, q.device)
+    out = torch.empty(q.shape[0], Hq, 128, device=q.device)
+    m.omnikv_decode_attention(consts.struct, cache.struct, q, part, S)
+    m.omnikv_combine(consts.struct, cache.struct, part, S, out)
+    torch.cuda.synchronize()
+    assert int(cache.error_word.item()) == 0
+    return out.cpu().numpy(), S
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_turbo_chunked_writes_bit_exact(cuda_device, bits):
+    import bit_kv_cache_pack_b200 as m
+    spec = with_bits(WORKLOADS["tiny"], bits, bits)
+    seed = 61
+    params, consts, ocfg = make_layer(spec, seed, 0, cuda_device, per_head=True, key_meta_format=TURBO)
+    assert m.omnikv_record_bytes_meta(bits, bits, TURBO) == (2176 if bits == 2 else 4224)
+    L = np.array([300], np.int32)
+    drift = key_drift(spec, seed, 0, 16, cuda_device)
+    k, v, mod = prefill_inputs(spec, seed, 0, params, drift, L, cuda_device)
+    gc = m.KVCache(1, 2, 320, bits, bits, cuda_device, key_meta_format=TURBO)
+    oc = codec.OracleCache(1, 2, 320, bits, bits, meta_format="turbo")
+    cuts = [0, 1, 3, 34, 67, 96, 97, 160, 191, 255, 300]
+    for a, b_ in zip(cuts[:-1], cuts[1:]):
+        _write_both(m, consts, ocfg, gc, oc, k[:, :, a:b_], v[:, :, a:b_], mod[:, a:b_])
+        _check(ocfg, oc, gc, v.cpu().numpy(), mod.cpu().numpy())
+    q = seeded_randn((1, 16, 128), cuda_device, 17).half()
+    ref = decode_dense(ocfg, oc, q.cpu().numpy())
+    for S in (1, 3, 0):
+        out, S = _decode(m, consts, upload_oracle_cache(oc, cuda_device), q, S, 16)
+        check_decode(out, ref, "turbo bits=%d S=%d" % (bits, S))
+
+
+def test_turbo_prefill_append_decode(cuda_device):
+    """The tiny workload's 2,048-token prefill and one appended token with turbo
+    keys; decode over the oracle's cache and over the GPU-written one with the
+    default split count (cooperative body) and one split (per-warp body), then the
+    fused decode step."""
+    import bit_kv_cache_pack_b200 as m
+    spec, seed = WORKLOADS["tiny"], 63
+    params, consts, ocfg = make_layer(spec, seed, 0, cuda_device, key_meta_format=TURBO)
+    L = seq_lengths(spec, seed)
+    cap = 2048 + 64
+    drift = key_drift(spec, seed, 0, cap // 32, cuda_device)
+    k, v, mod = prefill_inputs(spec, seed, 0, params, drift, L, cuda_device)
+    gc = m.KVCache(1, 2, cap, 2, 2, cuda_device, key_meta_format=TURBO)
+    oc = codec.OracleCache(1, 2, cap, 2, 2, meta_format="turbo")
+    _write_both(m, consts, ocfg, gc, oc, k, v, mod)
+    q, kn, vn, mn = decode_inputs(spec, seed, 0, 0, params, drift, L, cuda_device)
+    _write_both(m, consts, ocfg, gc, oc, kn, vn, mn)
+    v_all = torch.cat([v, vn], dim=2).cpu().numpy()
+    mod_all = torch.cat([mod, mn], dim=1).cpu().numpy()
+    mism = _check(ocfg, oc, gc, v_all, mod_all)
+    assert mism <= 1e-4 * v_all.size
+    ref = decode_dense(ocfg, oc, q.cpu().numpy())
+    for cache, what in ((upload_oracle_cache(oc, cuda_device), "oracle cache"), (gc, "gpu cache")):
+        for S in (0, 1):
+            out, S = _decode(m, consts, cache, q, S, 16)
+            check_decode(out, ref, "turbo %s S=%d" % (what, S))
+    q2, kn2, vn2, mn2 = decode_inputs(spec, seed, 0, 1, params, drift, L + 1, cuda_device)
+    S, fused = m.omnikv_step_splits(consts.struct, gc.struct, 0)
+    part = m.partials_tensor(1, 16, S, cuda_device)
+    out = torch.empty(1, 16, 128, device=cuda_device)
+    m.omnikv_decode_step(consts.struct, gc.struct, q2, kn2, vn2, mn2, part, 0, out)
+    codec.write_cache(ocfg, oc, kn2.cpu().numpy(), vn2.cpu().numpy(), mn2.cpu().numpy())
+    torch.cuda.synchronize()
+    assert int(gc.error_word.item()) == 0
+    check_decode(out.cpu().numpy(), decode_dense(ocfg, oc, q2.cpu().numpy()), "turbo decode step (fused=%d)" % fused)
+
+
+def test_codec_error_report_from_gpu_caches(cuda_device):
+    """One 2,048-token sequence of the omni30b shape (drift 1.0, 8 outlier channels
+    x 16), K2V2: the three codecs written by the GPU, dequantised, and measured
+    against the raw fp16 keys and values; TurboQuant proper uses the key rotation
+    for the values too (value basis R^T for every modality). The key metrics are
+    those of the oracle-written caches exactly (bit-exact key records); the output
+    MSE within the value codes' threshold effects."""
+    import bit_kv_cache_pack_b200 as m
+    from bit_kv_cache_pack_b200 import LayerConstants
+    import dataclasses
+    from synth.workloads import layer_params
+    spec = dataclasses.replace(WORKLOADS["omni30b-b8"], batch=1)
+    seed, T = 3, 2048
+    params = layer_params(spec, seed, 0)
+    H, Hq = spec.num_kv_heads, spec.num_q_heads
+    signs = params["key_signs"].numpy()
+    R = key_rotation_matrix(signs)
+    bases = {"omni-fp16": params["value_rot"].numpy(), "omni-mx": params["value_rot"].numpy(),
+             "turbo": np.broadcast_to(R.T.astype(np.float32), (H, 3, 128, 128)).copy()}
+    fmt = {"omni-fp16": ("fp16", 0), "omni-mx": ("mx", 1), "turbo": ("turbo", 2)}
+    drift = key_drift(spec, seed, 0, T // 32 + 1, cuda_device)
+    k, v, mod = prefill_inputs(spec, seed, 0, params, drift, np.array([T]), cuda_device)
+    q = decode_inputs(spec, seed, 0, 0, params, drift, np.array([T]), cuda_device)[0]
+    kn, vn, modn, qn = k.cpu().numpy(), v.cpu().numpy(), mod.cpu().numpy(), q.cpu().numpy()
+    kb = codebook(2)
+    G = Hq // H
+    report = {}
+    for name, (mf, code) in fmt.items():
+        consts = LayerConstants(kb, kb, signs, bases[name], Hq, cuda_device, key_meta_format=code)
+        ocfg = codec.OracleConfig(kb, kb, signs, bases[name], Hq, H)
+        gc = m.KVCache(1, H, T, 2, 2, cuda_device, key_meta_format=code)
+        m.omnikv_write_cache(consts.struct, gc.struct, k, v, mod, T)
+        torch.cuda.synchronize()
+        assert int(gc.error_word.item()) == 0
+        oc = codec.OracleCache(1, H, T, 2, 2, meta_format=mf)
+        codec.write_cache(ocfg, oc, kn, vn, modn)
+        gpu = codec.OracleCache(1, H, T, 2, 2, meta_format=mf)
+        gpu.records[:] = gc.records.cpu().numpy()
+        gpu.modality[:] = gc.modality.cpu().numpy()
+        gpu.seq_lens[:] = gc.seq_lens.cpu().numpy()
+        res = []
+        for cache in (gpu, oc):
+            per_head = []
+            for h in range(H):
+                kq, vq, md = dequantize(ocfg, cache, 0, h)
+                kh = kq @ R
+                vh = np.stack([bases[name][h, md[t]].astype(np.float64) @ vq[t] for t in range(T)])
+                per_head.append(attention_metrics(qn[0, h * G:(h + 1) * G], kn[0, h], vn[0, h], kh, vh))
+            res.append(tuple(float(np.mean([x[i] for x in per_head])) for i in range(3)))
+        (g_rm, g_kl, g_om), (o_rm, o_kl, o_om) = res
+        assert g_rm == o_rm and g_kl == o_kl, name                    # keys bit-exact
+        assert abs(g_om - o_om) <= 1e-3 * o_om, (name, g_om, o_om)    # value codes at thresholds
+        report[name] = res[0]
+    for name, (rm, kl, om) in report.items():
+        print("%-9s recon_mse %.4e  attn_kl %.4e  out_mse %.4e (GPU-written cache)" % (name, rm, kl, om))
+    # the pages' ordering (Table 3): the window codec reconstructs drifting keys better
+    assert report["omni-fp16"][0] < report["turbo"][0]
