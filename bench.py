@@ -90,9 +90,10 @@ def parse_args():
     ap.add_argument("--impl", default="omnikv", choices=["omnikv", "reference"])
     ap.add_argument("--workload", default="omni30b-b8", choices=sorted(WORKLOADS_KEYS))
     ap.add_argument("--no-graphs", action="store_true")
-    ap.add_argument("--layer", choices=["decode", "write"], default=None,
+    ap.add_argument("--layer", choices=["decode", "write", "calibrate"], default=None,
                     help="time one layer's decode (+ combine) or prefill cache write on --workload instead of "
-                         "the decode step; prints one JSON line per split count")
+                         "the decode step (one JSON line per split count), or the value-basis calibration of one "
+                         "(layer, kv head) from the workload's first sequence")
     ap.add_argument("--bits", type=int, default=0, help="with --layer: 2 or 4 (default: the workload's)")
     ap.add_argument("--meta", default="fp16", choices=sorted(META_FORMATS),
                     help="key metadata format: fp16 (m, s) pairs, mx (MXFP4, the pages' default) or turbo "
@@ -703,6 +704,23 @@ def run_layer(args):
                 ts.append(e0.elapsed_time(e1) * 1e3)
         return float(np.median(ts))
 
+    if args.layer == "calibrate":
+        # one (layer, kv head): the first sequence's values, weights from 4 decode queries
+        k, v, mod = prefill_inputs(dataclasses.replace(spec, batch=1), seed, 0, params, drift, np.array([T]), dev)
+        vals = v[0, 0].contiguous()
+        wts = torch.rand(T, generator=torch.Generator(device=dev).manual_seed(seed), device=dev)
+        ws = torch.empty(m.omnikv_calibrate_workspace_bytes(T) // 8 + 1, dtype=torch.float64, device=dev)
+        bases = torch.empty(3, 128, 128, dtype=torch.float32, device=dev)
+        lam = torch.empty(3, 128, dtype=torch.float64, device=dev)
+        mod0 = mod[0].contiguous()
+        us = timed(lambda: m.omnikv_calibrate_bases(vals, mod0, wts, T, ws, bases, lam))
+        gram_flop = 2.0 * T * 128 * 128  # each token's weighted outer product, fp64
+        fp64_peak = 148 * 64 * 2 * 1.965e9 / 1e12  # SMs x fp64 FMA lanes x 2 flop x max SM clock (TFLOP/s)
+        print(json.dumps({"layer": "calibrate", "workload": spec.name, "tokens": T, "us": round(us, 2),
+                          "gram_gflop": round(gram_flop / 1e9, 3),
+                          "fp64_tflops_over_whole_call": round(gram_flop / (us * 1e-6) / 1e12, 3),
+                          "fp64_peak_tflops_derived": round(fp64_peak, 1)}), flush=True)
+        return
     if args.layer == "write":
         k, v, mod = prefill_inputs(spec, seed, 0, params, drift, np.full(spec.batch, T), dev)
         c = m.KVCache(spec.batch, spec.num_kv_heads, cap, bits, bits, dev, key_meta_format=fmt)

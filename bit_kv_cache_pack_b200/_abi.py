@@ -34,7 +34,8 @@ EXPORTED = (
     "omnikv_status_string", "omnikv_abi_version", "omnikv_decode_static",
     "omnikv_dense_partials_bytes", "omnikv_dense_decode_bf16", "omnikv_decode_step",
     "omnikv_append_decode", "omnikv_combine_step", "omnikv_step_splits", "omnikv_write_cache_rotations",
-    "omnikv_test_decode_pending", "omnikv_record_bytes_meta",
+    "omnikv_test_decode_pending", "omnikv_record_bytes_meta", "omnikv_calibrate_workspace_bytes",
+    "omnikv_calibrate_bases",
 )
 OMNIKV_DECODE_STATIC_SCRATCH_BYTES = 8 << 20
 
@@ -105,6 +106,9 @@ def load() -> ctypes.CDLL:
     lib.omnikv_combine.restype = ctypes.c_int
     lib.omnikv_dense_partials_bytes.argtypes, lib.omnikv_dense_partials_bytes.restype = [I32, I32, I32], SZ
     lib.omnikv_dense_decode_bf16.argtypes = [P, P, P, I32, I32, I32, I32, I32, P, P, I32, P, P, P]
+    lib.omnikv_calibrate_workspace_bytes.argtypes, lib.omnikv_calibrate_workspace_bytes.restype = [I32], SZ
+    lib.omnikv_calibrate_bases.argtypes = [P, P, P, I32, P, SZ, P, P, P]
+    lib.omnikv_calibrate_bases.restype = ctypes.c_int
     lib.omnikv_dense_decode_bf16.restype = ctypes.c_int
     lib.omnikv_decode_step.argtypes = [cfgp, cachep, P, P, P, P, P, I32, P, P]
     lib.omnikv_decode_step.restype = ctypes.c_int
@@ -246,6 +250,19 @@ def omnikv_decode_static(cfg: OmniKVConfig, cache: OmniKVCache, q, out, num_spli
 
 def omnikv_dense_partials_bytes(batch: int, num_q_heads: int, num_splits: int) -> int:
     return int(load().omnikv_dense_partials_bytes(batch, num_q_heads, num_splits))
+
+
+def omnikv_calibrate_workspace_bytes(num_tokens: int) -> int:
+    return int(load().omnikv_calibrate_workspace_bytes(int(num_tokens)))
+
+
+def omnikv_calibrate_bases(values, modality, weights, num_tokens: int, workspace, bases, eigenvalues=None,
+                           stream=None) -> None:
+    """Value bases U_m of one (layer, kv head) from calibration values; see include/omnikv.h."""
+    st = load().omnikv_calibrate_bases(_ptr(values), _ptr(modality), _ptr(weights), int(num_tokens), _ptr(workspace),
+                                       int(workspace.numel() * workspace.element_size()), _ptr(bases),
+                                       _ptr(eigenvalues), _stream(stream))
+    _check(st, "omnikv_calibrate_bases")
 
 
 def omnikv_dense_decode_bf16(k_cache, v_cache, seq_lens, batch: int, num_q_heads: int, num_kv_heads: int,

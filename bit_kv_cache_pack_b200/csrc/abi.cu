@@ -427,6 +427,22 @@ omnikv_status omnikv_dense_decode_bf16(const void* k_cache, const void* v_cache,
   return OMNIKV_OK;
 }
 
+size_t omnikv_calibrate_workspace_bytes(int32_t num_tokens) { return calibrate_workspace_bytes(num_tokens); }
+
+omnikv_status omnikv_calibrate_bases(const void* values, const uint8_t* modality, const float* weights,
+                                     int32_t num_tokens, void* workspace, size_t workspace_bytes, float* bases,
+                                     double* eigenvalues, void* stream) {
+  if (!values || !modality || !weights || !workspace || !bases || num_tokens < 1) return OMNIKV_ERR_INVALID_ARG;
+  if (!aligned(values, 16) || !aligned(weights, 4) || !aligned(workspace, 16) || !aligned(bases, 4) ||
+      (eigenvalues && !aligned(eigenvalues, 8)))
+    return OMNIKV_ERR_INVALID_ARG;
+  if (workspace_bytes < calibrate_workspace_bytes(num_tokens)) return OMNIKV_ERR_CAPACITY;
+  if (launch_calibrate(static_cast<const __half*>(values), modality, weights, num_tokens, workspace, bases, eigenvalues,
+                       static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return OMNIKV_ERR_CUDA;
+  return OMNIKV_OK;
+}
+
 const char* omnikv_status_string(omnikv_status s) {
   switch (s) {
     case OMNIKV_OK: return "ok";

@@ -118,5 +118,8 @@ constexpr int kCoopMaxWindows = 16;
 int decode_body(int key_bits, int value_bits, int split_windows);
 int decode_ctas_per_sm(int body);  // resident decode CTAs per SM of a body on the current device
 cudaError_t launch_combine(const CombineParams& p, int batch, cudaStream_t stream);
+size_t calibrate_workspace_bytes(int num_tokens);  // 0 for num_tokens < 1
+cudaError_t launch_calibrate(const __half* values, const uint8_t* modality, const float* weights, int num_tokens,
+                             void* workspace, float* bases, double* eigenvalues, cudaStream_t stream);
 
 }  // namespace omnikv

@@ -299,6 +299,32 @@ OMNIKV_API omnikv_status omnikv_dense_decode_bf16(const void* k_cache, const voi
                                                   void* partials, int32_t num_splits, float* out,
                                                   int32_t* error_word, void* stream);
 
+/* Calibration of the per-modality value bases U_m of one (layer, kv head) from calibration values
+ * (paperpeel.com section 2.3 "Modality-aware value rotation": one basis per modality, calibrated
+ * once per model on calibration clips, section 3.1; pchao.org 方法概览: an attention-contribution-
+ * weighted covariance per modality and its eigendecomposition). For each modality m (ids 0, 1, 2;
+ * tokens with another id, or with a weight that is not positive, are ignored):
+ *   C_m = sum_t a_t (v_t - mu_m)(v_t - mu_m)^T / sum_t a_t, mu_m = sum_t a_t v_t / sum_t a_t (fp64);
+ *   E_m = the eigenvectors of C_m as columns, eigenvalues descending, each column's entry of
+ *         largest magnitude positive (the first on ties);
+ *   U_m = E_m H, H = 2^-3.5 H_128 (Sylvester; "a modality-aware correction of the Hadamard
+ *         rotation", paperpeel.com section 2.2); a modality without weight gets U_m = H.
+ *   values     : [num_tokens][128] fp16, device, 16-byte aligned
+ *   modality   : [num_tokens] u8, device;  weights: [num_tokens] fp32 a_t, device
+ *   workspace  : device scratch of at least omnikv_calibrate_workspace_bytes(num_tokens) bytes,
+ *                16-byte aligned, owned by the caller (contents undefined afterwards)
+ *   bases      : [3][128][128] fp32 out, device: U_m row-major, columns the basis (the layout of
+ *                omnikv_config.value_rot for one kv head)
+ *   eigenvalues: [3][128] fp64 out, device, descending (zeros for a modality without weight), or NULL
+ * Four stream-ordered launches (fp64 weighted Gram sums per token run, their reduction, a cyclic
+ * parallel Jacobi eigensolver per modality with at most 40 sweeps, sorting and the product with H).
+ * OMNIKV_ERR_INVALID_ARG: a null pointer, num_tokens < 1 or a misaligned pointer;
+ * OMNIKV_ERR_CAPACITY: workspace_bytes too small; OMNIKV_ERR_CUDA: a launch failed. */
+OMNIKV_API size_t omnikv_calibrate_workspace_bytes(int32_t num_tokens);
+OMNIKV_API omnikv_status omnikv_calibrate_bases(const void* values, const uint8_t* modality, const float* weights,
+                                                int32_t num_tokens, void* workspace, size_t workspace_bytes,
+                                                float* bases, double* eigenvalues, void* stream);
+
 /* Static text for a status code. */
 OMNIKV_API const char* omnikv_status_string(omnikv_status status);
 

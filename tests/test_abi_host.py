@@ -206,3 +206,26 @@ def test_step_split_rule(batch, tokens, want_s, want_fused):
     cache = _cache(batch=batch, cap_tokens=65536, max_seq_len=tokens)
     assert lib.omnikv_step_splits(ctypes.byref(_cfg()), ctypes.byref(cache), 0, ctypes.byref(f)) == want_s
     assert f.value == want_fused
+
+
+def test_calibration_arguments_rejected():
+    """Host checks of omnikv_calibrate_bases run before any launch (fake device
+    addresses are never dereferenced)."""
+    lib = _abi.load()
+    need = _abi.omnikv_calibrate_workspace_bytes(4096)
+    assert need > 0 and _abi.omnikv_calibrate_workspace_bytes(0) == 0
+    assert _abi.omnikv_calibrate_workspace_bytes(8192) >= need
+    A = 1 << 20  # an aligned fake address
+    ok = dict(values=A, modality=A, weights=A, num_tokens=4096, workspace=A, workspace_bytes=need, bases=A,
+              eigenvalues=0)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return lib.omnikv_calibrate_bases(a["values"], a["modality"], a["weights"], a["num_tokens"], a["workspace"],
+                                          a["workspace_bytes"], a["bases"], a["eigenvalues"], None)
+    assert call(values=0) == _abi.OMNIKV_ERR_INVALID_ARG
+    assert call(workspace=0) == _abi.OMNIKV_ERR_INVALID_ARG
+    assert call(num_tokens=0) == _abi.OMNIKV_ERR_INVALID_ARG
+    assert call(values=A + 8) == _abi.OMNIKV_ERR_INVALID_ARG       # values: 16-byte aligned
+    assert call(eigenvalues=A + 4) == _abi.OMNIKV_ERR_INVALID_ARG  # eigenvalues: 8-byte aligned
+    assert call(workspace_bytes=need - 1) == _abi.OMNIKV_ERR_CAPACITY
