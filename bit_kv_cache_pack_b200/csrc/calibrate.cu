@@ -23,8 +23,11 @@
 //      per round, 127 rounds per sweep; Golub and Van Loan, Matrix Computations,
 //      sections 8.5.2 "the symmetric Schur decomposition" and 8.5.3-8.5.5 on the
 //      cyclic and parallel orderings), accumulating the eigenvectors in the
-//      workspace, until the off-diagonal mass is below 1e-30 of the total (at most
-//      40 sweeps: the loop is bounded);
+//      workspace, until the off-diagonal mass is below 1e-26 of the total (an
+//      off-diagonal norm of 1e-13 of the matrix's; the sweeps converge
+//      quadratically, so the last one is far below) or after 40 sweeps (the loop
+//      is bounded; a singular covariance, fewer than 129 weighted tokens, keeps
+//      rounding noise in its null space and stops there);
 //   4. finish: rank the eigenvalues (descending, ties by index), apply the sign
 //      rule, multiply by H with a fast Walsh-Hadamard transform of every row, store
 //      U_m in fp32 and the sorted eigenvalues in fp64.
@@ -206,7 +209,7 @@ __global__ void __launch_bounds__(kJacThreads) jacobi_kernel(double* __restrict_
       }
       __syncthreads();
     }
-    // converged when the off-diagonal mass is below 1e-30 of the total
+    // converged when the off-diagonal mass is below 1e-26 of the total
     double off = 0.0, tot = 0.0;
     for (int e = tid; e < kMat; e += kJacThreads) {
       const double x = A[e] * A[e];
@@ -229,7 +232,7 @@ __global__ void __launch_bounds__(kJacThreads) jacobi_kernel(double* __restrict_
         o2 += red[w][0];
         t2 += red[w][1];
       }
-      s_done = (o2 <= 1e-30 * t2) ? 1 : 0;
+      s_done = (o2 <= 1e-26 * t2) ? 1 : 0;
     }
     __syncthreads();
   }

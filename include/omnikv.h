@@ -318,6 +318,8 @@ OMNIKV_API omnikv_status omnikv_dense_decode_bf16(const void* k_cache, const voi
  *   eigenvalues: [3][128] fp64 out, device, descending (zeros for a modality without weight), or NULL
  * Four stream-ordered launches (fp64 weighted Gram sums per token run, their reduction, a cyclic
  * parallel Jacobi eigensolver per modality with at most 40 sweeps, sorting and the product with H).
+ * A modality with fewer than 129 weighted tokens has a singular covariance: its null-space
+ * eigenvectors are not unique (any orthonormal basis of the null space is returned).
  * OMNIKV_ERR_INVALID_ARG: a null pointer, num_tokens < 1 or a misaligned pointer;
  * OMNIKV_ERR_CAPACITY: workspace_bytes too small; OMNIKV_ERR_CUDA: a launch failed. */
 OMNIKV_API size_t omnikv_calibrate_workspace_bytes(int32_t num_tokens);

@@ -4,6 +4,9 @@ eigendecomposition, U_m = E_m H) against the oracle (oracle/calibration.py, fp64
 with LAPACK's symmetric eigensolver): eigenvalues to 1e-9 of the largest, bases to
 2e-6 per entry (fp32 storage), orthogonality, the plain Hadamard rotation for a
 modality without weight, and invariance to tokens with zero weight or a foreign id.
+A modality with fewer weighted tokens than 129 has a singular covariance whose null
+space has no unique eigenbasis: there the eigenpairs with distinct nonzero
+eigenvalues are compared, and the rest are checked as eigenvectors (residual).
 
 Inputs: one (layer, kv head) of a workload's synthetic values (per-modality means
 and variances, the workload's modality layout) and, as the attention contribution
@@ -61,9 +64,10 @@ def _oracle_eigenvalues(values, mod, a):
     return out
 
 
-@pytest.mark.parametrize("name,T", [("omni3b-b16", 4096), ("omni30b-b8", 8192)])
+@pytest.mark.parametrize("name,T", [("omni30b-b8", 2048), ("omni30b-b8", 8192)])
 def test_bases_match_the_oracle(cuda_device, name, T):
     values, mod, a = _calibration_set(name, T, seed=5)
+    assert min(np.bincount(mod[a > 0], minlength=3)) >= 256  # full-rank covariances
     bases, lam = _gpu(values, mod, a, cuda_device)
     ref = calibrate_bases(values, mod, a)
     ref_lam = _oracle_eigenvalues(values, mod, a)
@@ -76,7 +80,7 @@ def test_bases_match_the_oracle(cuda_device, name, T):
 
 
 def test_modality_without_weight_keeps_the_hadamard_rotation(cuda_device):
-    values, mod, a = _calibration_set("omni3b-b16", 2048, seed=7)
+    values, mod, a = _calibration_set("omni30b-b8", 2048, seed=7)
     a = a.copy()
     a[mod == 1] = 0.0                  # audio: no weight at all
     mod = mod.copy()
@@ -90,7 +94,7 @@ def test_modality_without_weight_keeps_the_hadamard_rotation(cuda_device):
 
 
 def test_zero_weight_tokens_do_not_count(cuda_device):
-    values, mod, a = _calibration_set("omni3b-b16", 3000, seed=9)
+    values, mod, a = _calibration_set("omni30b-b8", 3000, seed=9)
     base, lam = _gpu(values, mod, a, cuda_device)
     # the same set with extra tokens of zero weight (random values) interleaved
     rng = np.random.default_rng(1)
@@ -102,3 +106,29 @@ def test_zero_weight_tokens_do_not_count(cuda_device):
     b2, lam2 = _gpu(v2[perm], m2[perm], a2[perm], cuda_device)
     assert np.abs(lam2 - lam).max() <= 1e-9 * np.abs(lam).max()
     assert np.abs(b2.astype(np.float64) - base.astype(np.float64)).max() <= 2e-6
+
+
+def test_singular_covariance_gives_valid_eigenpairs(cuda_device):
+    """omni3b's layout has 96 text tokens in 4,096: the text covariance has rank 95.
+    The eigenpairs with distinct nonzero eigenvalues match the oracle's; every
+    column is an eigenvector of C (residual) and the basis stays orthogonal."""
+    values, mod, a = _calibration_set("omni3b-b16", 4096, seed=5)
+    bases, lam = _gpu(values, mod, a, cuda_device)
+    ref = calibrate_bases(values, mod, a)
+    H = hadamard_normalised()
+    sel = (mod == 0) & (a > 0)
+    C = weighted_covariance(values[sel], a[sel])
+    ref_lam = _oracle_eigenvalues(values, mod, a)[0]
+    top = np.abs(ref_lam).max()
+    E = bases[0].astype(np.float64) @ H          # U = E H, H symmetric and orthogonal
+    E_ref = ref[0].astype(np.float64) @ H
+    assert np.abs(E.T @ E - np.eye(128)).max() < 1e-5
+    assert np.all(np.abs(lam[0] - ref_lam) <= 1e-9 * top)
+    gaps = np.minimum(np.abs(np.diff(ref_lam, prepend=np.inf)), np.abs(np.diff(ref_lam, append=-np.inf)))
+    distinct = (np.abs(ref_lam) > 1e-9 * top) & (gaps > 1e-6 * top)
+    assert distinct.sum() >= 90
+    assert np.abs(E[:, distinct] - E_ref[:, distinct]).max() <= 2e-5
+    resid = C @ E - E * lam[0][None, :]
+    assert np.abs(resid).max() <= 1e-5 * top
+    for mm in (1, 2):  # full-rank modalities
+        assert np.abs(bases[mm].astype(np.float64) - ref[mm].astype(np.float64)).max() <= 2e-6
