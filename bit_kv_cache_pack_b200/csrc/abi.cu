@@ -134,6 +134,7 @@ omnikv_status prepare_decode(const omnikv_config* cfg, const omnikv_cache* cache
   p->batch = cache->batch;
   p->len_add = 0;
   p->step_flags = nullptr;
+  p->append_ctas = 0;
   p->flag_wait_ns = kFlagWaitNs;
   return OMNIKV_OK;
 }
@@ -276,23 +277,36 @@ omnikv_status omnikv_combine(const omnikv_config* cfg, const omnikv_cache* cache
 
 namespace {
 
-// The split count of a decode step and whether its append runs inside the decode
-// launch, for the cache as the step sees it (max_seq_len already counting the
-// appended token). Fused only when every CTA of that launch is resident at once,
-// so a waiting warp never waits on an unscheduled CTA; with num_splits = 0 the
-// default is lowered (by at most half) to make it so.
-void plan_step(const omnikv_config* cfg, const omnikv_cache* after, int32_t num_splits, int32_t* S, bool* fused) {
+// The split count of a decode step, whether its append runs inside the decode
+// launch and with how many append CTAs, for the cache as the step sees it
+// (max_seq_len already counting the appended token). Fused only when every CTA of
+// that launch is resident at once, so a waiting warp never waits on an
+// unscheduled CTA. The append CTAs fill the slots the decode CTAs leave, each
+// appending for at most kMaxAppendsPerCta (sequence, kv head) units in turn (its
+// flags are read only by the last window of each split); with num_splits = 0 the
+// default split count is lowered (by at most half) when even that does not fit.
+constexpr long long kMaxAppendsPerCta = 4;
+
+void plan_step(const omnikv_config* cfg, const omnikv_cache* after, int32_t num_splits, int32_t* S, bool* fused,
+               int32_t* append_ctas = nullptr) {
   const long long units = (long long)after->batch * cfg->num_kv_heads;
+  const long long min_append = (units + kMaxAppendsPerCta - 1) / kMaxAppendsPerCta;
   *S = resolve_splits(cfg, after, num_splits);
   const long long resident = step_residency(cfg, after, *S);
-  *fused = units * (1 + (long long)*S) <= resident;
-  if (!*fused && num_splits == 0) {
+  long long A = units;
+  *fused = units * (long long)*S + min_append <= resident;
+  if (*fused) {
+    A = resident - units * (long long)*S;
+    if (A > units) A = units;
+  } else if (num_splits == 0) {
     const long long s_res = resident / units - 1;
     if (s_res >= 1 && 2 * s_res >= *S && units * (1 + s_res) <= step_residency(cfg, after, (int32_t)s_res)) {
       *S = (int32_t)s_res;
       *fused = true;
+      A = units;
     }
   }
+  if (append_ctas) *append_ctas = (int32_t)A;
 }
 
 }  // namespace
@@ -340,9 +354,9 @@ omnikv_status omnikv_append_decode(const omnikv_config* cfg, omnikv_cache* cache
   if ((long long)cache->max_seq_len + 1 > cache->cap_tokens) return OMNIKV_ERR_CAPACITY;
   omnikv_cache after = *cache;  // the decode sees the appended token
   after.max_seq_len += 1;
-  int32_t S;
+  int32_t S, A;
   bool fused;
-  plan_step(cfg, &after, num_splits, &S, &fused);
+  plan_step(cfg, &after, num_splits, &S, &fused, &A);
   DecodeParams dp;
   if ((st = prepare_decode(cfg, &after, q, partials, S, &dp)) != OMNIKV_OK) return st;
   WriteParams wp;
@@ -352,6 +366,7 @@ omnikv_status omnikv_append_decode(const omnikv_config* cfg, omnikv_cache* cache
   if (fused) {
     dp.len_add = 1;
     dp.step_flags = cache->step_flags;
+    dp.append_ctas = A;
     if (launch_decode_step(dp, wp, s) != cudaSuccess) return OMNIKV_ERR_CUDA;
   } else {
     if (launch_write(wp, cache->batch, s) != cudaSuccess) return OMNIKV_ERR_CUDA;

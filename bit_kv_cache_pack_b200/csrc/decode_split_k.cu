@@ -1301,25 +1301,28 @@ __global__ void __launch_bounds__(kThreads, body_ctas_per_sm(kBody))
   static_assert(sizeof(WindowSmem) <= sizeof(DecodeSmem), "append uses the decode shared memory");
   griddep_launch_dependents();
   const int H = p.num_kv_heads;
-  const int nappend = p.batch * H;
+  const int nappend = p.append_ctas;
   if ((int)blockIdx.x < nappend) {
     griddep_wait();
-    const int b = blockIdx.x / H, h = blockIdx.x % H;
-    const int L0 = w.seq_lens[b];
-    const int L1 = L0 + 1;
-    if (L0 >= 0 && L1 <= w.cap_tokens) {
-      quantize_window(w, b, h, L0 / kWindow, L0, L1, *reinterpret_cast<WindowSmem*>(&sm), threadIdx.x, 1, true);
-      if (h > 0 && threadIdx.x == 0) {  // the decode of head h reads the token's modality after h's flag
-        const int m = w.mod_new[b];
-        w.modality[(size_t)b * w.cap_tokens + L0] = (uint8_t)(m >= kMods ? kMods - 1 : m);
+    for (int u = blockIdx.x; u < p.batch * H; u += nappend) {
+      const int b = u / H, h = u % H;
+      const int L0 = w.seq_lens[b];
+      const int L1 = L0 + 1;
+      if (L0 >= 0 && L1 <= w.cap_tokens) {
+        quantize_window(w, b, h, L0 / kWindow, L0, L1, *reinterpret_cast<WindowSmem*>(&sm), threadIdx.x, 1, true);
+        if (h > 0 && threadIdx.x == 0) {  // the decode of head h reads the token's modality after h's flag
+          const int m = w.mod_new[b];
+          w.modality[(size_t)b * w.cap_tokens + L0] = (uint8_t)(m >= kMods ? kMods - 1 : m);
+        }
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x == 0)
+          asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(w.step_flags + (size_t)b * H + h), "r"(L1)
+                       : "memory");
+      } else if (threadIdx.x == 0 && h == 0) {
+        set_error(w.error_word, OMNIKV_DEVERR_CAPACITY);
       }
-      __threadfence();
-      __syncthreads();
-      if (threadIdx.x == 0)
-        asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(w.step_flags + (size_t)b * H + h), "r"(L1)
-                     : "memory");
-    } else if (threadIdx.x == 0 && h == 0) {
-      set_error(w.error_word, OMNIKV_DEVERR_CAPACITY);
+      __syncthreads();  // the shared memory is the next unit's
     }
     return;
   }
@@ -1436,7 +1439,7 @@ cudaError_t launch_decode_step(const DecodeParams& p, const WriteParams& w, cuda
   const int meta = p.key_meta;
   const cudaError_t e = prepare_kernels(body, meta);
   if (e != cudaSuccess) return e;
-  const dim3 grid(p.batch * p.num_kv_heads * (1 + p.num_splits));
+  const dim3 grid(p.append_ctas + p.batch * p.num_kv_heads * p.num_splits);
   const dim3 block(kThreads);
   if (body == kBodyGeneric) return launch_pdl(decode_step_kernel<kBodyGeneric, kMetaFp16>, grid, block, 0, stream, p, w);
   if (meta == kMetaMx)

@@ -56,6 +56,9 @@ struct DecodeParams {
   int len_add;
   const int32_t* step_flags;
   uint64_t flag_wait_ns;  // how long a copy waits for its step flag before giving up (OMNIKV_DEVERR_TIMEOUT)
+  // decode step only: the append CTAs in front of the decode CTAs; append CTA a
+  // appends for (sequence, kv head) units a, a + append_ctas, ... in turn
+  int append_ctas;
 };
 
 struct CombineParams {

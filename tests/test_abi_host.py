@@ -197,7 +197,7 @@ def test_default_split_rule(batch, tokens, bits, want):
 
 @pytest.mark.parametrize("batch,tokens,want_s,want_fused", [
     (1, 10240, 81, 1),    # 10,241 tokens after the append: 81 splits of 4 windows, 164 CTAs fit
-    (16, 32768, 8, 1),    # 9 per-warp splits would need 320 CTAs > 296: lowered to 8 (288 fit)
+    (16, 32768, 9, 1),    # 32 units x 9 per-warp splits = 288 CTAs + 8 append CTAs of 4 units each = 296
     (64, 32768, 8, 0),    # 128 units x 9 CTAs do not fit: append launch, then decode launch
 ])
 def test_step_split_rule(batch, tokens, want_s, want_fused):

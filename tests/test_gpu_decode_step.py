@@ -49,11 +49,14 @@ CASES = [
     (2, 8, [93, 40], 4, 200, 2),            # 2 x (1 + 200) CTAs: beyond residency -> four-call fallback
     (2, 8, [93, 250], 4, 0, 4),             # K4V4: the CUDA-core decode path with the fused append
     (2, 8, [700], 3, 1, 2),                 # one split of 22 windows: the per-warp body in the fused launch
+    # 16 x 2 units x 9 per-warp splits = 288 decode CTAs: the 8 append CTAs left
+    # in a 296-CTA wave append for 4 (sequence, kv head) units each
+    (2, 8, [4700 + 13 * i for i in range(16)], 2, 0, 2),
 ]
 
 
 @pytest.mark.parametrize("hkv,G,lengths,steps,splits,bits", CASES,
-                         ids=["b1-boundary", "ragged-b3", "h4", "fallback", "k4", "per-warp"])
+                         ids=["b1-boundary", "ragged-b3", "h4", "fallback", "k4", "per-warp", "shared-append-ctas"])
 def test_decode_step_matches_four_calls_and_oracle(cuda_device, hkv, G, lengths, steps, splits, bits):
     import bit_kv_cache_pack_b200 as m
     dev = cuda_device
