@@ -145,3 +145,60 @@ def decode_fused(cfg: OracleConfig, cache: OracleCache, q_fp16, num_splits: int 
                 o += (acc[:, m] / l[:, None]) @ U.T
             out[b, h * G:(h + 1) * G] = o
     return out
+
+
+# ----------------------------------------------------------------------------
+# streaming / captioning cache policy
+# ----------------------------------------------------------------------------
+STREAM_KEY_BLOCK = 128     # keys are quantised every 128 tokens (in 32-token windows)
+STREAM_VALUE_WINDOW = 128  # values keep a 128-token fp16 sliding window
+
+
+def stream_boundaries(T: int):
+    """The streaming policy of paperpeel.com section 3.1 ("Implementation details",
+    captioning: keys quantised every 128 tokens in groups of 32, values in a
+    128-token fp16 sliding window before quantisation). Readings:
+      s1  key blocks are aligned at absolute positions: the keys of positions
+          [0, KB) are read quantised, KB = 128 floor(T / 128); the others fp16;
+      s2  a value is quantised when it leaves the window of the newest 128
+          tokens: positions [0, VB) are read quantised, VB = max(0, T - 128);
+      s3  a quantised key or value is exactly what the ordinary cache write
+          produces (the key windows of a complete block are full; the value
+          codec is per token);
+      s4  fp16 keys and values enter attention as they are (original basis).
+    Returns (KB, VB)."""
+    return STREAM_KEY_BLOCK * (T // STREAM_KEY_BLOCK), max(0, T - STREAM_VALUE_WINDOW)
+
+
+def decode_dense_stream(cfg: OracleConfig, cache: OracleCache, k_raw, v_raw, q_fp16):
+    """decode_dense under the streaming policy: the cache holds every token's
+    record (written by the ordinary write); token t's key is the dequantised one
+    for t < KB and the raw fp16 key otherwise, its value the dequantised one for
+    t < VB and the raw fp16 value otherwise. k_raw, v_raw: [B][H][>= T_b][128] fp16
+    (the raw inputs of every cached position); q: [B][H_q][128]. fp64 result."""
+    q = np.asarray(q_fp16, dtype=np.float16).astype(F64)
+    B, Hq, _ = q.shape
+    G = cfg.num_q_heads // cfg.num_kv_heads
+    R = key_rotation_matrix(cfg.key_signs)
+    out = np.zeros((B, Hq, HEAD_DIM), F64)
+    for b in range(B):
+        T = int(cache.seq_lens[b])
+        if T == 0:
+            continue
+        KB, VB = stream_boundaries(T)
+        for h in range(cfg.num_kv_heads):
+            kq, vq, mod = dequantize(cfg, cache, b, h)
+            k = kq @ R
+            v = np.zeros_like(vq)
+            for m in range(NUM_MODALITIES):
+                U = np.asarray(cfg.value_rot[h, m], dtype=np.float32).astype(F64)
+                sel = mod == m
+                v[sel] = vq[sel] @ U.T
+            k[KB:T] = np.asarray(k_raw[b][h][KB:T], np.float16).astype(F64)
+            v[VB:T] = np.asarray(v_raw[b][h][VB:T], np.float16).astype(F64)
+            for g in range(G):
+                i = h * G + g
+                s = (k @ q[b, i]) / np.sqrt(HEAD_DIM)
+                p = np.exp(s - s.max())
+                out[b, i] = (p[:, None] * v).sum(axis=0) / p.sum()
+    return out
