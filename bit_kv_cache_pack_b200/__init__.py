@@ -12,6 +12,7 @@ from ._abi import (OMNIKV_DEVERR_CAPACITY, OMNIKV_ERR_CAPACITY, OMNIKV_ERR_CUDA,
                    omnikv_combine_step, omnikv_decode_attention, omnikv_decode_static,
                    omnikv_decode_step, omnikv_step_splits, omnikv_default_splits, omnikv_dense_decode_bf16,
                    omnikv_dense_partials_bytes, omnikv_partials_bytes,
-                   omnikv_record_bytes, omnikv_test_decode_pending, omnikv_write_cache,
+                   omnikv_record_bytes, omnikv_stream_decode, omnikv_stream_write_cache,
+                   omnikv_test_decode_pending, omnikv_write_cache,
                    omnikv_write_cache_rotations, status_string)
-from .layer import KVCache, LayerConstants, partials_tensor  # noqa: F401
+from .layer import KVCache, LayerConstants, partials_tensor, stream_rings  # noqa: F401

@@ -35,7 +35,7 @@ EXPORTED = (
     "omnikv_dense_partials_bytes", "omnikv_dense_decode_bf16", "omnikv_decode_step",
     "omnikv_append_decode", "omnikv_combine_step", "omnikv_step_splits", "omnikv_write_cache_rotations",
     "omnikv_test_decode_pending", "omnikv_record_bytes_meta", "omnikv_calibrate_workspace_bytes",
-    "omnikv_calibrate_bases",
+    "omnikv_calibrate_bases", "omnikv_stream_write_cache", "omnikv_stream_decode",
 )
 OMNIKV_DECODE_STATIC_SCRATCH_BYTES = 8 << 20
 
@@ -107,6 +107,10 @@ def load() -> ctypes.CDLL:
     lib.omnikv_dense_partials_bytes.argtypes, lib.omnikv_dense_partials_bytes.restype = [I32, I32, I32], SZ
     lib.omnikv_dense_decode_bf16.argtypes = [P, P, P, I32, I32, I32, I32, I32, P, P, I32, P, P, P]
     lib.omnikv_calibrate_workspace_bytes.argtypes, lib.omnikv_calibrate_workspace_bytes.restype = [I32], SZ
+    lib.omnikv_stream_write_cache.argtypes = [cfgp, cachep, P, P, P, P, P, I32, P]
+    lib.omnikv_stream_write_cache.restype = ctypes.c_int
+    lib.omnikv_stream_decode.argtypes = [cfgp, cachep, P, P, P, P, I32, P, P]
+    lib.omnikv_stream_decode.restype = ctypes.c_int
     lib.omnikv_calibrate_bases.argtypes = [P, P, P, I32, P, SZ, P, P, P]
     lib.omnikv_calibrate_bases.restype = ctypes.c_int
     lib.omnikv_dense_decode_bf16.restype = ctypes.c_int
@@ -250,6 +254,22 @@ def omnikv_decode_static(cfg: OmniKVConfig, cache: OmniKVCache, q, out, num_spli
 
 def omnikv_dense_partials_bytes(batch: int, num_q_heads: int, num_splits: int) -> int:
     return int(load().omnikv_dense_partials_bytes(batch, num_q_heads, num_splits))
+
+
+def omnikv_stream_write_cache(cfg: OmniKVConfig, cache: OmniKVCache, ring_k, ring_v, k_new, v_new, modality_new,
+                              n_new: int, stream=None) -> None:
+    """omnikv_write_cache plus the raw-input rings of the streaming policy; see include/omnikv.h."""
+    st = load().omnikv_stream_write_cache(ctypes.byref(cfg), ctypes.byref(cache), _ptr(ring_k), _ptr(ring_v),
+                                          _ptr(k_new), _ptr(v_new), _ptr(modality_new), int(n_new), _stream(stream))
+    _check(st, "omnikv_stream_write_cache")
+
+
+def omnikv_stream_decode(cfg: OmniKVConfig, cache: OmniKVCache, ring_k, ring_v, q, partials, num_splits: int, out,
+                         stream=None) -> None:
+    """Decode + combine under the streaming policy; see include/omnikv.h."""
+    st = load().omnikv_stream_decode(ctypes.byref(cfg), ctypes.byref(cache), _ptr(ring_k), _ptr(ring_v), _ptr(q),
+                                     _ptr(partials), int(num_splits), _ptr(out), _stream(stream))
+    _check(st, "omnikv_stream_decode")
 
 
 def omnikv_calibrate_workspace_bytes(num_tokens: int) -> int:

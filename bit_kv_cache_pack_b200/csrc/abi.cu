@@ -135,6 +135,7 @@ omnikv_status prepare_decode(const omnikv_config* cfg, const omnikv_cache* cache
   p->len_add = 0;
   p->step_flags = nullptr;
   p->append_ctas = 0;
+  p->stream = 0;
   p->flag_wait_ns = kFlagWaitNs;
   return OMNIKV_OK;
 }
@@ -439,6 +440,48 @@ omnikv_status omnikv_dense_decode_bf16(const void* k_cache, const void* v_cache,
   p.num_splits = S;
   p.split_chunks = nc > 0 ? (nc + S - 1) / S : 1;
   if (launch_dense(p, batch, static_cast<cudaStream_t>(stream)) != cudaSuccess) return OMNIKV_ERR_CUDA;
+  return OMNIKV_OK;
+}
+
+omnikv_status omnikv_stream_write_cache(const omnikv_config* cfg, omnikv_cache* cache, void* ring_k, void* ring_v,
+                                        const void* k_new, const void* v_new, const uint8_t* modality_new,
+                                        int32_t n_new, void* stream) {
+  omnikv_status st = check_config(cfg);
+  if (st != OMNIKV_OK) return st;
+  if ((st = check_cache(cache)) != OMNIKV_OK) return st;
+  if (n_new < 1 || !k_new || !v_new || !modality_new || !ring_k || !ring_v) return OMNIKV_ERR_INVALID_ARG;
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(ring_k, 16) || !aligned(ring_v, 16))
+    return OMNIKV_ERR_INVALID_ARG;
+  if ((long long)cache->max_seq_len + n_new > cache->cap_tokens) return OMNIKV_ERR_CAPACITY;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the raw inputs into their ring slots first (positions from the lengths before the write)
+  if (launch_stream_push(static_cast<const __half*>(k_new), static_cast<const __half*>(v_new), cache->seq_lens,
+                         static_cast<__half*>(ring_k), static_cast<__half*>(ring_v), cache->batch, cfg->num_kv_heads,
+                         n_new, s) != cudaSuccess)
+    return OMNIKV_ERR_CUDA;
+  return omnikv_write_cache(cfg, cache, k_new, v_new, modality_new, n_new, stream);
+}
+
+omnikv_status omnikv_stream_decode(const omnikv_config* cfg, const omnikv_cache* cache, const void* ring_k,
+                                   const void* ring_v, const void* q, void* partials, int32_t num_splits, float* out,
+                                   void* stream) {
+  if (!ring_k || !ring_v || !out) return OMNIKV_ERR_INVALID_ARG;
+  if (!aligned(ring_k, 16) || !aligned(ring_v, 16) || !aligned(out, 16)) return OMNIKV_ERR_INVALID_ARG;
+  DecodeParams dp;
+  omnikv_status st = prepare_decode(cfg, cache, q, partials, num_splits, &dp);
+  if (st != OMNIKV_OK) return st;
+  const int S = dp.num_splits;  // body splits 0 .. S-1 (the body's last, empty one is overwritten), tail split S
+  if (S + 1 > kMaxSplits) return OMNIKV_ERR_UNSUPPORTED;
+  dp.num_splits = S + 1;        // partials stride
+  dp.stream = 1;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (launch_decode(dp, cache->batch, s) != cudaSuccess) return OMNIKV_ERR_CUDA;
+  if (launch_stream_tail(dp, static_cast<const __half*>(ring_k), static_cast<const __half*>(ring_v), S, s) !=
+      cudaSuccess)
+    return OMNIKV_ERR_CUDA;
+  CombineParams cp;
+  if ((st = prepare_combine(cfg, cache, partials, S + 1, out, &cp)) != OMNIKV_OK) return st;
+  if (launch_combine(cp, cache->batch, s) != cudaSuccess) return OMNIKV_ERR_CUDA;
   return OMNIKV_OK;
 }
 

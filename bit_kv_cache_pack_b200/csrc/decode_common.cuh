@@ -69,6 +69,7 @@ __device__ __forceinline__ void split_range(const DecodeParams& p, int b, int sp
   const int L = p.seq_lens[b];
   const int La = L + p.len_add;  // a decode step's append happens only within the capacity
   T = max(0, min(La <= p.cap_tokens ? La : L, p.cap_tokens));
+  if (p.stream) T = kWindow * (max(0, T - 128) / kWindow);  // streaming policy: the packed body only
   const int nw = (T + kWindow - 1) / kWindow;
   w0 = min(split * p.split_windows, nw);
   w1 = min(w0 + p.split_windows, nw);

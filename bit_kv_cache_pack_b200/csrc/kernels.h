@@ -59,6 +59,9 @@ struct DecodeParams {
   // decode step only: the append CTAs in front of the decode CTAs; append CTA a
   // appends for (sequence, kv head) units a, a + append_ctas, ... in turn
   int append_ctas;
+  // streaming policy: the decode covers only the packed body, the windows before
+  // 32 floor(max(0, T - 128) / 32) (the tail is stream_tail_kernel's)
+  int stream;
 };
 
 struct CombineParams {
@@ -121,6 +124,10 @@ constexpr int kCoopMaxWindows = 16;
 int decode_body(int key_bits, int value_bits, int split_windows);
 int decode_ctas_per_sm(int body);  // resident decode CTAs per SM of a body on the current device
 cudaError_t launch_combine(const CombineParams& p, int batch, cudaStream_t stream);
+cudaError_t launch_stream_push(const __half* k_new, const __half* v_new, const int32_t* seq_lens, __half* ring_k,
+                               __half* ring_v, int batch, int num_kv_heads, int n_new, cudaStream_t stream);
+cudaError_t launch_stream_tail(const DecodeParams& p, const __half* ring_k, const __half* ring_v, int tail_split,
+                               cudaStream_t stream);
 size_t calibrate_workspace_bytes(int num_tokens);  // 0 for num_tokens < 1
 cudaError_t launch_calibrate(const __half* values, const uint8_t* modality, const float* weights, int num_tokens,
                              void* workspace, float* bases, double* eigenvalues, cudaStream_t stream);

@@ -68,6 +68,13 @@ class KVCache:
                            self.struct.max_seq_len, self.step_flags[b].data_ptr())
 
 
+def stream_rings(batch: int, num_kv_heads: int, device="cuda"):
+    """The raw fp16 key and value rings of the streaming policy, [B][H_kv][256][128] each."""
+    shape = (batch, num_kv_heads, 256, HEAD_DIM)
+    return (torch.zeros(shape, dtype=torch.float16, device=device),
+            torch.zeros(shape, dtype=torch.float16, device=device))
+
+
 def partials_tensor(batch: int, num_q_heads: int, num_splits: int, device="cuda") -> torch.Tensor:
     n = _abi.omnikv_partials_bytes(batch, num_q_heads, num_splits)
     return torch.empty(n // 4, dtype=torch.float32, device=device)

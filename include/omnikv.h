@@ -299,6 +299,32 @@ OMNIKV_API omnikv_status omnikv_dense_decode_bf16(const void* k_cache, const voi
                                                   void* partials, int32_t num_splits, float* out,
                                                   int32_t* error_word, void* stream);
 
+/* Streaming / captioning cache policy (paperpeel.com section 3.1, "Implementation details": keys are
+ * quantised every 128 tokens in groups of 32, values keep a 128-token fp16 sliding window before
+ * quantisation). With T tokens cached, the decode reads the keys of positions [0, KB) quantised,
+ * KB = 128 floor(T / 128) (blocks aligned at absolute positions), and the values of positions
+ * [0, VB) quantised, VB = max(0, T - 128); every other key and value enters attention as its raw
+ * fp16 input (original basis). Records are written for every token as by omnikv_write_cache (a
+ * quantised entry is exactly the ordinary write's); the raw inputs of the newest 256 positions are
+ * kept in caller-owned rings:
+ *   ring_k, ring_v : [batch][num_kv_heads][256][128] fp16 each, 16-byte aligned; position p of a
+ *                    sequence in slot p mod 256 (no initialisation needed).
+ * omnikv_stream_write_cache: omnikv_write_cache plus the copy of the last min(n_new, 256) tokens of
+ *   the write into the rings (at the positions the write gives them); the same arguments and errors.
+ * omnikv_stream_decode: decode + combine under the policy, three stream-ordered launches: the
+ *   ordinary decode over the windows before 32 floor(VB / 32) (splits 0 .. S-1), a tail kernel over
+ *   the remaining (at most 159) positions (split S; its raw values' sums are carried in modality 0's
+ *   rotated basis), and the combine over S + 1 splits.
+ *   num_splits: S, or 0 for omnikv_default_splits; partials: omnikv_partials_bytes(batch,
+ *   num_q_heads, S + 1) bytes; out: [batch][num_q_heads][128] fp32. Errors as omnikv_decode_attention
+ *   and omnikv_combine. */
+OMNIKV_API omnikv_status omnikv_stream_write_cache(const omnikv_config* cfg, omnikv_cache* cache, void* ring_k,
+                                                   void* ring_v, const void* k_new, const void* v_new,
+                                                   const uint8_t* modality_new, int32_t n_new, void* stream);
+OMNIKV_API omnikv_status omnikv_stream_decode(const omnikv_config* cfg, const omnikv_cache* cache,
+                                              const void* ring_k, const void* ring_v, const void* q, void* partials,
+                                              int32_t num_splits, float* out, void* stream);
+
 /* Calibration of the per-modality value bases U_m of one (layer, kv head) from calibration values
  * (paperpeel.com section 2.3 "Modality-aware value rotation": one basis per modality, calibrated
  * once per model on calibration clips, section 3.1; pchao.org 方法概览: an attention-contribution-
