@@ -100,6 +100,9 @@ def parse_args():
                          "(the TurboQuant key codec the pages compare against: one scale per token)")
     ap.add_argument("--batch", type=int, default=0, help="with --layer: override the workload's batch")
     ap.add_argument("--splits", default="0", help="with --layer decode: comma-separated split counts (0: default)")
+    ap.add_argument("--stream", action="store_true",
+                    help="with --layer decode: also time the streaming/captioning policy's decode "
+                         "(packed body + tail + combine, omnikv_stream_decode) over the same cache")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--clocks-csv", default=None, help="where to keep the nvidia-smi samples (default: a temp file)")
     return ap.parse_args()
@@ -736,11 +739,16 @@ def run_layer(args):
                           "error_word": int(c.error_word.item())}), flush=True)
         return
     cache = m.KVCache(spec.batch, spec.num_kv_heads, cap, bits, bits, dev, key_meta_format=fmt)
+    rings = m.stream_rings(spec.batch, spec.num_kv_heads, dev) if args.stream else None
     for b in range(spec.batch):
         k, v, mod = prefill_inputs(spec, seed, 0, params, drift, L, dev, batch_index=[b])
         n = int(L[b])
-        m.omnikv_write_cache(consts.struct, cache.sequence_view(b), k[:, :, :n].contiguous(),
-                             v[:, :, :n].contiguous(), mod[:, :n].contiguous(), n)
+        if rings is not None:
+            m.omnikv_stream_write_cache(consts.struct, cache.sequence_view(b), rings[0][b:b + 1], rings[1][b:b + 1],
+                                        k[:, :, :n].contiguous(), v[:, :, :n].contiguous(), mod[:, :n].contiguous(), n)
+        else:
+            m.omnikv_write_cache(consts.struct, cache.sequence_view(b), k[:, :, :n].contiguous(),
+                                 v[:, :, :n].contiguous(), mod[:, :n].contiguous(), n)
         del k, v, mod
     cache.struct.max_seq_len = T
     q = torch.randn(spec.batch, spec.num_q_heads, 128, device=dev).half()
@@ -755,6 +763,13 @@ def run_layer(args):
                           "combine_us": round(comb, 2), "GBps": round(byts / dec / 1e3, 1),
                           "frac": round(byts / dec / 1e3 / peak, 4), "error_word": int(cache.error_word.item())}),
               flush=True)
+        if rings is not None:
+            part2 = m.partials_tensor(spec.batch, spec.num_q_heads, S + 1, dev)
+            st = timed(lambda: m.omnikv_stream_decode(consts.struct, cache.struct, rings[0], rings[1], q, part2, S, out))
+            print(json.dumps({"layer": "stream-decode", "workload": spec.name, "meta": args.meta, "splits": S,
+                              "us": round(st, 2), "vs_decode_plus_combine": round(st / (dec + comb), 3),
+                              "what": "packed body + tail kernel (newest <= 159 positions) + combine, 3 launches"}),
+                  flush=True)
 
 
 def main():
