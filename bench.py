@@ -56,8 +56,8 @@ META_FORMATS = {"fp16": 0, "mx": 1, "turbo": 2}   # omnikv_config.key_meta_forma
 # next capture.
 TRAFFIC_CAPTURES = {
     ("qwen3-omni-30b-48L-b8-ctx65536", "fp16"): {
-        "sources_sha256": "799cd4759c72a470928c8d49d5aae5d6bc7a99b927e0bf951309ec3e40f878e9",
-        "bytes_per_launch": 173718528 + 8225024},
+        "sources_sha256": "bcb92b4de243d33d445c563ddb24818b6632cfcad38087d9e68aed22c47e721c",
+        "bytes_per_launch": 173743872 + 8676352},
 }
 KERNEL_SOURCES = ("decode_split_k.cu", "decode_common.cuh", "append.cuh", "common.cuh", "ptx.cuh", "kernels.h")
 
