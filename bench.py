@@ -764,11 +764,11 @@ def run_layer(args):
                           "frac": round(byts / dec / 1e3 / peak, 4), "error_word": int(cache.error_word.item())}),
               flush=True)
         if rings is not None:
-            part2 = m.partials_tensor(spec.batch, spec.num_q_heads, S + 1, dev)
+            part2 = m.partials_tensor(spec.batch, spec.num_q_heads, S + m._abi.OMNIKV_STREAM_TAIL_SPLITS, dev)
             st = timed(lambda: m.omnikv_stream_decode(consts.struct, cache.struct, rings[0], rings[1], q, part2, S, out))
             print(json.dumps({"layer": "stream-decode", "workload": spec.name, "meta": args.meta, "splits": S,
                               "us": round(st, 2), "vs_decode_plus_combine": round(st / (dec + comb), 3),
-                              "what": "packed body + tail kernel (newest <= 159 positions) + combine, 3 launches"}),
+                              "what": "packed body + tail kernel (newest <= 159 positions, 4 CTAs per kv head) + combine, 3 launches"}),
                   flush=True)
 
 

@@ -27,6 +27,7 @@ OMNIKV_DEVERR_RANGE = 0x10
 OMNIKV_META_FP16 = 0
 OMNIKV_META_MXFP4 = 1
 OMNIKV_META_TURBO = 2
+OMNIKV_STREAM_TAIL_SPLITS = 4  # partials of omnikv_stream_decode: S + this many splits
 
 EXPORTED = (
     "omnikv_record_bytes", "omnikv_partials_bytes", "omnikv_default_splits",

@@ -470,9 +470,10 @@ omnikv_status omnikv_stream_decode(const omnikv_config* cfg, const omnikv_cache*
   DecodeParams dp;
   omnikv_status st = prepare_decode(cfg, cache, q, partials, num_splits, &dp);
   if (st != OMNIKV_OK) return st;
-  const int S = dp.num_splits;  // body splits 0 .. S-1 (the body's last, empty one is overwritten), tail split S
-  if (S + 1 > kMaxSplits) return OMNIKV_ERR_UNSUPPORTED;
-  dp.num_splits = S + 1;        // partials stride
+  // body splits 0 .. S-1, tail splits S .. S+3 (the body's empty splits there are overwritten)
+  const int S = dp.num_splits;
+  if (S + kStreamTailSplits > kMaxSplits) return OMNIKV_ERR_UNSUPPORTED;
+  dp.num_splits = S + kStreamTailSplits;  // partials stride
   dp.stream = 1;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (launch_decode(dp, cache->batch, s) != cudaSuccess) return OMNIKV_ERR_CUDA;
@@ -480,7 +481,7 @@ omnikv_status omnikv_stream_decode(const omnikv_config* cfg, const omnikv_cache*
       cudaSuccess)
     return OMNIKV_ERR_CUDA;
   CombineParams cp;
-  if ((st = prepare_combine(cfg, cache, partials, S + 1, out, &cp)) != OMNIKV_OK) return st;
+  if ((st = prepare_combine(cfg, cache, partials, S + kStreamTailSplits, out, &cp)) != OMNIKV_OK) return st;
   if (launch_combine(cp, cache->batch, s) != cudaSuccess) return OMNIKV_ERR_CUDA;
   return OMNIKV_OK;
 }

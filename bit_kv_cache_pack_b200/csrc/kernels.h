@@ -126,6 +126,7 @@ int decode_ctas_per_sm(int body);  // resident decode CTAs per SM of a body on t
 cudaError_t launch_combine(const CombineParams& p, int batch, cudaStream_t stream);
 cudaError_t launch_stream_push(const __half* k_new, const __half* v_new, const int32_t* seq_lens, __half* ring_k,
                                __half* ring_v, int batch, int num_kv_heads, int n_new, cudaStream_t stream);
+constexpr int kStreamTailSplits = 4;  // splits the streaming decode's tail adds after the body's
 cudaError_t launch_stream_tail(const DecodeParams& p, const __half* ring_k, const __half* ring_v, int tail_split,
                                cudaStream_t stream);
 size_t calibrate_workspace_bytes(int num_tokens);  // 0 for num_tokens < 1

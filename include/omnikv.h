@@ -313,11 +313,12 @@ OMNIKV_API omnikv_status omnikv_dense_decode_bf16(const void* k_cache, const voi
  *   the write into the rings (at the positions the write gives them); the same arguments and errors.
  * omnikv_stream_decode: decode + combine under the policy, three stream-ordered launches: the
  *   ordinary decode over the windows before 32 floor(VB / 32) (splits 0 .. S-1), a tail kernel over
- *   the remaining (at most 159) positions (split S; its raw values' sums are carried in modality 0's
- *   rotated basis), and the combine over S + 1 splits.
+ *   the remaining (at most 159) positions in 4 chunks (splits S .. S+3; its raw values' sums are
+ *   carried in modality 0's rotated basis), and the combine over S + 4 splits.
  *   num_splits: S, or 0 for omnikv_default_splits; partials: omnikv_partials_bytes(batch,
- *   num_q_heads, S + 1) bytes; out: [batch][num_q_heads][128] fp32. Errors as omnikv_decode_attention
- *   and omnikv_combine. */
+ *   num_q_heads, S + OMNIKV_STREAM_TAIL_SPLITS) bytes; out: [batch][num_q_heads][128] fp32. Errors as
+ *   omnikv_decode_attention and omnikv_combine. */
+#define OMNIKV_STREAM_TAIL_SPLITS 4
 OMNIKV_API omnikv_status omnikv_stream_write_cache(const omnikv_config* cfg, omnikv_cache* cache, void* ring_k,
                                                    void* ring_v, const void* k_new, const void* v_new,
                                                    const uint8_t* modality_new, int32_t n_new, void* stream);

@@ -90,7 +90,7 @@ def test_stream_decode_matches_the_oracle(cuda_device, bits, fmt, lengths, steps
                 compare_records(ocfg, oc, grec, b, h, range((T + 31) // 32), vr_b[h], oc.modality[b])
         cache.records.copy_(torch.from_numpy(oc.records))
         S = splits or m.omnikv_default_splits(consts.struct, cache.struct)
-        part = m.partials_tensor(B, Hq, S + 1, dev)
+        part = m.partials_tensor(B, Hq, S + m._abi.OMNIKV_STREAM_TAIL_SPLITS, dev)
         out = torch.full((B, Hq, 128), float("nan"), device=dev)
         m.omnikv_stream_decode(consts.struct, cache.struct, ring_k, ring_v, q, part, S, out)
         torch.cuda.synchronize()
