@@ -229,3 +229,25 @@ def test_calibration_arguments_rejected():
     assert call(values=A + 8) == _abi.OMNIKV_ERR_INVALID_ARG       # values: 16-byte aligned
     assert call(eigenvalues=A + 4) == _abi.OMNIKV_ERR_INVALID_ARG  # eigenvalues: 8-byte aligned
     assert call(workspace_bytes=need - 1) == _abi.OMNIKV_ERR_CAPACITY
+
+
+def test_streaming_arguments_rejected():
+    """Host checks of the streaming entry points run before any launch."""
+    lib = _abi.load()
+    cfg, cache = _cfg(), _cache()
+
+    def write(ring_k=FAKE, ring_v=FAKE, k=FAKE, v=FAKE, mod=FAKE, n=1, c=None):
+        return lib.omnikv_stream_write_cache(ctypes.byref(cfg), ctypes.byref(c or cache), ring_k, ring_v, k, v, mod,
+                                             n, None)
+
+    def decode(ring_k=FAKE, ring_v=FAKE, q=FAKE, part=FAKE, S=0, out=FAKE):
+        return lib.omnikv_stream_decode(ctypes.byref(cfg), ctypes.byref(cache), ring_k, ring_v, q, part, S, out, None)
+    assert write(ring_k=0) == _abi.OMNIKV_ERR_INVALID_ARG
+    assert write(ring_v=FAKE + 8) == _abi.OMNIKV_ERR_INVALID_ARG        # rings: 16-byte aligned
+    assert write(n=0) == _abi.OMNIKV_ERR_INVALID_ARG
+    assert write(n=4096) == _abi.OMNIKV_ERR_CAPACITY                     # past cap_tokens
+    assert decode(ring_v=0) == _abi.OMNIKV_ERR_INVALID_ARG
+    assert decode(out=0) == _abi.OMNIKV_ERR_INVALID_ARG
+    assert decode(q=0) == _abi.OMNIKV_ERR_INVALID_ARG
+    assert decode(S=-1) == _abi.OMNIKV_ERR_INVALID_ARG
+    assert decode(S=4096) == _abi.OMNIKV_ERR_UNSUPPORTED  # 4096 body splits + 4 tail splits: past the 4096 limit
