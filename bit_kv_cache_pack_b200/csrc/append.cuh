@@ -38,11 +38,10 @@ __device__ __forceinline__ int kp_col(int t, int c) {
 // where ksigma_t == 0) for TurboQuant keys (scales in s_scale[0..31], bounds built
 // without c_0): thread c decides channel c for every token, then the codes are
 // packed 32 / BITS per token-major word.
-template <int BITS>
-__device__ __forceinline__ void key_code_words(WindowSmem& sm, uint8_t* kout, int nvalid, int tid, int bar_id,
-                                               bool turbo) {
+template <int BITS, bool kTurbo>
+__device__ __forceinline__ void key_code_words(WindowSmem& sm, uint8_t* kout, int nvalid, int tid, int bar_id) {
   constexpr int NB = (1 << BITS) - 1, cpw = 32 / BITS, wpt = kHeadDim / cpw;
-  if (!turbo) {
+  if constexpr (!kTurbo) {
     const int c = tid;
     const float s = sm.s_scale[c], m = sm.s_min[c];
     const ScaledBounds<NB> sb = scale_bounds(load_bounds<NB>(sm.bk), s);
@@ -89,6 +88,9 @@ __device__ __forceinline__ void key_code_words(WindowSmem& sm, uint8_t* kout, in
 // touches, in order, so a partial window always keeps its new raw keys in the
 // tail (otherwise only the first touched window does, and finish_write_kernel
 // copies those of a distinct partial last window).
+// kMeta: the key metadata format (kMetaFp16, kMetaMx, kMetaTurbo), a compile-time
+// choice so that each kernel carries only its format's code.
+template <int kMeta>
 __device__ void quantize_window(const WriteParams& p, int b, int h, int w, int L0, int L1, WindowSmem& sm, int tid,
                                 int bar_id, bool tail_any) {
   const int H = p.num_kv_heads;
@@ -97,7 +99,7 @@ __device__ void quantize_window(const WriteParams& p, int b, int h, int w, int L
   const int nvalid = p1 - p0;
   const int inew0 = max(L0 - p0, 0);  // first slot of this window holding a new token
 
-  const RecordLayout lay(p.key_bits, p.value_bits, p.key_meta);
+  const RecordLayout lay(p.key_bits, p.value_bits, kMeta);
   uint8_t* rec = p.records + ((size_t)(b * H + h) * p.cap_windows + w) * lay.bytes;
   const size_t seq_head = (size_t)b * H + h;
   __half* tail = p.key_tail + seq_head * kWindow * kHeadDim;
@@ -114,7 +116,7 @@ __device__ void quantize_window(const WriteParams& p, int b, int h, int w, int L
   const int lane = tid & 31;
   const int LK = 1 << p.key_bits;
   const int LV = 1 << p.value_bits;
-  const bool turbo = p.key_meta == kMetaTurbo;
+  constexpr bool turbo = kMeta == kMetaTurbo;
   const float kc0 = p.key_cb[0];
   if (tid < LK - 1)
     sm.bk[tid] = make_code_bound(__fmul_rn(__fadd_rn(p.key_cb[tid], p.key_cb[tid + 1]), 0.5f), turbo ? 0.0f : kc0);
@@ -217,7 +219,7 @@ __device__ void quantize_window(const WriteParams& p, int b, int h, int w, int L
   // ---- TurboQuant keys: one scale per token from the unrotated fp16 key, the
   // pairwise tree of the value scale (h = 64 across threads q ^ 2, h = 32 across
   // q ^ 1, then h = 16 .. 1 inside the thread's 32 channels)
-  if (turbo) {
+  if constexpr (turbo) {
     float x[32];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -253,7 +255,7 @@ __device__ void quantize_window(const WriteParams& p, int b, int h, int w, int L
       mn = fminf(mn, v);
       mx = fmaxf(mx, v);
     }
-    if (p.key_meta == kMetaMx) {
+    if constexpr (kMeta == kMetaMx) {
       // MXFP4: the warp's 32 channels form one block. The minimum is rounded to
       // the nearest E2M1 value of its block's exponent, then the scale it needs,
       // fp32((max - m^) / (c_last - c_0)) (0 if negative), on the scale block's grid.
@@ -296,9 +298,9 @@ __device__ void quantize_window(const WriteParams& p, int b, int h, int w, int L
 
   // ---- key codes, token-major words -----------------------------------------
   if (p.key_bits == 2)
-    key_code_words<2>(sm, rec + lay.k_off, nvalid, tid, bar_id, turbo);
+    key_code_words<2, turbo>(sm, rec + lay.k_off, nvalid, tid, bar_id);
   else
-    key_code_words<4>(sm, rec + lay.k_off, nvalid, tid, bar_id, turbo);
+    key_code_words<4, turbo>(sm, rec + lay.k_off, nvalid, tid, bar_id);
   group_sync(bar_id);  // kp is reused for values below
 
   // windows filled completely by this write get their values from vrot_tc
@@ -380,6 +382,17 @@ __device__ void quantize_window(const WriteParams& p, int b, int h, int w, int L
   }
 }
 
+
+// quantize_window for the format in p.key_meta (a kernel that serves every format).
+__device__ __forceinline__ void quantize_window_any(const WriteParams& p, int b, int h, int w, int L0, int L1,
+                                                    WindowSmem& sm, int tid, int bar_id, bool tail_any) {
+  if (p.key_meta == kMetaMx)
+    quantize_window<kMetaMx>(p, b, h, w, L0, L1, sm, tid, bar_id, tail_any);
+  else if (p.key_meta == kMetaTurbo)
+    quantize_window<kMetaTurbo>(p, b, h, w, L0, L1, sm, tid, bar_id, tail_any);
+  else
+    quantize_window<kMetaFp16>(p, b, h, w, L0, L1, sm, tid, bar_id, tail_any);
+}
 
 }  // namespace
 }  // namespace omnikv

@@ -1309,7 +1309,11 @@ __global__ void __launch_bounds__(kThreads, body_ctas_per_sm(kBody))
       const int L0 = w.seq_lens[b];
       const int L1 = L0 + 1;
       if (L0 >= 0 && L1 <= w.cap_tokens) {
-        quantize_window(w, b, h, L0 / kWindow, L0, L1, *reinterpret_cast<WindowSmem*>(&sm), threadIdx.x, 1, true);
+        if constexpr (kBody == kBodyGeneric)  // one instance serves every key format
+          quantize_window_any(w, b, h, L0 / kWindow, L0, L1, *reinterpret_cast<WindowSmem*>(&sm), threadIdx.x, 1, true);
+        else
+          quantize_window<kMeta>(w, b, h, L0 / kWindow, L0, L1, *reinterpret_cast<WindowSmem*>(&sm), threadIdx.x, 1,
+                                 true);
         if (h > 0 && threadIdx.x == 0) {  // the decode of head h reads the token's modality after h's flag
           const int m = w.mod_new[b];
           w.modality[(size_t)b * w.cap_tokens + L0] = (uint8_t)(m >= kMods ? kMods - 1 : m);

@@ -23,9 +23,12 @@ namespace omnikv {
 
 namespace {
 
-constexpr int kMaxAppendHeads = 8;  // kv heads of one sequence in one append CTA
+constexpr int kMaxAppendHeads = 4;  // kv heads of one sequence in one append CTA (512 threads: up to 128
+                                    // registers, so the window body does not spill)
 
-// One CTA per (window touched by the new positions, kv head, sequence).
+// One CTA per (window touched by the new positions, kv head, sequence); one
+// instance per key metadata format.
+template <int kMeta>
 __global__ void __launch_bounds__(kWriteThreads) kv_quant_pack_kernel(const WriteParams p) {
   __shared__ WindowSmem sm;
   griddep_launch_dependents();
@@ -39,12 +42,13 @@ __global__ void __launch_bounds__(kWriteThreads) kv_quant_pack_kernel(const Writ
   }
   const int w = L0 / kWindow + blockIdx.x;
   if (w * kWindow >= L1) return;
-  quantize_window(p, b, h, w, L0, L1, sm, threadIdx.x, 1, false);
+  quantize_window<kMeta>(p, b, h, w, L0, L1, sm, threadIdx.x, 1, false);
 }
 
 // Short appends (n_new < 32): one CTA per sequence, one group of 128 threads
 // per kv head; each group re-quantises the (one or two) touched windows in
 // order, and the CTA advances the length itself, so no second launch is needed.
+template <int kMeta>
 __global__ void __launch_bounds__(kWriteThreads * kMaxAppendHeads) kv_append_kernel(const WriteParams p) {
   extern __shared__ __align__(16) uint8_t append_smem[];
   griddep_launch_dependents();
@@ -59,7 +63,7 @@ __global__ void __launch_bounds__(kWriteThreads * kMaxAppendHeads) kv_append_ker
     return;
   }
   for (int w = L0 / kWindow; w * kWindow < L1; ++w) {
-    quantize_window(p, b, grp, w, L0, L1, sm, tid, 1 + grp, true);
+    quantize_window<kMeta>(p, b, grp, w, L0, L1, sm, tid, 1 + grp, true);
     group_sync(1 + grp);  // this window's tail reads are done before the next one writes it
   }
   __syncthreads();  // every group has read the old length
@@ -97,16 +101,20 @@ cudaError_t launch_write(const WriteParams& p_in, int batch, cudaStream_t stream
   if (p.n_new < kWindow && p.num_kv_heads <= kMaxAppendHeads) {
     p.tc_values = 0;
     const size_t smem = sizeof(WindowSmem) * p.num_kv_heads;
+    auto kern = p.key_meta == kMetaMx ? kv_append_kernel<kMetaMx>
+              : p.key_meta == kMetaTurbo ? kv_append_kernel<kMetaTurbo> : kv_append_kernel<kMetaFp16>;
     if (smem > 48 * 1024) {
-      const cudaError_t e = cudaFuncSetAttribute(kv_append_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
     }
-    return launch_pdl(kv_append_kernel, dim3(batch), dim3(kWriteThreads * p.num_kv_heads), smem, stream, p);
+    return launch_pdl(kern, dim3(batch), dim3(kWriteThreads * p.num_kv_heads), smem, stream, p);
   }
   p.tc_values = p.n_new >= kWindow ? 1 : 0;  // a write this long can fill whole windows
   const int slots = (p.n_new + kWindow - 1) / kWindow + 1;
   dim3 grid(slots, p.num_kv_heads, batch);
-  cudaError_t e = launch_pdl(kv_quant_pack_kernel, grid, dim3(kWriteThreads), 0, stream, p);
+  auto pack = p.key_meta == kMetaMx ? kv_quant_pack_kernel<kMetaMx>
+            : p.key_meta == kMetaTurbo ? kv_quant_pack_kernel<kMetaTurbo> : kv_quant_pack_kernel<kMetaFp16>;
+  cudaError_t e = launch_pdl(pack, grid, dim3(kWriteThreads), 0, stream, p);
   if (e != cudaSuccess) return e;
   if (p.tc_values) {
     e = launch_vrot_tc(p, batch, stream);
