@@ -16,6 +16,7 @@ struct __align__(16) WindowSmem {  // 16-byte multiple: per-group copies stay fl
   float s_min[kHeadDim], s_scale[kHeadDim];
   float s_sigma[kWindow];
   CodeBound bk[15], bv[15];  // code decision bounds (keys: after + c_0; values: none added)
+  float tb[kWindow][15];     // TurboQuant keys: each token's bounds scaled by its key scale
   uint8_t codes[kWindow][kHeadDim];  // key codes (token, channel) before packing
 };
 
@@ -52,15 +53,21 @@ __device__ __forceinline__ void key_code_words(WindowSmem& sm, uint8_t* kout, in
                                      ? code_from_scaled(sb, __fsub_rn(sm.kp[t][(t & 1) ? col1 : col0], m))
                                      : 0u);
   } else {
+    if (tid < kWindow) {  // thread t: token t's bounds, once
+      const ScaledBounds<NB> sb = scale_bounds(load_bounds<NB>(sm.bk), sm.s_scale[tid]);
+#pragma unroll
+      for (int j = 0; j < NB; ++j) sm.tb[tid][j] = sb.b[j];
+    }
+    group_sync(bar_id);
     const int c = tid;
-    const CodeBounds<NB> bd = load_bounds<NB>(sm.bk);
     const int col0 = kp_col(0, c), col1 = kp_col(1, c);
 #pragma unroll 2
     for (int t = 0; t < kWindow; ++t) {
       const float s = sm.s_scale[t];
-      sm.codes[t][c] = (uint8_t)((t < nvalid && s != 0.0f)
-                                     ? code_from_scaled(scale_bounds(bd, s), sm.kp[t][(t & 1) ? col1 : col0])
-                                     : 0u);
+      ScaledBounds<NB> sb;
+#pragma unroll
+      for (int j = 0; j < NB; ++j) sb.b[j] = sm.tb[t][j];
+      sm.codes[t][c] = (uint8_t)((t < nvalid && s != 0.0f) ? code_from_scaled(sb, sm.kp[t][(t & 1) ? col1 : col0]) : 0u);
     }
   }
   group_sync(bar_id);
