@@ -56,8 +56,8 @@ META_FORMATS = {"fp16": 0, "mx": 1, "turbo": 2}   # omnikv_config.key_meta_forma
 # next capture.
 TRAFFIC_CAPTURES = {
     ("qwen3-omni-30b-48L-b8-ctx65536", "fp16"): {
-        "sources_sha256": "bcb92b4de243d33d445c563ddb24818b6632cfcad38087d9e68aed22c47e721c",
-        "bytes_per_launch": 173743872 + 8676352},
+        "sources_sha256": "4c93b77c20c49f12f995dd0c422180b174a58631e5304729b8c3a82c18580375",
+        "bytes_per_launch": 173719808 + 8626432},
 }
 KERNEL_SOURCES = ("decode_split_k.cu", "decode_common.cuh", "append.cuh", "common.cuh", "ptx.cuh", "kernels.h")
 
