@@ -91,7 +91,8 @@ int32_t resolve_splits(const omnikv_config* cfg, const omnikv_cache* c, int32_t 
   const int nw = (c->max_seq_len + kWindow - 1) / kWindow;
   if (nw <= 0) return 1;
   const long long units = (long long)c->batch * cfg->num_kv_heads;
-  if (cfg->key_bits != 2 || cfg->value_bits != 2) return wave_splits(units, decode_ctas_per_sm(kBodyGeneric), nw);
+  if (cfg->key_bits != 2 || cfg->value_bits != 2)
+    return wave_splits(units, decode_ctas_per_sm(decode_body(cfg->key_bits, cfg->value_bits, meta_of(cfg->key_meta_format), 0)), nw);
   const int32_t s = wave_splits(units, decode_ctas_per_sm(kBodyCoop), nw);
   if (split_windows_of(c, s) <= kCoopMaxWindows) return s;
   return wave_splits(units, decode_ctas_per_sm(kBodyWarp), nw);
@@ -99,7 +100,7 @@ int32_t resolve_splits(const omnikv_config* cfg, const omnikv_cache* c, int32_t 
 
 // Resident CTAs of a decode-step launch with S splits (the residency of its body).
 long long step_residency(const omnikv_config* cfg, const omnikv_cache* c, int32_t S) {
-  const int body = decode_body(cfg->key_bits, cfg->value_bits, split_windows_of(c, S));
+  const int body = decode_body(cfg->key_bits, cfg->value_bits, meta_of(cfg->key_meta_format), split_windows_of(c, S));
   return (long long)decode_ctas_per_sm(body) * sm_count();
 }
 

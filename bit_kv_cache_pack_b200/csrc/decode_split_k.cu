@@ -179,7 +179,8 @@ __device__ __forceinline__ const __half2* window_meta_pairs(DecodeSmem& sm, cons
 // The split's maximum and denominator of head h; a split whose partial is not
 // finite (inputs outside the fp16 range of the operands) is reported and written
 // empty, so the combine gives it weight 0 and never reads its accumulators.
-__device__ __forceinline__ void write_split_ml(const DecodeParams& p, const DecodeSmem& sm, int b, int kvh, int h,
+template <class Smem>
+__device__ __forceinline__ void write_split_ml(const DecodeParams& p, const Smem& sm, int b, int kvh, int h,
                                                int split, float m, float l) {
   Partial* out = p.partials + ((size_t)b * p.num_kv_heads * p.group + kvh * p.group + h) * p.num_splits + split;
   const bool bad = ((sm.bad_heads >> h) & 1u) || !isfinite(l) || isnan(m) || m == INFINITY;
@@ -1178,6 +1179,506 @@ __device__ __forceinline__ void build_score_operand(DecodeSmem& sm, float k0scal
   }
 }
 
+// ---------------------------------------------------------------------------
+// tensor-core path for 4-bit caches (any codebook): the per-warp body
+// ---------------------------------------------------------------------------
+// A 16-level codebook is not linear in its code bits, so the codewords come from a
+// table: entry j of klut (vlut) holds the fp16 high and low parts of c_j - c_0 (of
+// c_j), hi = fp16(x), lo = fp16(x - hi), which carry x to ~22 bits. The window's
+// key scales move from the A to the B operand of the scores: B = q'_c s_gc 2^-E_w,
+// with a per-window power of two keeping it inside fp16, also as a high + low pair.
+// Each product is A_hi B_hi + A_hi B_lo + A_lo B_hi (A_lo B_lo is below 2^-22 of
+// it), accumulated in fp32: 3 MMAs per 16 x 16 x 8 tile where the 2-bit path needs
+// 4. Tokens are in natural order within a 16-token tile (score row r = value k-slot
+// r = token r), channels in natural order within a 16-channel chunk.
+constexpr int kStages4 = 2;                     // windows in flight per warp
+constexpr int kRec44 = 4672;                    // K4/V4 record bytes with fp16 key metadata (the largest)
+constexpr int kStageBytes4 = kRec44 + kWindow;  // record + modality ids
+
+template <int kMeta>
+struct Rec44 {
+  static constexpr int meta = 2048;
+  static constexpr int v = meta + meta_bytes_of(kMeta);
+  static constexpr int sigma = v + 2048;
+  static constexpr int bytes = sigma + 64;
+};
+
+struct __align__(16) DecodeSmem4 {
+  uint8_t stage[kWarps][kStages4][kStageBytes4];  // per-warp rings; also the final merge buffer
+  float qlane[32][36];  // lane (g, t): q' of head g at channels 16kc + 2t + {0, 1, 8, 9}, kc-major (rows padded)
+  float q[kMaxGroup][kHeadDim];                   // rotated queries (qpos layout), softmax scale folded in
+  uint32_t klut[16], vlut[16];                    // codeword tables: fp16 hi | lo << 16
+  uint64_t bar[kWarps][kStages4];
+  float mw[kWarps][kMaxGroup];
+  float lw[kWarps][kMaxGroup];
+  alignas(16) uint32_t mxpairs[kWarps][kHeadDim]; // MXFP4 caches: a warp's window metadata as fp16 (m, s) pairs
+  float qmax;                                     // max |q'| over the CTA's heads
+  uint32_t tmem_base;
+  uint32_t bad_heads;
+  int wabort[kWarps];
+};
+static_assert(offsetof(DecodeSmem4, qlane) % 16 == 0 && offsetof(DecodeSmem4, mxpairs) % 16 == 0 &&
+                  offsetof(DecodeSmem4, bar) % 8 == 0 && kStageBytes4 % 16 == 0, "aligned fields");
+static_assert(kWarps * 32 * 32 * 4 <= kWarps * kStages4 * kStageBytes4, "merge buffer");
+static_assert(sizeof(WindowSmem) <= sizeof(DecodeSmem4), "append uses the decode shared memory");
+
+__device__ __forceinline__ uint32_t lut_pair_lo(uint32_t e0, uint32_t e1) { return __byte_perm(e0, e1, 0x7632); }
+__device__ __forceinline__ uint32_t lut_pair_hi(uint32_t e0, uint32_t e1) { return __byte_perm(e0, e1, 0x5410); }
+
+// The A operand registers of byte `t` of a code word (two 4-bit codes: the even
+// k-slot in the low nibble): hi and lo parts from the table.
+__device__ __forceinline__ void lut_a(const uint32_t* lut, uint32_t w, int t, uint32_t& hi, uint32_t& lo) {
+  const uint32_t byte = (w >> (8 * t)) & 0xFFu;
+  const uint32_t e0 = lut[byte & 15u], e1 = lut[byte >> 4];
+  hi = lut_pair_hi(e0, e1);
+  lo = lut_pair_lo(e0, e1);
+}
+
+template <int kMeta>
+__device__ __forceinline__ void issue_window4(const DecodeParams& p, DecodeSmem4& sm, int warp, int stage,
+                                              const uint8_t* rec_base, int b, int kvh, int wi, int wait_win,
+                                              int wait_val) {
+  uint64_t* bar = &sm.bar[warp][stage];
+  if (wi == wait_win &&
+      !wait_flag(p.step_flags + (size_t)b * p.num_kv_heads + kvh, wait_val, p.flag_wait_ns)) {
+    set_error(p.error_word, OMNIKV_DEVERR_TIMEOUT);  // no copy of a stale record; the split is written empty
+    sm.wabort[warp] = 1;
+    mbar_arrive_expect_tx(bar, 0);
+    return;
+  }
+  uint8_t* dst = &sm.stage[warp][stage][0];
+  constexpr int rb = Rec44<kMeta>::bytes;
+  mbar_arrive_expect_tx(bar, rb + kWindow);
+  bulk_copy_g2s(dst, rec_base + (size_t)wi * rb, rb, bar);
+  bulk_copy_g2s(dst + rb, p.modality + (size_t)b * p.cap_tokens + (size_t)wi * kWindow, kWindow, bar);
+}
+
+template <int kMeta>
+__device__ void decode_mma4(const DecodeParams& p, DecodeSmem4& sm, int b, int kvh, int split, uint32_t tbase) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int G = p.group;
+  const int Hq = p.num_kv_heads * G;
+  int T, w0, w1;
+  split_range(p, b, split, T, w0, w1);
+  using L = Rec44<kMeta>;
+  const uint8_t* rec_base = p.records + ((size_t)(b * p.num_kv_heads + kvh) * p.cap_windows) * L::bytes;
+  int wa, we, wait_win, wait_val;
+  warp_windows(w0, w1, warp, wa, we);
+  step_window(p, b, wait_win, wait_val);
+  const int nmine = we - wa;
+  if (lane == 0) {
+    sm.wabort[warp] = 0;
+#pragma unroll
+    for (int s = 0; s < kStages4; ++s) mbar_init(&sm.bar[warp][s], 1);
+    fence_barrier_init();
+    for (int i = 0; i < kStages4 && i < nmine; ++i)
+      issue_window4<kMeta>(p, sm, warp, i, rec_base, b, kvh, wa + i, wait_win, wait_val);
+  }
+  __syncwarp();
+
+  WarpState st;
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    st.m[j] = -INFINITY;
+    st.l[j] = 0.0f;
+#pragma unroll
+    for (int m = 0; m < kMods; ++m) st.mref[m][j] = -INFINITY;
+  }
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+    for (int r = 0; r < 4; ++r) st.acc[mt][r] = 0.0f;
+  st.cur = -1;
+  st.parked = 0;
+  const float qmax = sm.qmax;
+
+  int failed_at = -1;
+  for (int i = 0; i < nmine; ++i) {
+    const int s = i % kStages4;
+    const int wi = wa + i;
+    const bool ok = mbar_wait_bounded(&sm.bar[warp][s], (i / kStages4) & 1, kWaitLimitNs) &&
+                    *reinterpret_cast<volatile int*>(&sm.wabort[warp]) == 0;
+    if (!__all_sync(0xffffffffu, ok)) {
+      failed_at = i;
+      break;
+    }
+    const uint8_t* stg = &sm.stage[warp][s][0];
+    const uint32_t* kw = reinterpret_cast<const uint32_t*>(stg);
+    const uint32_t* vw = reinterpret_cast<const uint32_t*>(stg + L::v);
+    const __half* sig = reinterpret_cast<const __half*>(stg + L::sigma);
+    const uint8_t* mods = stg + L::bytes;
+    const __half2* meta;
+    if constexpr (kMeta == kMetaMx) {
+      mx_window_pairs(stg + L::meta, sm.mxpairs[warp], lane);
+      meta = reinterpret_cast<const __half2*>(sm.mxpairs[warp]);
+    } else {
+      meta = reinterpret_cast<const __half2*>(stg + L::meta);
+    }
+
+    // ---- the window's score operand: q'_c s_c 2^-E (hi, lo) at this lane's
+    // B-fragment channels 16kc + 2t + {0, 1, 8, 9}, and the offset sum_c q'_c m_c
+    float qs[32];   // q'_c s_c, then the operand pairs
+    float off = 0.0f, smax = 0.0f;
+    {
+      const float4* ql = reinterpret_cast<const float4*>(&sm.qlane[lane][0]);
+#pragma unroll
+      for (int kc = 0; kc < 8; ++kc) {
+        const float4 q4 = ql[kc];
+        const uint2 ma = *reinterpret_cast<const uint2*>(meta + 16 * kc + 2 * t);      // channels 2t, 2t+1
+        const uint2 mb = *reinterpret_cast<const uint2*>(meta + 16 * kc + 8 + 2 * t);  // channels 8+2t, 9+2t
+        const float2 p0 = __half22float2(*reinterpret_cast<const __half2*>(&ma.x));
+        const float2 p1 = __half22float2(*reinterpret_cast<const __half2*>(&ma.y));
+        const float2 p2 = __half22float2(*reinterpret_cast<const __half2*>(&mb.x));
+        const float2 p3 = __half22float2(*reinterpret_cast<const __half2*>(&mb.y));
+        off = fmaf(q4.x, p0.x, off);
+        off = fmaf(q4.y, p1.x, off);
+        off = fmaf(q4.z, p2.x, off);
+        off = fmaf(q4.w, p3.x, off);
+        smax = fmaxf(smax, fmaxf(fmaxf(fabsf(p0.y), fabsf(p1.y)), fmaxf(fabsf(p2.y), fabsf(p3.y))));
+        qs[4 * kc + 0] = q4.x * p0.y;
+        qs[4 * kc + 1] = q4.y * p1.y;
+        qs[4 * kc + 2] = q4.z * p2.y;
+        qs[4 * kc + 3] = q4.w * p3.y;
+      }
+      off += __shfl_xor_sync(0xffffffffu, off, 1);
+      off += __shfl_xor_sync(0xffffffffu, off, 2);
+      smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 1));
+      smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 2));
+    }
+    const float off0 = __shfl_sync(0xffffffffu, off, 8 * t);      // head 2t
+    const float off1 = __shfl_sync(0xffffffffu, off, 8 * t + 4);  // head 2t + 1
+    // the largest |B| entry at most 2^14
+    const float bmax = qmax * smax;
+    int E = 0;
+    if (bmax > 0.0f && isfinite(bmax)) E = max(-100, min(100, (int)ceilf(log2f(bmax / 16384.0f))));
+    const float bscale = ldexpf(1.0f, -E), escale = ldexpf(1.0f, E);
+    uint32_t bq[8][4];  // per chunk: {hi (2t, 2t+1), hi (8+2t, 9+2t), lo (2t, 2t+1), lo (8+2t, 9+2t)}
+#pragma unroll
+    for (int kc = 0; kc < 8; ++kc) {
+      const float x0 = qs[4 * kc] * bscale, x1 = qs[4 * kc + 1] * bscale;
+      const float x2 = qs[4 * kc + 2] * bscale, x3 = qs[4 * kc + 3] * bscale;
+      const __half2 h01 = __floats2half2_rn(x0, x1), h23 = __floats2half2_rn(x2, x3);
+      const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+      const __half2 l01 = __floats2half2_rn(x0 - f01.x, x1 - f01.y), l23 = __floats2half2_rn(x2 - f23.x, x3 - f23.y);
+      bq[kc][0] = *reinterpret_cast<const uint32_t*>(&h01);
+      bq[kc][1] = *reinterpret_cast<const uint32_t*>(&h23);
+      bq[kc][2] = *reinterpret_cast<const uint32_t*>(&l01);
+      bq[kc][3] = *reinterpret_cast<const uint32_t*>(&l23);
+    }
+
+    // ---- scores of the two 16-token tiles: rows g, g + 8 = tokens 16h + g, 16h + g + 8
+    float sc[2][4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int tokA = 16 * h + g, tokB = tokA + 8;
+      const uint4* ka = reinterpret_cast<const uint4*>(kw + tokA * 16);
+      const uint4* kb = reinterpret_cast<const uint4*>(kw + tokB * 16);
+      float d[4] = {0.f, 0.f, 0.f, 0.f}, e[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        const uint4 wa4 = ka[q4], wb4 = kb[q4];  // words 4 q4 .. 4 q4 + 3: chunks 2 q4, 2 q4 + 1
+        const uint32_t wa[4] = {wa4.x, wa4.y, wa4.z, wa4.w}, wb[4] = {wb4.x, wb4.y, wb4.z, wb4.w};
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int kc = 2 * q4 + half;
+          uint32_t ahi[4], alo[4];
+          lut_a(sm.klut, wa[2 * half], t, ahi[0], alo[0]);      // row g, k-slots 2t, 2t+1
+          lut_a(sm.klut, wb[2 * half], t, ahi[1], alo[1]);      // row g + 8
+          lut_a(sm.klut, wa[2 * half + 1], t, ahi[2], alo[2]);  // row g, k-slots 2t+8, 2t+9
+          lut_a(sm.klut, wb[2 * half + 1], t, ahi[3], alo[3]);  // row g + 8
+          mma_f16_16816(d, ahi, bq[kc][0], bq[kc][1]);
+          mma_f16_16816(e, ahi, bq[kc][2], bq[kc][3]);
+          mma_f16_16816(e, alo, bq[kc][0], bq[kc][1]);
+        }
+      }
+      const int posA = wi * kWindow + tokA, posB = wi * kWindow + tokB;
+      sc[h][0] = posA < T ? fmaf(d[0] + e[0], escale, off0) : -INFINITY;
+      sc[h][1] = posA < T ? fmaf(d[1] + e[1], escale, off1) : -INFINITY;
+      sc[h][2] = posB < T ? fmaf(d[2] + e[2], escale, off0) : -INFINITY;
+      sc[h][3] = posB < T ? fmaf(d[3] + e[3], escale, off1) : -INFINITY;
+    }
+
+    // ---- online softmax over the window
+    float mx0 = fmaxf(fmaxf(sc[0][0], sc[0][2]), fmaxf(sc[1][0], sc[1][2]));
+    float mx1 = fmaxf(fmaxf(sc[0][1], sc[0][3]), fmaxf(sc[1][1], sc[1][3]));
+#pragma unroll
+    for (int o = 4; o <= 16; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+    }
+    const float mn0 = fmaxf(st.m[0], mx0), mn1 = fmaxf(st.m[1], mx1);
+    if (__any_sync(0xffffffffu, mn0 > st.m[0] || mn1 > st.m[1])) {
+      const float a0 = fast_exp2((st.m[0] - mn0) * kLog2e), a1 = fast_exp2((st.m[1] - mn1) * kLog2e);
+      st.l[0] *= a0;
+      st.l[1] *= a1;
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt) {
+        st.acc[mt][0] *= a0;
+        st.acc[mt][1] *= a1;
+        st.acc[mt][2] *= a0;
+        st.acc[mt][3] *= a1;
+      }
+      st.m[0] = mn0;
+      st.m[1] = mn1;
+    }
+    const float ms0 = st.m[0] * kLog2e, ms1 = st.m[1] * kLog2e;
+
+    // ---- value product per tile: rows g, g + 8 of m-tile mt = channels 16g + 2mt,
+    // 16g + 2mt + 1; k-slots 2t, 2t+1 (2t+8, 2t+9) = tokens 16h + 2t, +1 (+8)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int tokA = 16 * h + g, tokB = tokA + 8;
+      const float p0 = fast_exp2(fmaf(sc[h][0], kLog2e, -ms0));
+      const float p1 = fast_exp2(fmaf(sc[h][1], kLog2e, -ms1));
+      const float p2 = fast_exp2(fmaf(sc[h][2], kLog2e, -ms0));
+      const float p3 = fast_exp2(fmaf(sc[h][3], kLog2e, -ms1));
+      st.l[0] += p0 + p2;
+      st.l[1] += p1 + p3;
+      const float sgA = __half2float(sig[tokA]), sgB = __half2float(sig[tokB]);
+      const float w0v = p0 * sgA, w1v = p1 * sgA, w2v = p2 * sgB, w3v = p3 * sgB;
+      uint32_t bv[4];  // {hi (k 0..7), hi (k 8..15), lo (k 0..7), lo (k 8..15)}, transposed
+      split_pair_t(w0v, w1v, bv[0], bv[2]);
+      split_pair_t(w2v, w3v, bv[1], bv[3]);
+      const int mA = min((int)mods[tokA], 2), mB = min((int)mods[tokB], 2);
+      const uint32_t mbits = __reduce_or_sync(0xffffffffu, (1u << mA) | (1u << mB));
+      const int base = 16 * h;
+      const int mk0 = min((int)mods[base + 2 * t], 2), mk1 = min((int)mods[base + 2 * t + 1], 2);
+      const int mk2 = min((int)mods[base + 8 + 2 * t], 2), mk3 = min((int)mods[base + 9 + 2 * t], 2);
+      const uint4* r0 = reinterpret_cast<const uint4*>(vw + (2 * h) * kHeadDim + 16 * g);      // tokens 16h .. +7
+      const uint4* r1 = reinterpret_cast<const uint4*>(vw + (2 * h + 1) * kHeadDim + 16 * g);  // tokens 16h+8 .. +15
+      uint32_t todo = mbits;
+      int mm = (st.cur >= 0 && ((todo >> st.cur) & 1u)) ? st.cur : __ffs(todo) - 1;
+#pragma unroll 1
+      while (true) {
+        activate(st, mm, tbase, warp);
+        const bool single = mbits == (1u << mm);
+        const uint32_t msk01 = single ? 0xFFFFFFFFu : ((mk0 == mm ? 0x0000FFFFu : 0u) | (mk1 == mm ? 0xFFFF0000u : 0u));
+        const uint32_t msk23 = single ? 0xFFFFFFFFu : ((mk2 == mm ? 0x0000FFFFu : 0u) | (mk3 == mm ? 0xFFFF0000u : 0u));
+        const uint32_t bh0 = bv[0] & msk01, bh1 = bv[1] & msk23, bl0 = bv[2] & msk01, bl1 = bv[3] & msk23;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const uint4 u0w = r0[q4], u1w = r1[q4];  // channels 16g + 4 q4 .. + 3
+          const uint32_t x0[4] = {u0w.x, u0w.y, u0w.z, u0w.w}, x1[4] = {u1w.x, u1w.y, u1w.z, u1w.w};
+#pragma unroll
+          for (int e2 = 0; e2 < 2; ++e2) {
+            const int mt = 2 * q4 + e2;
+            uint32_t ahi[4], alo[4];
+            lut_a(sm.vlut, x0[2 * e2], t, ahi[0], alo[0]);      // channel 16g + 2mt, tokens 2t, 2t+1
+            lut_a(sm.vlut, x0[2 * e2 + 1], t, ahi[1], alo[1]);  // channel 16g + 2mt + 1
+            lut_a(sm.vlut, x1[2 * e2], t, ahi[2], alo[2]);      // channel 16g + 2mt, tokens 8+2t, 9+2t
+            lut_a(sm.vlut, x1[2 * e2 + 1], t, ahi[3], alo[3]);
+            mma_f16_16816(st.acc[mt], ahi, bh0, bh1);
+            mma_f16_16816(st.acc[mt], ahi, bl0, bl1);
+            mma_f16_16816(st.acc[mt], alo, bh0, bh1);
+          }
+        }
+        todo &= ~(1u << mm);
+        if (!todo) break;
+        mm = __ffs(todo) - 1;
+      }
+    }
+    __syncwarp();
+    if (lane == 0 && i + kStages4 < nmine) {
+      fence_proxy_async_smem();
+      issue_window4<kMeta>(p, sm, warp, s, rec_base, b, kvh, wa + i + kStages4, wait_win, wait_val);
+    }
+  }
+
+  if (__any_sync(0xffffffffu, failed_at >= 0)) {
+    const int f = __shfl_sync(0xffffffffu, failed_at, 0);
+    if (lane == 0) set_error(p.error_word, OMNIKV_DEVERR_TIMEOUT);
+    for (int j = f; j < nmine && j < f + kStages4; ++j)
+      mbar_wait_bounded(&sm.bar[warp][j % kStages4], (j / kStages4) & 1, kWaitLimitNs);
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      st.m[j] = -INFINITY;
+      st.l[j] = 0.0f;
+    }
+    st.cur = -1;
+    st.parked = 0;
+  }
+  if (st.cur >= 0) park_active(st, tbase, warp);
+
+  // ---- reduce the per-lane denominators over the 8 lanes sharing a column
+#pragma unroll
+  for (int o = 4; o <= 16; o <<= 1) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) st.l[j] += __shfl_xor_sync(0xffffffffu, st.l[j], o);
+  }
+  // ---- merge the 4 warps at their common max, one modality at a time
+  if (g == 0) {
+    sm.mw[warp][2 * t] = st.m[0];
+    sm.mw[warp][2 * t + 1] = st.m[1];
+  }
+  __syncthreads();  // also: all warps are done with their stage buffers
+  float M[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    float mm = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) mm = fmaxf(mm, sm.mw[w][2 * t + j]);
+    M[j] = mm;
+    const float f = (st.m[j] == -INFINITY) ? 0.0f : fast_exp2((st.m[j] - mm) * kLog2e);
+    st.l[j] *= f;
+  }
+  if (g == 0) {
+    sm.lw[warp][2 * t] = st.l[0];
+    sm.lw[warp][2 * t + 1] = st.l[1];
+  }
+  float* xbuf = reinterpret_cast<float*>(&sm.stage[0][0][0]);  // [warp][32 registers][32 lanes]
+#pragma unroll
+  for (int m = 0; m < kMods; ++m) {
+    unpark(st, m, tbase, warp, M[0], M[1]);  // zeros if this warp never saw modality m
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) xbuf[(warp * 32 + mt * 4 + r) * 32 + lane] = st.acc[mt][r];
+    __syncthreads();
+#pragma unroll
+    for (int e2 = 0; e2 < 2; ++e2) {
+      const int mt = 2 * warp + e2;
+      float v[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        float x = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) x += xbuf[(w * 32 + mt * 4 + r) * 32 + lane];
+        v[r] = x;
+      }
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int hh = 2 * t + j;
+        if (hh >= G) continue;
+        Partial* out = p.partials + ((size_t)b * Hq + kvh * G + hh) * p.num_splits + split;
+        *reinterpret_cast<float2*>(&out->acc[m][16 * g + 2 * mt]) = make_float2(v[j], v[j + 2]);
+        if (!isfinite(v[j]) || !isfinite(v[j + 2])) atomicOr(&sm.bad_heads, 1u << hh);
+      }
+    }
+    __syncthreads();
+  }
+  if (warp == 0 && g == 0) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int hh = 2 * t + j;
+      if (hh >= G) continue;
+      float l = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) l += sm.lw[w][hh];
+      write_split_ml(p, sm, b, kvh, hh, split, M[j], l);
+    }
+  }
+}
+
+// One decode CTA of the 4-bit tensor-core body.
+template <int kMeta>
+__device__ __forceinline__ void decode_cta4(const DecodeParams& p, DecodeSmem4& sm, int b, int kvh, int split) {
+  {
+    const size_t ubytes = (size_t)kMods * kHeadDim * kHeadDim * sizeof(float);
+    const size_t share = (ubytes + p.num_splits - 1) / p.num_splits;
+    const char* ub = reinterpret_cast<const char*>(p.value_rot) + (size_t)kvh * ubytes;
+    for (size_t off = (size_t)split * share + 128 * threadIdx.x; off < min(ubytes, (size_t)(split + 1) * share);
+         off += 128 * kThreads)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(ub + off));
+  }
+  rotate_queries(p, b, kvh, &sm.q[0][0]);
+  if (threadIdx.x < 16) {  // codeword tables: c_j - c_0 (keys), c_j (values), as fp16 hi | lo
+    const int j = threadIdx.x;
+    const int LK = 1 << p.key_bits, LV = 1 << p.value_bits;
+    const float dk = j < LK ? p.key_cb[j] - p.key_cb[0] : 0.0f;
+    const float dv = j < LV ? p.val_cb[j] : 0.0f;
+    const __half hk = __float2half_rn(dk), hv = __float2half_rn(dv);
+    const __half lk = __float2half_rn(dk - __half2float(hk)), lv = __float2half_rn(dv - __half2float(hv));
+    sm.klut[j] = (uint32_t)__half_as_ushort(hk) | ((uint32_t)__half_as_ushort(lk) << 16);
+    sm.vlut[j] = (uint32_t)__half_as_ushort(hv) | ((uint32_t)__half_as_ushort(lv) << 16);
+  }
+  if (threadIdx.x == 0) sm.bad_heads = 0u;
+  __syncthreads();  // every warp's rotated queries are written
+  {
+    float qm = 0.0f;
+    for (int e = threadIdx.x; e < kMaxGroup * kHeadDim; e += kThreads) qm = fmaxf(qm, fabsf((&sm.q[0][0])[e]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) qm = fmaxf(qm, __shfl_xor_sync(0xffffffffu, qm, o));
+    if ((threadIdx.x & 31) == 0) sm.lw[threadIdx.x >> 5][0] = qm;
+    // the lanes' B-fragment copy of the queries: lane (g, t), chunk kc: channels
+    // 16kc + 2t, 16kc + 2t + 1, 16kc + 8 + 2t, 16kc + 9 + 2t of head g
+    for (int e = threadIdx.x; e < 32 * 32; e += kThreads) {
+      const int ln = e >> 5, j = e & 31;
+      const int gg = ln >> 2, tt = ln & 3, kc = j >> 2, r = j & 3;
+      sm.qlane[ln][j] = sm.q[0][qpos(gg, 16 * kc + 2 * tt + (r & 1) + 8 * (r >> 1))];
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) sm.qmax = fmaxf(fmaxf(sm.lw[0][0], sm.lw[1][0]), fmaxf(sm.lw[2][0], sm.lw[3][0]));
+  __syncthreads();
+
+  griddep_wait();  // lengths and records may come from the previous launch
+  int T, w0, w1;
+  split_range(p, b, split, T, w0, w1);
+  if (w0 == w1) {
+    if (threadIdx.x < p.group) {
+      Partial* out = p.partials + ((size_t)b * p.num_kv_heads * p.group + kvh * p.group + threadIdx.x) * p.num_splits + split;
+      out->m = -INFINITY;
+      out->l = 0.0f;
+    }
+    return;
+  }
+  if (threadIdx.x < 32) tmem_alloc(&sm.tmem_base, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = sm.tmem_base;
+  decode_mma4<kMeta>(p, sm, b, kvh, split, tbase);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (threadIdx.x < 32) tmem_dealloc(tbase, kTmemCols);
+}
+
+template <int kMeta>
+__global__ void __launch_bounds__(kThreads, 2) decode_split_k4_kernel(const DecodeParams p) {
+  extern __shared__ __align__(16) uint8_t k4_smem[];
+  DecodeSmem4& sm = *reinterpret_cast<DecodeSmem4*>(k4_smem);
+  griddep_launch_dependents();
+  decode_cta4<kMeta>(p, sm, blockIdx.z, blockIdx.y, blockIdx.x);
+}
+
+template <int kMeta>
+__global__ void __launch_bounds__(kThreads, 2) decode_step4_kernel(const DecodeParams p, const WriteParams w) {
+  extern __shared__ __align__(16) uint8_t k4_smem[];
+  DecodeSmem4& sm = *reinterpret_cast<DecodeSmem4*>(k4_smem);
+  griddep_launch_dependents();
+  const int H = p.num_kv_heads;
+  const int nappend = p.append_ctas;
+  if ((int)blockIdx.x < nappend) {
+    griddep_wait();
+    for (int u = blockIdx.x; u < p.batch * H; u += nappend) {
+      const int b = u / H, h = u % H;
+      const int L0 = w.seq_lens[b];
+      const int L1 = L0 + 1;
+      if (L0 >= 0 && L1 <= w.cap_tokens) {
+        quantize_window<kMeta>(w, b, h, L0 / kWindow, L0, L1, *reinterpret_cast<WindowSmem*>(&sm), threadIdx.x, 1,
+                               true);
+        if (h > 0 && threadIdx.x == 0) {  // the decode of head h reads the token's modality after h's flag
+          const int m = w.mod_new[b];
+          w.modality[(size_t)b * w.cap_tokens + L0] = (uint8_t)(m >= kMods ? kMods - 1 : m);
+        }
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x == 0)
+          asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(w.step_flags + (size_t)b * H + h), "r"(L1)
+                       : "memory");
+      } else if (threadIdx.x == 0 && h == 0) {
+        set_error(w.error_word, OMNIKV_DEVERR_CAPACITY);
+      }
+      __syncthreads();  // the shared memory is the next unit's
+    }
+    return;
+  }
+  const int r = blockIdx.x - nappend;
+  decode_cta4<kMeta>(p, sm, r / (p.num_splits * H), (r / p.num_splits) % H, r % p.num_splits);
+}
+
 // One decode CTA: split `split` of kv head kvh of sequence b. kBody: the 4-bit
 // build (CUDA-core path only, no TMEM, more CTAs per SM), or a tensor-core build
 // (per-warp or cooperative body), whose kernels fall back to the CUDA-core path for
@@ -1351,6 +1852,29 @@ cudaError_t prefer_shared_carveout(Kernel kernel, std::atomic<uint64_t>& done) {
 
 std::atomic<uint64_t> g_carveout[2][kNumBodies][3];  // [decode, step][body][key metadata format]
 
+// The 4-bit tensor-core kernels take their shared memory dynamically (above the
+// 48 KB static limit): the attribute and the carveout, set once per device.
+template <typename Kernel>
+cudaError_t prepare_dynamic(Kernel kernel, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (1ull << dev) : 0ull;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(DecodeSmem4));
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
+
+template <int kMeta>
+cudaError_t prepare_tc4() {
+  const cudaError_t e = prepare_dynamic(decode_split_k4_kernel<kMeta>, g_carveout[0][kBodyTc4][kMeta]);
+  if (e != cudaSuccess) return e;
+  return prepare_dynamic(decode_step4_kernel<kMeta>, g_carveout[1][kBodyTc4][kMeta]);
+}
+
 template <int kBody, int kMeta>
 cudaError_t prepare_body() {
   const cudaError_t e = prefer_shared_carveout(decode_split_k_kernel<kBody, kMeta>, g_carveout[0][kBody][kMeta]);
@@ -1361,6 +1885,7 @@ cudaError_t prepare_body() {
 // The 4-bit build reads the metadata format at run time: one instance.
 cudaError_t prepare_kernels(int body, int meta) {
   if (body == kBodyGeneric) return prepare_body<kBodyGeneric, kMetaFp16>();
+  if (body == kBodyTc4) return meta == kMetaMx ? prepare_tc4<kMetaMx>() : prepare_tc4<kMetaFp16>();
   if (meta == kMetaMx) return body == kBodyWarp ? prepare_body<kBodyWarp, kMetaMx>() : prepare_body<kBodyCoop, kMetaMx>();
   if (meta == kMetaTurbo)
     return body == kBodyWarp ? prepare_body<kBodyWarp, kMetaTurbo>() : prepare_body<kBodyCoop, kMetaTurbo>();
@@ -1395,9 +1920,32 @@ cudaError_t body_attributes(cudaFuncAttributes* a) {
   return cudaSuccess;
 }
 
+template <int kMeta>
+cudaError_t tc4_attributes_of(cudaFuncAttributes* a) {
+  cudaError_t e = cudaFuncGetAttributes(a, decode_step4_kernel<kMeta>);
+  if (e != cudaSuccess) return e;
+  cudaFuncAttributes a2;
+  if ((e = cudaFuncGetAttributes(&a2, decode_split_k4_kernel<kMeta>)) != cudaSuccess) return e;
+  if (a2.numRegs > a->numRegs) a->numRegs = a2.numRegs;
+  if (a2.sharedSizeBytes > a->sharedSizeBytes) a->sharedSizeBytes = a2.sharedSizeBytes;
+  a->sharedSizeBytes += sizeof(DecodeSmem4);
+  return cudaSuccess;
+}
+
+cudaError_t tc4_attributes(cudaFuncAttributes* a) {
+  cudaError_t e = tc4_attributes_of<kMetaFp16>(a);
+  if (e != cudaSuccess) return e;
+  cudaFuncAttributes a2;
+  if ((e = tc4_attributes_of<kMetaMx>(&a2)) != cudaSuccess) return e;
+  if (a2.numRegs > a->numRegs) a->numRegs = a2.numRegs;
+  if (a2.sharedSizeBytes > a->sharedSizeBytes) a->sharedSizeBytes = a2.sharedSizeBytes;
+  return cudaSuccess;
+}
+
 }  // namespace
 
-int decode_body(int key_bits, int value_bits, int split_windows) {
+int decode_body(int key_bits, int value_bits, int key_meta, int split_windows) {
+  if (key_bits == 4 && value_bits == 4 && key_meta != kMetaTurbo) return kBodyTc4;
   if (key_bits != 2 || value_bits != 2) return kBodyGeneric;
   return split_windows <= kCoopMaxWindows ? kBodyCoop : kBodyWarp;
 }
@@ -1420,10 +1968,11 @@ int decode_ctas_per_sm(int body) {
   int regs_sm = 0, smem_sm = 0, smem_rsv = 0;
   const cudaError_t ea = body == kBodyWarp ? body_attributes<kBodyWarp>(&a)
                        : body == kBodyCoop ? body_attributes<kBodyCoop>(&a)
+                       : body == kBodyTc4  ? tc4_attributes(&a)
                                            : body_attributes<kBodyGeneric>(&a);
   if (prepare_kernels(body, kMetaFp16) != cudaSuccess ||
-      (body != kBodyGeneric && (prepare_kernels(body, kMetaMx) != cudaSuccess ||
-                                prepare_kernels(body, kMetaTurbo) != cudaSuccess)) ||
+      (body != kBodyGeneric && prepare_kernels(body, kMetaMx) != cudaSuccess) ||
+      ((body == kBodyWarp || body == kBodyCoop) && prepare_kernels(body, kMetaTurbo) != cudaSuccess) ||
       ea != cudaSuccess ||
       cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
@@ -1432,19 +1981,22 @@ int decode_ctas_per_sm(int body) {
   const int warp_regs = ((a.numRegs * 32 + 255) / 256) * 256;  // allocated per warp in units of 256
   const int by_regs = regs_sm / (warp_regs * kWarps);
   const int by_smem = smem_sm / ((int)a.sharedSizeBytes + smem_rsv);
-  const int by_tmem = body == kBodyWarp ? 512 / (int)kTmemCols : 64;  // only the per-warp body holds tensor memory
+  const int by_tmem = (body == kBodyWarp || body == kBodyTc4) ? 512 / (int)kTmemCols : 64;  // per-warp bodies hold tensor memory
   const int n = max(1, min(by_regs, min(by_smem, by_tmem)));
   if (dev < 64) cached[body][dev].store(n, std::memory_order_relaxed);
   return n;
 }
 
 cudaError_t launch_decode_step(const DecodeParams& p, const WriteParams& w, cudaStream_t stream) {
-  const int body = decode_body(p.key_bits, p.value_bits, p.split_windows);
   const int meta = p.key_meta;
+  const int body = decode_body(p.key_bits, p.value_bits, meta, p.split_windows);
   const cudaError_t e = prepare_kernels(body, meta);
   if (e != cudaSuccess) return e;
   const dim3 grid(p.append_ctas + p.batch * p.num_kv_heads * p.num_splits);
   const dim3 block(kThreads);
+  if (body == kBodyTc4)
+    return meta == kMetaMx ? launch_pdl(decode_step4_kernel<kMetaMx>, grid, block, sizeof(DecodeSmem4), stream, p, w)
+                           : launch_pdl(decode_step4_kernel<kMetaFp16>, grid, block, sizeof(DecodeSmem4), stream, p, w);
   if (body == kBodyGeneric) return launch_pdl(decode_step_kernel<kBodyGeneric, kMetaFp16>, grid, block, 0, stream, p, w);
   if (meta == kMetaMx)
     return body == kBodyWarp ? launch_pdl(decode_step_kernel<kBodyWarp, kMetaMx>, grid, block, 0, stream, p, w)
@@ -1457,12 +2009,15 @@ cudaError_t launch_decode_step(const DecodeParams& p, const WriteParams& w, cuda
 }
 
 cudaError_t launch_decode(const DecodeParams& p, int batch, cudaStream_t stream) {
-  const int body = decode_body(p.key_bits, p.value_bits, p.split_windows);
   const int meta = p.key_meta;
+  const int body = decode_body(p.key_bits, p.value_bits, meta, p.split_windows);
   const cudaError_t e = prepare_kernels(body, meta);
   if (e != cudaSuccess) return e;
   const dim3 grid(p.num_splits, p.num_kv_heads, batch);
   const dim3 block(kThreads);
+  if (body == kBodyTc4)
+    return meta == kMetaMx ? launch_pdl(decode_split_k4_kernel<kMetaMx>, grid, block, sizeof(DecodeSmem4), stream, p)
+                           : launch_pdl(decode_split_k4_kernel<kMetaFp16>, grid, block, sizeof(DecodeSmem4), stream, p);
   if (body == kBodyGeneric) return launch_pdl(decode_split_k_kernel<kBodyGeneric, kMetaFp16>, grid, block, 0, stream, p);
   if (meta == kMetaMx)
     return body == kBodyWarp ? launch_pdl(decode_split_k_kernel<kBodyWarp, kMetaMx>, grid, block, 0, stream, p)
