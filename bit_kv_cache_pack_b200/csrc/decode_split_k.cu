@@ -1180,35 +1180,40 @@ __device__ __forceinline__ void build_score_operand(DecodeSmem& sm, float k0scal
 }
 
 // ---------------------------------------------------------------------------
-// tensor-core path for 4-bit caches (any codebook): the per-warp body
+// tensor-core path for 4-bit caches over codeword tables: the per-warp table body
 // ---------------------------------------------------------------------------
-// A 16-level codebook is not linear in its code bits, so the codewords come from a
-// table: entry j of klut (vlut) holds the fp16 high and low parts of c_j - c_0 (of
-// c_j), hi = fp16(x), lo = fp16(x - hi), which carry x to ~22 bits. The window's
-// key scales move from the A to the B operand of the scores: B = q'_c s_gc 2^-E_w,
-// with a per-window power of two keeping it inside fp16, also as a high + low pair.
-// Each product is A_hi B_hi + A_hi B_lo + A_lo B_hi (A_lo B_lo is below 2^-22 of
-// it), accumulated in fp32: 3 MMAs per 16 x 16 x 8 tile where the 2-bit path needs
-// 4. Tokens are in natural order within a 16-token tile (score row r = value k-slot
-// r = token r), channels in natural order within a 16-channel chunk.
-constexpr int kStages4 = 2;                     // windows in flight per warp
-constexpr int kRec44 = 4672;                    // K4/V4 record bytes with fp16 key metadata (the largest)
-constexpr int kStageBytes4 = kRec44 + kWindow;  // record + modality ids
+// A 16-level codebook is not linear in its code bits, so the codewords come from
+// shared-memory tables, and the codebook needs no symmetry: each codeword is held
+// as an fp16 high and low part, hi = fp16(x), lo = fp16(x - hi), which carry x to
+// ~22 bits (keys: c_j - c_0, values: c_j). The window's key scales move from the A
+// to the B operand of the scores: B = q'_c s_gc 2^-E_w, with a per-window power of
+// two keeping it inside fp16, also as a high + low pair. Each product is
+// A_hi B_hi + A_hi B_lo + A_lo B_hi (A_lo B_lo is below 2^-22 of it), accumulated in
+// fp32: 3 MMAs per 16 x 16 x 8 tile; a register's two k-slots come from one code
+// byte. Tokens are in natural order within a 16-token tile (score row r = value
+// k-slot r = token r), channels in natural order within a 16-channel chunk.
+// (The same tables serve 2-bit codes in a register per code nibble, but there the
+// bit-plane bodies above are faster: 235.5 against 200.7 us per layer on the
+// 8 x 65,536-token decode.)
+constexpr int kLutRing = 9408;  // per-warp record ring: 2 windows of K4/V4 with fp16 metadata
 
 template <int kMeta>
-struct Rec44 {
-  static constexpr int meta = 2048;
+struct RecLut {
+  static constexpr int meta = 2048;                       // key codes: 32 tokens x 128 channels x 4 bits
   static constexpr int v = meta + meta_bytes_of(kMeta);
-  static constexpr int sigma = v + 2048;
+  static constexpr int sigma = v + 2048;                  // value codes
   static constexpr int bytes = sigma + 64;
+  static constexpr int stage = bytes + kWindow;           // record + modality ids
+  static constexpr int stages = kLutRing / stage;
+  static_assert(stage % 16 == 0 && stages >= 2, "ring of 16-byte aligned stages");
 };
 
-struct __align__(16) DecodeSmem4 {
-  uint8_t stage[kWarps][kStages4][kStageBytes4];  // per-warp rings; also the final merge buffer
+struct __align__(16) DecodeSmemLut {
+  uint8_t ring[kWarps][kLutRing];  // per-warp record rings; also the final merge buffer
   float qlane[32][36];  // lane (g, t): q' of head g at channels 16kc + 2t + {0, 1, 8, 9}, kc-major (rows padded)
   float q[kMaxGroup][kHeadDim];                   // rotated queries (qpos layout), softmax scale folded in
-  uint32_t klut[16], vlut[16];                    // codeword tables: fp16 hi | lo << 16
-  uint64_t bar[kWarps][kStages4];
+  uint32_t klut[16], vlut[16];                    // tables: fp16 hi | lo << 16 of each codeword
+  uint64_t bar[kWarps][2];
   float mw[kWarps][kMaxGroup];
   float lw[kWarps][kMaxGroup];
   alignas(16) uint32_t mxpairs[kWarps][kHeadDim]; // MXFP4 caches: a warp's window metadata as fp16 (m, s) pairs
@@ -1217,27 +1222,26 @@ struct __align__(16) DecodeSmem4 {
   uint32_t bad_heads;
   int wabort[kWarps];
 };
-static_assert(offsetof(DecodeSmem4, qlane) % 16 == 0 && offsetof(DecodeSmem4, mxpairs) % 16 == 0 &&
-                  offsetof(DecodeSmem4, bar) % 8 == 0 && kStageBytes4 % 16 == 0, "aligned fields");
-static_assert(kWarps * 32 * 32 * 4 <= kWarps * kStages4 * kStageBytes4, "merge buffer");
-static_assert(sizeof(WindowSmem) <= sizeof(DecodeSmem4), "append uses the decode shared memory");
+static_assert(offsetof(DecodeSmemLut, qlane) % 16 == 0 && offsetof(DecodeSmemLut, mxpairs) % 16 == 0 &&
+                  offsetof(DecodeSmemLut, bar) % 8 == 0 && kLutRing % 16 == 0, "aligned fields");
+static_assert(kWarps * 32 * 32 * 4 <= kWarps * kLutRing, "merge buffer");
+static_assert(sizeof(WindowSmem) <= sizeof(DecodeSmemLut), "append uses the decode shared memory");
+static_assert(RecLut<kMetaFp16>::stages == 2 && RecLut<kMetaMx>::stages == 2, "barriers per warp");
 
-__device__ __forceinline__ uint32_t lut_pair_lo(uint32_t e0, uint32_t e1) { return __byte_perm(e0, e1, 0x7632); }
-__device__ __forceinline__ uint32_t lut_pair_hi(uint32_t e0, uint32_t e1) { return __byte_perm(e0, e1, 0x5410); }
-
-// The A operand registers of byte `t` of a code word (two 4-bit codes: the even
-// k-slot in the low nibble): hi and lo parts from the table.
-__device__ __forceinline__ void lut_a(const uint32_t* lut, uint32_t w, int t, uint32_t& hi, uint32_t& lo) {
+// The A operand registers of byte `t` of a code word (two codes: the even k-slot in
+// the low nibble): hi and lo parts from the table.
+__device__ __forceinline__ void lut4_a(const uint32_t* lut, uint32_t w, int t, uint32_t& hi, uint32_t& lo) {
   const uint32_t byte = (w >> (8 * t)) & 0xFFu;
   const uint32_t e0 = lut[byte & 15u], e1 = lut[byte >> 4];
-  hi = lut_pair_hi(e0, e1);
-  lo = lut_pair_lo(e0, e1);
+  hi = __byte_perm(e0, e1, 0x5410);
+  lo = __byte_perm(e0, e1, 0x7632);
 }
 
 template <int kMeta>
-__device__ __forceinline__ void issue_window4(const DecodeParams& p, DecodeSmem4& sm, int warp, int stage,
-                                              const uint8_t* rec_base, int b, int kvh, int wi, int wait_win,
-                                              int wait_val) {
+__device__ __forceinline__ void issue_window_lut(const DecodeParams& p, DecodeSmemLut& sm, int warp, int stage,
+                                                 const uint8_t* rec_base, int b, int kvh, int wi, int wait_win,
+                                                 int wait_val) {
+  using L = RecLut<kMeta>;
   uint64_t* bar = &sm.bar[warp][stage];
   if (wi == wait_win &&
       !wait_flag(p.step_flags + (size_t)b * p.num_kv_heads + kvh, wait_val, p.flag_wait_ns)) {
@@ -1246,22 +1250,22 @@ __device__ __forceinline__ void issue_window4(const DecodeParams& p, DecodeSmem4
     mbar_arrive_expect_tx(bar, 0);
     return;
   }
-  uint8_t* dst = &sm.stage[warp][stage][0];
-  constexpr int rb = Rec44<kMeta>::bytes;
-  mbar_arrive_expect_tx(bar, rb + kWindow);
-  bulk_copy_g2s(dst, rec_base + (size_t)wi * rb, rb, bar);
-  bulk_copy_g2s(dst + rb, p.modality + (size_t)b * p.cap_tokens + (size_t)wi * kWindow, kWindow, bar);
+  uint8_t* dst = &sm.ring[warp][stage * L::stage];
+  mbar_arrive_expect_tx(bar, L::bytes + kWindow);
+  bulk_copy_g2s(dst, rec_base + (size_t)wi * L::bytes, L::bytes, bar);
+  bulk_copy_g2s(dst + L::bytes, p.modality + (size_t)b * p.cap_tokens + (size_t)wi * kWindow, kWindow, bar);
 }
 
 template <int kMeta>
-__device__ void decode_mma4(const DecodeParams& p, DecodeSmem4& sm, int b, int kvh, int split, uint32_t tbase) {
+__device__ void decode_mma_lut(const DecodeParams& p, DecodeSmemLut& sm, int b, int kvh, int split, uint32_t tbase) {
+  using L = RecLut<kMeta>;
+  constexpr int kSt = L::stages;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int G = p.group;
   const int Hq = p.num_kv_heads * G;
   int T, w0, w1;
   split_range(p, b, split, T, w0, w1);
-  using L = Rec44<kMeta>;
   const uint8_t* rec_base = p.records + ((size_t)(b * p.num_kv_heads + kvh) * p.cap_windows) * L::bytes;
   int wa, we, wait_win, wait_val;
   warp_windows(w0, w1, warp, wa, we);
@@ -1270,10 +1274,10 @@ __device__ void decode_mma4(const DecodeParams& p, DecodeSmem4& sm, int b, int k
   if (lane == 0) {
     sm.wabort[warp] = 0;
 #pragma unroll
-    for (int s = 0; s < kStages4; ++s) mbar_init(&sm.bar[warp][s], 1);
+    for (int s = 0; s < kSt; ++s) mbar_init(&sm.bar[warp][s], 1);
     fence_barrier_init();
-    for (int i = 0; i < kStages4 && i < nmine; ++i)
-      issue_window4<kMeta>(p, sm, warp, i, rec_base, b, kvh, wa + i, wait_win, wait_val);
+    for (int i = 0; i < kSt && i < nmine; ++i)
+      issue_window_lut<kMeta>(p, sm, warp, i, rec_base, b, kvh, wa + i, wait_win, wait_val);
   }
   __syncwarp();
 
@@ -1295,15 +1299,15 @@ __device__ void decode_mma4(const DecodeParams& p, DecodeSmem4& sm, int b, int k
 
   int failed_at = -1;
   for (int i = 0; i < nmine; ++i) {
-    const int s = i % kStages4;
+    const int s = i % kSt;
     const int wi = wa + i;
-    const bool ok = mbar_wait_bounded(&sm.bar[warp][s], (i / kStages4) & 1, kWaitLimitNs) &&
+    const bool ok = mbar_wait_bounded(&sm.bar[warp][s], (i / kSt) & 1, kWaitLimitNs) &&
                     *reinterpret_cast<volatile int*>(&sm.wabort[warp]) == 0;
     if (!__all_sync(0xffffffffu, ok)) {
       failed_at = i;
       break;
     }
-    const uint8_t* stg = &sm.stage[warp][s][0];
+    const uint8_t* stg = &sm.ring[warp][s * L::stage];
     const uint32_t* kw = reinterpret_cast<const uint32_t*>(stg);
     const uint32_t* vw = reinterpret_cast<const uint32_t*>(stg + L::v);
     const __half* sig = reinterpret_cast<const __half*>(stg + L::sigma);
@@ -1318,7 +1322,7 @@ __device__ void decode_mma4(const DecodeParams& p, DecodeSmem4& sm, int b, int k
 
     // ---- the window's score operand: q'_c s_c 2^-E (hi, lo) at this lane's
     // B-fragment channels 16kc + 2t + {0, 1, 8, 9}, and the offset sum_c q'_c m_c
-    float qs[32];   // q'_c s_c, then the operand pairs
+    float qs[32];
     float off = 0.0f, smax = 0.0f;
     {
       const float4* ql = reinterpret_cast<const float4*>(&sm.qlane[lane][0]);
@@ -1372,9 +1376,9 @@ __device__ void decode_mma4(const DecodeParams& p, DecodeSmem4& sm, int b, int k
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int tokA = 16 * h + g, tokB = tokA + 8;
+      float d[4] = {0.f, 0.f, 0.f, 0.f}, e[4] = {0.f, 0.f, 0.f, 0.f};
       const uint4* ka = reinterpret_cast<const uint4*>(kw + tokA * 16);
       const uint4* kb = reinterpret_cast<const uint4*>(kw + tokB * 16);
-      float d[4] = {0.f, 0.f, 0.f, 0.f}, e[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
         const uint4 wa4 = ka[q4], wb4 = kb[q4];  // words 4 q4 .. 4 q4 + 3: chunks 2 q4, 2 q4 + 1
@@ -1383,10 +1387,10 @@ __device__ void decode_mma4(const DecodeParams& p, DecodeSmem4& sm, int b, int k
         for (int half = 0; half < 2; ++half) {
           const int kc = 2 * q4 + half;
           uint32_t ahi[4], alo[4];
-          lut_a(sm.klut, wa[2 * half], t, ahi[0], alo[0]);      // row g, k-slots 2t, 2t+1
-          lut_a(sm.klut, wb[2 * half], t, ahi[1], alo[1]);      // row g + 8
-          lut_a(sm.klut, wa[2 * half + 1], t, ahi[2], alo[2]);  // row g, k-slots 2t+8, 2t+9
-          lut_a(sm.klut, wb[2 * half + 1], t, ahi[3], alo[3]);  // row g + 8
+          lut4_a(sm.klut, wa[2 * half], t, ahi[0], alo[0]);      // row g, k-slots 2t, 2t+1
+          lut4_a(sm.klut, wb[2 * half], t, ahi[1], alo[1]);      // row g + 8
+          lut4_a(sm.klut, wa[2 * half + 1], t, ahi[2], alo[2]);  // row g, k-slots 2t+8, 2t+9
+          lut4_a(sm.klut, wb[2 * half + 1], t, ahi[3], alo[3]);  // row g + 8
           mma_f16_16816(d, ahi, bq[kc][0], bq[kc][1]);
           mma_f16_16816(e, ahi, bq[kc][2], bq[kc][3]);
           mma_f16_16816(e, alo, bq[kc][0], bq[kc][1]);
@@ -1436,17 +1440,14 @@ __device__ void decode_mma4(const DecodeParams& p, DecodeSmem4& sm, int b, int k
       st.l[0] += p0 + p2;
       st.l[1] += p1 + p3;
       const float sgA = __half2float(sig[tokA]), sgB = __half2float(sig[tokB]);
-      const float w0v = p0 * sgA, w1v = p1 * sgA, w2v = p2 * sgB, w3v = p3 * sgB;
       uint32_t bv[4];  // {hi (k 0..7), hi (k 8..15), lo (k 0..7), lo (k 8..15)}, transposed
-      split_pair_t(w0v, w1v, bv[0], bv[2]);
-      split_pair_t(w2v, w3v, bv[1], bv[3]);
+      split_pair_t(p0 * sgA, p1 * sgA, bv[0], bv[2]);
+      split_pair_t(p2 * sgB, p3 * sgB, bv[1], bv[3]);
       const int mA = min((int)mods[tokA], 2), mB = min((int)mods[tokB], 2);
       const uint32_t mbits = __reduce_or_sync(0xffffffffu, (1u << mA) | (1u << mB));
       const int base = 16 * h;
       const int mk0 = min((int)mods[base + 2 * t], 2), mk1 = min((int)mods[base + 2 * t + 1], 2);
       const int mk2 = min((int)mods[base + 8 + 2 * t], 2), mk3 = min((int)mods[base + 9 + 2 * t], 2);
-      const uint4* r0 = reinterpret_cast<const uint4*>(vw + (2 * h) * kHeadDim + 16 * g);      // tokens 16h .. +7
-      const uint4* r1 = reinterpret_cast<const uint4*>(vw + (2 * h + 1) * kHeadDim + 16 * g);  // tokens 16h+8 .. +15
       uint32_t todo = mbits;
       int mm = (st.cur >= 0 && ((todo >> st.cur) & 1u)) ? st.cur : __ffs(todo) - 1;
 #pragma unroll 1
@@ -1456,6 +1457,8 @@ __device__ void decode_mma4(const DecodeParams& p, DecodeSmem4& sm, int b, int k
         const uint32_t msk01 = single ? 0xFFFFFFFFu : ((mk0 == mm ? 0x0000FFFFu : 0u) | (mk1 == mm ? 0xFFFF0000u : 0u));
         const uint32_t msk23 = single ? 0xFFFFFFFFu : ((mk2 == mm ? 0x0000FFFFu : 0u) | (mk3 == mm ? 0xFFFF0000u : 0u));
         const uint32_t bh0 = bv[0] & msk01, bh1 = bv[1] & msk23, bl0 = bv[2] & msk01, bl1 = bv[3] & msk23;
+        const uint4* r0 = reinterpret_cast<const uint4*>(vw + (2 * h) * kHeadDim + 16 * g);      // tokens 16h .. +7
+        const uint4* r1 = reinterpret_cast<const uint4*>(vw + (2 * h + 1) * kHeadDim + 16 * g);  // tokens 16h+8 .. +15
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           const uint4 u0w = r0[q4], u1w = r1[q4];  // channels 16g + 4 q4 .. + 3
@@ -1464,10 +1467,10 @@ __device__ void decode_mma4(const DecodeParams& p, DecodeSmem4& sm, int b, int k
           for (int e2 = 0; e2 < 2; ++e2) {
             const int mt = 2 * q4 + e2;
             uint32_t ahi[4], alo[4];
-            lut_a(sm.vlut, x0[2 * e2], t, ahi[0], alo[0]);      // channel 16g + 2mt, tokens 2t, 2t+1
-            lut_a(sm.vlut, x0[2 * e2 + 1], t, ahi[1], alo[1]);  // channel 16g + 2mt + 1
-            lut_a(sm.vlut, x1[2 * e2], t, ahi[2], alo[2]);      // channel 16g + 2mt, tokens 8+2t, 9+2t
-            lut_a(sm.vlut, x1[2 * e2 + 1], t, ahi[3], alo[3]);
+            lut4_a(sm.vlut, x0[2 * e2], t, ahi[0], alo[0]);      // channel 16g + 2mt, tokens 2t, 2t+1
+            lut4_a(sm.vlut, x0[2 * e2 + 1], t, ahi[1], alo[1]);  // channel 16g + 2mt + 1
+            lut4_a(sm.vlut, x1[2 * e2], t, ahi[2], alo[2]);      // channel 16g + 2mt, tokens 8+2t, 9+2t
+            lut4_a(sm.vlut, x1[2 * e2 + 1], t, ahi[3], alo[3]);
             mma_f16_16816(st.acc[mt], ahi, bh0, bh1);
             mma_f16_16816(st.acc[mt], ahi, bl0, bl1);
             mma_f16_16816(st.acc[mt], alo, bh0, bh1);
@@ -1479,17 +1482,17 @@ __device__ void decode_mma4(const DecodeParams& p, DecodeSmem4& sm, int b, int k
       }
     }
     __syncwarp();
-    if (lane == 0 && i + kStages4 < nmine) {
+    if (lane == 0 && i + kSt < nmine) {
       fence_proxy_async_smem();
-      issue_window4<kMeta>(p, sm, warp, s, rec_base, b, kvh, wa + i + kStages4, wait_win, wait_val);
+      issue_window_lut<kMeta>(p, sm, warp, s, rec_base, b, kvh, wa + i + kSt, wait_win, wait_val);
     }
   }
 
   if (__any_sync(0xffffffffu, failed_at >= 0)) {
     const int f = __shfl_sync(0xffffffffu, failed_at, 0);
     if (lane == 0) set_error(p.error_word, OMNIKV_DEVERR_TIMEOUT);
-    for (int j = f; j < nmine && j < f + kStages4; ++j)
-      mbar_wait_bounded(&sm.bar[warp][j % kStages4], (j / kStages4) & 1, kWaitLimitNs);
+    for (int j = f; j < nmine && j < f + kSt; ++j)
+      mbar_wait_bounded(&sm.bar[warp][j % kSt], (j / kSt) & 1, kWaitLimitNs);
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
       st.m[j] = -INFINITY;
@@ -1511,7 +1514,7 @@ __device__ void decode_mma4(const DecodeParams& p, DecodeSmem4& sm, int b, int k
     sm.mw[warp][2 * t] = st.m[0];
     sm.mw[warp][2 * t + 1] = st.m[1];
   }
-  __syncthreads();  // also: all warps are done with their stage buffers
+  __syncthreads();  // also: all warps are done with their rings
   float M[2];
 #pragma unroll
   for (int j = 0; j < 2; ++j) {
@@ -1526,7 +1529,7 @@ __device__ void decode_mma4(const DecodeParams& p, DecodeSmem4& sm, int b, int k
     sm.lw[warp][2 * t] = st.l[0];
     sm.lw[warp][2 * t + 1] = st.l[1];
   }
-  float* xbuf = reinterpret_cast<float*>(&sm.stage[0][0][0]);  // [warp][32 registers][32 lanes]
+  float* xbuf = reinterpret_cast<float*>(&sm.ring[0][0]);  // [warp][32 registers][32 lanes]
 #pragma unroll
   for (int m = 0; m < kMods; ++m) {
     unpark(st, m, tbase, warp, M[0], M[1]);  // zeros if this warp never saw modality m
@@ -1570,9 +1573,15 @@ __device__ void decode_mma4(const DecodeParams& p, DecodeSmem4& sm, int b, int k
   }
 }
 
-// One decode CTA of the 4-bit tensor-core body.
+__device__ __forceinline__ uint32_t half_pair_bits(float x, uint32_t& lo) {
+  const __half h = __float2half_rn(x);
+  lo = __half_as_ushort(__float2half_rn(x - __half2float(h)));
+  return __half_as_ushort(h);
+}
+
+// One decode CTA of the table body.
 template <int kMeta>
-__device__ __forceinline__ void decode_cta4(const DecodeParams& p, DecodeSmem4& sm, int b, int kvh, int split) {
+__device__ __forceinline__ void decode_cta_lut(const DecodeParams& p, DecodeSmemLut& sm, int b, int kvh, int split) {
   {
     const size_t ubytes = (size_t)kMods * kHeadDim * kHeadDim * sizeof(float);
     const size_t share = (ubytes + p.num_splits - 1) / p.num_splits;
@@ -1582,15 +1591,13 @@ __device__ __forceinline__ void decode_cta4(const DecodeParams& p, DecodeSmem4& 
       asm volatile("prefetch.global.L2 [%0];" ::"l"(ub + off));
   }
   rotate_queries(p, b, kvh, &sm.q[0][0]);
-  if (threadIdx.x < 16) {  // codeword tables: c_j - c_0 (keys), c_j (values), as fp16 hi | lo
+  if (threadIdx.x < 16) {  // codeword tables: c_j - c_0 (keys), c_j (values)
     const int j = threadIdx.x;
-    const int LK = 1 << p.key_bits, LV = 1 << p.value_bits;
-    const float dk = j < LK ? p.key_cb[j] - p.key_cb[0] : 0.0f;
-    const float dv = j < LV ? p.val_cb[j] : 0.0f;
-    const __half hk = __float2half_rn(dk), hv = __float2half_rn(dv);
-    const __half lk = __float2half_rn(dk - __half2float(hk)), lv = __float2half_rn(dv - __half2float(hv));
-    sm.klut[j] = (uint32_t)__half_as_ushort(hk) | ((uint32_t)__half_as_ushort(lk) << 16);
-    sm.vlut[j] = (uint32_t)__half_as_ushort(hv) | ((uint32_t)__half_as_ushort(lv) << 16);
+    uint32_t lk, lv;
+    const uint32_t hk = half_pair_bits(p.key_cb[j] - p.key_cb[0], lk);
+    const uint32_t hv = half_pair_bits(p.val_cb[j], lv);
+    sm.klut[j] = hk | (lk << 16);
+    sm.vlut[j] = hv | (lv << 16);
   }
   if (threadIdx.x == 0) sm.bad_heads = 0u;
   __syncthreads();  // every warp's rotated queries are written
@@ -1628,7 +1635,7 @@ __device__ __forceinline__ void decode_cta4(const DecodeParams& p, DecodeSmem4& 
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = sm.tmem_base;
-  decode_mma4<kMeta>(p, sm, b, kvh, split, tbase);
+  decode_mma_lut<kMeta>(p, sm, b, kvh, split, tbase);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -1636,17 +1643,17 @@ __device__ __forceinline__ void decode_cta4(const DecodeParams& p, DecodeSmem4& 
 }
 
 template <int kMeta>
-__global__ void __launch_bounds__(kThreads, 2) decode_split_k4_kernel(const DecodeParams p) {
-  extern __shared__ __align__(16) uint8_t k4_smem[];
-  DecodeSmem4& sm = *reinterpret_cast<DecodeSmem4*>(k4_smem);
+__global__ void __launch_bounds__(kThreads, 2) decode_split_lut_kernel(const DecodeParams p) {
+  extern __shared__ __align__(16) uint8_t lut_smem[];
+  DecodeSmemLut& sm = *reinterpret_cast<DecodeSmemLut*>(lut_smem);
   griddep_launch_dependents();
-  decode_cta4<kMeta>(p, sm, blockIdx.z, blockIdx.y, blockIdx.x);
+  decode_cta_lut<kMeta>(p, sm, blockIdx.z, blockIdx.y, blockIdx.x);
 }
 
 template <int kMeta>
-__global__ void __launch_bounds__(kThreads, 2) decode_step4_kernel(const DecodeParams p, const WriteParams w) {
-  extern __shared__ __align__(16) uint8_t k4_smem[];
-  DecodeSmem4& sm = *reinterpret_cast<DecodeSmem4*>(k4_smem);
+__global__ void __launch_bounds__(kThreads, 2) decode_step_lut_kernel(const DecodeParams p, const WriteParams w) {
+  extern __shared__ __align__(16) uint8_t lut_smem[];
+  DecodeSmemLut& sm = *reinterpret_cast<DecodeSmemLut*>(lut_smem);
   griddep_launch_dependents();
   const int H = p.num_kv_heads;
   const int nappend = p.append_ctas;
@@ -1676,7 +1683,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_step4_kernel(const DecodeP
     return;
   }
   const int r = blockIdx.x - nappend;
-  decode_cta4<kMeta>(p, sm, r / (p.num_splits * H), (r / p.num_splits) % H, r % p.num_splits);
+  decode_cta_lut<kMeta>(p, sm, r / (p.num_splits * H), (r / p.num_splits) % H, r % p.num_splits);
 }
 
 // One decode CTA: split `split` of kv head kvh of sequence b. kBody: the 4-bit
@@ -1852,8 +1859,8 @@ cudaError_t prefer_shared_carveout(Kernel kernel, std::atomic<uint64_t>& done) {
 
 std::atomic<uint64_t> g_carveout[2][kNumBodies][3];  // [decode, step][body][key metadata format]
 
-// The 4-bit tensor-core kernels take their shared memory dynamically (above the
-// 48 KB static limit): the attribute and the carveout, set once per device.
+// The table body's kernels take their shared memory dynamically (above the 48 KB
+// static limit): the attribute and the carveout, set once per device.
 template <typename Kernel>
 cudaError_t prepare_dynamic(Kernel kernel, std::atomic<uint64_t>& done) {
   int dev = 0;
@@ -1861,7 +1868,7 @@ cudaError_t prepare_dynamic(Kernel kernel, std::atomic<uint64_t>& done) {
   if (e != cudaSuccess) return e;
   const uint64_t bit = dev < 64 ? (1ull << dev) : 0ull;
   if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
-  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(DecodeSmem4));
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(DecodeSmemLut));
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
   if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
@@ -1869,10 +1876,10 @@ cudaError_t prepare_dynamic(Kernel kernel, std::atomic<uint64_t>& done) {
 }
 
 template <int kMeta>
-cudaError_t prepare_tc4() {
-  const cudaError_t e = prepare_dynamic(decode_split_k4_kernel<kMeta>, g_carveout[0][kBodyTc4][kMeta]);
+cudaError_t prepare_lut() {
+  const cudaError_t e = prepare_dynamic(decode_split_lut_kernel<kMeta>, g_carveout[0][kBodyLut][kMeta]);
   if (e != cudaSuccess) return e;
-  return prepare_dynamic(decode_step4_kernel<kMeta>, g_carveout[1][kBodyTc4][kMeta]);
+  return prepare_dynamic(decode_step_lut_kernel<kMeta>, g_carveout[1][kBodyLut][kMeta]);
 }
 
 template <int kBody, int kMeta>
@@ -1885,7 +1892,7 @@ cudaError_t prepare_body() {
 // The 4-bit build reads the metadata format at run time: one instance.
 cudaError_t prepare_kernels(int body, int meta) {
   if (body == kBodyGeneric) return prepare_body<kBodyGeneric, kMetaFp16>();
-  if (body == kBodyTc4) return meta == kMetaMx ? prepare_tc4<kMetaMx>() : prepare_tc4<kMetaFp16>();
+  if (body == kBodyLut) return meta == kMetaMx ? prepare_lut<kMetaMx>() : prepare_lut<kMetaFp16>();
   if (meta == kMetaMx) return body == kBodyWarp ? prepare_body<kBodyWarp, kMetaMx>() : prepare_body<kBodyCoop, kMetaMx>();
   if (meta == kMetaTurbo)
     return body == kBodyWarp ? prepare_body<kBodyWarp, kMetaTurbo>() : prepare_body<kBodyCoop, kMetaTurbo>();
@@ -1921,22 +1928,23 @@ cudaError_t body_attributes(cudaFuncAttributes* a) {
 }
 
 template <int kMeta>
-cudaError_t tc4_attributes_of(cudaFuncAttributes* a) {
-  cudaError_t e = cudaFuncGetAttributes(a, decode_step4_kernel<kMeta>);
+cudaError_t lut_attributes_of(cudaFuncAttributes* a) {
+  cudaError_t e = cudaFuncGetAttributes(a, decode_step_lut_kernel<kMeta>);
   if (e != cudaSuccess) return e;
   cudaFuncAttributes a2;
-  if ((e = cudaFuncGetAttributes(&a2, decode_split_k4_kernel<kMeta>)) != cudaSuccess) return e;
+  if ((e = cudaFuncGetAttributes(&a2, decode_split_lut_kernel<kMeta>)) != cudaSuccess) return e;
   if (a2.numRegs > a->numRegs) a->numRegs = a2.numRegs;
   if (a2.sharedSizeBytes > a->sharedSizeBytes) a->sharedSizeBytes = a2.sharedSizeBytes;
-  a->sharedSizeBytes += sizeof(DecodeSmem4);
+  a->sharedSizeBytes += sizeof(DecodeSmemLut);
   return cudaSuccess;
 }
 
-cudaError_t tc4_attributes(cudaFuncAttributes* a) {
-  cudaError_t e = tc4_attributes_of<kMetaFp16>(a);
+// Attributes of the table body over both metadata formats.
+cudaError_t lut_attributes(cudaFuncAttributes* a) {
+  cudaError_t e = lut_attributes_of<kMetaFp16>(a);
   if (e != cudaSuccess) return e;
   cudaFuncAttributes a2;
-  if ((e = tc4_attributes_of<kMetaMx>(&a2)) != cudaSuccess) return e;
+  if ((e = lut_attributes_of<kMetaMx>(&a2)) != cudaSuccess) return e;
   if (a2.numRegs > a->numRegs) a->numRegs = a2.numRegs;
   if (a2.sharedSizeBytes > a->sharedSizeBytes) a->sharedSizeBytes = a2.sharedSizeBytes;
   return cudaSuccess;
@@ -1945,7 +1953,7 @@ cudaError_t tc4_attributes(cudaFuncAttributes* a) {
 }  // namespace
 
 int decode_body(int key_bits, int value_bits, int key_meta, int split_windows) {
-  if (key_bits == 4 && value_bits == 4 && key_meta != kMetaTurbo) return kBodyTc4;
+  if (key_bits == 4 && value_bits == 4 && key_meta != kMetaTurbo) return kBodyLut;
   if (key_bits != 2 || value_bits != 2) return kBodyGeneric;
   return split_windows <= kCoopMaxWindows ? kBodyCoop : kBodyWarp;
 }
@@ -1968,7 +1976,7 @@ int decode_ctas_per_sm(int body) {
   int regs_sm = 0, smem_sm = 0, smem_rsv = 0;
   const cudaError_t ea = body == kBodyWarp ? body_attributes<kBodyWarp>(&a)
                        : body == kBodyCoop ? body_attributes<kBodyCoop>(&a)
-                       : body == kBodyTc4  ? tc4_attributes(&a)
+                       : body == kBodyLut  ? lut_attributes(&a)
                                            : body_attributes<kBodyGeneric>(&a);
   if (prepare_kernels(body, kMetaFp16) != cudaSuccess ||
       (body != kBodyGeneric && prepare_kernels(body, kMetaMx) != cudaSuccess) ||
@@ -1981,7 +1989,7 @@ int decode_ctas_per_sm(int body) {
   const int warp_regs = ((a.numRegs * 32 + 255) / 256) * 256;  // allocated per warp in units of 256
   const int by_regs = regs_sm / (warp_regs * kWarps);
   const int by_smem = smem_sm / ((int)a.sharedSizeBytes + smem_rsv);
-  const int by_tmem = (body == kBodyWarp || body == kBodyTc4) ? 512 / (int)kTmemCols : 64;  // per-warp bodies hold tensor memory
+  const int by_tmem = (body == kBodyWarp || body == kBodyLut) ? 512 / (int)kTmemCols : 64;  // per-warp bodies hold tensor memory
   const int n = max(1, min(by_regs, min(by_smem, by_tmem)));
   if (dev < 64) cached[body][dev].store(n, std::memory_order_relaxed);
   return n;
@@ -1994,9 +2002,10 @@ cudaError_t launch_decode_step(const DecodeParams& p, const WriteParams& w, cuda
   if (e != cudaSuccess) return e;
   const dim3 grid(p.append_ctas + p.batch * p.num_kv_heads * p.num_splits);
   const dim3 block(kThreads);
-  if (body == kBodyTc4)
-    return meta == kMetaMx ? launch_pdl(decode_step4_kernel<kMetaMx>, grid, block, sizeof(DecodeSmem4), stream, p, w)
-                           : launch_pdl(decode_step4_kernel<kMetaFp16>, grid, block, sizeof(DecodeSmem4), stream, p, w);
+  constexpr size_t lsm = sizeof(DecodeSmemLut);
+  if (body == kBodyLut)
+    return meta == kMetaMx ? launch_pdl(decode_step_lut_kernel<kMetaMx>, grid, block, lsm, stream, p, w)
+                           : launch_pdl(decode_step_lut_kernel<kMetaFp16>, grid, block, lsm, stream, p, w);
   if (body == kBodyGeneric) return launch_pdl(decode_step_kernel<kBodyGeneric, kMetaFp16>, grid, block, 0, stream, p, w);
   if (meta == kMetaMx)
     return body == kBodyWarp ? launch_pdl(decode_step_kernel<kBodyWarp, kMetaMx>, grid, block, 0, stream, p, w)
@@ -2015,9 +2024,10 @@ cudaError_t launch_decode(const DecodeParams& p, int batch, cudaStream_t stream)
   if (e != cudaSuccess) return e;
   const dim3 grid(p.num_splits, p.num_kv_heads, batch);
   const dim3 block(kThreads);
-  if (body == kBodyTc4)
-    return meta == kMetaMx ? launch_pdl(decode_split_k4_kernel<kMetaMx>, grid, block, sizeof(DecodeSmem4), stream, p)
-                           : launch_pdl(decode_split_k4_kernel<kMetaFp16>, grid, block, sizeof(DecodeSmem4), stream, p);
+  constexpr size_t lsm = sizeof(DecodeSmemLut);
+  if (body == kBodyLut)
+    return meta == kMetaMx ? launch_pdl(decode_split_lut_kernel<kMetaMx>, grid, block, lsm, stream, p)
+                           : launch_pdl(decode_split_lut_kernel<kMetaFp16>, grid, block, lsm, stream, p);
   if (body == kBodyGeneric) return launch_pdl(decode_split_k_kernel<kBodyGeneric, kMetaFp16>, grid, block, 0, stream, p);
   if (meta == kMetaMx)
     return body == kBodyWarp ? launch_pdl(decode_split_k_kernel<kBodyWarp, kMetaMx>, grid, block, 0, stream, p)

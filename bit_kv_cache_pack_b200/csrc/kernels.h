@@ -121,7 +121,7 @@ cudaError_t launch_decode_step(const DecodeParams& p, const WriteParams& w, cuda
 // kCoopMaxWindows windows; 4-bit keys and values with per-window key metadata: the
 // per-warp tensor-core body over codeword tables; other bit mixes and 4-bit
 // TurboQuant keys: the CUDA-core build.
-enum DecodeBody { kBodyWarp = 0, kBodyCoop = 1, kBodyGeneric = 2, kBodyTc4 = 3, kNumBodies = 4 };
+enum DecodeBody { kBodyWarp = 0, kBodyCoop = 1, kBodyGeneric = 2, kBodyLut = 3, kNumBodies = 4 };
 constexpr int kCoopMaxWindows = 16;
 int decode_body(int key_bits, int value_bits, int key_meta, int split_windows);
 int decode_ctas_per_sm(int body);  // resident decode CTAs per SM of a body on the current device

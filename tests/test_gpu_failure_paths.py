@@ -4,12 +4,13 @@
   appended token waits (bounded), gives up after the limit, copies no stale
   record and writes its split empty; the error word reports
   OMNIKV_DEVERR_TIMEOUT and the combined output stays finite. Run for each decode
-  body: the cooperative body (short splits), the per-warp body (long splits) and
-  the CUDA-core build (4-bit caches).
+  body: the cooperative body (short splits), the per-warp body (long splits), the
+  4-bit table body and the CUDA-core build (mixed bit widths).
 * Operand range: queries far larger than the fp16 score operand could hold
   unscaled decode within the tolerance (the operand carries a power of two);
-  value scales beyond the fp16 range of the value operand (sigma >= 565) are
-  reported as OMNIKV_DEVERR_RANGE with a finite output.
+  2-bit value scales beyond the fp16 range of the value operand (sigma >= 565)
+  are reported as OMNIKV_DEVERR_RANGE with a finite output; the 4-bit table body
+  takes them.
 """
 import time
 
@@ -39,10 +40,11 @@ def _oracle_cache(spec, seed, ocfg, params, L, cap, value_scale=1.0):
     return oc
 
 
-@pytest.mark.parametrize("bits,splits,body", [(2, 8, "cooperative"), (2, 1, "per-warp"), (4, 2, "CUDA-core")])
-def test_step_flag_that_never_arrives(cuda_device, bits, splits, body):
+@pytest.mark.parametrize("kb,vb,splits,body", [(2, 2, 8, "cooperative"), (2, 2, 1, "per-warp"),
+                                               (4, 4, 2, "4-bit tables"), (2, 4, 2, "CUDA-core")])
+def test_step_flag_that_never_arrives(cuda_device, kb, vb, splits, body):
     import bit_kv_cache_pack_b200 as m
-    spec = with_bits(WORKLOADS["tiny"], bits, bits)
+    spec = with_bits(WORKLOADS["tiny"], kb, vb)
     seed = 41
     params, consts, ocfg = make_layer(spec, seed, 0, cuda_device)
     L = np.array([1000], np.int32)                     # the appended token lands in window 31 (partial)
@@ -66,13 +68,14 @@ def test_step_flag_that_never_arrives(cuda_device, bits, splits, body):
     assert int(cache.seq_lens[0].item()) == int(L[0])  # the cache is unchanged
 
 
+@pytest.mark.parametrize("bits", [2, 4])
 @pytest.mark.parametrize("splits", [0, 1])
-def test_large_queries_decode_within_tolerance(cuda_device, splits):
+def test_large_queries_decode_within_tolerance(cuda_device, splits, bits):
     """Queries x 4096: the largest score-operand entry would be ~10x the fp16
-    maximum without the operand's power of two. Default splits run the
-    cooperative body, one split the per-warp body."""
+    maximum without the operand's power of two. 2-bit: default splits run the
+    cooperative body, one split the per-warp body; 4-bit: the table body."""
     import bit_kv_cache_pack_b200 as m
-    spec, seed = WORKLOADS["tiny"], 43
+    spec, seed = with_bits(WORKLOADS["tiny"], bits, bits), 43
     params, consts, ocfg = make_layer(spec, seed, 0, cuda_device)
     L = np.array([2048], np.int32)
     oc = _oracle_cache(spec, seed, ocfg, params, L, 2080)
@@ -86,7 +89,7 @@ def test_large_queries_decode_within_tolerance(cuda_device, splits):
     m.omnikv_combine(consts.struct, cache.struct, part, S, out)
     torch.cuda.synchronize()
     assert int(cache.error_word.item()) == 0
-    check_decode(out.cpu().numpy(), decode_dense(ocfg, oc, q.cpu().numpy()), "queries x 4096, S=%d" % S)
+    check_decode(out.cpu().numpy(), decode_dense(ocfg, oc, q.cpu().numpy()), "queries x 4096, K%d S=%d" % (bits, S))
 
 
 @pytest.mark.parametrize("splits", [0, 1])
@@ -110,3 +113,28 @@ def test_value_scales_out_of_range_are_reported(cuda_device, splits):
     torch.cuda.synchronize()
     assert int(cache.error_word.item()) & RANGE_BIT
     assert torch.isfinite(out).all()
+
+
+@pytest.mark.parametrize("splits", [0, 1])
+def test_4bit_large_value_scales_decode(cuda_device, splits):
+    """Values x 1024 on a 4-bit cache: the table body's value operand is the
+    softmax weight times sigma (at most 65504), so scales of several thousand
+    decode without a range report and within the tolerance relative to their size."""
+    import bit_kv_cache_pack_b200 as m
+    spec, seed = with_bits(WORKLOADS["tiny"], 4, 4), 47
+    params, consts, ocfg = make_layer(spec, seed, 0, cuda_device)
+    L = np.array([2048], np.int32)
+    oc = _oracle_cache(spec, seed, ocfg, params, L, 2080, value_scale=1024.0)
+    sig = oc.records[0, :, :, oc.off["sigma"]:].copy().view(np.float16).astype(np.float32)
+    assert sig.max() >= 565.0 and np.isfinite(sig).all()
+    cache = upload_oracle_cache(oc, cuda_device)
+    q = seeded_randn((1, spec.num_q_heads, 128), cuda_device, 9).half()
+    S = splits or m.omnikv_default_splits(consts.struct, cache.struct)
+    part = m.partials_tensor(1, spec.num_q_heads, S, cuda_device)
+    out = torch.empty(1, spec.num_q_heads, 128, device=cuda_device)
+    m.omnikv_decode_attention(consts.struct, cache.struct, q, part, S)
+    m.omnikv_combine(consts.struct, cache.struct, part, S, out)
+    torch.cuda.synchronize()
+    assert int(cache.error_word.item()) == 0
+    check_decode(out.cpu().numpy() / 1024.0, decode_dense(ocfg, oc, q.cpu().numpy()) / 1024.0,
+                 "K4 values x 1024, S=%d" % S)

@@ -109,41 +109,44 @@ def test_chunked_writes_and_tail(cuda_device, bits):
     check_decode(gpu_decode(consts, upload_oracle_cache(oc, cuda_device), q), ref, "bits=%d" % bits)
 
 
+@pytest.mark.parametrize("bits", [2, 4])
 @pytest.mark.parametrize("splits", [1, 2, 3, 5, 7, 64, 200])
-def test_decode_split_counts(cuda_device, splits):
-    """1,000 tokens (32 windows): one split of 32 windows runs the per-warp body; 16, 11,
-    7, 5 and 1 windows per split run the cooperative body (whole and partial window
-    groups)."""
+def test_decode_split_counts(cuda_device, splits, bits):
+    """1,000 tokens (32 windows). 2-bit: one split of 32 windows runs the per-warp
+    body; 16, 11, 7, 5 and 1 windows per split run the cooperative body (whole and
+    partial window groups). 4-bit: the per-warp table body at every split length
+    (one to four windows per warp, warps without windows)."""
     m = _abi()
-    spec, seed = WORKLOADS["tiny"], 5
+    spec, seed = with_bits(WORKLOADS["tiny"], bits, bits), 5
     params, consts, ocfg = make_layer(spec, seed, 0, cuda_device)
     L = np.array([1000], np.int32)
     drift = key_drift(spec, seed, 0, 32, cuda_device)
     k, v, mod = prefill_inputs(spec, seed, 0, params, drift, L, cuda_device)
-    oc = codec.OracleCache(1, 2, 1024, 2, 2)
+    oc = codec.OracleCache(1, 2, 1024, bits, bits)
     codec.write_cache(ocfg, oc, k.cpu().numpy(), v.cpu().numpy(), mod.cpu().numpy())
     for scale in (1.0, 3.0):  # 3x sharpens the attention (larger error amplification)
         g = torch.Generator(device=cuda_device).manual_seed(splits)
         q = (scale * torch.randn(1, 16, 128, device=cuda_device, generator=g)).half()
         ref = decode_dense(ocfg, oc, q.cpu().numpy())
         check_decode(gpu_decode(consts, upload_oracle_cache(oc, cuda_device), q, splits), ref,
-                     "S=%d scale=%g" % (splits, scale))
+                     "K%d S=%d scale=%g" % (bits, splits, scale))
 
 
-def test_decode_edge_cases(cuda_device):
+@pytest.mark.parametrize("bits", [2, 4])
+def test_decode_edge_cases(cuda_device, bits):
     """Batch of four: an empty sequence (zeros), a single token, a zero query
     (mean of the values) and a one-window sequence."""
     m = _abi()
-    spec, seed = WORKLOADS["tiny"], 6
+    spec, seed = with_bits(WORKLOADS["tiny"], bits, bits), 6
     params, consts, ocfg = make_layer(spec, seed, 0, cuda_device)
     drift = key_drift(spec, seed, 0, 4, cuda_device)
-    oc = codec.OracleCache(4, 2, 96, 2, 2)
-    gc = m.KVCache(4, 2, 96, 2, 2, cuda_device)
+    oc = codec.OracleCache(4, 2, 96, bits, bits)
+    gc = m.KVCache(4, 2, 96, bits, bits, cuda_device)
     for b, n in [(1, 1), (2, 70), (3, 32)]:
         k, v, mod = prefill_inputs(spec, seed + b, 0, params, drift, np.array([n]), cuda_device)
         view = gc.sequence_view(b)
         m.omnikv_write_cache(consts.struct, view, k.contiguous(), v.contiguous(), mod.contiguous(), n)
-        sub = codec.OracleCache(1, 2, 96, 2, 2)
+        sub = codec.OracleCache(1, 2, 96, bits, bits)
         codec.write_cache(ocfg, sub, k.cpu().numpy(), v.cpu().numpy(), mod.cpu().numpy())
         oc.records[b], oc.key_tail[b], oc.modality[b], oc.seq_lens[b] = (
             sub.records[0], sub.key_tail[0], sub.modality[0], sub.seq_lens[0])
@@ -155,7 +158,7 @@ def test_decode_edge_cases(cuda_device):
     ref = decode_dense(ocfg, oc, q.cpu().numpy())
     out = gpu_decode(consts, upload_oracle_cache(oc, cuda_device), q)
     assert np.all(out[0] == 0)
-    check_decode(out, ref, "edge cases")
+    check_decode(out, ref, "edge cases K%d" % bits)
 
 
 def test_device_capacity_check_sets_error_word(cuda_device):
@@ -197,23 +200,53 @@ def test_asymmetric_codebook_uses_generic_path(cuda_device):
     check_decode(gpu_decode(consts, upload_oracle_cache(oc, cuda_device), q, 3), ref, "asymmetric")
 
 
-@pytest.mark.parametrize("G,hkv", [(1, 4), (4, 2), (8, 1)])
-def test_group_sizes(cuda_device, G, hkv):
-    """GQA groups smaller than 8 leave tensor-core columns unused; every group
-    size up to 8 must match the oracle, with both 2-bit decode bodies (600 tokens:
-    one split of 19 windows runs the per-warp body, 4 splits the cooperative one)."""
+@pytest.mark.parametrize("splits", [1, 3])
+def test_4bit_codebook_with_full_fp32_mantissas(cuda_device, splits):
+    """The 4-bit tensor-core body holds each codeword as an fp16 high + low pair:
+    an asymmetric 16-level codebook whose entries use the whole fp32 mantissa (no
+    entry exact in fp16) still matches the oracle, keys and values."""
     import dataclasses
     m = _abi()
-    spec = dataclasses.replace(WORKLOADS["tiny"], num_q_heads=G * hkv, num_kv_heads=hkv)
+    spec, seed = with_bits(WORKLOADS["tiny"], 4, 4), 10
+    params, consts, ocfg = make_layer(spec, seed, 0, cuda_device)
+    rng = np.random.default_rng(10)
+    kb = np.sort(rng.normal(0.3, 1.1, 16)).astype(np.float32)
+    vb = np.sort(rng.normal(-0.2, 0.9, 16)).astype(np.float32)
+    assert np.all(np.diff(kb) > 0) and np.all(np.diff(vb) > 0)
+    assert not np.any(kb.astype(np.float16).astype(np.float32) == kb)
+    consts = m.LayerConstants(kb, vb, params["key_signs"], params["value_rot"], spec.num_q_heads, cuda_device)
+    ocfg = dataclasses.replace(ocfg, key_codebook=kb, value_codebook=vb)
+    L = np.array([700], np.int32)
+    drift = key_drift(spec, seed, 0, 22, cuda_device)
+    k, v, mod = prefill_inputs(spec, seed, 0, params, drift, L, cuda_device)
+    oc = codec.OracleCache(1, 2, 704, 4, 4)
+    codec.write_cache(ocfg, oc, k.cpu().numpy(), v.cpu().numpy(), mod.cpu().numpy())
+    for scale in (1.0, 3.0):
+        q = (scale * seeded_randn((1, 16, 128), cuda_device, 15)).half()
+        ref = decode_dense(ocfg, oc, q.cpu().numpy())
+        check_decode(gpu_decode(consts, upload_oracle_cache(oc, cuda_device), q, splits), ref,
+                     "K4 fp32 codebook S=%d scale=%g" % (splits, scale))
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+@pytest.mark.parametrize("G,hkv", [(1, 4), (4, 2), (8, 1)])
+def test_group_sizes(cuda_device, G, hkv, bits):
+    """GQA groups smaller than 8 leave tensor-core columns unused; every group
+    size up to 8 must match the oracle, with both 2-bit decode bodies (600 tokens:
+    one split of 19 windows runs the per-warp body, 4 splits the cooperative one)
+    and the 4-bit table body."""
+    import dataclasses
+    m = _abi()
+    spec = dataclasses.replace(with_bits(WORKLOADS["tiny"], bits, bits), num_q_heads=G * hkv, num_kv_heads=hkv)
     seed = 9
     params, consts, ocfg = make_layer(spec, seed, 0, cuda_device, per_head=True)
     L = np.array([600, 70], np.int32)
     spec2 = dataclasses.replace(spec, batch=2)
     drift = key_drift(spec2, seed, 0, 20, cuda_device)
     k, v, mod = prefill_inputs(spec2, seed, 0, params, drift, np.array([600, 600]), cuda_device)
-    oc = codec.OracleCache(2, hkv, 640, 2, 2)
+    oc = codec.OracleCache(2, hkv, 640, bits, bits)
     for b in range(2):
-        sub = codec.OracleCache(1, hkv, 640, 2, 2)
+        sub = codec.OracleCache(1, hkv, 640, bits, bits)
         n = int(L[b])
         codec.write_cache(ocfg, sub, k[b:b + 1, :, :n].cpu().numpy(), v[b:b + 1, :, :n].cpu().numpy(),
                           mod[b:b + 1, :n].cpu().numpy())
@@ -222,4 +255,4 @@ def test_group_sizes(cuda_device, G, hkv):
     q = seeded_randn((2, G * hkv, 128), cuda_device, 14 + G).half()
     ref = decode_dense(ocfg, oc, q.cpu().numpy())
     for S in (1, 4):
-        check_decode(gpu_decode(consts, upload_oracle_cache(oc, cuda_device), q, S), ref, "G=%d S=%d" % (G, S))
+        check_decode(gpu_decode(consts, upload_oracle_cache(oc, cuda_device), q, S), ref, "K%d G=%d S=%d" % (bits, G, S))
