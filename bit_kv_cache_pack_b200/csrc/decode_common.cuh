@@ -1,6 +1,7 @@
-// Device helpers shared by the decode kernels (decode_split_k.cu, decode_tc.cu):
+// Device helpers shared by the decode kernels (decode_split_k.cu, stream.cu):
 // rotated-query layout, split ranges, decode-step flags, and the CUDA-core decode
-// path (4-bit caches and codebooks that are not symmetric).
+// path (mixed bit widths, 4-bit TurboQuant keys, 2-bit codebooks that are not
+// symmetric).
 #pragma once
 
 #include <cstddef>
@@ -115,8 +116,8 @@ __device__ __forceinline__ float fast_exp2(float x) {
 }
 
 // ---------------------------------------------------------------------------
-// CUDA-core path (4-bit codes, or a codebook that is not symmetric): the CTA
-// decodes the split's windows one at a time from a double-buffered ring of bulk
+// CUDA-core path (mixed bit widths, 4-bit TurboQuant keys, or a 2-bit codebook
+// that is not symmetric): the CTA decodes the split's windows one at a time from a double-buffered ring of bulk
 // copies. Scores: four threads per token, thread q of token t holding channels
 // 4 j + q (j = 0..31), each dequantised once, k'_tc = m_c + s_c (c_code - c_0),
 // and used for the 8 query heads; two shuffles complete the dot products.
@@ -423,7 +424,7 @@ __device__ void decode_generic_t(const DecodeParams& p, GenSmem& g, const float*
 
 // The 2-bit builds reach the CUDA-core path only for a codebook that is not
 // symmetric: out of line there, so that the tensor-core paths stay compact in
-// the instruction cache. The 4-bit build inlines its three instances.
+// the instruction cache. The CUDA-core build inlines its three instances.
 template <class Sync>
 __device__ __noinline__ void decode_generic_asym(const DecodeParams& p, GenSmem& g, const float* qflat, int b,
                                                  int kvh, int split) {

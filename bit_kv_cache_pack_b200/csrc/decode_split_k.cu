@@ -49,10 +49,13 @@
 // two tokens of every value-operand register (k-slots 2t, 2t+1 -> tokens t,
 // t+8) sit 16 bits apart in one channel-major code word.
 //
-// CUDA-core path (4-bit codes, or a codebook that is not symmetric): the CTA
-// decodes a window at a time (four threads per token for the scores, a thread per
-// channel for the values), built into its own kernel for 4-bit caches (more CTAs
-// per SM, no tensor memory).
+// 4-bit codes (fp16 or MXFP4 key metadata): the per-warp table body, mma.sync
+// operands looked up per code byte in shared-memory codeword tables.
+//
+// CUDA-core path (mixed bit widths, 4-bit TurboQuant keys, or a 2-bit codebook
+// that is not symmetric): the CTA decodes a window at a time (four threads per
+// token for the scores, a thread per channel for the values), built into its own
+// kernel for the first two (more CTAs per SM, no tensor memory).
 //
 // Decode step (decode_step_kernel): the first batch x kv-head CTAs of the launch
 // append one token per (sequence, kv head) and publish the new length in a flag;
@@ -1786,7 +1789,7 @@ __device__ __forceinline__ void decode_cta(const DecodeParams& p, DecodeSmem& sm
 }
 
 // Registers for this many resident CTAs per SM: per-warp body 2 (its accumulators
-// need ~240 registers), cooperative body 3, 4-bit build 4.
+// need ~240 registers), cooperative body 3, CUDA-core build 4.
 __host__ __device__ constexpr int body_ctas_per_sm(int body) {
   return body == kBodyWarp ? 2 : body == kBodyCoop ? 3 : 4;
 }
@@ -1889,7 +1892,7 @@ cudaError_t prepare_body() {
   return prefer_shared_carveout(decode_step_kernel<kBody, kMeta>, g_carveout[1][kBody][kMeta]);
 }
 
-// The 4-bit build reads the metadata format at run time: one instance.
+// The CUDA-core build reads the metadata format at run time: one instance.
 cudaError_t prepare_kernels(int body, int meta) {
   if (body == kBodyGeneric) return prepare_body<kBodyGeneric, kMetaFp16>();
   if (body == kBodyLut) return meta == kMetaMx ? prepare_lut<kMetaMx>() : prepare_lut<kMetaFp16>();
