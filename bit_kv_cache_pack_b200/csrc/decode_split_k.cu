@@ -1046,7 +1046,7 @@ __device__ void decode_coop(const DecodeParams& p, DecodeSmem& sm, int b, int kv
 #pragma unroll 1
     for (int ww = 0; ww < kCoop; ++ww) {
       const uint8_t* rv = stg + ww * L::bytes + L::v;
-#pragma unroll
+#pragma unroll 1  // rolled: half the code (3 % faster at batch 1 and 2 than unrolled)
       for (int h = 0; h < 2; ++h) {
         const uint32_t tm = sm.tmask[ww][h];
         if (tm == 0u) continue;  // no window (the group's tail)
