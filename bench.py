@@ -56,8 +56,8 @@ META_FORMATS = {"fp16": 0, "mx": 1, "turbo": 2}   # omnikv_config.key_meta_forma
 # next capture.
 TRAFFIC_CAPTURES = {
     ("qwen3-omni-30b-48L-b8-ctx65536", "fp16"): {
-        "sources_sha256": "4c93b77c20c49f12f995dd0c422180b174a58631e5304729b8c3a82c18580375",
-        "bytes_per_launch": 173719808 + 8626432},
+        "sources_sha256": "bfd8f694b4bce03a68a8a11fcfe801258380d4cd26198d6caec73b331c52da6e",
+        "bytes_per_launch": 173710592 + 8660224},
 }
 KERNEL_SOURCES = ("decode_split_k.cu", "decode_common.cuh", "append.cuh", "common.cuh", "ptx.cuh", "kernels.h")
 
