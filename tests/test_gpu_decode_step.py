@@ -47,16 +47,19 @@ CASES = [
     (2, 8, [31, 64, 0], 3, 0, 2),           # a full window, a fresh window, an empty sequence
     (4, 8, [200, 17], 4, 0, 2),             # 4 kv heads, 32 query heads
     (2, 8, [93, 40], 4, 200, 2),            # 2 x (1 + 200) CTAs: beyond residency -> four-call fallback
-    (2, 8, [93, 250], 4, 0, 4),             # K4V4: the CUDA-core decode path with the fused append
+    (2, 8, [93, 250], 4, 0, 4),             # K4V4: the table body with the fused append
     (2, 8, [700], 3, 1, 2),                 # one split of 22 windows: the per-warp body in the fused launch
     # 16 x 2 units x 9 per-warp splits = 288 decode CTAs: the 8 append CTAs left
     # in a 296-CTA wave append for 4 (sequence, kv head) units each
     (2, 8, [4700 + 13 * i for i in range(16)], 2, 0, 2),
+    (2, 8, [700, 333], 3, 1, 4),            # K4V4, one split per (sequence, kv head): long table-body splits
+    (2, 8, [2300 + 13 * i for i in range(16)], 2, 0, 4),  # K4V4 with shared append CTAs (2 CTAs per SM)
 ]
 
 
 @pytest.mark.parametrize("hkv,G,lengths,steps,splits,bits", CASES,
-                         ids=["b1-boundary", "ragged-b3", "h4", "fallback", "k4", "per-warp", "shared-append-ctas"])
+                         ids=["b1-boundary", "ragged-b3", "h4", "fallback", "k4", "per-warp", "shared-append-ctas",
+                              "k4-one-split", "k4-shared-append-ctas"])
 def test_decode_step_matches_four_calls_and_oracle(cuda_device, hkv, G, lengths, steps, splits, bits):
     import bit_kv_cache_pack_b200 as m
     dev = cuda_device

@@ -98,6 +98,26 @@ def test_static_scratch_matches_allocated_partials(cuda_device):
 
 
 @pytest.mark.gpu
+def test_static_scratch_matches_allocated_partials_4bit(cuda_device):
+    """The same with 4-bit codes (the table body, which takes its shared memory
+    dynamically): bit-identical to the allocating path, within tolerance of the
+    oracle."""
+    import bit_kv_cache_pack_b200 as m
+    from synth.workloads import with_bits
+    spec, seed = with_bits(WORKLOADS["tiny"], 4, 4), 22
+    params, consts, ocfg = make_layer(spec, seed, 0, cuda_device)
+    oc = _oracle_cache(spec, seed, ocfg, params)
+    cache = upload_oracle_cache(oc, cuda_device)
+    for call, (qseed, S) in enumerate([(3, 5), (4, 0)]):
+        q = seeded_randn((1, spec.num_q_heads, 128), cuda_device, qseed).half()
+        S_used = S or m.omnikv_default_splits(consts.struct, cache.struct)
+        got = _static(m, consts, cache, q, S)
+        assert np.array_equal(got, _allocated(m, consts, cache, q, S_used)), "K4 call %d" % (call + 1)
+        check_decode(got, decode_dense(ocfg, oc, q.cpu().numpy()), "static scratch K4, call %d" % (call + 1))
+    assert int(cache.error_word.item()) == 0
+
+
+@pytest.mark.gpu
 def test_static_scratch_lowers_the_default_split_count(cuda_device):
     """Batch 64 x 16 query heads: the default split count does not fit the array
     (5405 entries hold 5 splits), so the call lowers it to 5 -- which also moves the
