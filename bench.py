@@ -17,9 +17,11 @@ barrier + synchronize around the timed region; the max over ranks is reported.
 All steps are replayed from one CUDA graph holding, per step, the L2 flush, the
 step's start event, exactly the C-ABI calls of the step, and its end event (no
 host gaps between steps). `value` has all inputs resident in HBM; `e2e` also
-copies each step's inputs (q, k, v and modality ids of every layer, packed in one
-pinned host buffer: one H2D copy) and the step's outputs back to the host
-(captured the same way).
+copies each step's inputs (q, k, v and modality ids of every layer, packed per
+layer in pinned host memory) and the step's outputs back to the host, inside the
+step's timed region, on side streams (layer 0's inputs first, the other layers'
+while layer 0 decodes; all outputs but the last layer's while it decodes), captured
+the same way.
 """
 from __future__ import annotations
 
@@ -275,15 +277,19 @@ class Workload:
         self.out = torch.empty(spec.layers, spec.batch, spec.num_q_heads, 128, dtype=torch.float32,
                                device=device)
 
-    def step_calls(self, s, q, k, v, mod, stream, dec_events=None):
+    def step_calls(self, s, q, k, v, mod, stream, dec_events=None, before=None, after=None):
         """The C-ABI calls of one decode step over all layers: omnikv_decode_step
         per layer (the append-and-decode launch, then the combine launch). With
         `dec_events` (a start/end pair), layer s % layers makes the same step as
         its two calls, omnikv_append_decode between the events, so the dominant
-        kernel (decode_step_kernel) is timed in place once per step."""
+        kernel (decode_step_kernel) is timed in place once per step. `before` and
+        `after` (called with the layer index) let the end-to-end run order each
+        layer after its input copy and its output copy after it."""
         m = self.m
         n = self.spec.layers
         for layer in range(n):
+            if before is not None:
+                before(layer)
             c, cache = self.consts[layer].struct, self.caches[layer].struct
             if dec_events is not None and layer == s % n:
                 dec_events[0].record(stream)
@@ -293,6 +299,8 @@ class Workload:
             else:
                 m.omnikv_decode_step(c, cache, q[layer], k[layer], v[layer], mod[layer], self.part, 0,
                                      self.out[layer], stream)
+            if after is not None:
+                after(layer)
 
     def launches_per_step(self, instrumented):
         """Library kernel launches in one step: 2 per layer (the append-and-decode
@@ -371,32 +379,69 @@ def run_gpu(args):
     dec_bytes = [wl.decode_bytes(s) for s in range(W, W + K)]
     total_ms = float(np.sum(step_ms))
 
-    # --- end to end through the C ABI with host buffers: per step the H2D copy of
-    # the step's inputs from pinned memory and the D2H copy of its outputs --------
-    # a step's inputs (q, k, v, modality ids of all layers) are packed in one pinned
-    # buffer and arrive with one H2D copy into 16-byte aligned device views
+    # --- end to end through the C ABI with host buffers: per step the H2D copies of
+    # the step's inputs from pinned memory and the D2H copies of its outputs ------
+    # a layer's inputs (q, k, v, modality ids) are packed in one pinned block
+    # (16-byte aligned device views). The copies run on side streams: layer 0's block
+    # first, the other layers' while layer 0 decodes; the outputs of all layers but
+    # the last while the last decodes, then the last one's. The step's timed region
+    # opens before its first input copy and closes after its last output copy.
     srcs = (wl.q, wl.k, wl.v, wl.mod)
-    sizes = [t[0].numel() * t[0].element_size() for t in srcs]
-    offs = [0]
-    for sz in sizes[:-1]:
-        offs.append(offs[-1] + (sz + 15) // 16 * 16)
-    nbytes = offs[-1] + sizes[-1]
-    hin = torch.empty((K, nbytes), dtype=torch.uint8).pin_memory()
+    nl = spec.layers
+    sizes = [t[0].numel() * t[0].element_size() for t in srcs]          # one step, all layers
+    lsizes = [sz // nl for sz in sizes]                                   # one layer
+    loffs = [0]
+    for sz in lsizes[:-1]:
+        loffs.append(loffs[-1] + (sz + 15) // 16 * 16)
+    lbytes = (loffs[-1] + lsizes[-1] + 15) // 16 * 16
+    hin = torch.empty((K, nl, lbytes), dtype=torch.uint8).pin_memory()
     for i in range(K):
-        for t, o, sz in zip(srcs, offs, sizes):
-            hin[i, o:o + sz].copy_(t[W + K + i].reshape(-1).view(torch.uint8).cpu())
-    din = torch.empty(nbytes, dtype=torch.uint8, device=dev)
-    dq, dk, dv, dm = (din[o:o + sz].view(t.dtype).view(t.shape[1:]) for t, o, sz in zip(srcs, offs, sizes))
+        for t, o, sz in zip(srcs, loffs, lsizes):
+            hin[i, :, o:o + sz].copy_(t[W + K + i].reshape(nl, -1).view(torch.uint8).cpu())
+    din = torch.empty((nl, lbytes), dtype=torch.uint8, device=dev)
+    dq, dk, dv, dm = ([din[l, o:o + sz].view(t.dtype).view(t.shape[2:]) for l in range(nl)]
+                      for t, o, sz in zip(srcs, loffs, lsizes))
     hout = torch.empty((K,) + tuple(wl.out.shape), dtype=torch.float32).pin_memory()
     e2e_ev = [(ev(), ev()) for _ in range(K)]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    sync = lambda: torch.cuda.Event()
+    fork_ev, join_ev = [sync() for _ in range(K)], [sync() for _ in range(K)]
+    in_ev = [[sync() for _ in range(2)] for _ in range(K)]
+    out_ev = [[sync() for _ in range(2)] for _ in range(K)]
 
     def e2e_steps(cs):
         for i in range(K):
             flush.zero_()
             e2e_ev[i][0].record(cs)
-            din.copy_(hin[i], non_blocking=True)
-            wl.step_calls(W + K + i, dq, dk, dv, dm, cs)
-            hout[i].copy_(wl.out, non_blocking=True)
+            fork_ev[i].record(cs)
+            s_in.wait_event(fork_ev[i])
+            s_out.wait_event(fork_ev[i])
+            with torch.cuda.stream(s_in):
+                din[0].copy_(hin[i, 0], non_blocking=True)
+                in_ev[i][0].record(s_in)
+                if nl > 1:
+                    din[1:].copy_(hin[i, 1:], non_blocking=True)
+                    in_ev[i][1].record(s_in)
+
+            def before(l, i=i):
+                if l < 2:
+                    cs.wait_event(in_ev[i][l])
+
+            def after(l, i=i):
+                if l < nl - 2:
+                    return
+                j = l - (nl - 2)  # 0: layers 0 .. nl - 2 are done; 1: the last layer
+                out_ev[i][j].record(cs)
+                s_out.wait_event(out_ev[i][j])
+                with torch.cuda.stream(s_out):
+                    if l == nl - 1:
+                        hout[i, l].copy_(wl.out[l], non_blocking=True)
+                    else:
+                        hout[i, :l + 1].copy_(wl.out[:l + 1], non_blocking=True)
+
+            wl.step_calls(W + K + i, dq, dk, dv, dm, cs, before=before, after=after)
+            join_ev[i].record(s_out)
+            cs.wait_event(join_ev[i])
             e2e_ev[i][1].record(cs)
     g2 = None
     if use_graphs:
