@@ -1,7 +1,6 @@
 // Device helpers shared by the decode kernels (decode_split_k.cu, stream.cu):
 // rotated-query layout, split ranges, decode-step flags, and the CUDA-core decode
-// path (mixed bit widths, 4-bit TurboQuant keys, 2-bit codebooks that are not
-// symmetric).
+// path (mixed bit widths, 2-bit codebooks that are not symmetric).
 #pragma once
 
 #include <cstddef>
@@ -116,8 +115,8 @@ __device__ __forceinline__ float fast_exp2(float x) {
 }
 
 // ---------------------------------------------------------------------------
-// CUDA-core path (mixed bit widths, 4-bit TurboQuant keys, or a 2-bit codebook
-// that is not symmetric): the CTA decodes the split's windows one at a time from a double-buffered ring of bulk
+// CUDA-core path (mixed bit widths, or a 2-bit codebook that is not symmetric):
+// the CTA decodes the split's windows one at a time from a double-buffered ring of bulk
 // copies. Scores: four threads per token, thread q of token t holding channels
 // 4 j + q (j = 0..31), each dequantised once, k'_tc = m_c + s_c (c_code - c_0),
 // and used for the 8 query heads; two shuffles complete the dot products.

@@ -49,13 +49,13 @@
 // two tokens of every value-operand register (k-slots 2t, 2t+1 -> tokens t,
 // t+8) sit 16 bits apart in one channel-major code word.
 //
-// 4-bit codes (fp16 or MXFP4 key metadata): the per-warp table body, mma.sync
-// operands looked up per code byte in shared-memory codeword tables.
+// 4-bit codes (every key format): the per-warp table body, mma.sync operands
+// looked up per code byte in shared-memory codeword tables.
 //
-// CUDA-core path (mixed bit widths, 4-bit TurboQuant keys, or a 2-bit codebook
-// that is not symmetric): the CTA decodes a window at a time (four threads per
-// token for the scores, a thread per channel for the values), built into its own
-// kernel for the first two (more CTAs per SM, no tensor memory).
+// CUDA-core path (mixed bit widths, or a 2-bit codebook that is not symmetric):
+// the CTA decodes a window at a time (four threads per token for the scores, a
+// thread per channel for the values), built into its own kernel for mixed bit
+// widths (more CTAs per SM, no tensor memory).
 //
 // Decode step (decode_step_kernel): the first batch x kv-head CTAs of the launch
 // append one token per (sequence, kv head) and publish the new length in a flag;
@@ -1231,7 +1231,8 @@ static_assert(offsetof(DecodeSmemLut, qlane) % 16 == 0 && offsetof(DecodeSmemLut
                   offsetof(DecodeSmemLut, bar) % 8 == 0 && kLutRing % 16 == 0, "aligned fields");
 static_assert(kWarps * 32 * 32 * 4 <= kWarps * kLutRing, "merge buffer");
 static_assert(sizeof(WindowSmem) <= sizeof(DecodeSmemLut), "append uses the decode shared memory");
-static_assert(RecLut<kMetaFp16>::stages == 2 && RecLut<kMetaMx>::stages == 2, "barriers per warp");
+static_assert(RecLut<kMetaFp16>::stages == 2 && RecLut<kMetaMx>::stages == 2 && RecLut<kMetaTurbo>::stages == 2,
+              "barriers per warp");
 
 // The A operand registers of byte `t` of a code word (two codes: the even k-slot in
 // the low nibble): hi and lo parts from the table.
@@ -1301,6 +1302,29 @@ __device__ void decode_mma_lut(const DecodeParams& p, DecodeSmemLut& sm, int b, 
   st.cur = -1;
   st.parked = 0;
   const float qmax = sm.qmax;
+  // TurboQuant keys (k'_tc = ksigma_t c_j): the score operand is q' alone, the same
+  // for every window, built here once; each score is its token's ksigma times the sum
+  uint32_t bqt[8][4];
+  float esct = 1.0f;
+  if constexpr (kMeta == kMetaTurbo) {
+    int E = 0;
+    if (qmax > 0.0f && isfinite(qmax)) E = max(-100, min(100, (int)ceilf(log2f(qmax / 16384.0f))));
+    const float bscale = ldexpf(1.0f, -E);
+    esct = ldexpf(1.0f, E);
+    const float4* ql = reinterpret_cast<const float4*>(&sm.qlane[lane][0]);
+#pragma unroll
+    for (int kc = 0; kc < 8; ++kc) {
+      const float4 q4 = ql[kc];
+      const float x0 = q4.x * bscale, x1 = q4.y * bscale, x2 = q4.z * bscale, x3 = q4.w * bscale;
+      const __half2 h01 = __floats2half2_rn(x0, x1), h23 = __floats2half2_rn(x2, x3);
+      const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+      const __half2 l01 = __floats2half2_rn(x0 - f01.x, x1 - f01.y), l23 = __floats2half2_rn(x2 - f23.x, x3 - f23.y);
+      bqt[kc][0] = *reinterpret_cast<const uint32_t*>(&h01);
+      bqt[kc][1] = *reinterpret_cast<const uint32_t*>(&h23);
+      bqt[kc][2] = *reinterpret_cast<const uint32_t*>(&l01);
+      bqt[kc][3] = *reinterpret_cast<const uint32_t*>(&l23);
+    }
+  }
 
   int failed_at = -1;
   for (int i = 0; i < nmine; ++i) {
@@ -1317,63 +1341,73 @@ __device__ void decode_mma_lut(const DecodeParams& p, DecodeSmemLut& sm, int b, 
     const uint32_t* vw = reinterpret_cast<const uint32_t*>(stg + L::v);
     const __half* sig = reinterpret_cast<const __half*>(stg + L::sigma);
     const uint8_t* mods = stg + L::bytes;
-    const __half2* meta;
-    if constexpr (kMeta == kMetaMx) {
-      mx_window_pairs(stg + L::meta, sm.mxpairs[warp], lane);
-      meta = reinterpret_cast<const __half2*>(sm.mxpairs[warp]);
+    const __half* ksig = reinterpret_cast<const __half*>(stg + L::meta);  // TurboQuant keys: per-token scales
+    uint32_t bq[8][4];  // per chunk: {hi (2t, 2t+1), hi (8+2t, 9+2t), lo (2t, 2t+1), lo (8+2t, 9+2t)}
+    float off0 = 0.0f, off1 = 0.0f, escale = esct;
+    if constexpr (kMeta == kMetaTurbo) {
+#pragma unroll
+      for (int kc = 0; kc < 8; ++kc)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) bq[kc][r] = bqt[kc][r];
     } else {
-      meta = reinterpret_cast<const __half2*>(stg + L::meta);
-    }
+      const __half2* meta;
+      if constexpr (kMeta == kMetaMx) {
+        mx_window_pairs(stg + L::meta, sm.mxpairs[warp], lane);
+        meta = reinterpret_cast<const __half2*>(sm.mxpairs[warp]);
+      } else {
+        meta = reinterpret_cast<const __half2*>(stg + L::meta);
+      }
 
-    // ---- the window's score operand: q'_c s_c 2^-E (hi, lo) at this lane's
-    // B-fragment channels 16kc + 2t + {0, 1, 8, 9}, and the offset sum_c q'_c m_c
-    float qs[32];
-    float off = 0.0f, smax = 0.0f;
-    {
-      const float4* ql = reinterpret_cast<const float4*>(&sm.qlane[lane][0]);
+      // ---- the window's score operand: q'_c s_c 2^-E (hi, lo) at this lane's
+      // B-fragment channels 16kc + 2t + {0, 1, 8, 9}, and the offset sum_c q'_c m_c
+      float qs[32];
+      float off = 0.0f, smax = 0.0f;
+      {
+        const float4* ql = reinterpret_cast<const float4*>(&sm.qlane[lane][0]);
+#pragma unroll
+        for (int kc = 0; kc < 8; ++kc) {
+          const float4 q4 = ql[kc];
+          const uint2 ma = *reinterpret_cast<const uint2*>(meta + 16 * kc + 2 * t);      // channels 2t, 2t+1
+          const uint2 mb = *reinterpret_cast<const uint2*>(meta + 16 * kc + 8 + 2 * t);  // channels 8+2t, 9+2t
+          const float2 p0 = __half22float2(*reinterpret_cast<const __half2*>(&ma.x));
+          const float2 p1 = __half22float2(*reinterpret_cast<const __half2*>(&ma.y));
+          const float2 p2 = __half22float2(*reinterpret_cast<const __half2*>(&mb.x));
+          const float2 p3 = __half22float2(*reinterpret_cast<const __half2*>(&mb.y));
+          off = fmaf(q4.x, p0.x, off);
+          off = fmaf(q4.y, p1.x, off);
+          off = fmaf(q4.z, p2.x, off);
+          off = fmaf(q4.w, p3.x, off);
+          smax = fmaxf(smax, fmaxf(fmaxf(fabsf(p0.y), fabsf(p1.y)), fmaxf(fabsf(p2.y), fabsf(p3.y))));
+          qs[4 * kc + 0] = q4.x * p0.y;
+          qs[4 * kc + 1] = q4.y * p1.y;
+          qs[4 * kc + 2] = q4.z * p2.y;
+          qs[4 * kc + 3] = q4.w * p3.y;
+        }
+        off += __shfl_xor_sync(0xffffffffu, off, 1);
+        off += __shfl_xor_sync(0xffffffffu, off, 2);
+        smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 1));
+        smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 2));
+      }
+      off0 = __shfl_sync(0xffffffffu, off, 8 * t);      // head 2t
+      off1 = __shfl_sync(0xffffffffu, off, 8 * t + 4);  // head 2t + 1
+      // the largest |B| entry at most 2^14
+      const float bmax = qmax * smax;
+      int E = 0;
+      if (bmax > 0.0f && isfinite(bmax)) E = max(-100, min(100, (int)ceilf(log2f(bmax / 16384.0f))));
+      const float bscale = ldexpf(1.0f, -E);
+      escale = ldexpf(1.0f, E);
 #pragma unroll
       for (int kc = 0; kc < 8; ++kc) {
-        const float4 q4 = ql[kc];
-        const uint2 ma = *reinterpret_cast<const uint2*>(meta + 16 * kc + 2 * t);      // channels 2t, 2t+1
-        const uint2 mb = *reinterpret_cast<const uint2*>(meta + 16 * kc + 8 + 2 * t);  // channels 8+2t, 9+2t
-        const float2 p0 = __half22float2(*reinterpret_cast<const __half2*>(&ma.x));
-        const float2 p1 = __half22float2(*reinterpret_cast<const __half2*>(&ma.y));
-        const float2 p2 = __half22float2(*reinterpret_cast<const __half2*>(&mb.x));
-        const float2 p3 = __half22float2(*reinterpret_cast<const __half2*>(&mb.y));
-        off = fmaf(q4.x, p0.x, off);
-        off = fmaf(q4.y, p1.x, off);
-        off = fmaf(q4.z, p2.x, off);
-        off = fmaf(q4.w, p3.x, off);
-        smax = fmaxf(smax, fmaxf(fmaxf(fabsf(p0.y), fabsf(p1.y)), fmaxf(fabsf(p2.y), fabsf(p3.y))));
-        qs[4 * kc + 0] = q4.x * p0.y;
-        qs[4 * kc + 1] = q4.y * p1.y;
-        qs[4 * kc + 2] = q4.z * p2.y;
-        qs[4 * kc + 3] = q4.w * p3.y;
+        const float x0 = qs[4 * kc] * bscale, x1 = qs[4 * kc + 1] * bscale;
+        const float x2 = qs[4 * kc + 2] * bscale, x3 = qs[4 * kc + 3] * bscale;
+        const __half2 h01 = __floats2half2_rn(x0, x1), h23 = __floats2half2_rn(x2, x3);
+        const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+        const __half2 l01 = __floats2half2_rn(x0 - f01.x, x1 - f01.y), l23 = __floats2half2_rn(x2 - f23.x, x3 - f23.y);
+        bq[kc][0] = *reinterpret_cast<const uint32_t*>(&h01);
+        bq[kc][1] = *reinterpret_cast<const uint32_t*>(&h23);
+        bq[kc][2] = *reinterpret_cast<const uint32_t*>(&l01);
+        bq[kc][3] = *reinterpret_cast<const uint32_t*>(&l23);
       }
-      off += __shfl_xor_sync(0xffffffffu, off, 1);
-      off += __shfl_xor_sync(0xffffffffu, off, 2);
-      smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 1));
-      smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 2));
-    }
-    const float off0 = __shfl_sync(0xffffffffu, off, 8 * t);      // head 2t
-    const float off1 = __shfl_sync(0xffffffffu, off, 8 * t + 4);  // head 2t + 1
-    // the largest |B| entry at most 2^14
-    const float bmax = qmax * smax;
-    int E = 0;
-    if (bmax > 0.0f && isfinite(bmax)) E = max(-100, min(100, (int)ceilf(log2f(bmax / 16384.0f))));
-    const float bscale = ldexpf(1.0f, -E), escale = ldexpf(1.0f, E);
-    uint32_t bq[8][4];  // per chunk: {hi (2t, 2t+1), hi (8+2t, 9+2t), lo (2t, 2t+1), lo (8+2t, 9+2t)}
-#pragma unroll
-    for (int kc = 0; kc < 8; ++kc) {
-      const float x0 = qs[4 * kc] * bscale, x1 = qs[4 * kc + 1] * bscale;
-      const float x2 = qs[4 * kc + 2] * bscale, x3 = qs[4 * kc + 3] * bscale;
-      const __half2 h01 = __floats2half2_rn(x0, x1), h23 = __floats2half2_rn(x2, x3);
-      const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
-      const __half2 l01 = __floats2half2_rn(x0 - f01.x, x1 - f01.y), l23 = __floats2half2_rn(x2 - f23.x, x3 - f23.y);
-      bq[kc][0] = *reinterpret_cast<const uint32_t*>(&h01);
-      bq[kc][1] = *reinterpret_cast<const uint32_t*>(&h23);
-      bq[kc][2] = *reinterpret_cast<const uint32_t*>(&l01);
-      bq[kc][3] = *reinterpret_cast<const uint32_t*>(&l23);
     }
 
     // ---- scores of the two 16-token tiles: rows g, g + 8 = tokens 16h + g, 16h + g + 8
@@ -1404,10 +1438,12 @@ __device__ void decode_mma_lut(const DecodeParams& p, DecodeSmemLut& sm, int b, 
         }
       }
       const int posA = wi * kWindow + tokA, posB = wi * kWindow + tokB;
-      const float r0 = posA < T ? fmaf(d[0] + e[0], escale, off0) : -INFINITY;
-      const float r1 = posA < T ? fmaf(d[1] + e[1], escale, off1) : -INFINITY;
-      const float r2 = posB < T ? fmaf(d[2] + e[2], escale, off0) : -INFINITY;
-      const float r3 = posB < T ? fmaf(d[3] + e[3], escale, off1) : -INFINITY;
+      const float kgA = kMeta == kMetaTurbo ? __half2float(ksig[tokA]) : 1.0f;
+      const float kgB = kMeta == kMetaTurbo ? __half2float(ksig[tokB]) : 1.0f;
+      const float r0 = posA < T ? kgA * fmaf(d[0] + e[0], escale, off0) : -INFINITY;
+      const float r1 = posA < T ? kgA * fmaf(d[1] + e[1], escale, off1) : -INFINITY;
+      const float r2 = posB < T ? kgB * fmaf(d[2] + e[2], escale, off0) : -INFINITY;
+      const float r3 = posB < T ? kgB * fmaf(d[3] + e[3], escale, off1) : -INFINITY;
       if (h == 0) {
         sc[0][0] = r0; sc[0][1] = r1; sc[0][2] = r2; sc[0][3] = r3;
       } else {
@@ -1603,10 +1639,10 @@ __device__ __forceinline__ void decode_cta_lut(const DecodeParams& p, DecodeSmem
       asm volatile("prefetch.global.L2 [%0];" ::"l"(ub + off));
   }
   rotate_queries(p, b, kvh, &sm.q[0][0]);
-  if (threadIdx.x < 16) {  // codeword tables: c_j - c_0 (keys), c_j (values)
+  if (threadIdx.x < 16) {  // codeword tables: c_j - c_0 (keys; c_j for TurboQuant keys), c_j (values)
     const int j = threadIdx.x;
     uint32_t lk, lv;
-    const uint32_t hk = half_pair_bits(p.key_cb[j] - p.key_cb[0], lk);
+    const uint32_t hk = half_pair_bits(kMeta == kMetaTurbo ? p.key_cb[j] : p.key_cb[j] - p.key_cb[0], lk);
     const uint32_t hv = half_pair_bits(p.val_cb[j], lv);
     sm.klut[j] = hk | (lk << 16);
     sm.vlut[j] = hv | (lv << 16);
@@ -1904,7 +1940,8 @@ cudaError_t prepare_body() {
 // The CUDA-core build reads the metadata format at run time: one instance.
 cudaError_t prepare_kernels(int body, int meta) {
   if (body == kBodyGeneric) return prepare_body<kBodyGeneric, kMetaFp16>();
-  if (body == kBodyLut) return meta == kMetaMx ? prepare_lut<kMetaMx>() : prepare_lut<kMetaFp16>();
+  if (body == kBodyLut)
+    return meta == kMetaMx ? prepare_lut<kMetaMx>() : meta == kMetaTurbo ? prepare_lut<kMetaTurbo>() : prepare_lut<kMetaFp16>();
   if (meta == kMetaMx) return body == kBodyWarp ? prepare_body<kBodyWarp, kMetaMx>() : prepare_body<kBodyCoop, kMetaMx>();
   if (meta == kMetaTurbo)
     return body == kBodyWarp ? prepare_body<kBodyWarp, kMetaTurbo>() : prepare_body<kBodyCoop, kMetaTurbo>();
@@ -1951,12 +1988,15 @@ cudaError_t lut_attributes_of(cudaFuncAttributes* a) {
   return cudaSuccess;
 }
 
-// Attributes of the table body over both metadata formats.
+// Attributes of the table body over every key metadata format.
 cudaError_t lut_attributes(cudaFuncAttributes* a) {
   cudaError_t e = lut_attributes_of<kMetaFp16>(a);
   if (e != cudaSuccess) return e;
   cudaFuncAttributes a2;
   if ((e = lut_attributes_of<kMetaMx>(&a2)) != cudaSuccess) return e;
+  if (a2.numRegs > a->numRegs) a->numRegs = a2.numRegs;
+  if (a2.sharedSizeBytes > a->sharedSizeBytes) a->sharedSizeBytes = a2.sharedSizeBytes;
+  if ((e = lut_attributes_of<kMetaTurbo>(&a2)) != cudaSuccess) return e;
   if (a2.numRegs > a->numRegs) a->numRegs = a2.numRegs;
   if (a2.sharedSizeBytes > a->sharedSizeBytes) a->sharedSizeBytes = a2.sharedSizeBytes;
   return cudaSuccess;
@@ -1965,7 +2005,7 @@ cudaError_t lut_attributes(cudaFuncAttributes* a) {
 }  // namespace
 
 int decode_body(int key_bits, int value_bits, int key_meta, int split_windows) {
-  if (key_bits == 4 && value_bits == 4 && key_meta != kMetaTurbo) return kBodyLut;
+  if (key_bits == 4 && value_bits == 4) return kBodyLut;
   if (key_bits != 2 || value_bits != 2) return kBodyGeneric;
   return split_windows <= kCoopMaxWindows ? kBodyCoop : kBodyWarp;
 }
@@ -1992,7 +2032,7 @@ int decode_ctas_per_sm(int body) {
                                            : body_attributes<kBodyGeneric>(&a);
   if (prepare_kernels(body, kMetaFp16) != cudaSuccess ||
       (body != kBodyGeneric && prepare_kernels(body, kMetaMx) != cudaSuccess) ||
-      ((body == kBodyWarp || body == kBodyCoop) && prepare_kernels(body, kMetaTurbo) != cudaSuccess) ||
+      (body != kBodyGeneric && prepare_kernels(body, kMetaTurbo) != cudaSuccess) ||
       ea != cudaSuccess ||
       cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
@@ -2016,8 +2056,9 @@ cudaError_t launch_decode_step(const DecodeParams& p, const WriteParams& w, cuda
   const dim3 block(kThreads);
   constexpr size_t lsm = sizeof(DecodeSmemLut);
   if (body == kBodyLut)
-    return meta == kMetaMx ? launch_pdl(decode_step_lut_kernel<kMetaMx>, grid, block, lsm, stream, p, w)
-                           : launch_pdl(decode_step_lut_kernel<kMetaFp16>, grid, block, lsm, stream, p, w);
+    return meta == kMetaMx      ? launch_pdl(decode_step_lut_kernel<kMetaMx>, grid, block, lsm, stream, p, w)
+           : meta == kMetaTurbo ? launch_pdl(decode_step_lut_kernel<kMetaTurbo>, grid, block, lsm, stream, p, w)
+                                : launch_pdl(decode_step_lut_kernel<kMetaFp16>, grid, block, lsm, stream, p, w);
   if (body == kBodyGeneric) return launch_pdl(decode_step_kernel<kBodyGeneric, kMetaFp16>, grid, block, 0, stream, p, w);
   if (meta == kMetaMx)
     return body == kBodyWarp ? launch_pdl(decode_step_kernel<kBodyWarp, kMetaMx>, grid, block, 0, stream, p, w)
@@ -2038,8 +2079,9 @@ cudaError_t launch_decode(const DecodeParams& p, int batch, cudaStream_t stream)
   const dim3 block(kThreads);
   constexpr size_t lsm = sizeof(DecodeSmemLut);
   if (body == kBodyLut)
-    return meta == kMetaMx ? launch_pdl(decode_split_lut_kernel<kMetaMx>, grid, block, lsm, stream, p)
-                           : launch_pdl(decode_split_lut_kernel<kMetaFp16>, grid, block, lsm, stream, p);
+    return meta == kMetaMx      ? launch_pdl(decode_split_lut_kernel<kMetaMx>, grid, block, lsm, stream, p)
+           : meta == kMetaTurbo ? launch_pdl(decode_split_lut_kernel<kMetaTurbo>, grid, block, lsm, stream, p)
+                                : launch_pdl(decode_split_lut_kernel<kMetaFp16>, grid, block, lsm, stream, p);
   if (body == kBodyGeneric) return launch_pdl(decode_split_k_kernel<kBodyGeneric, kMetaFp16>, grid, block, 0, stream, p);
   if (meta == kMetaMx)
     return body == kBodyWarp ? launch_pdl(decode_split_k_kernel<kBodyWarp, kMetaMx>, grid, block, 0, stream, p)

@@ -118,9 +118,8 @@ cudaError_t launch_decode_step(const DecodeParams& p, const WriteParams& w, cuda
 // Decode kernel bodies. 2-bit caches: the per-warp body (each warp streams its own
 // run of windows; registers for 2 CTAs per SM) for long splits, the cooperative
 // body (the CTA takes 4 windows at a time; 3 CTAs per SM) for splits of at most
-// kCoopMaxWindows windows; 4-bit keys and values with per-window key metadata: the
-// per-warp tensor-core body over codeword tables; other bit mixes and 4-bit
-// TurboQuant keys: the CUDA-core build.
+// kCoopMaxWindows windows; 4-bit keys and values (every key format): the per-warp
+// tensor-core body over codeword tables; other bit mixes: the CUDA-core build.
 enum DecodeBody { kBodyWarp = 0, kBodyCoop = 1, kBodyGeneric = 2, kBodyLut = 3, kNumBodies = 4 };
 constexpr int kCoopMaxWindows = 16;
 int decode_body(int key_bits, int value_bits, int key_meta, int split_windows);

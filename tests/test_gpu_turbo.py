@@ -82,20 +82,21 @@ def test_turbo_chunked_writes_bit_exact(cuda_device, bits):
         check_decode(out, ref, "turbo bits=%d S=%d" % (bits, S))
 
 
-def test_turbo_prefill_append_decode(cuda_device):
+@pytest.mark.parametrize("bits", [2, 4])
+def test_turbo_prefill_append_decode(cuda_device, bits):
     """The tiny workload's 2,048-token prefill and one appended token with turbo
     keys; decode over the oracle's cache and over the GPU-written one with the
-    default split count (cooperative body) and one split (per-warp body), then the
-    fused decode step."""
+    default split count (2-bit: cooperative body) and one split (2-bit: per-warp
+    body; 4-bit: the table body either way), then the fused decode step."""
     import bit_kv_cache_pack_b200 as m
-    spec, seed = WORKLOADS["tiny"], 63
+    spec, seed = with_bits(WORKLOADS["tiny"], bits, bits), 63
     params, consts, ocfg = make_layer(spec, seed, 0, cuda_device, key_meta_format=TURBO)
     L = seq_lengths(spec, seed)
     cap = 2048 + 64
     drift = key_drift(spec, seed, 0, cap // 32, cuda_device)
     k, v, mod = prefill_inputs(spec, seed, 0, params, drift, L, cuda_device)
-    gc = m.KVCache(1, 2, cap, 2, 2, cuda_device, key_meta_format=TURBO)
-    oc = codec.OracleCache(1, 2, cap, 2, 2, meta_format="turbo")
+    gc = m.KVCache(1, 2, cap, bits, bits, cuda_device, key_meta_format=TURBO)
+    oc = codec.OracleCache(1, 2, cap, bits, bits, meta_format="turbo")
     _write_both(m, consts, ocfg, gc, oc, k, v, mod)
     q, kn, vn, mn = decode_inputs(spec, seed, 0, 0, params, drift, L, cuda_device)
     _write_both(m, consts, ocfg, gc, oc, kn, vn, mn)
@@ -107,7 +108,7 @@ def test_turbo_prefill_append_decode(cuda_device):
     for cache, what in ((upload_oracle_cache(oc, cuda_device), "oracle cache"), (gc, "gpu cache")):
         for S in (0, 1):
             out, S = _decode(m, consts, cache, q, S, 16)
-            check_decode(out, ref, "turbo %s S=%d" % (what, S))
+            check_decode(out, ref, "turbo K%d %s S=%d" % (bits, what, S))
     q2, kn2, vn2, mn2 = decode_inputs(spec, seed, 0, 1, params, drift, L + 1, cuda_device)
     S, fused = m.omnikv_step_splits(consts.struct, gc.struct, 0)
     part = m.partials_tensor(1, 16, S, cuda_device)
