@@ -7,15 +7,19 @@
 // block of 128:
 //   0. before waiting on the decode launch: this warp's 4 rows of U_m for the 3
 //      modalities go into registers (they do not depend on the decode);
-//   1. warp 0: M = max_s m_s, weights e_s = exp(m_s - M), l = sum_s l_s e_s,
-//      each lane's (m, l) pairs loaded together;
-//   2. a_m[c] = sum_s acc_{s,m}[c] e_s / l, the splits read as 16-byte vectors,
-//      two threads per vector column, 16 loads in flight per thread, splits of
-//      weight 0 not read;
+//   1. warp w merges the splits s = w, w + 8, ... as they arrive: a split's (m, l)
+//      and its 384 accumulators (three 16-byte vectors per lane) are loaded
+//      together, kBatch splits at a time, and folded in with a running maximum
+//      (the running sums rescaled when it grows; splits with m = -inf skipped);
+//   2. the 8 warps' (max, sum, accumulators) merge through shared memory at their
+//      common maximum M: a_m[c] = sum_s acc_{s,m}[c] e^(m_s - M) / l with
+//      l = sum_s l_s e^(m_s - M);
 //   3. out[j] = sum_m sum_c U_m[j][c] a_m[c] for the block's rows: one warp per 4
 //      rows, lanes over c, warp reduction.
-// The row blocks of a head merge the same partials (read from L2); splitting the
-// rows keeps every step one memory round trip deep when there are few heads.
+// The merge needs no maximum before the first accumulator load, so up to 8 kBatch
+// splits are one memory round trip deep. The row blocks of a head merge the same
+// partials (read from L2); splitting the rows keeps every step short when there
+// are few heads.
 // A sequence without tokens (all m_s = -inf) yields zeros.
 #include "common.cuh"
 #include "kernels.h"
@@ -27,10 +31,11 @@ namespace {
 
 constexpr int kCombineThreads = 256;
 constexpr int kWarpsC = kCombineThreads / 32;
-constexpr int kMaxSplitsSmem = 4096;
+constexpr int kMaxSplitsSmem = 4096;  // the library's split limit
+constexpr int kBatch = 3;             // splits per warp in flight
 
 template <int kRowBlocks>
-__global__ void __launch_bounds__(kCombineThreads)
+__global__ void __launch_bounds__(kCombineThreads, 2)
 combine_inverse_rotate_kernel(const CombineParams p) {
   constexpr int kRowsPerWarp = kHeadDim / kRowBlocks / kWarpsC;  // 4 or 16
   const int g = blockIdx.x / kRowBlocks;  // query head within the group
@@ -43,11 +48,9 @@ combine_inverse_rotate_kernel(const CombineParams p) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qh = kvh * G + g;
 
-  __shared__ float w[kMaxSplitsSmem];   // split maxima, then weights
-  __shared__ float wl[kMaxSplitsSmem];  // split denominators
-  __shared__ __align__(16) float4 red[2][96];
+  __shared__ __align__(16) float4 wacc[kWarpsC][96];  // each warp's accumulators, at its own max
+  __shared__ float wmax[kWarpsC], wsum[kWarpsC];
   __shared__ __align__(16) float a[kMods * kHeadDim];
-  __shared__ float s_l;
 
   griddep_launch_dependents();
   // ---- 0. value-basis rows (constant input): this warp's rows j0 .., lanes over
@@ -70,77 +73,70 @@ combine_inverse_rotate_kernel(const CombineParams p) {
     if (L >= 0 && L + p.len_add <= p.cap_tokens) p.seq_lens[b] = L + p.len_add;
   }
 
-  // ---- 1. split weights (warp 0): every lane loads (m, l) of all its splits at
-  // once (one memory round trip for up to 128 splits), then the max, the weights
-  // e_s and l = sum_s l_s e_s
-  if (warp == 0) {
-    constexpr int kPer = 4;  // splits per lane per pass
-    float M = -INFINITY;
-    for (int base = 0; base < S; base += 32 * kPer) {
-      float2 ml[kPer];
+  // ---- 1. each warp folds in its splits as they arrive (running maximum)
+  {
+    float mw = -INFINITY, lw = 0.0f;
+    float4 aw[3] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f),
+                    make_float4(0.f, 0.f, 0.f, 0.f)};
+    for (int s0 = warp; s0 < S; s0 += kWarpsC * kBatch) {
+      float2 ml[kBatch];
+      float4 v[kBatch][3];
 #pragma unroll
-      for (int i = 0; i < kPer; ++i) {
-        const int s = base + 32 * i + lane;
-        ml[i] = s < S ? *reinterpret_cast<const float2*>(&part[s].m) : make_float2(-INFINITY, 0.0f);
+      for (int i = 0; i < kBatch; ++i) {
+        const int sp = s0 + kWarpsC * i;
+        ml[i] = sp < S ? *reinterpret_cast<const float2*>(&part[sp].m) : make_float2(-INFINITY, 0.0f);
+        // the accumulators of an empty split (m = -inf) are never written: loaded
+        // (the memory is the split's own) but not used
+        const float4* src = reinterpret_cast<const float4*>(part[sp < S ? sp : s0].acc);
+#pragma unroll
+        for (int j = 0; j < 3; ++j) v[i][j] = src[lane + 32 * j];
       }
 #pragma unroll
-      for (int i = 0; i < kPer; ++i) {
-        const int s = base + 32 * i + lane;
-        if (s < S) {
-          w[s] = ml[i].x;
-          wl[s] = ml[i].y;
+      for (int i = 0; i < kBatch; ++i) {
+        if (ml[i].x == -INFINITY) continue;  // warp-uniform
+        const float mn = fmaxf(mw, ml[i].x);
+        const float fo = mw == -INFINITY ? 0.0f : expf(mw - mn);
+        const float fn = expf(ml[i].x - mn);
+        lw = lw * fo + ml[i].y * fn;
+#pragma unroll
+        for (int j = 0; j < 3; ++j) {
+          aw[j].x = fmaf(v[i][j].x, fn, aw[j].x * fo);
+          aw[j].y = fmaf(v[i][j].y, fn, aw[j].y * fo);
+          aw[j].z = fmaf(v[i][j].z, fn, aw[j].z * fo);
+          aw[j].w = fmaf(v[i][j].w, fn, aw[j].w * fo);
         }
-        M = fmaxf(M, ml[i].x);
+        mw = mn;
       }
     }
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float l = 0.0f;
-    for (int s = lane; s < S; s += 32) {
-      const float ms = w[s];
-      const float e = (ms == -INFINITY) ? 0.0f : expf(ms - M);
-      w[s] = e;
-      if (e != 0.0f) l += wl[s] * e;
+    for (int j = 0; j < 3; ++j) wacc[warp][lane + 32 * j] = aw[j];
+    if (lane == 0) {
+      wmax[warp] = mw;
+      wsum[warp] = lw;
     }
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-    if (lane == 0) s_l = l;
   }
   __syncthreads();
 
-  // ---- 2. weighted sum over splits: column c4 (of 96 float4), half h of the
-  // splits, kU loads in flight per thread (splits of weight 0 are not read)
-  {
-    const int c4 = tid & 127, h = tid >> 7;
-    if (c4 < 96) {
-      constexpr int kU = 16;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int s0 = h; s0 < S; s0 += 2 * kU) {
-        float4 v[kU];
-        float e[kU];
-#pragma unroll
-        for (int i = 0; i < kU; ++i) {
-          const int s = s0 + 2 * i;
-          e[i] = s < S ? w[s] : 0.0f;
-          v[i] = e[i] != 0.0f ? reinterpret_cast<const float4*>(part[s].acc)[c4] : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-#pragma unroll
-        for (int i = 0; i < kU; ++i) {
-          acc.x = fmaf(v[i].x, e[i], acc.x);
-          acc.y = fmaf(v[i].y, e[i], acc.y);
-          acc.z = fmaf(v[i].z, e[i], acc.z);
-          acc.w = fmaf(v[i].w, e[i], acc.w);
-        }
-      }
-      red[h][c4] = acc;
-    }
-  }
-  __syncthreads();
+  // ---- 2. the warps' partial merges at their common maximum
   if (tid < 96) {
-    const float inv = s_l > 0.0f ? 1.0f / s_l : 0.0f;
-    const float4 x = red[0][tid], y = red[1][tid];
-    reinterpret_cast<float4*>(a)[tid] =
-        make_float4((x.x + y.x) * inv, (x.y + y.y) * inv, (x.z + y.z) * inv, (x.w + y.w) * inv);
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarpsC; ++w) M = fmaxf(M, wmax[w]);
+    float l = 0.0f;
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int w = 0; w < kWarpsC; ++w) {
+      if (wmax[w] == -INFINITY) continue;
+      const float e = expf(wmax[w] - M);
+      l = fmaf(wsum[w], e, l);
+      const float4 y = wacc[w][tid];
+      x.x = fmaf(y.x, e, x.x);
+      x.y = fmaf(y.y, e, x.y);
+      x.z = fmaf(y.z, e, x.z);
+      x.w = fmaf(y.w, e, x.w);
+    }
+    const float inv = l > 0.0f ? 1.0f / l : 0.0f;
+    reinterpret_cast<float4*>(a)[tid] = make_float4(x.x * inv, x.y * inv, x.z * inv, x.w * inv);
   }
   __syncthreads();
 
