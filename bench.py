@@ -58,8 +58,8 @@ META_FORMATS = {"fp16": 0, "mx": 1, "turbo": 2}   # omnikv_config.key_meta_forma
 # next capture.
 TRAFFIC_CAPTURES = {
     ("qwen3-omni-30b-48L-b8-ctx65536", "fp16"): {
-        "sources_sha256": "bfd8f694b4bce03a68a8a11fcfe801258380d4cd26198d6caec73b331c52da6e",
-        "bytes_per_launch": 173710592 + 8660224},
+        "sources_sha256": "e667514f81980f6b28074c51c3f79cb8d4094517921d6e109946c792ce697e40",
+        "bytes_per_launch": 173712384 + 8849664},
 }
 KERNEL_SOURCES = ("decode_split_k.cu", "decode_common.cuh", "append.cuh", "common.cuh", "ptx.cuh", "kernels.h")
 
