@@ -54,12 +54,13 @@ CASES = [
     (2, 8, [4700 + 13 * i for i in range(16)], 2, 0, 2),
     (2, 8, [700, 333], 3, 1, 4),            # K4V4, one split per (sequence, kv head): long table-body splits
     (2, 8, [2300 + 13 * i for i in range(16)], 2, 0, 4),  # K4V4 with shared append CTAs (2 CTAs per SM)
+    (2, 8, [93, 40], 4, 200, 4),            # K4V4 beyond residency -> four-call fallback
 ]
 
 
 @pytest.mark.parametrize("hkv,G,lengths,steps,splits,bits", CASES,
                          ids=["b1-boundary", "ragged-b3", "h4", "fallback", "k4", "per-warp", "shared-append-ctas",
-                              "k4-one-split", "k4-shared-append-ctas"])
+                              "k4-one-split", "k4-shared-append-ctas", "k4-fallback"])
 def test_decode_step_matches_four_calls_and_oracle(cuda_device, hkv, G, lengths, steps, splits, bits):
     import bit_kv_cache_pack_b200 as m
     dev = cuda_device
